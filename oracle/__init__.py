@@ -1,0 +1,21 @@
+"""Double-precision CPU oracle of the SparseGPT layer solver.
+
+Test infrastructure: only the tests, the smoke check and the CPU-baseline leg
+of the bench use it. See ``sparsegpt_ref`` for what it computes and which
+passages of the pages each step follows.
+"""
+
+from .sparsegpt_ref import (  # noqa: F401
+    NotPositiveDefinite,
+    bits_to_mask,
+    damp,
+    hessian,
+    inverse_cholesky_upper,
+    mask_bits,
+    pack24,
+    parse_pattern,
+    prune_layer,
+    recon_error,
+    sweep,
+    unpack24,
+)

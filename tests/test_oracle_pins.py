@@ -1,0 +1,346 @@
+"""Pins of the double-precision oracle to facts the pages and mathematics fix.
+
+Each check is independent of the oracle's own routines: brute-force least
+squares on the activations X (numpy lstsq, no Cholesky), sub-matrix solves,
+closed forms, hand-computed fixtures from the pages, and invariants. The last
+test plants plausible mistakes in a copy of the oracle and checks that these
+pins catch every one.
+"""
+
+import inspect
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import sparsegpt_ref as ref
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _layer(rng, r=6, d=16, n=64, scale_spread=1.0):
+    s = np.exp(scale_spread * rng.standard_normal(d))
+    X = rng.standard_normal((n, d)) * s
+    W = rng.standard_normal((r, d)) / math.sqrt(d)
+    return W, X
+
+
+def _factor(X, damp_ratio=0.01):
+    H = oracle.hessian(X)
+    Hd, _ = oracle.damp(H, damp_ratio)
+    return H, Hd, oracle.inverse_cholesky_upper(Hd)
+
+
+# ---------------------------------------------------------------- references
+
+def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None):
+    """Sequential OBS written as explicit least-squares re-fits.
+
+    For each column q in order: decide the mask if the pattern decides here
+    (saliency w_c^2 / [(H_d[c:, c:])^-1]_00 on the current weights), set a
+    pruned weight to zero, then re-fit every column right of q to minimise
+    (w - w^) H_d (w - w^)^T with the columns <= q frozen. Uses general linear
+    solves only: no Cholesky, no U, no blocking.
+    """
+    kind, n_keep, m_grp, sparsity = ref.parse_pattern(pattern)
+    assert kind == "nm" or forced_mask is not None
+    r, d = W.shape
+    sal_den = np.array([np.linalg.inv(Hd[c:, c:])[0, 0] for c in range(d)])
+    out = np.array(W, dtype=np.float64)
+    mask = np.ones((r, d), dtype=bool) if forced_mask is None else forced_mask.copy()
+    for row in range(r):
+        w0 = np.array(W[row], dtype=np.float64)
+        cur = w0.copy()
+        for q in range(d):
+            if forced_mask is None and q % m_grp == 0:
+                S = cur[q:q + m_grp] ** 2 / sal_den[q:q + m_grp]
+                order = sorted(range(m_grp), key=lambda j: (-S[j], j))
+                mask[row, q:q + m_grp] = False
+                mask[row, [q + j for j in order[:n_keep]]] = True
+            if not mask[row, q]:
+                cur[q] = 0.0
+                if q + 1 < d:
+                    D_fixed = w0[:q + 1] - cur[:q + 1]
+                    rhs = Hd[q + 1:, :q + 1] @ D_fixed
+                    D_free = -np.linalg.solve(Hd[q + 1:, q + 1:], rhs)
+                    cur[q + 1:] = w0[q + 1:] - D_free
+        out[row] = cur
+    return out, mask
+
+
+def lstsq_fixed(X, w, fixed_idx, fixed_val):
+    """argmin over the free weights of ||X (w - w^)||^2 with some fixed."""
+    d = X.shape[1]
+    free = [j for j in range(d) if j not in set(fixed_idx)]
+    y = X @ w - X[:, fixed_idx] @ np.asarray(fixed_val, dtype=np.float64)
+    sol = np.linalg.lstsq(X[:, free], y, rcond=None)[0]
+    wh = np.zeros(d)
+    wh[fixed_idx] = fixed_val
+    wh[free] = sol
+    return wh
+
+
+# ---------------------------------------------------------------- the pins
+
+def test_hessian_hand_example():
+    g = _golden("hessian_2x2.json")
+    H = oracle.hessian(np.array(g["X_tokens_by_channels"]))
+    assert np.array_equal(H, np.array(g["H"]))
+
+
+def test_hessian_quadratic_form(rng):
+    X = rng.standard_normal((37, 9)) * np.exp(rng.standard_normal(9))
+    H = oracle.hessian(X, chunk=5)          # chunking must not matter
+    v = rng.standard_normal(9)
+    assert np.allclose(v @ H @ v, 2.0 / 37 * np.sum((X @ v) ** 2), rtol=1e-12)
+    assert np.array_equal(H, H.T)
+
+
+def test_damping_closed_form():
+    d = 10
+    H = np.diag(np.arange(1.0, d + 1))
+    Hd, lam = oracle.damp(H, 0.01)
+    assert lam == pytest.approx(0.01 * (d + 1) / 2, rel=1e-15)
+    assert np.allclose(np.diag(Hd), np.arange(1.0, d + 1) + lam, rtol=1e-15)
+
+
+def test_inverse_cholesky_is_the_unique_factor(rng):
+    _, X = _layer(rng, d=12, n=40)
+    _, Hd, U = _factor(X)
+    assert np.all(np.tril(U, -1) == 0)
+    assert np.all(np.diag(U) > 0)
+    assert np.allclose(U.T @ U @ Hd, np.eye(12), atol=1e-10)
+    # saliency denominator: U_cc^2 = [(H_d[c:, c:])^-1]_00
+    for c in range(12):
+        assert U[c, c] ** 2 == pytest.approx(np.linalg.inv(Hd[c:, c:])[0, 0], rel=1e-10)
+
+
+def test_not_positive_definite_raises():
+    with pytest.raises(oracle.NotPositiveDefinite):
+        oracle.prune_layer(np.ones((2, 4)), H=np.zeros((4, 4)))
+    H = np.eye(4)
+    H[2, 2] = -50.0
+    with pytest.raises(oracle.NotPositiveDefinite):
+        oracle.prune_layer(np.ones((2, 4)), H=H)
+
+
+def test_worked_example_24():
+    """Diagonal H: no compensation, 2:4 keeps the two largest |w|."""
+    g = _golden("worked_example_24.json")
+    W = np.array([g["dense"]])
+    out = oracle.prune_layer(W, H=3.0 * np.eye(4), pattern="2:4", blocksize=4)
+    assert np.array_equal(out["W"][0], np.array(g["sparse_24"]))
+    assert np.flatnonzero(out["mask"][0]).tolist() == g["kept_positions"]
+    assert out["meta"][0, 0] == 0 | (3 << 2)
+    assert np.array_equal(out["values"][0], np.array([0.42, 0.31]))
+
+
+def test_single_weight_obs_equals_least_squares(rng):
+    """Removing one weight = re-fit of the later weights on X ([SGPT] 八)."""
+    W, X = _layer(rng, r=3, d=8, n=50)
+    _, Hd, U = _factor(X, damp_ratio=0.0)
+    for q in range(8):
+        forced = np.ones_like(W, dtype=bool)
+        forced[:, q] = False
+        out = oracle.sweep(W, U, "2:4", blocksize=4, forced_mask=forced)
+        for row in range(3):
+            fixed = list(range(q + 1))
+            vals = list(W[row, :q]) + [0.0]
+            wh = lstsq_fixed(X, W[row], fixed, vals)
+            assert np.allclose(out["W"][row], wh, atol=1e-10), (q, row)
+    # q = 0 is textbook OBS: delta = -(w_q / [H^-1]_qq) H^-1 e_q
+    Hinv = np.linalg.inv(Hd)
+    forced = np.ones_like(W, dtype=bool)
+    forced[:, 0] = False
+    out = oracle.sweep(W, U, "2:4", blocksize=8, forced_mask=forced)
+    for row in range(3):
+        obs = W[row] - W[row, 0] / Hinv[0, 0] * Hinv[:, 0]
+        assert np.allclose(out["W"][row], obs, atol=1e-12)
+
+
+@pytest.mark.parametrize("blocksize", [4, 8, 16])
+def test_sweep_equals_frozen_prefix_least_squares(rng, blocksize):
+    W, X = _layer(rng, r=5, d=16, n=60, scale_spread=1.5)
+    _, Hd, U = _factor(X)
+    out = oracle.sweep(W, U, "2:4", blocksize=blocksize)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, "2:4")
+    assert np.array_equal(out["mask"], ref_mask)
+    assert np.allclose(out["W"], ref_W, atol=1e-11)
+    # forced, arbitrary (non-2:4) mask
+    forced = rng.random(W.shape) < 0.6
+    out = oracle.sweep(W, U, "2:4", blocksize=blocksize, forced_mask=forced)
+    ref_W, _ = frozen_prefix_sweep(W, Hd, "2:4", forced_mask=forced)
+    assert np.allclose(out["W"], ref_W, atol=1e-11)
+
+
+def test_diagonal_hessian_is_wanda_and_magnitude(rng):
+    """H diagonal: U diagonal, no compensation, keep the largest w^2 H_ii."""
+    r, d, n = 7, 16, 64
+    # tokens that each excite one channel give an exactly diagonal X^T X
+    X = np.zeros((n, d))
+    X[np.arange(n), np.arange(n) % d] = rng.standard_normal(n) * 3
+    W = rng.standard_normal((r, d))
+    out = oracle.prune_layer(W, X=X, pattern="2:4", damp_ratio=0.0, blocksize=8)
+    kept = out["mask"]
+    assert np.array_equal(out["W"][kept], W[kept])           # bit-unchanged
+    assert np.all(out["W"][~kept] == 0.0)
+    wanda = np.abs(W) * np.linalg.norm(X, axis=0)            # [SGPT] 十八
+    for g in range(d // 4):
+        top2 = np.argsort(-wanda[:, 4 * g:4 * g + 4], axis=1, kind="stable")[:, :2]
+        for row in range(r):
+            assert set(np.flatnonzero(kept[row, 4 * g:4 * g + 4])) == set(top2[row])
+    # H = c I: plain magnitude pruning ([SGPT] 五)
+    out = oracle.prune_layer(W, H=2.5 * np.eye(d), pattern="2:4")
+    for g in range(d // 4):
+        top2 = np.argsort(-np.abs(W[:, 4 * g:4 * g + 4]), axis=1, kind="stable")[:, :2]
+        for row in range(r):
+            assert set(np.flatnonzero(out["mask"][row, 4 * g:4 * g + 4])) == set(top2[row])
+
+
+def test_never_below_brute_force_optimum(rng):
+    """d_in = 8: compare with all C(4,2)^2 = 36 masks, each optimally re-fit."""
+    W, X = _layer(rng, r=4, d=8, n=40, scale_spread=1.0)
+    out = oracle.prune_layer(W, X=X, pattern="2:4", blocksize=8)
+    pairs = list(itertools.combinations(range(4), 2))
+    for row in range(4):
+        err_sgpt = np.sum((X @ (W[row] - out["W"][row])) ** 2)
+        best = math.inf
+        own = None
+        for a, b in itertools.product(pairs, pairs):
+            keep = list(a) + [4 + j for j in b]
+            pruned = [j for j in range(8) if j not in keep]
+            wh = np.zeros(8)
+            wh[keep] = np.linalg.lstsq(X[:, keep], X @ W[row], rcond=None)[0]
+            err = np.sum((X @ (W[row] - wh)) ** 2)
+            best = min(best, err)
+            if not out["mask"][row, pruned].any():
+                own = err
+        assert err_sgpt >= best * (1 - 1e-12)
+        assert err_sgpt >= own * (1 - 1e-12)
+
+
+def test_exact_counts_and_compression_table(rng):
+    W, X = _layer(rng, r=12, d=32, n=80)
+    _, _, U = _factor(X)
+    out = oracle.sweep(W, U, "2:4", blocksize=16)
+    groups = out["mask"].reshape(12, 8, 4).sum(axis=2)
+    assert np.all(groups == 2)
+    assert np.all(out["W"][~out["mask"]] == 0.0)
+    for ratio, approx in _golden("compression_table.json")["rows"]:
+        s = 1.0 - 1.0 / ratio
+        assert abs(s - approx) < 0.005
+        out = oracle.sweep(W, U, f"unstructured:{s}", blocksize=16)
+        for b0 in range(0, 32, 16):
+            pruned = (~out["mask"][:, b0:b0 + 16]).sum()
+            assert pruned == math.floor(s * 12 * 16)
+        assert np.all(out["W"][~out["mask"]] == 0.0)
+
+
+def test_unstructured_picks_smallest_saliency_with_tiebreak():
+    # U = I: saliency = w^2; equal magnitudes tie and break by (row, col)
+    W = np.array([[1.0, -1.0, 3.0, 1.0],
+                  [2.0, 1.0, -1.0, 5.0]])
+    out = oracle.sweep(W, np.eye(4), "unstructured:0.5", blocksize=4)
+    # k = 4 pruned: the five |w| = 1 entries in (row, col) order, first four
+    expect = np.ones_like(W, dtype=bool)
+    for rc in [(0, 0), (0, 1), (0, 3), (1, 1)]:
+        expect[rc] = False
+    assert np.array_equal(out["mask"], expect)
+    # all pruned saliencies <= all kept ones on a random tile
+    rng = np.random.default_rng(3)
+    W = rng.standard_normal((9, 8))
+    U = np.diag(rng.uniform(0.5, 2.0, 8))
+    out = oracle.sweep(W, U, "unstructured:0.7", blocksize=8)
+    S = (W / np.diag(U)) ** 2
+    assert S[~out["mask"]].max() <= S[out["mask"]].min()
+    assert (~out["mask"]).sum() == math.floor(0.7 * 72)
+
+
+def test_telescoping_loss(rng):
+    W, X = _layer(rng, r=6, d=24, n=70)
+    _, Hd, U = _factor(X)
+    for pat in ["2:4", "unstructured:0.6"]:
+        out = oracle.sweep(W, U, pat, blocksize=8)
+        dW = W - out["W"]
+        assert out["loss"].sum() == pytest.approx(np.trace(dW @ Hd @ dW.T), rel=1e-10)
+        assert np.allclose(out["loss"], np.einsum("ij,jk,ik->i", dW, Hd, dW), rtol=1e-10)
+
+
+def test_scale_invariance(rng):
+    W, X = _layer(rng, r=5, d=16, n=50)
+    a = oracle.prune_layer(W, X=X, pattern="2:4", blocksize=8)
+    b = oracle.prune_layer(W, X=3.0 * X, pattern="2:4", blocksize=8)
+    assert np.array_equal(a["mask"], b["mask"])
+    assert np.allclose(a["W"], b["W"], rtol=1e-10, atol=1e-13)
+    c = oracle.prune_layer(W * np.array([[2.0], [1], [0.5], [4], [1]]), X=X,
+                           pattern="2:4", blocksize=8)
+    assert np.array_equal(a["mask"], c["mask"])
+    assert np.allclose(c["W"][0], 2.0 * a["W"][0], rtol=1e-12, atol=1e-14)
+
+
+def test_blocksize_and_row_independence(rng):
+    W, X = _layer(rng, r=6, d=32, n=90, scale_spread=1.2)
+    _, _, U = _factor(X)
+    outs = [oracle.sweep(W, U, "2:4", blocksize=b) for b in (4, 8, 16, 32)]
+    for o in outs[1:]:
+        assert np.array_equal(o["mask"], outs[0]["mask"])
+        assert np.allclose(o["W"], outs[0]["W"], atol=1e-12)
+    sub = oracle.sweep(W[[1, 4]], U, "2:4", blocksize=16)
+    assert np.array_equal(sub["mask"], outs[2]["mask"][[1, 4]])
+    assert np.allclose(sub["W"], outs[2]["W"][[1, 4]], atol=1e-14)
+
+
+def test_pack_roundtrip_and_bits(rng):
+    W, X = _layer(rng, r=5, d=64, n=100)
+    out = oracle.prune_layer(W, X=X, pattern="2:4", blocksize=32)
+    back = oracle.unpack24(out["values"], out["meta"], 64)
+    assert np.array_equal(back, out["W"])
+    words = oracle.mask_bits(out["mask"])
+    assert words.shape == (5, 2) and words.dtype == np.uint32
+    assert np.array_equal(oracle.bits_to_mask(words, 64), out["mask"])
+    bad = out["mask"].copy()
+    bad[0, :4] = True
+    with pytest.raises(ValueError):
+        oracle.pack24(out["W"], bad)
+
+
+# ---------------------------------------------------------------- mutations
+
+_MUTATIONS = [
+    ("wrong sign of the compensation", "W1[:, q:] -= np.outer(e, U[c, c:i2])",
+     "W1[:, q:] += np.outer(e, U[c, c:i2])"),
+    ("dropped lazy trailing update", "W[:, i2:] -= E1 @ U[i1:i2, i2:]", "pass"),
+    ("transposed U in the trailing update", "W[:, i2:] -= E1 @ U[i1:i2, i2:]",
+     "W[:, i2:] -= E1 @ U.T[i1:i2, i2:]"),
+    ("error not divided by U_qq", "e = (w - p) / U[c, c]", "e = (w - p)"),
+    ("saliency on the starting weights", "S = (W1[:, q:q + m_grp] / diagU[c:c + m_grp]) ** 2",
+     "S = (W[:, c:c + m_grp] / diagU[c:c + m_grp]) ** 2"),
+    ("saliency without U", "S = (W1[:, q:q + m_grp] / diagU[c:c + m_grp]) ** 2",
+     "S = (W1[:, q:q + m_grp]) ** 2"),
+    ("off-by-one in the rank-1 update", "W1[:, q:] -= np.outer(e, U[c, c:i2])",
+     "W1[:, q + 1:] -= np.outer(e, U[c, c:i2 - 1])"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", _MUTATIONS, ids=[m[0] for m in _MUTATIONS])
+def test_pins_catch_planted_mistakes(rng, name, old, new):
+    src = inspect.getsource(ref.sweep)
+    assert old in src, name
+    ns = dict(vars(ref))
+    exec(src.replace(old, new), ns)
+    mutated = ns["sweep"]
+    W, X = _layer(rng, r=5, d=16, n=60, scale_spread=1.5)
+    _, Hd, U = _factor(X)
+    got = mutated(W, U, "2:4", blocksize=8)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, "2:4")
+    same = np.array_equal(got["mask"], ref_mask) and np.allclose(got["W"], ref_W, atol=1e-9)
+    assert not same, f"pins did not catch: {name}"
