@@ -1,0 +1,174 @@
+/*
+ * sgpt.h - C ABI of the B200 (sm_100a) SparseGPT layer solver.
+ *
+ * The operation: given the weights W [d_out x d_in] of one linear layer and
+ * calibration inputs X [n_tok x d_in], find a sparse W^ whose outputs W^X stay
+ * as close as possible to WX under an N:M or unstructured sparsity pattern,
+ * compensating every removed weight in the remaining weights of its row.
+ *   - Problem statement: SparseGPT review ("SparseGPT: Massive Language Models
+ *     Can Be Accurately Pruned in One-Shot", devpress.csdn.net), section 六.
+ *   - Hessian proxy H = X X^T: same page, section 七.
+ *   - Optimal-Brain-Surgeon removal with compensation: section 八.
+ *   - Layer-wise pipeline, columns processed block by block: section 十一.
+ *   - N:M (2:4) semi-structured sparsity: section 十四 14.4.
+ *   - 2:4 storage, values plus 2-bit position metadata: "LLM 2:4 structured
+ *     sparsity production guide" (oh-bug.com), section "2:4 结构化稀疏的核心机制
+ *     与生产状态分类".
+ *
+ * Conventions for every call below.
+ *   - All array arguments are DEVICE pointers into memory the caller owns
+ *     (allocated by the caller, e.g. through PyTorch). The library never
+ *     allocates, frees or synchronises, except sgpt_sync_status.
+ *   - Matrices are row-major. X is bf16 passed as raw 16-bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call
+ *     only enqueues work on that stream.
+ *   - `ws`/`ws_bytes` is caller-provided device scratch, at least
+ *     sgpt_workspace_bytes() bytes, 256-byte aligned. It is not kept between
+ *     calls.
+ *   - Argument errors are reported synchronously as the return value, before
+ *     anything is enqueued. Numeric errors found on the device (a matrix that
+ *     is not positive definite, non-finite values, a bounded wait that ran out,
+ *     a mask that breaks 2:4) are written to `*dev_info` (device int). Kernels
+ *     record only the first error, and every kernel of a later call that sees
+ *     a non-zero *dev_info returns without touching its outputs. Clear it with
+ *     sgpt_info_clear, read it with sgpt_sync_status.
+ *     dev_info values: 0 ok; k > 0 pivot k (1-based column of H) was not
+ *     positive; SGPT_INFO_NONFINITE; SGPT_INFO_TIMEOUT; SGPT_INFO_BAD_MASK.
+ *   - Size limits: 32 <= d_in <= 32768 and d_in % 32 == 0; 1 <= d_out <=
+ *     16777216; ldw >= d_in and ldw % 4 == 0; every pointer 16-byte aligned.
+ */
+#ifndef SGPT_H_
+#define SGPT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SGPT_ABI_VERSION 1
+
+typedef enum sgpt_status {
+  SGPT_OK = 0,
+  SGPT_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or parameter   */
+  SGPT_ERR_NOT_PD = 2,      /* damped H has a non-positive pivot           */
+  SGPT_ERR_NONFINITE = 3,   /* NaN/Inf met in H, U or W                    */
+  SGPT_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up          */
+  SGPT_ERR_CUDA = 5,        /* a CUDA runtime call failed                  */
+  SGPT_ERR_UNSUPPORTED = 6, /* valid request this build does not implement */
+  SGPT_ERR_BAD_MASK = 7,    /* pack: a group does not keep exactly 2 of 4  */
+  SGPT_ERR_WORKSPACE = 8    /* ws too small or misaligned                  */
+} sgpt_status;
+
+/* Non-pivot codes written to *dev_info. */
+#define SGPT_INFO_NONFINITE (-1)
+#define SGPT_INFO_TIMEOUT (-2)
+#define SGPT_INFO_BAD_MASK (-3)
+
+#define SGPT_PATTERN_UNSTRUCTURED 0
+#define SGPT_PATTERN_NM 1
+
+typedef struct sgpt_params {
+  int pattern;    /* SGPT_PATTERN_UNSTRUCTURED or SGPT_PATTERN_NM            */
+  int n, m;       /* N:M - keep n of every m consecutive inputs (2 and 4)    */
+  float sparsity; /* unstructured - fraction pruned in each block, [0, 1)    */
+  int blocksize;  /* columns per OBS block: 32, 64, 96 or 128                */
+  float damp;     /* damping ratio (0.01 = 1% of the mean diagonal), >= 0    */
+  int forced;     /* 1: mask_bits is an INPUT and no selection is made       */
+} sgpt_params;
+
+/* Human-readable name of a status. Never NULL. */
+const char* sgpt_status_string(sgpt_status s);
+
+/* SGPT_ABI_VERSION of the loaded library. */
+int sgpt_abi_version(void);
+
+/* Diagnostics: number of kernels this library has enqueued since it was
+ * loaded (all devices, all streams). Memsets and copies are not counted. */
+uint64_t sgpt_kernel_launches(void);
+
+/* Scratch bytes needed by any call below for these sizes (n_tok only matters
+ * for the Hessian; pass 0 when H is given). */
+size_t sgpt_workspace_bytes(int d_out, int d_in, int64_t n_tok, const sgpt_params* p);
+
+/* *dev_info = 0, enqueued on `stream`. */
+sgpt_status sgpt_info_clear(int* dev_info, void* stream);
+
+/* Blocking: waits for `stream`, reads *dev_info and maps it to a status
+ * (0 -> OK, k > 0 -> NOT_PD, other codes as named above). */
+sgpt_status sgpt_sync_status(const int* dev_info, void* stream);
+
+/* H += X^T X  (SparseGPT review, section 七: H = X X^T with X as channels x
+ * tokens; here X is tokens x channels, so the same matrix is X^T X).
+ *   H   [d_in x d_in] fp32, full symmetric matrix, updated in place; both
+ *       triangles are written. Zero it first (sgpt_hessian_zero) to start a
+ *       new accumulation; call repeatedly to stream token chunks.
+ *   X   [n_tok x d_in] bf16 bit patterns, row-major, 16-byte aligned rows.
+ * Products are exact in fp32; sums are fp32 (tensor cores, fixed order). */
+sgpt_status sgpt_hessian_zero(float* H, int d_in, void* stream);
+sgpt_status sgpt_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tok, int d_in,
+                                    void* ws, size_t ws_bytes, int* dev_info, void* stream);
+
+/* U = upper Cholesky factor of H_d^-1, with H_d = (2/n_total) H + lambda I,
+ * lambda = damp * mean(diag((2/n_total) H)); H_d^-1 = U^T U, U_ii > 0.
+ *   H   [d_in x d_in] fp32, the accumulated X^T X; only the upper triangle
+ *       (i <= j) is read. Not modified (unless U == H).
+ *   U   [d_in x d_in] fp32 output; zeros below the diagonal. May alias H.
+ * Errors on the device: pivot k not positive -> *dev_info = k (NOT_PD);
+ * non-finite diagonal -> NONFINITE. U is then unspecified. */
+sgpt_status sgpt_factor(const float* H, int64_t n_total, int d_in, float damp, float* U,
+                        void* ws, size_t ws_bytes, int* dev_info, void* stream);
+
+/* The blocked OBS sweep (SparseGPT review, sections 八 and 十一): for each
+ * block of p->blocksize columns, select the mask (N:M at the first column of
+ * each group of m, on the weights as compensated so far, keeping the n largest
+ * w_c^2 / U_cc^2, ties to the lower column; or unstructured: exactly
+ * floor(sparsity * d_out * width) of the block's smallest saliencies, ties by
+ * row then column), then for each column q: e = (w_q - p_q) / U_qq, subtract
+ * e * U[q, q:] from the rest of the block, and after the block subtract
+ * Err * U[block, right of block] from every later column.
+ *   W          [d_out x ldw] fp32, in: dense weights, out: pruned weights.
+ *   U          from sgpt_factor (same d_in).
+ *   mask_bits  [d_out x d_in/32] uint32, bit c%32 of word c/32 = 1 if kept;
+ *              output, or input when p->forced.
+ *   row_loss   [d_out] fp32 or NULL: sum over the row of e^2 (accumulated
+ *              in place: zero it first).
+ * The result of an N:M run does not depend on blocksize. */
+sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U,
+                       const sgpt_params* p, uint32_t* mask_bits, float* row_loss,
+                       void* ws, size_t ws_bytes, int* dev_info, void* stream);
+
+/* 2:4 packing (2:4 production guide, section on the 2:4 mechanism):
+ *   values [d_out x d_in/2] fp32: the two kept weights of each group of four,
+ *          in column order;
+ *   meta   [d_out x d_in/32] uint32: group g of a row is the 4-bit code
+ *          a | (b << 2) (a < b kept positions) in bits [4(g%8), 4(g%8)+4) of
+ *          word g/8.
+ * A group whose mask does not keep exactly two sets *dev_info = BAD_MASK. */
+sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint32_t* mask_bits,
+                        float* values, uint32_t* meta, int* dev_info, void* stream);
+
+/* Layer reconstruction error (SparseGPT review, section 六, the objective):
+ * num_den[0] = tr(dW H dW^T), num_den[1] = tr(W0 H W0^T), dW = W0 - W, in
+ * fp64 on the device. H is the full symmetric matrix (undamped; any positive
+ * scale). Both W0 and W use leading dimension ldw. */
+sgpt_status sgpt_recon_error(const float* W0, const float* W, int d_out, int d_in, int ldw,
+                             const float* H, double* num_den, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* One layer end to end: if X != NULL, H = X^T X over its n_tok rows, else H
+ * must already hold that sum; then U = sgpt_factor(H), sgpt_prune, and for
+ * 2:4 sgpt_pack24 (values/meta may be NULL to skip packing). U and H must
+ * not alias. *dev_info is cleared first. */
+sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint16_t* X,
+                             int64_t n_tok, float* H, float* U, const sgpt_params* p,
+                             uint32_t* mask_bits, float* values, uint32_t* meta,
+                             float* row_loss, void* ws, size_t ws_bytes, int* dev_info,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SGPT_H_ */

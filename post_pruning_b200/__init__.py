@@ -1,0 +1,30 @@
+"""B200-native SparseGPT layer solver: Python binding of the libsgpt C ABI.
+
+The solver (Hessian accumulation, damped factorisation, blocked OBS sweep
+with 2:4 or unstructured masks, 2:4 packing) runs in hand-written sm_100a CUDA
+kernels inside ``libsgpt.so``; see ``include/sgpt.h`` for the contract.
+"""
+
+from .sgpt import (  # noqa: F401
+    EXPORTS,
+    HostPruner,
+    LIB_PATH,
+    LayerBuffers,
+    Params,
+    SgptError,
+    factor,
+    hessian_accumulate,
+    hessian_zero,
+    info_clear,
+    kernel_launches,
+    lib,
+    new_info,
+    pack24,
+    prune,
+    prune_layer,
+    raise_on_info,
+    recon_error,
+    sync_status,
+    workspace,
+    workspace_bytes,
+)

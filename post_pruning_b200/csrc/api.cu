@@ -1,0 +1,195 @@
+// C ABI of the solver: argument checks, workspace carving and launch order.
+// Nothing here computes; every step runs in the kernels of the other files.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "../../include/sgpt.h"
+#include "common.cuh"
+#include "kernels.h"
+
+#include <atomic>
+
+namespace sgpt {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace sgpt
+
+namespace {
+
+using namespace sgpt;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool valid_din(int d_in) { return d_in >= 32 && d_in <= 32768 && d_in % 32 == 0; }
+bool valid_dout(int d_out) { return d_out >= 1 && d_out <= (1 << 24); }
+
+sgpt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SGPT_OK : SGPT_ERR_CUDA; }
+
+sgpt_status check_params(const sgpt_params* p) {
+  if (!p) return SGPT_ERR_INVALID_ARG;
+  if (p->blocksize < 32 || p->blocksize > kMaxBlock || p->blocksize % 32) return SGPT_ERR_INVALID_ARG;
+  if (!(p->damp >= 0.f) || !std::isfinite(p->damp)) return SGPT_ERR_INVALID_ARG;
+  if (p->forced != 0 && p->forced != 1) return SGPT_ERR_INVALID_ARG;
+  if (p->pattern == SGPT_PATTERN_NM) {
+    if (p->n <= 0 || p->m <= 0 || p->n > p->m) return SGPT_ERR_INVALID_ARG;
+    if (!(p->n == 2 && p->m == 4)) return SGPT_ERR_UNSUPPORTED;
+  } else if (p->pattern == SGPT_PATTERN_UNSTRUCTURED) {
+    if (!(p->sparsity >= 0.f && p->sparsity < 1.f)) return SGPT_ERR_INVALID_ARG;
+  } else {
+    return SGPT_ERR_INVALID_ARG;
+  }
+  return SGPT_OK;
+}
+
+sgpt_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return SGPT_OK;
+  if (!ws || !aligned256(ws) || have < need) return SGPT_ERR_WORKSPACE;
+  return SGPT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sgpt_status_string(sgpt_status s) {
+  switch (s) {
+    case SGPT_OK: return "ok";
+    case SGPT_ERR_INVALID_ARG: return "invalid argument";
+    case SGPT_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case SGPT_ERR_NONFINITE: return "non-finite value";
+    case SGPT_ERR_TIMEOUT: return "device-side wait timed out";
+    case SGPT_ERR_CUDA: return "CUDA runtime error";
+    case SGPT_ERR_UNSUPPORTED: return "unsupported by this build";
+    case SGPT_ERR_BAD_MASK: return "mask breaks the 2:4 pattern";
+    case SGPT_ERR_WORKSPACE: return "workspace too small or misaligned";
+  }
+  return "unknown status";
+}
+
+int sgpt_abi_version(void) { return SGPT_ABI_VERSION; }
+
+uint64_t sgpt_kernel_launches(void) { return sgpt::g_launches.load(std::memory_order_relaxed); }
+
+size_t sgpt_workspace_bytes(int d_out, int d_in, int64_t n_tok, const sgpt_params* p) {
+  (void)p;
+  if (!valid_din(d_in) || !valid_dout(d_out) || n_tok < 0) return 0;
+  size_t need = std::max(factor_ws_bytes(d_in), prune_ws_bytes(d_out));
+  if (n_tok > 0) need = std::max(need, hessian_ws_bytes(d_in, n_tok));
+  return need;
+}
+
+sgpt_status sgpt_info_clear(int* dev_info, void* stream) {
+  if (!dev_info) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(dev_info, 0, sizeof(int), as_stream(stream)));
+}
+
+sgpt_status sgpt_sync_status(const int* dev_info, void* stream) {
+  if (!dev_info) return SGPT_ERR_INVALID_ARG;
+  int h = 0;
+  if (cudaMemcpyAsync(&h, dev_info, sizeof(int), cudaMemcpyDeviceToHost, as_stream(stream)) != cudaSuccess)
+    return SGPT_ERR_CUDA;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SGPT_ERR_CUDA;
+  if (h == 0) return SGPT_OK;
+  if (h > 0) return SGPT_ERR_NOT_PD;
+  if (h == SGPT_INFO_NONFINITE) return SGPT_ERR_NONFINITE;
+  if (h == SGPT_INFO_TIMEOUT) return SGPT_ERR_TIMEOUT;
+  if (h == SGPT_INFO_BAD_MASK) return SGPT_ERR_BAD_MASK;
+  return SGPT_ERR_CUDA;
+}
+
+sgpt_status sgpt_hessian_zero(float* H, int d_in, void* stream) {
+  if (!H || !aligned16(H) || !valid_din(d_in)) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(H, 0, (size_t)d_in * d_in * sizeof(float), as_stream(stream)));
+}
+
+sgpt_status sgpt_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tok, int d_in, void* ws,
+                                    size_t ws_bytes, int* dev_info, void* stream) {
+  if (!H || !X || !aligned16(H) || !aligned16(X) || !valid_din(d_in) || n_tok < 0 || !dev_info)
+    return SGPT_ERR_INVALID_ARG;
+  if (n_tok > (int64_t)INT32_MAX) return SGPT_ERR_INVALID_ARG;   // TMA coordinates are 32-bit
+  if (n_tok == 0) return SGPT_OK;
+  sgpt_status s = check_ws(ws, ws_bytes, hessian_ws_bytes(d_in, n_tok));
+  if (s != SGPT_OK) return s;
+  cudaError_t e = launch_hessian_tc(H, X, n_tok, d_in, ws, dev_info, as_stream(stream));
+  if (e == cudaErrorNotSupported) return SGPT_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+sgpt_status sgpt_factor(const float* H, int64_t n_total, int d_in, float damp, float* U, void* ws,
+                        size_t ws_bytes, int* dev_info, void* stream) {
+  if (!H || !U || !dev_info || !aligned16(H) || !aligned16(U) || !valid_din(d_in) || n_total <= 0)
+    return SGPT_ERR_INVALID_ARG;
+  if (!(damp >= 0.f) || !std::isfinite(damp)) return SGPT_ERR_INVALID_ARG;
+  sgpt_status s = check_ws(ws, ws_bytes, factor_ws_bytes(d_in));
+  if (s != SGPT_OK) return s;
+  return from_cuda(launch_factor(H, n_total, d_in, damp, U, ws, dev_info, as_stream(stream)));
+}
+
+sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U, const sgpt_params* p,
+                       uint32_t* mask_bits, float* row_loss, void* ws, size_t ws_bytes, int* dev_info,
+                       void* stream) {
+  if (!W || !U || !mask_bits || !dev_info || !aligned16(W) || !aligned16(U) || !aligned16(mask_bits))
+    return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
+  sgpt_status s = check_params(p);
+  if (s != SGPT_OK) return s;
+  s = check_ws(ws, ws_bytes, prune_ws_bytes(d_out));
+  if (s != SGPT_OK) return s;
+  return from_cuda(launch_prune(W, d_out, d_in, ldw, U, *p, mask_bits, row_loss, ws, dev_info,
+                                as_stream(stream)));
+}
+
+sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint32_t* mask_bits,
+                        float* values, uint32_t* meta, int* dev_info, void* stream) {
+  if (!W || !mask_bits || !values || !meta || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(mask_bits) || !aligned16(meta))
+    return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_pack24(W, ldw, d_out, d_in, mask_bits, values, meta, dev_info, as_stream(stream)));
+}
+
+sgpt_status sgpt_recon_error(const float* W0, const float* W, int d_out, int d_in, int ldw, const float* H,
+                             double* num_den, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!W0 || !W || !H || !num_den) return SGPT_ERR_INVALID_ARG;
+  if (!aligned16(W0) || !aligned16(W) || !aligned16(H) || (reinterpret_cast<uintptr_t>(num_den) & 7u))
+    return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_recon(W0, W, d_out, d_in, ldw, H, num_den, as_stream(stream)));
+}
+
+sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint16_t* X, int64_t n_tok,
+                             float* H, float* U, const sgpt_params* p, uint32_t* mask_bits, float* values,
+                             uint32_t* meta, float* row_loss, void* ws, size_t ws_bytes, int* dev_info,
+                             void* stream) {
+  if (!H || !U || H == U || n_tok <= 0 || !dev_info) return SGPT_ERR_INVALID_ARG;
+  sgpt_status s = check_params(p);
+  if (s != SGPT_OK) return s;
+  if (!valid_din(d_in) || !valid_dout(d_out)) return SGPT_ERR_INVALID_ARG;
+  s = check_ws(ws, ws_bytes, sgpt_workspace_bytes(d_out, d_in, X ? n_tok : 0, p));
+  if (s != SGPT_OK) return s;
+  const bool pack = p->pattern == SGPT_PATTERN_NM && values && meta;
+  if ((values || meta) && !pack) return SGPT_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if ((s = sgpt_info_clear(dev_info, stream)) != SGPT_OK) return s;
+  if (X) {
+    if ((s = sgpt_hessian_zero(H, d_in, stream)) != SGPT_OK) return s;
+    if ((s = sgpt_hessian_accumulate(H, X, n_tok, d_in, ws, ws_bytes, dev_info, stream)) != SGPT_OK) return s;
+  }
+  if ((s = sgpt_factor(H, n_tok, d_in, p->damp, U, ws, ws_bytes, dev_info, stream)) != SGPT_OK) return s;
+  if (row_loss && cudaMemsetAsync(row_loss, 0, (size_t)d_out * sizeof(float), st) != cudaSuccess)
+    return SGPT_ERR_CUDA;
+  if ((s = sgpt_prune(W, d_out, d_in, ldw, U, p, mask_bits, row_loss, ws, ws_bytes, dev_info, stream)) != SGPT_OK)
+    return s;
+  if (pack) s = sgpt_pack24(W, d_out, d_in, ldw, mask_bits, values, meta, dev_info, stream);
+  return s;
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Shared device helpers of the SparseGPT solver kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sgpt.h"
+
+namespace sgpt {
+
+constexpr int kNumSMs = 148;          // B200
+constexpr int kTile = 128;            // square tile of H, R, U and the GEMMs
+constexpr int kMaxBlock = 128;        // widest OBS block held by the sweep
+
+// Bounded spin: a device-side wait gives up after this many polls and
+// records SGPT_INFO_TIMEOUT instead of hanging the GPU.
+constexpr long long kSpinLimit = 1ll << 26;
+
+// First error wins; later kernels of the chain see it and return early.
+__device__ __forceinline__ void set_info(int* info, int code) {
+  if (info) atomicCAS(info, 0, code);
+}
+
+__device__ __forceinline__ bool info_set(const int* info) {
+  return info && *(volatile const int*)info != 0;
+}
+
+// The same test taken once per CTA (every thread of the block must call it):
+// thread 0 reads the word and the answer is shared, so a CTA never splits
+// into threads that return and threads that wait at a barrier.
+__device__ __forceinline__ bool cta_info_set(const int* info) {
+  return __syncthreads_or(threadIdx.x == 0 && info_set(info)) != 0;
+}
+
+__device__ __forceinline__ float4 ld4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ void st4(float* p, float4 v) {
+  *reinterpret_cast<float4*>(p) = v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ long long cdivll(long long a, long long b) {
+  return (a + b - 1) / b;
+}
+
+// Saliency of weight w in a column whose U diagonal is u: (w / u)^2 in fp32
+// with IEEE division. Every kernel that ranks weights calls this one function,
+// so the selection kernels and the sweep agree bit for bit.
+__device__ __forceinline__ float saliency(float w, float u) {
+  float t = __fdiv_rn(w, u);
+  return __fmul_rn(t, t);
+}
+
+// Host-side count of kernel launches (diagnostics, sgpt_kernel_launches).
+void count_launches(unsigned long long n);
+
+// Host-side workspace carving: consecutive 256-byte aligned sub-buffers.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+}  // namespace sgpt

@@ -1,0 +1,370 @@
+// H += X^T X on the 5th-generation tensor cores (SparseGPT review, section 七:
+// the Hessian proxy of a linear layer is the Gram matrix of its inputs).
+//
+// X is bf16 [n x d] row-major, so both GEMM operands of C = X^T X are the same
+// tensor read "MN-major": for C[i][j] = sum_t X[t][i] X[t][j], A(i, t) and
+// B(j, t) are contiguous along i and j. One CTA owns a 128 x 256 tile of H
+// whose rows i0.. and columns j0.. meet the upper triangle (H is symmetric:
+// only those tiles are computed, and every element i <= j is written to both
+// H[i][j] and H[j][i]). Tokens are split across CTAs when there are too few
+// tiles to fill the GPU; split partials are summed in split order by the CTA
+// that finishes a tile last (deterministic).
+//
+// Per CTA: warp 0 lane 0 streams 64-token stages with TMA (128-byte swizzle,
+// one box = 64 tokens x 64 channels), warp 1 lane 0 issues
+// tcgen05.mma.kind::f16 (M=128, N=256, K=16, bf16 in, fp32 accumulate in
+// TMEM, 256 columns), and all four warps drain TMEM with tcgen05.ld after the
+// last MMA commits. Every wait is bounded; a wait that runs out records
+// SGPT_INFO_TIMEOUT.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sgpt {
+
+namespace {
+
+constexpr int kM = 128;              // tile rows (i)
+constexpr int kN = 256;              // tile columns (j)
+constexpr int kBK = 64;              // tokens per stage
+constexpr int kStages = 4;
+constexpr int kBox = kBK * 64 * 2;   // bytes of one 64-token x 64-channel box
+constexpr int kAStage = 2 * kBox;    // 16 KB
+constexpr int kBStage = 4 * kBox;    // 32 KB
+constexpr int kStageBytes = kAStage + kBStage;
+constexpr int kThreads = 128;
+constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr long long kWaitCycles = 4000000000ll;   // ~2 s at the B200 boost clock
+
+// instruction descriptor: D fp32, A/B bf16, both MN-major, N=256, M=128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                            ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor, MN-major operand, 128-byte swizzle:
+// atoms of 64 channels x 8 tokens (1 KB); LBO = stride between 64-channel
+// atoms (one TMA box), SBO = stride between 8-token groups (1 KB).
+__device__ __forceinline__ uint64_t mn_desc(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fff);
+  d |= (uint64_t)((kBox >> 4) & 0x3fff) << 16;     // leading byte offset
+  d |= (uint64_t)((1024 >> 4) & 0x3fff) << 32;     // stride byte offset
+  d |= (uint64_t)1 << 46;                          // descriptor version (sm100)
+  d |= (uint64_t)2 << 61;                          // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.b32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false if the barrier phase did not complete in time.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+        "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+        "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Tiles meeting the upper triangle, band by band: band ti (rows ti*128..)
+// holds the 256-wide column tiles tj >= ti/2, so it starts at tile
+// ti*tn - floor(ti/2)*floor((ti-1)/2).
+__host__ __device__ inline long long band_start(int ti, int tn) {
+  return (long long)ti * tn - (long long)(ti / 2) * ((ti - 1) / 2);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
+    const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int d, long long n,
+    int nsplit, long long per, float* __restrict__ part, unsigned int* __restrict__ tickets,
+    int* info) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  __shared__ int failed;
+  __shared__ unsigned int last;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / nsplit, split = blockIdx.x - (blockIdx.x / nsplit) * nsplit;
+  // tile -> (band ti, column tile tj)
+  const int tn = (d + kN - 1) / kN;
+  int ti = 0;
+  {
+    int lo = 0, hi = (d + kM - 1) / kM - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (band_start(mid, tn) <= tile) lo = mid;
+      else hi = mid - 1;
+    }
+    ti = lo;
+  }
+  const int tj = ti / 2 + (int)(tile - band_start(ti, tn));
+  const int i0 = ti * kM, j0 = tj * kN;
+  const long long t_begin = (long long)split * per;
+  const long long t_end = t_begin + per < n ? t_begin + per : n;
+  const int iters = (int)((t_end - t_begin + kBK - 1) / kBK);
+
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages), done = smem_u32(bars + 2 * kStages);
+
+  if (threadIdx.x == 0) {
+    failed = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = cta_info_set(info) || iters <= 0;
+
+  if (!skip && warp == 0 && lane == 0) {
+    // TMA producer
+    int issued = 0;
+    for (int it = 0; it < iters; ++it) {
+      const int s = it % kStages;
+      const uint32_t par = ((it / kStages) & 1) ^ 1;
+      if (it >= kStages && !mbar_wait(empty0 + 8 * s, par)) {
+        failed = 1;
+        break;
+      }
+      const uint32_t bar = full0 + 8 * s;
+      mbar_expect_tx(bar, kStageBytes);
+      const int y = (int)(t_begin + (long long)it * kBK);
+      const uint32_t a = s0 + s * kStageBytes, b = a + kAStage;
+      tma_load_2d(a, &xmap, bar, i0, y);
+      tma_load_2d(a + kBox, &xmap, bar, i0 + 64, y);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tma_load_2d(b + c * kBox, &xmap, bar, j0 + 64 * c, y);
+      ++issued;
+    }
+    // never leave with copies in flight: wait for every stage that was armed
+    for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
+      if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
+  } else if (!skip && warp == 1 && lane == 0) {
+    // MMA issuer
+    for (int it = 0; it < iters; ++it) {
+      const int s = it % kStages;
+      if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+        failed = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = s0 + s * kStageBytes, b = a + kAStage;
+#pragma unroll
+      for (int ks = 0; ks < kBK / 16; ++ks)
+        mma_bf16(tmem, mn_desc(a + ks * 2048), mn_desc(b + ks * 2048), (it | ks) != 0);
+      mma_commit(empty0 + 8 * s);
+    }
+    mma_commit(done);
+  }
+
+  // Epilogue: every warp waits for the accumulator, then reads its 32 lanes.
+  bool have = !skip;
+  if (have) {
+    __syncwarp();
+    if (!mbar_wait(done, 0)) {
+      failed = 1;
+      have = false;
+    }
+  }
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (failed) {
+    have = false;
+    if (threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
+  }
+
+  const int i = i0 + warp * 32 + lane;   // TMEM lane = tile row
+  if (have) {
+    float* dst = nsplit > 1 ? part + (size_t)blockIdx.x * kM * kN + (size_t)(warp * 32 + lane) * kN : nullptr;
+#pragma unroll 1
+    for (int c = 0; c < kN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
+      if (nsplit > 1) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          st4(dst + c * 32 + e, make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])));
+      } else if (i < d) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = j0 + c * 32 + e;
+          if (j < i || j >= d) continue;
+          const float x = __uint_as_float(v[e]);
+          H[(long long)i * d + j] += x;
+          if (j != i) H[(long long)j * d + i] += x;
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
+
+  if (nsplit > 1 && !failed && !skip) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = (atomicAdd(&tickets[tile], 1u) == (unsigned)nsplit - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    // the last CTA of the tile sums the partials in split order
+    const float* base = part + (size_t)tile * nsplit * kM * kN;
+    for (int e = threadIdx.x; e < kM * kN; e += kThreads) {
+      const int r = e / kN, c = e - (e / kN) * kN;
+      const int ii = i0 + r, jj = j0 + c;
+      if (ii >= d || jj >= d || jj < ii) continue;
+      float sum = 0.f;
+      for (int p = 0; p < nsplit; ++p) sum += __ldcg(base + (size_t)p * kM * kN + e);
+      H[(long long)ii * d + jj] += sum;
+      if (jj != ii) H[(long long)jj * d + ii] += sum;
+    }
+    if (threadIdx.x == 0) tickets[tile] = 0;
+  }
+}
+
+// ----------------------------------------------------------------- host
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+struct Plan {
+  int tiles, nsplit;
+  long long per;
+};
+
+Plan plan(int d, long long n) {
+  const int tm = (d + kM - 1) / kM, tn = (d + kN - 1) / kN;
+  const int tiles = (int)band_start(tm, tn);
+  // split tokens when the tiles alone cannot fill the GPU
+  long long ns = 1;
+  if (tiles < kNumSMs) ns = (kNumSMs + tiles - 1) / tiles;
+  const long long max_split = (n + 4 * kBK - 1) / (4 * kBK);   // >= 4 stages per split
+  ns = std::max<long long>(1, std::min(ns, max_split));
+  long long per = ((n + ns - 1) / ns + kBK - 1) / kBK * kBK;
+  ns = (n + per - 1) / per;
+  return {tiles, (int)std::max<long long>(1, ns), per};
+}
+
+}  // namespace
+
+size_t hessian_ws_bytes(int d, long long n) {
+  const Plan p = plan(d, n);
+  Carve c(nullptr);
+  c.take<unsigned int>((size_t)p.tiles);
+  if (p.nsplit > 1) c.take<float>((size_t)p.tiles * p.nsplit * kM * kN);
+  return c.off + 256;
+}
+
+cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, void* ws, int* info,
+                              cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const Plan p = plan(d, n);
+  Carve c(ws);
+  unsigned int* tickets = c.take<unsigned int>((size_t)p.tiles);
+  float* part = p.nsplit > 1 ? c.take<float>((size_t)p.tiles * p.nsplit * kM * kN) : nullptr;
+
+  cudaMemsetAsync(tickets, 0, sizeof(unsigned int) * p.tiles, st);
+
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kBK};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    attr = true;
+  }
+  hessian_tc_kernel<<<p.tiles * p.nsplit, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, tickets,
+                                                                 info);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sgpt

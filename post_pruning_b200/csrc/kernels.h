@@ -1,0 +1,38 @@
+// Internal launchers behind the C ABI (host side, one translation unit each).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "../../include/sgpt.h"
+
+namespace sgpt {
+
+// factor.cu
+size_t factor_ws_bytes(int d);
+size_t factor_part_tiles(int d);
+int trtri_splits(int K, int s);
+cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, float* U, void* ws,
+                          int* info, cudaStream_t st);
+
+// sweep.cu
+size_t prune_ws_bytes(int d_out);
+cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* U,
+                         const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
+                         int* info, cudaStream_t st);
+
+// pack.cu
+cudaError_t launch_pack24(const float* W, long long ldw, int rows, int d, const uint32_t* mask,
+                          float* values, uint32_t* meta, int* info, cudaStream_t st);
+cudaError_t launch_recon(const float* W0, const float* W, int rows, int d, long long ldw,
+                         const float* H, double* num_den, cudaStream_t st);
+
+// hessian_tc.cu
+size_t hessian_ws_bytes(int d, long long n);
+cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, void* ws, int* info,
+                              cudaStream_t st);
+
+}  // namespace sgpt

@@ -1,0 +1,122 @@
+// 2:4 packing and the layer reconstruction error.
+//
+// Packing follows the 2:4 production guide (oh-bug.com, section on the 2:4
+// mechanism): of every four consecutive weights along the input dimension two
+// are kept, stored in column order, and their positions are recorded as
+// 2-bit indices.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "kernels.h"
+
+namespace sgpt {
+
+// One thread per (row, 32 columns): 8 groups, one mask word, one meta word,
+// 32 weights in, 16 values out.
+__global__ void __launch_bounds__(256) pack24_kernel(const float* __restrict__ W, long long ldw,
+                                                     int rows, int d,
+                                                     const uint32_t* __restrict__ mask,
+                                                     float* __restrict__ values,
+                                                     uint32_t* __restrict__ meta, int* info) {
+  if (info_set(info)) return;
+  const int wpr = d / 32;
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (long long)rows * wpr) return;
+  const int row = (int)(t / wpr), wd = (int)(t - (long long)row * wpr);
+  const uint32_t m = mask[t];
+  const float* src = W + (long long)row * ldw + wd * 32;
+  float* dst = values + (long long)row * (d / 2) + wd * 16;
+  uint32_t code = 0;
+  bool bad = false;
+#pragma unroll
+  for (int g2 = 0; g2 < 4; ++g2) {           // two groups per float4 pair
+    float out[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int g = 2 * g2 + h;
+      const uint32_t nib = (m >> (4 * g)) & 0xfu;
+      const float4 x = ld4(src + 4 * g);
+      bad |= __popc(nib) != 2;
+      const int a = __ffs(nib) - 1;                  // lowest kept
+      const int b = 31 - __clz(nib);                 // highest kept
+      const int aa = a < 0 ? 0 : a, bb = b < 0 ? 0 : b;
+      out[2 * h] = aa == 0 ? x.x : aa == 1 ? x.y : aa == 2 ? x.z : x.w;
+      out[2 * h + 1] = bb == 0 ? x.x : bb == 1 ? x.y : bb == 2 ? x.z : x.w;
+      code |= (uint32_t)((aa | (bb << 2)) & 0xf) << (4 * g);
+    }
+    st4(dst + 4 * g2, make_float4(out[0], out[1], out[2], out[3]));
+  }
+  meta[t] = code;
+  if (bad) set_info(info, SGPT_INFO_BAD_MASK);
+}
+
+cudaError_t launch_pack24(const float* W, long long ldw, int rows, int d, const uint32_t* mask,
+                          float* values, uint32_t* meta, int* info, cudaStream_t st) {
+  const long long n = (long long)rows * (d / 32);
+  pack24_kernel<<<(unsigned)cdivll(n, 256), 256, 0, st>>>(W, ldw, rows, d, mask, values, meta, info);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------- reconstruction error
+
+// out += sum over the tile of (A H)[m][n] * A[m][n], A = W0 - W (diff) or W0.
+template <class OA>
+__global__ void __launch_bounds__(kGemmThreads) quad_form_kernel(OA A, const float* __restrict__ H,
+                                                                 int d, const float* __restrict__ P,
+                                                                 const float* __restrict__ Q,
+                                                                 long long ldw, int rows,
+                                                                 double* __restrict__ out) {
+  extern __shared__ float smem[];
+  __shared__ double red[kGemmThreads / 32];
+  const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile;
+  A.i0 = m0;
+  A.I = rows - m0;
+  float acc[8][8];
+  zero_acc(acc);
+  const OpIContig B{H, d, n0, d - n0, d};
+  gemm_tile(A, B, 0, d, acc, smem);
+  double s = 0.0;
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const int m = m0 + acc_row(a);
+    if (m >= rows) continue;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int n = n0 + acc_col(h);
+      if (n >= d) continue;
+      const long long o = (long long)m * ldw + n;
+      float4 p = ld4(P + o);
+      if (Q) {
+        const float4 q = ld4(Q + o);
+        p.x -= q.x; p.y -= q.y; p.z -= q.z; p.w -= q.w;
+      }
+      s += (double)acc[a][4 * h + 0] * p.x + (double)acc[a][4 * h + 1] * p.y +
+           (double)acc[a][4 * h + 2] * p.z + (double)acc[a][4 * h + 3] * p.w;
+    }
+  }
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kGemmThreads / 32; ++w) t += red[w];
+    atomicAdd(out, t);
+  }
+}
+
+cudaError_t launch_recon(const float* W0, const float* W, int rows, int d, long long ldw,
+                         const float* H, double* num_den, cudaStream_t st) {
+  cudaMemsetAsync(num_den, 0, 2 * sizeof(double), st);
+  dim3 grid(cdiv(d, kTile), cdiv(rows, kTile));
+  const OpKContigDiff dA{W0, W, ldw, 0, rows, d};
+  quad_form_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(dA, H, d, W0, W, ldw, rows, num_den);
+  count_launches(1);
+  const OpKContig A0{W0, ldw, 0, rows, d};
+  quad_form_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(A0, H, d, W0, nullptr, ldw, rows, num_den + 1);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace sgpt

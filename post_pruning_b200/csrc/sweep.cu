@@ -1,0 +1,320 @@
+// The blocked OBS column sweep (SparseGPT review, sections 八 and 十一).
+//
+// Per block of `bw` <= 128 columns starting at i1:
+//   1. (unstructured) exact k-selection of the block's smallest saliencies
+//      over all d_out rows: radix select on a 64-bit key (saliency bits, then
+//      row * bw + column), select_pass_kernel, one 8-bit digit per launch;
+//   2. sweep_kernel: every row's 128 columns are processed in order in
+//      registers: mask decision (2:4 at each group start on the compensated
+//      weights), e = (w_q - p_q) / U_qq, rank-1 update of the rest of the
+//      block with the U row held in shared memory;
+//   3. trailing_kernel: W[:, i2:] -= Err * U[i1:i2, i2:] (FP32 SIMT product).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "kernels.h"
+
+namespace sgpt {
+
+// ---------------------------------------------------------------- sweep
+
+constexpr int kSweepRows = 16;             // rows per CTA
+constexpr int kSeg = 16;                   // columns per thread
+constexpr int kTpr = kMaxBlock / kSeg;     // threads per row (8)
+constexpr int kSweepThreads = kSweepRows * kTpr;
+constexpr size_t kSweepSmem = (size_t)kMaxBlock * kMaxBlock * sizeof(float);
+
+enum SweepMode { kModeNM24 = 0, kModeThreshold = 1, kModeForced = 2 };
+
+__device__ __forceinline__ unsigned long long sal_key(float w, float u, unsigned idx) {
+  return ((unsigned long long)__float_as_uint(saliency(w, u)) << 32) | idx;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
+    float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
+    const float* __restrict__ U, uint32_t* __restrict__ mask, float* __restrict__ row_loss,
+    float* __restrict__ Err, const unsigned long long* __restrict__ thr, int* info) {
+  if (cta_info_set(info)) return;
+  extern __shared__ float Us[];   // [128][128]: U[i1 + a][i1 + b]
+  const int tid = threadIdx.x;
+  for (int e = tid * 4; e < kMaxBlock * kMaxBlock; e += kSweepThreads * 4) {
+    const int a = e >> 7, b = e & 127;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (a < bw && b < bw) v = ld4(U + (long long)(i1 + a) * d + i1 + b);
+    st4(Us + e, v);
+  }
+  __syncthreads();
+
+  const int lane = tid & 31;
+  const int seg = tid % kTpr;                      // column segment of this thread
+  const int row = blockIdx.x * kSweepRows + tid / kTpr;
+  const bool live = row < rows && seg * kSeg < bw;
+  const int c0 = seg * kSeg;                       // block-relative first column
+  float w[kSeg], err[kSeg];
+  uint32_t keep = 0xffffu;
+  bool bad = false;
+  float* wrow = W + (long long)row * ldw + i1 + c0;
+#pragma unroll
+  for (int v = 0; v < kSeg / 4; ++v) {
+    float4 x = live ? ld4(wrow + 4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    w[4 * v + 0] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+  }
+#pragma unroll
+  for (int j = 0; j < kSeg; ++j) {
+    err[j] = 0.f;
+    bad |= !isfinite(w[j]);
+  }
+  if (MODE == kModeThreshold && live) {
+    const unsigned long long t = *thr;
+    keep = 0;
+#pragma unroll
+    for (int j = 0; j < kSeg; ++j) {
+      const unsigned idx = (unsigned)row * (unsigned)bw + (unsigned)(c0 + j);
+      if (sal_key(w[j], Us[(c0 + j) * kMaxBlock + c0 + j], idx) >= t) keep |= 1u << j;
+    }
+  }
+  if (MODE == kModeForced && live) {
+    const uint32_t word = mask[(long long)row * (d / 32) + (i1 + c0) / 32];
+    keep = (word >> ((i1 + c0) & 31)) & 0xffffu;
+  }
+  float loss = 0.f;
+
+#pragma unroll
+  for (int qs = 0; qs < kTpr; ++qs) {
+    if (qs * kSeg >= bw) break;
+#pragma unroll
+    for (int qj = 0; qj < kSeg; ++qj) {
+      const int q = qs * kSeg + qj;
+      float e = 0.f;
+      if (seg == qs) {
+        if (MODE == kModeNM24 && (qj & 3) == 0) {
+          // 2 of 4 on the compensated weights; ties keep the lower column.
+          float s[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) s[t] = saliency(w[qj + t], Us[(q + t) * kMaxBlock + q + t]);
+          uint32_t g = 0;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            int rank = 0;   // how many of the group beat column t
+#pragma unroll
+            for (int o = 0; o < 4; ++o)
+              if (o != t && (s[o] > s[t] || (s[o] == s[t] && o < t))) ++rank;
+            if (rank < 2) g |= 1u << t;
+          }
+          keep = (keep & ~(0xfu << qj)) | (g << qj);
+        }
+        const float wq = w[qj];
+        const bool kept = (keep >> qj) & 1u;
+        e = kept ? 0.f : __fdiv_rn(wq, Us[q * kMaxBlock + q]);
+        w[qj] = kept ? wq : 0.f;
+        err[qj] = e;
+        loss = fmaf(e, e, loss);
+      }
+      e = __shfl_sync(0xffffffffu, e, (lane & ~(kTpr - 1)) | qs);
+      if (seg >= qs && e != 0.f) {
+        const float* urow = Us + q * kMaxBlock + c0;
+        float u[kSeg];
+#pragma unroll
+        for (int v = 0; v < kSeg / 4; ++v) {
+          const float4 x = ld4(urow + 4 * v);
+          u[4 * v + 0] = x.x; u[4 * v + 1] = x.y; u[4 * v + 2] = x.z; u[4 * v + 3] = x.w;
+        }
+        if (seg > qs) {
+#pragma unroll
+          for (int j = 0; j < kSeg; ++j) w[j] = fmaf(-e, u[j], w[j]);
+        } else {
+#pragma unroll
+          for (int j = qj + 1; j < kSeg; ++j) w[j] = fmaf(-e, u[j], w[j]);
+        }
+      }
+    }
+  }
+
+  // Loss of the row: sum over its kTpr threads.
+  float tot = loss;
+#pragma unroll
+  for (int o = 1; o < kTpr; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  bad |= !isfinite(tot);
+  // Mask words: segments 2p and 2p+1 make one 32-bit word.
+  const uint32_t other = __shfl_down_sync(0xffffffffu, keep, 1);
+  if (live) {
+#pragma unroll
+    for (int v = 0; v < kSeg / 4; ++v) st4(wrow + 4 * v, make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
+    float* erow = Err + (long long)row * kMaxBlock + c0;
+#pragma unroll
+    for (int v = 0; v < kSeg / 4; ++v) st4(erow + 4 * v, make_float4(err[4 * v], err[4 * v + 1], err[4 * v + 2], err[4 * v + 3]));
+    if (MODE != kModeForced && (seg & 1) == 0) {
+      const uint32_t hi = (c0 + kSeg < bw) ? other : 0u;
+      mask[(long long)row * (d / 32) + (i1 + c0) / 32] = (keep & 0xffffu) | (hi << 16);
+    }
+    if (seg == 0 && row_loss) row_loss[row] += tot;
+    if (bad) set_info(info, SGPT_INFO_NONFINITE);
+  }
+}
+
+// --------------------------------------------------------- trailing update
+
+// W[:, i2:] -= Err[:, :bw] * U[i1:i1+bw, i2:]
+__global__ void __launch_bounds__(kGemmThreads) trailing_kernel(
+    float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
+    const float* __restrict__ U, const float* __restrict__ Err, const int* info) {
+  if (cta_info_set(info)) return;
+  extern __shared__ float smem[];
+  const int i2 = i1 + bw;
+  const int n0 = i2 + blockIdx.x * kTile;
+  const int m0 = blockIdx.y * kTile;
+  float acc[8][8];
+  zero_acc(acc);
+  const OpKContig A{Err, kMaxBlock, m0, rows - m0, bw};
+  const OpIContig B{U + (long long)i1 * d, d, n0, d - n0, bw};
+  gemm_tile(A, B, 0, bw, acc, smem);
+  store_tile(W + (long long)m0 * ldw + n0, ldw, rows - m0, d - n0, acc, -1.f, 1.f);
+}
+
+// ------------------------------------------------ unstructured selection
+
+struct SelState {
+  unsigned long long prefix;   // key bits fixed so far
+  unsigned long long thr;      // exclusive threshold: pruned iff key < thr
+  unsigned int k_rem;          // rank still to place inside the prefix bin
+  int done;
+  unsigned int ticket;
+  unsigned int pad;
+  unsigned int hist[256];
+};
+
+__global__ void select_init_kernel(SelState* st, unsigned int k) {
+  const int t = threadIdx.x;
+  if (t < 256) st->hist[t] = 0;
+  if (t == 0) {
+    st->prefix = 0;
+    st->thr = 0;
+    st->k_rem = k;
+    st->done = (k == 0);
+    st->ticket = 0;
+  }
+}
+
+// Pass p histograms digit p (bits 63-8p .. 56-8p) of the keys that match the
+// prefix found so far. The last CTA to finish picks the digit holding the
+// k-th smallest key and either finishes (the whole bin is pruned) or narrows
+// the prefix for the next pass.
+__global__ void __launch_bounds__(256) select_pass_kernel(
+    const float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
+    const float* __restrict__ U, SelState* st, int pass, const int* info) {
+  if (cta_info_set(info) || st->done) return;
+  __shared__ unsigned int h[256];
+  __shared__ float ud[kMaxBlock];
+  __shared__ unsigned int last;
+  const int t = threadIdx.x;
+  h[t] = 0;
+  if (t < bw) ud[t] = U[(long long)(i1 + t) * d + i1 + t];
+  __syncthreads();
+  const int shift = 56 - 8 * pass;
+  const unsigned long long prefix = st->prefix;
+  const long long total4 = (long long)rows * (bw / 4);
+  for (long long e = (long long)blockIdx.x * 256 + t; e < total4; e += (long long)gridDim.x * 256) {
+    const int row = (int)(e / (bw / 4));
+    const int c = (int)(e - (long long)row * (bw / 4)) * 4;
+    const float4 x = ld4(W + (long long)row * ldw + i1 + c);
+    const float v[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const unsigned long long key = sal_key(v[j], ud[c + j], (unsigned)row * (unsigned)bw + (unsigned)(c + j));
+      if (pass == 0 || (key >> (shift + 8)) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+    }
+  }
+  __syncthreads();
+  if (h[t]) atomicAdd(&st->hist[t], h[t]);
+  __threadfence();
+  __syncthreads();
+  if (t == 0) last = (atomicAdd(&st->ticket, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (t == 0) {
+    unsigned int cum = 0, digit = 0, cnt = 0;
+    const unsigned int k = st->k_rem;
+    for (int b = 0; b < 256; ++b) {
+      const unsigned int c = __ldcg(&st->hist[b]);
+      if (cum + c >= k) { digit = b; cnt = c; break; }
+      cum += c;
+    }
+    const unsigned int krem = k - cum;
+    const unsigned long long pre = (prefix << 8) | digit;
+    st->prefix = pre;
+    st->k_rem = krem;
+    if (cnt == krem) {
+      st->done = 1;
+      st->thr = (pre << shift) + (1ull << shift);   // every key of the bin is pruned
+    }
+    st->ticket = 0;
+  }
+  __syncthreads();
+  st->hist[t] = 0;
+}
+
+// ----------------------------------------------------------------- driver
+
+size_t prune_ws_bytes(int d_out) {
+  Carve c(nullptr);
+  c.take<float>((size_t)d_out * kMaxBlock);   // Err
+  c.take<SelState>(1);
+  return c.off + 256;
+}
+
+cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* U,
+                         const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
+                         int* info, cudaStream_t st) {
+  Carve c(ws);
+  float* Err = c.take<float>((size_t)rows * kMaxBlock);
+  SelState* sel = c.take<SelState>(1);
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(sweep_kernel<kModeNM24>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    cudaFuncSetAttribute(sweep_kernel<kModeThreshold>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    cudaFuncSetAttribute(sweep_kernel<kModeForced>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    attr_done = true;
+  }
+  const int B = p.blocksize;
+  const int sweep_grid = cdiv(rows, kSweepRows);
+  for (int i1 = 0; i1 < d; i1 += B) {
+    const int bw = min(B, d - i1);
+    if (p.forced) {
+      sweep_kernel<kModeForced><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+      count_launches(1);
+    } else if (p.pattern == SGPT_PATTERN_NM) {
+      sweep_kernel<kModeNM24><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+      count_launches(1);
+    } else {
+      const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
+      select_init_kernel<<<1, 256, 0, st>>>(sel, (unsigned int)kk);
+      count_launches(1);
+      const long long total4 = (long long)rows * (bw / 4);
+      const int g = (int)std::min<long long>(cdivll(total4, 256 * 8), 4 * kNumSMs);
+      for (int pass = 0; pass < 8; ++pass) {
+        select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, sel, pass, info);
+        count_launches(1);
+      }
+      sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, &sel->thr, info);
+      count_launches(1);
+    }
+    const int i2 = i1 + bw;
+    if (i2 < d) {
+      dim3 grid(cdiv(d - i2, kTile), cdiv(rows, kTile));
+      trailing_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(W, ldw, rows, d, i1, bw, U, Err, info);
+      count_launches(1);
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sgpt

@@ -1,0 +1,359 @@
+"""Python binding of libsgpt (the C ABI declared in include/sgpt.h).
+
+Argument marshalling only: every function here checks tensor dtypes, devices
+and shapes, passes raw device pointers and the current CUDA stream to the
+C entry point of the same name, and turns a non-OK status into SgptError.
+All arithmetic of the solver runs in the library's CUDA kernels; PyTorch only
+provides device memory and streams. There is no fallback: if the library is
+missing, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsgpt.so")
+
+SGPT_OK = 0
+STATUS_NAMES = {
+    0: "OK", 1: "INVALID_ARG", 2: "NOT_PD", 3: "NONFINITE", 4: "TIMEOUT",
+    5: "CUDA", 6: "UNSUPPORTED", 7: "BAD_MASK", 8: "WORKSPACE",
+}
+PATTERN_UNSTRUCTURED = 0
+PATTERN_NM = 1
+
+EXPORTS = (
+    "sgpt_status_string", "sgpt_abi_version", "sgpt_kernel_launches", "sgpt_workspace_bytes",
+    "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
+    "sgpt_hessian_accumulate", "sgpt_factor", "sgpt_prune", "sgpt_pack24",
+    "sgpt_recon_error", "sgpt_prune_layer",
+)
+
+
+class SgptError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{where}: SGPT_{'ERR_' if status else ''}{self.name} ({status})")
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("pattern", ctypes.c_int), ("n", ctypes.c_int), ("m", ctypes.c_int),
+                ("sparsity", ctypes.c_float), ("blocksize", ctypes.c_int),
+                ("damp", ctypes.c_float), ("forced", ctypes.c_int)]
+
+
+@dataclass(frozen=True)
+class Params:
+    """Sparsity pattern and solver knobs (mirrors sgpt_params)."""
+    pattern: str = "2:4"        # "2:4" or "unstructured:<fraction>"
+    blocksize: int = 128
+    damp: float = 0.01
+    forced: bool = False
+
+    @property
+    def is_nm(self) -> bool:
+        return not self.pattern.startswith("unstructured")
+
+    @property
+    def sparsity(self) -> float:
+        return 0.0 if self.is_nm else float(self.pattern.split(":")[1])
+
+    def to_c(self) -> _Params:
+        if self.is_nm:
+            n, m = (int(x) for x in self.pattern.split(":"))
+            return _Params(PATTERN_NM, n, m, 0.0, self.blocksize, self.damp, int(self.forced))
+        return _Params(PATTERN_UNSTRUCTURED, 0, 0, self.sparsity, self.blocksize, self.damp,
+                       int(self.forced))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsgpt.so once; raise loudly if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m post_pruning_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    pp = ctypes.POINTER(_Params)
+    sig = {
+        "sgpt_status_string": (ctypes.c_char_p, [i32]),
+        "sgpt_abi_version": (i32, []),
+        "sgpt_kernel_launches": (ctypes.c_uint64, []),
+        "sgpt_workspace_bytes": (sz, [i32, i32, i64, pp]),
+        "sgpt_info_clear": (i32, [vp, vp]),
+        "sgpt_sync_status": (i32, [vp, vp]),
+        "sgpt_hessian_zero": (i32, [vp, i32, vp]),
+        "sgpt_hessian_accumulate": (i32, [vp, vp, i64, i32, vp, sz, vp, vp]),
+        "sgpt_factor": (i32, [vp, i64, i32, ctypes.c_float, vp, vp, sz, vp, vp]),
+        "sgpt_prune": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, sz, vp, vp]),
+        "sgpt_pack24": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
+        "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
+                                   vp, sz, vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+# ------------------------------------------------------------------ helpers
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _rowmajor(t: torch.Tensor, name: str) -> int:
+    """Leading dimension of a 2-D tensor with unit column stride."""
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with contiguous rows")
+    return t.stride(0)
+
+
+def _check(status: int, where: str):
+    if status != SGPT_OK:
+        raise SgptError(status, where)
+
+
+def kernel_launches() -> int:
+    """Kernels libsgpt has enqueued since it was loaded."""
+    return int(lib().sgpt_kernel_launches())
+
+
+def workspace_bytes(d_out: int, d_in: int, n_tok: int = 0, params: Params | None = None) -> int:
+    p = (params or Params()).to_c()
+    return int(lib().sgpt_workspace_bytes(d_out, d_in, n_tok, ctypes.byref(p)))
+
+
+def workspace(d_out: int, d_in: int, n_tok: int = 0, params: Params | None = None,
+              device="cuda") -> torch.Tensor:
+    """A byte tensor large enough for every call at these sizes."""
+    return torch.empty(workspace_bytes(d_out, d_in, n_tok, params), dtype=torch.uint8, device=device)
+
+
+def new_info(device="cuda") -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+# ------------------------------------------------------------- entry points
+
+def info_clear(dev_info: torch.Tensor, stream=None):
+    _check(lib().sgpt_info_clear(_ptr(dev_info), _stream(stream)), "sgpt_info_clear")
+
+
+def sync_status(dev_info: torch.Tensor, stream=None) -> int:
+    """Blocking; returns the status code (0 = OK) without raising."""
+    return int(lib().sgpt_sync_status(_ptr(dev_info), _stream(stream)))
+
+
+def raise_on_info(dev_info: torch.Tensor, stream=None, where="device"):
+    _check(sync_status(dev_info, stream), where)
+
+
+def hessian_zero(H: torch.Tensor, stream=None):
+    _dev(H, torch.float32, "H")
+    _check(lib().sgpt_hessian_zero(_ptr(H), H.shape[0], _stream(stream)), "sgpt_hessian_zero")
+
+
+def hessian_accumulate(H: torch.Tensor, X: torch.Tensor, ws: torch.Tensor, dev_info: torch.Tensor,
+                       stream=None):
+    _dev(H, torch.float32, "H")
+    _dev(X, torch.bfloat16, "X")
+    d = H.shape[0]
+    if H.shape != (d, d) or not H.is_contiguous() or X.dim() != 2 or X.shape[1] != d or not X.is_contiguous():
+        raise ValueError("H must be [d, d] and X [n, d], both contiguous")
+    _check(lib().sgpt_hessian_accumulate(_ptr(H), _ptr(X), X.shape[0], d, _ptr(ws), ws.numel(),
+                                         _ptr(dev_info), _stream(stream)), "sgpt_hessian_accumulate")
+
+
+def factor(H: torch.Tensor, n_total: int, damp: float, U: torch.Tensor, ws: torch.Tensor,
+           dev_info: torch.Tensor, stream=None):
+    _dev(H, torch.float32, "H")
+    _dev(U, torch.float32, "U")
+    d = H.shape[0]
+    if H.shape != (d, d) or U.shape != (d, d) or not H.is_contiguous() or not U.is_contiguous():
+        raise ValueError("H and U must be contiguous [d, d]")
+    _check(lib().sgpt_factor(_ptr(H), n_total, d, damp, _ptr(U), _ptr(ws), ws.numel(), _ptr(dev_info),
+                             _stream(stream)), "sgpt_factor")
+
+
+def prune(W: torch.Tensor, U: torch.Tensor, params: Params, mask: torch.Tensor, ws: torch.Tensor,
+          dev_info: torch.Tensor, row_loss: torch.Tensor | None = None, stream=None):
+    _dev(W, torch.float32, "W")
+    _dev(U, torch.float32, "U")
+    _dev(mask, torch.int32, "mask")
+    ldw = _rowmajor(W, "W")
+    r, d = W.shape
+    if mask.shape != (r, d // 32) or not mask.is_contiguous():
+        raise ValueError("mask must be contiguous int32 [d_out, d_in/32]")
+    if row_loss is not None:
+        _dev(row_loss, torch.float32, "row_loss")
+    p = params.to_c()
+    _check(lib().sgpt_prune(_ptr(W), r, d, ldw, _ptr(U), ctypes.byref(p), _ptr(mask), _ptr(row_loss),
+                            _ptr(ws), ws.numel(), _ptr(dev_info), _stream(stream)), "sgpt_prune")
+
+
+def pack24(W: torch.Tensor, mask: torch.Tensor, values: torch.Tensor, meta: torch.Tensor,
+           dev_info: torch.Tensor, stream=None):
+    _dev(W, torch.float32, "W")
+    _dev(values, torch.float32, "values")
+    _dev(mask, torch.int32, "mask")
+    _dev(meta, torch.int32, "meta")
+    ldw = _rowmajor(W, "W")
+    r, d = W.shape
+    if values.shape != (r, d // 2) or meta.shape != (r, d // 32):
+        raise ValueError("values must be [d_out, d_in/2] and meta [d_out, d_in/32]")
+    _check(lib().sgpt_pack24(_ptr(W), r, d, ldw, _ptr(mask), _ptr(values), _ptr(meta), _ptr(dev_info),
+                             _stream(stream)), "sgpt_pack24")
+
+
+def recon_error(W0: torch.Tensor, W: torch.Tensor, H: torch.Tensor, num_den: torch.Tensor,
+                stream=None):
+    """num_den (float64 [2], device) = (tr(dW H dW^T), tr(W0 H W0^T))."""
+    _dev(W0, torch.float32, "W0")
+    _dev(W, torch.float32, "W")
+    _dev(H, torch.float32, "H")
+    _dev(num_den, torch.float64, "num_den")
+    ldw = _rowmajor(W, "W")
+    if _rowmajor(W0, "W0") != ldw or W0.shape != W.shape:
+        raise ValueError("W0 and W must share shape and leading dimension")
+    r, d = W.shape
+    _check(lib().sgpt_recon_error(_ptr(W0), _ptr(W), r, d, ldw, _ptr(H), _ptr(num_den), None, 0,
+                                  _stream(stream)), "sgpt_recon_error")
+
+
+def prune_layer(W: torch.Tensor, H: torch.Tensor, U: torch.Tensor, params: Params,
+                mask: torch.Tensor, ws: torch.Tensor, dev_info: torch.Tensor,
+                X: torch.Tensor | None = None, n_tok: int | None = None,
+                values: torch.Tensor | None = None, meta: torch.Tensor | None = None,
+                row_loss: torch.Tensor | None = None, stream=None):
+    """One layer end to end (sgpt_prune_layer); X None means H holds X^T X."""
+    _dev(W, torch.float32, "W")
+    _dev(H, torch.float32, "H")
+    _dev(U, torch.float32, "U")
+    _dev(mask, torch.int32, "mask")
+    ldw = _rowmajor(W, "W")
+    r, d = W.shape
+    if X is not None:
+        _dev(X, torch.bfloat16, "X")
+        if X.dim() != 2 or X.shape[1] != d or not X.is_contiguous():
+            raise ValueError("X must be contiguous [n, d_in]")
+        n_tok = X.shape[0]
+    if n_tok is None:
+        raise ValueError("n_tok is required when H is given")
+    p = params.to_c()
+    _check(lib().sgpt_prune_layer(_ptr(W), r, d, ldw, _ptr(X), n_tok, _ptr(H), _ptr(U), ctypes.byref(p),
+                                  _ptr(mask), _ptr(values), _ptr(meta), _ptr(row_loss), _ptr(ws),
+                                  ws.numel(), _ptr(dev_info), _stream(stream)), "sgpt_prune_layer")
+
+
+# --------------------------------------------------------------- conveniences
+
+@dataclass
+class LayerBuffers:
+    """Device buffers for pruning one layer shape (allocated once, reused)."""
+    d_out: int
+    d_in: int
+    n_tok: int
+    H: torch.Tensor
+    U: torch.Tensor
+    mask: torch.Tensor
+    values: torch.Tensor
+    meta: torch.Tensor
+    row_loss: torch.Tensor
+    ws: torch.Tensor
+    info: torch.Tensor
+
+    @classmethod
+    def allocate(cls, d_out: int, d_in: int, n_tok: int, device="cuda") -> "LayerBuffers":
+        f32 = dict(dtype=torch.float32, device=device)
+        i32 = dict(dtype=torch.int32, device=device)
+        return cls(d_out, d_in, n_tok,
+                   H=torch.empty((d_in, d_in), **f32), U=torch.empty((d_in, d_in), **f32),
+                   mask=torch.empty((d_out, d_in // 32), **i32),
+                   values=torch.empty((d_out, d_in // 2), **f32),
+                   meta=torch.empty((d_out, d_in // 32), **i32),
+                   row_loss=torch.empty(d_out, **f32),
+                   ws=workspace(d_out, d_in, n_tok, device=device),
+                   info=new_info(device))
+
+    def run(self, W: torch.Tensor, X: torch.Tensor | None, params: Params, stream=None):
+        pack = params.is_nm
+        prune_layer(W, self.H, self.U, params, self.mask, self.ws, self.info, X=X,
+                    n_tok=self.n_tok, values=self.values if pack else None,
+                    meta=self.meta if pack else None, row_loss=self.row_loss, stream=stream)
+
+
+class HostPruner:
+    """End-to-end pruning from host memory through the public API.
+
+    Owns the device buffers of one layer shape and pinned host outputs.
+    run() copies W and X from (pinned) host memory to the device, prunes the
+    layer from X with sgpt_prune_layer, copies the pruned weights, the mask
+    and (for 2:4) the packed values and metadata back to the host, and checks
+    the device status. All copies are enqueued on the current stream.
+    """
+
+    def __init__(self, d_out: int, d_in: int, n_tok: int, device="cuda"):
+        self.bufs = LayerBuffers.allocate(d_out, d_in, n_tok, device)
+        self.W = torch.empty((d_out, d_in), dtype=torch.float32, device=device)
+        self.X = torch.empty((n_tok, d_in), dtype=torch.bfloat16, device=device)
+        pin = dict(pin_memory=True)
+        self.W_out = torch.empty((d_out, d_in), dtype=torch.float32, **pin)
+        self.mask_out = torch.empty((d_out, d_in // 32), dtype=torch.int32, **pin)
+        self.values_out = torch.empty((d_out, d_in // 2), dtype=torch.float32, **pin)
+        self.meta_out = torch.empty((d_out, d_in // 32), dtype=torch.int32, **pin)
+
+    def h2d_bytes(self) -> int:
+        return self.W.numel() * 4 + self.X.numel() * 2
+
+    def d2h_bytes(self, params: Params) -> int:
+        b = self.W_out.numel() * 4 + self.mask_out.numel() * 4
+        if params.is_nm:
+            b += self.values_out.numel() * 4 + self.meta_out.numel() * 4
+        return b
+
+    def enqueue(self, W_host: torch.Tensor, X_host: torch.Tensor | None, params: Params, stream=None):
+        """Copies and pruning, all asynchronous; X_host None reuses the X on
+        the device from the previous call."""
+        self.W.copy_(W_host, non_blocking=True)
+        if X_host is not None:
+            self.X.copy_(X_host, non_blocking=True)
+        self.bufs.run(self.W, self.X, params, stream=stream)
+        self.W_out.copy_(self.W, non_blocking=True)
+        self.mask_out.copy_(self.bufs.mask, non_blocking=True)
+        if params.is_nm:
+            self.values_out.copy_(self.bufs.values, non_blocking=True)
+            self.meta_out.copy_(self.bufs.meta, non_blocking=True)
+
+    def run(self, W_host: torch.Tensor, X_host: torch.Tensor, params: Params, stream=None):
+        self.enqueue(W_host, X_host, params, stream)
+        raise_on_info(self.bufs.info, stream, "HostPruner.run")
+        if params.is_nm:
+            return self.W_out, self.mask_out, self.values_out, self.meta_out
+        return self.W_out, self.mask_out, None, None

@@ -1,0 +1,114 @@
+"""The C-ABI library loads and exports every entry point include/sgpt.h
+declares; argument errors are rejected before anything touches a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import post_pruning_b200 as pp
+from post_pruning_b200 import sgpt as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sgpt.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|sgpt_status|int|size_t|uint64_t)\s+(sgpt_\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(pp.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = pp.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert L.sgpt_abi_version() == 1
+
+
+def test_status_strings():
+    L = pp.lib()
+    for code in range(0, 9):
+        assert L.sgpt_status_string(code)
+    assert L.sgpt_status_string(123) == b"unknown status"
+
+
+def test_workspace_bytes():
+    p = S.Params("2:4").to_c()
+    L = pp.lib()
+    ws = L.sgpt_workspace_bytes(4096, 11008, 131072, ctypes.byref(p))
+    # at least the factor's d x d scratch
+    assert ws >= 11008 * 11008 * 4
+    assert L.sgpt_workspace_bytes(4096, 100, 0, ctypes.byref(p)) == 0      # d_in % 32
+    assert L.sgpt_workspace_bytes(0, 256, 0, ctypes.byref(p)) == 0          # d_out
+    assert pp.workspace_bytes(256, 256, 2048) > 0
+
+
+FAKE = 1 << 20          # an aligned non-null address; never dereferenced
+MISALIGNED = FAKE + 4
+
+
+@pytest.mark.parametrize("case", [
+    "null_W", "bad_din", "bad_ldw", "bad_blocksize", "bad_sparsity", "nm_unsupported",
+    "misaligned", "bad_pattern", "negative_damp",
+])
+def test_prune_rejects_bad_arguments(case):
+    L = pp.lib()
+    p = S.Params("2:4").to_c()
+    args = dict(W=FAKE, r=64, d=256, ldw=256, U=FAKE, mask=FAKE)
+    if case == "null_W":
+        args["W"] = None
+    elif case == "bad_din":
+        args["d"] = 250
+        args["ldw"] = 252
+    elif case == "bad_ldw":
+        args["ldw"] = 255
+    elif case == "bad_blocksize":
+        p.blocksize = 100
+    elif case == "bad_sparsity":
+        p = S.Params("unstructured:1.0").to_c()
+    elif case == "nm_unsupported":
+        p = S.Params("4:8").to_c()
+    elif case == "misaligned":
+        args["mask"] = MISALIGNED
+    elif case == "bad_pattern":
+        p.pattern = 7
+    elif case == "negative_damp":
+        p.damp = -0.5
+    st = L.sgpt_prune(args["W"], args["r"], args["d"], args["ldw"], args["U"], ctypes.byref(p),
+                      args["mask"], None, FAKE, 1 << 30, FAKE, None)
+    expected = 6 if case == "nm_unsupported" else 1
+    assert st == expected, (case, st)
+
+
+def test_other_entry_points_validate():
+    L = pp.lib()
+    assert L.sgpt_factor(None, 10, 256, 0.01, FAKE, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_factor(FAKE, 0, 256, 0.01, FAKE, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_factor(FAKE, 10, 256, 0.01, FAKE, FAKE, 16, FAKE, None) == 8     # workspace
+    assert L.sgpt_factor(FAKE, 10, 256, 0.01, FAKE, FAKE + 16, 1 << 30, FAKE, None) == 8
+    assert L.sgpt_hessian_accumulate(FAKE, MISALIGNED, 100, 256, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_hessian_accumulate(FAKE, FAKE, 100, 96 + 8, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_pack24(FAKE, 8, 64, 64, FAKE, FAKE, None, FAKE, None) == 1
+    assert L.sgpt_recon_error(FAKE, FAKE, 8, 64, 60, FAKE, FAKE, None, 0, None) == 1
+    assert L.sgpt_info_clear(None, None) == 1
+    assert L.sgpt_sync_status(None, None) == 1
+    p = S.Params("2:4").to_c()
+    # H and U must not alias; values without meta is an error
+    assert L.sgpt_prune_layer(FAKE, 8, 64, 64, None, 10, FAKE, FAKE, ctypes.byref(p), FAKE, None, None,
+                              None, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_prune_layer(FAKE, 8, 64, 64, None, 10, FAKE, FAKE + 4096, ctypes.byref(p), FAKE, FAKE,
+                              None, None, FAKE, 1 << 30, FAKE, None) == 1
+
+
+def test_python_binding_requires_cuda_tensors():
+    import torch
+    W = torch.zeros(4, 64)
+    with pytest.raises(TypeError):
+        pp.hessian_zero(W)

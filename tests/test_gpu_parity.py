@@ -1,0 +1,258 @@
+"""CUDA path vs the float64 oracle, through the C ABI, on seeded inputs.
+
+Sizes the oracle finishes in seconds that span several 128-tiles and ragged
+tails (d_in not a multiple of 128, d_out not a multiple of 16, token counts
+not a multiple of 64), plus the full OPT-125M-shaped layer (768 x 768,
+262,144 tokens) in the launch configuration the bench times.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import post_pruning_b200 as pp
+from workloads import CONFIGS, LayerSpec, bf16_bits_to_f64, gen_activations, gen_weights
+
+from parity import assert_parity, compare, f32, gpu_prune_layer
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    CONFIGS["layer256"][0],
+    LayerSpec("ragged", d_in=320, d_out=200, n_tok=3000, sigma=1.5, p_out=0.02, f_out=30.0, seed=1),
+    LayerSpec("tall", d_in=128, d_out=1000, n_tok=777, seed=2),
+]
+
+
+def _inputs(spec, device="cpu"):
+    X = gen_activations(spec, device=device)
+    W = gen_weights(spec, device="cpu")
+    return W, X
+
+
+def _oracle_factor(H_sum_f32: np.ndarray, n: int, damp=0.01):
+    H = H_sum_f32.astype(np.float64) * (2.0 / n)
+    Hd, _ = oracle.damp(H, damp)
+    return H, oracle.inverse_cholesky_upper(Hd)
+
+
+# ------------------------------------------------------------ Hessian
+
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
+def test_hessian_matches_oracle(spec):
+    W, X = _inputs(spec)
+    dev = torch.device("cuda")
+    H = torch.zeros(spec.d_in, spec.d_in, device=dev)
+    ws = pp.workspace(spec.d_out, spec.d_in, spec.n_tok)
+    info = pp.new_info()
+    pp.hessian_accumulate(H, X.to(dev), ws, info)
+    pp.raise_on_info(info)
+    Hg = H.cpu().numpy().astype(np.float64)
+    X64 = bf16_bits_to_f64(X).numpy()
+    ref = X64.T @ X64                              # the sum, unscaled
+    absref = np.abs(X64).T @ np.abs(X64)
+    assert np.array_equal(Hg, Hg.T)
+    err = np.abs(Hg - ref)
+    # fp32 accumulation over n tokens of exact bf16 products
+    assert np.all(err <= 1e-5 * absref + 1e-30), float((err / (absref + 1e-30)).max())
+    # streaming: two chunks accumulate to the same matrix
+    h = spec.n_tok // 3 // 64 * 64 + 64
+    H2 = torch.zeros_like(H)
+    pp.hessian_accumulate(H2, X[:h].to(dev).contiguous(), ws, info)
+    pp.hessian_accumulate(H2, X[h:].to(dev).contiguous(), ws, info)
+    pp.raise_on_info(info)
+    assert np.all(np.abs(H2.cpu().numpy() - ref) <= 1e-5 * absref + 1e-30)
+
+
+# ------------------------------------------------------------ factor
+
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
+def test_factor_matches_oracle(spec):
+    W, X = _inputs(spec)
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)           # same fp32 input to both sides
+    H, U_ref = _oracle_factor(Hs, spec.n_tok)
+    dev = torch.device("cuda")
+    Hd = torch.from_numpy(Hs).to(dev)
+    U = torch.empty_like(Hd)
+    ws = pp.workspace(spec.d_out, spec.d_in)
+    info = pp.new_info()
+    pp.factor(Hd, spec.n_tok, 0.01, U, ws, info)
+    pp.raise_on_info(info)
+    Ug = U.cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert np.all(np.diag(Ug) > 0)
+    rel_rows = np.linalg.norm(Ug - U_ref, axis=1) / np.linalg.norm(U_ref, axis=1)
+    assert rel_rows.max() < 1e-4, rel_rows.max()
+    # in place (U aliases H) gives the same factor
+    pp.factor(Hd, spec.n_tok, 0.01, Hd, ws, info)
+    pp.raise_on_info(info)
+    assert torch.equal(Hd, U)
+
+
+# ------------------------------------------------------------ sweep
+
+PATTERNS = [pp.Params("2:4"), pp.Params("2:4", blocksize=32), pp.Params("unstructured:0.5"),
+            pp.Params("unstructured:0.7", blocksize=64)]
+
+
+@pytest.mark.parametrize("p", PATTERNS, ids=lambda p: f"{p.pattern}-b{p.blocksize}")
+@pytest.mark.parametrize("spec", SMALL[:2], ids=lambda s: s.name)
+def test_sweep_matches_oracle_given_H(spec, p):
+    W, X = _inputs(spec)
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)
+    H, U_ref = _oracle_factor(Hs, spec.n_tok)
+    gpu = gpu_prune_layer(W, None, p, H_sum=torch.from_numpy(Hs), n_tok=spec.n_tok)
+    m = compare(gpu, W.numpy().astype(np.float64), H, U_ref, p)
+    assert_parity(m, p)
+
+
+def test_forced_mask_reproduces_oracle():
+    spec = SMALL[1]
+    W, X = _inputs(spec)
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)
+    H, U = _oracle_factor(Hs, spec.n_tok)
+    rng = np.random.default_rng(5)
+    forced = rng.random((spec.d_out, spec.d_in)) < 0.55
+    p = pp.Params("unstructured:0.5", forced=True)
+    gpu = gpu_prune_layer(W, None, p, H_sum=torch.from_numpy(Hs), n_tok=spec.n_tok, forced_mask=forced)
+    ref = oracle.sweep(W.numpy().astype(np.float64), U, "unstructured:0.5", 128, forced_mask=forced)
+    assert np.array_equal(gpu["mask"], forced)
+    assert np.all(gpu["W"][~forced] == 0.0)
+    rel = np.linalg.norm(gpu["W"] - ref["W"]) / np.linalg.norm(ref["W"])
+    assert rel < 1e-4, rel
+    assert np.allclose(gpu["row_loss"], ref["loss"], rtol=1e-3)
+
+
+# ------------------------------------------------------------ end to end
+
+@pytest.mark.parametrize("p", [pp.Params("2:4"), pp.Params("unstructured:0.5")], ids=["2:4", "u50"])
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
+def test_prune_layer_from_X(spec, p):
+    W, X = _inputs(spec)
+    gpu = gpu_prune_layer(W, X, p)
+    X64 = bf16_bits_to_f64(X).numpy()
+    H = oracle.hessian(X64)
+    Hd, _ = oracle.damp(H, 0.01)
+    U = oracle.inverse_cholesky_upper(Hd)
+    m = compare(gpu, W.numpy().astype(np.float64), H, U, p)
+    assert_parity(m, p)
+
+
+def test_full_opt125m_layer_from_X():
+    """The full 768 x 768 layer with 262,144 tokens, as the bench runs it."""
+    spec = CONFIGS["opt125m_768"][0]
+    X = gen_activations(spec, device="cuda")
+    W = gen_weights(spec)
+    X64 = bf16_bits_to_f64(X.cpu()).numpy()
+    H = oracle.hessian(X64)
+    Hd, _ = oracle.damp(H, 0.01)
+    U = oracle.inverse_cholesky_upper(Hd)
+    for run in spec.runs:
+        p = pp.Params(run)
+        gpu = gpu_prune_layer(W, X, p)
+        m = compare(gpu, W.numpy().astype(np.float64), H, U, p)
+        assert_parity(m, p)
+
+
+# ------------------------------------------------------------ properties
+
+def test_24_result_independent_of_blocksize():
+    spec = SMALL[0]
+    W, X = _inputs(spec)
+    a = gpu_prune_layer(W, X, pp.Params("2:4", blocksize=128))
+    b = gpu_prune_layer(W, X, pp.Params("2:4", blocksize=32))
+    assert np.mean(a["mask"] == b["mask"]) > 0.999
+    agree = np.all(a["mask"] == b["mask"], axis=1)
+    rel = np.linalg.norm(a["W"][agree] - b["W"][agree]) / np.linalg.norm(a["W"][agree])
+    assert rel < 1e-4
+
+
+def test_diagonal_hessian_keeps_survivors_bit_exact():
+    """Tokens that each excite one channel give a diagonal H: no compensation."""
+    d, r, n = 256, 64, 4096
+    X = torch.zeros(n, d)
+    g = torch.Generator().manual_seed(3)
+    X[torch.arange(n), torch.arange(n) % d] = torch.randn(n, generator=g) * 3
+    X = X.to(torch.bfloat16)
+    W = torch.randn(r, d, generator=g)
+    gpu = gpu_prune_layer(W, X, pp.Params("2:4"))
+    kept = gpu["mask"]
+    assert np.array_equal(gpu["W"][kept], W.numpy()[kept])
+    X64 = bf16_bits_to_f64(X).numpy()
+    lam = 0.01 * np.mean(np.diag(oracle.hessian(X64)))
+    score = W.numpy().astype(np.float64) ** 2 * (np.diag(oracle.hessian(X64)) + lam)
+    top2 = np.argsort(-score.reshape(r, -1, 4), axis=2, kind="stable")[:, :, :2]
+    want = np.zeros((r, d // 4, 4), dtype=bool)
+    np.put_along_axis(want, top2, True, axis=2)
+    assert np.mean(want.reshape(r, d) == kept) > 0.999
+
+
+def test_deterministic():
+    spec = SMALL[1]
+    W, X = _inputs(spec)
+    a = gpu_prune_layer(W, X, pp.Params("unstructured:0.5"))
+    b = gpu_prune_layer(W, X, pp.Params("unstructured:0.5"))
+    assert np.array_equal(a["W"], b["W"]) and np.array_equal(a["mask"], b["mask"])
+    assert np.array_equal(a["H"], b["H"]) and np.array_equal(a["U"], b["U"])
+
+
+def test_recon_error_matches_oracle():
+    spec = SMALL[1]
+    W, X = _inputs(spec)
+    gpu = gpu_prune_layer(W, X, pp.Params("2:4"))
+    dev = torch.device("cuda")
+    nd = torch.zeros(2, dtype=torch.float64, device=dev)
+    Hd = torch.from_numpy(gpu["H"]).to(dev)
+    pp.recon_error(W.to(dev), torch.from_numpy(gpu["W"]).to(dev), Hd, nd)
+    num, den = nd.cpu().tolist()
+    rnum, rden = oracle.recon_error(W.numpy(), gpu["W"], gpu["H"].astype(np.float64))
+    assert num == pytest.approx(rnum, rel=1e-4)
+    assert den == pytest.approx(rden, rel=1e-5)
+
+
+# ------------------------------------------------------------ error paths
+
+def test_not_positive_definite_is_reported():
+    d, r = 128, 16
+    dev = torch.device("cuda")
+    H = torch.zeros(d, d, device=dev)          # lambda = 0 -> zero pivot
+    U = torch.empty_like(H)
+    ws = pp.workspace(r, d)
+    info = pp.new_info()
+    pp.factor(H, 100, 0.01, U, ws, info)
+    assert pp.sync_status(info) == 2
+    # a later call in the chain leaves its outputs alone
+    W = torch.ones(r, d, device=dev)
+    mask = torch.zeros(r, d // 32, dtype=torch.int32, device=dev)
+    pp.prune(W, U, pp.Params("2:4"), mask, ws, info)
+    assert pp.sync_status(info) == 2
+    assert torch.all(W == 1) and torch.all(mask == 0)
+
+
+def test_nonfinite_is_reported():
+    d = 64
+    dev = torch.device("cuda")
+    H = torch.eye(d, device=dev)
+    H[3, 3] = float("nan")
+    U = torch.empty_like(H)
+    info = pp.new_info()
+    pp.factor(H, 10, 0.01, U, pp.workspace(8, d), info)
+    assert pp.sync_status(info) == 3
+
+
+def test_bad_mask_is_reported():
+    d, r = 64, 8
+    dev = torch.device("cuda")
+    W = torch.randn(r, d, device=dev)
+    mask = torch.full((r, d // 32), -1, dtype=torch.int32, device=dev)     # keeps all 4
+    vals = torch.empty(r, d // 2, device=dev)
+    meta = torch.empty(r, d // 32, dtype=torch.int32, device=dev)
+    info = pp.new_info()
+    pp.pack24(W, mask, vals, meta, info)
+    assert pp.sync_status(info) == 7
