@@ -72,97 +72,188 @@ __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict
 
 // ------------------------------------------------------- diagonal blocks
 //
-// One CTA factors the diagonal block A_kk = R_kk R_kk^T (R_kk upper) in
-// float64 and inverts it: U_kk = R_kk^-1. Layout in shared memory: one
-// 128 x 129 float64 array; R in the strict upper triangle, U transposed in
-// the strict lower triangle (A[j][i] = U[i][j], i < j), diagonals apart.
+// One CTA factors the diagonal block A_kk = R_kk R_kk^T (R_kk upper) and
+// inverts it, U_kk = R_kk^-1, in float64. 256 threads form a 16 x 16 grid;
+// thread (ty, tx) keeps A[i][l] for i = ty + 16a, l = tx + 16c (a, c < 8) in
+// registers (cyclic layout, so the shrinking active triangle stays spread
+// over all threads). Each pivot j costs one barrier: column j of the current
+// matrix is broadcast through a double-buffered shared vector, every thread
+// applies the rank-1 update A[i][l] -= a_ij a_lj / a_jj to its entries with
+// i <= l < j, and the owners of column j-1 publish it for the next pivot.
+// The inverse runs the same way over rows: X[i][.] = B[i][.] / r_ii, then
+// B[l][.] -= r_li X[i][.] for l < i, with B = I initially and R in shared
+// memory.
 
-constexpr int kDiagThreads = 512;
+constexpr int kDiagThreads = 256;
 constexpr int kDiagLd = kTile + 1;
-constexpr size_t kDiagSmem = (size_t)kTile * kDiagLd * sizeof(double) + 2 * kTile * sizeof(double);
+constexpr size_t kDiagSmem = (size_t)kTile * kDiagLd * sizeof(double);
 
-__global__ void __launch_bounds__(kDiagThreads) diag_factor_kernel(const float* __restrict__ Rws,
-                                                                   int d, int k,
-                                                                   float* __restrict__ Ukk,
-                                                                   float* __restrict__ U,
-                                                                   int* info) {
+__global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const float* __restrict__ Rws,
+                                                                      int d, int k,
+                                                                      float* __restrict__ Ukk,
+                                                                      float* __restrict__ U,
+                                                                      int* info) {
   if (cta_info_set(info)) return;
-  extern __shared__ double sm[];
-  double* A = sm;                        // [128][129]
-  double* dR = sm + kTile * kDiagLd;     // R_ii
-  double* dU = dR + kTile;               // U_ii
+  extern __shared__ double Rs[];            // [128][129], R after the factorisation
+  __shared__ double vec[2][kTile];          // broadcast column (factor) / row (inverse)
+  __shared__ double piv[2][3];              // 1/a_jj, 1/sqrt(a_jj), sqrt(a_jj)
   __shared__ int bad;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int b0 = k * kTile;
   const int b = min(kTile, d - b0);
-  for (int idx = tid; idx < b * b; idx += kDiagThreads) {
-    const int i = idx / b, j = idx - (idx / b) * b;
-    if (i <= j) A[i * kDiagLd + j] = (double)Rws[(long long)(b0 + i) * d + b0 + j];
-  }
+  double r[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = ty + 16 * a, l = tx + 16 * c;
+      r[a][c] = (i <= l && l < b) ? (double)Rws[(long long)(b0 + i) * d + b0 + l] : 0.0;
+    }
   if (tid == 0) bad = 0;
   __syncthreads();
 
-  // Reverse Cholesky: for j = b-1 .. 0: r_jj = sqrt(a_jj); r_ij = a_ij / r_jj
-  // (i < j); a_il -= r_ij r_lj for i <= l < j.
-  const int ty = tid >> 5, tx = tid & 31;   // 16 x 32 thread grid
-  for (int j = b - 1; j >= 0; --j) {
-    if (tid == 0) {
-      const double piv = A[j * kDiagLd + j];
-      if (!(piv > 0.0)) bad = isfinite(piv) ? (b0 + j + 1) : SGPT_INFO_NONFINITE;
-      else dR[j] = sqrt(piv);
+  // publish column j (entries i <= j) and its pivot into buffer p
+  auto publish_col = [&](int j, int p) {
+    if (tx != (j & 15)) return;
+    const int cj = j >> 4;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (c != cj) continue;
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const int i = ty + 16 * a;
+        if (i > j) continue;
+        vec[p][i] = r[a][c];
+        if (i == j) {
+          const double pv = r[a][c];
+          if (!(pv > 0.0)) {
+            bad = isfinite(pv) ? (b0 + j + 1) : SGPT_INFO_NONFINITE;
+            piv[p][0] = piv[p][1] = piv[p][2] = 0.0;
+          } else {
+            const double sq = sqrt(pv);
+            piv[p][0] = 1.0 / pv;
+            piv[p][1] = 1.0 / sq;
+            piv[p][2] = sq;
+          }
+        }
+      }
     }
+  };
+
+  publish_col(b - 1, 0);
+  for (int j = b - 1, p = 0; j >= 0; --j, p ^= 1) {
     __syncthreads();
     if (bad) {
       if (tid == 0) set_info(info, bad);
       return;
     }
-    const double rjj = dR[j];
-    for (int i = tid; i < j; i += kDiagThreads) A[i * kDiagLd + j] /= rjj;
-    __syncthreads();
-    for (int i = ty; i < j; i += 16) {
-      const double rij = A[i * kDiagLd + j];
-      for (int l = i + tx; l < j; l += 32) A[i * kDiagLd + l] -= rij * A[l * kDiagLd + j];
+    const double pinv = piv[p][0], rs = piv[p][1], sq = piv[p][2];
+    double ci[8], cl[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      const int i = ty + 16 * a;
+      ci[a] = i <= j ? vec[p][i] * pinv : 0.0;
     }
-    __syncthreads();
-  }
-
-  // Inverse, bottom row first: X[i][j] = B[i][j] / r_ii (j >= i), then
-  // B[l][j] -= r_li X[i][j] for l < i <= j. B starts as the identity.
-  for (int idx = tid; idx < b * b; idx += kDiagThreads) {
-    const int i = idx / b, j = idx - (idx / b) * b;
-    if (i > j) A[i * kDiagLd + j] = 0.0;
-  }
-  for (int i = tid; i < b; i += kDiagThreads) dU[i] = 1.0;
-  __syncthreads();
-  for (int i = b - 1; i >= 0; --i) {
-    const double inv = 1.0 / dR[i];
-    for (int j = i + tid; j < b; j += kDiagThreads) {
-      if (j == i) dU[i] *= inv;
-      else A[j * kDiagLd + i] *= inv;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int l = tx + 16 * c;
+      cl[c] = l <= j ? vec[p][l] : 0.0;
     }
-    __syncthreads();
-    // rows l < i, columns j >= i
-    for (int l = ty; l < i; l += 16) {
-      const double rli = A[l * kDiagLd + i];
-      for (int j = i + tx; j < b; j += 32) {
-        const double x = (j == i) ? dU[i] : A[j * kDiagLd + i];
-        A[j * kDiagLd + l] -= rli * x;
+    // rank-1 update of the leading j x j upper triangle
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      const int i = ty + 16 * a;
+      if (i >= j) continue;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int l = tx + 16 * c;
+        if (l >= i && l < j) r[a][c] = fma(-ci[a], cl[c], r[a][c]);
       }
     }
+    // column j becomes column j of R
+    if (tx == (j & 15)) {
+      const int cj = j >> 4;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c != cj) continue;
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          const int i = ty + 16 * a;
+          if (i < j) r[a][c] *= rs;
+          else if (i == j) r[a][c] = sq;
+        }
+      }
+    }
+    if (j > 0) publish_col(j - 1, p ^ 1);
+  }
+
+  // R to shared memory; registers become B = I
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = ty + 16 * a, l = tx + 16 * c;
+      Rs[i * kDiagLd + l] = (i <= l && l < b) ? r[a][c] : 0.0;
+      r[a][c] = (i == l && i < b) ? 1.0 : 0.0;
+    }
+
+  // publish row i of X = B[i][.] / r_ii (entries j >= i) into buffer p; the
+  // owners keep X in their registers.
+  auto publish_row = [&](int i, int p) {
+    if (ty != (i & 15)) return;
+    const int ai = i >> 4;
+    const double inv = 1.0 / Rs[i * kDiagLd + i];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      if (a != ai) continue;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int l = tx + 16 * c;
+        if (l < i || l >= b) continue;
+        r[a][c] *= inv;
+        vec[p][l] = r[a][c];
+      }
+    }
+  };
+
+  __syncthreads();
+  publish_row(b - 1, 0);
+  for (int i = b - 1, p = 0; i > 0; --i, p ^= 1) {
     __syncthreads();
+    double xr[8], rc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int l = tx + 16 * c;
+      xr[c] = (l >= i && l < b) ? vec[p][l] : 0.0;
+    }
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      const int row = ty + 16 * a;
+      rc[a] = row < i ? Rs[row * kDiagLd + i] : 0.0;
+    }
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      const int row = ty + 16 * a;
+      if (row >= i) continue;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int l = tx + 16 * c;
+        if (l >= i && l < b) r[a][c] = fma(-rc[a], xr[c], r[a][c]);
+      }
+    }
+    publish_row(i - 1, p ^ 1);
   }
 
   // Write U_kk (upper, zeros below) to the output and to the block cache.
-  for (int idx = tid; idx < kTile * kTile; idx += kDiagThreads) {
-    const int i = idx >> 7, j = idx & 127;
-    float v = 0.f;
-    if (i < b && j < b) {
-      if (i == j) v = (float)dU[i];
-      else if (i < j) v = (float)A[j * kDiagLd + i];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = ty + 16 * a, l = tx + 16 * c;
+      const float v = (i <= l && l < b) ? (float)r[a][c] : 0.f;
+      Ukk[i * kTile + l] = v;
+      if (i < b && l < b) U[(long long)(b0 + i) * d + b0 + l] = v;
     }
-    Ukk[idx] = v;
-    if (i < b && j < b) U[(long long)(b0 + i) * d + b0 + j] = v;
-  }
 }
 
 // ------------------------------------------------- off-diagonal products

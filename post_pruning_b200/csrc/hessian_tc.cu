@@ -315,9 +315,10 @@ struct Plan {
 Plan plan(int d, long long n) {
   const int tm = (d + kM - 1) / kM, tn = (d + kN - 1) / kN;
   const int tiles = (int)band_start(tm, tn);
-  // split tokens when the tiles alone cannot fill the GPU
+  // split tokens when the tiles alone cannot fill the GPU, keeping the grid
+  // within one wave (one CTA per SM: the stages take most of shared memory)
   long long ns = 1;
-  if (tiles < kNumSMs) ns = (kNumSMs + tiles - 1) / tiles;
+  if (tiles < kNumSMs) ns = kNumSMs / tiles;
   const long long max_split = (n + 4 * kBK - 1) / (4 * kBK);   // >= 4 stages per split
   ns = std::max<long long>(1, std::min(ns, max_split));
   long long per = ((n + ns - 1) / ns + kBK - 1) / kBK * kBK;
