@@ -139,6 +139,28 @@ sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U,
                        const sgpt_params* p, uint32_t* mask_bits, float* row_loss,
                        void* ws, size_t ws_bytes, int* dev_info, void* stream);
 
+/* Allocation-free variant of sgpt_prune. No counterpart in the pages: it
+ * exists for callers that cannot provide device memory at the call site -
+ * for instance code running in a framework plugin or a real-time loop whose
+ * execution path forbids allocation, or a process whose device memory is
+ * wholly owned by another allocator - and so cannot pass the workspace
+ * sgpt_prune needs. Same arguments, results and device-status behaviour as
+ * sgpt_prune, minus ws/ws_bytes: the scratch (the d_out x 128 fp32 error
+ * block and the selection state, about 4 MiB) lives in a fixed device array
+ * inside the library, which every GPU that loads the library keeps until
+ * the process exits. The library allocates nothing here.
+ *   - d_out must not exceed SGPT_NOALLOC_MAX_ROWS (else SGPT_ERR_INVALID_ARG).
+ *   - The first call on each device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race and must be serialised by the
+ *     caller. Nothing in the array needs clearing between calls. */
+#define SGPT_NOALLOC_MAX_ROWS 8192
+sgpt_status sgpt_prune_noalloc(float* W, int d_out, int d_in, int ldw, const float* U,
+                               const sgpt_params* p, uint32_t* mask_bits, float* row_loss,
+                               int* dev_info, void* stream);
+
 /* 2:4 packing (2:4 production guide, section on the 2:4 mechanism):
  *   values [d_out x d_in/2] fp32: the two kept weights of each group of four,
  *          in column order;

@@ -22,6 +22,7 @@ from .sgpt import (  # noqa: F401
     pack24,
     prune,
     prune_layer,
+    prune_noalloc,
     raise_on_info,
     recon_error,
     sync_status,

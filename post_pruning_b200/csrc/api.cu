@@ -145,6 +145,19 @@ sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U, c
                                 as_stream(stream)));
 }
 
+sgpt_status sgpt_prune_noalloc(float* W, int d_out, int d_in, int ldw, const float* U, const sgpt_params* p,
+                               uint32_t* mask_bits, float* row_loss, int* dev_info, void* stream) {
+  if (!W || !U || !mask_bits || !dev_info || !aligned16(W) || !aligned16(U) || !aligned16(mask_bits))
+    return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  if (d_out > SGPT_NOALLOC_MAX_ROWS) return SGPT_ERR_INVALID_ARG;
+  if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
+  sgpt_status s = check_params(p);
+  if (s != SGPT_OK) return s;
+  return from_cuda(launch_prune_noalloc(W, d_out, d_in, ldw, U, *p, mask_bits, row_loss, dev_info,
+                                        as_stream(stream)));
+}
+
 sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint32_t* mask_bits,
                         float* values, uint32_t* meta, int* dev_info, void* stream) {
   if (!W || !mask_bits || !values || !meta || !dev_info) return SGPT_ERR_INVALID_ARG;

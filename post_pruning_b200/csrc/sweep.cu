@@ -13,6 +13,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
@@ -274,6 +275,97 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
   Carve c(ws);
   float* Err = c.take<float>((size_t)rows * kMaxBlock);
   SelState* sel = c.take<SelState>(1);
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(sweep_kernel<kModeNM24>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    cudaFuncSetAttribute(sweep_kernel<kModeThreshold>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    cudaFuncSetAttribute(sweep_kernel<kModeForced>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    attr_done = true;
+  }
+  const int B = p.blocksize;
+  const int sweep_grid = cdiv(rows, kSweepRows);
+  for (int i1 = 0; i1 < d; i1 += B) {
+    const int bw = min(B, d - i1);
+    if (p.forced) {
+      sweep_kernel<kModeForced><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+      count_launches(1);
+    } else if (p.pattern == SGPT_PATTERN_NM) {
+      sweep_kernel<kModeNM24><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+      count_launches(1);
+    } else {
+      const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
+      select_init_kernel<<<1, 256, 0, st>>>(sel, (unsigned int)kk);
+      count_launches(1);
+      const long long total4 = (long long)rows * (bw / 4);
+      const int g = (int)std::min<long long>(cdivll(total4, 256 * 8), 4 * kNumSMs);
+      for (int pass = 0; pass < 8; ++pass) {
+        select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, sel, pass, info);
+        count_launches(1);
+      }
+      sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, &sel->thr, info);
+      count_launches(1);
+    }
+    const int i2 = i1 + bw;
+    if (i2 < d) {
+      dim3 grid(cdiv(d - i2, kTile), cdiv(rows, kTile));
+      trailing_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(W, ldw, rows, d, i1, bw, U, Err, info);
+      count_launches(1);
+    }
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------ allocation-free variant
+//
+// sgpt_prune needs scratch for the error block of the current OBS block
+// (d_out x 128 fp32) and for the selection state. The allocation-free entry
+// takes that scratch from the fixed device array below instead of a caller
+// workspace. Every device that loads this library holds the array until the
+// process exits. All calls share it, so calls that overlap on the GPU (two
+// streams, or two host threads) race; nothing in it has to start at zero
+// (the error block is written before it is read and the selection state is
+// re-initialised for every block).
+
+constexpr size_t kNoAllocErrBytes = (size_t)SGPT_NOALLOC_MAX_ROWS * kMaxBlock * sizeof(float);
+constexpr size_t kNoAllocScratchBytes = kNoAllocErrBytes + 4096;
+static_assert(sizeof(SelState) <= 4096, "selection state must fit the scratch tail");
+
+static __device__ __align__(256) unsigned char g_prune_scratch[kNoAllocScratchBytes];
+
+// In host code g_prune_scratch names a host-side stand-in, not device memory;
+// the device address must come from cudaGetSymbolAddress with the device
+// current. It is looked up once per device, on the first call there.
+static std::mutex g_scratch_mu;
+static void* g_scratch_addr[256];
+
+static cudaError_t prune_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_prune_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const float* U,
+                                 const sgpt_params& p, uint32_t* mask, float* row_loss, int* info,
+                                 cudaStream_t st) {
+  if (rows > SGPT_NOALLOC_MAX_ROWS) return cudaErrorInvalidValue;
+  void* base = nullptr;
+  cudaError_t e = prune_scratch(&base);
+  if (e != cudaSuccess) return e;
+  float* Err = static_cast<float*>(base);
+  SelState* sel = reinterpret_cast<SelState*>(static_cast<char*>(base) + kNoAllocErrBytes);
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(sweep_kernel<kModeNM24>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);

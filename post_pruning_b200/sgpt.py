@@ -30,7 +30,7 @@ PATTERN_NM = 1
 EXPORTS = (
     "sgpt_status_string", "sgpt_abi_version", "sgpt_kernel_launches", "sgpt_workspace_bytes",
     "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
-    "sgpt_hessian_accumulate", "sgpt_factor", "sgpt_prune", "sgpt_pack24",
+    "sgpt_hessian_accumulate", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
     "sgpt_recon_error", "sgpt_prune_layer",
 )
 
@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "sgpt_hessian_accumulate": (i32, [vp, vp, i64, i32, vp, sz, vp, vp]),
         "sgpt_factor": (i32, [vp, i64, i32, ctypes.c_float, vp, vp, sz, vp, vp]),
         "sgpt_prune": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, sz, vp, vp]),
+        "sgpt_prune_noalloc": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, vp]),
         "sgpt_pack24": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
         "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
@@ -216,6 +217,29 @@ def prune(W: torch.Tensor, U: torch.Tensor, params: Params, mask: torch.Tensor, 
     p = params.to_c()
     _check(lib().sgpt_prune(_ptr(W), r, d, ldw, _ptr(U), ctypes.byref(p), _ptr(mask), _ptr(row_loss),
                             _ptr(ws), ws.numel(), _ptr(dev_info), _stream(stream)), "sgpt_prune")
+
+
+NOALLOC_MAX_ROWS = 8192
+
+
+def prune_noalloc(W: torch.Tensor, U: torch.Tensor, params: Params, mask: torch.Tensor,
+                  dev_info: torch.Tensor, row_loss: torch.Tensor | None = None, stream=None):
+    """sgpt_prune without a workspace, for callers that cannot allocate device
+    memory where they call it: the scratch is a fixed array inside the library
+    (d_out <= NOALLOC_MAX_ROWS). Calls that overlap on the GPU race on it."""
+    _dev(W, torch.float32, "W")
+    _dev(U, torch.float32, "U")
+    _dev(mask, torch.int32, "mask")
+    ldw = _rowmajor(W, "W")
+    r, d = W.shape
+    if mask.shape != (r, d // 32) or not mask.is_contiguous():
+        raise ValueError("mask must be contiguous int32 [d_out, d_in/32]")
+    if row_loss is not None:
+        _dev(row_loss, torch.float32, "row_loss")
+    p = params.to_c()
+    _check(lib().sgpt_prune_noalloc(_ptr(W), r, d, ldw, _ptr(U), ctypes.byref(p), _ptr(mask),
+                                    _ptr(row_loss), _ptr(dev_info), _stream(stream)),
+           "sgpt_prune_noalloc")
 
 
 def pack24(W: torch.Tensor, mask: torch.Tensor, values: torch.Tensor, meta: torch.Tensor,
