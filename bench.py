@@ -31,19 +31,31 @@ sys.path.insert(0, ROOT)
 METRIC = "SparseGPT per-layer prune time & weights/s on 1 B200; % of HBM/tensor roofline"
 UNIT = "weights/s"
 CONFIG = "opt125m_768"
+WORKLOADS = {
+    "layer256": "256x256 layer, 2048 tokens, 2:4",
+    "llama7b_down": ("Llama-7B MLP down-proj: W 4096x11008 fp32, X 131072x11008 bf16 (lognormal sigma=1.5, "
+                     "0.5% outlier channels x50), 2:4"),
+    "llama7b_q": ("Llama-7B q_proj: W 4096x4096 fp32, X 262144x4096 bf16, unstructured 50/70/80% "
+                  "(three layer prunes per step)"),
+    "qwen3_32b_block": ("Qwen3-32B-shaped block: q 5120->8192, k/v 5120->1024, o 8192->5120, gate/up "
+                        "5120->25600, down 25600->5120, 131072 tokens, 2:4; H and U shared by q/k/v and by "
+                        "gate/up (4 Hessians, 7 sweeps per step)"),
+}
 WORKLOAD = ("OPT-125M-shaped linear layer: W 768x768 fp32 ~N(0,1/768); X 262144x768 bf16 "
             "(128 seqs x 2048 tokens, lognormal(sigma=1) channel scales, 1% outlier channels x20); "
             "two layer prunes per step from X: 2:4 and unstructured 50%; blocksize 128; damp 0.01")
+WORKLOADS[CONFIG] = WORKLOAD
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", default=CONFIG, help="workload (default: the OPT-125M-shaped layer)")
     return ap.parse_args()
 
 
@@ -78,7 +90,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"],
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -173,14 +185,33 @@ def reference_arm(args, spec):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ ranks
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time: every rank contributes its own device time and
+    all ranks receive the maximum (one all-reduce, outside the timed region)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(weights_per_rank_step: int, steps: int, world: int, t_slowest: float) -> dict:
+    """Whole-job throughput of `world` replicas (weak scaling): all ranks'
+    units over the slowest rank's time."""
+    total = weights_per_rank_step * steps * world
+    return {"value": total / t_slowest, "ms_per_step": t_slowest * 1e3 / steps}
+
+
 # ------------------------------------------------------------------ native
 
 def main():
     args = parse()
     from workloads import CONFIGS
-    spec = CONFIGS[CONFIG][0]
     if args.impl == "reference":
-        reference_arm(args, spec)
+        reference_arm(args, CONFIGS[CONFIG][0])
         return
 
     import torch
@@ -199,38 +230,59 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     stream = torch.cuda.current_stream()
-    X = gen_activations(spec, device=dev)
-    W0 = gen_weights(spec, device=dev)
-    runs = [pp.Params(r) for r in spec.runs]
-    r, d, n = spec.d_out, spec.d_in, spec.n_tok
-    bufs = [pp.LayerBuffers.allocate(r, d, n, dev) for _ in runs]
-    Ws = [W0.clone() for _ in runs]
+    # A job is one activation input: its Hessian and factor are computed once,
+    # then every weight matrix reading that input is swept (and 2:4 packed).
+    # The OPT-125M workload prunes its layer twice from X (one job per run);
+    # the Qwen3-32B block has four inputs shared by q/k/v, o, gate/up, down.
+    jobs = []
+    specs = CONFIGS[args.config]
+    if len(specs) == 1:
+        sp = specs[0]
+        X = gen_activations(sp, device=dev)
+        for run in sp.runs:
+            jobs.append((sp, X, [(sp, pp.Params(run))]))
+    else:
+        by_x = {}
+        for sp in specs:
+            by_x.setdefault(sp.x_key, []).append(sp)
+        for key, group in by_x.items():
+            X = gen_activations(group[0], device=dev)
+            jobs.append((group[0], X, [(sp, pp.Params(sp.runs[0])) for sp in group]))
+    layers = []      # (W0, W, LayerGraphs)
+    job_graphs = []
+    for xs, X, mats in jobs:
+        first = None
+        gl = []
+        for sp, p in mats:
+            W0 = gen_weights(sp, device=dev)
+            W = W0.clone()
+            if first is None:
+                b = pp.LayerBuffers.allocate(sp.d_out, sp.d_in, xs.n_tok, dev)
+                g = pp.LayerGraphs(b, W, X, p)
+                first = b
+            else:
+                b = pp.LayerBuffers.sharing(first, sp.d_out, dev)
+                g = pp.LayerGraphs(b, W, None, p, phases=("prune", "pack"))
+            layers.append((W0, W, g))
+            gl.append(g)
+        job_graphs.append(gl)
+    weights_per_step = sum(sp.weights for _, _, mats in jobs for sp, _ in mats)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    PH = pp.LayerGraphs.PHASES
 
     def one_step(ev=None):
-        for k, (p, b, W) in enumerate(zip(runs, bufs, Ws)):
-            info = b.info
-            pp.info_clear(info)
-            if ev is not None:
-                ev[k][0].record(stream)
-            pp.hessian_zero(b.H)
-            pp.hessian_accumulate(b.H, X, b.ws, info)
-            if ev is not None:
-                ev[k][1].record(stream)
-            pp.factor(b.H, n, p.damp, b.U, b.ws, info)
-            if ev is not None:
-                ev[k][2].record(stream)
-            b.row_loss.zero_()
-            pp.prune(W, b.U, p, b.mask, b.ws, info, row_loss=b.row_loss)
-            if ev is not None:
-                ev[k][3].record(stream)
-            if p.is_nm:
-                pp.pack24(W, b.mask, b.values, b.meta, info)
-            if ev is not None:
-                ev[k][4].record(stream)
+        # ev[j][phase] pairs of events around every graph of job j
+        for j, gl in enumerate(job_graphs):
+            for g in gl:
+                for name in g.phases:
+                    if ev is not None:
+                        ev[j][name][0].record(stream)
+                    g.graphs[name].replay()
+                    if ev is not None:
+                        ev[j][name][1].record(stream)
 
     def prep():
-        for W in Ws:
+        for W0, W, _ in layers:
             W.copy_(W0)
         flush.zero_()
 
@@ -238,67 +290,83 @@ def main():
         prep()
         one_step()
     torch.cuda.synchronize()
-    for b in bufs:
-        pp.raise_on_info(b.info, where="warm-up")
+    for _, _, g in layers:
+        pp.raise_on_info(g.bufs.info, where="warm-up")
 
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in runs] for _ in range(args.steps)]
+    def mk():
+        return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    # one event pair per (job, phase); graphs of the same phase in a job share it
+    evs = [[{name: mk() for name in PH} for _ in job_graphs] for _ in range(args.steps)]
+    step_ev = [mk() for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(0.3)               # let the sampler produce its first line
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = pp.kernel_launches()
     wall0 = time.perf_counter()
-    for s in range(args.steps):
+    phase = {name: 0.0 for name in PH}
+    for s_ in range(args.steps):
         prep()
-        one_step(evs[s])
+        step_ev[s_][0].record(stream)
+        for j, gl in enumerate(job_graphs):
+            for name in PH:
+                e0, e1 = evs[s_][j][name]
+                ran = False
+                for g in gl:
+                    if name in g.graphs:
+                        if not ran:
+                            e0.record(stream)
+                            ran = True
+                        g.graphs[name].replay()
+                if ran:
+                    e1.record(stream)
+        step_ev[s_][1].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
-    launches = pp.kernel_launches() - launches0
+    launches = pp.kernel_launches() - launches0 + args.steps * sum(sum(g.kernels.values()) for _, _, g in layers)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    for b in bufs:
-        pp.raise_on_info(b.info, where="timed steps")
+    for _, _, g in layers:
+        pp.raise_on_info(g.bufs.info, where="timed steps")
 
-    # per-step device time and phase breakdown
-    step_ms = [sum(e[k][0].elapsed_time(e[k][4]) for k in range(len(runs))) for e in evs]
-    phase = {"hessian": 0.0, "factor": 0.0, "sweep": 0.0, "pack": 0.0}
-    names = list(phase)
-    for e in evs:
-        for k in range(len(runs)):
-            for j, nm in enumerate(names):
-                phase[nm] += e[k][j].elapsed_time(e[k][j + 1])
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    for s_ in range(args.steps):
+        for j, gl in enumerate(job_graphs):
+            for name in PH:
+                if any(name in g.graphs for g in gl):
+                    e0, e1 = evs[s_][j][name]
+                    phase[name] += e0.elapsed_time(e1)
     phase = {k: v / args.steps for k, v in phase.items()}
-    t_rank = sum(step_ms) / 1e3
-    if world > 1:
-        t = torch.tensor([t_rank], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_rank = float(t.item())
-    weights = spec.weights * len(runs) * args.steps * world
-    value = weights / t_rank
-    ms_per_step = t_rank * 1e3 / args.steps
+    t_rank = max_over_ranks(sum(step_ms) / 1e3, dist if world > 1 else None, dev)
+    agg = aggregate(weights_per_step, args.steps, world, t_rank)
+    value, ms_per_step = agg["value"], agg["ms_per_step"]
+    spec = jobs[0][0]
+    n_hess = len(jobs)
+    n, d = spec.n_tok, spec.d_in
 
-    # roofline of the dominant kernel: the tensor-core Hessian (one launch per run)
+    # roofline of the dominant kernel: the tensor-core Hessian (one launch per job)
     hbm, bf16_burst, bf16_sust, peak_kind = peaks()
-    hess_ms = phase["hessian"] / len(runs)
-    hess_flops = n * d * (d + 1)            # the symmetric half X^T X needs
-    achieved = hess_flops / (hess_ms * 1e-3) / 1e12
+    hess_flops = sum(xs.n_tok * xs.d_in * (xs.d_in + 1) for xs, _, _ in jobs)
+    achieved = hess_flops / (phase["hessian"] * 1e-3) / 1e12
     roofline = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": achieved,
                 "peak": bf16_burst, "unit": "TFLOP/s", "frac": achieved / bf16_burst,
                 "traffic": None, "peak_kind": f"{peak_kind} bf16 burst",
-                "work": f"n*d*(d+1) = {hess_flops:.4g} flop per launch (upper triangle incl. diagonal)"}
+                "work": f"n*d*(d+1) = {hess_flops / n_hess:.4g} flop per launch (upper triangle incl. "
+                        f"diagonal), {n_hess} launches per step"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "input_dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "per_gpu_layers_per_step": len(runs),
-                   "l2": "flushed between steps (256 MiB write, untimed); X is 403 MB > 126 MB L2",
+        "config": {"workload": WORKLOADS.get(args.config, args.config), "name": args.config,
+                   "weights_per_step": weights_per_step,
+                   "launch": "each phase of each layer replayed as a captured CUDA graph",
+                   "l2": "flushed between steps (256 MiB write, untimed); every X exceeds the 126 MB L2",
                    "parallelism": f"replicas x{world}"},
-        "per_layer_ms": {p.pattern: sum(e[k][0].elapsed_time(e[k][4]) for e in evs) / args.steps
-                         for k, p in enumerate(runs)},
         "phases_ms_per_step": phase,
         "roofline": roofline,
         "gpu_launches": launches,
@@ -306,38 +374,40 @@ def main():
         "wall_s_timed": wall,
     }
 
-    # end to end through the public API with host buffers (rank-local)
-    if not args.no_e2e:
-        hp = [pp.HostPruner(r, d, n, dev) for _ in runs]
-        X_host = X.cpu().pin_memory()
-        W_host = W0.cpu().pin_memory()
+    # end to end through the public API with host buffers (rank-local), for
+    # workloads whose layers each read their own input
+    single = all(len(m) == 1 for _, _, m in jobs)
+    if not args.no_e2e and single:
+        hp = [(pp.HostPruner(sp.d_out, sp.d_in, xs.n_tok, dev), p, xs, sp) for xs, _, ((sp, p),) in jobs]
+        X_host = {id(X): X.cpu().pin_memory() for _, X, _ in jobs}
+        W_host = [layers[k][0].cpu().pin_memory() for k in range(len(layers))]
+        xs_of = [X for _, X, _ in jobs]
+
+        def e2e_step():
+            for k, (h, p, xs, sp) in enumerate(hp):
+                h.enqueue(W_host[k], X_host[id(xs_of[k])], p)
+
         for _ in range(max(1, args.warmup // 2)):
-            for p, h in zip(runs, hp):
-                h.enqueue(W_host, X_host, p)
+            e2e_step()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ks = max(1, args.steps // 2)
         e0.record(stream)
         for _ in range(ks):
-            for p, h in zip(runs, hp):
-                h.enqueue(W_host, X_host, p)
+            e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        for h in hp:
+        for h, _, _, _ in hp:
             pp.raise_on_info(h.bufs.info, where="e2e")
-        t_e2e = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_e2e = float(t.item())
-        line["e2e"] = {"value": spec.weights * len(runs) * ks * world / t_e2e, "unit": UNIT,
-                       "h2d_bytes_per_step": sum(h.h2d_bytes() for h in hp),
-                       "d2h_bytes_per_step": sum(h.d2h_bytes(p) for h, p in zip(hp, runs)),
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
+        line["e2e"] = {"value": weights_per_step * ks * world / t_e2e, "unit": UNIT,
+                       "h2d_bytes_per_step": sum(h.h2d_bytes() for h, _, _, _ in hp),
+                       "d2h_bytes_per_step": sum(h.d2h_bytes(p) for h, p, _, _ in hp),
                        "ms_per_step": t_e2e * 1e3 / ks,
-                       "note": "each run copies W and X from pinned host memory and its results back"}
+                       "note": "each layer prune copies W and X from pinned host memory and its results back"}
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, t, cores, sample = cpu_baseline(spec, X[:32768].cpu(), W0.cpu())
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and len(specs) == 1:
+        v, t, cores, sample = cpu_baseline(spec, jobs[0][1][:32768].cpu(), layers[0][0].cpu())
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": sample, "seconds": t}
     if world > 1:

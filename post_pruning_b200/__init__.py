@@ -10,6 +10,7 @@ from .sgpt import (  # noqa: F401
     HostPruner,
     LIB_PATH,
     LayerBuffers,
+    LayerGraphs,
     Params,
     SgptError,
     factor,

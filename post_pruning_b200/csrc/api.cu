@@ -78,7 +78,7 @@ uint64_t sgpt_kernel_launches(void) { return sgpt::g_launches.load(std::memory_o
 size_t sgpt_workspace_bytes(int d_out, int d_in, int64_t n_tok, const sgpt_params* p) {
   (void)p;
   if (!valid_din(d_in) || !valid_dout(d_out) || n_tok < 0) return 0;
-  size_t need = std::max(factor_ws_bytes(d_in), prune_ws_bytes(d_out));
+  size_t need = std::max(factor_ws_bytes(d_in), prune_ws_bytes(d_out, d_in));
   if (n_tok > 0) need = std::max(need, hessian_ws_bytes(d_in, n_tok));
   return need;
 }
@@ -139,7 +139,7 @@ sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U, c
   if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
   sgpt_status s = check_params(p);
   if (s != SGPT_OK) return s;
-  s = check_ws(ws, ws_bytes, prune_ws_bytes(d_out));
+  s = check_ws(ws, ws_bytes, prune_ws_bytes(d_out, d_in));
   if (s != SGPT_OK) return s;
   return from_cuda(launch_prune(W, d_out, d_in, ldw, U, *p, mask_bits, row_loss, ws, dev_info,
                                 as_stream(stream)));

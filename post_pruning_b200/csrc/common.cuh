@@ -56,6 +56,13 @@ __device__ __forceinline__ float saliency(float w, float u) {
   return __fmul_rn(t, t);
 }
 
+// x rounded to TF32 (10 explicit mantissa bits, ties away from zero); the
+// remainder x - tf32_hi(x) is exact in fp32. Used to split fp32 operands into
+// the hi/lo planes of the three-product tensor-core GEMM.
+__device__ __forceinline__ float tf32_hi(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
+}
+
 // Host-side count of kernel launches (diagnostics, sgpt_kernel_launches).
 void count_launches(unsigned long long n);
 

@@ -10,12 +10,15 @@
 // the sweep consumes it.
 //
 // Blocking: 128 x 128 tiles. Diagonal blocks are factored and inverted in
-// float64 in shared memory by one CTA; all off-diagonal work (panel solve,
-// rank-128 updates, triangular inverse) runs as FP32 SIMT tile products.
+// shared memory by one CTA; the panel solve and the V scaling are FP32 SIMT
+// tile products; the rank-128 updates of the leading part and the
+// triangular inverse (the d^3/3 + d^3/3 flops) run on the tensor cores as
+// FP32-accurate three-product TF32 GEMMs (gemm_tc.cu).
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.h"
 #include "kernels.h"
 
 namespace sgpt {
@@ -73,20 +76,41 @@ __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict
 // ------------------------------------------------------- diagonal blocks
 //
 // One CTA factors the diagonal block A_kk = R_kk R_kk^T (R_kk upper) and
-// inverts it, U_kk = R_kk^-1, in float64. 256 threads form a 16 x 16 grid;
-// thread (ty, tx) keeps A[i][l] for i = ty + 16a, l = tx + 16c (a, c < 8) in
-// registers (cyclic layout, so the shrinking active triangle stays spread
-// over all threads). Each pivot j costs one barrier: column j of the current
-// matrix is broadcast through a double-buffered shared vector, every thread
-// applies the rank-1 update A[i][l] -= a_ij a_lj / a_jj to its entries with
-// i <= l < j, and the owners of column j-1 publish it for the next pivot.
-// The inverse runs the same way over rows: X[i][.] = B[i][.] / r_ii, then
-// B[l][.] -= r_li X[i][.] for l < i, with B = I initially and R in shared
-// memory.
+// inverts it, U_kk = R_kk^-1, in FP32 shared memory. The block is treated as
+// up to 4 x 4 sub-blocks of 32 (width b = 32..128), processed from the last
+// 32-panel to the first:
+//   1. warp 0 factors the 32 x 32 diagonal sub-block D_pp = R_pp R_pp^T (lane
+//      = row, pivots broadcast by shuffles, no CTA barrier) and inverts R_pp
+//      (lane = column, back substitution against R_pp in shared memory);
+//   2. panel: R_ip = A_ip U_pp^T for the sub-blocks above (one warp each);
+//   3. update: A_ij -= R_ip R_jp^T for the leading sub-blocks (one warp each).
+// Then V_pm = U_pp R_pm and the off-diagonal blocks of U along the
+// anti-diagonals, U_pq = -sum_{m=p+1..q} V_pm U_mq.
+// Warp-level 32 x 32 products keep one operand column per lane in registers
+// and read the other operand's rows as broadcast 16-byte loads.
 
 constexpr int kDiagThreads = 256;
-constexpr int kDiagLd = kTile + 1;
-constexpr size_t kDiagSmem = (size_t)kTile * kDiagLd * sizeof(double);
+constexpr int kDiagLd = kTile + 4;     // 16-byte aligned rows
+constexpr size_t kDiagSmem = 2 * (size_t)kTile * kDiagLd * sizeof(float);
+
+// acc[i] = sum_k A[i][k] * b[k] for the 32 rows of A (row stride kDiagLd,
+// 16-byte aligned, read as broadcasts), b in registers.
+__device__ __forceinline__ void rows_dot32(const float* A, const float (&b)[32], float (&acc)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float* a = A + i * kDiagLd;
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(a + k);
+      s = fmaf(x.x, b[k], s);
+      s = fmaf(x.y, b[k + 1], s);
+      s = fmaf(x.z, b[k + 2], s);
+      s = fmaf(x.w, b[k + 3], s);
+    }
+    acc[i] = s;
+  }
+}
 
 __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const float* __restrict__ Rws,
                                                                       int d, int k,
@@ -94,166 +118,161 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
                                                                       float* __restrict__ U,
                                                                       int* info) {
   if (cta_info_set(info)) return;
-  extern __shared__ double Rs[];            // [128][129], R after the factorisation
-  __shared__ double vec[2][kTile];          // broadcast column (factor) / row (inverse)
-  __shared__ double piv[2][3];              // 1/a_jj, 1/sqrt(a_jj), sqrt(a_jj)
+  extern __shared__ __align__(16) float dsm[];
+  float* S = dsm;                        // A, becoming R (upper)
+  float* Ui = dsm + kTile * kDiagLd;     // U (upper)
+  __shared__ float rinv[kTile];
   __shared__ int bad;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b0 = k * kTile;
-  const int b = min(kTile, d - b0);
-  double r[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int i = ty + 16 * a, l = tx + 16 * c;
-      r[a][c] = (i <= l && l < b) ? (double)Rws[(long long)(b0 + i) * d + b0 + l] : 0.0;
-    }
+  const int b = min(kTile, d - b0);      // a multiple of 32
+  const int np = b >> 5;
+  for (int e = tid; e < kTile * kTile; e += kDiagThreads) {
+    const int i = e >> 7, l = e & 127;
+    S[i * kDiagLd + l] = (i <= l && l < b) ? Rws[(long long)(b0 + i) * d + b0 + l] : 0.f;
+    Ui[i * kDiagLd + l] = 0.f;
+  }
   if (tid == 0) bad = 0;
   __syncthreads();
 
-  // publish column j (entries i <= j) and its pivot into buffer p
-  auto publish_col = [&](int j, int p) {
-    if (tx != (j & 15)) return;
-    const int cj = j >> 4;
+  for (int p = np - 1; p >= 0; --p) {
+    const int c0 = p * 32;
+    if (warp == 0) {
+      // ---- reverse Cholesky of the 32 x 32 diagonal sub-block, lane = row
+      float dr[32];
+      float* row = S + (c0 + lane) * kDiagLd + c0;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      if (c != cj) continue;
+      for (int l = 0; l < 32; ++l) dr[l] = row[l];
+      int fail = 0;
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const int i = ty + 16 * a;
-        if (i > j) continue;
-        vec[p][i] = r[a][c];
-        if (i == j) {
-          const double pv = r[a][c];
-          if (!(pv > 0.0)) {
-            bad = isfinite(pv) ? (b0 + j + 1) : SGPT_INFO_NONFINITE;
-            piv[p][0] = piv[p][1] = piv[p][2] = 0.0;
-          } else {
-            const double sq = sqrt(pv);
-            piv[p][0] = 1.0 / pv;
-            piv[p][1] = 1.0 / sq;
-            piv[p][2] = sq;
-          }
+      for (int j = 31; j >= 0; --j) {
+        const float piv = __shfl_sync(0xffffffffu, dr[j], j);
+        if (!(piv > 0.f) && fail == 0) fail = isfinite(piv) ? (b0 + c0 + j + 1) : SGPT_INFO_NONFINITE;
+        const float sq = sqrtf(piv);
+        const float inv = 1.0f / sq;
+        const float rij = lane < j ? dr[j] * inv : (lane == j ? sq : 0.f);
+#pragma unroll
+        for (int l = 0; l < j; ++l) {
+          const float rlj = __shfl_sync(0xffffffffu, rij, l);
+          if (lane <= l) dr[l] = fmaf(-rij, rlj, dr[l]);
         }
+        dr[j] = rij;
       }
+#pragma unroll
+      for (int l = 0; l < 32; ++l) row[l] = lane <= l ? dr[l] : 0.f;
+      if (fail && lane == 0) bad = fail;
     }
-  };
-
-  publish_col(b - 1, 0);
-  for (int j = b - 1, p = 0; j >= 0; --j, p ^= 1) {
     __syncthreads();
     if (bad) {
       if (tid == 0) set_info(info, bad);
       return;
     }
-    const double pinv = piv[p][0], rs = piv[p][1], sq = piv[p][2];
-    double ci[8], cl[8];
+    if (warp == 0) {
+      rinv[c0 + lane] = 1.0f / S[(c0 + lane) * kDiagLd + c0 + lane];
+      __syncwarp();
+      // ---- U_pp = R_pp^-1, lane = column j: back substitution from the bottom
+      float u[32];
+      const float* R = S + c0 * kDiagLd + c0;
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int i = ty + 16 * a;
-      ci[a] = i <= j ? vec[p][i] * pinv : 0.0;
-    }
+      for (int i = 31; i >= 0; --i) {
+        float sacc = (i == lane) ? 1.f : 0.f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int l = tx + 16 * c;
-      cl[c] = l <= j ? vec[p][l] : 0.0;
-    }
-    // rank-1 update of the leading j x j upper triangle
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int i = ty + 16 * a;
-      if (i >= j) continue;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int l = tx + 16 * c;
-        if (l >= i && l < j) r[a][c] = fma(-ci[a], cl[c], r[a][c]);
+        for (int m = i + 1; m < 32; ++m) sacc = fmaf(-R[i * kDiagLd + m], u[m], sacc);
+        u[i] = (i <= lane) ? sacc * rinv[c0 + i] : 0.f;
       }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Ui[(c0 + i) * kDiagLd + c0 + lane] = u[i];
     }
-    // column j becomes column j of R
-    if (tx == (j & 15)) {
-      const int cj = j >> 4;
+    __syncthreads();
+    if (p == 0) break;
+    // ---- panel: R_ip = A_ip U_pp^T, rows blocks i < p (in place)
+    if (warp < p) {
+      float bcol[32], acc[32];
+      const float* ur = Ui + (c0 + lane) * kDiagLd + c0;    // row `lane` of U_pp = column of U_pp^T
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (c != cj) continue;
+      for (int m = 0; m < 32; m += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(ur + m);
+        bcol[m] = x.x; bcol[m + 1] = x.y; bcol[m + 2] = x.z; bcol[m + 3] = x.w;
+      }
+      float* Ablk = S + (warp * 32) * kDiagLd + c0;
+      rows_dot32(Ablk, bcol, acc);
+      __syncwarp();
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const int i = ty + 16 * a;
-          if (i < j) r[a][c] *= rs;
-          else if (i == j) r[a][c] = sq;
+      for (int i = 0; i < 32; ++i) Ablk[i * kDiagLd + lane] = acc[i];
+    }
+    __syncthreads();
+    // ---- update of the leading sub-blocks: A_ij -= R_ip R_jp^T, i <= j < p
+    {
+      const int pairs = p * (p + 1) / 2;
+      if (warp < pairs) {
+        int jj = 0;
+        while ((jj + 1) * (jj + 2) / 2 <= warp) ++jj;
+        const int ii = warp - jj * (jj + 1) / 2;          // ii <= jj
+        float bcol[32], acc[32];
+        const float* rp = S + (jj * 32 + lane) * kDiagLd + c0;   // row of R_jp = column of R_jp^T
+#pragma unroll
+        for (int m = 0; m < 32; m += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(rp + m);
+          bcol[m] = x.x; bcol[m + 1] = x.y; bcol[m + 2] = x.z; bcol[m + 3] = x.w;
         }
+        rows_dot32(S + (ii * 32) * kDiagLd + c0, bcol, acc);
+        float* C = S + (ii * 32) * kDiagLd + jj * 32;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) C[i * kDiagLd + lane] -= acc[i];
       }
     }
-    if (j > 0) publish_col(j - 1, p ^ 1);
+    __syncthreads();
   }
 
-  // R to shared memory; registers become B = I
+  // ---- V_pm = U_pp R_pm (p < m), in place over R_pm: lane = column of R_pm
+  {
+    const int pairs = np * (np - 1) / 2;
+    if (warp < pairs) {
+      int mm = 0;
+      while ((mm + 1) * (mm + 2) / 2 <= warp) ++mm;
+      const int pp = warp - mm * (mm + 1) / 2;            // pp <= mm
+      mm += 1;                                             // pp < mm
+      float bcol[32], acc[32];
+      float* Rpm = S + (pp * 32) * kDiagLd + mm * 32;
 #pragma unroll
-  for (int a = 0; a < 8; ++a)
+      for (int kk = 0; kk < 32; ++kk) bcol[kk] = Rpm[kk * kDiagLd + lane];
+      rows_dot32(Ui + (pp * 32) * kDiagLd + pp * 32, bcol, acc);
+      __syncwarp();
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int i = ty + 16 * a, l = tx + 16 * c;
-      Rs[i * kDiagLd + l] = (i <= l && l < b) ? r[a][c] : 0.0;
-      r[a][c] = (i == l && i < b) ? 1.0 : 0.0;
+      for (int i = 0; i < 32; ++i) Rpm[i * kDiagLd + lane] = acc[i];
     }
-
-  // publish row i of X = B[i][.] / r_ii (entries j >= i) into buffer p; the
-  // owners keep X in their registers.
-  auto publish_row = [&](int i, int p) {
-    if (ty != (i & 15)) return;
-    const int ai = i >> 4;
-    const double inv = 1.0 / Rs[i * kDiagLd + i];
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      if (a != ai) continue;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int l = tx + 16 * c;
-        if (l < i || l >= b) continue;
-        r[a][c] *= inv;
-        vec[p][l] = r[a][c];
-      }
-    }
-  };
-
+  }
   __syncthreads();
-  publish_row(b - 1, 0);
-  for (int i = b - 1, p = 0; i > 0; --i, p ^= 1) {
-    __syncthreads();
-    double xr[8], rc[8];
+  // ---- off-diagonal blocks of U by anti-diagonals: U_pq = -sum V_pm U_mq
+  for (int sd = 1; sd < np; ++sd) {
+    if (warp < np - sd) {
+      const int pp = warp, qq = warp + sd;
+      float acc[32];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int l = tx + 16 * c;
-      xr[c] = (l >= i && l < b) ? vec[p][l] : 0.0;
-    }
+      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+      for (int mm = pp + 1; mm <= qq; ++mm) {
+        float bcol[32], part[32];
+        const float* Umq = Ui + (mm * 32) * kDiagLd + qq * 32;
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int row = ty + 16 * a;
-      rc[a] = row < i ? Rs[row * kDiagLd + i] : 0.0;
-    }
+        for (int kk = 0; kk < 32; ++kk) bcol[kk] = Umq[kk * kDiagLd + lane];
+        rows_dot32(S + (pp * 32) * kDiagLd + mm * 32, bcol, part);
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int row = ty + 16 * a;
-      if (row >= i) continue;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int l = tx + 16 * c;
-        if (l >= i && l < b) r[a][c] = fma(-rc[a], xr[c], r[a][c]);
+        for (int i = 0; i < 32; ++i) acc[i] += part[i];
       }
+      float* Upq = Ui + (pp * 32) * kDiagLd + qq * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Upq[i * kDiagLd + lane] = -acc[i];
     }
-    publish_row(i - 1, p ^ 1);
+    __syncthreads();
   }
 
   // Write U_kk (upper, zeros below) to the output and to the block cache.
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int i = ty + 16 * a, l = tx + 16 * c;
-      const float v = (i <= l && l < b) ? (float)r[a][c] : 0.f;
-      Ukk[i * kTile + l] = v;
-      if (i < b && l < b) U[(long long)(b0 + i) * d + b0 + l] = v;
-    }
+  for (int e = tid * 4; e < kTile * kTile; e += kDiagThreads * 4) {
+    const int i = e >> 7, l = e & 127;
+    const float4 v = *reinterpret_cast<const float4*>(Ui + i * kDiagLd + l);
+    st4(Ukk + e, v);
+    if (i < b && l < b) st4(U + (long long)(b0 + i) * d + b0 + l, v);
+  }
 }
 
 // ------------------------------------------------- off-diagonal products
@@ -284,22 +303,6 @@ __device__ __forceinline__ void upper_tile_index(int t, int& i, int& j) {
   i = t - jj * (jj + 1) / 2;
 }
 
-// Rank-128 update of the leading part: A_ij -= R_ik R_jk^T, i <= j < k.
-__global__ void __launch_bounds__(kGemmThreads) syrk_kernel(float* __restrict__ Rws, int d, int k,
-                                                            const int* info) {
-  if (cta_info_set(info)) return;
-  extern __shared__ float smem[];
-  int i, j;
-  upper_tile_index(blockIdx.x, i, j);
-  const int bk = min(kTile, d - k * kTile);
-  float acc[8][8];
-  zero_acc(acc);
-  const OpKContig A{Rws + k * kTile, d, i * kTile, kTile, bk};
-  const OpKContig B{Rws + k * kTile, d, j * kTile, kTile, bk};
-  gemm_tile(A, B, 0, bk, acc, smem);
-  store_tile(Rws + (long long)i * kTile * d + j * kTile, d, kTile, kTile, acc, -1.f, 1.f);
-}
-
 // V_im = U_ii R_im for every off-diagonal block i < m (in place over R).
 __global__ void __launch_bounds__(kGemmThreads) vscale_kernel(float* __restrict__ Rws, int d,
                                                               const float* __restrict__ Udiag,
@@ -318,68 +321,41 @@ __global__ void __launch_bounds__(kGemmThreads) vscale_kernel(float* __restrict_
   store_tile(Rws + (long long)i * kTile * d + m * kTile, d, kTile, bm, acc, 1.f, 0.f);
 }
 
-// Anti-diagonal s of U: U_ij = -sum_{m=i+1..j} V_im U_mj, j = i + s.
-// Split over m into `nsplit` chunks; partial tiles go to `part`, and the CTA
-// that finishes a tile last sums its partials in split order (deterministic).
-__global__ void __launch_bounds__(kGemmThreads) trtri_kernel(const float* __restrict__ V,
-                                                             float* __restrict__ U, int d, int s,
-                                                             int nsplit, float* __restrict__ part,
-                                                             unsigned int* __restrict__ tickets,
-                                                             const int* info) {
-  if (cta_info_set(info)) return;
-  extern __shared__ float smem[];
-  __shared__ unsigned int last;
-  const int tile = blockIdx.x / nsplit;
-  const int split = blockIdx.x - tile * nsplit;
-  const int i = tile, j = tile + s;
-  const int bj = min(kTile, d - j * kTile);
-  const int k_lo = (i + 1) * kTile, k_hi = min((j + 1) * kTile, d);
-  const int nblk = s;                       // blocks m = i+1 .. j
-  const int per = cdiv(nblk, nsplit);
-  const int kb = k_lo + split * per * kTile;
-  const int ke = min(k_hi, kb + per * kTile);
-  float acc[8][8];
-  zero_acc(acc);
-  const OpKContig A{V, d, i * kTile, kTile, k_hi};
-  const OpIContig B{U, d, j * kTile, bj, k_hi};
-  gemm_tile(A, B, kb, ke, acc, smem);
-  float* Ut = U + (long long)i * kTile * d + j * kTile;
-  if (nsplit == 1) {
-    store_tile(Ut, d, kTile, bj, acc, -1.f, 0.f);
-    return;
-  }
-  float* mine = part + ((size_t)blockIdx.x) * kTile * kTile;
-  store_tile(mine, kTile, kTile, bj, acc, 1.f, 0.f);
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = (atomicAdd(&tickets[tile], 1u) == (unsigned)nsplit - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  const float* base = part + (size_t)tile * nsplit * kTile * kTile;
-  for (int e = threadIdx.x * 4; e < kTile * bj; e += kGemmThreads * 4) {
-    const int r = e / bj, c = e - (e / bj) * bj;
-    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = 0; p < nsplit; ++p) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (size_t)p * kTile * kTile + r * kTile + c));
-      sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-    }
-    st4(Ut + (long long)r * d + c, make_float4(-sum.x, -sum.y, -sum.z, -sum.w));
-  }
-  if (threadIdx.x == 0) tickets[tile] = 0;
-}
-
 // ----------------------------------------------------------------- driver
 
-size_t factor_ws_bytes(int d) {
-  Carve c(nullptr);
+struct FactorWs {
+  double* lam;
+  float* R;        // H_d, then R, then V; finally the hi plane of V
+  float* Udiag;    // U_kk blocks, 128 x 128 each
+  float* P_hi;     // hi/lo planes of the current panel (d x 128)
+  float* P_lo;
+  float* V_lo;     // lo plane of V (d x d)
+  float* U_hi;     // hi/lo planes of U (d x d)
+  float* U_lo;
+  float* part;     // split partials of the triangular inverse
+};
+
+static FactorWs carve_factor(void* ws, int d, size_t* bytes) {
+  Carve c(ws);
   const int K = cdiv(d, kTile);
-  c.take<double>(4);
-  c.take<float>((size_t)d * d);                      // R, then V
-  c.take<float>((size_t)K * kTile * kTile);          // U_kk cache
-  c.take<unsigned int>((size_t)K + 32);              // tickets
-  c.take<float>(factor_part_tiles(d) * kTile * kTile);
-  return c.off + 256;
+  FactorWs w;
+  w.lam = c.take<double>(4);
+  w.R = c.take<float>((size_t)d * d);
+  w.Udiag = c.take<float>((size_t)K * kTile * kTile);
+  w.P_hi = c.take<float>((size_t)d * kTile);
+  w.P_lo = c.take<float>((size_t)d * kTile);
+  w.V_lo = c.take<float>((size_t)d * d);
+  w.U_hi = c.take<float>((size_t)d * d);
+  w.U_lo = c.take<float>((size_t)d * d);
+  w.part = c.take<float>(factor_part_tiles(d) * kTile * kTile);
+  if (bytes) *bytes = c.off + 256;
+  return w;
+}
+
+size_t factor_ws_bytes(int d) {
+  size_t b = 0;
+  carve_factor(nullptr, d, &b);
+  return b;
 }
 
 size_t factor_part_tiles(int d) {
@@ -402,43 +378,67 @@ int trtri_splits(int K, int s) {
 
 cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, float* U, void* ws,
                           int* info, cudaStream_t st) {
-  Carve c(ws);
   const int K = cdiv(d, kTile);
-  double* lam = c.take<double>(4);
-  float* R = c.take<float>((size_t)d * d);
-  float* Udiag = c.take<float>((size_t)K * kTile * kTile);
-  unsigned int* tickets = c.take<unsigned int>((size_t)K + 32);
-  float* part = c.take<float>(factor_part_tiles(d) * kTile * kTile);
+  const FactorWs w = carve_factor(ws, d, nullptr);
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(diag_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
     attr_done = true;
   }
   const double scale = 2.0 / (double)n_total;
-  cudaMemsetAsync(tickets, 0, ((size_t)K + 32) * sizeof(unsigned int), st);
   if (U != H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
-  damp_lambda_kernel<<<1, 1024, 0, st>>>(H, d, scale, (double)damp, lam, info);
+  damp_lambda_kernel<<<1, 1024, 0, st>>>(H, d, scale, (double)damp, w.lam, info);
   count_launches(1);
-  scale_damp_kernel<<<dim3(cdiv(d, 4 * 128), d), 128, 0, st>>>(H, R, d, scale, lam, info);
+  scale_damp_kernel<<<dim3(cdiv(d, 4 * 128), d), 128, 0, st>>>(H, w.R, d, scale, w.lam, info);
   count_launches(1);
   if (U == H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
+  cudaError_t e = cudaSuccess;
   for (int k = K - 1; k >= 0; --k) {
-    diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, st>>>(R, d, k, Udiag + (size_t)k * kTile * kTile, U, info);
+    diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, st>>>(w.R, d, k, w.Udiag + (size_t)k * kTile * kTile, U, info);
     count_launches(1);
     if (k == 0) break;
-    panel_kernel<<<k, kGemmThreads, kGemmSmemBytes, st>>>(R, d, k, Udiag + (size_t)k * kTile * kTile, info);
+    const int bk = min(kTile, d - k * kTile);
+    panel_kernel<<<k, kGemmThreads, kGemmSmemBytes, st>>>(w.R, d, k, w.Udiag + (size_t)k * kTile * kTile, info);
     count_launches(1);
-    syrk_kernel<<<k * (k + 1) / 2, kGemmThreads, kGemmSmemBytes, st>>>(R, d, k, info);
-    count_launches(1);
+    // rank-bk update of the leading upper tiles on the tensor cores
+    if ((e = tc::launch_split(w.R + k * kTile, d, k * kTile, bk, w.P_hi, w.P_lo, kTile, info, st)) != cudaSuccess)
+      return e;
+    const tc::Operand P{w.P_hi, w.P_lo, (long long)k * kTile, kTile, kTile};
+    tc::Job job{};
+    job.mode = 1;
+    job.kdim = bk;
+    job.C = w.R;
+    job.ldc = d;
+    job.Mlim = job.Nlim = k * kTile;
+    job.alpha = -1.f;
+    job.beta = 1.f;
+    if ((e = tc::launch_gemm(P, P, false, job, k * (k + 1) / 2, info, st)) != cudaSuccess) return e;
   }
   if (K > 1) {
-    vscale_kernel<<<K * (K - 1) / 2, kGemmThreads, kGemmSmemBytes, st>>>(R, d, Udiag, info);
+    vscale_kernel<<<K * (K - 1) / 2, kGemmThreads, kGemmSmemBytes, st>>>(w.R, d, w.Udiag, info);
     count_launches(1);
-  }
-  for (int s = 1; s < K; ++s) {
-    const int ns = trtri_splits(K, s);
-    trtri_kernel<<<(K - s) * ns, kGemmThreads, kGemmSmemBytes, st>>>(R, U, d, s, ns, part, tickets, info);
-    count_launches(1);
+    // planes of V (hi in place over R) and of U (its diagonal blocks so far)
+    if ((e = tc::launch_split(w.R, d, d, d, w.R, w.V_lo, d, info, st)) != cudaSuccess) return e;
+    if ((e = tc::launch_split(U, d, d, d, w.U_hi, w.U_lo, d, info, st)) != cudaSuccess) return e;
+    const tc::Operand V{w.R, w.V_lo, d, d, d};
+    const tc::Operand Up{w.U_hi, w.U_lo, d, d, d};
+    for (int s = 1; s < K; ++s) {
+      tc::Job job{};
+      job.mode = 2;
+      job.s = s;
+      job.nsplit = trtri_splits(K, s);
+      job.nblk = K;
+      job.dlim = d;
+      job.C = U;
+      job.ldc = d;
+      job.Mlim = job.Nlim = d;
+      job.alpha = -1.f;
+      job.beta = 0.f;
+      job.C_hi = w.U_hi;
+      job.C_lo = w.U_lo;
+      job.part = w.part;
+      if ((e = tc::launch_gemm(V, Up, true, job, (K - s) * job.nsplit, info, st)) != cudaSuccess) return e;
+    }
   }
   return cudaGetLastError();
 }

@@ -1,0 +1,454 @@
+// FP32-accurate matrix products on the 5th-generation tensor cores.
+//
+// C = alpha * A B + beta * C with A, B fp32. Each operand is held as two
+// planes, x = hi + lo with hi = x rounded to TF32 (10 explicit mantissa
+// bits) and lo = x - hi (exact), and every K step issues three
+// tcgen05.mma.kind::tf32 products, hi*hi + hi*lo + lo*hi, into one fp32 TMEM
+// accumulator (the lo*lo term is below fp32 resolution). The error per
+// product is about 2^-21 relative, against 2^-24 for a plain fp32 FMA and
+// 2^-11 for a single TF32 product.
+//
+// Used for the rank-128 updates and the triangular inverse of the
+// factorisation and for the lazy trailing update of the OBS sweep.
+//
+// CTA tile 128 x 128, K in chunks of 32 (one 128-byte swizzle row of fp32),
+// three-stage TMA ring (no multicast); warp 0 lane 0 loads, warp 1 lane 0
+// issues MMAs, warps 2-5 drain TMEM (warp w reads lanes 32*(w%4)..).
+// A is always K-major (row-major M x K); B is K-major (row-major N x K) or
+// MN-major (row-major K x N). Every wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "gemm_tc.h"
+#include "kernels.h"
+
+namespace sgpt {
+namespace tc {
+
+namespace {
+
+constexpr int kM = 128, kN = 128, kKC = 32;
+constexpr int kStages = 3;
+constexpr int kPlane = kM * kKC * 4;            // 16 KB: one operand plane of one stage
+constexpr int kStageBytes = 4 * kPlane;         // A hi/lo, B hi/lo
+constexpr int kThreads = 192;
+constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256;
+constexpr long long kWaitCycles = 4000000000ll;
+
+__host__ __device__ constexpr uint32_t make_idesc(bool b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(kN >> 3) << 17) |
+         ((uint32_t)(kM >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// K-major operand, 128-byte swizzle: 8-row groups of 1 KB.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fff);
+  d |= (uint64_t)1 << 16;                         // leading byte offset (unused when swizzled)
+  d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: next 8 rows
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// MN-major 32-bit operand: the 128-byte swizzle with 32-byte granules
+// (descriptor layout SWIZZLE_128B_BASE32B, filled by TMA's
+// SWIZZLE_128B_ATOM_32B). Atoms are 32 columns x 4 K rows (512 bytes);
+// LBO = next 32 columns (one 32-column x 32-row TMA box, 4 KB), SBO = next
+// 4 K rows. The plain 128-byte swizzle (16-byte granules) is not a valid
+// MN-major form for 32-bit elements.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fff);
+  d |= (uint64_t)(4096 >> 4) << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)1 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.b32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mma_tf32(uint32_t tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+        "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+        "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tri_index(int t, int& i, int& j) {
+  int jj = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+  while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
+  while (jj * (jj + 1) / 2 > t) --jj;
+  j = jj;
+  i = t - jj * (jj + 1) / 2;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
+    const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
+    const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo, const Job job,
+    const int b_mn, int* info) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  __shared__ int failed;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- which tile and which K range
+  int m0 = 0, n0 = 0, kb = 0, ke = 0, split = 0, tile = 0;
+  if (job.mode == 0) {
+    m0 = (blockIdx.x / job.nt) * kM;
+    n0 = (blockIdx.x % job.nt) * kN;
+    ke = job.kdim;
+  } else if (job.mode == 1) {
+    int i, j;
+    tri_index(blockIdx.x, i, j);
+    m0 = i * kM;
+    n0 = j * kN;
+    ke = job.kdim;
+  } else {
+    tile = blockIdx.x / job.nsplit;
+    split = blockIdx.x - tile * job.nsplit;
+    const int i = tile, j = tile + job.s;
+    m0 = i * kM;
+    n0 = j * kN;
+    const int lo = (i + 1) * kM, hi = min((j + 1) * kM, job.dlim);
+    const int per = ((job.s + job.nsplit - 1) / job.nsplit) * kM;
+    kb = min(hi, lo + split * per);
+    ke = min(hi, kb + per);
+  }
+  const int iters = (ke - kb + kKC - 1) / kKC;
+  const uint32_t idesc = make_idesc(b_mn != 0);
+
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages), done = smem_u32(bars + 2 * kStages);
+  if (threadIdx.x == 0) {
+    failed = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = cta_info_set(info);
+
+  if (!skip && iters > 0 && warp == 0 && lane == 0) {
+    int issued = 0;
+    for (int it = 0; it < iters; ++it) {
+      const int s = it % kStages;
+      if (it >= kStages && !mbar_wait(empty0 + 8 * s, ((it / kStages) & 1) ^ 1)) {
+        failed = 1;
+        break;
+      }
+      const uint32_t bar = full0 + 8 * s;
+      mbar_expect_tx(bar, kStageBytes);
+      const uint32_t st = s0 + s * kStageBytes;
+      const int k = kb + it * kKC;
+      tma_2d(st, &a_hi, bar, job.a_x0 + k, job.a_y0 + m0);
+      tma_2d(st + kPlane, &a_lo, bar, job.a_x0 + k, job.a_y0 + m0);
+      if (b_mn) {
+#pragma unroll
+        for (int c = 0; c < kN / 32; ++c) {
+          tma_2d(st + 2 * kPlane + c * 4096, &b_hi, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
+          tma_2d(st + 3 * kPlane + c * 4096, &b_lo, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
+        }
+      } else {
+        tma_2d(st + 2 * kPlane, &b_hi, bar, job.b_x0 + k, job.b_y0 + n0);
+        tma_2d(st + 3 * kPlane, &b_lo, bar, job.b_x0 + k, job.b_y0 + n0);
+      }
+      ++issued;
+    }
+    for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
+      if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
+  } else if (!skip && iters > 0 && warp == 1 && lane == 0) {
+    for (int it = 0; it < iters; ++it) {
+      const int s = it % kStages;
+      if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+        failed = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t st = s0 + s * kStageBytes;
+#pragma unroll
+      for (int ks = 0; ks < kKC / 8; ++ks) {
+        const uint64_t ah = kmajor_desc(st + ks * 32), al = kmajor_desc(st + kPlane + ks * 32);
+        uint64_t bh, bl;
+        if (b_mn) {
+          bh = mnmajor_desc(st + 2 * kPlane + ks * 1024);
+          bl = mnmajor_desc(st + 3 * kPlane + ks * 1024);
+        } else {
+          bh = kmajor_desc(st + 2 * kPlane + ks * 32);
+          bl = kmajor_desc(st + 3 * kPlane + ks * 32);
+        }
+        const uint32_t first = (it == 0 && ks == 0) ? 0u : 1u;
+        mma_tf32(tmem, al, bh, idesc, first);   // small terms first
+        mma_tf32(tmem, ah, bl, idesc, 1u);
+        mma_tf32(tmem, ah, bh, idesc, 1u);
+      }
+      mma_commit(empty0 + 8 * s);
+    }
+    mma_commit(done);
+  }
+
+  bool have = !skip && iters > 0;
+  if (have && warp >= 2) {
+    __syncwarp();
+    if (!mbar_wait(done, 0)) {
+      failed = 1;
+      have = false;
+    }
+  }
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
+
+  if (!skip && !failed && warp >= 2) {
+    const int q = warp & 3;
+    const int m = q * 32 + lane;               // tile row = TMEM lane
+    const bool partial = job.mode == 2 && job.nsplit > 1;
+#pragma unroll 1
+    for (int cc = 0; cc < kN / 32; ++cc) {
+      uint32_t v[32];
+      if (iters > 0) {
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + cc * 32, v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (partial) {
+        float* dst = job.part + (size_t)blockIdx.x * kM * kN + (size_t)m * kN + cc * 32;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          st4(dst + e, make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                                   __uint_as_float(v[e + 3])));
+        continue;
+      }
+      const int row = m0 + m;
+      if (row >= job.Mlim) continue;
+      const long long off = (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + n0 + cc * 32;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const int col = n0 + cc * 32 + e;
+        if (col >= job.Nlim) break;
+        float o[4];
+        float4 old = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (job.beta != 0.f) old = ld4(job.C + off + e);
+        o[0] = fmaf(job.alpha, __uint_as_float(v[e + 0]), job.beta * old.x);
+        o[1] = fmaf(job.alpha, __uint_as_float(v[e + 1]), job.beta * old.y);
+        o[2] = fmaf(job.alpha, __uint_as_float(v[e + 2]), job.beta * old.z);
+        o[3] = fmaf(job.alpha, __uint_as_float(v[e + 3]), job.beta * old.w);
+        st4(job.C + off + e, make_float4(o[0], o[1], o[2], o[3]));
+        if (job.C_hi) {
+          float h4[4], l4[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            h4[t] = tf32_hi(o[t]);
+            l4[t] = o[t] - h4[t];
+          }
+          st4(job.C_hi + off + e, make_float4(h4[0], h4[1], h4[2], h4[3]));
+          st4(job.C_lo + off + e, make_float4(l4[0], l4[1], l4[2], l4[3]));
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
+}
+
+// Anti-diagonal split partials -> C = alpha * sum (+ hi/lo planes), in split order.
+__global__ void __launch_bounds__(256) antidiag_reduce_kernel(const Job job, const int* info) {
+  if (cta_info_set(info)) return;
+  const int tiles = job.nblk - job.s;
+  const long long quads = (long long)tiles * (kM * kN / 4);
+  for (long long qd = (long long)blockIdx.x * blockDim.x + threadIdx.x; qd < quads;
+       qd += (long long)gridDim.x * blockDim.x) {
+    const int tile = (int)(qd / (kM * kN / 4));
+    const int e = (int)(qd - (long long)tile * (kM * kN / 4)) * 4;
+    const int m = e / kN, n = e % kN;
+    const int row = tile * kM + m, col = (tile + job.s) * kN + n;
+    if (row >= job.Mlim || col >= job.Nlim) continue;
+    const float* src = job.part + (size_t)tile * job.nsplit * kM * kN + e;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p = 0; p < job.nsplit; ++p) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + (size_t)p * kM * kN));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const float o[4] = {job.alpha * acc.x, job.alpha * acc.y, job.alpha * acc.z, job.alpha * acc.w};
+    const long long off = (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + col;
+    st4(job.C + off, make_float4(o[0], o[1], o[2], o[3]));
+    if (job.C_hi) {
+      float h4[4], l4[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        h4[t] = tf32_hi(o[t]);
+        l4[t] = o[t] - h4[t];
+      }
+      st4(job.C_hi + off, make_float4(h4[0], h4[1], h4[2], h4[3]));
+      st4(job.C_lo + off, make_float4(l4[0], l4[1], l4[2], l4[3]));
+    }
+  }
+}
+
+// hi/lo planes of a row-major block: rows x cols (cols % 4 == 0).
+// In place is allowed (hi == src): every element is read before it is written.
+__global__ void split_planes_kernel(const float* src, long long ld, int rows, int cols, float* hi, float* lo,
+                                    long long ldo, const int* info) {
+  if (info_set(info)) return;
+  const long long quads = (long long)rows * (cols / 4);
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < quads;
+       q += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(q / (cols / 4)), c = (int)(q - (long long)r * (cols / 4)) * 4;
+    const float4 x = ld4(src + (long long)r * ld + c);
+    const float4 h = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+    st4(hi + (long long)r * ldo + c, h);
+    st4(lo + (long long)r * ldo + c, make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Tensor map over a row-major fp32 matrix [rows x cols] with leading dimension
+// ld; box = box_x (inner, fp32 elements) x box_y rows, 128-byte swizzle
+// (32-byte granules for MN-major operands).
+bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, long long ld, int box_x, int box_y,
+              bool mn_major) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_y};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_split(const float* src, long long ld, int rows, int cols, float* hi, float* lo, long long ldo,
+                         const int* info, cudaStream_t st) {
+  const long long quads = (long long)rows * (cols / 4);
+  if (quads == 0) return cudaSuccess;
+  const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
+  split_planes_kernel<<<g, 256, 0, st>>>(src, ld, rows, cols, hi, lo, ldo, info);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
+                        cudaStream_t st) {
+  if (grid <= 0) return cudaSuccess;
+  CUtensorMap ah, al, bh, bl;
+  if (!make_map(&ah, A.hi, A.rows, A.cols, A.ld, kKC, kM, false) ||
+      !make_map(&al, A.lo, A.rows, A.cols, A.ld, kKC, kM, false))
+    return cudaErrorInvalidValue;
+  if (b_mn) {
+    if (!make_map(&bh, B.hi, B.rows, B.cols, B.ld, 32, kKC, true) ||
+        !make_map(&bl, B.lo, B.rows, B.cols, B.ld, 32, kKC, true))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&bh, B.hi, B.rows, B.cols, B.ld, kKC, kN, false) ||
+        !make_map(&bl, B.lo, B.rows, B.cols, B.ld, kKC, kN, false))
+      return cudaErrorInvalidValue;
+  }
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    attr = true;
+  }
+  gemm_tf32x3_kernel<<<grid, kThreads, kSmem, st>>>(ah, al, bh, bl, job, b_mn ? 1 : 0, info);
+  count_launches(1);
+  if (job.mode == 2 && job.nsplit > 1) {
+    const long long quads = (long long)(job.nblk - job.s) * (kM * kN / 4);
+    const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
+    antidiag_reduce_kernel<<<g, 256, 0, st>>>(job, info);
+    count_launches(1);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace sgpt

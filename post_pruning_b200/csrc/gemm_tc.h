@@ -1,0 +1,52 @@
+// FP32-accurate tensor-core products (three TF32 products per K step), see
+// gemm_tc.cu. Host-side interface used by the factorisation and the sweep.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace sgpt {
+namespace tc {
+
+// One fp32 operand as hi/lo planes, both row-major rows x cols with leading
+// dimension ld (ld % 4 == 0, 16-byte aligned bases).
+struct Operand {
+  const float* hi;
+  const float* lo;
+  long long rows, cols, ld;
+};
+
+// What one launch computes; tile sizes are 128 x 128.
+//  mode 0: dense grid of mt x nt tiles, K = kdim.
+//  mode 1: tiles (i, j), i <= j, enumerated column by column, K = kdim.
+//  mode 2: tiles (i, i + s) for i < nblk - s, K = [(i+1)*128, min((i+s+1)*128, dlim)),
+//          split into nsplit ranges whose partials are reduced in order.
+// A(m, k) is read at (x = a_x0 + k, y = a_y0 + m0 + m); B(k, n) at
+// (x = b_x0 + k, y = b_y0 + n0 + n) if K-major, (x = b_x0 + n0 + n, y = b_y0 + k)
+// if MN-major. C(m, n) = alpha * acc + beta * C at
+// C[(c_row0 + m0 + m) * ldc + c_col0 + n0 + n] for m0+m < Mlim, n0+n < Nlim;
+// C_hi/C_lo (optional) receive the hi/lo planes of the result.
+struct Job {
+  int mode;
+  int mt, nt;
+  int s, nsplit, nblk;
+  int kdim;
+  int dlim;
+  int a_x0, a_y0, b_x0, b_y0;
+  float* C;
+  long long ldc;
+  int c_row0, c_col0, Mlim, Nlim;
+  float alpha, beta;
+  float* C_hi;
+  float* C_lo;
+  float* part;
+};
+
+constexpr int kTileTC = 128;
+
+cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
+                        cudaStream_t st);
+cudaError_t launch_split(const float* src, long long ld, int rows, int cols, float* hi, float* lo, long long ldo,
+                         const int* info, cudaStream_t st);
+
+}  // namespace tc
+}  // namespace sgpt

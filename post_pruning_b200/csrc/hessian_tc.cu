@@ -7,15 +7,19 @@
 // whose rows i0.. and columns j0.. meet the upper triangle (H is symmetric:
 // only those tiles are computed, and every element i <= j is written to both
 // H[i][j] and H[j][i]). Tokens are split across CTAs when there are too few
-// tiles to fill the GPU; split partials are summed in split order by the CTA
-// that finishes a tile last (deterministic).
+// tiles to fill the GPU; split partials are summed in split order
+// by a separate reduction kernel (deterministic).
 //
 // Per CTA: warp 0 lane 0 streams 64-token stages with TMA (128-byte swizzle,
 // one box = 64 tokens x 64 channels), warp 1 lane 0 issues
 // tcgen05.mma.kind::f16 (M=128, N=256, K=16, bf16 in, fp32 accumulate in
-// TMEM, 256 columns), and all four warps drain TMEM with tcgen05.ld after the
-// last MMA commits. Every wait is bounded; a wait that runs out records
-// SGPT_INFO_TIMEOUT.
+// TMEM). The tensor-core accumulator loses a fraction of an ulp per step on
+// long sums of positive terms (the diagonal of X^T X drifts low by about 1e-3
+// relative over 16k steps), so each TMEM accumulator only ever sums one chunk
+// of 512 tokens: two 256-column accumulators alternate, and eight epilogue
+// warps drain each finished chunk into FP32 running sums in registers
+// (round-to-nearest adds) while the MMAs fill the other one. Every wait is
+// bounded; a wait that runs out records SGPT_INFO_TIMEOUT.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -34,7 +38,10 @@ constexpr int kBox = kBK * 64 * 2;   // bytes of one 64-token x 64-channel box
 constexpr int kAStage = 2 * kBox;    // 16 KB
 constexpr int kBStage = 4 * kBox;    // 32 KB
 constexpr int kStageBytes = kAStage + kBStage;
-constexpr int kThreads = 128;
+constexpr int kEpiWarps = 8;                  // warps 2..9 drain TMEM
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // warp 0: TMA, warp 1: MMA
+constexpr int kChunkIters = 8;                // stages (512 tokens) per TMEM accumulation
+constexpr int kTmemCols = 2 * kN;             // two accumulators, double-buffered
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 constexpr long long kWaitCycles = 4000000000ll;   // ~2 s at the B200 boost clock
 
@@ -61,6 +68,9 @@ __device__ __forceinline__ uint64_t mn_desc(uint32_t addr) {
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -103,7 +113,8 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+// 32 consecutive accumulator columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -113,8 +124,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
         "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Tiles meeting the upper triangle, band by band: band ti (rows ti*128..)
 // holds the 256-wide column tiles tj >= ti/2, so it starts at tile
@@ -127,15 +138,13 @@ __host__ __device__ inline long long band_start(int ti, int tn) {
 
 __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int d, long long n,
-    int nsplit, long long per, float* __restrict__ part, unsigned int* __restrict__ tickets,
-    int* info) {
+    int nsplit, long long per, float* __restrict__ part, int* info) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
   __shared__ int failed;
-  __shared__ unsigned int last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x / nsplit, split = blockIdx.x - (blockIdx.x / nsplit) * nsplit;
@@ -156,9 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   const long long t_begin = (long long)split * per;
   const long long t_end = t_begin + per < n ? t_begin + per : n;
   const int iters = (int)((t_end - t_begin + kBK - 1) / kBK);
+  const int nchunks = (iters + kChunkIters - 1) / kChunkIters;
 
   const uint32_t s0 = smem_u32(smem);
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages), done = smem_u32(bars + 2 * kStages);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
+  const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16;
 
   if (threadIdx.x == 0) {
     failed = 0;
@@ -166,12 +177,15 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, kEpiWarps);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kN));
+                 "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -179,6 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
   const bool skip = cta_info_set(info) || iters <= 0;
+
+  // Epilogue state: warp w (2..9) owns TMEM lanes 32*(w%4).. (tile rows) and
+  // columns 128*((w-2)/4).. of each accumulator; its running sums live in
+  // registers and are updated with correctly rounded FP32 adds.
+  const int q = warp & 3, h = (warp - 2) >> 2;
+  float acc[128];
+#pragma unroll
+  for (int e = 0; e < 128; ++e) acc[e] = 0.f;
 
   if (!skip && warp == 0 && lane == 0) {
     // TMA producer
@@ -204,86 +226,118 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
       if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
   } else if (!skip && warp == 1 && lane == 0) {
-    // MMA issuer
-    for (int it = 0; it < iters; ++it) {
-      const int s = it % kStages;
-      if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+    // MMA issuer: chunk c accumulates kChunkIters stages into buffer c & 1
+    for (int c = 0; c < nchunks && !failed; ++c) {
+      const int b = c & 1;
+      if (c >= 2 && !mbar_wait(tempty0 + 8 * b, ((c >> 1) - 1) & 1)) {
         failed = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a = s0 + s * kStageBytes, b = a + kAStage;
-#pragma unroll
-      for (int ks = 0; ks < kBK / 16; ++ks)
-        mma_bf16(tmem, mn_desc(a + ks * 2048), mn_desc(b + ks * 2048), (it | ks) != 0);
-      mma_commit(empty0 + 8 * s);
-    }
-    mma_commit(done);
-  }
-
-  // Epilogue: every warp waits for the accumulator, then reads its 32 lanes.
-  bool have = !skip;
-  if (have) {
-    __syncwarp();
-    if (!mbar_wait(done, 0)) {
-      failed = 1;
-      have = false;
-    }
-  }
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  __syncthreads();
-  if (failed) {
-    have = false;
-    if (threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
-  }
-
-  const int i = i0 + warp * 32 + lane;   // TMEM lane = tile row
-  if (have) {
-    float* dst = nsplit > 1 ? part + (size_t)blockIdx.x * kM * kN + (size_t)(warp * 32 + lane) * kN : nullptr;
-#pragma unroll 1
-    for (int c = 0; c < kN / 32; ++c) {
-      uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
-      if (nsplit > 1) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          st4(dst + c * 32 + e, make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])));
-      } else if (i < d) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = j0 + c * 32 + e;
-          if (j < i || j >= d) continue;
-          const float x = __uint_as_float(v[e]);
-          H[(long long)i * d + j] += x;
-          if (j != i) H[(long long)j * d + i] += x;
+      const uint32_t acc_t = tmem + (uint32_t)(b * kN);
+      const int it_end = min(iters, (c + 1) * kChunkIters);
+      for (int it = c * kChunkIters; it < it_end; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+          failed = 1;
+          break;
         }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a = s0 + s * kStageBytes, bb = a + kAStage;
+#pragma unroll
+        for (int ks = 0; ks < kBK / 16; ++ks)
+          mma_bf16(acc_t, mn_desc(a + ks * 2048), mn_desc(bb + ks * 2048), (it != c * kChunkIters) || ks != 0);
+        mma_commit(empty0 + 8 * s);
+      }
+      mma_commit(tfull0 + 8 * b);
+    }
+  } else if (!skip && warp >= 2) {
+    // Drain every chunk into the running sums, then hand the buffer back.
+    for (int c = 0; c < nchunks; ++c) {
+      const int b = c & 1;
+      if (!mbar_wait(tfull0 + 8 * b, (c >> 1) & 1)) {
+        failed = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kN + h * 128);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32_nowait(base + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[cc * 32 + e] += __uint_as_float(v[e]);
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * b);
+    }
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
+  if (!skip && !failed && warp >= 2) {
+    const int r = q * 32 + lane;              // tile row
+    const int i = i0 + r;
+    if (nsplit > 1) {
+      float* dst = part + (size_t)blockIdx.x * kM * kN + (size_t)r * kN + h * 128;
+#pragma unroll
+      for (int e = 0; e < 128; e += 4) st4(dst + e, make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]));
+    } else if (i < d) {
+#pragma unroll
+      for (int e = 0; e < 128; ++e) {
+        const int j = j0 + h * 128 + e;
+        if (j < i || j >= d) continue;
+        H[(long long)i * d + j] += acc[e];
+        if (j != i) H[(long long)j * d + i] += acc[e];
       }
     }
   }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
 
-  if (nsplit > 1 && !failed && !skip) {
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last = (atomicAdd(&tickets[tile], 1u) == (unsigned)nsplit - 1);
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    // the last CTA of the tile sums the partials in split order
-    const float* base = part + (size_t)tile * nsplit * kM * kN;
-    for (int e = threadIdx.x; e < kM * kN; e += kThreads) {
-      const int r = e / kN, c = e - (e / kN) * kN;
-      const int ii = i0 + r, jj = j0 + c;
-      if (ii >= d || jj >= d || jj < ii) continue;
-      float sum = 0.f;
-      for (int p = 0; p < nsplit; ++p) sum += __ldcg(base + (size_t)p * kM * kN + e);
-      H[(long long)ii * d + jj] += sum;
-      if (jj != ii) H[(long long)jj * d + ii] += sum;
+// Split partials -> H: every element of every tile sums its nsplit partials
+// in split order (deterministic) and adds the sum to H[i][j] and H[j][i].
+__global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __restrict__ part,
+                                                             float* __restrict__ H, int d, int tiles,
+                                                             int nsplit, const int* info) {
+  if (cta_info_set(info)) return;
+  const int tn = (d + kN - 1) / kN;
+  const long long quads = (long long)tiles * (kM * kN / 4);
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < quads;
+       q += (long long)gridDim.x * blockDim.x) {
+    const int tile = (int)(q / (kM * kN / 4));
+    const int e = (int)(q - (long long)tile * (kM * kN / 4)) * 4;
+    int ti = 0;
+    {
+      int lo = 0, hi = (d + kM - 1) / kM - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (band_start(mid, tn) <= tile) lo = mid;
+        else hi = mid - 1;
+      }
+      ti = lo;
     }
-    if (threadIdx.x == 0) tickets[tile] = 0;
+    const int tj = ti / 2 + (int)(tile - band_start(ti, tn));
+    const int i = ti * kM + e / kN, j0 = tj * kN + (e % kN);
+    if (i >= d || j0 >= d || j0 + 3 < i) continue;
+    const float* src = part + (size_t)tile * nsplit * kM * kN + e;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p = 0; p < nsplit; ++p) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + (size_t)p * kM * kN));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int j = j0 + t;
+      if (j < i || j >= d) continue;
+      H[(long long)i * d + j] += a[t];
+      if (j != i) H[(long long)j * d + i] += a[t];
+    }
   }
 }
 
@@ -331,7 +385,6 @@ Plan plan(int d, long long n) {
 size_t hessian_ws_bytes(int d, long long n) {
   const Plan p = plan(d, n);
   Carve c(nullptr);
-  c.take<unsigned int>((size_t)p.tiles);
   if (p.nsplit > 1) c.take<float>((size_t)p.tiles * p.nsplit * kM * kN);
   return c.off + 256;
 }
@@ -343,10 +396,8 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
   if (!enc) return cudaErrorNotSupported;
   const Plan p = plan(d, n);
   Carve c(ws);
-  unsigned int* tickets = c.take<unsigned int>((size_t)p.tiles);
   float* part = p.nsplit > 1 ? c.take<float>((size_t)p.tiles * p.nsplit * kM * kN) : nullptr;
 
-  cudaMemsetAsync(tickets, 0, sizeof(unsigned int) * p.tiles, st);
 
   CUtensorMap map;
   const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n};
@@ -362,9 +413,14 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
     cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     attr = true;
   }
-  hessian_tc_kernel<<<p.tiles * p.nsplit, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, tickets,
-                                                                 info);
+  hessian_tc_kernel<<<p.tiles * p.nsplit, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info);
   count_launches(1);
+  if (p.nsplit > 1) {
+    const long long quads = (long long)p.tiles * (kM * kN / 4);
+    const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
+    hessian_reduce_kernel<<<g, 256, 0, st>>>(part, H, d, p.tiles, p.nsplit, info);
+    count_launches(1);
+  }
   return cudaGetLastError();
 }
 

@@ -19,7 +19,7 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
                           int* info, cudaStream_t st);
 
 // sweep.cu
-size_t prune_ws_bytes(int d_out);
+size_t prune_ws_bytes(int d_out, int d_in);
 cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* U,
                          const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
                          int* info, cudaStream_t st);

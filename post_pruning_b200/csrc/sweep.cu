@@ -8,7 +8,8 @@
 //      registers: mask decision (2:4 at each group start on the compensated
 //      weights), e = (w_q - p_q) / U_qq, rank-1 update of the rest of the
 //      block with the U row held in shared memory;
-//   3. trailing_kernel: W[:, i2:] -= Err * U[i1:i2, i2:] (FP32 SIMT product).
+//   3. W[:, i2:] -= Err * U[i1:i2, i2:] as an FP32-accurate tensor-core GEMM
+//      (three TF32 products on hi/lo planes of Err and U, gemm_tc.cu).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -17,6 +18,7 @@
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.h"
 #include "kernels.h"
 
 namespace sgpt {
@@ -39,7 +41,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
     const float* __restrict__ U, uint32_t* __restrict__ mask, float* __restrict__ row_loss,
-    float* __restrict__ Err, const unsigned long long* __restrict__ thr, int* info) {
+    float* __restrict__ Err, float* __restrict__ Err_lo, const unsigned long long* __restrict__ thr,
+    int* info) {
   if (cta_info_set(info)) return;
   extern __shared__ float Us[];   // [128][128]: U[i1 + a][i1 + b]
   const int tid = threadIdx.x;
@@ -85,7 +88,10 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
   }
   float loss = 0.f;
 
-#pragma unroll
+  // Segments run as a loop (not unrolled) to keep the body small enough for
+  // the instruction cache; the 16 columns of a segment are unrolled so that
+  // every register index is static.
+#pragma unroll 1
   for (int qs = 0; qs < kTpr; ++qs) {
     if (qs * kSeg >= bw) break;
 #pragma unroll
@@ -147,6 +153,16 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 #pragma unroll
     for (int v = 0; v < kSeg / 4; ++v) st4(wrow + 4 * v, make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
     float* erow = Err + (long long)row * kMaxBlock + c0;
+    if (Err_lo) {
+      // hi/lo planes for the tensor-core trailing update
+      float* lrow = Err_lo + (long long)row * kMaxBlock + c0;
+#pragma unroll
+      for (int j = 0; j < kSeg; ++j) {
+        const float h = tf32_hi(err[j]);
+        lrow[j] = err[j] - h;
+        err[j] = h;
+      }
+    }
 #pragma unroll
     for (int v = 0; v < kSeg / 4; ++v) st4(erow + 4 * v, make_float4(err[4 * v], err[4 * v + 1], err[4 * v + 2], err[4 * v + 3]));
     if (MODE != kModeForced && (seg & 1) == 0) {
@@ -219,15 +235,29 @@ __global__ void __launch_bounds__(256) select_pass_kernel(
   const int shift = 56 - 8 * pass;
   const unsigned long long prefix = st->prefix;
   const long long total4 = (long long)rows * (bw / 4);
-  for (long long e = (long long)blockIdx.x * 256 + t; e < total4; e += (long long)gridDim.x * 256) {
-    const int row = (int)(e / (bw / 4));
-    const int c = (int)(e - (long long)row * (bw / 4)) * 4;
-    const float4 x = ld4(W + (long long)row * ldw + i1 + c);
-    const float v[4] = {x.x, x.y, x.z, x.w};
+  // The trip count is uniform across the block so that every lane of a warp
+  // takes part in the warp-wide match below.
+  for (long long base = (long long)blockIdx.x * 256; base < total4; base += (long long)gridDim.x * 256) {
+    const long long e = base + t;
+    const bool act = e < total4;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    int row = 0, c = 0;
+    if (act) {
+      row = (int)(e / (bw / 4));
+      c = (int)(e - (long long)row * (bw / 4)) * 4;
+      const float4 x = ld4(W + (long long)row * ldw + i1 + c);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const unsigned long long key = sal_key(v[j], ud[c + j], (unsigned)row * (unsigned)bw + (unsigned)(c + j));
-      if (pass == 0 || (key >> (shift + 8)) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+      const unsigned long long key =
+          act ? sal_key(v[j], ud[c + j], (unsigned)row * (unsigned)bw + (unsigned)(c + j)) : 0ull;
+      const bool mine = act && (pass == 0 || (key >> (shift + 8)) == prefix);
+      // Most keys share a few digits (saliencies span a narrow exponent
+      // range): aggregate equal digits within the warp before the atomic.
+      const unsigned bin = mine ? (unsigned)((key >> shift) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (mine && (t & 31) == (__ffs(peers) - 1)) atomicAdd(&h[bin], (unsigned)__popc(peers));
     }
   }
   __syncthreads();
@@ -262,19 +292,36 @@ __global__ void __launch_bounds__(256) select_pass_kernel(
 
 // ----------------------------------------------------------------- driver
 
-size_t prune_ws_bytes(int d_out) {
-  Carve c(nullptr);
-  c.take<float>((size_t)d_out * kMaxBlock);   // Err
-  c.take<SelState>(1);
-  return c.off + 256;
+struct PruneWs {
+  float* Err_hi;   // error block of the current OBS block, hi/lo planes (d_out x 128)
+  float* Err_lo;
+  float* U_hi;     // hi/lo planes of U (d_in x d_in)
+  float* U_lo;
+  SelState* sel;
+};
+
+static PruneWs carve_prune(void* ws, int d_out, int d_in, size_t* bytes) {
+  Carve c(ws);
+  PruneWs w;
+  w.Err_hi = c.take<float>((size_t)d_out * kMaxBlock);
+  w.Err_lo = c.take<float>((size_t)d_out * kMaxBlock);
+  w.U_hi = c.take<float>((size_t)d_in * d_in);
+  w.U_lo = c.take<float>((size_t)d_in * d_in);
+  w.sel = c.take<SelState>(1);
+  if (bytes) *bytes = c.off + 256;
+  return w;
+}
+
+size_t prune_ws_bytes(int d_out, int d_in) {
+  size_t b = 0;
+  carve_prune(nullptr, d_out, d_in, &b);
+  return b;
 }
 
 cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* U,
                          const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
                          int* info, cudaStream_t st) {
-  Carve c(ws);
-  float* Err = c.take<float>((size_t)rows * kMaxBlock);
-  SelState* sel = c.take<SelState>(1);
+  const PruneWs w = carve_prune(ws, rows, d, nullptr);
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(sweep_kernel<kModeNM24>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
@@ -282,37 +329,53 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
     cudaFuncSetAttribute(sweep_kernel<kModeForced>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
     attr_done = true;
   }
+  cudaError_t e = tc::launch_split(U, d, d, d, w.U_hi, w.U_lo, d, info, st);
+  if (e != cudaSuccess) return e;
+  const tc::Operand Ep{w.Err_hi, w.Err_lo, rows, kMaxBlock, kMaxBlock};
+  const tc::Operand Up{w.U_hi, w.U_lo, d, d, d};
   const int B = p.blocksize;
   const int sweep_grid = cdiv(rows, kSweepRows);
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
     if (p.forced) {
       sweep_kernel<kModeForced><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info);
       count_launches(1);
     } else if (p.pattern == SGPT_PATTERN_NM) {
       sweep_kernel<kModeNM24><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info);
       count_launches(1);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
-      select_init_kernel<<<1, 256, 0, st>>>(sel, (unsigned int)kk);
+      select_init_kernel<<<1, 256, 0, st>>>(w.sel, (unsigned int)kk);
       count_launches(1);
       const long long total4 = (long long)rows * (bw / 4);
       const int g = (int)std::min<long long>(cdivll(total4, 256 * 8), 4 * kNumSMs);
       for (int pass = 0; pass < 8; ++pass) {
-        select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, sel, pass, info);
+        select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, w.sel, pass, info);
         count_launches(1);
       }
       sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, &sel->thr, info);
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, info);
       count_launches(1);
     }
     const int i2 = i1 + bw;
     if (i2 < d) {
-      dim3 grid(cdiv(d - i2, kTile), cdiv(rows, kTile));
-      trailing_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(W, ldw, rows, d, i1, bw, U, Err, info);
-      count_launches(1);
+      tc::Job job{};
+      job.mode = 0;
+      job.mt = cdiv(rows, kTile);
+      job.nt = cdiv(d - i2, kTile);
+      job.kdim = bw;
+      job.b_x0 = i2;
+      job.b_y0 = i1;
+      job.C = W;
+      job.ldc = ldw;
+      job.c_col0 = i2;
+      job.Mlim = rows;
+      job.Nlim = d - i2;
+      job.alpha = -1.f;
+      job.beta = 1.f;
+      if ((e = tc::launch_gemm(Ep, Up, true, job, job.mt * job.nt, info, st)) != cudaSuccess) return e;
     }
   }
   return cudaGetLastError();
@@ -379,11 +442,11 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
     const int bw = min(B, d - i1);
     if (p.forced) {
       sweep_kernel<kModeForced><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info);
       count_launches(1);
     } else if (p.pattern == SGPT_PATTERN_NM) {
       sweep_kernel<kModeNM24><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, info);
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info);
       count_launches(1);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
@@ -396,7 +459,7 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
         count_launches(1);
       }
       sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, &sel->thr, info);
+          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info);
       count_launches(1);
     }
     const int i2 = i1 + bw;

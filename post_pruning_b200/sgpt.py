@@ -314,11 +314,21 @@ class LayerBuffers:
     info: torch.Tensor
 
     @classmethod
-    def allocate(cls, d_out: int, d_in: int, n_tok: int, device="cuda") -> "LayerBuffers":
+    def sharing(cls, other: "LayerBuffers", d_out: int, device="cuda") -> "LayerBuffers":
+        """Buffers for another weight matrix that reads the same input: it
+        shares H and U (factor once, sweep each matrix) and has its own
+        outputs and workspace."""
+        mine = cls.allocate(d_out, other.d_in, 0, device, with_hu=False)
+        mine.H, mine.U, mine.n_tok = other.H, other.U, other.n_tok
+        return mine
+
+    @classmethod
+    def allocate(cls, d_out: int, d_in: int, n_tok: int, device="cuda", with_hu: bool = True) -> "LayerBuffers":
         f32 = dict(dtype=torch.float32, device=device)
         i32 = dict(dtype=torch.int32, device=device)
+        hu = (d_in, d_in) if with_hu else (0, 0)
         return cls(d_out, d_in, n_tok,
-                   H=torch.empty((d_in, d_in), **f32), U=torch.empty((d_in, d_in), **f32),
+                   H=torch.empty(hu, **f32), U=torch.empty(hu, **f32),
                    mask=torch.empty((d_out, d_in // 32), **i32),
                    values=torch.empty((d_out, d_in // 2), **f32),
                    meta=torch.empty((d_out, d_in // 32), **i32),
@@ -331,6 +341,59 @@ class LayerBuffers:
         prune_layer(W, self.H, self.U, params, self.mask, self.ws, self.info, X=X,
                     n_tok=self.n_tok, values=self.values if pack else None,
                     meta=self.meta if pack else None, row_loss=self.row_loss, stream=stream)
+
+
+class LayerGraphs:
+    """The four phases of one layer prune captured as CUDA graphs.
+
+    hessian (zero + accumulate), factor, prune (row loss cleared + sweep) and,
+    for 2:4, pack. Replaying them in order does exactly what
+    LayerBuffers.run does, with the launch overhead of one graph per phase.
+    Capture reads no data: buffers are bound by address, so W and X must
+    stay where they were at capture time. Replay on the current stream with
+    replay(), or phase by phase through .graphs.
+    """
+
+    PHASES = ("hessian", "factor", "prune", "pack")
+
+    def __init__(self, bufs: LayerBuffers, W: torch.Tensor, X: torch.Tensor | None, params: Params,
+                 phases=PHASES):
+        self.bufs, self.W, self.X, self.params = bufs, W, X, params
+        self.phases = tuple(ph for ph in phases if not (ph == "pack" and not params.is_nm))
+        # one eager pass first: per-process kernel attributes are set outside capture
+        self._eager()
+        torch.cuda.synchronize()
+        self.graphs = {}
+        self.kernels = {}        # libsgpt kernels captured in each graph
+        for name in self.phases:
+            g = torch.cuda.CUDAGraph()
+            before = kernel_launches()
+            with torch.cuda.graph(g):
+                self._phase(name)
+            self.kernels[name] = kernel_launches() - before
+            self.graphs[name] = g
+
+    def _phase(self, name: str):
+        b, p = self.bufs, self.params
+        if name == "hessian":
+            info_clear(b.info)
+            hessian_zero(b.H)
+            hessian_accumulate(b.H, self.X, b.ws, b.info)
+        elif name == "factor":
+            factor(b.H, b.n_tok, p.damp, b.U, b.ws, b.info)
+        elif name == "prune":
+            b.row_loss.zero_()
+            prune(self.W, b.U, p, b.mask, b.ws, b.info, row_loss=b.row_loss)
+        elif name == "pack":
+            pack24(self.W, b.mask, b.values, b.meta, b.info)
+
+    def _eager(self):
+        for name in self.phases:
+            self._phase(name)
+
+    def replay(self):
+        for g in self.graphs.values():
+            g.replay()
 
 
 class HostPruner:

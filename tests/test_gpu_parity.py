@@ -256,3 +256,29 @@ def test_bad_mask_is_reported():
     info = pp.new_info()
     pp.pack24(W, mask, vals, meta, info)
     assert pp.sync_status(info) == 7
+
+
+def test_hessian_long_accumulation():
+    """Many tokens per CTA (d = 2048: 72 tiles, two token splits of 32,768):
+    sums of positive terms must not drift (sampled entries vs float64)."""
+    spec = LayerSpec("long", d_in=2048, d_out=128, n_tok=65536, seed=4)
+    dev = torch.device("cuda")
+    X = gen_activations(spec, device=dev)
+    H = torch.zeros(spec.d_in, spec.d_in, device=dev)
+    info = pp.new_info()
+    pp.hessian_accumulate(H, X, pp.workspace(spec.d_out, spec.d_in, spec.n_tok), info)
+    pp.raise_on_info(info)
+    Xh = bf16_bits_to_f64(X.cpu()).numpy()
+    rng = np.random.default_rng(0)
+    cols = rng.choice(spec.d_in, 48, replace=False)
+    Hh = H.cpu().numpy().astype(np.float64)
+    for c in cols:
+        ref = float(np.dot(Xh[:, c], Xh[:, c]))
+        # an accumulator that drifts by a fraction of an ulp per MMA step is
+        # off by ~1e-3 here; chunked accumulation keeps it near 1e-6
+        assert abs(Hh[c, c] - ref) <= 1e-5 * ref, (c, Hh[c, c] / ref - 1)
+    for a, b in zip(cols[:24], cols[24:]):
+        ref = float(np.dot(Xh[:, a], Xh[:, b]))
+        absref = float(np.dot(np.abs(Xh[:, a]), np.abs(Xh[:, b])))
+        assert abs(Hh[a, b] - ref) <= 2e-6 * absref
+        assert Hh[a, b] == Hh[b, a]
