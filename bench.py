@@ -37,6 +37,7 @@ WORKLOADS = {
                      "0.5% outlier channels x50), 2:4"),
     "llama7b_q": ("Llama-7B q_proj: W 4096x4096 fp32, X 262144x4096 bf16, unstructured 50/70/80% "
                   "(three layer prunes per step)"),
+    "profile_4096": "4096x4096 layer, 32768 tokens, 2:4 (profiler captures)",
     "qwen3_32b_block": ("Qwen3-32B-shaped block: q 5120->8192, k/v 5120->1024, o 8192->5120, gate/up "
                         "5120->25600, down 25600->5120, 131072 tokens, 2:4; H and U shared by q/k/v and by "
                         "gate/up (4 Hessians, 7 sweeps per step)"),
@@ -57,6 +58,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", default=CONFIG, help="workload (default: the OPT-125M-shaped layer)")
     return ap.parse_args()
+
+
+# DRAM bytes (read + write) of one hessian_tc_kernel launch, from the ncu
+# capture summarised in profiles/hessian_tc_kernel_opt125m_768.md; re-capture
+# when the kernel changes.
+HESSIAN_TRAFFIC = {"opt125m_768": 407.7e6}
 
 
 def peaks():
@@ -353,7 +360,8 @@ def main():
     achieved = hess_flops / (phase["hessian"] * 1e-3) / 1e12
     roofline = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": achieved,
                 "peak": bf16_burst, "unit": "TFLOP/s", "frac": achieved / bf16_burst,
-                "traffic": None, "peak_kind": f"{peak_kind} bf16 burst",
+                "traffic": HESSIAN_TRAFFIC.get(args.config), "traffic_unit": "bytes per launch",
+                "peak_kind": f"{peak_kind} bf16 burst",
                 "work": f"n*d*(d+1) = {hess_flops / n_hess:.4g} flop per launch (upper triangle incl. "
                         f"diagonal), {n_hess} launches per step"}
 

@@ -48,11 +48,12 @@ __host__ __device__ __forceinline__ long long cdivll(long long a, long long b) {
   return (a + b - 1) / b;
 }
 
-// Saliency of weight w in a column whose U diagonal is u: (w / u)^2 in fp32
-// with IEEE division. Every kernel that ranks weights calls this one function,
-// so the selection kernels and the sweep agree bit for bit.
-__device__ __forceinline__ float saliency(float w, float u) {
-  float t = __fdiv_rn(w, u);
+// Saliency w^2 / U_cc^2 of weight w in a column whose U diagonal has the
+// reciprocal inv_u = 1 / U_cc (IEEE-rounded once per column): (w * inv_u)^2
+// in fp32. Every kernel that ranks weights calls this one function with the
+// same reciprocal, so the selection kernels and the sweep agree bit for bit.
+__device__ __forceinline__ float saliency(float w, float inv_u) {
+  const float t = __fmul_rn(w, inv_u);
   return __fmul_rn(t, t);
 }
 

@@ -10,14 +10,15 @@
 // the sweep consumes it.
 //
 // Blocking: 128 x 128 tiles. Diagonal blocks are factored and inverted in
-// shared memory by one CTA; the panel solve and the V scaling are FP32 SIMT
-// tile products; the rank-128 updates of the leading part and the
-// triangular inverse (the d^3/3 + d^3/3 flops) run on the tensor cores as
-// FP32-accurate three-product TF32 GEMMs (gemm_tc.cu).
+// shared memory by one CTA; every other product (the panel R_ik = A_ik
+// U_kk^T, the rank-128 updates of the leading part, V_im = U_ii R_im and
+// the triangular inverse) runs on the tensor cores as an FP32-accurate
+// three-product TF32 GEMM (gemm_tc.cu). Operands move between those GEMMs
+// as hi/lo planes written by the producing epilogue, so no separate split
+// pass runs except once for the last column block.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
-#include "gemm_simt.cuh"
 #include "gemm_tc.h"
 #include "kernels.h"
 
@@ -90,47 +91,88 @@ __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict
 // and read the other operand's rows as broadcast 16-byte loads.
 
 constexpr int kDiagThreads = 256;
+constexpr int kDiagWarps = kDiagThreads / 32;
 constexpr int kDiagLd = kTile + 4;     // 16-byte aligned rows
-constexpr size_t kDiagSmem = 2 * (size_t)kTile * kDiagLd * sizeof(float);
+constexpr size_t kDiagSmem = 3 * (size_t)kTile * kDiagLd * sizeof(float);
 
-// acc[i] = sum_k A[i][k] * b[k] for the 32 rows of A (row stride kDiagLd,
-// 16-byte aligned, read as broadcasts), b in registers.
-__device__ __forceinline__ void rows_dot32(const float* A, const float (&b)[32], float (&acc)[32]) {
+// sum_k a[k] * b[k] over 32 entries: a is a shared-memory row (16-byte
+// aligned, read as broadcasts), b is in registers.
+__device__ __forceinline__ float row_dot32(const float* a, const float (&b)[32]) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float* a = A + i * kDiagLd;
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(a + k);
-      s = fmaf(x.x, b[k], s);
-      s = fmaf(x.y, b[k + 1], s);
-      s = fmaf(x.z, b[k + 2], s);
-      s = fmaf(x.w, b[k + 3], s);
-    }
-    acc[i] = s;
+  for (int k = 0; k < 32; k += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(a + k);
+    s0 = fmaf(x.x, b[k], s0);
+    s1 = fmaf(x.y, b[k + 1], s1);
+    s2 = fmaf(x.z, b[k + 2], s2);
+    s3 = fmaf(x.w, b[k + 3], s3);
   }
+  return (s0 + s1) + (s2 + s3);
 }
 
+// Row `lane` of a 32-wide shared-memory block into registers.
+__device__ __forceinline__ void load_row32(const float* blk, int lane, float (&b)[32]) {
+  const float* r = blk + lane * kDiagLd;
+#pragma unroll
+  for (int k = 0; k < 32; k += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(r + k);
+    b[k] = x.x; b[k + 1] = x.y; b[k + 2] = x.z; b[k + 3] = x.w;
+  }
+}
+// Column `lane` of a 32 x 32 shared-memory block into registers.
+__device__ __forceinline__ void load_col32(const float* blk, int lane, float (&b)[32]) {
+#pragma unroll
+  for (int k = 0; k < 32; ++k) b[k] = blk[k * kDiagLd + lane];
+}
+
+// 1/sqrt(x) to about 1 ulp: the hardware estimate and one Newton step.
+__device__ __forceinline__ float rsqrt_nr(float x) {
+  const float y = rsqrtf(x);
+  return y * fmaf(-0.5f * x * y, y, 1.5f);
+}
+
+// Units of work for the eight warps: (32 x 32 block, 8-row quarter) pairs.
+__device__ __forceinline__ void tri_pair(int t, int& i, int& j) {   // t -> (i <= j)
+  int jj = 0;
+  while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
+  j = jj;
+  i = t - jj * (jj + 1) / 2;
+}
+
+// One CTA factors the diagonal block A_kk = R_kk R_kk^T (R_kk upper) and
+// inverts it, U_kk = R_kk^-1, in FP32 shared memory, as up to 4 x 4
+// sub-blocks of 32 processed from the last 32-panel to the first:
+//   1. warp 0 factors the panel's 32 x 32 diagonal sub-block (lane = row; the
+//      pivot column is broadcast by shuffles) and inverts it
+//      (lane = column, back substitution);
+//   2. R_ip = A_ip U_pp^T for the sub-blocks above, and
+//   3. A_ij -= R_ip R_jp^T for the leading sub-blocks, both spread over all
+//      warps in 8-row units (lane = output column).
+// Then V_pm = U_pp R_pm and the off-diagonal blocks of U along the
+// anti-diagonals, U_pq = -sum_{m=p+1..q} V_pm U_mq, in the same units.
 __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const float* __restrict__ Rws,
                                                                       int d, int k,
-                                                                      float* __restrict__ Ukk,
                                                                       float* __restrict__ U,
+                                                                      float* __restrict__ U_hi,
+                                                                      float* __restrict__ U_lo,
                                                                       int* info) {
   if (cta_info_set(info)) return;
   extern __shared__ __align__(16) float dsm[];
-  float* S = dsm;                        // A, becoming R (upper)
-  float* Ui = dsm + kTile * kDiagLd;     // U (upper)
+  float* S = dsm;                            // A, becoming R (upper)
+  float* Ui = dsm + kTile * kDiagLd;         // U (upper)
+  float* Vb = dsm + 2 * kTile * kDiagLd;     // V_pm blocks
   __shared__ float rinv[kTile];
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b0 = k * kTile;
-  const int b = min(kTile, d - b0);      // a multiple of 32
+  const int b = min(kTile, d - b0);          // a multiple of 32
   const int np = b >> 5;
-  for (int e = tid; e < kTile * kTile; e += kDiagThreads) {
+  for (int e = tid * 4; e < kTile * kTile; e += kDiagThreads * 4) {
     const int i = e >> 7, l = e & 127;
-    S[i * kDiagLd + l] = (i <= l && l < b) ? Rws[(long long)(b0 + i) * d + b0 + l] : 0.f;
-    Ui[i * kDiagLd + l] = 0.f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < b && l < b) v = ld4(Rws + (long long)(b0 + i) * d + b0 + l);
+    st4(S + i * kDiagLd + l, v);             // only entries i <= l are ever read
+    st4(Ui + i * kDiagLd + l, make_float4(0.f, 0.f, 0.f, 0.f));
   }
   if (tid == 0) bad = 0;
   __syncthreads();
@@ -138,215 +180,170 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
   for (int p = np - 1; p >= 0; --p) {
     const int c0 = p * 32;
     if (warp == 0) {
-      // ---- reverse Cholesky of the 32 x 32 diagonal sub-block, lane = row
+      // ---- reverse Cholesky of the 32 x 32 diagonal sub-block, lane = row.
+      // Pivot j: r_jj = sqrt(a_jj), r_ij = a_ij / r_jj (i < j), then
+      // a_il -= r_ij r_lj for l < j. Entries below the diagonal (l < i)
+      // take the update too but are never read, and are zeroed on output.
       float dr[32];
       float* row = S + (c0 + lane) * kDiagLd + c0;
-#pragma unroll
-      for (int l = 0; l < 32; ++l) dr[l] = row[l];
+      load_row32(S + c0 * kDiagLd + c0, lane, dr);
       int fail = 0;
 #pragma unroll
       for (int j = 31; j >= 0; --j) {
         const float piv = __shfl_sync(0xffffffffu, dr[j], j);
         if (!(piv > 0.f) && fail == 0) fail = isfinite(piv) ? (b0 + c0 + j + 1) : SGPT_INFO_NONFINITE;
-        const float sq = sqrtf(piv);
-        const float inv = 1.0f / sq;
-        const float rij = lane < j ? dr[j] * inv : (lane == j ? sq : 0.f);
+        const float rs = rsqrt_nr(piv);
+        const float rij = lane < j ? dr[j] * rs : (lane == j ? piv * rs : 0.f);
+        dr[j] = rij;
+        if (j == 0) break;
 #pragma unroll
         for (int l = 0; l < j; ++l) {
-          const float rlj = __shfl_sync(0xffffffffu, rij, l);
-          if (lane <= l) dr[l] = fmaf(-rij, rlj, dr[l]);
+          const float c = __shfl_sync(0xffffffffu, rij, l);
+          dr[l] = fmaf(-rij, c, dr[l]);
         }
-        dr[j] = rij;
       }
 #pragma unroll
-      for (int l = 0; l < 32; ++l) row[l] = lane <= l ? dr[l] : 0.f;
+      for (int l = 0; l < 32; l += 4)
+        *reinterpret_cast<float4*>(row + l) =
+            make_float4(lane <= l ? dr[l] : 0.f, lane <= l + 1 ? dr[l + 1] : 0.f,
+                        lane <= l + 2 ? dr[l + 2] : 0.f, lane <= l + 3 ? dr[l + 3] : 0.f);
+      rinv[c0 + lane] = 1.0f / row[lane];
       if (fail && lane == 0) bad = fail;
+      __syncwarp();
+      // ---- U_pp = R_pp^-1, lane = column j: back substitution from the
+      // bottom, u_i = (delta_ij - sum_{m>i} r_im u_m) / r_ii.
+      float u[32];
+      const float* R = S + c0 * kDiagLd + c0;
+#pragma unroll
+      for (int i = 31; i >= 0; --i) {
+        const float* ri = R + i * kDiagLd;
+        float a0 = (i == lane) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int m = i + 1; m < 32; ++m) {
+          const float r = ri[m];
+          if ((m & 3) == 0) a0 = fmaf(-r, u[m], a0);
+          else if ((m & 3) == 1) a1 = fmaf(-r, u[m], a1);
+          else if ((m & 3) == 2) a2 = fmaf(-r, u[m], a2);
+          else a3 = fmaf(-r, u[m], a3);
+        }
+        u[i] = (i <= lane) ? ((a0 + a1) + (a2 + a3)) * rinv[c0 + i] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Ui[(c0 + i) * kDiagLd + c0 + lane] = u[i];
     }
     __syncthreads();
     if (bad) {
       if (tid == 0) set_info(info, bad);
       return;
     }
-    if (warp == 0) {
-      rinv[c0 + lane] = 1.0f / S[(c0 + lane) * kDiagLd + c0 + lane];
-      __syncwarp();
-      // ---- U_pp = R_pp^-1, lane = column j: back substitution from the bottom
-      float u[32];
-      const float* R = S + c0 * kDiagLd + c0;
-#pragma unroll
-      for (int i = 31; i >= 0; --i) {
-        float sacc = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-        for (int m = i + 1; m < 32; ++m) sacc = fmaf(-R[i * kDiagLd + m], u[m], sacc);
-        u[i] = (i <= lane) ? sacc * rinv[c0 + i] : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) Ui[(c0 + i) * kDiagLd + c0 + lane] = u[i];
-    }
-    __syncthreads();
     if (p == 0) break;
-    // ---- panel: R_ip = A_ip U_pp^T, rows blocks i < p (in place)
-    if (warp < p) {
-      float bcol[32], acc[32];
-      const float* ur = Ui + (c0 + lane) * kDiagLd + c0;    // row `lane` of U_pp = column of U_pp^T
+    // ---- panel: R_ip = A_ip U_pp^T for the row blocks i < p (in place);
+    // unit = 8 rows, lane = output column j with row j of U_pp in registers.
+    {
+      float bu[32];
+      load_row32(Ui + c0 * kDiagLd + c0, lane, bu);
+      for (int unit = warp; unit < p * 4; unit += kDiagWarps) {
+        float* A = S + (unit * 8) * kDiagLd + c0;
+        float v[8];
 #pragma unroll
-      for (int m = 0; m < 32; m += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(ur + m);
-        bcol[m] = x.x; bcol[m + 1] = x.y; bcol[m + 2] = x.z; bcol[m + 3] = x.w;
+        for (int i = 0; i < 8; ++i) v[i] = row_dot32(A + i * kDiagLd, bu);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) A[i * kDiagLd + lane] = v[i];
       }
-      float* Ablk = S + (warp * 32) * kDiagLd + c0;
-      rows_dot32(Ablk, bcol, acc);
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) Ablk[i * kDiagLd + lane] = acc[i];
     }
     __syncthreads();
     // ---- update of the leading sub-blocks: A_ij -= R_ip R_jp^T, i <= j < p
     {
-      const int pairs = p * (p + 1) / 2;
-      if (warp < pairs) {
-        int jj = 0;
-        while ((jj + 1) * (jj + 2) / 2 <= warp) ++jj;
-        const int ii = warp - jj * (jj + 1) / 2;          // ii <= jj
-        float bcol[32], acc[32];
-        const float* rp = S + (jj * 32 + lane) * kDiagLd + c0;   // row of R_jp = column of R_jp^T
+      const int units = p * (p + 1) / 2 * 4;
+      for (int unit = warp; unit < units; unit += kDiagWarps) {
+        int ii, jj;
+        tri_pair(unit >> 2, ii, jj);
+        const int r0 = ii * 32 + (unit & 3) * 8;
+        float br[32];
+        load_row32(S + (jj * 32) * kDiagLd + c0, lane, br);   // row `lane` of R_jp
+        float* C = S + r0 * kDiagLd + jj * 32;
+        const float* Ai = S + r0 * kDiagLd + c0;
 #pragma unroll
-        for (int m = 0; m < 32; m += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(rp + m);
-          bcol[m] = x.x; bcol[m + 1] = x.y; bcol[m + 2] = x.z; bcol[m + 3] = x.w;
-        }
-        rows_dot32(S + (ii * 32) * kDiagLd + c0, bcol, acc);
-        float* C = S + (ii * 32) * kDiagLd + jj * 32;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) C[i * kDiagLd + lane] -= acc[i];
+        for (int i = 0; i < 8; ++i) C[i * kDiagLd + lane] -= row_dot32(Ai + i * kDiagLd, br);
       }
     }
     __syncthreads();
   }
 
-  // ---- V_pm = U_pp R_pm (p < m), in place over R_pm: lane = column of R_pm
+  // ---- V_pm = U_pp R_pm (p < m) into Vb; unit = 8 rows, lane = column
   {
-    const int pairs = np * (np - 1) / 2;
-    if (warp < pairs) {
-      int mm = 0;
-      while ((mm + 1) * (mm + 2) / 2 <= warp) ++mm;
-      const int pp = warp - mm * (mm + 1) / 2;            // pp <= mm
-      mm += 1;                                             // pp < mm
-      float bcol[32], acc[32];
-      float* Rpm = S + (pp * 32) * kDiagLd + mm * 32;
+    const int units = np * (np - 1) / 2 * 4;
+    for (int unit = warp; unit < units; unit += kDiagWarps) {
+      int pp, mm;
+      tri_pair(unit >> 2, pp, mm);      // pp <= mm-1
+      mm += 1;
+      const int r0 = (unit & 3) * 8;
+      float bcol[32];
+      load_col32(S + (pp * 32) * kDiagLd + mm * 32, lane, bcol);
+      const float* Upp = Ui + (pp * 32 + r0) * kDiagLd + pp * 32;
+      float* V = Vb + (pp * 32 + r0) * kDiagLd + mm * 32;
 #pragma unroll
-      for (int kk = 0; kk < 32; ++kk) bcol[kk] = Rpm[kk * kDiagLd + lane];
-      rows_dot32(Ui + (pp * 32) * kDiagLd + pp * 32, bcol, acc);
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) Rpm[i * kDiagLd + lane] = acc[i];
+      for (int i = 0; i < 8; ++i) V[i * kDiagLd + lane] = row_dot32(Upp + i * kDiagLd, bcol);
     }
   }
   __syncthreads();
   // ---- off-diagonal blocks of U by anti-diagonals: U_pq = -sum V_pm U_mq
   for (int sd = 1; sd < np; ++sd) {
-    if (warp < np - sd) {
-      const int pp = warp, qq = warp + sd;
-      float acc[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    const int units = (np - sd) * 4;
+    for (int unit = warp; unit < units; unit += kDiagWarps) {
+      const int pp = unit >> 2, qq = pp + sd, r0 = (unit & 3) * 8;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int mm = pp + 1; mm <= qq; ++mm) {
-        float bcol[32], part[32];
-        const float* Umq = Ui + (mm * 32) * kDiagLd + qq * 32;
+        float bcol[32];
+        load_col32(Ui + (mm * 32) * kDiagLd + qq * 32, lane, bcol);
+        const float* V = Vb + (pp * 32 + r0) * kDiagLd + mm * 32;
 #pragma unroll
-        for (int kk = 0; kk < 32; ++kk) bcol[kk] = Umq[kk * kDiagLd + lane];
-        rows_dot32(S + (pp * 32) * kDiagLd + mm * 32, bcol, part);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] += part[i];
+        for (int i = 0; i < 8; ++i) acc[i] += row_dot32(V + i * kDiagLd, bcol);
       }
-      float* Upq = Ui + (pp * 32) * kDiagLd + qq * 32;
+      float* Upq = Ui + (pp * 32 + r0) * kDiagLd + qq * 32;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) Upq[i * kDiagLd + lane] = -acc[i];
+      for (int i = 0; i < 8; ++i) Upq[i * kDiagLd + lane] = -acc[i];
     }
     __syncthreads();
   }
 
-  // Write U_kk (upper, zeros below) to the output and to the block cache.
+  // Write U_kk (upper, zeros below) and its hi/lo planes.
   for (int e = tid * 4; e < kTile * kTile; e += kDiagThreads * 4) {
     const int i = e >> 7, l = e & 127;
+    if (i >= b || l >= b) continue;
     const float4 v = *reinterpret_cast<const float4*>(Ui + i * kDiagLd + l);
-    st4(Ukk + e, v);
-    if (i < b && l < b) st4(U + (long long)(b0 + i) * d + b0 + l, v);
+    const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+    const long long off = (long long)(b0 + i) * d + b0 + l;
+    st4(U + off, v);
+    st4(U_hi + off, h);
+    st4(U_lo + off, make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w));
   }
-}
-
-// ------------------------------------------------- off-diagonal products
-
-// Panel: R_ik = A_ik U_kk^T for every row block i < k (in place).
-__global__ void __launch_bounds__(kGemmThreads) panel_kernel(float* __restrict__ Rws, int d, int k,
-                                                             const float* __restrict__ Ukk,
-                                                             const int* info) {
-  if (cta_info_set(info)) return;
-  extern __shared__ float smem[];
-  const int i = blockIdx.x;
-  const int bk = min(kTile, d - k * kTile);
-  float acc[8][8];
-  zero_acc(acc);
-  const OpKContig A{Rws + k * kTile, d, i * kTile, kTile, bk};
-  const OpKContig B{Ukk, kTile, 0, bk, bk};
-  gemm_tile(A, B, 0, bk, acc, smem);
-  store_tile(Rws + (long long)i * kTile * d + k * kTile, d, kTile, bk, acc, 1.f, 0.f);
-}
-
-__device__ __forceinline__ void upper_tile_index(int t, int& i, int& j) {
-  // t enumerates (i <= j) row by row: row i holds tiles j = i .. n-1; with n
-  // unknown here we enumerate by j instead: column j holds i = 0..j.
-  int jj = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-  while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
-  while (jj * (jj + 1) / 2 > t) --jj;
-  j = jj;
-  i = t - jj * (jj + 1) / 2;
-}
-
-// V_im = U_ii R_im for every off-diagonal block i < m (in place over R).
-__global__ void __launch_bounds__(kGemmThreads) vscale_kernel(float* __restrict__ Rws, int d,
-                                                              const float* __restrict__ Udiag,
-                                                              const int* info) {
-  if (cta_info_set(info)) return;
-  extern __shared__ float smem[];
-  int i, m;
-  upper_tile_index(blockIdx.x, i, m);   // i <= m-1 enumerated as (i, m-1)
-  m += 1;
-  const int bm = min(kTile, d - m * kTile);
-  float acc[8][8];
-  zero_acc(acc);
-  const OpKContig A{Udiag + (size_t)i * kTile * kTile, kTile, 0, kTile, kTile};
-  const OpIContig B{Rws + (long long)i * kTile * d, d, m * kTile, bm, kTile};
-  gemm_tile(A, B, 0, kTile, acc, smem);
-  store_tile(Rws + (long long)i * kTile * d + m * kTile, d, kTile, bm, acc, 1.f, 0.f);
 }
 
 // ----------------------------------------------------------------- driver
 
 struct FactorWs {
   double* lam;
-  float* R;        // H_d, then R, then V; finally the hi plane of V
-  float* Udiag;    // U_kk blocks, 128 x 128 each
-  float* P_hi;     // hi/lo planes of the current panel (d x 128)
-  float* P_lo;
-  float* V_lo;     // lo plane of V (d x d)
+  float* R;        // H_d, then R; the hi plane of R_ik and then of V_ik above the diagonal blocks
+  float* V_lo;     // lo plane of R_ik, then of V_ik (d x d)
   float* U_hi;     // hi/lo planes of U (d x d)
   float* U_lo;
+  float* A_hi;     // hi/lo planes of the next column block of the updated H_d (d x 128)
+  float* A_lo;
   float* part;     // split partials of the triangular inverse
 };
 
 static FactorWs carve_factor(void* ws, int d, size_t* bytes) {
   Carve c(ws);
-  const int K = cdiv(d, kTile);
   FactorWs w;
   w.lam = c.take<double>(4);
   w.R = c.take<float>((size_t)d * d);
-  w.Udiag = c.take<float>((size_t)K * kTile * kTile);
-  w.P_hi = c.take<float>((size_t)d * kTile);
-  w.P_lo = c.take<float>((size_t)d * kTile);
   w.V_lo = c.take<float>((size_t)d * d);
   w.U_hi = c.take<float>((size_t)d * d);
   w.U_lo = c.take<float>((size_t)d * d);
+  w.A_hi = c.take<float>((size_t)d * kTile);
+  w.A_lo = c.take<float>((size_t)d * kTile);
   w.part = c.take<float>(factor_part_tiles(d) * kTile * kTile);
   if (bytes) *bytes = c.off + 256;
   return w;
@@ -393,35 +390,71 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
   count_launches(1);
   if (U == H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
   cudaError_t e = cudaSuccess;
+  // planes of the last column block above its diagonal block
+  if (K > 1 && (e = tc::launch_split(w.R + (K - 1) * kTile, d, (K - 1) * kTile, d - (K - 1) * kTile, w.A_hi,
+                                     w.A_lo, kTile, info, st)) != cudaSuccess)
+    return e;
   for (int k = K - 1; k >= 0; --k) {
-    diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, st>>>(w.R, d, k, w.Udiag + (size_t)k * kTile * kTile, U, info);
+    const int c0 = k * kTile, bk = min(kTile, d - c0);
+    diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, st>>>(w.R, d, k, U, w.U_hi, w.U_lo, info);
     count_launches(1);
     if (k == 0) break;
-    const int bk = min(kTile, d - k * kTile);
-    panel_kernel<<<k, kGemmThreads, kGemmSmemBytes, st>>>(w.R, d, k, w.Udiag + (size_t)k * kTile * kTile, info);
-    count_launches(1);
-    // rank-bk update of the leading upper tiles on the tensor cores
-    if ((e = tc::launch_split(w.R + k * kTile, d, k * kTile, bk, w.P_hi, w.P_lo, kTile, info, st)) != cudaSuccess)
-      return e;
-    const tc::Operand P{w.P_hi, w.P_lo, (long long)k * kTile, kTile, kTile};
-    tc::Job job{};
-    job.mode = 1;
-    job.kdim = bk;
-    job.C = w.R;
-    job.ldc = d;
-    job.Mlim = job.Nlim = k * kTile;
-    job.alpha = -1.f;
-    job.beta = 1.f;
-    if ((e = tc::launch_gemm(P, P, false, job, k * (k + 1) / 2, info, st)) != cudaSuccess) return e;
+    {
+      // panel R_ik = A_ik U_kk^T for the rows above, written as hi/lo planes
+      // (hi over R, lo into V_lo)
+      const tc::Operand A{w.A_hi, w.A_lo, c0, bk, kTile};
+      const tc::Operand B{w.U_hi + (long long)c0 * d + c0, w.U_lo + (long long)c0 * d + c0, bk, bk, d};
+      tc::Job job{};
+      job.mode = 0;
+      job.mt = k;
+      job.nt = 1;
+      job.kdim = bk;
+      job.ldc = d;
+      job.c_col0 = c0;
+      job.Mlim = c0;
+      job.Nlim = bk;
+      job.alpha = 1.f;
+      job.C_hi = w.R;
+      job.C_lo = w.V_lo;
+      if ((e = tc::launch_gemm(A, B, false, job, k, info, st)) != cudaSuccess) return e;
+    }
+    {
+      // rank-bk update of the leading upper tiles, A_ij -= R_ik R_jk^T; the
+      // tiles of column block k-1 also write the planes the next panel reads
+      const tc::Operand P{w.R + c0, w.V_lo + c0, c0, bk, d};
+      tc::Job job{};
+      job.mode = 1;
+      job.kdim = bk;
+      job.C = w.R;
+      job.ldc = d;
+      job.Mlim = job.Nlim = c0;
+      job.alpha = -1.f;
+      job.beta = 1.f;
+      job.C_hi = w.A_hi;
+      job.C_lo = w.A_lo;
+      job.ldp = kTile;
+      job.p_col0 = c0 - kTile;
+      job.planes_one_col = 1;
+      job.planes_n0 = c0 - kTile;
+      if ((e = tc::launch_gemm(P, P, false, job, k * (k + 1) / 2, info, st)) != cudaSuccess) return e;
+    }
   }
   if (K > 1) {
-    vscale_kernel<<<K * (K - 1) / 2, kGemmThreads, kGemmSmemBytes, st>>>(w.R, d, w.Udiag, info);
-    count_launches(1);
-    // planes of V (hi in place over R) and of U (its diagonal blocks so far)
-    if ((e = tc::launch_split(w.R, d, d, d, w.R, w.V_lo, d, info, st)) != cudaSuccess) return e;
-    if ((e = tc::launch_split(U, d, d, d, w.U_hi, w.U_lo, d, info, st)) != cudaSuccess) return e;
-    const tc::Operand V{w.R, w.V_lo, d, d, d};
-    const tc::Operand Up{w.U_hi, w.U_lo, d, d, d};
+    // V_im = U_ii R_im above the diagonal blocks, as planes in place of R_im's
+    const tc::Operand Ud{w.U_hi, w.U_lo, d, d, d};
+    const tc::Operand Rp{w.R, w.V_lo, d, d, d};
+    {
+      tc::Job job{};
+      job.mode = 3;
+      job.dlim = d;
+      job.ldc = d;
+      job.Mlim = job.Nlim = d;
+      job.alpha = 1.f;
+      job.C_hi = w.R;
+      job.C_lo = w.V_lo;
+      if ((e = tc::launch_gemm(Ud, Rp, true, job, K * (K - 1) / 2, info, st)) != cudaSuccess) return e;
+    }
+    // off-diagonal blocks of U by anti-diagonals, U_pq = -sum_{m=p+1..q} V_pm U_mq
     for (int s = 1; s < K; ++s) {
       tc::Job job{};
       job.mode = 2;
@@ -437,7 +470,7 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
       job.C_hi = w.U_hi;
       job.C_lo = w.U_lo;
       job.part = w.part;
-      if ((e = tc::launch_gemm(V, Up, true, job, (K - s) * job.nsplit, info, st)) != cudaSuccess) return e;
+      if ((e = tc::launch_gemm(Rp, Ud, true, job, (K - s) * job.nsplit, info, st)) != cudaSuccess) return e;
     }
   }
   return cudaGetLastError();

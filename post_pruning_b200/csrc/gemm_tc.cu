@@ -11,9 +11,11 @@
 // Used for the rank-128 updates and the triangular inverse of the
 // factorisation and for the lazy trailing update of the OBS sweep.
 //
-// CTA tile 128 x 128, K in chunks of 32 (one 128-byte swizzle row of fp32),
-// three-stage TMA ring (no multicast); warp 0 lane 0 loads, warp 1 lane 0
-// issues MMAs, warps 2-5 drain TMEM (warp w reads lanes 32*(w%4)..).
+// CTA tile 128 x 128, K in chunks of 16 (one 64-byte swizzle row of fp32),
+// three-stage TMA ring in 96 KB (no multicast) so that two CTAs share an SM;
+// warp 0 lane 0 loads, warp 1 lane 0 issues MMAs, warps 2-5 drain TMEM
+// (warp w reads lanes 32*(w%4)..) into a shared staging tile and then update
+// C a whole row per warp instruction (coalesced).
 // A is always K-major (row-major M x K); B is K-major (row-major N x K) or
 // MN-major (row-major K x N). Every wait is bounded.
 #include <cuda.h>
@@ -30,12 +32,14 @@ namespace tc {
 
 namespace {
 
-constexpr int kM = 128, kN = 128, kKC = 32;
+constexpr int kM = 128, kN = 128, kKC = 16;
 constexpr int kStages = 3;
-constexpr int kPlane = kM * kKC * 4;            // 16 KB: one operand plane of one stage
+constexpr int kPlane = kM * kKC * 4;            // 8 KB: one operand plane of one stage
 constexpr int kStageBytes = 4 * kPlane;         // A hi/lo, B hi/lo
 constexpr int kThreads = 192;
+constexpr int kStageLd = kN + 4;                // epilogue staging row (floats)
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256;
+static_assert((size_t)kM * kStageLd * 4 <= (size_t)kStages * kStageBytes, "staging must fit the stages");
 constexpr long long kWaitCycles = 4000000000ll;
 
 __host__ __device__ constexpr uint32_t make_idesc(bool b_mn) {
@@ -47,26 +51,27 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// K-major operand, 128-byte swizzle: 8-row groups of 1 KB.
+// K-major operand, 64-byte swizzle (a K chunk of 16 fp32 is one 64-byte
+// row): 8-row groups of 512 bytes.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3fff);
   d |= (uint64_t)1 << 16;                         // leading byte offset (unused when swizzled)
-  d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: next 8 rows
+  d |= (uint64_t)(512 >> 4) << 32;                // stride byte offset: next 8 rows
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)4 << 61;                         // SWIZZLE_64B
   return d;
 }
 // MN-major 32-bit operand: the 128-byte swizzle with 32-byte granules
 // (descriptor layout SWIZZLE_128B_BASE32B, filled by TMA's
 // SWIZZLE_128B_ATOM_32B). Atoms are 32 columns x 4 K rows (512 bytes);
-// LBO = next 32 columns (one 32-column x 32-row TMA box, 4 KB), SBO = next
+// LBO = next 32 columns (one 32-column x 16-row TMA box, 2 KB), SBO = next
 // 4 K rows. The plain 128-byte swizzle (16-byte granules) is not a valid
 // MN-major form for 32-bit elements.
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3fff);
-  d |= (uint64_t)(4096 >> 4) << 16;
+  d |= (uint64_t)(2048 >> 4) << 16;
   d |= (uint64_t)(512 >> 4) << 32;
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)1 << 61;
@@ -134,7 +139,7 @@ __device__ __forceinline__ void tri_index(int t, int& i, int& j) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
+__global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
     const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
     const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo, const Job job,
     const int b_mn, int* info) {
@@ -158,6 +163,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
     m0 = i * kM;
     n0 = j * kN;
     ke = job.kdim;
+  } else if (job.mode == 3) {
+    int i, j;
+    tri_index(blockIdx.x, i, j);
+    m0 = i * kM;
+    n0 = (j + 1) * kN;
+    kb = m0;
+    ke = min(m0 + kM, job.dlim);
   } else {
     tile = blockIdx.x / job.nsplit;
     split = blockIdx.x - tile * job.nsplit;
@@ -211,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
       if (b_mn) {
 #pragma unroll
         for (int c = 0; c < kN / 32; ++c) {
-          tma_2d(st + 2 * kPlane + c * 4096, &b_hi, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
-          tma_2d(st + 3 * kPlane + c * 4096, &b_lo, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
+          tma_2d(st + 2 * kPlane + c * 2048, &b_hi, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
+          tma_2d(st + 3 * kPlane + c * 2048, &b_lo, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
         }
       } else {
         tma_2d(st + 2 * kPlane, &b_hi, bar, job.b_x0 + k, job.b_y0 + n0);
@@ -252,6 +264,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
     mma_commit(done);
   }
 
+  const bool partial = job.mode == 2 && job.nsplit > 1;
+  const bool read_c = !partial && job.C != nullptr && job.beta != 0.f;
+  if (!skip && read_c && warp >= 2) {
+    // Bring this warp's 32 rows of C toward L2 while the main loop runs.
+    const int row = m0 + (warp - 2) * 32 + lane;
+    if (row < job.Mlim && n0 < job.Nlim) {
+      const float* p = job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + n0;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(min(kN, job.Nlim - n0) * 4)
+                   : "memory");
+    }
+  }
   bool have = !skip && iters > 0;
   if (have && warp >= 2) {
     __syncwarp();
@@ -265,9 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
   if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
 
   if (!skip && !failed && warp >= 2) {
+    // TMEM -> shared staging tile (the stage buffers are free once the last
+    // MMA has committed), then whole rows per warp to global memory.
+    float* T = reinterpret_cast<float*>(smem);
     const int q = warp & 3;
     const int m = q * 32 + lane;               // tile row = TMEM lane
-    const bool partial = job.mode == 2 && job.nsplit > 1;
 #pragma unroll 1
     for (int cc = 0; cc < kN / 32; ++cc) {
       uint32_t v[32];
@@ -277,38 +302,52 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      if (partial) {
-        float* dst = job.part + (size_t)blockIdx.x * kM * kN + (size_t)m * kN + cc * 32;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          st4(dst + e, make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                                   __uint_as_float(v[e + 3])));
-        continue;
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(T + m * kStageLd + cc * 32 + e) =
+            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                        __uint_as_float(v[e + 3]));
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");    // the four epilogue warps
+    const int col = lane * 4;                  // this lane's four columns of a row
+    const bool planes = job.C_hi != nullptr && (!job.planes_one_col || n0 == job.planes_n0);
+    const long long ldp = job.ldp ? job.ldp : job.ldc;
+    const bool col_ok = n0 + col < job.Nlim;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 32; r0 += 8) {
+      float4 a[8], old[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {            // all loads of 8 rows first
+        const int mr = (warp - 2) * 32 + r0 + u;
+        a[u] = *reinterpret_cast<const float4*>(T + mr * kStageLd + col);
+        old[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (read_c && col_ok && m0 + mr < job.Mlim)
+          old[u] = ld4(job.C + (long long)(job.c_row0 + m0 + mr) * job.ldc + job.c_col0 + n0 + col);
       }
-      const int row = m0 + m;
-      if (row >= job.Mlim) continue;
-      const long long off = (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + n0 + cc * 32;
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const int col = n0 + cc * 32 + e;
-        if (col >= job.Nlim) break;
-        float o[4];
-        float4 old = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (job.beta != 0.f) old = ld4(job.C + off + e);
-        o[0] = fmaf(job.alpha, __uint_as_float(v[e + 0]), job.beta * old.x);
-        o[1] = fmaf(job.alpha, __uint_as_float(v[e + 1]), job.beta * old.y);
-        o[2] = fmaf(job.alpha, __uint_as_float(v[e + 2]), job.beta * old.z);
-        o[3] = fmaf(job.alpha, __uint_as_float(v[e + 3]), job.beta * old.w);
-        st4(job.C + off + e, make_float4(o[0], o[1], o[2], o[3]));
-        if (job.C_hi) {
+      for (int u = 0; u < 8; ++u) {
+        const int mr = (warp - 2) * 32 + r0 + u;
+        if (partial) {
+          st4(job.part + (size_t)blockIdx.x * kM * kN + (size_t)mr * kN + col, a[u]);
+          continue;
+        }
+        const int row = m0 + mr;
+        if (row >= job.Mlim || !col_ok) continue;
+        const float o[4] = {fmaf(job.alpha, a[u].x, job.beta * old[u].x), fmaf(job.alpha, a[u].y, job.beta * old[u].y),
+                            fmaf(job.alpha, a[u].z, job.beta * old[u].z), fmaf(job.alpha, a[u].w, job.beta * old[u].w)};
+        if (job.C)
+          st4(job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + n0 + col,
+              make_float4(o[0], o[1], o[2], o[3]));
+        if (planes) {
+          const long long off = (long long)(job.c_row0 + row) * ldp + job.c_col0 + n0 + col - job.p_col0;
           float h4[4], l4[4];
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             h4[t] = tf32_hi(o[t]);
             l4[t] = o[t] - h4[t];
           }
-          st4(job.C_hi + off + e, make_float4(h4[0], h4[1], h4[2], h4[3]));
-          st4(job.C_lo + off + e, make_float4(l4[0], l4[1], l4[2], l4[3]));
+          st4(job.C_hi + off, make_float4(h4[0], h4[1], h4[2], h4[3]));
+          st4(job.C_lo + off, make_float4(l4[0], l4[1], l4[2], l4[3]));
         }
       }
     }
@@ -337,9 +376,9 @@ __global__ void __launch_bounds__(256) antidiag_reduce_kernel(const Job job, con
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     const float o[4] = {job.alpha * acc.x, job.alpha * acc.y, job.alpha * acc.z, job.alpha * acc.w};
-    const long long off = (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + col;
-    st4(job.C + off, make_float4(o[0], o[1], o[2], o[3]));
+    if (job.C) st4(job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + col, make_float4(o[0], o[1], o[2], o[3]));
     if (job.C_hi) {
+      const long long off = (long long)(job.c_row0 + row) * (job.ldp ? job.ldp : job.ldc) + job.c_col0 + col - job.p_col0;
       float h4[4], l4[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -389,8 +428,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // Tensor map over a row-major fp32 matrix [rows x cols] with leading dimension
-// ld; box = box_x (inner, fp32 elements) x box_y rows, 128-byte swizzle
-// (32-byte granules for MN-major operands).
+// ld; box = box_x (inner, fp32 elements) x box_y rows; 64-byte swizzle for
+// K-major operands (16-float rows), 128-byte swizzle with 32-byte granules
+// for MN-major ones (32-float rows).
 bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, long long ld, int box_x, int box_y,
               bool mn_major) {
   EncodeTiledFn enc = encode_fn();
@@ -401,7 +441,7 @@ bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, lo
   const cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE,
-             mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+             mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_64B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -20,11 +20,16 @@ struct Operand {
 //  mode 1: tiles (i, j), i <= j, enumerated column by column, K = kdim.
 //  mode 2: tiles (i, i + s) for i < nblk - s, K = [(i+1)*128, min((i+s+1)*128, dlim)),
 //          split into nsplit ranges whose partials are reduced in order.
+//  mode 3: tiles (i, m), i < m, enumerated like mode 1 over (i, m - 1),
+//          K = [i*128, min((i+1)*128, dlim)).
 // A(m, k) is read at (x = a_x0 + k, y = a_y0 + m0 + m); B(k, n) at
 // (x = b_x0 + k, y = b_y0 + n0 + n) if K-major, (x = b_x0 + n0 + n, y = b_y0 + k)
 // if MN-major. C(m, n) = alpha * acc + beta * C at
-// C[(c_row0 + m0 + m) * ldc + c_col0 + n0 + n] for m0+m < Mlim, n0+n < Nlim;
-// C_hi/C_lo (optional) receive the hi/lo planes of the result.
+// C[(c_row0 + m0 + m) * ldc + c_col0 + n0 + n] for m0+m < Mlim, n0+n < Nlim
+// (C may be null: no fp32 result). C_hi/C_lo (optional) receive the hi/lo
+// planes of the result at [(c_row0 + m0 + m) * ldp + c_col0 + n0 + n - p_col0]
+// (ldp = 0: ldc), from every tile or, with planes_one_col, only from the
+// tiles whose n0 == planes_n0.
 struct Job {
   int mode;
   int mt, nt;
@@ -38,6 +43,9 @@ struct Job {
   float alpha, beta;
   float* C_hi;
   float* C_lo;
+  long long ldp;
+  int p_col0;
+  int planes_one_col, planes_n0;
   float* part;
 };
 

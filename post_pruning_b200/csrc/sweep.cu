@@ -6,7 +6,8 @@
 //      row * bw + column), select_pass_kernel, one 8-bit digit per launch;
 //   2. sweep_kernel: every row's 128 columns are processed in order in
 //      registers: mask decision (2:4 at each group start on the compensated
-//      weights), e = (w_q - p_q) / U_qq, rank-1 update of the rest of the
+//      weights), e = (w_q - p_q) / U_qq (as a product with the reciprocal),
+//      rank-1 update of the rest of the
 //      block with the U row held in shared memory;
 //   3. W[:, i2:] -= Err * U[i1:i2, i2:] as an FP32-accurate tensor-core GEMM
 //      (three TF32 products on hi/lo planes of Err and U, gemm_tc.cu).
@@ -33,8 +34,8 @@ constexpr size_t kSweepSmem = (size_t)kMaxBlock * kMaxBlock * sizeof(float);
 
 enum SweepMode { kModeNM24 = 0, kModeThreshold = 1, kModeForced = 2 };
 
-__device__ __forceinline__ unsigned long long sal_key(float w, float u, unsigned idx) {
-  return ((unsigned long long)__float_as_uint(saliency(w, u)) << 32) | idx;
+__device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsigned idx) {
+  return ((unsigned long long)__float_as_uint(saliency(w, inv_u)) << 32) | idx;
 }
 
 template <int MODE>
@@ -45,6 +46,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     int* info) {
   if (cta_info_set(info)) return;
   extern __shared__ float Us[];   // [128][128]: U[i1 + a][i1 + b]
+  __shared__ float Uinv[kMaxBlock];   // 1 / U_qq of the block's columns
   const int tid = threadIdx.x;
   for (int e = tid * 4; e < kMaxBlock * kMaxBlock; e += kSweepThreads * 4) {
     const int a = e >> 7, b = e & 127;
@@ -52,6 +54,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     if (a < bw && b < bw) v = ld4(U + (long long)(i1 + a) * d + i1 + b);
     st4(Us + e, v);
   }
+  if (tid < kMaxBlock) Uinv[tid] = tid < bw ? 1.0f / U[(long long)(i1 + tid) * d + i1 + tid] : 0.f;
   __syncthreads();
 
   const int lane = tid & 31;
@@ -79,7 +82,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 #pragma unroll
     for (int j = 0; j < kSeg; ++j) {
       const unsigned idx = (unsigned)row * (unsigned)bw + (unsigned)(c0 + j);
-      if (sal_key(w[j], Us[(c0 + j) * kMaxBlock + c0 + j], idx) >= t) keep |= 1u << j;
+      if (sal_key(w[j], Uinv[c0 + j], idx) >= t) keep |= 1u << j;
     }
   }
   if (MODE == kModeForced && live) {
@@ -88,55 +91,70 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
   }
   float loss = 0.f;
 
+  // Columns are taken four at a time (one N:M group; a group never straddles
+  // two threads). The owner of the group decides its mask, computes the four
+  // errors in order with the in-group updates done locally, and broadcasts
+  // them; every thread then applies the rank-4 update to its later columns.
+  // Arithmetically this is the column-by-column sweep with the updates of
+  // the four columns to the columns right of the group summed together.
   // Segments run as a loop (not unrolled) to keep the body small enough for
-  // the instruction cache; the 16 columns of a segment are unrolled so that
-  // every register index is static.
+  // the instruction cache; the groups of a segment are unrolled so that every
+  // register index is static.
+  const int src = (lane & ~(kTpr - 1));
 #pragma unroll 1
   for (int qs = 0; qs < kTpr; ++qs) {
     if (qs * kSeg >= bw) break;
 #pragma unroll
-    for (int qj = 0; qj < kSeg; ++qj) {
-      const int q = qs * kSeg + qj;
-      float e = 0.f;
+    for (int g = 0; g < kSeg / 4; ++g) {
+      const int qj0 = 4 * g, q0 = qs * kSeg + qj0;
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
       if (seg == qs) {
-        if (MODE == kModeNM24 && (qj & 3) == 0) {
+        if (MODE == kModeNM24) {
           // 2 of 4 on the compensated weights; ties keep the lower column.
-          float s[4];
+          float sl[4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) s[t] = saliency(w[qj + t], Us[(q + t) * kMaxBlock + q + t]);
-          uint32_t g = 0;
+          for (int t = 0; t < 4; ++t) sl[t] = saliency(w[qj0 + t], Uinv[q0 + t]);
+          uint32_t gm = 0;
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             int rank = 0;   // how many of the group beat column t
 #pragma unroll
             for (int o = 0; o < 4; ++o)
-              if (o != t && (s[o] > s[t] || (s[o] == s[t] && o < t))) ++rank;
-            if (rank < 2) g |= 1u << t;
+              if (o != t && (sl[o] > sl[t] || (sl[o] == sl[t] && o < t))) ++rank;
+            if (rank < 2) gm |= 1u << t;
           }
-          keep = (keep & ~(0xfu << qj)) | (g << qj);
+          keep = (keep & ~(0xfu << qj0)) | (gm << qj0);
         }
-        const float wq = w[qj];
-        const bool kept = (keep >> qj) & 1u;
-        e = kept ? 0.f : __fdiv_rn(wq, Us[q * kMaxBlock + q]);
-        w[qj] = kept ? wq : 0.f;
-        err[qj] = e;
-        loss = fmaf(e, e, loss);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int qj = qj0 + t, q = q0 + t;
+          const float wq = w[qj];
+          const bool kept = (keep >> qj) & 1u;
+          e[t] = kept ? 0.f : __fmul_rn(wq, Uinv[q]);
+          w[qj] = kept ? wq : 0.f;
+          err[qj] = e[t];
+          loss = fmaf(e[t], e[t], loss);
+          const float* urow = Us + q * kMaxBlock + c0;
+#pragma unroll
+          for (int jj = qj + 1; jj < qj0 + 4; ++jj) w[jj] = fmaf(-e[t], urow[jj], w[jj]);
+        }
       }
-      e = __shfl_sync(0xffffffffu, e, (lane & ~(kTpr - 1)) | qs);
-      if (seg >= qs && e != 0.f) {
-        const float* urow = Us + q * kMaxBlock + c0;
-        float u[kSeg];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) e[t] = __shfl_sync(0xffffffffu, e[t], src | qs);
+      if (seg >= qs && (e[0] != 0.f || e[1] != 0.f || e[2] != 0.f || e[3] != 0.f)) {
+        // columns of this segment right of the group
 #pragma unroll
         for (int v = 0; v < kSeg / 4; ++v) {
-          const float4 x = ld4(urow + 4 * v);
-          u[4 * v + 0] = x.x; u[4 * v + 1] = x.y; u[4 * v + 2] = x.z; u[4 * v + 3] = x.w;
-        }
-        if (seg > qs) {
-#pragma unroll
-          for (int j = 0; j < kSeg; ++j) w[j] = fmaf(-e, u[j], w[j]);
-        } else {
-#pragma unroll
-          for (int j = qj + 1; j < kSeg; ++j) w[j] = fmaf(-e, u[j], w[j]);
+          const bool right = (seg > qs) || (4 * v > qj0);
+          if (!right) continue;
+          float4 u0 = ld4(Us + (q0 + 0) * kMaxBlock + c0 + 4 * v);
+          float4 u1 = ld4(Us + (q0 + 1) * kMaxBlock + c0 + 4 * v);
+          float4 u2 = ld4(Us + (q0 + 2) * kMaxBlock + c0 + 4 * v);
+          float4 u3 = ld4(Us + (q0 + 3) * kMaxBlock + c0 + 4 * v);
+          w[4 * v + 0] = fmaf(-e[3], u3.x, fmaf(-e[2], u2.x, fmaf(-e[1], u1.x, fmaf(-e[0], u0.x, w[4 * v + 0]))));
+          w[4 * v + 1] = fmaf(-e[3], u3.y, fmaf(-e[2], u2.y, fmaf(-e[1], u1.y, fmaf(-e[0], u0.y, w[4 * v + 1]))));
+          w[4 * v + 2] = fmaf(-e[3], u3.z, fmaf(-e[2], u2.z, fmaf(-e[1], u1.z, fmaf(-e[0], u0.z, w[4 * v + 2]))));
+          w[4 * v + 3] = fmaf(-e[3], u3.w, fmaf(-e[2], u2.w, fmaf(-e[1], u1.w, fmaf(-e[0], u0.w, w[4 * v + 3]))));
         }
       }
     }
@@ -230,7 +248,7 @@ __global__ void __launch_bounds__(256) select_pass_kernel(
   __shared__ unsigned int last;
   const int t = threadIdx.x;
   h[t] = 0;
-  if (t < bw) ud[t] = U[(long long)(i1 + t) * d + i1 + t];
+  if (t < bw) ud[t] = 1.0f / U[(long long)(i1 + t) * d + i1 + t];   // same reciprocal as the sweep
   __syncthreads();
   const int shift = 56 - 8 * pass;
   const unsigned long long prefix = st->prefix;
@@ -350,7 +368,7 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
       select_init_kernel<<<1, 256, 0, st>>>(w.sel, (unsigned int)kk);
       count_launches(1);
       const long long total4 = (long long)rows * (bw / 4);
-      const int g = (int)std::min<long long>(cdivll(total4, 256 * 8), 4 * kNumSMs);
+      const int g = (int)std::min<long long>(cdivll(total4, 256), 8 * kNumSMs);
       for (int pass = 0; pass < 8; ++pass) {
         select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, w.sel, pass, info);
         count_launches(1);

@@ -200,4 +200,7 @@ CONFIGS = {
                                   "unstructured:0.8"))],
     # Qwen3-32B-shaped decoder block
     "qwen3_32b_block": _qwen_block(),
+    # a Llama-7B-wide layer with a short calibration set, sized for profiler
+    # captures of the factorisation and sweep kernels (X 268 MB > L2)
+    "profile_4096": [LayerSpec("profile_4096", 4096, 4096, 32768, runs=("2:4",))],
 }
