@@ -18,6 +18,9 @@
 // pass runs except once for the last column block.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <mutex>
+
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "kernels.h"
@@ -358,50 +361,107 @@ size_t factor_ws_bytes(int d) {
 size_t factor_part_tiles(int d) {
   const int K = cdiv(d, kTile);
   size_t best = 0;
-  for (int s = 1; s < K; ++s) {
-    const size_t t = (size_t)(K - s) * trtri_splits(K, s);
-    if (t > best) best = t;
-  }
+  for (int t = 1; t < K; ++t) best = std::max(best, (size_t)t * urow_splits(t));
   return best;
 }
 
-int trtri_splits(int K, int s) {
-  // aim for two CTAs per SM on each anti-diagonal, at least 2 blocks of m each
-  const int tiles = K - s;
-  int n = cdiv(2 * kNumSMs, tiles);
-  n = min(n, max(1, s / 2));
-  return max(1, n);
+int urow_splits(int tiles) {
+  // a block row of U with `tiles` tiles whose K lengths are 1..tiles blocks:
+  // split the long ones so the row fills about one wave, at least 2 blocks
+  // of K per split
+  return std::max(1, std::min(tiles / 2, kNumSMs / tiles));
 }
 
-cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, float* U, void* ws,
-                          int* info, cudaStream_t st) {
-  const int K = cdiv(d, kTile);
-  const FactorWs w = carve_factor(ws, d, nullptr);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(diag_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
-    attr_done = true;
+namespace {
+
+// The factorisation's internal streams (per device): the critical chain
+// diag(k) -> panel(k) -> update of column block k-1 -> diag(k-1) on `crit`;
+// the rest of each rank-128 update on `upd`; the V and U block rows, which
+// nothing in the chain waits for, on `rows`. They fork from and join back to
+// the caller's stream, so the whole factorisation is ordered on it (and
+// captures into one graph).
+struct FactorStreams {
+  cudaStream_t crit = nullptr, upd = nullptr, rows = nullptr;
+  cudaEvent_t fork = nullptr, diag_done = nullptr, panel_done = nullptr, upd_done = nullptr;
+  cudaEvent_t join[3] = {nullptr, nullptr, nullptr};
+};
+
+std::mutex g_streams_mu;
+
+cudaError_t factor_streams(FactorStreams** out) {
+  static FactorStreams per_dev[64];
+  static bool made[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  FactorStreams& f = per_dev[dev];
+  if (!made[dev]) {
+    int lo = 0, hi = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&f.crit, cudaStreamNonBlocking, hi)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&f.upd, cudaStreamNonBlocking, lo)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&f.rows, cudaStreamNonBlocking, lo)) != cudaSuccess) return e;
+    cudaEvent_t* evs[] = {&f.fork, &f.diag_done, &f.panel_done, &f.upd_done, &f.join[0], &f.join[1], &f.join[2]};
+    for (cudaEvent_t* ev : evs)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    made[dev] = true;
   }
-  const double scale = 2.0 / (double)n_total;
-  if (U != H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
-  damp_lambda_kernel<<<1, 1024, 0, st>>>(H, d, scale, (double)damp, w.lam, info);
-  count_launches(1);
-  scale_damp_kernel<<<dim3(cdiv(d, 4 * 128), d), 128, 0, st>>>(H, w.R, d, scale, w.lam, info);
-  count_launches(1);
-  if (U == H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
+  *out = &f;
+  return cudaSuccess;
+}
+
+// s2 waits for everything enqueued on s1 so far.
+cudaError_t after(cudaStream_t s2, cudaStream_t s1, cudaEvent_t ev) {
+  cudaError_t e = cudaEventRecord(ev, s1);
+  return e != cudaSuccess ? e : cudaStreamWaitEvent(s2, ev, 0);
+}
+
+// The block-column loop and the V / U block rows (see the file comment).
+cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const FactorStreams& f) {
+  const int K = cdiv(d, kTile);
+  const tc::Operand Ud{w.U_hi, w.U_lo, d, d, d};
+  const tc::Operand Rp{w.R, w.V_lo, d, d, d};
   cudaError_t e = cudaSuccess;
-  // planes of the last column block above its diagonal block
-  if (K > 1 && (e = tc::launch_split(w.R + (K - 1) * kTile, d, (K - 1) * kTile, d - (K - 1) * kTile, w.A_hi,
-                                     w.A_lo, kTile, info, st)) != cudaSuccess)
-    return e;
+  bool upd_pending = false;
   for (int k = K - 1; k >= 0; --k) {
     const int c0 = k * kTile, bk = min(kTile, d - c0);
-    diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, st>>>(w.R, d, k, U, w.U_hi, w.U_lo, info);
+    diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, f.crit>>>(w.R, d, k, U, w.U_hi, w.U_lo, info);
     count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (k < K - 1) {
+      // block row k: V_km = U_kk R_km (planes in place of R_km's), then
+      // U_kq = -sum_{m=k+1..q} V_km U_mq, reading the U rows below it
+      if ((e = after(f.rows, f.crit, f.diag_done)) != cudaSuccess) return e;
+      tc::Job v{};
+      v.mode = 3;
+      v.s = k;
+      v.dlim = d;
+      v.ldc = d;
+      v.Mlim = v.Nlim = d;
+      v.alpha = 1.f;
+      v.C_hi = w.R;
+      v.C_lo = w.V_lo;
+      if ((e = tc::launch_gemm(Ud, Rp, true, v, K - 1 - k, info, f.rows)) != cudaSuccess) return e;
+      tc::Job u{};
+      u.mode = 2;
+      u.s = k;
+      u.nsplit = urow_splits(K - 1 - k);
+      u.nblk = K;
+      u.dlim = d;
+      u.C = U;
+      u.ldc = d;
+      u.Mlim = u.Nlim = d;
+      u.alpha = -1.f;
+      u.C_hi = w.U_hi;
+      u.C_lo = w.U_lo;
+      u.part = w.part;
+      if ((e = tc::launch_gemm(Rp, Ud, true, u, (K - 1 - k) * u.nsplit, info, f.rows)) != cudaSuccess) return e;
+    }
     if (k == 0) break;
     {
-      // panel R_ik = A_ik U_kk^T for the rows above, written as hi/lo planes
-      // (hi over R, lo into V_lo)
+      // panel R_ik = A_ik U_kk^T for the rows above, as hi/lo planes (hi
+      // over R, lo into V_lo)
       const tc::Operand A{w.A_hi, w.A_lo, c0, bk, kTile};
       const tc::Operand B{w.U_hi + (long long)c0 * d + c0, w.U_lo + (long long)c0 * d + c0, bk, bk, d};
       tc::Job job{};
@@ -416,64 +476,74 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
       job.alpha = 1.f;
       job.C_hi = w.R;
       job.C_lo = w.V_lo;
-      if ((e = tc::launch_gemm(A, B, false, job, k, info, st)) != cudaSuccess) return e;
+      if ((e = tc::launch_gemm(A, B, false, job, k, info, f.crit)) != cudaSuccess) return e;
     }
-    {
-      // rank-bk update of the leading upper tiles, A_ij -= R_ik R_jk^T; the
-      // tiles of column block k-1 also write the planes the next panel reads
-      const tc::Operand P{w.R + c0, w.V_lo + c0, c0, bk, d};
-      tc::Job job{};
-      job.mode = 1;
-      job.kdim = bk;
-      job.C = w.R;
-      job.ldc = d;
-      job.Mlim = job.Nlim = c0;
-      job.alpha = -1.f;
-      job.beta = 1.f;
-      job.C_hi = w.A_hi;
-      job.C_lo = w.A_lo;
-      job.ldp = kTile;
-      job.p_col0 = c0 - kTile;
-      job.planes_one_col = 1;
-      job.planes_n0 = c0 - kTile;
-      if ((e = tc::launch_gemm(P, P, false, job, k * (k + 1) / 2, info, st)) != cudaSuccess) return e;
+    // rank-bk update A_ij -= R_ik R_jk^T of the leading upper tiles: column
+    // block k-1 on the chain (its tiles also write the planes the next panel
+    // reads), the tiles left of it on `upd`, after the previous step's
+    if (upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
+    const tc::Operand P{w.R + c0, w.V_lo + c0, c0, bk, d};
+    tc::Job job{};
+    job.mode = 1;
+    job.kdim = bk;
+    job.C = w.R;
+    job.ldc = d;
+    job.Mlim = job.Nlim = c0;
+    job.alpha = -1.f;
+    job.beta = 1.f;
+    if (k >= 2) {
+      if ((e = after(f.upd, f.crit, f.panel_done)) != cudaSuccess) return e;
+      if ((e = tc::launch_gemm(P, P, false, job, (k - 1) * k / 2, info, f.upd)) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(f.upd_done, f.upd)) != cudaSuccess) return e;
+      upd_pending = true;
     }
+    job.t0 = (k - 1) * k / 2;
+    job.C_hi = w.A_hi;
+    job.C_lo = w.A_lo;
+    job.ldp = kTile;
+    job.p_col0 = c0 - kTile;
+    if ((e = tc::launch_gemm(P, P, false, job, k, info, f.crit)) != cudaSuccess) return e;
   }
-  if (K > 1) {
-    // V_im = U_ii R_im above the diagonal blocks, as planes in place of R_im's
-    const tc::Operand Ud{w.U_hi, w.U_lo, d, d, d};
-    const tc::Operand Rp{w.R, w.V_lo, d, d, d};
-    {
-      tc::Job job{};
-      job.mode = 3;
-      job.dlim = d;
-      job.ldc = d;
-      job.Mlim = job.Nlim = d;
-      job.alpha = 1.f;
-      job.C_hi = w.R;
-      job.C_lo = w.V_lo;
-      if ((e = tc::launch_gemm(Ud, Rp, true, job, K * (K - 1) / 2, info, st)) != cudaSuccess) return e;
-    }
-    // off-diagonal blocks of U by anti-diagonals, U_pq = -sum_{m=p+1..q} V_pm U_mq
-    for (int s = 1; s < K; ++s) {
-      tc::Job job{};
-      job.mode = 2;
-      job.s = s;
-      job.nsplit = trtri_splits(K, s);
-      job.nblk = K;
-      job.dlim = d;
-      job.C = U;
-      job.ldc = d;
-      job.Mlim = job.Nlim = d;
-      job.alpha = -1.f;
-      job.beta = 0.f;
-      job.C_hi = w.U_hi;
-      job.C_lo = w.U_lo;
-      job.part = w.part;
-      if ((e = tc::launch_gemm(Rp, Ud, true, job, (K - s) * job.nsplit, info, st)) != cudaSuccess) return e;
-    }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, float* U, void* ws,
+                          int* info, cudaStream_t st) {
+  const int K = cdiv(d, kTile);
+  const FactorWs w = carve_factor(ws, d, nullptr);
+  std::lock_guard<std::mutex> lock(g_streams_mu);
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(diag_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
+    attr_done = true;
   }
-  return cudaGetLastError();
+  FactorStreams* f = nullptr;
+  cudaError_t e = factor_streams(&f);
+  if (e != cudaSuccess) return e;
+  const double scale = 2.0 / (double)n_total;
+  if (U != H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
+  damp_lambda_kernel<<<1, 1024, 0, st>>>(H, d, scale, (double)damp, w.lam, info);
+  count_launches(1);
+  scale_damp_kernel<<<dim3(cdiv(d, 4 * 128), d), 128, 0, st>>>(H, w.R, d, scale, w.lam, info);
+  count_launches(1);
+  if (U == H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
+  // planes of the last column block above its diagonal block
+  if (K > 1 && (e = tc::launch_split(w.R + (K - 1) * kTile, d, (K - 1) * kTile, d - (K - 1) * kTile, w.A_hi,
+                                     w.A_lo, kTile, info, st)) != cudaSuccess)
+    return e;
+  if ((e = cudaEventRecord(f->fork, st)) != cudaSuccess) return e;
+  for (cudaStream_t s : {f->crit, f->upd, f->rows})
+    if ((e = cudaStreamWaitEvent(s, f->fork, 0)) != cudaSuccess) return e;
+  e = factor_blocks(w, d, U, info, *f);
+  // always join, also after an error, so that a capture stays well formed
+  const cudaStream_t side[3] = {f->crit, f->upd, f->rows};
+  for (int i = 0; i < 3; ++i) {
+    const cudaError_t e2 = after(st, side[i], f->join[i]);
+    if (e == cudaSuccess) e = e2;
+  }
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sgpt

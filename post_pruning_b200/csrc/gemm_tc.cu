@@ -159,25 +159,23 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
     ke = job.kdim;
   } else if (job.mode == 1) {
     int i, j;
-    tri_index(blockIdx.x, i, j);
+    tri_index(job.t0 + (int)blockIdx.x, i, j);
     m0 = i * kM;
     n0 = j * kN;
     ke = job.kdim;
   } else if (job.mode == 3) {
-    int i, j;
-    tri_index(blockIdx.x, i, j);
-    m0 = i * kM;
-    n0 = (j + 1) * kN;
+    m0 = job.s * kM;
+    n0 = (job.s + 1 + (int)blockIdx.x) * kN;
     kb = m0;
     ke = min(m0 + kM, job.dlim);
   } else {
     tile = blockIdx.x / job.nsplit;
     split = blockIdx.x - tile * job.nsplit;
-    const int i = tile, j = tile + job.s;
+    const int i = job.s, j = job.s + 1 + tile;
     m0 = i * kM;
     n0 = j * kN;
     const int lo = (i + 1) * kM, hi = min((j + 1) * kM, job.dlim);
-    const int per = ((job.s + job.nsplit - 1) / job.nsplit) * kM;
+    const int per = ((j - i + job.nsplit - 1) / job.nsplit) * kM;
     kb = min(hi, lo + split * per);
     ke = min(hi, kb + per);
   }
@@ -357,17 +355,17 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
 }
 
-// Anti-diagonal split partials -> C = alpha * sum (+ hi/lo planes), in split order.
-__global__ void __launch_bounds__(256) antidiag_reduce_kernel(const Job job, const int* info) {
+// Split partials of a block row -> C = alpha * sum (+ hi/lo planes), in split order.
+__global__ void __launch_bounds__(256) rowsplit_reduce_kernel(const Job job, const int* info) {
   if (cta_info_set(info)) return;
-  const int tiles = job.nblk - job.s;
+  const int tiles = job.nblk - 1 - job.s;
   const long long quads = (long long)tiles * (kM * kN / 4);
   for (long long qd = (long long)blockIdx.x * blockDim.x + threadIdx.x; qd < quads;
        qd += (long long)gridDim.x * blockDim.x) {
     const int tile = (int)(qd / (kM * kN / 4));
     const int e = (int)(qd - (long long)tile * (kM * kN / 4)) * 4;
     const int m = e / kN, n = e % kN;
-    const int row = tile * kM + m, col = (tile + job.s) * kN + n;
+    const int row = job.s * kM + m, col = (job.s + 1 + tile) * kN + n;
     if (row >= job.Mlim || col >= job.Nlim) continue;
     const float* src = job.part + (size_t)tile * job.nsplit * kM * kN + e;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -482,9 +480,9 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
   gemm_tf32x3_kernel<<<grid, kThreads, kSmem, st>>>(ah, al, bh, bl, job, b_mn ? 1 : 0, info);
   count_launches(1);
   if (job.mode == 2 && job.nsplit > 1) {
-    const long long quads = (long long)(job.nblk - job.s) * (kM * kN / 4);
+    const long long quads = (long long)(job.nblk - 1 - job.s) * (kM * kN / 4);
     const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
-    antidiag_reduce_kernel<<<g, 256, 0, st>>>(job, info);
+    rowsplit_reduce_kernel<<<g, 256, 0, st>>>(job, info);
     count_launches(1);
   }
   return cudaGetLastError();

@@ -17,11 +17,11 @@ struct Operand {
 
 // What one launch computes; tile sizes are 128 x 128.
 //  mode 0: dense grid of mt x nt tiles, K = kdim.
-//  mode 1: tiles (i, j), i <= j, enumerated column by column, K = kdim.
-//  mode 2: tiles (i, i + s) for i < nblk - s, K = [(i+1)*128, min((i+s+1)*128, dlim)),
-//          split into nsplit ranges whose partials are reduced in order.
-//  mode 3: tiles (i, m), i < m, enumerated like mode 1 over (i, m - 1),
-//          K = [i*128, min((i+1)*128, dlim)).
+//  mode 1: tiles (i, j), i <= j, enumerated column by column from tile t0, K = kdim.
+//  mode 2: tiles (s, s + 1 + t) for t < nblk - 1 - s (one block row of U),
+//          K = [(s+1)*128, min((s+2+t)*128, dlim)), split into nsplit ranges
+//          whose partials are reduced in order.
+//  mode 3: tiles (s, s + 1 + t) for t < nblk - 1 - s, K = [s*128, min((s+1)*128, dlim)).
 // A(m, k) is read at (x = a_x0 + k, y = a_y0 + m0 + m); B(k, n) at
 // (x = b_x0 + k, y = b_y0 + n0 + n) if K-major, (x = b_x0 + n0 + n, y = b_y0 + k)
 // if MN-major. C(m, n) = alpha * acc + beta * C at
@@ -33,6 +33,7 @@ struct Operand {
 struct Job {
   int mode;
   int mt, nt;
+  int t0;
   int s, nsplit, nblk;
   int kdim;
   int dlim;

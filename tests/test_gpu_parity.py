@@ -93,6 +93,54 @@ def test_factor_matches_oracle(spec):
     assert torch.equal(Hd, U)
 
 
+# 17 column blocks with a 32-wide last one: the block-column loop runs its
+# rank-128 updates, V and U block rows on internal streams and joins them
+# back to the caller's stream, so check it eager, on a side stream behind a
+# pending producer, and captured in a CUDA graph.
+WIDE = LayerSpec("wide_2080", d_in=2080, d_out=64, n_tok=4096, sigma=1.5, seed=11)
+
+
+def test_factor_many_blocks_streams_and_graph():
+    spec = WIDE
+    X64 = bf16_bits_to_f64(gen_activations(spec)).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)
+    _, U_ref = _oracle_factor(Hs, spec.n_tok)
+    dev = torch.device("cuda")
+    ws = pp.workspace(spec.d_out, spec.d_in)
+    info = pp.new_info()
+
+    Hd = torch.from_numpy(Hs).to(dev)
+    U = torch.empty_like(Hd)
+    pp.factor(Hd, spec.n_tok, 0.01, U, ws, info)
+    pp.raise_on_info(info)
+    Ug = U.cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0) and np.all(np.diag(Ug) > 0)
+    rel_rows = np.linalg.norm(Ug - U_ref, axis=1) / np.linalg.norm(U_ref, axis=1)
+    assert rel_rows.max() < 1e-4, rel_rows.max()
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        H2 = torch.zeros_like(Hd)
+        H2.copy_(Hd)                       # the producer is still queued on `side`
+        U2 = torch.full_like(Hd, float("nan"))
+        pp.factor(H2, spec.n_tok, 0.01, U2, ws, info)
+    torch.cuda.synchronize()
+    pp.raise_on_info(info)
+    assert torch.equal(U2, U)
+
+    U3 = torch.full_like(Hd, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        pp.factor(Hd, spec.n_tok, 0.01, U3, ws, info)
+    g.replay()
+    torch.cuda.synchronize()
+    pp.raise_on_info(info)
+    assert torch.equal(U3, U)
+    del g
+
+
 # ------------------------------------------------------------ sweep
 
 PATTERNS = [pp.Params("2:4"), pp.Params("2:4", blocksize=32), pp.Params("unstructured:0.5"),
