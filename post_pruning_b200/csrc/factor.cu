@@ -82,16 +82,21 @@ __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict
 // One CTA factors the diagonal block A_kk = R_kk R_kk^T (R_kk upper) and
 // inverts it, U_kk = R_kk^-1, in FP32 shared memory. The block is treated as
 // up to 4 x 4 sub-blocks of 32 (width b = 32..128), processed from the last
-// 32-panel to the first:
-//   1. warp 0 factors the 32 x 32 diagonal sub-block D_pp = R_pp R_pp^T (lane
-//      = row, pivots broadcast by shuffles, no CTA barrier) and inverts R_pp
-//      (lane = column, back substitution against R_pp in shared memory);
-//   2. panel: R_ip = A_ip U_pp^T for the sub-blocks above (one warp each);
-//   3. update: A_ij -= R_ip R_jp^T for the leading sub-blocks (one warp each).
-// Then V_pm = U_pp R_pm and the off-diagonal blocks of U along the
-// anti-diagonals, U_pq = -sum_{m=p+1..q} V_pm U_mq.
-// Warp-level 32 x 32 products keep one operand column per lane in registers
-// and read the other operand's rows as broadcast 16-byte loads.
+// 32-panel p to the first. The pivots are the only serial chain, so one warp
+// runs them while the other seven do everything else around it:
+//   warp 0, per panel p: waits until D_pp is fully updated, factors it,
+//     D_pp = R_pp R_pp^T (lane = row, pivots broadcast by shuffles), inverts
+//     it, U_pp = R_pp^-1 (lane = column, column-form back substitution), and
+//     signals;
+//   warps 1-7, per panel p, once U_pp is there: the panel R_ip = A_ip U_pp^T
+//     for the sub-blocks above; the update A_ij -= R_ip R_jp^T, the next
+//     diagonal sub-block first (then warp 0 may go on) and the rest after;
+//     then block row p of U: V_pm = U_pp R_pm and
+//     U_pq = -sum_{m=p+1..q} V_pm U_mq (rows below p are final by then).
+// Warp 0 and the workers meet on two named barriers (one each way), the
+// workers among themselves on a third. Warp-level 32 x 32 products keep one
+// operand column per lane in registers and read the other operand's rows as
+// broadcast 16-byte loads, in units of 8 rows.
 
 constexpr int kDiagThreads = 256;
 constexpr int kDiagWarps = kDiagThreads / 32;
@@ -142,17 +147,77 @@ __device__ __forceinline__ void tri_pair(int t, int& i, int& j) {   // t -> (i <
   i = t - jj * (jj + 1) / 2;
 }
 
-// One CTA factors the diagonal block A_kk = R_kk R_kk^T (R_kk upper) and
-// inverts it, U_kk = R_kk^-1, in FP32 shared memory, as up to 4 x 4
-// sub-blocks of 32 processed from the last 32-panel to the first:
-//   1. warp 0 factors the panel's 32 x 32 diagonal sub-block (lane = row; the
-//      pivot column is broadcast by shuffles) and inverts it
-//      (lane = column, back substitution);
-//   2. R_ip = A_ip U_pp^T for the sub-blocks above, and
-//   3. A_ij -= R_ip R_jp^T for the leading sub-blocks, both spread over all
-//      warps in 8-row units (lane = output column).
-// Then V_pm = U_pp R_pm and the off-diagonal blocks of U along the
-// anti-diagonals, U_pq = -sum_{m=p+1..q} V_pm U_mq, in the same units.
+// Named CTA barriers: `count` threads take part; bar_arrive does not wait.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+constexpr int kBarUReady = 1;    // warp 0 -> workers: U_pp (and R_pp) written
+constexpr int kBarDReady = 2;    // workers -> warp 0: next diagonal sub-block updated
+constexpr int kBarWorkers = 3;   // the seven worker warps among themselves
+constexpr int kWorkers = kDiagWarps - 1;
+
+// C[8 rows][lane] (+)= sum_k A[8 rows][k] * b[k] for a unit of 8 rows.
+__device__ __forceinline__ void unit_dot8(const float* A, const float (&b)[32], float (&acc)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] += row_dot32(A + i * kDiagLd, b);
+}
+
+// Warp 0's part for panel p: factor the 32 x 32 diagonal sub-block at
+// (c0, c0) of S in place (reverse Cholesky, lane = row) and write its
+// inverse into Ui; returns the first failing column + 1 (or
+// SGPT_INFO_NONFINITE), 0 if every pivot was positive.
+__device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* rinv, int c0, int col0, int lane) {
+  // Pivot j: r_jj = sqrt(a_jj), r_ij = a_ij / r_jj (i < j), then
+  // a_il -= r_ij r_lj for l < j. Column j-1 is updated first and the next
+  // pivot is broadcast before the rest of the update is issued. Entries
+  // below the diagonal (l < i) take the update too but are never read, and
+  // are zeroed on output.
+  float dr[32];
+  float* row = S + (c0 + lane) * kDiagLd + c0;
+  load_row32(S + c0 * kDiagLd + c0, lane, dr);
+  int fail = 0;
+  float piv = __shfl_sync(0xffffffffu, dr[31], 31);
+#pragma unroll
+  for (int j = 31; j >= 0; --j) {
+    if (!(piv > 0.f) && fail == 0) fail = isfinite(piv) ? (col0 + j + 1) : SGPT_INFO_NONFINITE;
+    const float rs = rsqrt_nr(piv);
+    const float rij = lane < j ? dr[j] * rs : (lane == j ? piv * rs : 0.f);
+    dr[j] = rij;
+    if (j == 0) break;
+    dr[j - 1] = fmaf(-rij, __shfl_sync(0xffffffffu, rij, j - 1), dr[j - 1]);
+    const float next = __shfl_sync(0xffffffffu, dr[j - 1], j - 1);
+#pragma unroll
+    for (int l = j - 2; l >= 0; --l) dr[l] = fmaf(-rij, __shfl_sync(0xffffffffu, rij, l), dr[l]);
+    piv = next;
+  }
+#pragma unroll
+  for (int l = 0; l < 32; l += 4)
+    *reinterpret_cast<float4*>(row + l) =
+        make_float4(lane <= l ? dr[l] : 0.f, lane <= l + 1 ? dr[l + 1] : 0.f, lane <= l + 2 ? dr[l + 2] : 0.f,
+                    lane <= l + 3 ? dr[l + 3] : 0.f);
+  rinv[c0 + lane] = 1.0f / row[lane];      // this lane's own diagonal entry
+  __syncwarp();
+  // U_pp = R_pp^-1, lane = column: back substitution from the bottom in
+  // column form, u_m = acc_m / r_mm, then acc_i -= r_im u_m for i < m (row
+  // m-1 first: it is the next step's).
+  float u[32];
+  const float* R = S + c0 * kDiagLd + c0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+  for (int m = 31; m >= 0; --m) {
+    u[m] = (m <= lane) ? u[m] * rinv[c0 + m] : 0.f;
+#pragma unroll
+    for (int i = m - 1; i >= 0; --i) u[i] = fmaf(-R[i * kDiagLd + m], u[m], u[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) Ui[(c0 + i) * kDiagLd + c0 + lane] = u[i];
+  return fail;
+}
+
 __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const float* __restrict__ Rws,
                                                                       int d, int k,
                                                                       float* __restrict__ U,
@@ -170,145 +235,108 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
   const int b0 = k * kTile;
   const int b = min(kTile, d - b0);          // a multiple of 32
   const int np = b >> 5;
-  for (int e = tid * 4; e < kTile * kTile; e += kDiagThreads * 4) {
-    const int i = e >> 7, l = e & 127;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < b && l < b) v = ld4(Rws + (long long)(b0 + i) * d + b0 + l);
-    st4(S + i * kDiagLd + l, v);             // only entries i <= l are ever read
-    st4(Ui + i * kDiagLd + l, make_float4(0.f, 0.f, 0.f, 0.f));
+  {
+    // all sixteen loads of this thread in flight before the first store
+    constexpr int kPer = kTile * kTile / 4 / kDiagThreads;
+    float4 v[kPer];
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = (tid + t * kDiagThreads) * 4, i = e >> 7, l = e & 127;
+      v[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < b && l < b) v[t] = ld4(Rws + (long long)(b0 + i) * d + b0 + l);
+    }
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = (tid + t * kDiagThreads) * 4, i = e >> 7, l = e & 127;
+      st4(S + i * kDiagLd + l, v[t]);        // only entries i <= l are ever read
+      st4(Ui + i * kDiagLd + l, make_float4(0.f, 0.f, 0.f, 0.f));
+    }
   }
   if (tid == 0) bad = 0;
   __syncthreads();
 
-  for (int p = np - 1; p >= 0; --p) {
-    const int c0 = p * 32;
-    if (warp == 0) {
-      // ---- reverse Cholesky of the 32 x 32 diagonal sub-block, lane = row.
-      // Pivot j: r_jj = sqrt(a_jj), r_ij = a_ij / r_jj (i < j), then
-      // a_il -= r_ij r_lj for l < j. Entries below the diagonal (l < i)
-      // take the update too but are never read, and are zeroed on output.
-      float dr[32];
-      float* row = S + (c0 + lane) * kDiagLd + c0;
-      load_row32(S + c0 * kDiagLd + c0, lane, dr);
-      int fail = 0;
+  // Every thread runs the same barrier sequence whatever the data; a failed
+  // pivot is reported after the loop (the values are then discarded).
+  if (warp == 0) {
+    for (int p = np - 1; p >= 0; --p) {
+      if (p < np - 1) bar_sync(kBarDReady, kDiagThreads);
+      const int fail = pivot_panel(S, Ui, rinv, p * 32, b0 + p * 32, lane);
+      if (fail && lane == 0 && bad == 0) bad = fail;
+      bar_arrive(kBarUReady, kDiagThreads);
+    }
+  } else {
+    const int w = warp - 1;
+    for (int p = np - 1; p >= 0; --p) {
+      const int c0 = p * 32;
+      bar_sync(kBarUReady, kDiagThreads);
+      if (p > 0) {
+        {
+          // panel: R_ip = A_ip U_pp^T for i < p, in place; lane = column j
+          // with row j of U_pp in registers
+          float bu[32];
+          load_row32(Ui + c0 * kDiagLd + c0, lane, bu);
+          for (int unit = w; unit < p * 4; unit += kWorkers) {
+            float* A = S + (unit * 8) * kDiagLd + c0;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            unit_dot8(A, bu, acc);
+            __syncwarp();
 #pragma unroll
-      for (int j = 31; j >= 0; --j) {
-        const float piv = __shfl_sync(0xffffffffu, dr[j], j);
-        if (!(piv > 0.f) && fail == 0) fail = isfinite(piv) ? (b0 + c0 + j + 1) : SGPT_INFO_NONFINITE;
-        const float rs = rsqrt_nr(piv);
-        const float rij = lane < j ? dr[j] * rs : (lane == j ? piv * rs : 0.f);
-        dr[j] = rij;
-        if (j == 0) break;
+            for (int i = 0; i < 8; ++i) A[i * kDiagLd + lane] = acc[i];
+          }
+        }
+        bar_sync(kBarWorkers, kWorkers * 32);
+        // update A_ij -= R_ip R_jp^T for i <= j < p: the sub-block (p-1, p-1)
+        // first (four units), then warp 0 may factor it
+        const int units = p * (p + 1) / 2 * 4;
+        if (w >= 4) bar_arrive(kBarDReady, kDiagThreads);   // no unit among the first four
+        for (int unit = w; unit < units; unit += kWorkers) {
+          // unit order: the last pair (p-1, p-1) first, then the others
+          const int t = (unit < 4) ? (units / 4 - 1) : ((unit - 4) >> 2);
+          int ii, jj;
+          tri_pair(t, ii, jj);
+          const int r0 = ii * 32 + (unit & 3) * 8;
+          float br[32];
+          load_row32(S + (jj * 32) * kDiagLd + c0, lane, br);   // row `lane` of R_jp
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          unit_dot8(S + r0 * kDiagLd + c0, br, acc);
+          float* C = S + r0 * kDiagLd + jj * 32;
 #pragma unroll
-        for (int l = 0; l < j; ++l) {
-          const float c = __shfl_sync(0xffffffffu, rij, l);
-          dr[l] = fmaf(-rij, c, dr[l]);
+          for (int i = 0; i < 8; ++i) C[i * kDiagLd + lane] -= acc[i];
+          if (unit < 4) bar_arrive(kBarDReady, kDiagThreads);   // each of workers 0-3, once
         }
       }
+      // block row p of U (the rows below are final): V_pm = U_pp R_pm ...
+      if (p < np - 1) {
+        const int nm = np - 1 - p;
+        for (int unit = w; unit < nm * 4; unit += kWorkers) {
+          const int m = p + 1 + (unit >> 2), r0 = c0 + (unit & 3) * 8;
+          float bcol[32];
+          load_col32(S + c0 * kDiagLd + m * 32, lane, bcol);   // column `lane` of R_pm
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          unit_dot8(Ui + r0 * kDiagLd + c0, bcol, acc);
 #pragma unroll
-      for (int l = 0; l < 32; l += 4)
-        *reinterpret_cast<float4*>(row + l) =
-            make_float4(lane <= l ? dr[l] : 0.f, lane <= l + 1 ? dr[l + 1] : 0.f,
-                        lane <= l + 2 ? dr[l + 2] : 0.f, lane <= l + 3 ? dr[l + 3] : 0.f);
-      rinv[c0 + lane] = 1.0f / row[lane];
-      if (fail && lane == 0) bad = fail;
-      __syncwarp();
-      // ---- U_pp = R_pp^-1, lane = column j: back substitution from the
-      // bottom, u_i = (delta_ij - sum_{m>i} r_im u_m) / r_ii.
-      float u[32];
-      const float* R = S + c0 * kDiagLd + c0;
-#pragma unroll
-      for (int i = 31; i >= 0; --i) {
-        const float* ri = R + i * kDiagLd;
-        float a0 = (i == lane) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int m = i + 1; m < 32; ++m) {
-          const float r = ri[m];
-          if ((m & 3) == 0) a0 = fmaf(-r, u[m], a0);
-          else if ((m & 3) == 1) a1 = fmaf(-r, u[m], a1);
-          else if ((m & 3) == 2) a2 = fmaf(-r, u[m], a2);
-          else a3 = fmaf(-r, u[m], a3);
+          for (int i = 0; i < 8; ++i) Vb[(r0 + i) * kDiagLd + m * 32 + lane] = acc[i];
         }
-        u[i] = (i <= lane) ? ((a0 + a1) + (a2 + a3)) * rinv[c0 + i] : 0.f;
+        bar_sync(kBarWorkers, kWorkers * 32);
+        // ... then U_pq = -sum_{m=p+1..q} V_pm U_mq
+        for (int unit = w; unit < nm * 4; unit += kWorkers) {
+          const int q = p + 1 + (unit >> 2), r0 = c0 + (unit & 3) * 8;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int m = p + 1; m <= q; ++m) {
+            float bcol[32];
+            load_col32(Ui + (m * 32) * kDiagLd + q * 32, lane, bcol);   // column `lane` of U_mq
+            unit_dot8(Vb + r0 * kDiagLd + m * 32, bcol, acc);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) Ui[(r0 + i) * kDiagLd + q * 32 + lane] = -acc[i];
+        }
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) Ui[(c0 + i) * kDiagLd + c0 + lane] = u[i];
-    }
-    __syncthreads();
-    if (bad) {
-      if (tid == 0) set_info(info, bad);
-      return;
-    }
-    if (p == 0) break;
-    // ---- panel: R_ip = A_ip U_pp^T for the row blocks i < p (in place);
-    // unit = 8 rows, lane = output column j with row j of U_pp in registers.
-    {
-      float bu[32];
-      load_row32(Ui + c0 * kDiagLd + c0, lane, bu);
-      for (int unit = warp; unit < p * 4; unit += kDiagWarps) {
-        float* A = S + (unit * 8) * kDiagLd + c0;
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = row_dot32(A + i * kDiagLd, bu);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) A[i * kDiagLd + lane] = v[i];
-      }
-    }
-    __syncthreads();
-    // ---- update of the leading sub-blocks: A_ij -= R_ip R_jp^T, i <= j < p
-    {
-      const int units = p * (p + 1) / 2 * 4;
-      for (int unit = warp; unit < units; unit += kDiagWarps) {
-        int ii, jj;
-        tri_pair(unit >> 2, ii, jj);
-        const int r0 = ii * 32 + (unit & 3) * 8;
-        float br[32];
-        load_row32(S + (jj * 32) * kDiagLd + c0, lane, br);   // row `lane` of R_jp
-        float* C = S + r0 * kDiagLd + jj * 32;
-        const float* Ai = S + r0 * kDiagLd + c0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) C[i * kDiagLd + lane] -= row_dot32(Ai + i * kDiagLd, br);
-      }
-    }
-    __syncthreads();
-  }
-
-  // ---- V_pm = U_pp R_pm (p < m) into Vb; unit = 8 rows, lane = column
-  {
-    const int units = np * (np - 1) / 2 * 4;
-    for (int unit = warp; unit < units; unit += kDiagWarps) {
-      int pp, mm;
-      tri_pair(unit >> 2, pp, mm);      // pp <= mm-1
-      mm += 1;
-      const int r0 = (unit & 3) * 8;
-      float bcol[32];
-      load_col32(S + (pp * 32) * kDiagLd + mm * 32, lane, bcol);
-      const float* Upp = Ui + (pp * 32 + r0) * kDiagLd + pp * 32;
-      float* V = Vb + (pp * 32 + r0) * kDiagLd + mm * 32;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) V[i * kDiagLd + lane] = row_dot32(Upp + i * kDiagLd, bcol);
     }
   }
   __syncthreads();
-  // ---- off-diagonal blocks of U by anti-diagonals: U_pq = -sum V_pm U_mq
-  for (int sd = 1; sd < np; ++sd) {
-    const int units = (np - sd) * 4;
-    for (int unit = warp; unit < units; unit += kDiagWarps) {
-      const int pp = unit >> 2, qq = pp + sd, r0 = (unit & 3) * 8;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int mm = pp + 1; mm <= qq; ++mm) {
-        float bcol[32];
-        load_col32(Ui + (mm * 32) * kDiagLd + qq * 32, lane, bcol);
-        const float* V = Vb + (pp * 32 + r0) * kDiagLd + mm * 32;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += row_dot32(V + i * kDiagLd, bcol);
-      }
-      float* Upq = Ui + (pp * 32 + r0) * kDiagLd + qq * 32;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) Upq[i * kDiagLd + lane] = -acc[i];
-    }
-    __syncthreads();
+  if (bad) {
+    if (tid == 0) set_info(info, bad);
+    return;
   }
 
   // Write U_kk (upper, zeros below) and its hi/lo planes.

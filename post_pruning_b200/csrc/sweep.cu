@@ -3,7 +3,8 @@
 // Per block of `bw` <= 128 columns starting at i1:
 //   1. (unstructured) exact k-selection of the block's smallest saliencies
 //      over all d_out rows: radix select on a 64-bit key (saliency bits, then
-//      row * bw + column), select_pass_kernel, one 8-bit digit per launch;
+//      row * bw + column), one cooperative launch of select_kernel with a
+//      grid barrier per 8-bit digit;
 //   2. sweep_kernel: every row's 128 columns are processed in order in
 //      registers: mask decision (2:4 at each group start on the compensated
 //      weights), e = (w_q - p_q) / U_qq (as a product with the reciprocal),
@@ -214,98 +215,164 @@ __global__ void __launch_bounds__(kGemmThreads) trailing_kernel(
 // ------------------------------------------------ unstructured selection
 
 struct SelState {
-  unsigned long long prefix;   // key bits fixed so far
-  unsigned long long thr;      // exclusive threshold: pruned iff key < thr
-  unsigned int k_rem;          // rank still to place inside the prefix bin
-  int done;
-  unsigned int ticket;
+  unsigned long long thr;      // pruned iff key < thr
+  unsigned int arrive;         // grid barrier counter
   unsigned int pad;
-  unsigned int hist[256];
+  unsigned int hist[8][256];   // one histogram per digit pass
 };
 
-__global__ void select_init_kernel(SelState* st, unsigned int k) {
+constexpr int kSelThreads = 512;
+constexpr long long kGridWaitCycles = 2000000000ll;
+
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Barrier over the whole grid (the launch is cooperative, so every CTA is
+// resident). The wait is bounded: on timeout the CTA records
+// SGPT_INFO_TIMEOUT and the caller returns.
+__device__ bool grid_sync(unsigned int* ctr, unsigned int target, int* info, int* failed) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const long long t0 = clock64();
+    while (ld_acquire(ctr) < target) {
+      if (clock64() - t0 > kGridWaitCycles) {
+        set_info(info, SGPT_INFO_TIMEOUT);
+        *failed = 1;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *failed == 0;
+}
+
+// Exact k-selection over the block's d_out x bw saliency keys in one
+// cooperative launch: a radix select on the 64-bit key, one 8-bit digit per
+// pass, most significant first (four passes on the saliency bits, four on
+// the index that breaks ties). Each pass histograms the digit of the keys
+// that match the prefix fixed so far; after a grid barrier every CTA scans
+// the same global histogram and takes the same decision, so a pass needs one
+// barrier. It stops as soon as the rank falls on a whole bin (usually after
+// the saliency passes). st must be zeroed before the launch; CTA 0 writes
+// the threshold.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(
+    const float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
+    const float* __restrict__ U, SelState* st, unsigned int k, int* info) {
+  if (cta_info_set(info)) return;
+  __shared__ unsigned int h[256];
+  __shared__ float ud[kMaxBlock];
+  __shared__ unsigned int wsum[kSelThreads / 32];
+  __shared__ unsigned long long s_prefix;
+  __shared__ unsigned int s_krem;
+  __shared__ int s_done, s_failed;
   const int t = threadIdx.x;
-  if (t < 256) st->hist[t] = 0;
+  if (t < bw) ud[t] = 1.0f / U[(long long)(i1 + t) * d + i1 + t];   // same reciprocal as the sweep
   if (t == 0) {
-    st->prefix = 0;
-    st->thr = 0;
-    st->k_rem = k;
-    st->done = (k == 0);
-    st->ticket = 0;
+    s_prefix = 0;
+    s_krem = k;
+    s_done = (k == 0);
+    s_failed = 0;
+  }
+  const long long total4 = (long long)rows * (bw / 4);
+  unsigned long long thr = 0;
+  for (int pass = 0; pass < 8; ++pass) {
+    if (t < 256) h[t] = 0;
+    __syncthreads();
+    if (s_done) break;
+    const int shift = 56 - 8 * pass;
+    const unsigned long long prefix = s_prefix;
+    // trip count uniform across the CTA: every lane takes part in the match
+    for (long long base = (long long)blockIdx.x * kSelThreads; base < total4;
+         base += (long long)gridDim.x * kSelThreads) {
+      const long long e = base + t;
+      const bool act = e < total4;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      int row = 0, c = 0;
+      if (act) {
+        row = (int)(e / (bw / 4));
+        c = (int)(e - (long long)row * (bw / 4)) * 4;
+        const float4 x = ld4(W + (long long)row * ldw + i1 + c);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const unsigned long long key =
+            act ? sal_key(v[j], ud[c + j], (unsigned)row * (unsigned)bw + (unsigned)(c + j)) : 0ull;
+        const bool mine = act && (pass == 0 || (key >> (shift + 8)) == prefix);
+        // saliencies span a narrow exponent range, so a warp holds few
+        // distinct digits: one shared atomic per digit and warp
+        const unsigned bin = mine ? (unsigned)((key >> shift) & 255u) : 256u;
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (mine && (t & 31) == (__ffs(peers) - 1)) atomicAdd(&h[bin], (unsigned)__popc(peers));
+      }
+    }
+    __syncthreads();
+    if (t < 256 && h[t]) atomicAdd(&st->hist[pass][t], h[t]);
+    if (!grid_sync(&st->arrive, (unsigned)(pass + 1) * gridDim.x, info, &s_failed)) return;
+    // every CTA: inclusive scan of the 256 bins and the bin holding rank k
+    const unsigned int cnt = (t < 256) ? __ldcg(&st->hist[pass][t]) : 0u;
+    unsigned int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if ((t & 31) >= o) inc += y;
+    }
+    if ((t & 31) == 31) wsum[t >> 5] = inc;
+    __syncthreads();
+    for (int w = 0; w < (t >> 5); ++w) inc += wsum[w];
+    const unsigned int kr = s_krem;
+    const unsigned int exc = inc - cnt;
+    __syncthreads();                          // everyone has read s_krem
+    if (t < 256 && cnt > 0 && exc < kr && kr <= inc) {
+      const unsigned int krem = kr - exc;
+      const unsigned long long pre = (prefix << 8) | (unsigned long long)t;
+      s_prefix = pre;
+      s_krem = krem;
+      if (cnt == krem) {
+        s_done = 1;
+        thr = (pre << shift) + (1ull << shift);   // every key of the bin is pruned
+        if (blockIdx.x == 0) st->thr = thr;
+      }
+    }
+    __syncthreads();
   }
 }
 
-// Pass p histograms digit p (bits 63-8p .. 56-8p) of the keys that match the
-// prefix found so far. The last CTA to finish picks the digit holding the
-// k-th smallest key and either finishes (the whole bin is pruned) or narrows
-// the prefix for the next pass.
-__global__ void __launch_bounds__(256) select_pass_kernel(
-    const float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
-    const float* __restrict__ U, SelState* st, int pass, const int* info) {
-  if (cta_info_set(info) || st->done) return;
-  __shared__ unsigned int h[256];
-  __shared__ float ud[kMaxBlock];
-  __shared__ unsigned int last;
-  const int t = threadIdx.x;
-  h[t] = 0;
-  if (t < bw) ud[t] = 1.0f / U[(long long)(i1 + t) * d + i1 + t];   // same reciprocal as the sweep
-  __syncthreads();
-  const int shift = 56 - 8 * pass;
-  const unsigned long long prefix = st->prefix;
+static cudaError_t launch_select(const float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
+                                 SelState* sel, unsigned int k, int* info, cudaStream_t st) {
+  static int max_grid = 0;
+  cudaError_t e = cudaSuccess;
+  if (!max_grid) {
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kSelThreads, 0)) != cudaSuccess)
+      return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    max_grid = std::max(1, std::min(per_sm, 2) * sms);
+  }
+  if ((e = cudaMemsetAsync(sel, 0, sizeof(SelState), st)) != cudaSuccess) return e;
   const long long total4 = (long long)rows * (bw / 4);
-  // The trip count is uniform across the block so that every lane of a warp
-  // takes part in the warp-wide match below.
-  for (long long base = (long long)blockIdx.x * 256; base < total4; base += (long long)gridDim.x * 256) {
-    const long long e = base + t;
-    const bool act = e < total4;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    int row = 0, c = 0;
-    if (act) {
-      row = (int)(e / (bw / 4));
-      c = (int)(e - (long long)row * (bw / 4)) * 4;
-      const float4 x = ld4(W + (long long)row * ldw + i1 + c);
-      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const unsigned long long key =
-          act ? sal_key(v[j], ud[c + j], (unsigned)row * (unsigned)bw + (unsigned)(c + j)) : 0ull;
-      const bool mine = act && (pass == 0 || (key >> (shift + 8)) == prefix);
-      // Most keys share a few digits (saliencies span a narrow exponent
-      // range): aggregate equal digits within the warp before the atomic.
-      const unsigned bin = mine ? (unsigned)((key >> shift) & 255u) : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (mine && (t & 31) == (__ffs(peers) - 1)) atomicAdd(&h[bin], (unsigned)__popc(peers));
-    }
-  }
-  __syncthreads();
-  if (h[t]) atomicAdd(&st->hist[t], h[t]);
-  __threadfence();
-  __syncthreads();
-  if (t == 0) last = (atomicAdd(&st->ticket, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  if (t == 0) {
-    unsigned int cum = 0, digit = 0, cnt = 0;
-    const unsigned int k = st->k_rem;
-    for (int b = 0; b < 256; ++b) {
-      const unsigned int c = __ldcg(&st->hist[b]);
-      if (cum + c >= k) { digit = b; cnt = c; break; }
-      cum += c;
-    }
-    const unsigned int krem = k - cum;
-    const unsigned long long pre = (prefix << 8) | digit;
-    st->prefix = pre;
-    st->k_rem = krem;
-    if (cnt == krem) {
-      st->done = 1;
-      st->thr = (pre << shift) + (1ull << shift);   // every key of the bin is pruned
-    }
-    st->ticket = 0;
-  }
-  __syncthreads();
-  st->hist[t] = 0;
+  const int grid = (int)std::max<long long>(1, std::min<long long>(cdivll(total4, kSelThreads), max_grid));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, select_kernel, W, ldw, rows, d, i1, bw, U, sel, k, info);
+  count_launches(1);
+  return e;
 }
 
 // ----------------------------------------------------------------- driver
@@ -365,14 +432,8 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
       count_launches(1);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
-      select_init_kernel<<<1, 256, 0, st>>>(w.sel, (unsigned int)kk);
-      count_launches(1);
-      const long long total4 = (long long)rows * (bw / 4);
-      const int g = (int)std::min<long long>(cdivll(total4, 256), 8 * kNumSMs);
-      for (int pass = 0; pass < 8; ++pass) {
-        select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, w.sel, pass, info);
-        count_launches(1);
-      }
+      if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
+        return e;
       sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
           W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, info);
       count_launches(1);
@@ -411,8 +472,8 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
 // re-initialised for every block).
 
 constexpr size_t kNoAllocErrBytes = (size_t)SGPT_NOALLOC_MAX_ROWS * kMaxBlock * sizeof(float);
-constexpr size_t kNoAllocScratchBytes = kNoAllocErrBytes + 4096;
-static_assert(sizeof(SelState) <= 4096, "selection state must fit the scratch tail");
+constexpr size_t kNoAllocScratchBytes = kNoAllocErrBytes + 16384;
+static_assert(sizeof(SelState) <= 16384, "selection state must fit the scratch tail");
 
 static __device__ __align__(256) unsigned char g_prune_scratch[kNoAllocScratchBytes];
 
@@ -468,14 +529,8 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
       count_launches(1);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
-      select_init_kernel<<<1, 256, 0, st>>>(sel, (unsigned int)kk);
-      count_launches(1);
-      const long long total4 = (long long)rows * (bw / 4);
-      const int g = (int)std::min<long long>(cdivll(total4, 256 * 8), 4 * kNumSMs);
-      for (int pass = 0; pass < 8; ++pass) {
-        select_pass_kernel<<<g, 256, 0, st>>>(W, ldw, rows, d, i1, bw, U, sel, pass, info);
-        count_launches(1);
-      }
+      if ((e = launch_select(W, ldw, rows, d, i1, bw, U, sel, (unsigned int)kk, info, st)) != cudaSuccess)
+        return e;
       sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
           W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info);
       count_launches(1);
