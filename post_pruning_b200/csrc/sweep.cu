@@ -5,11 +5,11 @@
 //      over all d_out rows: radix select on a 64-bit key (saliency bits, then
 //      row * bw + column), one cooperative launch of select_kernel with a
 //      grid barrier per 8-bit digit;
-//   2. sweep_kernel: every row's 128 columns are processed in order in
-//      registers: mask decision (2:4 at each group start on the compensated
-//      weights), e = (w_q - p_q) / U_qq (as a product with the reciprocal),
-//      rank-1 update of the rest of the
-//      block with the U row held in shared memory;
+//   2. sweep_kernel: one warp per row, one 4-column group per lane; the
+//      groups are processed in order: mask decision (2:4 at each group start
+//      on the compensated weights), e = (w_q - p_q) / U_qq (as a product with
+//      the reciprocal), rank-4 update of the rest of the block with the U
+//      rows held in shared memory;
 //   3. W[:, i2:] -= Err * U[i1:i2, i2:] as an FP32-accurate tensor-core GEMM
 //      (three TF32 products on hi/lo planes of Err and U, gemm_tc.cu).
 #include <cuda_runtime.h>
@@ -27,10 +27,8 @@ namespace sgpt {
 
 // ---------------------------------------------------------------- sweep
 
-constexpr int kSweepRows = 16;             // rows per CTA
-constexpr int kSeg = 16;                   // columns per thread
-constexpr int kTpr = kMaxBlock / kSeg;     // threads per row (8)
-constexpr int kSweepThreads = kSweepRows * kTpr;
+constexpr int kSweepRows = 8;              // rows per CTA, one warp each
+constexpr int kSweepThreads = kSweepRows * 32;
 constexpr size_t kSweepSmem = (size_t)kMaxBlock * kMaxBlock * sizeof(float);
 
 enum SweepMode { kModeNM24 = 0, kModeThreshold = 1, kModeForced = 2 };
@@ -39,6 +37,17 @@ __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsi
   return ((unsigned long long)__float_as_uint(saliency(w, inv_u)) << 32) | idx;
 }
 
+// One warp per row; lane l owns the block's columns 4l .. 4l+3, i.e. one
+// 4-column group (an N:M group never straddles two lanes). Groups are taken
+// in order. For group g every lane receives lane g's four weights, decides
+// the group's mask (2:4: on the compensated weights, at the group start) and
+// computes its four errors in column order with the in-group updates, all
+// lanes alike; lane g keeps the result and every lane right of it applies
+// the rank-4 update to its four columns. Arithmetically this is the
+// column-by-column sweep with the updates of the four columns to the columns
+// right of the group summed together. The chain per group is one shuffle,
+// the four in-group steps and one rank-4 update; the U values are loaded
+// before the weights arrive.
 template <int MODE>
 __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
@@ -49,146 +58,146 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
   extern __shared__ float Us[];   // [128][128]: U[i1 + a][i1 + b]
   __shared__ float Uinv[kMaxBlock];   // 1 / U_qq of the block's columns
   const int tid = threadIdx.x;
+  // U block to shared memory with asynchronous 16-byte copies, all in
+  // flight at once (rows are 16-byte aligned: i1 and d are multiples of 32)
   for (int e = tid * 4; e < kMaxBlock * kMaxBlock; e += kSweepThreads * 4) {
     const int a = e >> 7, b = e & 127;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (a < bw && b < bw) v = ld4(U + (long long)(i1 + a) * d + i1 + b);
-    st4(Us + e, v);
+    if (a < bw && b < bw)
+      cp_async16(Us + e, U + (long long)(i1 + a) * d + i1 + b);
+    else
+      st4(Us + e, make_float4(0.f, 0.f, 0.f, 0.f));
   }
+  cp_async_commit();
   if (tid < kMaxBlock) Uinv[tid] = tid < bw ? 1.0f / U[(long long)(i1 + tid) * d + i1 + tid] : 0.f;
-  __syncthreads();
 
   const int lane = tid & 31;
-  const int seg = tid % kTpr;                      // column segment of this thread
-  const int row = blockIdx.x * kSweepRows + tid / kTpr;
-  const bool live = row < rows && seg * kSeg < bw;
-  const int c0 = seg * kSeg;                       // block-relative first column
-  float w[kSeg], err[kSeg];
-  uint32_t keep = 0xffffu;
-  bool bad = false;
+  const int row = blockIdx.x * kSweepRows + (tid >> 5);
+  const int ngroups = bw >> 2;
+  const bool live = row < rows;
+  const bool mine = live && lane < ngroups;
+  const int c0 = 4 * lane;                         // block-relative first column
   float* wrow = W + (long long)row * ldw + i1 + c0;
-#pragma unroll
-  for (int v = 0; v < kSeg / 4; ++v) {
-    float4 x = live ? ld4(wrow + 4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
-    w[4 * v + 0] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+  float w[4] = {0.f, 0.f, 0.f, 0.f}, err[4] = {0.f, 0.f, 0.f, 0.f};
+  if (mine) {
+    const float4 x = ld4(wrow);
+    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
   }
-#pragma unroll
-  for (int j = 0; j < kSeg; ++j) {
-    err[j] = 0.f;
-    bad |= !isfinite(w[j]);
+  bool bad = !(isfinite(w[0]) && isfinite(w[1]) && isfinite(w[2]) && isfinite(w[3]));
+  uint32_t keep = 0xfu;
+  if (MODE == kModeForced && mine) {
+    const uint32_t word = mask[(long long)row * (d / 32) + (i1 + c0) / 32];
+    keep = (word >> ((i1 + c0) & 31)) & 0xfu;
   }
-  if (MODE == kModeThreshold && live) {
+  cp_async_wait_all();
+  __syncthreads();
+  if (MODE == kModeThreshold && mine) {
     const unsigned long long t = *thr;
     keep = 0;
 #pragma unroll
-    for (int j = 0; j < kSeg; ++j) {
+    for (int j = 0; j < 4; ++j) {
       const unsigned idx = (unsigned)row * (unsigned)bw + (unsigned)(c0 + j);
       if (sal_key(w[j], Uinv[c0 + j], idx) >= t) keep |= 1u << j;
     }
   }
-  if (MODE == kModeForced && live) {
-    const uint32_t word = mask[(long long)row * (d / 32) + (i1 + c0) / 32];
-    keep = (word >> ((i1 + c0) & 31)) & 0xffffu;
-  }
   float loss = 0.f;
+  // keep bit t of every lane, for the threshold and forced modes
+  uint32_t kb[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) kb[t] = __ballot_sync(0xffffffffu, (keep >> t) & 1u);
 
-  // Columns are taken four at a time (one N:M group; a group never straddles
-  // two threads). The owner of the group decides its mask, computes the four
-  // errors in order with the in-group updates done locally, and broadcasts
-  // them; every thread then applies the rank-4 update to its later columns.
-  // Arithmetically this is the column-by-column sweep with the updates of
-  // the four columns to the columns right of the group summed together.
-  // Segments run as a loop (not unrolled) to keep the body small enough for
-  // the instruction cache; the groups of a segment are unrolled so that every
-  // register index is static.
-  const int src = (lane & ~(kTpr - 1));
 #pragma unroll 1
-  for (int qs = 0; qs < kTpr; ++qs) {
-    if (qs * kSeg >= bw) break;
+  for (int g = 0; g < ngroups; ++g) {
+    const int q0 = 4 * g;
+    // everything that does not depend on the weights first: the owner's
+    // four rows of U at this lane's columns, its in-group entries and the
+    // reciprocal diagonal
+    const float4 u0 = ld4(Us + (q0 + 0) * kMaxBlock + c0);
+    const float4 u1 = ld4(Us + (q0 + 1) * kMaxBlock + c0);
+    const float4 u2 = ld4(Us + (q0 + 2) * kMaxBlock + c0);
+    const float4 u3 = ld4(Us + (q0 + 3) * kMaxBlock + c0);
+    const float4 g0 = ld4(Us + (q0 + 0) * kMaxBlock + q0);
+    const float4 g1 = ld4(Us + (q0 + 1) * kMaxBlock + q0);
+    const float4 g2 = ld4(Us + (q0 + 2) * kMaxBlock + q0);
+    const float4 ri = ld4(Uinv + q0);
+    // every lane takes the owner's weights and computes its group the same
+    // way, so no lane waits for a second broadcast
+    float wo[4];
 #pragma unroll
-    for (int g = 0; g < kSeg / 4; ++g) {
-      const int qj0 = 4 * g, q0 = qs * kSeg + qj0;
-      float e[4] = {0.f, 0.f, 0.f, 0.f};
-      if (seg == qs) {
-        if (MODE == kModeNM24) {
-          // 2 of 4 on the compensated weights; ties keep the lower column.
-          float sl[4];
+    for (int t = 0; t < 4; ++t) wo[t] = __shfl_sync(0xffffffffu, w[t], g);
+    const float r[4] = {ri.x, ri.y, ri.z, ri.w};
+    uint32_t km;
+    if (MODE == kModeNM24) {
+      // 2 of 4 on the compensated weights; ties keep the lower column.
+      float sl[4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) sl[t] = saliency(w[qj0 + t], Uinv[q0 + t]);
-          uint32_t gm = 0;
+      for (int t = 0; t < 4; ++t) sl[t] = saliency(wo[t], r[t]);
+      km = 0;
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            int rank = 0;   // how many of the group beat column t
+      for (int t = 0; t < 4; ++t) {
+        int rank = 0;   // how many of the group beat column t
 #pragma unroll
-            for (int o = 0; o < 4; ++o)
-              if (o != t && (sl[o] > sl[t] || (sl[o] == sl[t] && o < t))) ++rank;
-            if (rank < 2) gm |= 1u << t;
-          }
-          keep = (keep & ~(0xfu << qj0)) | (gm << qj0);
-        }
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int qj = qj0 + t, q = q0 + t;
-          const float wq = w[qj];
-          const bool kept = (keep >> qj) & 1u;
-          e[t] = kept ? 0.f : __fmul_rn(wq, Uinv[q]);
-          w[qj] = kept ? wq : 0.f;
-          err[qj] = e[t];
-          loss = fmaf(e[t], e[t], loss);
-          const float* urow = Us + q * kMaxBlock + c0;
-#pragma unroll
-          for (int jj = qj + 1; jj < qj0 + 4; ++jj) w[jj] = fmaf(-e[t], urow[jj], w[jj]);
-        }
+        for (int o = 0; o < 4; ++o)
+          if (o != t && (sl[o] > sl[t] || (sl[o] == sl[t] && o < t))) ++rank;
+        if (rank < 2) km |= 1u << t;
       }
+    } else {
+      km = ((kb[0] >> g) & 1u) | (((kb[1] >> g) & 1u) << 1) | (((kb[2] >> g) & 1u) << 2) | (((kb[3] >> g) & 1u) << 3);
+    }
+    float e[4];
+    e[0] = (km & 1u) ? 0.f : __fmul_rn(wo[0], r[0]);
+    wo[1] = fmaf(-e[0], g0.y, wo[1]);
+    wo[2] = fmaf(-e[0], g0.z, wo[2]);
+    wo[3] = fmaf(-e[0], g0.w, wo[3]);
+    e[1] = (km & 2u) ? 0.f : __fmul_rn(wo[1], r[1]);
+    wo[2] = fmaf(-e[1], g1.z, wo[2]);
+    wo[3] = fmaf(-e[1], g1.w, wo[3]);
+    e[2] = (km & 4u) ? 0.f : __fmul_rn(wo[2], r[2]);
+    wo[3] = fmaf(-e[2], g2.w, wo[3]);
+    e[3] = (km & 8u) ? 0.f : __fmul_rn(wo[3], r[3]);
+    if (lane == g) {
+      // the owner keeps its group's result
 #pragma unroll
-      for (int t = 0; t < 4; ++t) e[t] = __shfl_sync(0xffffffffu, e[t], src | qs);
-      if (seg >= qs && (e[0] != 0.f || e[1] != 0.f || e[2] != 0.f || e[3] != 0.f)) {
-        // columns of this segment right of the group
-#pragma unroll
-        for (int v = 0; v < kSeg / 4; ++v) {
-          const bool right = (seg > qs) || (4 * v > qj0);
-          if (!right) continue;
-          float4 u0 = ld4(Us + (q0 + 0) * kMaxBlock + c0 + 4 * v);
-          float4 u1 = ld4(Us + (q0 + 1) * kMaxBlock + c0 + 4 * v);
-          float4 u2 = ld4(Us + (q0 + 2) * kMaxBlock + c0 + 4 * v);
-          float4 u3 = ld4(Us + (q0 + 3) * kMaxBlock + c0 + 4 * v);
-          w[4 * v + 0] = fmaf(-e[3], u3.x, fmaf(-e[2], u2.x, fmaf(-e[1], u1.x, fmaf(-e[0], u0.x, w[4 * v + 0]))));
-          w[4 * v + 1] = fmaf(-e[3], u3.y, fmaf(-e[2], u2.y, fmaf(-e[1], u1.y, fmaf(-e[0], u0.y, w[4 * v + 1]))));
-          w[4 * v + 2] = fmaf(-e[3], u3.z, fmaf(-e[2], u2.z, fmaf(-e[1], u1.z, fmaf(-e[0], u0.z, w[4 * v + 2]))));
-          w[4 * v + 3] = fmaf(-e[3], u3.w, fmaf(-e[2], u2.w, fmaf(-e[1], u1.w, fmaf(-e[0], u0.w, w[4 * v + 3]))));
-        }
+      for (int t = 0; t < 4; ++t) {
+        w[t] = ((km >> t) & 1u) ? wo[t] : 0.f;
+        err[t] = e[t];
+        loss = fmaf(e[t], e[t], loss);
       }
+      keep = km;
+    } else if (lane > g) {
+      w[0] = fmaf(-e[3], u3.x, fmaf(-e[2], u2.x, fmaf(-e[1], u1.x, fmaf(-e[0], u0.x, w[0]))));
+      w[1] = fmaf(-e[3], u3.y, fmaf(-e[2], u2.y, fmaf(-e[1], u1.y, fmaf(-e[0], u0.y, w[1]))));
+      w[2] = fmaf(-e[3], u3.z, fmaf(-e[2], u2.z, fmaf(-e[1], u1.z, fmaf(-e[0], u0.z, w[2]))));
+      w[3] = fmaf(-e[3], u3.w, fmaf(-e[2], u2.w, fmaf(-e[1], u1.w, fmaf(-e[0], u0.w, w[3]))));
     }
   }
 
-  // Loss of the row: sum over its kTpr threads.
+  // Loss of the row: sum over the warp.
   float tot = loss;
 #pragma unroll
-  for (int o = 1; o < kTpr; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  for (int o = 1; o < 32; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
   bad |= !isfinite(tot);
-  // Mask words: segments 2p and 2p+1 make one 32-bit word.
-  const uint32_t other = __shfl_down_sync(0xffffffffu, keep, 1);
-  if (live) {
-#pragma unroll
-    for (int v = 0; v < kSeg / 4; ++v) st4(wrow + 4 * v, make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
+  // Mask words: lanes 8m .. 8m+7 make the word of columns 32m .. 32m+31.
+  uint32_t bits = mine ? (keep & 0xfu) << (4 * (lane & 7)) : 0u;
+  bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
+  bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
+  bits |= __shfl_xor_sync(0xffffffffu, bits, 4);
+  if (mine) {
+    st4(wrow, make_float4(w[0], w[1], w[2], w[3]));
     float* erow = Err + (long long)row * kMaxBlock + c0;
     if (Err_lo) {
       // hi/lo planes for the tensor-core trailing update
-      float* lrow = Err_lo + (long long)row * kMaxBlock + c0;
+      float lo[4];
 #pragma unroll
-      for (int j = 0; j < kSeg; ++j) {
+      for (int j = 0; j < 4; ++j) {
         const float h = tf32_hi(err[j]);
-        lrow[j] = err[j] - h;
+        lo[j] = err[j] - h;
         err[j] = h;
       }
+      st4(Err_lo + (long long)row * kMaxBlock + c0, make_float4(lo[0], lo[1], lo[2], lo[3]));
     }
-#pragma unroll
-    for (int v = 0; v < kSeg / 4; ++v) st4(erow + 4 * v, make_float4(err[4 * v], err[4 * v + 1], err[4 * v + 2], err[4 * v + 3]));
-    if (MODE != kModeForced && (seg & 1) == 0) {
-      const uint32_t hi = (c0 + kSeg < bw) ? other : 0u;
-      mask[(long long)row * (d / 32) + (i1 + c0) / 32] = (keep & 0xffffu) | (hi << 16);
-    }
-    if (seg == 0 && row_loss) row_loss[row] += tot;
+    st4(erow, make_float4(err[0], err[1], err[2], err[3]));
+    if (MODE != kModeForced && (lane & 7) == 0) mask[(long long)row * (d / 32) + (i1 + c0) / 32] = bits;
+    if (lane == 0 && row_loss) row_loss[row] += tot;
     if (bad) set_info(info, SGPT_INFO_NONFINITE);
   }
 }
