@@ -11,11 +11,14 @@
 // Used for the rank-128 updates and the triangular inverse of the
 // factorisation and for the lazy trailing update of the OBS sweep.
 //
-// CTA tile 128 x 128, K in chunks of 16 (one 64-byte swizzle row of fp32),
+// CTA tile 128 x 128, K in steps of 16 (one 64-byte swizzle row of fp32),
 // three-stage TMA ring in 96 KB (no multicast) so that two CTAs share an SM;
 // warp 0 lane 0 loads, warp 1 lane 0 issues MMAs, warps 2-5 drain TMEM
 // (warp w reads lanes 32*(w%4)..) into a shared staging tile and then update
-// C a whole row per warp instruction (coalesced).
+// C a whole row per warp instruction (coalesced). TMEM accumulates at most
+// 128 of K: a longer K alternates between two TMEM accumulators and the
+// epilogue warps sum the chunks in FP32 registers (a long accumulation inside
+// TMEM loses accuracy).
 // A is always K-major (row-major M x K); B is K-major (row-major N x K) or
 // MN-major (row-major K x N). Every wait is bounded.
 #include <cuda.h>
@@ -41,6 +44,8 @@ constexpr int kStageLd = kN + 4;                // epilogue staging row (floats)
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256;
 static_assert((size_t)kM * kStageLd * 4 <= (size_t)kStages * kStageBytes, "staging must fit the stages");
 constexpr long long kWaitCycles = 4000000000ll;
+constexpr int kChunk = 8;                       // K steps (128 of K) per TMEM accumulation
+constexpr int kTmemCols = 2 * kN;               // two accumulators: one fills while one drains
 
 __host__ __device__ constexpr uint32_t make_idesc(bool b_mn) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(kN >> 3) << 17) |
@@ -80,6 +85,9 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -147,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
   __shared__ int failed;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -183,19 +191,24 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
   const uint32_t idesc = make_idesc(b_mn != 0);
 
   const uint32_t s0 = smem_u32(smem);
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages), done = smem_u32(bars + 2 * kStages);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
+  const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16;
+  const int nchunks = (iters + kChunk - 1) / kChunk;
   if (threadIdx.x == 0) {
     failed = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 4);            // the four epilogue warps
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kN));
+                 "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -233,33 +246,45 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
     for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
       if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
   } else if (!skip && iters > 0 && warp == 1 && lane == 0) {
-    for (int it = 0; it < iters; ++it) {
-      const int s = it % kStages;
-      if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+    // chunk c (kChunk K steps) accumulates into TMEM buffer c & 1; a long K
+    // is summed chunk by chunk in FP32 registers by the epilogue warps
+    for (int c = 0; c < nchunks && !failed; ++c) {
+      const int b = c & 1;
+      if (c >= 2 && !mbar_wait(tempty0 + 8 * b, ((c >> 1) - 1) & 1)) {
         failed = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t st = s0 + s * kStageBytes;
-#pragma unroll
-      for (int ks = 0; ks < kKC / 8; ++ks) {
-        const uint64_t ah = kmajor_desc(st + ks * 32), al = kmajor_desc(st + kPlane + ks * 32);
-        uint64_t bh, bl;
-        if (b_mn) {
-          bh = mnmajor_desc(st + 2 * kPlane + ks * 1024);
-          bl = mnmajor_desc(st + 3 * kPlane + ks * 1024);
-        } else {
-          bh = kmajor_desc(st + 2 * kPlane + ks * 32);
-          bl = kmajor_desc(st + 3 * kPlane + ks * 32);
+      const uint32_t acc_t = tmem + (uint32_t)(b * kN);
+      const int it_end = min(iters, (c + 1) * kChunk);
+      for (int it = c * kChunk; it < it_end; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+          failed = 1;
+          break;
         }
-        const uint32_t first = (it == 0 && ks == 0) ? 0u : 1u;
-        mma_tf32(tmem, al, bh, idesc, first);   // small terms first
-        mma_tf32(tmem, ah, bl, idesc, 1u);
-        mma_tf32(tmem, ah, bh, idesc, 1u);
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t st = s0 + s * kStageBytes;
+#pragma unroll
+        for (int ks = 0; ks < kKC / 8; ++ks) {
+          const uint64_t ah = kmajor_desc(st + ks * 32), al = kmajor_desc(st + kPlane + ks * 32);
+          uint64_t bh, bl;
+          if (b_mn) {
+            bh = mnmajor_desc(st + 2 * kPlane + ks * 1024);
+            bl = mnmajor_desc(st + 3 * kPlane + ks * 1024);
+          } else {
+            bh = kmajor_desc(st + 2 * kPlane + ks * 32);
+            bl = kmajor_desc(st + 3 * kPlane + ks * 32);
+          }
+          const uint32_t first = (it == c * kChunk && ks == 0) ? 0u : 1u;
+          mma_tf32(acc_t, al, bh, idesc, first);   // small terms first
+          mma_tf32(acc_t, ah, bl, idesc, 1u);
+          mma_tf32(acc_t, ah, bh, idesc, 1u);
+        }
+        mma_commit(empty0 + 8 * s);
       }
-      mma_commit(empty0 + 8 * s);
+      mma_commit(tfull0 + 8 * b);
     }
-    mma_commit(done);
   }
 
   const bool partial = job.mode == 2 && job.nsplit > 1;
@@ -273,40 +298,64 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
                    : "memory");
     }
   }
-  bool have = !skip && iters > 0;
-  if (have && warp >= 2) {
-    __syncwarp();
-    if (!mbar_wait(done, 0)) {
-      failed = 1;
-      have = false;
+  // Epilogue warps: TMEM -> shared staging tile. Warp w reads TMEM lanes
+  // 32*(w%4).. (tile rows). One chunk goes straight to the staging tile;
+  // several are summed in FP32 registers first (each thread holds its row).
+  // The stage buffers are free for staging once the last chunk is in.
+  float* T = reinterpret_cast<float*>(smem);
+  const int q = warp & 3;
+  const int m = q * 32 + lane;                 // tile row = TMEM lane
+  if (!skip && warp >= 2) {
+    if (iters == 0) {
+#pragma unroll 1
+      for (int e = 0; e < kN; e += 4) *reinterpret_cast<float4*>(T + m * kStageLd + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else if (nchunks == 1) {
+      __syncwarp();
+      if (!mbar_wait(tfull0, 0)) failed = 1;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll 1
+      for (int cc = 0; cc < kN / 32 && !failed; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + cc * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(T + m * kStageLd + cc * 32 + e) =
+              make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                          __uint_as_float(v[e + 3]));
+      }
+    } else {
+      float acc[kN];
+#pragma unroll
+      for (int e = 0; e < kN; ++e) acc[e] = 0.f;
+      for (int c = 0; c < nchunks; ++c) {
+        const int b = c & 1;
+        __syncwarp();
+        if (!mbar_wait(tfull0 + 8 * b, (c >> 1) & 1)) {
+          failed = 1;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+        for (int cc = 0; cc < kN / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kN + cc * 32), v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc[cc * 32 + e] += __uint_as_float(v[e]);
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty0 + 8 * b);
+      }
+#pragma unroll
+      for (int e = 0; e < kN; e += 4)
+        *reinterpret_cast<float4*>(T + m * kStageLd + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
     }
   }
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
 
   if (!skip && !failed && warp >= 2) {
-    // TMEM -> shared staging tile (the stage buffers are free once the last
-    // MMA has committed), then whole rows per warp to global memory.
-    float* T = reinterpret_cast<float*>(smem);
-    const int q = warp & 3;
-    const int m = q * 32 + lane;               // tile row = TMEM lane
-#pragma unroll 1
-    for (int cc = 0; cc < kN / 32; ++cc) {
-      uint32_t v[32];
-      if (iters > 0) {
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + cc * 32, v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0u;
-      }
-#pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(T + m * kStageLd + cc * 32 + e) =
-            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                        __uint_as_float(v[e + 3]));
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");    // the four epilogue warps
     const int col = lane * 4;                  // this lane's four columns of a row
     const bool planes = job.C_hi != nullptr && (!job.planes_one_col || n0 == job.planes_n0);
     const long long ldp = job.ldp ? job.ldp : job.ldc;
@@ -352,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
 // Split partials of a block row -> C = alpha * sum (+ hi/lo planes), in split order.
