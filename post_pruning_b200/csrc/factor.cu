@@ -388,16 +388,14 @@ size_t factor_ws_bytes(int d) {
 
 size_t factor_part_tiles(int d) {
   const int K = cdiv(d, kTile);
-  size_t best = 0;
-  for (int t = 1; t < K; ++t) best = std::max(best, (size_t)t * urow_splits(t));
-  return best;
+  return K > 1 ? (size_t)tc::row_items(K - 1, urow_splits(K - 1)) : 0;
 }
 
 int urow_splits(int tiles) {
   // a block row of U with `tiles` tiles whose K lengths are 1..tiles blocks:
-  // split the long ones so the row fills about one wave, at least 2 blocks
-  // of K per split
-  return std::max(1, std::min(tiles / 2, kNumSMs / tiles));
+  // long ranges are cut into pieces of 8 blocks (1024 of K) so that the
+  // row's items are short and balance across SMs; short rows are not cut
+  return tiles > 8 ? 8 : 0;
 }
 
 namespace {
@@ -445,6 +443,10 @@ cudaError_t after(cudaStream_t s2, cudaStream_t s1, cudaEvent_t ev) {
   return e != cudaSuccess ? e : cudaStreamWaitEvent(s2, ev, 0);
 }
 
+// Off-chain GEMMs are persistent kernels that would otherwise hold every SM
+// for their whole duration; they leave some to the chain's launches.
+constexpr int kOffChainCtas = kNumSMs - 16;
+
 // The block-column loop and the V / U block rows (see the file comment).
 cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const FactorStreams& f) {
   const int K = cdiv(d, kTile);
@@ -470,6 +472,7 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
       v.alpha = 1.f;
       v.C_hi = w.R;
       v.C_lo = w.V_lo;
+      v.max_ctas = kOffChainCtas;
       if ((e = tc::launch_gemm(Ud, Rp, true, v, K - 1 - k, info, f.rows)) != cudaSuccess) return e;
       tc::Job u{};
       u.mode = 2;
@@ -484,7 +487,9 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
       u.C_hi = w.U_hi;
       u.C_lo = w.U_lo;
       u.part = w.part;
-      if ((e = tc::launch_gemm(Rp, Ud, true, u, (K - 1 - k) * u.nsplit, info, f.rows)) != cudaSuccess) return e;
+      u.max_ctas = kOffChainCtas;
+      if ((e = tc::launch_gemm(Rp, Ud, true, u, tc::row_items(K - 1 - k, u.nsplit), info, f.rows)) != cudaSuccess)
+        return e;
     }
     if (k == 0) break;
     {
@@ -521,7 +526,9 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
     job.beta = 1.f;
     if (k >= 2) {
       if ((e = after(f.upd, f.crit, f.panel_done)) != cudaSuccess) return e;
+      job.max_ctas = kOffChainCtas;
       if ((e = tc::launch_gemm(P, P, false, job, (k - 1) * k / 2, info, f.upd)) != cudaSuccess) return e;
+      job.max_ctas = 0;
       if ((e = cudaEventRecord(f.upd_done, f.upd)) != cudaSuccess) return e;
       upd_pending = true;
     }

@@ -11,14 +11,15 @@
 // Used for the rank-128 updates and the triangular inverse of the
 // factorisation and for the lazy trailing update of the OBS sweep.
 //
-// CTA tile 128 x 128, K in steps of 16 (one 64-byte swizzle row of fp32),
-// three-stage TMA ring in 96 KB (no multicast) so that two CTAs share an SM;
-// warp 0 lane 0 loads, warp 1 lane 0 issues MMAs, warps 2-5 drain TMEM
-// (warp w reads lanes 32*(w%4)..) into a shared staging tile and then update
-// C a whole row per warp instruction (coalesced). TMEM accumulates at most
-// 128 of K: a longer K alternates between two TMEM accumulators and the
-// epilogue warps sum the chunks in FP32 registers (a long accumulation inside
-// TMEM loses accuracy).
+// Output tiles of 128 x 128, K in stages of 32 (one 128-byte swizzle row of
+// fp32) through a two-stage TMA ring of 64 KB stages (no multicast). Persistent: one CTA per
+// SM walks its share of the launch's tiles; warp 0 lane 0 loads, warp 1 lane
+// 0 issues MMAs, warps 2-9 drain TMEM, combine it with the C tile that TMA
+// brought into shared memory one tile ahead, and write whole rows per warp
+// instruction (coalesced). TMEM accumulates at most 128
+// of K per accumulator; two accumulators alternate, so a tile's epilogue
+// overlaps the next tile's main loop and a longer K is summed chunk by chunk
+// in FP32 registers (a long accumulation inside TMEM loses accuracy).
 // A is always K-major (row-major M x K); B is K-major (row-major N x K) or
 // MN-major (row-major K x N). Every wait is bounded.
 #include <cuda.h>
@@ -35,16 +36,18 @@ namespace tc {
 
 namespace {
 
-constexpr int kM = 128, kN = 128, kKC = 16;
-constexpr int kStages = 3;
-constexpr int kPlane = kM * kKC * 4;            // 8 KB: one operand plane of one stage
+constexpr int kM = 128, kN = 128, kKC = 32;   // K per stage: one 128-byte swizzle row of fp32
+constexpr int kStages = 2;
+constexpr int kPlane = kM * kKC * 4;            // 16 KB: one operand plane of one stage
 constexpr int kStageBytes = 4 * kPlane;         // A hi/lo, B hi/lo
-constexpr int kThreads = 192;
-constexpr int kStageLd = kN + 4;                // epilogue staging row (floats)
-constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256;
-static_assert((size_t)kM * kStageLd * 4 <= (size_t)kStages * kStageBytes, "staging must fit the stages");
+constexpr int kEpiWarps = 8;                    // two per TMEM lane quadrant, 64 columns each
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // producer, MMA issuer, epilogue
+// Epilogue tile: 128 x 128 fp32 as four 32-column groups of 128 rows x 128
+// bytes, 16-byte chunks XOR-swizzled by row % 8 (TMA's 128-byte swizzle).
+constexpr size_t kStagingBytes = (size_t)kM * kN * 4;
+constexpr size_t kSmem = (size_t)kStages * kStageBytes + kStagingBytes + 1024 + 256;
 constexpr long long kWaitCycles = 4000000000ll;
-constexpr int kChunk = 8;                       // K steps (128 of K) per TMEM accumulation
+constexpr int kChunk = 128 / kKC;               // stages (128 of K) per TMEM accumulation
 constexpr int kTmemCols = 2 * kN;               // two accumulators: one fills while one drains
 
 __host__ __device__ constexpr uint32_t make_idesc(bool b_mn) {
@@ -56,27 +59,27 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// K-major operand, 64-byte swizzle (a K chunk of 16 fp32 is one 64-byte
-// row): 8-row groups of 512 bytes.
+// K-major operand, 128-byte swizzle (a K stage of 32 fp32 is one 128-byte
+// row): 8-row groups of 1024 bytes.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3fff);
   d |= (uint64_t)1 << 16;                         // leading byte offset (unused when swizzled)
-  d |= (uint64_t)(512 >> 4) << 32;                // stride byte offset: next 8 rows
+  d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: next 8 rows
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)4 << 61;                         // SWIZZLE_64B
+  d |= (uint64_t)2 << 61;                         // SWIZZLE_128B
   return d;
 }
 // MN-major 32-bit operand: the 128-byte swizzle with 32-byte granules
 // (descriptor layout SWIZZLE_128B_BASE32B, filled by TMA's
 // SWIZZLE_128B_ATOM_32B). Atoms are 32 columns x 4 K rows (512 bytes);
-// LBO = next 32 columns (one 32-column x 16-row TMA box, 2 KB), SBO = next
+// LBO = next 32 columns (one 32-column x kKC-row TMA box), SBO = next
 // 4 K rows. The plain 128-byte swizzle (16-byte granules) is not a valid
 // MN-major form for 32-bit elements.
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3fff);
-  d |= (uint64_t)(2048 >> 4) << 16;
+  d |= (uint64_t)((kKC * 128) >> 4) << 16;
   d |= (uint64_t)(512 >> 4) << 32;
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)1 << 61;
@@ -147,63 +150,94 @@ __device__ __forceinline__ void tri_index(int t, int& i, int& j) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
+// Items before tile t of a split block row: tile t' has t' / b + 1 pieces.
+__host__ __device__ __forceinline__ int split_prefix(int t, int b) {
+  const int a = t / b;
+  return t + b * a * (a - 1) / 2 + a * (t - b * a);
+}
+
+// Work item w of a launch: its output tile (m0, n0) and K range [kb, ke).
+struct Item {
+  int m0, n0, kb, ke;
+};
+
+__device__ __forceinline__ Item decode_item(const Job& job, int w) {
+  Item it{0, 0, 0, 0};
+  if (job.mode == 0) {
+    it.m0 = (w / job.nt) * kM;
+    it.n0 = (w % job.nt) * kN;
+    it.ke = job.kdim;
+  } else if (job.mode == 1) {
+    int i, j;
+    tri_index(job.t0 + w, i, j);
+    it.m0 = i * kM;
+    it.n0 = j * kN;
+    it.ke = job.kdim;
+  } else if (job.mode == 3) {
+    it.m0 = job.s * kM;
+    it.n0 = (job.s + 1 + w) * kN;
+    it.kb = it.m0;
+    it.ke = min(it.m0 + kM, job.dlim);
+  } else {
+    int tile = w, piece = 0;
+    if (job.nsplit > 0) {                     // the tile whose pieces hold item w
+      int lo = 0, hi = job.nblk - 1 - job.s;  // split_prefix(lo) <= w < split_prefix(hi)
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (split_prefix(mid, job.nsplit) <= w) lo = mid; else hi = mid;
+      }
+      tile = lo;
+      piece = w - split_prefix(lo, job.nsplit);
+    }
+    const int i = job.s, j = job.s + 1 + tile;
+    it.m0 = i * kM;
+    it.n0 = j * kN;
+    const int lo = (i + 1) * kM, hi = min((j + 1) * kM, job.dlim);
+    if (job.nsplit > 0) {
+      it.kb = min(hi, lo + piece * job.nsplit * kM);
+      it.ke = min(hi, it.kb + job.nsplit * kM);
+    } else {
+      it.kb = lo;
+      it.ke = hi;
+    }
+  }
+  return it;
+}
+
+// Persistent: CTA c takes items c, c + gridDim.x, ... The TMA ring runs
+// through the K steps of all its items without a break; the MMA warp fills
+// one TMEM accumulator per unit of at most kChunk K steps, alternating two,
+// while the epilogue warps drain the other, so one tile's epilogue overlaps
+// the next tile's main loop.
+__global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
     const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
     const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo, const Job job,
-    const int b_mn, int* info) {
+    const __grid_constant__ CUtensorMap c_map, const int b_mn, const int items, int* info) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  unsigned char* T = smem + kStages * kStageBytes;   // epilogue tile (C in, result out)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kStagingBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   __shared__ int failed;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (cta_info_set(info)) return;
 
-  // ---- which tile and which K range
-  int m0 = 0, n0 = 0, kb = 0, ke = 0, split = 0, tile = 0;
-  if (job.mode == 0) {
-    m0 = (blockIdx.x / job.nt) * kM;
-    n0 = (blockIdx.x % job.nt) * kN;
-    ke = job.kdim;
-  } else if (job.mode == 1) {
-    int i, j;
-    tri_index(job.t0 + (int)blockIdx.x, i, j);
-    m0 = i * kM;
-    n0 = j * kN;
-    ke = job.kdim;
-  } else if (job.mode == 3) {
-    m0 = job.s * kM;
-    n0 = (job.s + 1 + (int)blockIdx.x) * kN;
-    kb = m0;
-    ke = min(m0 + kM, job.dlim);
-  } else {
-    tile = blockIdx.x / job.nsplit;
-    split = blockIdx.x - tile * job.nsplit;
-    const int i = job.s, j = job.s + 1 + tile;
-    m0 = i * kM;
-    n0 = j * kN;
-    const int lo = (i + 1) * kM, hi = min((j + 1) * kM, job.dlim);
-    const int per = ((j - i + job.nsplit - 1) / job.nsplit) * kM;
-    kb = min(hi, lo + split * per);
-    ke = min(hi, kb + per);
-  }
-  const int iters = (ke - kb + kKC - 1) / kKC;
   const uint32_t idesc = make_idesc(b_mn != 0);
-
   const uint32_t s0 = smem_u32(smem);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
-  const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16;
-  const int nchunks = (iters + kChunk - 1) / kChunk;
+  const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16, cfull = tfull0 + 32;
   if (threadIdx.x == 0) {
     failed = 0;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(full0 + 8 * st, 1);
+      mbar_init(empty0 + 8 * st, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, 4);            // the four epilogue warps
+      mbar_init(tempty0 + 8 * b, kEpiWarps);
     }
+    mbar_init(cfull, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -215,196 +249,195 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_tf32x3_kernel(
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
-  const bool skip = cta_info_set(info);
 
-  if (!skip && iters > 0 && warp == 0 && lane == 0) {
-    int issued = 0;
-    for (int it = 0; it < iters; ++it) {
-      const int s = it % kStages;
-      if (it >= kStages && !mbar_wait(empty0 + 8 * s, ((it / kStages) & 1) ^ 1)) {
-        failed = 1;
-        break;
-      }
-      const uint32_t bar = full0 + 8 * s;
-      mbar_expect_tx(bar, kStageBytes);
-      const uint32_t st = s0 + s * kStageBytes;
-      const int k = kb + it * kKC;
-      tma_2d(st, &a_hi, bar, job.a_x0 + k, job.a_y0 + m0);
-      tma_2d(st + kPlane, &a_lo, bar, job.a_x0 + k, job.a_y0 + m0);
-      if (b_mn) {
-#pragma unroll
-        for (int c = 0; c < kN / 32; ++c) {
-          tma_2d(st + 2 * kPlane + c * 2048, &b_hi, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
-          tma_2d(st + 3 * kPlane + c * 2048, &b_lo, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
-        }
-      } else {
-        tma_2d(st + 2 * kPlane, &b_hi, bar, job.b_x0 + k, job.b_y0 + n0);
-        tma_2d(st + 3 * kPlane, &b_lo, bar, job.b_x0 + k, job.b_y0 + n0);
-      }
-      ++issued;
-    }
-    for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
-      if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
-  } else if (!skip && iters > 0 && warp == 1 && lane == 0) {
-    // chunk c (kChunk K steps) accumulates into TMEM buffer c & 1; a long K
-    // is summed chunk by chunk in FP32 registers by the epilogue warps
-    for (int c = 0; c < nchunks && !failed; ++c) {
-      const int b = c & 1;
-      if (c >= 2 && !mbar_wait(tempty0 + 8 * b, ((c >> 1) - 1) & 1)) {
-        failed = 1;
-        break;
-      }
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t acc_t = tmem + (uint32_t)(b * kN);
-      const int it_end = min(iters, (c + 1) * kChunk);
-      for (int it = c * kChunk; it < it_end; ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
-          failed = 1;
-          break;
-        }
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t st = s0 + s * kStageBytes;
-#pragma unroll
-        for (int ks = 0; ks < kKC / 8; ++ks) {
-          const uint64_t ah = kmajor_desc(st + ks * 32), al = kmajor_desc(st + kPlane + ks * 32);
-          uint64_t bh, bl;
-          if (b_mn) {
-            bh = mnmajor_desc(st + 2 * kPlane + ks * 1024);
-            bl = mnmajor_desc(st + 3 * kPlane + ks * 1024);
-          } else {
-            bh = kmajor_desc(st + 2 * kPlane + ks * 32);
-            bl = kmajor_desc(st + 3 * kPlane + ks * 32);
+  if (warp == 0) {
+    if (lane == 0) {
+      // TMA producer: the K steps of every item, one stage each
+      int g = 0;                                  // stage uses so far
+      for (int w = blockIdx.x; w < items && !failed; w += gridDim.x) {
+        const Item it = decode_item(job, w);
+        const int iters = (it.ke - it.kb + kKC - 1) / kKC;
+        for (int i = 0; i < iters; ++i, ++g) {
+          const int st = g % kStages;
+          if (g >= kStages && !mbar_wait(empty0 + 8 * st, ((g / kStages) & 1) ^ 1)) {
+            failed = 1;
+            break;
           }
-          const uint32_t first = (it == c * kChunk && ks == 0) ? 0u : 1u;
-          mma_tf32(acc_t, al, bh, idesc, first);   // small terms first
-          mma_tf32(acc_t, ah, bl, idesc, 1u);
-          mma_tf32(acc_t, ah, bh, idesc, 1u);
-        }
-        mma_commit(empty0 + 8 * s);
-      }
-      mma_commit(tfull0 + 8 * b);
-    }
-  }
-
-  const bool partial = job.mode == 2 && job.nsplit > 1;
-  const bool read_c = !partial && job.C != nullptr && job.beta != 0.f;
-  if (!skip && read_c && warp >= 2) {
-    // Bring this warp's 32 rows of C toward L2 while the main loop runs.
-    const int row = m0 + (warp - 2) * 32 + lane;
-    if (row < job.Mlim && n0 < job.Nlim) {
-      const float* p = job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + n0;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(min(kN, job.Nlim - n0) * 4)
-                   : "memory");
-    }
-  }
-  // Epilogue warps: TMEM -> shared staging tile. Warp w reads TMEM lanes
-  // 32*(w%4).. (tile rows). One chunk goes straight to the staging tile;
-  // several are summed in FP32 registers first (each thread holds its row).
-  // The stage buffers are free for staging once the last chunk is in.
-  float* T = reinterpret_cast<float*>(smem);
-  const int q = warp & 3;
-  const int m = q * 32 + lane;                 // tile row = TMEM lane
-  if (!skip && warp >= 2) {
-    if (iters == 0) {
-#pragma unroll 1
-      for (int e = 0; e < kN; e += 4) *reinterpret_cast<float4*>(T + m * kStageLd + e) = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else if (nchunks == 1) {
-      __syncwarp();
-      if (!mbar_wait(tfull0, 0)) failed = 1;
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll 1
-      for (int cc = 0; cc < kN / 32 && !failed; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + cc * 32, v);
+          const uint32_t bar = full0 + 8 * st;
+          mbar_expect_tx(bar, kStageBytes);
+          const uint32_t sa = s0 + st * kStageBytes;
+          const int k = it.kb + i * kKC;
+          tma_2d(sa, &a_hi, bar, job.a_x0 + k, job.a_y0 + it.m0);
+          tma_2d(sa + kPlane, &a_lo, bar, job.a_x0 + k, job.a_y0 + it.m0);
+          if (b_mn) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(T + m * kStageLd + cc * 32 + e) =
-              make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                          __uint_as_float(v[e + 3]));
-      }
-    } else {
-      float acc[kN];
-#pragma unroll
-      for (int e = 0; e < kN; ++e) acc[e] = 0.f;
-      for (int c = 0; c < nchunks; ++c) {
-        const int b = c & 1;
-        __syncwarp();
-        if (!mbar_wait(tfull0 + 8 * b, (c >> 1) & 1)) {
-          failed = 1;
-          break;
+            for (int c = 0; c < kN / 32; ++c) {
+              tma_2d(sa + 2 * kPlane + c * kKC * 128, &b_hi, bar, job.b_x0 + it.n0 + 32 * c, job.b_y0 + k);
+              tma_2d(sa + 3 * kPlane + c * kKC * 128, &b_lo, bar, job.b_x0 + it.n0 + 32 * c, job.b_y0 + k);
+            }
+          } else {
+            tma_2d(sa + 2 * kPlane, &b_hi, bar, job.b_x0 + k, job.b_y0 + it.n0);
+            tma_2d(sa + 3 * kPlane, &b_lo, bar, job.b_x0 + k, job.b_y0 + it.n0);
+          }
         }
+      }
+      // never leave with copies in flight: wait for every stage still armed
+      for (int x = (g > kStages ? g - kStages : 0); x < g; ++x)
+        if (!mbar_wait(full0 + 8 * (x % kStages), (x / kStages) & 1)) failed = 1;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MMA issuer: unit u (<= kChunk K steps of one item) into TMEM buffer u & 1
+      int g = 0, u = 0;
+      for (int w = blockIdx.x; w < items && !failed; w += gridDim.x) {
+        const Item it = decode_item(job, w);
+        const int iters = (it.ke - it.kb + kKC - 1) / kKC;
+        for (int c0 = 0; c0 < iters && !failed; c0 += kChunk, ++u) {
+          const int b = u & 1;
+          if (u >= 2 && !mbar_wait(tempty0 + 8 * b, ((u >> 1) - 1) & 1)) {
+            failed = 1;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint32_t acc_t = tmem + (uint32_t)(b * kN);
+          const int c1 = min(iters, c0 + kChunk);
+          for (int i = c0; i < c1; ++i, ++g) {
+            const int st = g % kStages;
+            if (!mbar_wait(full0 + 8 * st, (g / kStages) & 1)) {
+              failed = 1;
+              break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t sa = s0 + st * kStageBytes;
+#pragma unroll
+            for (int ks = 0; ks < kKC / 8; ++ks) {
+              const uint64_t ah = kmajor_desc(sa + ks * 32), al = kmajor_desc(sa + kPlane + ks * 32);
+              uint64_t bh, bl;
+              if (b_mn) {
+                bh = mnmajor_desc(sa + 2 * kPlane + ks * 1024);
+                bl = mnmajor_desc(sa + 3 * kPlane + ks * 1024);
+              } else {
+                bh = kmajor_desc(sa + 2 * kPlane + ks * 32);
+                bl = kmajor_desc(sa + 3 * kPlane + ks * 32);
+              }
+              const uint32_t first = (i == c0 && ks == 0) ? 0u : 1u;
+              mma_tf32(acc_t, al, bh, idesc, first);   // small terms first
+              mma_tf32(acc_t, ah, bl, idesc, 1u);
+              mma_tf32(acc_t, ah, bh, idesc, 1u);
+            }
+            mma_commit(empty0 + 8 * st);
+          }
+          mma_commit(tfull0 + 8 * b);
+        }
+      }
+    }
+  } else {
+    // Epilogue warps: warp w reads TMEM lanes 32*(w%4).. (tile rows) and
+    // columns 64*h.., h = (w-2)/4, and sums an item's units in FP32
+    // registers (one unit: just copied). C arrives by TMA in the epilogue
+    // tile, requested one item ahead; each thread forms alpha * acc +
+    // beta * C for its row in place, and the warps write whole rows out
+    // (coalesced) with the optional hi/lo planes.
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const int m = q * 32 + lane;                  // tile row = TMEM lane
+    const int ew = warp - 2;                      // 0..7: rows 16*ew.. in the write-out
+    const bool partial = job.mode == 2 && job.nsplit > 0;
+    const bool read_c = !partial && job.C != nullptr && job.beta != 0.f;
+    const long long ldp = job.ldp ? job.ldp : job.ldc;
+    const bool issuer = (warp == 2 && lane == 0);
+    auto load_c = [&](int ww) {                   // TMA of item ww's C tile (four 32-column groups)
+      const Item nx = decode_item(job, ww);
+      mbar_expect_tx(cfull, (uint32_t)kStagingBytes);
+#pragma unroll
+      for (int g4 = 0; g4 < 4; ++g4)
+        tma_2d(smem_u32(T) + g4 * (kM * 128), &c_map, cfull, job.c_col0 + nx.n0 + 32 * g4, job.c_row0 + nx.m0);
+    };
+    int c_issued = 0;                             // C tiles requested (issuer only)
+    if (read_c && issuer && (int)blockIdx.x < items) {
+      load_c(blockIdx.x);
+      ++c_issued;
+    }
+    int u = 0, nitem = 0;
+    for (int w = blockIdx.x; w < items; w += gridDim.x, ++nitem) {
+      const Item it = decode_item(job, w);
+      const int iters = (it.ke - it.kb + kKC - 1) / kKC;
+      float acc[64];
+#pragma unroll
+      for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+      for (int c0 = 0; c0 < iters; c0 += kChunk, ++u) {
+        const int b = u & 1;
+        if (!failed && !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1)) failed = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (!failed) {
 #pragma unroll
-        for (int cc = 0; cc < kN / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kN + cc * 32), v);
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kN + h * 64 + cc * 32), v);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) acc[cc * 32 + e] += __uint_as_float(v[e]);
+            for (int e = 0; e < 32; ++e) acc[cc * 32 + e] += __uint_as_float(v[e]);
+          }
         }
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty0 + 8 * b);
       }
+      if (read_c && !failed && !mbar_wait(cfull, nitem & 1)) failed = 1;
+      // this thread's 64 columns = 16 chunks of 16 bytes in groups 2h, 2h+1
 #pragma unroll
-      for (int e = 0; e < kN; e += 4)
-        *reinterpret_cast<float4*>(T + m * kStageLd + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+      for (int cj = 0; cj < 16; ++cj) {
+        const int g4 = 2 * h + (cj >> 3), j = cj & 7;
+        float4* pch = reinterpret_cast<float4*>(T + g4 * (kM * 128) + m * 128 + ((j ^ (m & 7)) << 4));
+        float4 o = make_float4(acc[4 * cj], acc[4 * cj + 1], acc[4 * cj + 2], acc[4 * cj + 3]);
+        if (!partial) {
+          const float4 cv = read_c ? *pch : make_float4(0.f, 0.f, 0.f, 0.f);
+          o = make_float4(fmaf(job.alpha, o.x, job.beta * cv.x), fmaf(job.alpha, o.y, job.beta * cv.y),
+                          fmaf(job.alpha, o.z, job.beta * cv.z), fmaf(job.alpha, o.w, job.beta * cv.w));
+        }
+        *pch = o;
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
+      if (!failed) {
+        const bool planes = job.C_hi != nullptr && (!job.planes_one_col || it.n0 == job.planes_n0);
+        const int cn = lane * 4;                  // lane = 16-byte chunk of the row
+        const bool col_ok = it.n0 + cn < job.Nlim;
+        const int g4 = lane >> 3, j = lane & 7;
+#pragma unroll 4
+        for (int x = 0; x < 16; ++x) {
+          const int mr = ew * 16 + x;
+          const float4 o = *reinterpret_cast<const float4*>(T + g4 * (kM * 128) + mr * 128 + ((j ^ (mr & 7)) << 4));
+          if (partial) {
+            st4(job.part + (size_t)w * kM * kN + (size_t)mr * kN + cn, o);
+            continue;
+          }
+          const int row = it.m0 + mr;
+          if (row >= job.Mlim || !col_ok) continue;
+          if (job.C) st4(job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + it.n0 + cn, o);
+          if (planes) {
+            const long long off = (long long)(job.c_row0 + row) * ldp + job.c_col0 + it.n0 + cn - job.p_col0;
+            const float4 hv = make_float4(tf32_hi(o.x), tf32_hi(o.y), tf32_hi(o.z), tf32_hi(o.w));
+            st4(job.C_hi + off, hv);
+            st4(job.C_lo + off, make_float4(o.x - hv.x, o.y - hv.y, o.z - hv.z, o.w - hv.w));
+          }
+        }
+      }
+      // every read of the tile is done: the next item's C may come in
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
+      if (read_c && issuer && !failed && w + (int)gridDim.x < items) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        load_c(w + gridDim.x);
+        ++c_issued;
+      }
     }
+    // never leave with a C copy in flight (after a timeout some were not waited for)
+    if (read_c && issuer && c_issued > 0) mbar_wait(cfull, (c_issued - 1) & 1);
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
-
-  if (!skip && !failed && warp >= 2) {
-    const int col = lane * 4;                  // this lane's four columns of a row
-    const bool planes = job.C_hi != nullptr && (!job.planes_one_col || n0 == job.planes_n0);
-    const long long ldp = job.ldp ? job.ldp : job.ldc;
-    const bool col_ok = n0 + col < job.Nlim;
-#pragma unroll 1
-    for (int r0 = 0; r0 < 32; r0 += 8) {
-      float4 a[8], old[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {            // all loads of 8 rows first
-        const int mr = (warp - 2) * 32 + r0 + u;
-        a[u] = *reinterpret_cast<const float4*>(T + mr * kStageLd + col);
-        old[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (read_c && col_ok && m0 + mr < job.Mlim)
-          old[u] = ld4(job.C + (long long)(job.c_row0 + m0 + mr) * job.ldc + job.c_col0 + n0 + col);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int mr = (warp - 2) * 32 + r0 + u;
-        if (partial) {
-          st4(job.part + (size_t)blockIdx.x * kM * kN + (size_t)mr * kN + col, a[u]);
-          continue;
-        }
-        const int row = m0 + mr;
-        if (row >= job.Mlim || !col_ok) continue;
-        const float o[4] = {fmaf(job.alpha, a[u].x, job.beta * old[u].x), fmaf(job.alpha, a[u].y, job.beta * old[u].y),
-                            fmaf(job.alpha, a[u].z, job.beta * old[u].z), fmaf(job.alpha, a[u].w, job.beta * old[u].w)};
-        if (job.C)
-          st4(job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + n0 + col,
-              make_float4(o[0], o[1], o[2], o[3]));
-        if (planes) {
-          const long long off = (long long)(job.c_row0 + row) * ldp + job.c_col0 + n0 + col - job.p_col0;
-          float h4[4], l4[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            h4[t] = tf32_hi(o[t]);
-            l4[t] = o[t] - h4[t];
-          }
-          st4(job.C_hi + off, make_float4(h4[0], h4[1], h4[2], h4[3]));
-          st4(job.C_lo + off, make_float4(l4[0], l4[1], l4[2], l4[3]));
-        }
-      }
-    }
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-// Split partials of a block row -> C = alpha * sum (+ hi/lo planes), in split order.
+// Split partials of a block row -> C = alpha * sum (+ hi/lo planes), in piece order.
 __global__ void __launch_bounds__(256) rowsplit_reduce_kernel(const Job job, const int* info) {
   if (cta_info_set(info)) return;
   const int tiles = job.nblk - 1 - job.s;
@@ -416,9 +449,10 @@ __global__ void __launch_bounds__(256) rowsplit_reduce_kernel(const Job job, con
     const int m = e / kN, n = e % kN;
     const int row = job.s * kM + m, col = (job.s + 1 + tile) * kN + n;
     if (row >= job.Mlim || col >= job.Nlim) continue;
-    const float* src = job.part + (size_t)tile * job.nsplit * kM * kN + e;
+    const int p0 = split_prefix(tile, job.nsplit), np = tile / job.nsplit + 1;
+    const float* src = job.part + (size_t)p0 * kM * kN + e;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = 0; p < job.nsplit; ++p) {
+    for (int p = 0; p < np; ++p) {
       const float4 v = __ldcs(reinterpret_cast<const float4*>(src + (size_t)p * kM * kN));
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
@@ -475,8 +509,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // Tensor map over a row-major fp32 matrix [rows x cols] with leading dimension
-// ld; box = box_x (inner, fp32 elements) x box_y rows; 64-byte swizzle for
-// K-major operands (16-float rows), 128-byte swizzle with 32-byte granules
+// ld; box = box_x (inner, fp32 elements) x box_y rows; 128-byte swizzle for
+// K-major operands (32-float rows), 128-byte swizzle with 32-byte granules
 // for MN-major ones (32-float rows).
 bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, long long ld, int box_x, int box_y,
               bool mn_major) {
@@ -488,12 +522,28 @@ bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, lo
   const cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE,
-             mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+             mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map over C for the epilogue: boxes of 32 columns x 128 rows with the
+// 128-byte swizzle.
+bool make_map_c(CUtensorMap* m, const float* p, long long rows, long long cols, long long ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {32, (cuuint32_t)kM};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
+
+int row_items(int tiles, int blocks) { return blocks > 0 ? split_prefix(tiles, blocks) : tiles; }
 
 cudaError_t launch_split(const float* src, long long ld, int rows, int cols, float* hi, float* lo, long long ldo,
                          const int* info, cudaStream_t st) {
@@ -526,9 +576,17 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
     cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     attr = true;
   }
-  gemm_tf32x3_kernel<<<grid, kThreads, kSmem, st>>>(ah, al, bh, bl, job, b_mn ? 1 : 0, info);
+  // persistent: one CTA per SM at most, fewer when the job leaves SMs to others
+  const int ctas = std::min(grid, job.max_ctas > 0 ? std::min(job.max_ctas, kNumSMs) : kNumSMs);
+  // C comes in by TMA when it is read (beta != 0); otherwise the map is unused
+  CUtensorMap cm = ah;
+  const bool partial = job.mode == 2 && job.nsplit > 0;
+  if (!partial && job.C && job.beta != 0.f &&
+      !make_map_c(&cm, job.C, (long long)job.c_row0 + job.Mlim, (long long)job.c_col0 + job.Nlim, job.ldc))
+    return cudaErrorInvalidValue;
+  gemm_tf32x3_kernel<<<ctas, kThreads, kSmem, st>>>(ah, al, bh, bl, job, cm, b_mn ? 1 : 0, grid, info);
   count_launches(1);
-  if (job.mode == 2 && job.nsplit > 1) {
+  if (job.mode == 2 && job.nsplit > 0) {
     const long long quads = (long long)(job.nblk - 1 - job.s) * (kM * kN / 4);
     const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
     rowsplit_reduce_kernel<<<g, 256, 0, st>>>(job, info);

@@ -19,8 +19,10 @@ struct Operand {
 //  mode 0: dense grid of mt x nt tiles, K = kdim.
 //  mode 1: tiles (i, j), i <= j, enumerated column by column from tile t0, K = kdim.
 //  mode 2: tiles (s, s + 1 + t) for t < nblk - 1 - s (one block row of U),
-//          K = [(s+1)*128, min((s+2+t)*128, dlim)), split into nsplit ranges
-//          whose partials are reduced in order.
+//          K = [(s+1)*128, min((s+2+t)*128, dlim)); with nsplit > 0 that
+//          range is cut into pieces of nsplit blocks (tile t has
+//          floor(t / nsplit) + 1 of them, items in tile order), whose
+//          partials are then reduced in order.
 //  mode 3: tiles (s, s + 1 + t) for t < nblk - 1 - s, K = [s*128, min((s+1)*128, dlim)).
 // A(m, k) is read at (x = a_x0 + k, y = a_y0 + m0 + m); B(k, n) at
 // (x = b_x0 + k, y = b_y0 + n0 + n) if K-major, (x = b_x0 + n0 + n, y = b_y0 + k)
@@ -48,9 +50,13 @@ struct Job {
   int p_col0;
   int planes_one_col, planes_n0;
   float* part;
+  int max_ctas;      // persistent CTAs at most (0: one per SM)
 };
 
 constexpr int kTileTC = 128;
+
+// Items of a mode-2 row of `tiles` tiles split into pieces of `blocks` blocks.
+int row_items(int tiles, int blocks);
 
 cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
                         cudaStream_t st);
