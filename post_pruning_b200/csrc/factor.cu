@@ -171,8 +171,8 @@ __device__ __forceinline__ void unit_dot8(const float* A, const float (&b)[32], 
 // SGPT_INFO_NONFINITE), 0 if every pivot was positive.
 __device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* rinv, int c0, int col0, int lane) {
   // Pivot j: r_jj = sqrt(a_jj), r_ij = a_ij / r_jj (i < j), then
-  // a_il -= r_ij r_lj for l < j. Column j-1 is updated first and the next
-  // pivot is broadcast before the rest of the update is issued. Entries
+  // a_il -= r_ij r_lj for l < j. The next pivot is broadcast before the
+  // rest of the update is issued. Entries
   // below the diagonal (l < i) take the update too but are never read, and
   // are zeroed on output.
   float dr[32];
@@ -187,10 +187,12 @@ __device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* rinv, int
     const float rij = lane < j ? dr[j] * rs : (lane == j ? piv * rs : 0.f);
     dr[j] = rij;
     if (j == 0) break;
-    dr[j - 1] = fmaf(-rij, __shfl_sync(0xffffffffu, rij, j - 1), dr[j - 1]);
-    const float next = __shfl_sync(0xffffffffu, dr[j - 1], j - 1);
+    // lane j-1 forms its next pivot from its own r_{j-1,j} (no shuffle on
+    // the chain), then broadcasts it; the other lanes' updates follow
+    const float own = fmaf(-rij, rij, dr[j - 1]);
+    const float next = __shfl_sync(0xffffffffu, own, j - 1);
 #pragma unroll
-    for (int l = j - 2; l >= 0; --l) dr[l] = fmaf(-rij, __shfl_sync(0xffffffffu, rij, l), dr[l]);
+    for (int l = j - 1; l >= 0; --l) dr[l] = fmaf(-rij, __shfl_sync(0xffffffffu, rij, l), dr[l]);
     piv = next;
   }
 #pragma unroll

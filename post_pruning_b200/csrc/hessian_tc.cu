@@ -136,6 +136,35 @@ __host__ __device__ inline long long band_start(int ti, int tn) {
 
 }  // namespace
 
+// H[i][j] += S[r][c] and, for j != i, H[j][i] += S[r][c] over the upper
+// part (j >= i) of the 64 x 64 block at rows i0.., columns j0.. (S in shared
+// memory, row stride ld). Both passes are coalesced: rows of H along c,
+// then the mirrored rows along r (a column of S).
+constexpr int kSLd = 65;
+constexpr int kTileLd = kN + 1;
+__device__ void flush_block(const float* S, int ld, int i0, int j0, float* __restrict__ H, int d, int t, int nt) {
+  for (int q = t; q < 64 * 16; q += nt) {
+    const int r = q >> 4, c4 = (q & 15) * 4, i = i0 + r;
+    if (i >= d) continue;
+    const long long row = (long long)i * d;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int j = j0 + c4 + x;
+      if (j >= i && j < d) H[row + j] += S[r * ld + c4 + x];
+    }
+  }
+  for (int q = t; q < 64 * 16; q += nt) {
+    const int c = q >> 4, r4 = (q & 15) * 4, j = j0 + c;
+    if (j >= d) continue;
+    const long long row = (long long)j * d;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int i = i0 + r4 + x;
+      if (i < j && i < d) H[row + i] += S[(r4 + x) * ld + c];
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int d, long long n,
     int nsplit, long long per, float* __restrict__ part, int* info) {
@@ -285,32 +314,43 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       float* dst = part + (size_t)blockIdx.x * kM * kN + (size_t)r * kN + h * 128;
 #pragma unroll
       for (int e = 0; e < 128; e += 4) st4(dst + e, make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]));
-    } else if (i < d) {
+    }
+  }
+  if (!skip && !failed && nsplit == 1 && warp >= 2) {
+    // H += tile (and its mirror) through shared memory, by the epilogue
+    // warps (named barrier 1): the whole tile is staged in the stage buffers,
+    // free now that every MMA has completed, then flushed 64 x 64 at a time
+    float* S = reinterpret_cast<float*>(smem);
+    const int et = threadIdx.x - 64;            // epilogue thread 0..255
+    const int r = q * 32 + lane;
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        const int j = j0 + h * 128 + e;
-        if (j < i || j >= d) continue;
-        H[(long long)i * d + j] += acc[e];
-        if (j != i) H[(long long)j * d + i] += acc[e];
-      }
+    for (int e = 0; e < 128; ++e) S[r * kTileLd + h * 128 + e] = acc[e];
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    for (int blk = 0; blk < (kM / 64) * (kN / 64); ++blk) {
+      const int br = blk / (kN / 64), bc = blk % (kN / 64);
+      const int bi0 = i0 + 64 * br, bj0 = j0 + 64 * bc;
+      if (bi0 < d && bj0 < d && bj0 + 63 >= bi0)  // the block meets the upper triangle
+        flush_block(S + (64 * br) * kTileLd + 64 * bc, kTileLd, bi0, bj0, H, d, et, 256);
     }
   }
   __syncthreads();
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-// Split partials -> H: every element of every tile sums its nsplit partials
-// in split order (deterministic) and adds the sum to H[i][j] and H[j][i].
-__global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __restrict__ part,
-                                                             float* __restrict__ H, int d, int tiles,
-                                                             int nsplit, const int* info) {
+// Split partials -> H: one CTA per 64 x 64 block of a tile, one thread per
+// four elements, sums the block's nsplit partials in split order
+// (deterministic; up to eight loads in flight per thread), then adds the sum
+// to H and to its mirror through shared memory.
+constexpr int kReduceThreads = 1024;
+__global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const float* __restrict__ part,
+                                                                        float* __restrict__ H, int d, int tiles,
+                                                                        int nsplit, const int* info) {
   if (cta_info_set(info)) return;
+  __shared__ float S[64 * kSLd];
   const int tn = (d + kN - 1) / kN;
-  const long long quads = (long long)tiles * (kM * kN / 4);
-  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < quads;
-       q += (long long)gridDim.x * blockDim.x) {
-    const int tile = (int)(q / (kM * kN / 4));
-    const int e = (int)(q - (long long)tile * (kM * kN / 4)) * 4;
+  const int t = threadIdx.x, r = t >> 4, c4 = (t & 15) * 4;
+  for (int blk = blockIdx.x; blk < tiles * 8; blk += gridDim.x) {
+    const int tile = blk >> 3, br = (blk & 7) >> 2, bc = blk & 3;
     int ti = 0;
     {
       int lo = 0, hi = (d + kM - 1) / kM - 1;
@@ -322,22 +362,29 @@ __global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __rest
       ti = lo;
     }
     const int tj = ti / 2 + (int)(tile - band_start(ti, tn));
-    const int i = ti * kM + e / kN, j0 = tj * kN + (e % kN);
-    if (i >= d || j0 >= d || j0 + 3 < i) continue;
-    const float* src = part + (size_t)tile * nsplit * kM * kN + e;
+    const int bi0 = ti * kM + 64 * br, bj0 = tj * kN + 64 * bc;
+    if (!(bi0 < d && bj0 < d && bj0 + 63 >= bi0)) continue;   // block-uniform
+    const float* src = part + (size_t)tile * nsplit * kM * kN + (size_t)(64 * br + r) * kN + 64 * bc + c4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = 0; p < nsplit; ++p) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + (size_t)p * kM * kN));
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+    for (int p0 = 0; p0 < nsplit; p0 += 8) {
+      float4 v[8];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int j = j0 + t;
-      if (j < i || j >= d) continue;
-      H[(long long)i * d + j] += a[t];
-      if (j != i) H[(long long)j * d + i] += a[t];
+      for (int pp = 0; pp < 8; ++pp)
+        v[pp] = (p0 + pp < nsplit) ? __ldcs(reinterpret_cast<const float4*>(src + (size_t)(p0 + pp) * kM * kN))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int pp = 0; pp < 8; ++pp)
+        if (p0 + pp < nsplit) {
+          acc.x += v[pp].x; acc.y += v[pp].y; acc.z += v[pp].z; acc.w += v[pp].w;
+        }
     }
+    S[r * kSLd + c4] = acc.x;
+    S[r * kSLd + c4 + 1] = acc.y;
+    S[r * kSLd + c4 + 2] = acc.z;
+    S[r * kSLd + c4 + 3] = acc.w;
+    __syncthreads();
+    flush_block(S, kSLd, bi0, bj0, H, d, t, kReduceThreads);
+    __syncthreads();
   }
 }
 
@@ -416,9 +463,8 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
   hessian_tc_kernel<<<p.tiles * p.nsplit, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info);
   count_launches(1);
   if (p.nsplit > 1) {
-    const long long quads = (long long)p.tiles * (kM * kN / 4);
-    const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
-    hessian_reduce_kernel<<<g, 256, 0, st>>>(part, H, d, p.tiles, p.nsplit, info);
+    const int g = (int)std::min<long long>((long long)p.tiles * 8, 8 * kNumSMs);
+    hessian_reduce_kernel<<<g, kReduceThreads, 0, st>>>(part, H, d, p.tiles, p.nsplit, info);
     count_launches(1);
   }
   return cudaGetLastError();
