@@ -27,8 +27,8 @@ namespace sgpt {
 
 // ---------------------------------------------------------------- sweep
 
-constexpr int kSweepRows = 8;              // rows per CTA, one warp each
-constexpr int kSweepThreads = kSweepRows * 32;
+constexpr int kSweepWarps = 8;             // warps per CTA
+constexpr int kSweepThreads = kSweepWarps * 32;
 constexpr size_t kSweepSmem = (size_t)kMaxBlock * kMaxBlock * sizeof(float);
 
 enum SweepMode { kModeNM24 = 0, kModeThreshold = 1, kModeForced = 2 };
@@ -37,23 +37,30 @@ __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsi
   return ((unsigned long long)__float_as_uint(saliency(w, inv_u)) << 32) | idx;
 }
 
-// One warp per row; lane l owns the block's columns 4l .. 4l+3, i.e. one
-// 4-column group (an N:M group never straddles two lanes). Groups are taken
-// in order. For group g every lane receives lane g's four weights, decides
-// the group's mask (2:4: on the compensated weights, at the group start) and
-// computes its four errors in column order with the in-group updates, all
-// lanes alike; lane g keeps the result and every lane right of it applies
-// the rank-4 update to its four columns. Arithmetically this is the
-// column-by-column sweep with the updates of the four columns to the columns
-// right of the group summed together. The chain per group is one shuffle,
-// the four in-group steps and one rank-4 update; the U values are loaded
-// before the weights arrive.
-template <int MODE>
+// ROWS rows per warp, 32/ROWS lanes per row; lane l of a row owns the
+// 4-column groups l, l + 32/ROWS, ... of its row (an N:M group never
+// straddles two lanes; the interleave keeps every shared-memory row read of
+// the warp contiguous).
+// Groups are taken in order. For group g every lane of the row receives the
+// owner lane's four weights, decides the group's mask (2:4: on the
+// compensated weights, at the group start) and computes its four errors in
+// column order with the in-group updates, all lanes alike; the owner keeps
+// the result and applies the group's update to its own later group, and
+// every lane right of it applies the rank-4 update to its columns.
+// Arithmetically this is the column-by-column sweep with the updates of the
+// four columns to the columns right of the group summed together. The chain
+// per group is one shuffle, the four in-group steps and one rank-4 update;
+// the U values are loaded before the weights arrive. Two rows per warp halve
+// the owner work per row (for tall layers); one row per warp gives more
+// parallelism to short ones.
+template <int MODE, int ROWS>
 __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
     const float* __restrict__ U, uint32_t* __restrict__ mask, float* __restrict__ row_loss,
     float* __restrict__ Err, float* __restrict__ Err_lo, const unsigned long long* __restrict__ thr,
     int* info) {
+  constexpr int LPR = 32 / ROWS;                 // lanes per row
+  constexpr int CPL = 4 * ROWS;                  // columns per lane
   if (cta_info_set(info)) return;
   extern __shared__ float Us[];   // [128][128]: U[i1 + a][i1 + b]
   __shared__ float Uinv[kMaxBlock];   // 1 / U_qq of the block's columns
@@ -71,22 +78,44 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
   if (tid < kMaxBlock) Uinv[tid] = tid < bw ? 1.0f / U[(long long)(i1 + tid) * d + i1 + tid] : 0.f;
 
   const int lane = tid & 31;
-  const int row = blockIdx.x * kSweepRows + (tid >> 5);
+  const int sub = lane / LPR, sl = lane % LPR;   // row within the warp, lane within the row
+  const int base = sub * LPR;                    // first lane of this row
+  const int row = (blockIdx.x * kSweepWarps + (tid >> 5)) * ROWS + sub;
   const int ngroups = bw >> 2;
+  constexpr int SPAN = 4 * LPR;                  // columns between a lane's groups
   const bool live = row < rows;
-  const bool mine = live && lane < ngroups;
-  const int c0 = 4 * lane;                         // block-relative first column
+  const bool mine = live;
+  const int c0 = 4 * sl;                         // block-relative first column of group v: c0 + v * SPAN
   float* wrow = W + (long long)row * ldw + i1 + c0;
-  float w[4] = {0.f, 0.f, 0.f, 0.f}, err[4] = {0.f, 0.f, 0.f, 0.f};
-  if (mine) {
-    const float4 x = ld4(wrow);
-    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+  float w[CPL], err[CPL];
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) {
+    w[j] = 0.f;
+    err[j] = 0.f;
   }
-  bool bad = !(isfinite(w[0]) && isfinite(w[1]) && isfinite(w[2]) && isfinite(w[3]));
-  uint32_t keep = 0xfu;
+  if (mine) {
+#pragma unroll
+    for (int v = 0; v < ROWS; ++v) {
+      if (c0 + v * SPAN < bw) {
+        const float4 x = ld4(wrow + v * SPAN);
+        w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+      }
+    }
+  }
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) bad |= !isfinite(w[j]);
+  uint32_t keep = (1u << CPL) - 1u;
   if (MODE == kModeForced && mine) {
-    const uint32_t word = mask[(long long)row * (d / 32) + (i1 + c0) / 32];
-    keep = (word >> ((i1 + c0) & 31)) & 0xfu;
+    keep = 0;
+#pragma unroll
+    for (int v = 0; v < ROWS; ++v) {
+      const int c = c0 + v * SPAN;
+      if (c < bw) {
+        const uint32_t word = mask[(long long)row * (d / 32) + (i1 + c) / 32];
+        keep |= ((word >> ((i1 + c) & 31)) & 0xfu) << (4 * v);
+      }
+    }
   }
   cp_async_wait_all();
   __syncthreads();
@@ -94,112 +123,158 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     const unsigned long long t = *thr;
     keep = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const unsigned idx = (unsigned)row * (unsigned)bw + (unsigned)(c0 + j);
-      if (sal_key(w[j], Uinv[c0 + j], idx) >= t) keep |= 1u << j;
+    for (int j = 0; j < CPL; ++j) {
+      const int c = c0 + (j >> 2) * SPAN + (j & 3);
+      const unsigned idx = (unsigned)row * (unsigned)bw + (unsigned)c;
+      if (c < bw && sal_key(w[j], Uinv[c], idx) >= t) keep |= 1u << j;
     }
   }
   float loss = 0.f;
-  // keep bit t of every lane, for the threshold and forced modes
-  uint32_t kb[4];
+  // keep bit j of every lane, for the threshold and forced modes
+  uint32_t kb[CPL];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) kb[t] = __ballot_sync(0xffffffffu, (keep >> t) & 1u);
+  for (int j = 0; j < CPL; ++j) kb[j] = __ballot_sync(0xffffffffu, (keep >> j) & 1u);
 
+#pragma unroll
+  for (int gi = 0; gi < ROWS; ++gi) {
+    const int gend = min(LPR, (bw - gi * SPAN) / 4);   // groups of this column span inside the block
 #pragma unroll 1
-  for (int g = 0; g < ngroups; ++g) {
-    const int q0 = 4 * g;
-    // everything that does not depend on the weights first: the owner's
-    // four rows of U at this lane's columns, its in-group entries and the
-    // reciprocal diagonal
-    const float4 u0 = ld4(Us + (q0 + 0) * kMaxBlock + c0);
-    const float4 u1 = ld4(Us + (q0 + 1) * kMaxBlock + c0);
-    const float4 u2 = ld4(Us + (q0 + 2) * kMaxBlock + c0);
-    const float4 u3 = ld4(Us + (q0 + 3) * kMaxBlock + c0);
-    const float4 g0 = ld4(Us + (q0 + 0) * kMaxBlock + q0);
-    const float4 g1 = ld4(Us + (q0 + 1) * kMaxBlock + q0);
-    const float4 g2 = ld4(Us + (q0 + 2) * kMaxBlock + q0);
-    const float4 ri = ld4(Uinv + q0);
-    // every lane takes the owner's weights and computes its group the same
-    // way, so no lane waits for a second broadcast
-    float wo[4];
+    for (int gp = 0; gp < gend; ++gp) {
+      const int q0 = gi * SPAN + 4 * gp;         // the group's first column (group order = column order)
+      const int owner = base + gp;
+      // U values that do not depend on the weights first: the group's four
+      // rows at this lane's columns, its in-group entries, the reciprocals
+      float4 ur[4][ROWS];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) wo[t] = __shfl_sync(0xffffffffu, w[t], g);
-    const float r[4] = {ri.x, ri.y, ri.z, ri.w};
-    uint32_t km;
-    if (MODE == kModeNM24) {
-      // 2 of 4 on the compensated weights; ties keep the lower column.
-      float sl[4];
+      for (int t = 0; t < 4; ++t)
 #pragma unroll
-      for (int t = 0; t < 4; ++t) sl[t] = saliency(wo[t], r[t]);
-      km = 0;
+        for (int v = 0; v < ROWS; ++v)
+          ur[t][v] = (v >= gi) ? ld4(Us + (q0 + t) * kMaxBlock + c0 + v * SPAN) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 g0 = ld4(Us + (q0 + 0) * kMaxBlock + q0);
+      const float4 g1 = ld4(Us + (q0 + 1) * kMaxBlock + q0);
+      const float4 g2 = ld4(Us + (q0 + 2) * kMaxBlock + q0);
+      const float4 ri = ld4(Uinv + q0);
+      float wo[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        int rank = 0;   // how many of the group beat column t
+      for (int t = 0; t < 4; ++t) wo[t] = __shfl_sync(0xffffffffu, w[4 * gi + t], owner);
+      const float r[4] = {ri.x, ri.y, ri.z, ri.w};
+      uint32_t km;
+      if (MODE == kModeNM24) {
+        // 2 of 4 on the compensated weights; ties keep the lower column.
+        float slv[4];
 #pragma unroll
-        for (int o = 0; o < 4; ++o)
-          if (o != t && (sl[o] > sl[t] || (sl[o] == sl[t] && o < t))) ++rank;
-        if (rank < 2) km |= 1u << t;
+        for (int t = 0; t < 4; ++t) slv[t] = saliency(wo[t], r[t]);
+        km = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          int rank = 0;   // how many of the group beat column t
+#pragma unroll
+          for (int o = 0; o < 4; ++o)
+            if (o != t && (slv[o] > slv[t] || (slv[o] == slv[t] && o < t))) ++rank;
+          if (rank < 2) km |= 1u << t;
+        }
+      } else {
+        km = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) km |= ((kb[4 * gi + t] >> owner) & 1u) << t;
       }
-    } else {
-      km = ((kb[0] >> g) & 1u) | (((kb[1] >> g) & 1u) << 1) | (((kb[2] >> g) & 1u) << 2) | (((kb[3] >> g) & 1u) << 3);
-    }
-    float e[4];
-    e[0] = (km & 1u) ? 0.f : __fmul_rn(wo[0], r[0]);
-    wo[1] = fmaf(-e[0], g0.y, wo[1]);
-    wo[2] = fmaf(-e[0], g0.z, wo[2]);
-    wo[3] = fmaf(-e[0], g0.w, wo[3]);
-    e[1] = (km & 2u) ? 0.f : __fmul_rn(wo[1], r[1]);
-    wo[2] = fmaf(-e[1], g1.z, wo[2]);
-    wo[3] = fmaf(-e[1], g1.w, wo[3]);
-    e[2] = (km & 4u) ? 0.f : __fmul_rn(wo[2], r[2]);
-    wo[3] = fmaf(-e[2], g2.w, wo[3]);
-    e[3] = (km & 8u) ? 0.f : __fmul_rn(wo[3], r[3]);
-    if (lane == g) {
-      // the owner keeps its group's result
+      float e[4];
+      e[0] = (km & 1u) ? 0.f : __fmul_rn(wo[0], r[0]);
+      wo[1] = fmaf(-e[0], g0.y, wo[1]);
+      wo[2] = fmaf(-e[0], g0.z, wo[2]);
+      wo[3] = fmaf(-e[0], g0.w, wo[3]);
+      e[1] = (km & 2u) ? 0.f : __fmul_rn(wo[1], r[1]);
+      wo[2] = fmaf(-e[1], g1.z, wo[2]);
+      wo[3] = fmaf(-e[1], g1.w, wo[3]);
+      e[2] = (km & 4u) ? 0.f : __fmul_rn(wo[2], r[2]);
+      wo[3] = fmaf(-e[2], g2.w, wo[3]);
+      e[3] = (km & 8u) ? 0.f : __fmul_rn(wo[3], r[3]);
+      if (sl == gp) {
+        // the owner keeps its group's result
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        w[t] = ((km >> t) & 1u) ? wo[t] : 0.f;
-        err[t] = e[t];
-        loss = fmaf(e[t], e[t], loss);
+        for (int t = 0; t < 4; ++t) {
+          w[4 * gi + t] = ((km >> t) & 1u) ? wo[t] : 0.f;
+          err[4 * gi + t] = e[t];
+          loss = fmaf(e[t], e[t], loss);
+        }
+        keep = (keep & ~(0xfu << (4 * gi))) | (km << (4 * gi));
       }
-      keep = km;
-    } else if (lane > g) {
-      w[0] = fmaf(-e[3], u3.x, fmaf(-e[2], u2.x, fmaf(-e[1], u1.x, fmaf(-e[0], u0.x, w[0]))));
-      w[1] = fmaf(-e[3], u3.y, fmaf(-e[2], u2.y, fmaf(-e[1], u1.y, fmaf(-e[0], u0.y, w[1]))));
-      w[2] = fmaf(-e[3], u3.z, fmaf(-e[2], u2.z, fmaf(-e[1], u1.z, fmaf(-e[0], u0.z, w[2]))));
-      w[3] = fmaf(-e[3], u3.w, fmaf(-e[2], u2.w, fmaf(-e[1], u1.w, fmaf(-e[0], u0.w, w[3]))));
+      // the rank-4 update of every column right of the group: this lane's
+      // later groups (v > gi) always, group gi if the lane is right of the owner
+#pragma unroll
+      for (int v = 0; v < ROWS; ++v) {
+        if (v > gi || (v == gi && sl > gp)) {
+          w[4 * v + 0] = fmaf(-e[3], ur[3][v].x, fmaf(-e[2], ur[2][v].x, fmaf(-e[1], ur[1][v].x, fmaf(-e[0], ur[0][v].x, w[4 * v + 0]))));
+          w[4 * v + 1] = fmaf(-e[3], ur[3][v].y, fmaf(-e[2], ur[2][v].y, fmaf(-e[1], ur[1][v].y, fmaf(-e[0], ur[0][v].y, w[4 * v + 1]))));
+          w[4 * v + 2] = fmaf(-e[3], ur[3][v].z, fmaf(-e[2], ur[2][v].z, fmaf(-e[1], ur[1][v].z, fmaf(-e[0], ur[0][v].z, w[4 * v + 2]))));
+          w[4 * v + 3] = fmaf(-e[3], ur[3][v].w, fmaf(-e[2], ur[2][v].w, fmaf(-e[1], ur[1][v].w, fmaf(-e[0], ur[0][v].w, w[4 * v + 3]))));
+        }
+      }
     }
   }
 
-  // Loss of the row: sum over the warp.
+  // Loss of the row: sum over its lanes.
   float tot = loss;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  for (int o = 1; o < LPR; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
   bad |= !isfinite(tot);
-  // Mask words: lanes 8m .. 8m+7 make the word of columns 32m .. 32m+31.
-  uint32_t bits = mine ? (keep & 0xfu) << (4 * (lane & 7)) : 0u;
-  bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
-  bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
-  bits |= __shfl_xor_sync(0xffffffffu, bits, 4);
-  if (mine) {
-    st4(wrow, make_float4(w[0], w[1], w[2], w[3]));
-    float* erow = Err + (long long)row * kMaxBlock + c0;
-    if (Err_lo) {
-      // hi/lo planes for the tensor-core trailing update
-      float lo[4];
+  // Mask words: for each of its groups v, lanes 8m .. 8m+7 of a row hold the
+  // columns of word (v * SPAN) / 32 + m.
+  uint32_t bits[ROWS];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float h = tf32_hi(err[j]);
-        lo[j] = err[j] - h;
-        err[j] = h;
+  for (int v = 0; v < ROWS; ++v) {
+    bits[v] = mine ? ((keep >> (4 * v)) & 0xfu) << (4 * (sl & 7)) : 0u;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) bits[v] |= __shfl_xor_sync(0xffffffffu, bits[v], o);
+  }
+  if (mine) {
+#pragma unroll
+    for (int v = 0; v < ROWS; ++v) {
+      const int c = c0 + v * SPAN;
+      if (c >= bw) continue;
+      st4(wrow + v * SPAN, make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]));
+      float ev[4] = {err[4 * v], err[4 * v + 1], err[4 * v + 2], err[4 * v + 3]};
+      if (Err_lo) {
+        // hi/lo planes for the tensor-core trailing update
+        float lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float h = tf32_hi(ev[j]);
+          lo[j] = ev[j] - h;
+          ev[j] = h;
+        }
+        st4(Err_lo + (long long)row * kMaxBlock + c, make_float4(lo[0], lo[1], lo[2], lo[3]));
       }
-      st4(Err_lo + (long long)row * kMaxBlock + c0, make_float4(lo[0], lo[1], lo[2], lo[3]));
+      st4(Err + (long long)row * kMaxBlock + c, make_float4(ev[0], ev[1], ev[2], ev[3]));
+      if (MODE != kModeForced && (sl & 7) == 0) mask[(long long)row * (d / 32) + (i1 + c) / 32] = bits[v];
     }
-    st4(erow, make_float4(err[0], err[1], err[2], err[3]));
-    if (MODE != kModeForced && (lane & 7) == 0) mask[(long long)row * (d / 32) + (i1 + c0) / 32] = bits;
-    if (lane == 0 && row_loss) row_loss[row] += tot;
+    if (sl == 0 && row_loss) row_loss[row] += tot;
     if (bad) set_info(info, SGPT_INFO_NONFINITE);
   }
+}
+
+// Rows per warp for a layer: two for tall layers (halves the instructions
+// per row), one for short ones (twice the warps in flight).
+static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 2 : 1; }
+
+template <int MODE>
+static void launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
+                         uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
+                         const unsigned long long* thr, int* info, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaFuncSetAttribute(sweep_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    cudaFuncSetAttribute(sweep_kernel<MODE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    attr_done = true;
+  }
+  const int grid = cdiv(rows, kSweepWarps * rpw);
+  if (rpw == 2)
+    sweep_kernel<MODE, 2><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
+                                                                   Err_lo, thr, info);
+  else
+    sweep_kernel<MODE, 1><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
+                                                                   Err_lo, thr, info);
+  count_launches(1);
 }
 
 // --------------------------------------------------------- trailing update
@@ -416,36 +491,24 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
                          const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
                          int* info, cudaStream_t st) {
   const PruneWs w = carve_prune(ws, rows, d, nullptr);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(sweep_kernel<kModeNM24>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    cudaFuncSetAttribute(sweep_kernel<kModeThreshold>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    cudaFuncSetAttribute(sweep_kernel<kModeForced>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    attr_done = true;
-  }
   cudaError_t e = tc::launch_split(U, d, d, d, w.U_hi, w.U_lo, d, info, st);
   if (e != cudaSuccess) return e;
   const tc::Operand Ep{w.Err_hi, w.Err_lo, rows, kMaxBlock, kMaxBlock};
   const tc::Operand Up{w.U_hi, w.U_lo, d, d, d};
   const int B = p.blocksize;
-  const int sweep_grid = cdiv(rows, kSweepRows);
+  const int rpw = sweep_rows_per_warp(rows);
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
     if (p.forced) {
-      sweep_kernel<kModeForced><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info);
-      count_launches(1);
+      launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info, st);
     } else if (p.pattern == SGPT_PATTERN_NM) {
-      sweep_kernel<kModeNM24><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info);
-      count_launches(1);
+      launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info, st);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
-      sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, info);
-      count_launches(1);
+      launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr,
+                                   info, st);
     }
     const int i2 = i1 + bw;
     if (i2 < d) {
@@ -517,32 +580,19 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
   if (e != cudaSuccess) return e;
   float* Err = static_cast<float*>(base);
   SelState* sel = reinterpret_cast<SelState*>(static_cast<char*>(base) + kNoAllocErrBytes);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(sweep_kernel<kModeNM24>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    cudaFuncSetAttribute(sweep_kernel<kModeThreshold>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    cudaFuncSetAttribute(sweep_kernel<kModeForced>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    attr_done = true;
-  }
   const int B = p.blocksize;
-  const int sweep_grid = cdiv(rows, kSweepRows);
+  const int rpw = sweep_rows_per_warp(rows);
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
     if (p.forced) {
-      sweep_kernel<kModeForced><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info);
-      count_launches(1);
+      launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info, st);
     } else if (p.pattern == SGPT_PATTERN_NM) {
-      sweep_kernel<kModeNM24><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info);
-      count_launches(1);
+      launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info, st);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
-      sweep_kernel<kModeThreshold><<<sweep_grid, kSweepThreads, kSweepSmem, st>>>(
-          W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info);
-      count_launches(1);
+      launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info, st);
     }
     const int i2 = i1 + bw;
     if (i2 < d) {
