@@ -305,7 +305,7 @@ struct SelState {
   unsigned int hist[8][256];   // one histogram per digit pass
 };
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 1024;
 constexpr long long kGridWaitCycles = 2000000000ll;
 
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
@@ -344,12 +344,15 @@ __device__ bool grid_sync(unsigned int* ctr, unsigned int target, int* info, int
 // that match the prefix fixed so far; after a grid barrier every CTA scans
 // the same global histogram and takes the same decision, so a pass needs one
 // barrier. It stops as soon as the rank falls on a whole bin (usually after
-// the saliency passes). st must be zeroed before the launch; CTA 0 writes
-// the threshold.
+// the saliency passes). The first pass scores the weights and keeps each
+// CTA's saliency bits in shared memory for the later passes (when they fit;
+// otherwise every pass rescores W); the index of quad e's element j is
+// 4e + j. st must be zeroed before the launch; CTA 0 writes the threshold.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
-    const float* __restrict__ U, SelState* st, unsigned int k, int* info) {
+    const float* __restrict__ U, SelState* st, unsigned int k, int keep_bits, int* info) {
   if (cta_info_set(info)) return;
+  extern __shared__ unsigned int skey[];        // this CTA's saliency bits, if keep_bits
   __shared__ unsigned int h[256];
   __shared__ float ud[kMaxBlock];
   __shared__ unsigned int wsum[kSelThreads / 32];
@@ -365,7 +368,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     s_failed = 0;
   }
   const long long total4 = (long long)rows * (bw / 4);
-  unsigned long long thr = 0;
   for (int pass = 0; pass < 8; ++pass) {
     if (t < 256) h[t] = 0;
     __syncthreads();
@@ -373,22 +375,30 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const int shift = 56 - 8 * pass;
     const unsigned long long prefix = s_prefix;
     // trip count uniform across the CTA: every lane takes part in the match
+    int it = 0;
     for (long long base = (long long)blockIdx.x * kSelThreads; base < total4;
-         base += (long long)gridDim.x * kSelThreads) {
+         base += (long long)gridDim.x * kSelThreads, ++it) {
       const long long e = base + t;
       const bool act = e < total4;
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      int row = 0, c = 0;
+      unsigned int sb[4] = {0u, 0u, 0u, 0u};
       if (act) {
-        row = (int)(e / (bw / 4));
-        c = (int)(e - (long long)row * (bw / 4)) * 4;
-        const float4 x = ld4(W + (long long)row * ldw + i1 + c);
-        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        if (pass > 0 && keep_bits) {
+          const uint4 x = *reinterpret_cast<const uint4*>(skey + 4 * (it * kSelThreads + t));
+          sb[0] = x.x; sb[1] = x.y; sb[2] = x.z; sb[3] = x.w;
+        } else {
+          const int row = (int)(e / (bw / 4));
+          const int c = (int)(e - (long long)row * (bw / 4)) * 4;
+          const float4 x = ld4(W + (long long)row * ldw + i1 + c);
+          const float v[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sb[j] = (unsigned int)(sal_key(v[j], ud[c + j], 0u) >> 32);
+          if (pass == 0 && keep_bits)
+            *reinterpret_cast<uint4*>(skey + 4 * (it * kSelThreads + t)) = make_uint4(sb[0], sb[1], sb[2], sb[3]);
+        }
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const unsigned long long key =
-            act ? sal_key(v[j], ud[c + j], (unsigned)row * (unsigned)bw + (unsigned)(c + j)) : 0ull;
+        const unsigned long long key = act ? (((unsigned long long)sb[j] << 32) | (unsigned long long)(4 * e + j)) : 0ull;
         const bool mine = act && (pass == 0 || (key >> (shift + 8)) == prefix);
         // saliencies span a narrow exponent range, so a warp holds few
         // distinct digits: one shared atomic per digit and warp
@@ -421,40 +431,49 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       s_krem = krem;
       if (cnt == krem) {
         s_done = 1;
-        thr = (pre << shift) + (1ull << shift);   // every key of the bin is pruned
-        if (blockIdx.x == 0) st->thr = thr;
+        if (blockIdx.x == 0) st->thr = (pre << shift) + (1ull << shift);   // every key of the bin is pruned
       }
     }
     __syncthreads();
   }
 }
 
+constexpr int kSelMaxSmem = 160 * 1024;         // bytes of saliency bits a CTA keeps
+
 static cudaError_t launch_select(const float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
                                  SelState* sel, unsigned int k, int* info, cudaStream_t st) {
   static int max_grid = 0;
   cudaError_t e = cudaSuccess;
   if (!max_grid) {
+    if ((e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxSmem)) !=
+        cudaSuccess)
+      return e;
     int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kSelThreads, 0)) != cudaSuccess)
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kSelThreads, kSelMaxSmem)) !=
+        cudaSuccess)
       return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    max_grid = std::max(1, std::min(per_sm, 2) * sms);
+    max_grid = std::max(1, std::min(per_sm, 1) * sms);   // one CTA per SM: fewer histogram merges
   }
   if ((e = cudaMemsetAsync(sel, 0, sizeof(SelState), st)) != cudaSuccess) return e;
   const long long total4 = (long long)rows * (bw / 4);
   const int grid = (int)std::max<long long>(1, std::min<long long>(cdivll(total4, kSelThreads), max_grid));
+  const long long iters = cdivll(total4, (long long)grid * kSelThreads);
+  const long long bytes = iters * kSelThreads * 16;
+  const int keep_bits = bytes <= kSelMaxSmem ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = keep_bits ? (size_t)bytes : 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, select_kernel, W, ldw, rows, d, i1, bw, U, sel, k, info);
+  e = cudaLaunchKernelEx(&cfg, select_kernel, W, ldw, rows, d, i1, bw, U, sel, k, keep_bits, info);
   count_launches(1);
   return e;
 }
