@@ -513,20 +513,29 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
       job.C_lo = w.V_lo;
       if ((e = tc::launch_gemm(A, B, false, job, k, info, f.crit)) != cudaSuccess) return e;
     }
-    // rank-bk update A_ij -= R_ik R_jk^T of the leading upper tiles: column
-    // block k-1 on the chain (its tiles also write the planes the next panel
-    // reads), the tiles left of it on `upd`, after the previous step's
-    if (upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
-    const tc::Operand P{w.R + c0, w.V_lo + c0, c0, bk, d};
+    // Rank updates A_ij -= R_ik R_jk^T of the leading upper tiles, by pairs
+    // of block columns (k, k-1): the first of a pair updates only column
+    // block k-1 (on the chain; its tiles also write the planes the next
+    // panel reads); the second updates column block k-2 with both panels
+    // (K = 256, on the chain) and the tiles left of it with both panels on
+    // `upd`, so that the bulk of the trailing matrix is read and written once
+    // per two block columns. The chain waits for the previous bulk update
+    // before it touches tiles that update also wrote.
+    const bool second = ((K - 1 - k) & 1) != 0;  // k is the second block of its pair
+    // K of this step's updates: panel k, or panels k and k+1 (the last block
+    // may be narrower than 128)
+    const int kp = second ? std::min(2 * kTile, d - c0) : bk;
+    if (!second && upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
+    const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
     tc::Job job{};
     job.mode = 1;
-    job.kdim = bk;
+    job.kdim = kp;
     job.C = w.R;
     job.ldc = d;
     job.Mlim = job.Nlim = c0;
     job.alpha = -1.f;
     job.beta = 1.f;
-    if (k >= 2) {
+    if (second && k >= 2) {
       if ((e = after(f.upd, f.crit, f.panel_done)) != cudaSuccess) return e;
       job.max_ctas = kOffChainCtas;
       if ((e = tc::launch_gemm(P, P, false, job, (k - 1) * k / 2, info, f.upd)) != cudaSuccess) return e;
