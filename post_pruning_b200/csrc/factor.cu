@@ -448,6 +448,8 @@ cudaError_t after(cudaStream_t s2, cudaStream_t s1, cudaEvent_t ev) {
 // Off-chain GEMMs are persistent kernels that would otherwise hold every SM
 // for their whole duration; they leave some to the chain's launches.
 constexpr int kOffChainCtas = kNumSMs - 16;
+// Block columns from which the trailing updates go by pairs.
+constexpr int kPairFrom = 16;
 
 // The block-column loop and the V / U block rows (see the file comment).
 cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const FactorStreams& f) {
@@ -521,11 +523,16 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
     // `upd`, so that the bulk of the trailing matrix is read and written once
     // per two block columns. The chain waits for the previous bulk update
     // before it touches tiles that update also wrote.
-    const bool second = ((K - 1 - k) & 1) != 0;  // k is the second block of its pair
+    // (pairs only pay off for wide matrices: for a few blocks the longer
+    // column update on the chain costs more than the bulk traffic saved)
+    const bool paired = K >= kPairFrom;
+    const bool second = paired && ((K - 1 - k) & 1) != 0;   // k is the second block of its pair
     // K of this step's updates: panel k, or panels k and k+1 (the last block
     // may be narrower than 128)
     const int kp = second ? std::min(2 * kTile, d - c0) : bk;
     if (!second && upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
+    // (unpaired: every step updates column block k-1 on the chain and the
+    // tiles left of it on `upd`, with panel k alone)
     const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
     tc::Job job{};
     job.mode = 1;
@@ -535,7 +542,7 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
     job.Mlim = job.Nlim = c0;
     job.alpha = -1.f;
     job.beta = 1.f;
-    if (second && k >= 2) {
+    if ((second || !paired) && k >= 2) {
       if ((e = after(f.upd, f.crit, f.panel_done)) != cudaSuccess) return e;
       job.max_ctas = kOffChainCtas;
       if ((e = tc::launch_gemm(P, P, false, job, (k - 1) * k / 2, info, f.upd)) != cudaSuccess) return e;
