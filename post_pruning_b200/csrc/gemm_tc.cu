@@ -89,6 +89,18 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
+// 16-byte shared-memory accesses by 32-bit shared address (the epilogue
+// tile's address is computed by aligning an integer, which the compiler can
+// no longer see as shared memory).
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts4(uint32_t addr, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -228,6 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
   const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16, cfull = tfull0 + 32;
   if (threadIdx.x == 0) {
+    // descriptors into the TMA unit's cache before the first copy needs them
+    const CUtensorMap* maps[5] = {&a_hi, &a_lo, &b_hi, &b_lo, &c_map};
+    for (int i = 0; i < 5; ++i)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(maps[i])) : "memory");
     failed = 0;
     for (int st = 0; st < kStages; ++st) {
       mbar_init(full0 + 8 * st, 1);
@@ -345,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
     const bool read_c = !partial && job.C != nullptr && job.beta != 0.f;
     const long long ldp = job.ldp ? job.ldp : job.ldc;
     const bool issuer = (warp == 2 && lane == 0);
+    const uint32_t t_s = smem_u32(T);             // the epilogue tile as a shared address
     auto load_c = [&](int ww) {                   // TMA of item ww's C tile (four 32-column groups)
       const Item nx = decode_item(job, ww);
       mbar_expect_tx(cfull, (uint32_t)kStagingBytes);
@@ -386,14 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
 #pragma unroll
       for (int cj = 0; cj < 16; ++cj) {
         const int g4 = 2 * h + (cj >> 3), j = cj & 7;
-        float4* pch = reinterpret_cast<float4*>(T + g4 * (kM * 128) + m * 128 + ((j ^ (m & 7)) << 4));
+        const uint32_t pch = t_s + g4 * (kM * 128) + m * 128 + ((j ^ (m & 7)) << 4);
         float4 o = make_float4(acc[4 * cj], acc[4 * cj + 1], acc[4 * cj + 2], acc[4 * cj + 3]);
         if (!partial) {
-          const float4 cv = read_c ? *pch : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 cv = read_c ? lds4(pch) : make_float4(0.f, 0.f, 0.f, 0.f);
           o = make_float4(fmaf(job.alpha, o.x, job.beta * cv.x), fmaf(job.alpha, o.y, job.beta * cv.y),
                           fmaf(job.alpha, o.z, job.beta * cv.z), fmaf(job.alpha, o.w, job.beta * cv.w));
         }
-        *pch = o;
+        sts4(pch, o);
       }
       asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
       if (!failed) {
@@ -404,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
 #pragma unroll 4
         for (int x = 0; x < 16; ++x) {
           const int mr = ew * 16 + x;
-          const float4 o = *reinterpret_cast<const float4*>(T + g4 * (kM * 128) + mr * 128 + ((j ^ (mr & 7)) << 4));
+          const float4 o = lds4(t_s + g4 * (kM * 128) + mr * 128 + ((j ^ (mr & 7)) << 4));
           if (partial) {
             st4(job.part + (size_t)w * kM * kN + (size_t)mr * kN + cn, o);
             continue;

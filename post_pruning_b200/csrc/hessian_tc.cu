@@ -142,7 +142,14 @@ __host__ __device__ inline long long band_start(int ti, int tn) {
 // then the mirrored rows along r (a column of S).
 constexpr int kSLd = 65;
 constexpr int kTileLd = kN + 1;
-__device__ void flush_block(const float* S, int ld, int i0, int j0, float* __restrict__ H, int d, int t, int nt) {
+__device__ __forceinline__ float lds1(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+// (S is a 32-bit shared-memory address: the staging area may have been
+// aligned through an integer, which hides its address space from the compiler)
+__device__ void flush_block(uint32_t S, int ld, int i0, int j0, float* __restrict__ H, int d, int t, int nt) {
   for (int q = t; q < 64 * 16; q += nt) {
     const int r = q >> 4, c4 = (q & 15) * 4, i = i0 + r;
     if (i >= d) continue;
@@ -150,7 +157,7 @@ __device__ void flush_block(const float* S, int ld, int i0, int j0, float* __res
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       const int j = j0 + c4 + x;
-      if (j >= i && j < d) H[row + j] += S[r * ld + c4 + x];
+      if (j >= i && j < d) H[row + j] += lds1(S + 4u * (uint32_t)(r * ld + c4 + x));
     }
   }
   for (int q = t; q < 64 * 16; q += nt) {
@@ -160,7 +167,7 @@ __device__ void flush_block(const float* S, int ld, int i0, int j0, float* __res
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
       const int i = i0 + r4 + x;
-      if (i < j && i < d) H[row + i] += S[(r4 + x) * ld + c];
+      if (i < j && i < d) H[row + i] += lds1(S + 4u * (uint32_t)((r4 + x) * ld + c));
     }
   }
 }
@@ -201,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16;
 
   if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
     failed = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -320,17 +328,18 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     // H += tile (and its mirror) through shared memory, by the epilogue
     // warps (named barrier 1): the whole tile is staged in the stage buffers,
     // free now that every MMA has completed, then flushed 64 x 64 at a time
-    float* S = reinterpret_cast<float*>(smem);
+    const uint32_t S = smem_u32(smem);
     const int et = threadIdx.x - 64;            // epilogue thread 0..255
     const int r = q * 32 + lane;
 #pragma unroll
-    for (int e = 0; e < 128; ++e) S[r * kTileLd + h * 128 + e] = acc[e];
+    for (int e = 0; e < 128; ++e)
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(S + 4u * (uint32_t)(r * kTileLd + h * 128 + e)), "f"(acc[e]) : "memory");
     asm volatile("bar.sync 1, 256;" ::: "memory");
     for (int blk = 0; blk < (kM / 64) * (kN / 64); ++blk) {
       const int br = blk / (kN / 64), bc = blk % (kN / 64);
       const int bi0 = i0 + 64 * br, bj0 = j0 + 64 * bc;
       if (bi0 < d && bj0 < d && bj0 + 63 >= bi0)  // the block meets the upper triangle
-        flush_block(S + (64 * br) * kTileLd + 64 * bc, kTileLd, bi0, bj0, H, d, et, 256);
+        flush_block(S + 4u * (uint32_t)((64 * br) * kTileLd + 64 * bc), kTileLd, bi0, bj0, H, d, et, 256);
     }
   }
   __syncthreads();
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const fl
     S[r * kSLd + c4 + 2] = acc.z;
     S[r * kSLd + c4 + 3] = acc.w;
     __syncthreads();
-    flush_block(S, kSLd, bi0, bj0, H, d, t, kReduceThreads);
+    flush_block(smem_u32(S), kSLd, bi0, bj0, H, d, t, kReduceThreads);
     __syncthreads();
   }
 }
