@@ -6,6 +6,8 @@ all rows; the GPU runs the whole layer from X through the C ABI. Slow: the
 oracle's Hessian alone is 4e13 float64 flops on the host.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -17,6 +19,11 @@ from workloads import CONFIGS, bf16_bits_to_f64, gen_activations, gen_weights
 from parity import assert_parity, compare, gpu_prune_layer
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+# The two largest Qwen groups take 3 and 5 minutes of host time for the
+# oracle alone; they run when SGPT_LONG_TESTS=1.
+long_test = pytest.mark.skipif(os.environ.get("SGPT_LONG_TESTS") != "1",
+                               reason="oracle takes minutes; set SGPT_LONG_TESTS=1")
 
 
 def _oracle_h(X: torch.Tensor) -> np.ndarray:
@@ -91,12 +98,13 @@ def _qwen_group(x_key):
         assert_parity(m, p)
 
 
-@pytest.mark.parametrize("x_key", [0, 1, 2], ids=["qkv", "o", "gate_up"])
+@pytest.mark.parametrize("x_key", [0, 1, pytest.param(2, marks=long_test)], ids=["qkv", "o", "gate_up"])
 def test_qwen3_block_shared_hessian(x_key):
     """q/k/v share one H and U, o has its own, gate/up share one."""
     _qwen_group(x_key)
 
 
+@long_test
 def test_qwen3_block_down_proj():
     """d_in = 25,600: the oracle's Hessian alone is ~9e13 float64 flops."""
     _qwen_group(3)
