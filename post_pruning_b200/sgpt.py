@@ -425,13 +425,16 @@ class HostPruner:
             b += self.values_out.numel() * 4 + self.meta_out.numel() * 4
         return b
 
-    def enqueue(self, W_host: torch.Tensor, X_host: torch.Tensor | None, params: Params, stream=None):
-        """Copies and pruning, all asynchronous; X_host None reuses the X on
-        the device from the previous call."""
+    def enqueue(self, W_host: torch.Tensor, X_host: torch.Tensor | None, params: Params, stream=None,
+                X_device: torch.Tensor | None = None):
+        """Copies and pruning, all asynchronous. X_host None reuses the X on
+        the device from the previous call; X_device prunes from an X already
+        on the device (for example another pruner's, when several layers read
+        the same input)."""
         self.W.copy_(W_host, non_blocking=True)
-        if X_host is not None:
+        if X_device is None and X_host is not None:
             self.X.copy_(X_host, non_blocking=True)
-        self.bufs.run(self.W, self.X, params, stream=stream)
+        self.bufs.run(self.W, self.X if X_device is None else X_device, params, stream=stream)
         self.W_out.copy_(self.W, non_blocking=True)
         self.mask_out.copy_(self.bufs.mask, non_blocking=True)
         if params.is_nm:
