@@ -8,7 +8,9 @@
 // only those tiles are computed, and every element i <= j is written to both
 // H[i][j] and H[j][i]). Tokens are split across CTAs when there are too few
 // tiles to fill the GPU; split partials are summed in split order
-// by a separate reduction kernel (deterministic).
+// by a separate reduction kernel (deterministic). Tiles are numbered in
+// super-blocks of 2048 x 2048 channels so that the CTAs resident together
+// share most of the columns of X they stream (L2 reuse).
 //
 // Per CTA: warp 0 lane 0 streams 64-token stages with TMA (128-byte swizzle,
 // one box = 64 tokens x 64 channels), warp 1 lane 0 issues
@@ -127,11 +129,47 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[3
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Tiles meeting the upper triangle, band by band: band ti (rows ti*128..)
-// holds the 256-wide column tiles tj >= ti/2, so it starts at tile
-// ti*tn - floor(ti/2)*floor((ti-1)/2).
+// Number of tiles meeting the upper triangle in the first ti row tiles: row
+// tile ti (rows ti*128..) meets the 256-wide column tiles tj >= ti/2, so
+// this is ti*tn - floor(ti/2)*floor((ti-1)/2).
 __host__ __device__ inline long long band_start(int ti, int tn) {
   return (long long)ti * tn - (long long)(ti / 2) * ((ti - 1) / 2);
+}
+
+// Tiles meeting the upper triangle in super-blocks of 2G row tiles by G
+// column tiles (G*256 channels each way), super-block rows in order and, in
+// each, the diagonal super-block first; tiles row by row inside a
+// super-block. CTAs that run together then read a few thousand channels of X
+// rather than all of them.
+constexpr int kGroup = 8;
+__host__ __device__ inline void grouped_tile(long long t, int tm, int tn, int& ti, int& tj) {
+  const int G = kGroup;
+  for (int I = 0;; ++I) {
+    const int r0 = 2 * G * I, nr = (r0 + 2 * G < tm ? r0 + 2 * G : tm) - r0;
+    const int c_hi = G * (I + 1) < tn ? G * (I + 1) : tn;
+    long long diag = 0;
+    for (int r = r0; r < r0 + nr; ++r) diag += c_hi - r / 2;
+    if (t < diag) {
+      int r = r0;
+      while (t >= c_hi - r / 2) { t -= c_hi - r / 2; ++r; }
+      ti = r;
+      tj = r / 2 + (int)t;
+      return;
+    }
+    t -= diag;
+    const long long rest = (long long)nr * (tn - c_hi > 0 ? tn - c_hi : 0);
+    if (t < rest || r0 + nr >= tm) {
+      const long long per_sb = (long long)nr * G;
+      const int k = (int)(t / per_sb);
+      const int w = (int)(t - (long long)k * per_sb);
+      const int c0 = c_hi + k * G;
+      const int nc = tn - c0 < G ? tn - c0 : G;
+      ti = r0 + w / nc;
+      tj = c0 + w % nc;
+      return;
+    }
+    t -= rest;
+  }
 }
 
 }  // namespace
@@ -184,19 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x / nsplit, split = blockIdx.x - (blockIdx.x / nsplit) * nsplit;
-  // tile -> (band ti, column tile tj)
-  const int tn = (d + kN - 1) / kN;
-  int ti = 0;
-  {
-    int lo = 0, hi = (d + kM - 1) / kM - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (band_start(mid, tn) <= tile) lo = mid;
-      else hi = mid - 1;
-    }
-    ti = lo;
-  }
-  const int tj = ti / 2 + (int)(tile - band_start(ti, tn));
+  int ti, tj;
+  grouped_tile(tile, (d + kM - 1) / kM, (d + kN - 1) / kN, ti, tj);
   const int i0 = ti * kM, j0 = tj * kN;
   const long long t_begin = (long long)split * per;
   const long long t_end = t_begin + per < n ? t_begin + per : n;
@@ -360,17 +387,8 @@ __global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const fl
   const int t = threadIdx.x, r = t >> 4, c4 = (t & 15) * 4;
   for (int blk = blockIdx.x; blk < tiles * 8; blk += gridDim.x) {
     const int tile = blk >> 3, br = (blk & 7) >> 2, bc = blk & 3;
-    int ti = 0;
-    {
-      int lo = 0, hi = (d + kM - 1) / kM - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (band_start(mid, tn) <= tile) lo = mid;
-        else hi = mid - 1;
-      }
-      ti = lo;
-    }
-    const int tj = ti / 2 + (int)(tile - band_start(ti, tn));
+    int ti, tj;
+    grouped_tile(tile, (d + kM - 1) / kM, tn, ti, tj);
     const int bi0 = ti * kM + 64 * br, bj0 = tj * kN + 64 * bc;
     if (!(bi0 < d && bj0 < d && bj0 + 63 >= bi0)) continue;   // block-uniform
     const float* src = part + (size_t)tile * nsplit * kM * kN + (size_t)(64 * br + r) * kN + 64 * bc + c4;

@@ -67,6 +67,27 @@ def test_hessian_matches_oracle(spec):
     assert np.all(np.abs(H2.cpu().numpy() - ref) <= 1e-5 * absref + 1e-30)
 
 
+@pytest.mark.parametrize("d", [2592, 4192])
+def test_hessian_super_block_order(d):
+    """Widths whose tiles span several 2048-channel super-blocks, with ragged
+    last super-blocks: 2592 (131 tiles, token-split, so the reduction decodes
+    the same tile order) and 4192 (305 tiles, unsplit). Every element of H is
+    compared with the float64 sum."""
+    spec = LayerSpec("wide", d_in=d, d_out=16, n_tok=1000, seed=7)
+    dev = torch.device("cuda")
+    X = gen_activations(spec, device="cpu")
+    H = torch.zeros(d, d, device=dev)
+    info = pp.new_info()
+    pp.hessian_accumulate(H, X.to(dev), pp.workspace(spec.d_out, d, spec.n_tok), info)
+    pp.raise_on_info(info)
+    X64 = bf16_bits_to_f64(X).numpy()
+    ref = X64.T @ X64
+    absref = np.abs(X64).T @ np.abs(X64)
+    Hg = H.cpu().numpy().astype(np.float64)
+    assert np.array_equal(Hg, Hg.T)
+    assert np.all(np.abs(Hg - ref) <= 1e-5 * absref + 1e-30)
+
+
 # ------------------------------------------------------------ factor
 
 @pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
