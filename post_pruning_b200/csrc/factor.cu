@@ -10,12 +10,16 @@
 // the sweep consumes it.
 //
 // Blocking: 128 x 128 tiles. Diagonal blocks are factored and inverted in
-// shared memory by one CTA; every other product (the panel R_ik = A_ik
-// U_kk^T, the rank-128 updates of the leading part, V_im = U_ii R_im and
-// the triangular inverse) runs on the tensor cores as an FP32-accurate
-// three-product TF32 GEMM (gemm_tc.cu). Operands move between those GEMMs
-// as hi/lo planes written by the producing epilogue, so no separate split
-// pass runs except once for the last column block.
+// shared memory by one CTA. The serial chain from one diagonal block to the
+// next is diag(k) -> chain step(k) -> diag(k-1): the chain step forms, in
+// plain FP32 on 136 CTAs, the one panel tile R_{k-1,k} and the update of
+// diagonal block k-1 that diag(k-1) waits for. Every other product (the
+// panel R_ik = A_ik U_kk^T of the rows above, the rank-128 updates of the
+// leading part, V_im = U_ii R_im and the triangular inverse) runs off the
+// chain on the tensor cores as an FP32-accurate three-product TF32 GEMM
+// (gemm_tc.cu). Operands move between those GEMMs as hi/lo planes written
+// by the producing epilogue, so no separate split pass runs except once for
+// the last column block.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -354,6 +358,158 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
   }
 }
 
+// ------------------------------------------------------------- chain step
+//
+// Right after diag(s), on the critical chain: the next diagonal block is
+// made ready without waiting for the panel product and the trailing update
+// of block column s, which then run off the chain:
+//   R_{s-1,s} = A_{s-1,s} U_ss^T           (its hi/lo planes replace the tile,
+//                                           as the panel product does for the
+//                                           rows above),
+//   D = A_{s-1,s-1} - R_{s-1,s} R_{s-1,s}^T (upper triangle, in place).
+// A_{s-1,s} is read from the hi/lo planes of block column s (hi + lo is the
+// fp32 value exactly), so the in-place planes of R never race with a read.
+// One CTA per 8 x 8 block (I, J), I <= J, of D (136 CTAs, one wave): it
+// forms rows I and J of R_{s-1,s} itself in plain FP32 (U_ss has zeros
+// below its diagonal, so each dot starts near the diagonal), then its block
+// of D; the CTAs with I == J also write the planes of their 8 rows of R.
+constexpr int kChainG = 8;
+constexpr int kChainBlocks = kTile / kChainG;                       // 16
+constexpr int kChainCtas = kChainBlocks * (kChainBlocks + 1) / 2;   // 136
+constexpr int kChainThreads = 256;
+constexpr int kChainLd = kTile + 4;                                 // 16-byte aligned rows
+constexpr size_t kChainSmem = (size_t)(kTile + 4 * kChainG) * kChainLd * sizeof(float);
+
+__global__ void __launch_bounds__(kChainThreads) chain_step_kernel(
+    float* __restrict__ Rw, float* __restrict__ V_lo, const float* __restrict__ A_hi,
+    const float* __restrict__ A_lo, const float* __restrict__ U, int d, int s, const int* info) {
+  if (cta_info_set(info)) return;
+  extern __shared__ __align__(16) float csm[];
+  float* Us = csm;                                // U_ss rows j, columns l (zeros outside)
+  float* As = csm + kTile * kChainLd;             // rows I then J of A_{s-1,s} (hi), then of R
+  float* Al = As + 2 * kChainG * kChainLd;        // the same rows, lo plane
+  const int tid = threadIdx.x;
+  // blockIdx.x -> (I, J), I <= J, column by column
+  int J = 0;
+  while ((J + 1) * (J + 2) / 2 <= (int)blockIdx.x) ++J;
+  const int I = (int)blockIdx.x - J * (J + 1) / 2;
+  const int c0 = s * kTile, bk = min(kTile, d - c0), r0 = c0 - kTile;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  // this thread's entry of the D block (phase 2), fetched early
+  const int o = tid >> 2, sl = tid & 3, da = o >> 3, db = o & 7;
+  const bool d_out = sl == 0 && (I < J || da <= db);
+  float* const d_ptr = Rw + (long long)(r0 + I * kChainG + da) * d + r0 + J * kChainG + db;
+  const float a_old = d_out ? *d_ptr : 0.f;
+  // U_ss (the chunks that reach the upper triangle) and both planes of the
+  // 16 A rows, all copies in flight at once
+#pragma unroll
+  for (int q = 0; q < kTile * kTile / 4 / kChainThreads; ++q) {
+    const int e = tid + q * kChainThreads, j = e >> 5, l = (e & 31) * 4;
+    float* dst = Us + j * kChainLd + l;
+    if (j < bk && l < bk && l + 4 > j) cp_async16(dst, U + (long long)(c0 + j) * d + c0 + l);
+    else *reinterpret_cast<float4*>(dst) = zero;
+  }
+#pragma unroll
+  for (int q = 0; q < 2 * kChainG * kTile / 4 / kChainThreads; ++q) {
+    const int e = tid + q * kChainThreads, r = e >> 5, l = (e & 31) * 4;
+    const int row = r0 + (r < kChainG ? I * kChainG + r : J * kChainG + r - kChainG);
+    if (l < bk) {
+      cp_async16(As + r * kChainLd + l, A_hi + (long long)row * kTile + l);
+      cp_async16(Al + r * kChainLd + l, A_lo + (long long)row * kTile + l);
+    } else {
+      *reinterpret_cast<float4*>(As + r * kChainLd + l) = zero;
+      *reinterpret_cast<float4*>(Al + r * kChainLd + l) = zero;
+    }
+  }
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+  // A = hi + lo (exact)
+#pragma unroll
+  for (int q = 0; q < 2 * kChainG * kTile / 4 / kChainThreads; ++q) {
+    const int e = tid + q * kChainThreads, r = e >> 5, l = (e & 31) * 4;
+    float4* x = reinterpret_cast<float4*>(As + r * kChainLd + l);
+    const float4 y = *reinterpret_cast<const float4*>(Al + r * kChainLd + l);
+    const float4 v = *x;
+    *x = make_float4(v.x + y.x, v.y + y.y, v.z + y.z, v.w + y.w);
+  }
+  __syncthreads();
+  // R[r][j] = sum_l A[r][l] U[j][l]: thread -> column j and half h of the
+  // l range, with U[j][64h..64h+64) in registers and the A rows read as
+  // broadcasts; warps whose half of U_ss is below the diagonal (h = 0,
+  // j >= 64) skip it. The h = 1 sums go through the lo-plane buffer, free by
+  // then, and are added to the h = 0 ones.
+  {
+    const int w = tid >> 5, h = w & 1, j = ((w >> 1) << 5) | (tid & 31);
+    float res[2 * kChainG];
+#pragma unroll
+    for (int r = 0; r < 2 * kChainG; ++r) res[r] = 0.f;
+    if (h == 1 || j < 64) {   // warp-uniform
+      float u[64];
+      const float* ur = Us + j * kChainLd + 64 * h;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = *reinterpret_cast<const float4*>(ur + 4 * c);
+        u[4 * c] = v.x; u[4 * c + 1] = v.y; u[4 * c + 2] = v.z; u[4 * c + 3] = v.w;
+      }
+#pragma unroll
+      for (int r = 0; r < 2 * kChainG; ++r) {
+        const float* ar = As + r * kChainLd + 64 * h;
+        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float4 x = *reinterpret_cast<const float4*>(ar + 4 * c);
+          p0 = fmaf(x.x, u[4 * c], p0);
+          p1 = fmaf(x.y, u[4 * c + 1], p1);
+          p0 = fmaf(x.z, u[4 * c + 2], p0);
+          p1 = fmaf(x.w, u[4 * c + 3], p1);
+        }
+        res[r] = p0 + p1;
+      }
+    }
+    if (h == 1) {
+#pragma unroll
+      for (int r = 0; r < 2 * kChainG; ++r) Al[r * kChainLd + j] = res[r];
+    }
+    __syncthreads();   // every thread is done reading the A rows
+    if (h == 0) {
+#pragma unroll
+      for (int r = 0; r < 2 * kChainG; ++r) As[r * kChainLd + j] = res[r] + Al[r * kChainLd + j];
+    }
+  }
+  __syncthreads();
+  // planes of rows I of R (the diagonal CTAs), coalesced
+  if (I == J) {
+    for (int e = tid; e < kChainG * (kTile / 4); e += kChainThreads) {
+      const int r = e >> 5, l = (e & 31) * 4;
+      if (l >= bk) continue;
+      const float4 v = *reinterpret_cast<const float4*>(As + r * kChainLd + l);
+      const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+      const long long off = (long long)(r0 + I * kChainG + r) * d + c0 + l;
+      st4(Rw + off, h);
+      st4(V_lo + off, make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w));
+    }
+  }
+  // D block: four threads per entry, a quarter of the K range each
+  {
+    const float* x = As + da * kChainLd;
+    const float* y = As + (kChainG + db) * kChainLd;
+    float s0 = 0.f, s1 = 0.f;
+    for (int l = 32 * sl; l < min(32 * sl + 32, bk); l += 4) {
+      const float4 p = *reinterpret_cast<const float4*>(x + l);
+      const float4 q = *reinterpret_cast<const float4*>(y + l);
+      s0 = fmaf(p.x, q.x, s0);
+      s1 = fmaf(p.y, q.y, s1);
+      s0 = fmaf(p.z, q.z, s0);
+      s1 = fmaf(p.w, q.w, s1);
+    }
+    float t = s0 + s1;
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    if (d_out) *d_ptr = a_old - t;
+  }
+}
+
 // ----------------------------------------------------------------- driver
 
 struct FactorWs {
@@ -403,15 +559,17 @@ int urow_splits(int tiles) {
 namespace {
 
 // The factorisation's internal streams (per device): the critical chain
-// diag(k) -> panel(k) -> update of column block k-1 -> diag(k-1) on `crit`;
-// the rest of each rank-128 update on `upd`; the V and U block rows, which
-// nothing in the chain waits for, on `rows`. They fork from and join back to
-// the caller's stream, so the whole factorisation is ordered on it (and
+// diag(k) -> chain step(k) -> diag(k-1) on `crit`; the panel product of
+// the rows above and the update of block column k-1 on `pan`; the rest of
+// each trailing update on `upd`; the V and U block rows, which nothing in
+// the chain waits for, on `rows`. They fork from and join back to the
+// caller's stream, so the whole factorisation is ordered on it (and
 // captures into one graph).
 struct FactorStreams {
-  cudaStream_t crit = nullptr, upd = nullptr, rows = nullptr;
-  cudaEvent_t fork = nullptr, diag_done = nullptr, panel_done = nullptr, upd_done = nullptr;
-  cudaEvent_t join[3] = {nullptr, nullptr, nullptr};
+  cudaStream_t crit = nullptr, pan = nullptr, upd = nullptr, rows = nullptr;
+  cudaEvent_t fork = nullptr, diag_done = nullptr, chain_done = nullptr, panel_done = nullptr,
+              pan_done = nullptr, upd_done = nullptr;
+  cudaEvent_t join[4] = {nullptr, nullptr, nullptr, nullptr};
 };
 
 std::mutex g_streams_mu;
@@ -428,9 +586,11 @@ cudaError_t factor_streams(FactorStreams** out) {
     int lo = 0, hi = 0;
     if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithPriority(&f.crit, cudaStreamNonBlocking, hi)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&f.pan, cudaStreamNonBlocking, hi)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithPriority(&f.upd, cudaStreamNonBlocking, lo)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithPriority(&f.rows, cudaStreamNonBlocking, lo)) != cudaSuccess) return e;
-    cudaEvent_t* evs[] = {&f.fork, &f.diag_done, &f.panel_done, &f.upd_done, &f.join[0], &f.join[1], &f.join[2]};
+    cudaEvent_t* evs[] = {&f.fork,     &f.diag_done, &f.chain_done, &f.panel_done, &f.pan_done,
+                          &f.upd_done, &f.join[0],   &f.join[1],    &f.join[2],    &f.join[3]};
     for (cudaEvent_t* ev : evs)
       if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
     made[dev] = true;
@@ -451,22 +611,45 @@ constexpr int kOffChainCtas = kNumSMs - 16;
 // Block columns from which the trailing updates go by pairs.
 constexpr int kPairFrom = 16;
 
-// The block-column loop and the V / U block rows (see the file comment).
+// Upper tiles of the leading part are numbered column by column: tile
+// (i, j), i <= j, is number j (j + 1) / 2 + i.
+inline int tri_start(int j) { return j * (j + 1) / 2; }
+
+// The block-column loop (see the file comment). Step k:
+//   crit: diag(k); chain step(k) (R_{k-1,k} and the updated diagonal block
+//         k-1), after the updates of the step before have written the tiles
+//         it reads;
+//   rows: V and U block rows k, once diag(k) is done and nothing reads
+//         block row k of R any more;
+//   pan:  panel R_ik = A_ik U_kk^T for the rows i < k-1, then the update of
+//         block column k-1 (rows above its diagonal block), which also
+//         writes the planes the next panel reads;
+//   upd:  the update of the block columns left of k-1.
+// From kPairFrom block columns on, the updates go by pairs of steps
+// (k+1, k): the first one updates block column k-1 and the diagonal tile of
+// column k-2 with panel k+1 alone (both are needed before the next two chain
+// steps); the second one updates everything left of block column k with
+// both panels (K = 256), so that the bulk of the trailing matrix is read and
+// written once per two block columns.
 cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const FactorStreams& f) {
   const int K = cdiv(d, kTile);
   const tc::Operand Ud{w.U_hi, w.U_lo, d, d, d};
   const tc::Operand Rp{w.R, w.V_lo, d, d, d};
+  const bool paired = K >= kPairFrom;
   cudaError_t e = cudaSuccess;
-  bool upd_pending = false;
+  bool pan_pending = false, upd_pending = false;
   for (int k = K - 1; k >= 0; --k) {
     const int c0 = k * kTile, bk = min(kTile, d - c0);
     diag_factor_kernel<<<1, kDiagThreads, kDiagSmem, f.crit>>>(w.R, d, k, U, w.U_hi, w.U_lo, info);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(f.diag_done, f.crit)) != cudaSuccess) return e;
     if (k < K - 1) {
       // block row k: V_km = U_kk R_km (planes in place of R_km's), then
-      // U_kq = -sum_{m=k+1..q} V_km U_mq, reading the U rows below it
-      if ((e = after(f.rows, f.crit, f.diag_done)) != cudaSuccess) return e;
+      // U_kq = -sum_{m=k+1..q} V_km U_mq, reading the U rows below it; the
+      // last reader of R_{k,k+1} is the column update of the step before
+      if ((e = cudaStreamWaitEvent(f.rows, f.diag_done, 0)) != cudaSuccess) return e;
+      if (pan_pending && (e = cudaStreamWaitEvent(f.rows, f.pan_done, 0)) != cudaSuccess) return e;
       tc::Job v{};
       v.mode = 3;
       v.s = k;
@@ -496,66 +679,88 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
         return e;
     }
     if (k == 0) break;
+    // chain step: tiles (k-1, k) and (k-1, k-1) hold every earlier panel's
+    // update once the last column update and the last bulk update are done
+    if (pan_pending && (e = cudaStreamWaitEvent(f.crit, f.pan_done, 0)) != cudaSuccess) return e;
+    if (upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
+    chain_step_kernel<<<kChainCtas, kChainThreads, kChainSmem, f.crit>>>(w.R, w.V_lo, w.A_hi, w.A_lo, U, d, k,
+                                                                          info);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(f.chain_done, f.crit)) != cudaSuccess) return e;
+    if (k == 1) continue;   // block 0 is all the chain step touches
+
+    const bool second = paired && ((K - 1 - k) & 1) != 0;   // k is the second step of its pair
+    const bool first = paired && !second;
+    // K of this step's updates: panel k, or panels k and k+1 (the last block
+    // may be narrower than 128)
+    const int kp = second ? std::min(2 * kTile, d - c0) : bk;
+    const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
     {
-      // panel R_ik = A_ik U_kk^T for the rows above, as hi/lo planes (hi
-      // over R, lo into V_lo)
+      // panel R_ik = A_ik U_kk^T for i < k-1, as hi/lo planes (hi over R,
+      // lo into V_lo)
+      if ((e = cudaStreamWaitEvent(f.pan, f.diag_done, 0)) != cudaSuccess) return e;
       const tc::Operand A{w.A_hi, w.A_lo, c0, bk, kTile};
       const tc::Operand B{w.U_hi + (long long)c0 * d + c0, w.U_lo + (long long)c0 * d + c0, bk, bk, d};
       tc::Job job{};
       job.mode = 0;
-      job.mt = k;
+      job.mt = k - 1;
       job.nt = 1;
       job.kdim = bk;
       job.ldc = d;
       job.c_col0 = c0;
-      job.Mlim = c0;
+      job.Mlim = c0 - kTile;
       job.Nlim = bk;
       job.alpha = 1.f;
       job.C_hi = w.R;
       job.C_lo = w.V_lo;
-      if ((e = tc::launch_gemm(A, B, false, job, k, info, f.crit)) != cudaSuccess) return e;
-    }
-    // Rank updates A_ij -= R_ik R_jk^T of the leading upper tiles, by pairs
-    // of block columns (k, k-1): the first of a pair updates only column
-    // block k-1 (on the chain; its tiles also write the planes the next
-    // panel reads); the second updates column block k-2 with both panels
-    // (K = 256, on the chain) and the tiles left of it with both panels on
-    // `upd`, so that the bulk of the trailing matrix is read and written once
-    // per two block columns. The chain waits for the previous bulk update
-    // before it touches tiles that update also wrote.
-    // (pairs only pay off for wide matrices: for a few blocks the longer
-    // column update on the chain costs more than the bulk traffic saved)
-    const bool paired = K >= kPairFrom;
-    const bool second = paired && ((K - 1 - k) & 1) != 0;   // k is the second block of its pair
-    // K of this step's updates: panel k, or panels k and k+1 (the last block
-    // may be narrower than 128)
-    const int kp = second ? std::min(2 * kTile, d - c0) : bk;
-    if (!second && upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
-    // (unpaired: every step updates column block k-1 on the chain and the
-    // tiles left of it on `upd`, with panel k alone)
-    const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
-    tc::Job job{};
-    job.mode = 1;
-    job.kdim = kp;
-    job.C = w.R;
-    job.ldc = d;
-    job.Mlim = job.Nlim = c0;
-    job.alpha = -1.f;
-    job.beta = 1.f;
-    if ((second || !paired) && k >= 2) {
-      if ((e = after(f.upd, f.crit, f.panel_done)) != cudaSuccess) return e;
       job.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(P, P, false, job, (k - 1) * k / 2, info, f.upd)) != cudaSuccess) return e;
-      job.max_ctas = 0;
+      if ((e = tc::launch_gemm(A, B, false, job, k - 1, info, f.pan)) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(f.panel_done, f.pan)) != cudaSuccess) return e;
+    }
+    {
+      // block column k-1 above its diagonal block (and, for the first step
+      // of a pair, the diagonal tile of block column k-2, which comes just
+      // before it in the numbering); the planes of block column k-1 for the
+      // next panel
+      if ((e = cudaStreamWaitEvent(f.pan, f.chain_done, 0)) != cudaSuccess) return e;
+      tc::Job job{};
+      job.mode = 1;
+      job.kdim = kp;
+      job.t0 = tri_start(k - 1) - (first ? 1 : 0);
+      job.C = w.R;
+      job.ldc = d;
+      job.Mlim = job.Nlim = c0;
+      job.alpha = -1.f;
+      job.beta = 1.f;
+      job.C_hi = w.A_hi;
+      job.C_lo = w.A_lo;
+      job.ldp = kTile;
+      job.p_col0 = c0 - kTile;
+      job.planes_one_col = first ? 1 : 0;
+      job.planes_n0 = c0 - kTile;
+      job.max_ctas = kOffChainCtas;
+      if ((e = tc::launch_gemm(P, P, false, job, (k - 1) + (first ? 1 : 0), info, f.pan)) != cudaSuccess)
+        return e;
+      if ((e = cudaEventRecord(f.pan_done, f.pan)) != cudaSuccess) return e;
+      pan_pending = true;
+    }
+    if (!first) {
+      // the block columns left of k-1
+      if ((e = cudaStreamWaitEvent(f.upd, f.panel_done, 0)) != cudaSuccess) return e;
+      tc::Job job{};
+      job.mode = 1;
+      job.kdim = kp;
+      job.C = w.R;
+      job.ldc = d;
+      job.Mlim = job.Nlim = c0;
+      job.alpha = -1.f;
+      job.beta = 1.f;
+      job.max_ctas = kOffChainCtas;
+      if ((e = tc::launch_gemm(P, P, false, job, tri_start(k - 1), info, f.upd)) != cudaSuccess) return e;
       if ((e = cudaEventRecord(f.upd_done, f.upd)) != cudaSuccess) return e;
       upd_pending = true;
     }
-    job.t0 = (k - 1) * k / 2;
-    job.C_hi = w.A_hi;
-    job.C_lo = w.A_lo;
-    job.ldp = kTile;
-    job.p_col0 = c0 - kTile;
-    if ((e = tc::launch_gemm(P, P, false, job, k, info, f.crit)) != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
@@ -570,6 +775,7 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
   static bool attr_done = false;
   if (!attr_done) {
     cudaFuncSetAttribute(diag_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
+    cudaFuncSetAttribute(chain_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChainSmem);
     attr_done = true;
   }
   FactorStreams* f = nullptr;
@@ -587,12 +793,12 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
                                      w.A_lo, kTile, info, st)) != cudaSuccess)
     return e;
   if ((e = cudaEventRecord(f->fork, st)) != cudaSuccess) return e;
-  for (cudaStream_t s : {f->crit, f->upd, f->rows})
+  for (cudaStream_t s : {f->crit, f->pan, f->upd, f->rows})
     if ((e = cudaStreamWaitEvent(s, f->fork, 0)) != cudaSuccess) return e;
   e = factor_blocks(w, d, U, info, *f);
   // always join, also after an error, so that a capture stays well formed
-  const cudaStream_t side[3] = {f->crit, f->upd, f->rows};
-  for (int i = 0; i < 3; ++i) {
+  const cudaStream_t side[4] = {f->crit, f->pan, f->upd, f->rows};
+  for (int i = 0; i < 4; ++i) {
     const cudaError_t e2 = after(st, side[i], f->join[i]);
     if (e == cudaSuccess) e = e2;
   }
