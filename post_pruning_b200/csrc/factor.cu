@@ -89,23 +89,30 @@ __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict
 // 32-panel p to the first. The pivots are the only serial chain, so one warp
 // runs them while the other seven do everything else around it:
 //   warp 0, per panel p: waits until D_pp is fully updated, factors it,
-//     D_pp = R_pp R_pp^T (lane = row, pivots broadcast by shuffles), inverts
-//     it, U_pp = R_pp^-1 (lane = column, column-form back substitution), and
-//     signals;
-//   warps 1-7, per panel p, once U_pp is there: the panel R_ip = A_ip U_pp^T
-//     for the sub-blocks above; the update A_ij -= R_ip R_jp^T, the next
-//     diagonal sub-block first (then warp 0 may go on) and the rest after;
-//     then block row p of U: V_pm = U_pp R_pm and
-//     U_pq = -sum_{m=p+1..q} V_pm U_mq (rows below p are final by then).
-// Warp 0 and the workers meet on two named barriers (one each way), the
-// workers among themselves on a third. Warp-level 32 x 32 products keep one
-// operand column per lane in registers and read the other operand's rows as
-// broadcast 16-byte loads, in units of 8 rows.
+//     D_pp = R_pp R_pp^T (lane = row; each pivot's column of R goes through
+//     a small shared buffer that every lane reads as broadcasts), inverts
+//     it, U_pp = R_pp^-1 (lane = column, back substitution reading that
+//     buffer), and signals;
+//   warps 1-4 then form the panel row R_{p-1,p} = A_{p-1,p} U_pp^T and
+//     update D_{p-1,p-1} -= R_{p-1,p} R_{p-1,p}^T, the only products the
+//     next pivots wait for, and signal warp 0;
+//   warps 5-7 meanwhile form the other panel rows R_ip (i < p-1); then all
+//     seven do the remaining updates A_ij -= R_ip R_jp^T and block row p of
+//     U, U_pq = -U_pp T_pq (q > p), from sums T_pq = sum_{m=p+1..q} R_pm U_mq
+//     that earlier panels accumulated; then add the terms R_ip U_pq (q >= p)
+//     to the sums T_iq of the rows above, and store the 32 finished rows of
+//     U (with their hi/lo planes) while the next panel's pivots run.
+// So after the last pivot only U_0q = -U_00 T_0q and the store of 32 rows
+// remain. Warp 0 and the workers meet on two named barriers (one each way),
+// the workers among themselves on two more. Warp-level 32 x 32 products
+// keep one operand column per lane in registers and read the other
+// operand's rows as broadcast 16-byte loads, in units of 8 rows.
 
 constexpr int kDiagThreads = 256;
 constexpr int kDiagWarps = kDiagThreads / 32;
 constexpr int kDiagLd = kTile + 4;     // 16-byte aligned rows
-constexpr size_t kDiagSmem = 3 * (size_t)kTile * kDiagLd * sizeof(float);
+constexpr int kPivLd = 36;             // pivot column buffer: 32 rows of 32 (+4)
+constexpr size_t kDiagSmem = (3 * (size_t)kTile * kDiagLd + 32 * kPivLd) * sizeof(float);
 
 // sum_k a[k] * b[k] over 32 entries: a is a shared-memory row (16-byte
 // aligned, read as broadcasts), b is in registers.
@@ -143,8 +150,8 @@ __device__ __forceinline__ float rsqrt_nr(float x) {
   return y * fmaf(-0.5f * x * y, y, 1.5f);
 }
 
-// Units of work for the eight warps: (32 x 32 block, 8-row quarter) pairs.
-__device__ __forceinline__ void tri_pair(int t, int& i, int& j) {   // t -> (i <= j)
+// t -> (i, j), i <= j, column by column.
+__device__ __forceinline__ void tri_pair(int t, int& i, int& j) {
   int jj = 0;
   while ((jj + 1) * (jj + 2) / 2 <= t) ++jj;
   j = jj;
@@ -158,10 +165,13 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
 __device__ __forceinline__ void bar_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
-constexpr int kBarUReady = 1;    // warp 0 -> workers: U_pp (and R_pp) written
-constexpr int kBarDReady = 2;    // workers -> warp 0: next diagonal sub-block updated
-constexpr int kBarWorkers = 3;   // the seven worker warps among themselves
 constexpr int kWorkers = kDiagWarps - 1;
+constexpr int kCritWarps = 4;                    // workers 0-3: the next pivots' products
+constexpr int kBarUReady = 1;    // warp 0 -> workers: U_pp (and R_pp) written        (all 256)
+constexpr int kBarDReady = 2;    // workers 0-3 -> warp 0: D_{p-1,p-1} updated       (160)
+constexpr int kBarCrit = 3;      // workers 0-3 among themselves                     (128)
+constexpr int kBarWorkers = 4;   // the seven workers among themselves               (224)
+constexpr int kDReadyCount = 32 * (1 + kCritWarps);
 
 // C[8 rows][lane] (+)= sum_k A[8 rows][k] * b[k] for a unit of 8 rows.
 __device__ __forceinline__ void unit_dot8(const float* A, const float (&b)[32], float (&acc)[8]) {
@@ -171,14 +181,17 @@ __device__ __forceinline__ void unit_dot8(const float* A, const float (&b)[32], 
 
 // Warp 0's part for panel p: factor the 32 x 32 diagonal sub-block at
 // (c0, c0) of S in place (reverse Cholesky, lane = row) and write its
-// inverse into Ui; returns the first failing column + 1 (or
-// SGPT_INFO_NONFINITE), 0 if every pivot was positive.
-__device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* rinv, int c0, int col0, int lane) {
+// inverse into Ui; Pc is a 32 x kPivLd buffer that ends up holding R_pp^T.
+// Returns the first failing column + 1 (or SGPT_INFO_NONFINITE), 0 if every
+// pivot was positive.
+__device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* Pc, float* rinv, int c0, int col0,
+                                           int lane) {
   // Pivot j: r_jj = sqrt(a_jj), r_ij = a_ij / r_jj (i < j), then
-  // a_il -= r_ij r_lj for l < j. The next pivot is broadcast before the
-  // rest of the update is issued. Entries
-  // below the diagonal (l < i) take the update too but are never read, and
-  // are zeroed on output.
+  // a_il -= r_ij r_lj for l < j. Lane j-1 forms the next pivot from its own
+  // r_{j-1,j} and broadcasts it; column j of R goes to Pc[j][.], from where
+  // every lane reads r_lj (l < j) as 16-byte broadcasts for the rest of its
+  // update. Entries below the diagonal (l < i) take the update too but are
+  // never read, and are zeroed on output.
   float dr[32];
   float* row = S + (c0 + lane) * kDiagLd + c0;
   load_row32(S + c0 * kDiagLd + c0, lane, dr);
@@ -190,13 +203,19 @@ __device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* rinv, int
     const float rs = rsqrt_nr(piv);
     const float rij = lane < j ? dr[j] * rs : (lane == j ? piv * rs : 0.f);
     dr[j] = rij;
+    Pc[j * kPivLd + lane] = rij;
     if (j == 0) break;
-    // lane j-1 forms its next pivot from its own r_{j-1,j} (no shuffle on
-    // the chain), then broadcasts it; the other lanes' updates follow
     const float own = fmaf(-rij, rij, dr[j - 1]);
     const float next = __shfl_sync(0xffffffffu, own, j - 1);
+    __syncwarp();
 #pragma unroll
-    for (int l = j - 1; l >= 0; --l) dr[l] = fmaf(-rij, __shfl_sync(0xffffffffu, rij, l), dr[l]);
+    for (int l4 = 0; l4 < j; l4 += 4) {
+      const float4 c = *reinterpret_cast<const float4*>(Pc + j * kPivLd + l4);
+      dr[l4] = fmaf(-rij, c.x, dr[l4]);
+      if (l4 + 1 < j) dr[l4 + 1] = fmaf(-rij, c.y, dr[l4 + 1]);
+      if (l4 + 2 < j) dr[l4 + 2] = fmaf(-rij, c.z, dr[l4 + 2]);
+      if (l4 + 3 < j) dr[l4 + 3] = fmaf(-rij, c.w, dr[l4 + 3]);
+    }
     piv = next;
   }
 #pragma unroll
@@ -204,20 +223,25 @@ __device__ __forceinline__ int pivot_panel(float* S, float* Ui, float* rinv, int
     *reinterpret_cast<float4*>(row + l) =
         make_float4(lane <= l ? dr[l] : 0.f, lane <= l + 1 ? dr[l + 1] : 0.f, lane <= l + 2 ? dr[l + 2] : 0.f,
                     lane <= l + 3 ? dr[l + 3] : 0.f);
-  rinv[c0 + lane] = 1.0f / row[lane];      // this lane's own diagonal entry
+  rinv[c0 + lane] = 1.0f / Pc[lane * kPivLd + lane];   // 1 / r_ii, written by this lane
   __syncwarp();
   // U_pp = R_pp^-1, lane = column: back substitution from the bottom in
-  // column form, u_m = acc_m / r_mm, then acc_i -= r_im u_m for i < m (row
-  // m-1 first: it is the next step's).
+  // column form, u_m = acc_m / r_mm, then acc_i -= r_im u_m for i < m, with
+  // r_im = Pc[m][i] read as 16-byte broadcasts.
   float u[32];
-  const float* R = S + c0 * kDiagLd + c0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) u[i] = (i == lane) ? 1.f : 0.f;
 #pragma unroll
   for (int m = 31; m >= 0; --m) {
     u[m] = (m <= lane) ? u[m] * rinv[c0 + m] : 0.f;
 #pragma unroll
-    for (int i = m - 1; i >= 0; --i) u[i] = fmaf(-R[i * kDiagLd + m], u[m], u[i]);
+    for (int i4 = 0; i4 < m; i4 += 4) {
+      const float4 c = *reinterpret_cast<const float4*>(Pc + m * kPivLd + i4);
+      u[i4] = fmaf(-c.x, u[m], u[i4]);
+      if (i4 + 1 < m) u[i4 + 1] = fmaf(-c.y, u[m], u[i4 + 1]);
+      if (i4 + 2 < m) u[i4 + 2] = fmaf(-c.z, u[m], u[i4 + 2]);
+      if (i4 + 3 < m) u[i4 + 3] = fmaf(-c.w, u[m], u[i4 + 3]);
+    }
   }
 #pragma unroll
   for (int i = 0; i < 32; ++i) Ui[(c0 + i) * kDiagLd + c0 + lane] = u[i];
@@ -233,8 +257,9 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
   if (cta_info_set(info)) return;
   extern __shared__ __align__(16) float dsm[];
   float* S = dsm;                            // A, becoming R (upper)
-  float* Ui = dsm + kTile * kDiagLd;         // U (upper)
-  float* Vb = dsm + 2 * kTile * kDiagLd;     // V_pm blocks
+  float* Ui = dsm + kTile * kDiagLd;         // U (upper, zeros below)
+  float* T = dsm + 2 * kTile * kDiagLd;      // sums T_pq of the block rows of U still to come
+  float* Pc = dsm + 3 * kTile * kDiagLd;     // warp 0's pivot columns
   __shared__ float rinv[kTile];
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -262,11 +287,11 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
   __syncthreads();
 
   // Every thread runs the same barrier sequence whatever the data; a failed
-  // pivot is reported after the loop (the values are then discarded).
+  // pivot is reported at the end (the values are then meaningless).
   if (warp == 0) {
     for (int p = np - 1; p >= 0; --p) {
-      if (p < np - 1) bar_sync(kBarDReady, kDiagThreads);
-      const int fail = pivot_panel(S, Ui, rinv, p * 32, b0 + p * 32, lane);
+      if (p < np - 1) bar_sync(kBarDReady, kDReadyCount);
+      const int fail = pivot_panel(S, Ui, Pc, rinv, p * 32, b0 + p * 32, lane);
       if (fail && lane == 0 && bad == 0) bad = fail;
       bar_arrive(kBarUReady, kDiagThreads);
     }
@@ -276,86 +301,95 @@ __global__ void __launch_bounds__(kDiagThreads, 1) diag_factor_kernel(const floa
       const int c0 = p * 32;
       bar_sync(kBarUReady, kDiagThreads);
       if (p > 0) {
-        {
-          // panel: R_ip = A_ip U_pp^T for i < p, in place; lane = column j
-          // with row j of U_pp in registers
-          float bu[32];
-          load_row32(Ui + c0 * kDiagLd + c0, lane, bu);
-          for (int unit = w; unit < p * 4; unit += kWorkers) {
-            float* A = S + (unit * 8) * kDiagLd + c0;
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            unit_dot8(A, bu, acc);
-            __syncwarp();
+        // panel R_ip = A_ip U_pp^T in place; lane = column j with row j of
+        // U_pp in registers. Workers 0-3 take row block p-1 (the next
+        // pivots need it), workers 4-6 the rows above.
+        float bu[32];
+        load_row32(Ui + c0 * kDiagLd + c0, lane, bu);
+        const int first = w < kCritWarps ? (p - 1) * 4 + w : w - kCritWarps;
+        const int last = w < kCritWarps ? first + 1 : (p - 1) * 4;
+        const int step = w < kCritWarps ? 1 : kWorkers - kCritWarps;
+        for (int unit = first; unit < last; unit += step) {
+          float* A = S + (unit * 8) * kDiagLd + c0;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          unit_dot8(A, bu, acc);
+          __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) A[i * kDiagLd + lane] = acc[i];
-          }
+          for (int i = 0; i < 8; ++i) A[i * kDiagLd + lane] = acc[i];
         }
-        bar_sync(kBarWorkers, kWorkers * 32);
-        // update A_ij -= R_ip R_jp^T for i <= j < p: the sub-block (p-1, p-1)
-        // first (four units), then warp 0 may factor it
-        const int units = p * (p + 1) / 2 * 4;
-        if (w >= 4) bar_arrive(kBarDReady, kDiagThreads);   // no unit among the first four
-        for (int unit = w; unit < units; unit += kWorkers) {
-          // unit order: the last pair (p-1, p-1) first, then the others
-          const int t = (unit < 4) ? (units / 4 - 1) : ((unit - 4) >> 2);
-          int ii, jj;
-          tri_pair(t, ii, jj);
-          const int r0 = ii * 32 + (unit & 3) * 8;
+        if (w < kCritWarps) {
+          // D_{p-1,p-1} -= R_{p-1,p} R_{p-1,p}^T, quarter w, then warp 0 may go on
+          bar_sync(kBarCrit, 32 * kCritWarps);
+          const int r0 = (p - 1) * 32 + w * 8;
           float br[32];
-          load_row32(S + (jj * 32) * kDiagLd + c0, lane, br);   // row `lane` of R_jp
+          load_row32(S + ((p - 1) * 32) * kDiagLd + c0, lane, br);   // row `lane` of R_{p-1,p}
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           unit_dot8(S + r0 * kDiagLd + c0, br, acc);
-          float* C = S + r0 * kDiagLd + jj * 32;
+          float* C = S + r0 * kDiagLd + (p - 1) * 32;
 #pragma unroll
           for (int i = 0; i < 8; ++i) C[i * kDiagLd + lane] -= acc[i];
-          if (unit < 4) bar_arrive(kBarDReady, kDiagThreads);   // each of workers 0-3, once
+          bar_arrive(kBarDReady, kDReadyCount);
+        }
+        bar_sync(kBarWorkers, kWorkers * 32);   // every panel row is there
+      }
+      {
+        // the other updates A_ij -= R_ip R_jp^T (i <= j < p, but not
+        // (p-1, p-1)), then block row p of U: U_pq = -U_pp T_pq (q > p)
+        const int n_upd = p > 0 ? (p * (p + 1) / 2 - 1) * 4 : 0;
+        const int n_u = (np - 1 - p) * 4;
+        for (int unit = w; unit < n_upd + n_u; unit += kWorkers) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          if (unit < n_upd) {
+            int ii, jj;
+            tri_pair(unit >> 2, ii, jj);   // pairs below t = p(p+1)/2 - 1, i.e. all but (p-1, p-1)
+            const int r0 = ii * 32 + (unit & 3) * 8;
+            float br[32];
+            load_row32(S + (jj * 32) * kDiagLd + c0, lane, br);   // row `lane` of R_jp
+            unit_dot8(S + r0 * kDiagLd + c0, br, acc);
+            float* C = S + r0 * kDiagLd + jj * 32;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) C[i * kDiagLd + lane] -= acc[i];
+          } else {
+            const int u = unit - n_upd, q = p + 1 + (u >> 2), r0 = c0 + (u & 3) * 8;
+            float bt[32];
+            load_col32(T + c0 * kDiagLd + q * 32, lane, bt);      // column `lane` of T_pq
+            unit_dot8(Ui + r0 * kDiagLd + c0, bt, acc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) Ui[(r0 + i) * kDiagLd + q * 32 + lane] = -acc[i];
+          }
         }
       }
-      // block row p of U (the rows below are final): V_pm = U_pp R_pm ...
-      if (p < np - 1) {
-        const int nm = np - 1 - p;
-        for (int unit = w; unit < nm * 4; unit += kWorkers) {
-          const int m = p + 1 + (unit >> 2), r0 = c0 + (unit & 3) * 8;
-          float bcol[32];
-          load_col32(S + c0 * kDiagLd + m * 32, lane, bcol);   // column `lane` of R_pm
+      bar_sync(kBarWorkers, kWorkers * 32);   // block row p of U is final
+      {
+        // T_iq += R_ip U_pq for i < p, q >= p (the first term, q == p,
+        // starts the sum), and the store of rows c0..c0+31 of U
+        const int n_t = p * (np - p) * 4;
+        for (int unit = w; unit < n_t; unit += kWorkers) {
+          const int pair = unit >> 2, i = pair / (np - p), q = p + pair % (np - p);
+          const int r0 = i * 32 + (unit & 3) * 8;
+          float bu2[32];
+          load_col32(Ui + c0 * kDiagLd + q * 32, lane, bu2);    // column `lane` of U_pq
           float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          unit_dot8(Ui + r0 * kDiagLd + c0, bcol, acc);
+          unit_dot8(S + r0 * kDiagLd + c0, bu2, acc);
+          float* C = T + r0 * kDiagLd + q * 32;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) Vb[(r0 + i) * kDiagLd + m * 32 + lane] = acc[i];
+          for (int x = 0; x < 8; ++x) C[x * kDiagLd + lane] = (q == p ? 0.f : C[x * kDiagLd + lane]) + acc[x];
         }
-        bar_sync(kBarWorkers, kWorkers * 32);
-        // ... then U_pq = -sum_{m=p+1..q} V_pm U_mq
-        for (int unit = w; unit < nm * 4; unit += kWorkers) {
-          const int q = p + 1 + (unit >> 2), r0 = c0 + (unit & 3) * 8;
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          for (int m = p + 1; m <= q; ++m) {
-            float bcol[32];
-            load_col32(Ui + (m * 32) * kDiagLd + q * 32, lane, bcol);   // column `lane` of U_mq
-            unit_dot8(Vb + r0 * kDiagLd + m * 32, bcol, acc);
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) Ui[(r0 + i) * kDiagLd + q * 32 + lane] = -acc[i];
+        for (int e = tid - 32; e < 32 * (kTile / 4); e += kWorkers * 32) {
+          const int i = c0 + (e >> 5), l = (e & 31) * 4;
+          if (l >= b) continue;
+          const float4 v = *reinterpret_cast<const float4*>(Ui + i * kDiagLd + l);
+          const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+          const long long off = (long long)(b0 + i) * d + b0 + l;
+          st4(U + off, v);
+          st4(U_hi + off, h);
+          st4(U_lo + off, make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w));
         }
       }
     }
   }
   __syncthreads();
-  if (bad) {
-    if (tid == 0) set_info(info, bad);
-    return;
-  }
-
-  // Write U_kk (upper, zeros below) and its hi/lo planes.
-  for (int e = tid * 4; e < kTile * kTile; e += kDiagThreads * 4) {
-    const int i = e >> 7, l = e & 127;
-    if (i >= b || l >= b) continue;
-    const float4 v = *reinterpret_cast<const float4*>(Ui + i * kDiagLd + l);
-    const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-    const long long off = (long long)(b0 + i) * d + b0 + l;
-    st4(U + off, v);
-    st4(U_hi + off, h);
-    st4(U_lo + off, make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w));
-  }
+  if (bad && tid == 0) set_info(info, bad);
 }
 
 // ------------------------------------------------------------- chain step
