@@ -548,13 +548,14 @@ __global__ void __launch_bounds__(kChainThreads) chain_step_kernel(
 
 struct FactorWs {
   double* lam;
-  float* R;        // H_d, then R; the hi plane of R_ik and then of V_ik above the diagonal blocks
-  float* V_lo;     // lo plane of R_ik, then of V_ik (d x d)
+  float* R;        // H_d, then R; the hi plane of R_ik above the diagonal blocks
+  float* V_lo;     // lo plane of R_ik (d x d)
   float* U_hi;     // hi/lo planes of U (d x d)
   float* U_lo;
   float* A_hi;     // hi/lo planes of the next column block of the updated H_d (d x 128)
   float* A_lo;
-  float* part;     // split partials of the triangular inverse
+  float* T_hi;     // hi/lo planes of the next block row of the sums T (128 x d)
+  float* T_lo;
 };
 
 static FactorWs carve_factor(void* ws, int d, size_t* bytes) {
@@ -567,7 +568,8 @@ static FactorWs carve_factor(void* ws, int d, size_t* bytes) {
   w.U_lo = c.take<float>((size_t)d * d);
   w.A_hi = c.take<float>((size_t)d * kTile);
   w.A_lo = c.take<float>((size_t)d * kTile);
-  w.part = c.take<float>(factor_part_tiles(d) * kTile * kTile);
+  w.T_hi = c.take<float>((size_t)kTile * d);
+  w.T_lo = c.take<float>((size_t)kTile * d);
   if (bytes) *bytes = c.off + 256;
   return w;
 }
@@ -576,18 +578,6 @@ size_t factor_ws_bytes(int d) {
   size_t b = 0;
   carve_factor(nullptr, d, &b);
   return b;
-}
-
-size_t factor_part_tiles(int d) {
-  const int K = cdiv(d, kTile);
-  return K > 1 ? (size_t)tc::row_items(K - 1, urow_splits(K - 1)) : 0;
-}
-
-int urow_splits(int tiles) {
-  // a block row of U with `tiles` tiles whose K lengths are 1..tiles blocks:
-  // long ranges are cut into pieces of 8 blocks (1024 of K) so that the
-  // row's items are short and balance across SMs; short rows are not cut
-  return tiles > 8 ? 8 : 0;
 }
 
 namespace {
@@ -653,12 +643,17 @@ inline int tri_start(int j) { return j * (j + 1) / 2; }
 //   crit: diag(k); chain step(k) (R_{k-1,k} and the updated diagonal block
 //         k-1), after the updates of the step before have written the tiles
 //         it reads;
-//   rows: V and U block rows k, once diag(k) is done and nothing reads
-//         block row k of R any more;
 //   pan:  panel R_ik = A_ik U_kk^T for the rows i < k-1, then the update of
 //         block column k-1 (rows above its diagonal block), which also
 //         writes the planes the next panel reads;
-//   upd:  the update of the block columns left of k-1.
+//   upd:  the update of the block columns left of k-1;
+//   rows: block row k of U, U_kq = -U_kk T_kq (q > k), then the step's
+//         terms R_ik U_kq (i < k, q >= k) of the sums
+//         T_iq = sum_{m=i+1..q} R_im U_mq: one rank-128 product over the
+//         whole rectangle above and right of block k. T lives in the
+//         still-unused upper part of U (zero at the start); the product that
+//         completes block row k-1 of T also writes its hi/lo planes, which
+//         the next block row of U reads.
 // From kPairFrom block columns on, the updates go by pairs of steps
 // (k+1, k): the first one updates block column k-1 and the diagonal tile of
 // column k-2 with panel k+1 alone (both are needed before the next two chain
@@ -669,6 +664,7 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
   const int K = cdiv(d, kTile);
   const tc::Operand Ud{w.U_hi, w.U_lo, d, d, d};
   const tc::Operand Rp{w.R, w.V_lo, d, d, d};
+  const tc::Operand Tp{w.T_hi, w.T_lo, kTile, d, d};
   const bool paired = K >= kPairFrom;
   cudaError_t e = cudaSuccess;
   bool pan_pending = false, upd_pending = false;
@@ -678,122 +674,141 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(f.diag_done, f.crit)) != cudaSuccess) return e;
-    if (k < K - 1) {
-      // block row k: V_km = U_kk R_km (planes in place of R_km's), then
-      // U_kq = -sum_{m=k+1..q} V_km U_mq, reading the U rows below it; the
-      // last reader of R_{k,k+1} is the column update of the step before
-      if ((e = cudaStreamWaitEvent(f.rows, f.diag_done, 0)) != cudaSuccess) return e;
-      if (pan_pending && (e = cudaStreamWaitEvent(f.rows, f.pan_done, 0)) != cudaSuccess) return e;
-      tc::Job v{};
-      v.mode = 3;
-      v.s = k;
-      v.dlim = d;
-      v.ldc = d;
-      v.Mlim = v.Nlim = d;
-      v.alpha = 1.f;
-      v.C_hi = w.R;
-      v.C_lo = w.V_lo;
-      v.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(Ud, Rp, true, v, K - 1 - k, info, f.rows)) != cudaSuccess) return e;
-      tc::Job u{};
-      u.mode = 2;
-      u.s = k;
-      u.nsplit = urow_splits(K - 1 - k);
-      u.nblk = K;
-      u.dlim = d;
-      u.C = U;
-      u.ldc = d;
-      u.Mlim = u.Nlim = d;
-      u.alpha = -1.f;
-      u.C_hi = w.U_hi;
-      u.C_lo = w.U_lo;
-      u.part = w.part;
-      u.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(Rp, Ud, true, u, tc::row_items(K - 1 - k, u.nsplit), info, f.rows)) != cudaSuccess)
-        return e;
+    if (k > 0) {
+      // chain step: tiles (k-1, k) and (k-1, k-1) hold every earlier panel's
+      // update once the last column update and the last bulk update are done
+      if (pan_pending && (e = cudaStreamWaitEvent(f.crit, f.pan_done, 0)) != cudaSuccess) return e;
+      if (upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
+      chain_step_kernel<<<kChainCtas, kChainThreads, kChainSmem, f.crit>>>(w.R, w.V_lo, w.A_hi, w.A_lo, U, d,
+                                                                            k, info);
+      count_launches(1);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      if ((e = cudaEventRecord(f.chain_done, f.crit)) != cudaSuccess) return e;
     }
-    if (k == 0) break;
-    // chain step: tiles (k-1, k) and (k-1, k-1) hold every earlier panel's
-    // update once the last column update and the last bulk update are done
-    if (pan_pending && (e = cudaStreamWaitEvent(f.crit, f.pan_done, 0)) != cudaSuccess) return e;
-    if (upd_pending && (e = cudaStreamWaitEvent(f.crit, f.upd_done, 0)) != cudaSuccess) return e;
-    chain_step_kernel<<<kChainCtas, kChainThreads, kChainSmem, f.crit>>>(w.R, w.V_lo, w.A_hi, w.A_lo, U, d, k,
-                                                                          info);
-    count_launches(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(f.chain_done, f.crit)) != cudaSuccess) return e;
-    if (k == 1) continue;   // block 0 is all the chain step touches
-
-    const bool second = paired && ((K - 1 - k) & 1) != 0;   // k is the second step of its pair
-    const bool first = paired && !second;
-    // K of this step's updates: panel k, or panels k and k+1 (the last block
-    // may be narrower than 128)
-    const int kp = second ? std::min(2 * kTile, d - c0) : bk;
-    const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
-    {
-      // panel R_ik = A_ik U_kk^T for i < k-1, as hi/lo planes (hi over R,
-      // lo into V_lo)
-      if ((e = cudaStreamWaitEvent(f.pan, f.diag_done, 0)) != cudaSuccess) return e;
-      const tc::Operand A{w.A_hi, w.A_lo, c0, bk, kTile};
-      const tc::Operand B{w.U_hi + (long long)c0 * d + c0, w.U_lo + (long long)c0 * d + c0, bk, bk, d};
+    if (k >= 2) {   // block 0 is all the chain step of k = 1 touches
+      const bool second = paired && ((K - 1 - k) & 1) != 0;   // k is the second step of its pair
+      const bool first = paired && !second;
+      // K of this step's updates: panel k, or panels k and k+1 (the last
+      // block may be narrower than 128)
+      const int kp = second ? std::min(2 * kTile, d - c0) : bk;
+      const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
+      {
+        // panel R_ik = A_ik U_kk^T for i < k-1, as hi/lo planes (hi over R,
+        // lo into V_lo)
+        if ((e = cudaStreamWaitEvent(f.pan, f.diag_done, 0)) != cudaSuccess) return e;
+        const tc::Operand A{w.A_hi, w.A_lo, c0, bk, kTile};
+        const tc::Operand B{w.U_hi + (long long)c0 * d + c0, w.U_lo + (long long)c0 * d + c0, bk, bk, d};
+        tc::Job job{};
+        job.mode = 0;
+        job.mt = k - 1;
+        job.nt = 1;
+        job.kdim = bk;
+        job.ldc = d;
+        job.c_col0 = c0;
+        job.Mlim = c0 - kTile;
+        job.Nlim = bk;
+        job.alpha = 1.f;
+        job.C_hi = w.R;
+        job.C_lo = w.V_lo;
+        job.max_ctas = kOffChainCtas;
+        if ((e = tc::launch_gemm(A, B, false, job, k - 1, info, f.pan)) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(f.panel_done, f.pan)) != cudaSuccess) return e;
+      }
+      {
+        // block column k-1 above its diagonal block (and, for the first
+        // step of a pair, the diagonal tile of block column k-2, which comes
+        // just before it in the numbering); the planes of block column k-1
+        // for the next panel
+        if ((e = cudaStreamWaitEvent(f.pan, f.chain_done, 0)) != cudaSuccess) return e;
+        tc::Job job{};
+        job.mode = 1;
+        job.kdim = kp;
+        job.t0 = tri_start(k - 1) - (first ? 1 : 0);
+        job.C = w.R;
+        job.ldc = d;
+        job.Mlim = job.Nlim = c0;
+        job.alpha = -1.f;
+        job.beta = 1.f;
+        job.C_hi = w.A_hi;
+        job.C_lo = w.A_lo;
+        job.ldp = kTile;
+        job.p_col0 = c0 - kTile;
+        job.planes_one_col = first ? 1 : 0;
+        job.planes_n0 = c0 - kTile;
+        job.max_ctas = kOffChainCtas;
+        if ((e = tc::launch_gemm(P, P, false, job, (k - 1) + (first ? 1 : 0), info, f.pan)) != cudaSuccess)
+          return e;
+        if ((e = cudaEventRecord(f.pan_done, f.pan)) != cudaSuccess) return e;
+        pan_pending = true;
+      }
+      if (!first) {
+        // the block columns left of k-1
+        if ((e = cudaStreamWaitEvent(f.upd, f.panel_done, 0)) != cudaSuccess) return e;
+        tc::Job job{};
+        job.mode = 1;
+        job.kdim = kp;
+        job.C = w.R;
+        job.ldc = d;
+        job.Mlim = job.Nlim = c0;
+        job.alpha = -1.f;
+        job.beta = 1.f;
+        job.max_ctas = kOffChainCtas;
+        if ((e = tc::launch_gemm(P, P, false, job, tri_start(k - 1), info, f.upd)) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(f.upd_done, f.upd)) != cudaSuccess) return e;
+        upd_pending = true;
+      }
+    }
+    // rows: U_kq = -U_kk T_kq for q > k (T's block row k is complete: its
+    // last term came from step k+1, on this stream)
+    if ((e = cudaStreamWaitEvent(f.rows, f.diag_done, 0)) != cudaSuccess) return e;
+    if (k < K - 1) {
       tc::Job job{};
       job.mode = 0;
-      job.mt = k - 1;
-      job.nt = 1;
+      job.mt = 1;
+      job.nt = K - 1 - k;
+      job.kdim = kTile;
+      job.a_x0 = job.a_y0 = c0;
+      job.b_x0 = c0 + kTile;
+      job.C = U;
+      job.ldc = d;
+      job.c_row0 = c0;
+      job.c_col0 = c0 + kTile;
+      job.Mlim = kTile;
+      job.Nlim = d - c0 - kTile;
+      job.alpha = -1.f;
+      job.C_hi = w.U_hi;
+      job.C_lo = w.U_lo;
+      job.max_ctas = kOffChainCtas;
+      if ((e = tc::launch_gemm(Ud, Tp, true, job, K - 1 - k, info, f.rows)) != cudaSuccess) return e;
+    }
+    if (k > 0) {
+      // T_iq += R_ik U_kq for i < k, q >= k (rows [0, c0), columns [c0, d)),
+      // with the planes of T's block row k-1, which this term completes
+      if ((e = cudaStreamWaitEvent(f.rows, f.chain_done, 0)) != cudaSuccess) return e;
+      if (k >= 2 && (e = cudaStreamWaitEvent(f.rows, f.panel_done, 0)) != cudaSuccess) return e;
+      tc::Job job{};
+      job.mode = 0;
+      job.mt = k;
+      job.nt = K - k;
       job.kdim = bk;
+      job.a_x0 = c0;
+      job.b_x0 = c0;
+      job.b_y0 = c0;
+      job.C = U;
       job.ldc = d;
       job.c_col0 = c0;
-      job.Mlim = c0 - kTile;
-      job.Nlim = bk;
+      job.Mlim = c0;
+      job.Nlim = d - c0;
       job.alpha = 1.f;
-      job.C_hi = w.R;
-      job.C_lo = w.V_lo;
-      job.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(A, B, false, job, k - 1, info, f.pan)) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(f.panel_done, f.pan)) != cudaSuccess) return e;
-    }
-    {
-      // block column k-1 above its diagonal block (and, for the first step
-      // of a pair, the diagonal tile of block column k-2, which comes just
-      // before it in the numbering); the planes of block column k-1 for the
-      // next panel
-      if ((e = cudaStreamWaitEvent(f.pan, f.chain_done, 0)) != cudaSuccess) return e;
-      tc::Job job{};
-      job.mode = 1;
-      job.kdim = kp;
-      job.t0 = tri_start(k - 1) - (first ? 1 : 0);
-      job.C = w.R;
-      job.ldc = d;
-      job.Mlim = job.Nlim = c0;
-      job.alpha = -1.f;
       job.beta = 1.f;
-      job.C_hi = w.A_hi;
-      job.C_lo = w.A_lo;
-      job.ldp = kTile;
-      job.p_col0 = c0 - kTile;
-      job.planes_one_col = first ? 1 : 0;
-      job.planes_n0 = c0 - kTile;
+      job.C_hi = w.T_hi;
+      job.C_lo = w.T_lo;
+      job.ldp = d;
+      job.p_row0 = c0 - kTile;
+      job.planes_one_row = 1;
+      job.planes_m0 = c0 - kTile;
       job.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(P, P, false, job, (k - 1) + (first ? 1 : 0), info, f.pan)) != cudaSuccess)
-        return e;
-      if ((e = cudaEventRecord(f.pan_done, f.pan)) != cudaSuccess) return e;
-      pan_pending = true;
-    }
-    if (!first) {
-      // the block columns left of k-1
-      if ((e = cudaStreamWaitEvent(f.upd, f.panel_done, 0)) != cudaSuccess) return e;
-      tc::Job job{};
-      job.mode = 1;
-      job.kdim = kp;
-      job.C = w.R;
-      job.ldc = d;
-      job.Mlim = job.Nlim = c0;
-      job.alpha = -1.f;
-      job.beta = 1.f;
-      job.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(P, P, false, job, tri_start(k - 1), info, f.upd)) != cudaSuccess) return e;
-      if ((e = cudaEventRecord(f.upd_done, f.upd)) != cudaSuccess) return e;
-      upd_pending = true;
+      if ((e = tc::launch_gemm(Rp, Ud, true, job, k * (K - k), info, f.rows)) != cudaSuccess) return e;
     }
   }
   return cudaSuccess;

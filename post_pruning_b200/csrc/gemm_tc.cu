@@ -8,8 +8,9 @@
 // product is about 2^-21 relative, against 2^-24 for a plain fp32 FMA and
 // 2^-11 for a single TF32 product.
 //
-// Used for the rank-128 updates and the triangular inverse of the
-// factorisation and for the lazy trailing update of the OBS sweep.
+// Used for the panel products, the rank-128 updates and the triangular
+// inverse of the factorisation and for the lazy trailing update of the OBS
+// sweep.
 //
 // Output tiles of 128 x 128, K in stages of 32 (one 128-byte swizzle row of
 // fp32) through a two-stage TMA ring of 64 KB stages (no multicast). Persistent: one CTA per
@@ -162,11 +163,6 @@ __device__ __forceinline__ void tri_index(int t, int& i, int& j) {
 
 }  // namespace
 
-// Items before tile t of a split block row: tile t' has t' / b + 1 pieces.
-__host__ __device__ __forceinline__ int split_prefix(int t, int b) {
-  const int a = t / b;
-  return t + b * a * (a - 1) / 2 + a * (t - b * a);
-}
 
 // Work item w of a launch: its output tile (m0, n0) and K range [kb, ke).
 struct Item {
@@ -185,33 +181,6 @@ __device__ __forceinline__ Item decode_item(const Job& job, int w) {
     it.m0 = i * kM;
     it.n0 = j * kN;
     it.ke = job.kdim;
-  } else if (job.mode == 3) {
-    it.m0 = job.s * kM;
-    it.n0 = (job.s + 1 + w) * kN;
-    it.kb = it.m0;
-    it.ke = min(it.m0 + kM, job.dlim);
-  } else {
-    int tile = w, piece = 0;
-    if (job.nsplit > 0) {                     // the tile whose pieces hold item w
-      int lo = 0, hi = job.nblk - 1 - job.s;  // split_prefix(lo) <= w < split_prefix(hi)
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (split_prefix(mid, job.nsplit) <= w) lo = mid; else hi = mid;
-      }
-      tile = lo;
-      piece = w - split_prefix(lo, job.nsplit);
-    }
-    const int i = job.s, j = job.s + 1 + tile;
-    it.m0 = i * kM;
-    it.n0 = j * kN;
-    const int lo = (i + 1) * kM, hi = min((j + 1) * kM, job.dlim);
-    if (job.nsplit > 0) {
-      it.kb = min(hi, lo + piece * job.nsplit * kM);
-      it.ke = min(hi, it.kb + job.nsplit * kM);
-    } else {
-      it.kb = lo;
-      it.ke = hi;
-    }
   }
   return it;
 }
@@ -357,8 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
     const int q = warp & 3, h = (warp - 2) >> 2;
     const int m = q * 32 + lane;                  // tile row = TMEM lane
     const int ew = warp - 2;                      // 0..7: rows 16*ew.. in the write-out
-    const bool partial = job.mode == 2 && job.nsplit > 0;
-    const bool read_c = !partial && job.C != nullptr && job.beta != 0.f;
+    const bool read_c = job.C != nullptr && job.beta != 0.f;
     const long long ldp = job.ldp ? job.ldp : job.ldc;
     const bool issuer = (warp == 2 && lane == 0);
     const uint32_t t_s = smem_u32(T);             // the epilogue tile as a shared address
@@ -405,16 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
         const int g4 = 2 * h + (cj >> 3), j = cj & 7;
         const uint32_t pch = t_s + g4 * (kM * 128) + m * 128 + ((j ^ (m & 7)) << 4);
         float4 o = make_float4(acc[4 * cj], acc[4 * cj + 1], acc[4 * cj + 2], acc[4 * cj + 3]);
-        if (!partial) {
-          const float4 cv = read_c ? lds4(pch) : make_float4(0.f, 0.f, 0.f, 0.f);
-          o = make_float4(fmaf(job.alpha, o.x, job.beta * cv.x), fmaf(job.alpha, o.y, job.beta * cv.y),
-                          fmaf(job.alpha, o.z, job.beta * cv.z), fmaf(job.alpha, o.w, job.beta * cv.w));
-        }
+        const float4 cv = read_c ? lds4(pch) : make_float4(0.f, 0.f, 0.f, 0.f);
+        o = make_float4(fmaf(job.alpha, o.x, job.beta * cv.x), fmaf(job.alpha, o.y, job.beta * cv.y),
+                        fmaf(job.alpha, o.z, job.beta * cv.z), fmaf(job.alpha, o.w, job.beta * cv.w));
         sts4(pch, o);
       }
       asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
       if (!failed) {
-        const bool planes = job.C_hi != nullptr && (!job.planes_one_col || it.n0 == job.planes_n0);
+        const bool planes = job.C_hi != nullptr && (!job.planes_one_col || it.n0 == job.planes_n0) &&
+                            (!job.planes_one_row || it.m0 == job.planes_m0);
         const int cn = lane * 4;                  // lane = 16-byte chunk of the row
         const bool col_ok = it.n0 + cn < job.Nlim;
         const int g4 = lane >> 3, j = lane & 7;
@@ -422,15 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
         for (int x = 0; x < 16; ++x) {
           const int mr = ew * 16 + x;
           const float4 o = lds4(t_s + g4 * (kM * 128) + mr * 128 + ((j ^ (mr & 7)) << 4));
-          if (partial) {
-            st4(job.part + (size_t)w * kM * kN + (size_t)mr * kN + cn, o);
-            continue;
-          }
           const int row = it.m0 + mr;
           if (row >= job.Mlim || !col_ok) continue;
           if (job.C) st4(job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + it.n0 + cn, o);
           if (planes) {
-            const long long off = (long long)(job.c_row0 + row) * ldp + job.c_col0 + it.n0 + cn - job.p_col0;
+            const long long off =
+                (long long)(job.c_row0 + row - job.p_row0) * ldp + job.c_col0 + it.n0 + cn - job.p_col0;
             const float4 hv = make_float4(tf32_hi(o.x), tf32_hi(o.y), tf32_hi(o.z), tf32_hi(o.w));
             st4(job.C_hi + off, hv);
             st4(job.C_lo + off, make_float4(o.x - hv.x, o.y - hv.y, o.z - hv.z, o.w - hv.w));
@@ -452,41 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
   __syncthreads();
   if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
-}
-
-// Split partials of a block row -> C = alpha * sum (+ hi/lo planes), in piece order.
-__global__ void __launch_bounds__(256) rowsplit_reduce_kernel(const Job job, const int* info) {
-  if (cta_info_set(info)) return;
-  const int tiles = job.nblk - 1 - job.s;
-  const long long quads = (long long)tiles * (kM * kN / 4);
-  for (long long qd = (long long)blockIdx.x * blockDim.x + threadIdx.x; qd < quads;
-       qd += (long long)gridDim.x * blockDim.x) {
-    const int tile = (int)(qd / (kM * kN / 4));
-    const int e = (int)(qd - (long long)tile * (kM * kN / 4)) * 4;
-    const int m = e / kN, n = e % kN;
-    const int row = job.s * kM + m, col = (job.s + 1 + tile) * kN + n;
-    if (row >= job.Mlim || col >= job.Nlim) continue;
-    const int p0 = split_prefix(tile, job.nsplit), np = tile / job.nsplit + 1;
-    const float* src = job.part + (size_t)p0 * kM * kN + e;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = 0; p < np; ++p) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + (size_t)p * kM * kN));
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    const float o[4] = {job.alpha * acc.x, job.alpha * acc.y, job.alpha * acc.z, job.alpha * acc.w};
-    if (job.C) st4(job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0 + col, make_float4(o[0], o[1], o[2], o[3]));
-    if (job.C_hi) {
-      const long long off = (long long)(job.c_row0 + row) * (job.ldp ? job.ldp : job.ldc) + job.c_col0 + col - job.p_col0;
-      float h4[4], l4[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        h4[t] = tf32_hi(o[t]);
-        l4[t] = o[t] - h4[t];
-      }
-      st4(job.C_hi + off, make_float4(h4[0], h4[1], h4[2], h4[3]));
-      st4(job.C_lo + off, make_float4(l4[0], l4[1], l4[2], l4[3]));
-    }
-  }
 }
 
 // hi/lo planes of a row-major block: rows x cols (cols % 4 == 0).
@@ -560,7 +489,6 @@ bool make_map_c(CUtensorMap* m, const float* p, long long rows, long long cols, 
 
 }  // namespace
 
-int row_items(int tiles, int blocks) { return blocks > 0 ? split_prefix(tiles, blocks) : tiles; }
 
 cudaError_t launch_split(const float* src, long long ld, int rows, int cols, float* hi, float* lo, long long ldo,
                          const int* info, cudaStream_t st) {
@@ -597,18 +525,11 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
   const int ctas = std::min(grid, job.max_ctas > 0 ? std::min(job.max_ctas, kNumSMs) : kNumSMs);
   // C comes in by TMA when it is read (beta != 0); otherwise the map is unused
   CUtensorMap cm = ah;
-  const bool partial = job.mode == 2 && job.nsplit > 0;
-  if (!partial && job.C && job.beta != 0.f &&
+  if (job.C && job.beta != 0.f &&
       !make_map_c(&cm, job.C, (long long)job.c_row0 + job.Mlim, (long long)job.c_col0 + job.Nlim, job.ldc))
     return cudaErrorInvalidValue;
   gemm_tf32x3_kernel<<<ctas, kThreads, kSmem, st>>>(ah, al, bh, bl, job, cm, b_mn ? 1 : 0, grid, info);
   count_launches(1);
-  if (job.mode == 2 && job.nsplit > 0) {
-    const long long quads = (long long)(job.nblk - 1 - job.s) * (kM * kN / 4);
-    const int g = (int)std::min<long long>((quads + 255) / 256, 8 * kNumSMs);
-    rowsplit_reduce_kernel<<<g, 256, 0, st>>>(job, info);
-    count_launches(1);
-  }
   return cudaGetLastError();
 }
 

@@ -18,27 +18,19 @@ struct Operand {
 // What one launch computes; tile sizes are 128 x 128.
 //  mode 0: dense grid of mt x nt tiles, K = kdim.
 //  mode 1: tiles (i, j), i <= j, enumerated column by column from tile t0, K = kdim.
-//  mode 2: tiles (s, s + 1 + t) for t < nblk - 1 - s (one block row of U),
-//          K = [(s+1)*128, min((s+2+t)*128, dlim)); with nsplit > 0 that
-//          range is cut into pieces of nsplit blocks (tile t has
-//          floor(t / nsplit) + 1 of them, items in tile order), whose
-//          partials are then reduced in order.
-//  mode 3: tiles (s, s + 1 + t) for t < nblk - 1 - s, K = [s*128, min((s+1)*128, dlim)).
 // A(m, k) is read at (x = a_x0 + k, y = a_y0 + m0 + m); B(k, n) at
 // (x = b_x0 + k, y = b_y0 + n0 + n) if K-major, (x = b_x0 + n0 + n, y = b_y0 + k)
 // if MN-major. C(m, n) = alpha * acc + beta * C at
 // C[(c_row0 + m0 + m) * ldc + c_col0 + n0 + n] for m0+m < Mlim, n0+n < Nlim
 // (C may be null: no fp32 result). C_hi/C_lo (optional) receive the hi/lo
-// planes of the result at [(c_row0 + m0 + m) * ldp + c_col0 + n0 + n - p_col0]
-// (ldp = 0: ldc), from every tile or, with planes_one_col, only from the
-// tiles whose n0 == planes_n0.
+// planes of the result at [(c_row0 + m0 + m - p_row0) * ldp + c_col0 + n0 + n
+// - p_col0] (ldp = 0: ldc), from every tile or only from the tiles whose
+// n0 == planes_n0 (planes_one_col) and whose m0 == planes_m0 (planes_one_row).
 struct Job {
   int mode;
   int mt, nt;
   int t0;
-  int s, nsplit, nblk;
   int kdim;
-  int dlim;
   int a_x0, a_y0, b_x0, b_y0;
   float* C;
   long long ldc;
@@ -47,16 +39,13 @@ struct Job {
   float* C_hi;
   float* C_lo;
   long long ldp;
-  int p_col0;
+  int p_row0, p_col0;
   int planes_one_col, planes_n0;
-  float* part;
+  int planes_one_row, planes_m0;
   int max_ctas;      // persistent CTAs at most (0: one per SM)
 };
 
 constexpr int kTileTC = 128;
-
-// Items of a mode-2 row of `tiles` tiles split into pieces of `blocks` blocks.
-int row_items(int tiles, int blocks);
 
 cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
                         cudaStream_t st);

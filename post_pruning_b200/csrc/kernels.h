@@ -13,8 +13,6 @@ namespace sgpt {
 
 // factor.cu
 size_t factor_ws_bytes(int d);
-size_t factor_part_tiles(int d);
-int urow_splits(int tiles);
 cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, float* U, void* ws,
                           int* info, cudaStream_t st);
 
