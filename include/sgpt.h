@@ -110,6 +110,13 @@ sgpt_status sgpt_hessian_zero(float* H, int d_in, void* stream);
 sgpt_status sgpt_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tok, int d_in,
                                     void* ws, size_t ws_bytes, int* dev_info, void* stream);
 
+/* H = X^T X: the same sums as sgpt_hessian_zero followed by
+ * sgpt_hessian_accumulate, but H is only written (its old contents are never
+ * read), which saves the zeroing and a read of H. Same arguments and errors
+ * as sgpt_hessian_accumulate; n_tok == 0 gives H = 0. */
+sgpt_status sgpt_hessian_compute(float* H, const uint16_t* X, int64_t n_tok, int d_in,
+                                 void* ws, size_t ws_bytes, int* dev_info, void* stream);
+
 /* U = upper Cholesky factor of H_d^-1, with H_d = (2/n_total) H + lambda I,
  * lambda = damp * mean(diag((2/n_total) H)); H_d^-1 = U^T U, U_ii > 0.
  *   H   [d_in x d_in] fp32, the accumulated X^T X; only the upper triangle

@@ -15,6 +15,7 @@ from .sgpt import (  # noqa: F401
     SgptError,
     factor,
     hessian_accumulate,
+    hessian_compute,
     hessian_zero,
     info_clear,
     kernel_launches,

@@ -107,17 +107,29 @@ sgpt_status sgpt_hessian_zero(float* H, int d_in, void* stream) {
   return from_cuda(cudaMemsetAsync(H, 0, (size_t)d_in * d_in * sizeof(float), as_stream(stream)));
 }
 
-sgpt_status sgpt_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tok, int d_in, void* ws,
-                                    size_t ws_bytes, int* dev_info, void* stream) {
+namespace {
+sgpt_status hessian(float* H, const uint16_t* X, int64_t n_tok, int d_in, void* ws, size_t ws_bytes, int* dev_info,
+                    void* stream, bool set) {
   if (!H || !X || !aligned16(H) || !aligned16(X) || !valid_din(d_in) || n_tok < 0 || !dev_info)
     return SGPT_ERR_INVALID_ARG;
   if (n_tok > (int64_t)INT32_MAX) return SGPT_ERR_INVALID_ARG;   // TMA coordinates are 32-bit
-  if (n_tok == 0) return SGPT_OK;
+  if (n_tok == 0) return set ? sgpt_hessian_zero(H, d_in, stream) : SGPT_OK;
   sgpt_status s = check_ws(ws, ws_bytes, hessian_ws_bytes(d_in, n_tok));
   if (s != SGPT_OK) return s;
-  cudaError_t e = launch_hessian_tc(H, X, n_tok, d_in, ws, dev_info, as_stream(stream));
+  cudaError_t e = launch_hessian_tc(H, X, n_tok, d_in, ws, dev_info, as_stream(stream), set);
   if (e == cudaErrorNotSupported) return SGPT_ERR_UNSUPPORTED;
   return from_cuda(e);
+}
+}  // namespace
+
+sgpt_status sgpt_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tok, int d_in, void* ws,
+                                    size_t ws_bytes, int* dev_info, void* stream) {
+  return hessian(H, X, n_tok, d_in, ws, ws_bytes, dev_info, stream, false);
+}
+
+sgpt_status sgpt_hessian_compute(float* H, const uint16_t* X, int64_t n_tok, int d_in, void* ws,
+                                 size_t ws_bytes, int* dev_info, void* stream) {
+  return hessian(H, X, n_tok, d_in, ws, ws_bytes, dev_info, stream, true);
 }
 
 sgpt_status sgpt_factor(const float* H, int64_t n_total, int d_in, float damp, float* U, void* ws,
@@ -192,10 +204,7 @@ sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint1
   if ((values || meta) && !pack) return SGPT_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
   if ((s = sgpt_info_clear(dev_info, stream)) != SGPT_OK) return s;
-  if (X) {
-    if ((s = sgpt_hessian_zero(H, d_in, stream)) != SGPT_OK) return s;
-    if ((s = sgpt_hessian_accumulate(H, X, n_tok, d_in, ws, ws_bytes, dev_info, stream)) != SGPT_OK) return s;
-  }
+  if (X && (s = sgpt_hessian_compute(H, X, n_tok, d_in, ws, ws_bytes, dev_info, stream)) != SGPT_OK) return s;
   if ((s = sgpt_factor(H, n_tok, d_in, p->damp, U, ws, ws_bytes, dev_info, stream)) != SGPT_OK) return s;
   if (row_loss && cudaMemsetAsync(row_loss, 0, (size_t)d_out * sizeof(float), st) != cudaSuccess)
     return SGPT_ERR_CUDA;

@@ -51,6 +51,8 @@ constexpr long long kWaitCycles = 4000000000ll;   // ~2 s at the B200 boost cloc
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                             ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
 
+constexpr uint32_t kIdesc128 = (kIdesc & ~(0x3fu << 17)) | ((uint32_t)(128 >> 3) << 17);
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -104,11 +106,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+__device__ __forceinline__ void mma_bf16(uint32_t tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -172,12 +175,45 @@ __host__ __device__ inline void grouped_tile(long long t, int tm, int tn, int& t
   }
 }
 
+// Widths with few 128-blocks (K(K+1)/2 <= one CTA per SM) cover the upper
+// triangle with 128 x 128 squares rather than 128 x 256 band tiles, which
+// would compute up to a third of their area below the diagonal. Row block a
+// takes the squares (a, (a + o) mod K) for o = 0, 1, ...: (K+1)/2 of them
+// for odd K; for even K, K/2 + 1 for a < K/2 and K/2 for the others. That
+// is every unordered pair {a, c} exactly once; a square with c < a holds
+// the transpose of the upper square (c, a). Then rows with an odd count are
+// taken two at a time and the one square they share moves to the other
+// row, which leaves at most one odd row. Consecutive squares of a row share
+// the row block's A and make one 128 x 256 tile (B = column blocks c1 and
+// c2, which need not be adjacent); the one odd square left is a 128 x 128
+// tile, which takes about as long per token as a full one. Every tile gets
+// the same number of token splits, and each CTA writes its partial sums for
+// the reduction kernel.
+constexpr int kMaxPairCtas = 148;
+struct PairWork {
+  unsigned char a, c1, c2, nsq;   // row block, column blocks of the one or two squares
+  int t0, t1;                     // token range
+};
+struct PairTile {
+  unsigned char a, c1, c2, nsq;
+  short first, ns;                // CTAs first .. first + ns - 1, in token order
+};
+struct PairWorks {
+  int ncta;                       // 0: band tiles instead
+  PairWork w[kMaxPairCtas];
+};
+struct PairTiles {
+  int ntiles;
+  PairTile t[kMaxPairCtas];
+};
+
 }  // namespace
 
 // H[i][j] += S[r][c] and, for j != i, H[j][i] += S[r][c] over the upper
 // part (j >= i) of the 64 x 64 block at rows i0.., columns j0.. (S in shared
-// memory, row stride ld). Both passes are coalesced: rows of H along c,
-// then the mirrored rows along r (a column of S).
+// memory, element (r, c) at r * rs + c * cs: a transposed view passes the
+// strides swapped). Both passes are coalesced: rows of H along c, then the
+// mirrored rows along r (a column of S).
 constexpr int kSLd = 65;
 constexpr int kTileLd = kN + 1;
 __device__ __forceinline__ float lds1(uint32_t addr) {
@@ -187,32 +223,52 @@ __device__ __forceinline__ float lds1(uint32_t addr) {
 }
 // (S is a 32-bit shared-memory address: the staging area may have been
 // aligned through an integer, which hides its address space from the compiler)
-__device__ void flush_block(uint32_t S, int ld, int i0, int j0, float* __restrict__ H, int d, int t, int nt) {
+__device__ void flush_block(uint32_t S, int rs, int cs, int i0, int j0, float* __restrict__ H, int d, int t,
+                            int nt, bool set) {
+  // d is a multiple of 32 and every group starts at a multiple of 4, so a
+  // group that starts inside H ends inside it; groups wholly on one side of
+  // the diagonal go as one 16-byte access (a store when `set`: H = the sum
+  // instead of H += the sum)
   for (int q = t; q < 64 * 16; q += nt) {
-    const int r = q >> 4, c4 = (q & 15) * 4, i = i0 + r;
-    if (i >= d) continue;
-    const long long row = (long long)i * d;
+    const int r = q >> 4, c4 = (q & 15) * 4, i = i0 + r, j = j0 + c4;
+    if (i >= d || j >= d || j + 3 < i) continue;
+    float v[4];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int j = j0 + c4 + x;
-      if (j >= i && j < d) H[row + j] += lds1(S + 4u * (uint32_t)(r * ld + c4 + x));
+    for (int x = 0; x < 4; ++x) v[x] = lds1(S + 4u * (uint32_t)(r * rs + (c4 + x) * cs));
+    float* p = H + (long long)i * d + j;
+    if (j >= i) {
+      float4 h = set ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<float4*>(p);
+      h.x += v[0]; h.y += v[1]; h.z += v[2]; h.w += v[3];
+      *reinterpret_cast<float4*>(p) = h;
+    } else {
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        if (j + x >= i) p[x] = (set ? 0.f : p[x]) + v[x];
     }
   }
   for (int q = t; q < 64 * 16; q += nt) {
-    const int c = q >> 4, r4 = (q & 15) * 4, j = j0 + c;
-    if (j >= d) continue;
-    const long long row = (long long)j * d;
+    const int c = q >> 4, r4 = (q & 15) * 4, j = j0 + c, i = i0 + r4;
+    if (j >= d || i >= d || i >= j) continue;
+    float v[4];
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int i = i0 + r4 + x;
-      if (i < j && i < d) H[row + i] += lds1(S + 4u * (uint32_t)((r4 + x) * ld + c));
+    for (int x = 0; x < 4; ++x) v[x] = lds1(S + 4u * (uint32_t)((r4 + x) * rs + c * cs));
+    float* p = H + (long long)j * d + i;
+    if (i + 3 < j) {
+      float4 h = set ? make_float4(0.f, 0.f, 0.f, 0.f) : *reinterpret_cast<float4*>(p);
+      h.x += v[0]; h.y += v[1]; h.z += v[2]; h.w += v[3];
+      *reinterpret_cast<float4*>(p) = h;
+    } else {
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        if (i + x < j) p[x] = (set ? 0.f : p[x]) + v[x];
     }
   }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int d, long long n,
-    int nsplit, long long per, float* __restrict__ part, int* info) {
+    int nsplit, long long per, float* __restrict__ part, int* info, const __grid_constant__ PairWorks pw,
+    int set) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -221,12 +277,28 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   __shared__ int failed;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x / nsplit, split = blockIdx.x - (blockIdx.x / nsplit) * nsplit;
-  int ti, tj;
-  grouped_tile(tile, (d + kM - 1) / kM, (d + kN - 1) / kN, ti, tj);
-  const int i0 = ti * kM, j0 = tj * kN;
-  const long long t_begin = (long long)split * per;
-  const long long t_end = t_begin + per < n ? t_begin + per : n;
+  const bool paired = pw.ncta > 0;
+  int i0, j1, j2, nsq = 2;                    // row channels; B = channels j1.. and j2.. (128 each)
+  long long t_begin, t_end;
+  if (paired) {
+    const PairWork wk = pw.w[blockIdx.x];
+    i0 = wk.a * kM;
+    nsq = wk.nsq;
+    j1 = wk.c1 * kM;
+    j2 = wk.c2 * kM;
+    t_begin = wk.t0;
+    t_end = wk.t1;
+  } else {
+    const int tile = blockIdx.x / nsplit, split = blockIdx.x - (blockIdx.x / nsplit) * nsplit;
+    int ti, tj;
+    grouped_tile(tile, (d + kM - 1) / kM, (d + kN - 1) / kN, ti, tj);
+    i0 = ti * kM;
+    j1 = tj * kN;
+    j2 = j1 + 128;
+    t_begin = (long long)split * per;
+    t_end = t_begin + per < n ? t_begin + per : n;
+  }
+  const int j0 = j1;
   const int iters = (int)((t_end - t_begin + kBK - 1) / kBK);
   const int nchunks = (iters + kChunkIters - 1) / kChunkIters;
 
@@ -277,13 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
         break;
       }
       const uint32_t bar = full0 + 8 * s;
-      mbar_expect_tx(bar, kStageBytes);
+      mbar_expect_tx(bar, kAStage + 2 * nsq * kBox);
       const int y = (int)(t_begin + (long long)it * kBK);
       const uint32_t a = s0 + s * kStageBytes, b = a + kAStage;
       tma_load_2d(a, &xmap, bar, i0, y);
       tma_load_2d(a + kBox, &xmap, bar, i0 + 64, y);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tma_load_2d(b + c * kBox, &xmap, bar, j0 + 64 * c, y);
+      for (int c = 0; c < 4; ++c)
+        if (c < 2 * nsq) tma_load_2d(b + c * kBox, &xmap, bar, (c < 2 ? j1 : j2) + 64 * (c & 1), y);
       ++issued;
     }
     // never leave with copies in flight: wait for every stage that was armed
@@ -291,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
   } else if (!skip && warp == 1 && lane == 0) {
     // MMA issuer: chunk c accumulates kChunkIters stages into buffer c & 1
+    const uint32_t idesc = nsq == 2 ? kIdesc : kIdesc128;
     for (int c = 0; c < nchunks && !failed; ++c) {
       const int b = c & 1;
       if (c >= 2 && !mbar_wait(tempty0 + 8 * b, ((c >> 1) - 1) & 1)) {
@@ -310,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
         const uint32_t a = s0 + s * kStageBytes, bb = a + kAStage;
 #pragma unroll
         for (int ks = 0; ks < kBK / 16; ++ks)
-          mma_bf16(acc_t, mn_desc(a + ks * 2048), mn_desc(bb + ks * 2048), (it != c * kChunkIters) || ks != 0);
+          mma_bf16(acc_t, mn_desc(a + ks * 2048), mn_desc(bb + ks * 2048), idesc,
+                   (it != c * kChunkIters) || ks != 0);
         mma_commit(empty0 + 8 * s);
       }
       mma_commit(tfull0 + 8 * b);
@@ -325,13 +400,15 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kN + h * 128);
+      if (h < nsq) {                          // a one-square tile has no second half
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld32_nowait(base + cc * 32, v);
-        tmem_wait_ld();
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tmem_ld32_nowait(base + cc * 32, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) acc[cc * 32 + e] += __uint_as_float(v[e]);
+          for (int e = 0; e < 32; ++e) acc[cc * 32 + e] += __uint_as_float(v[e]);
+        }
       }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
@@ -345,13 +422,13 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   if (!skip && !failed && warp >= 2) {
     const int r = q * 32 + lane;              // tile row
     const int i = i0 + r;
-    if (nsplit > 1) {
+    if (paired || nsplit > 1) {
       float* dst = part + (size_t)blockIdx.x * kM * kN + (size_t)r * kN + h * 128;
 #pragma unroll
       for (int e = 0; e < 128; e += 4) st4(dst + e, make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]));
     }
   }
-  if (!skip && !failed && nsplit == 1 && warp >= 2) {
+  if (!skip && !failed && !paired && nsplit == 1 && warp >= 2) {
     // H += tile (and its mirror) through shared memory, by the epilogue
     // warps (named barrier 1): the whole tile is staged in the stage buffers,
     // free now that every MMA has completed, then flushed 64 x 64 at a time
@@ -366,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       const int br = blk / (kN / 64), bc = blk % (kN / 64);
       const int bi0 = i0 + 64 * br, bj0 = j0 + 64 * bc;
       if (bi0 < d && bj0 < d && bj0 + 63 >= bi0)  // the block meets the upper triangle
-        flush_block(S + 4u * (uint32_t)((64 * br) * kTileLd + 64 * bc), kTileLd, bi0, bj0, H, d, et, 256);
+        flush_block(S + 4u * (uint32_t)((64 * br) * kTileLd + 64 * bc), kTileLd, 1, bi0, bj0, H, d, et, 256,
+                    set != 0);
     }
   }
   __syncthreads();
@@ -380,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
 constexpr int kReduceThreads = 1024;
 __global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const float* __restrict__ part,
                                                                         float* __restrict__ H, int d, int tiles,
-                                                                        int nsplit, const int* info) {
+                                                                        int nsplit, const int* info, int set) {
   if (cta_info_set(info)) return;
   __shared__ float S[64 * kSLd];
   const int tn = (d + kN - 1) / kN;
@@ -410,7 +488,53 @@ __global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const fl
     S[r * kSLd + c4 + 2] = acc.z;
     S[r * kSLd + c4 + 3] = acc.w;
     __syncthreads();
-    flush_block(smem_u32(S), kSLd, bi0, bj0, H, d, t, kReduceThreads);
+    flush_block(smem_u32(S), kSLd, 1, bi0, bj0, H, d, t, kReduceThreads, set != 0);
+    __syncthreads();
+  }
+}
+
+// Square tiles' partials -> H: one CTA per 64 x 64 block of a square
+// (four per square; the lower one of a diagonal square holds nothing
+// needed), summing the tile's partials in token order, then adding the sum
+// to H and its mirror; a square below the diagonal is flushed through its
+// transposed view, which lies above it.
+__global__ void __launch_bounds__(kReduceThreads) hessian_pair_reduce_kernel(const float* __restrict__ part,
+                                                                             float* __restrict__ H, int d,
+                                                                             const __grid_constant__ PairTiles pt,
+                                                                             const int* info, int set) {
+  if (cta_info_set(info)) return;
+  __shared__ float S[64 * kSLd];
+  const int t = threadIdx.x, r = t >> 4, c4 = (t & 15) * 4;
+  for (int gb = blockIdx.x;; gb += gridDim.x) {
+    int ti = 0, base = 0;
+    while (ti < pt.ntiles && gb >= base + 4 * pt.t[ti].nsq) base += 4 * pt.t[ti++].nsq;
+    if (ti >= pt.ntiles) break;                                // block-uniform
+    const PairTile tl = pt.t[ti];
+    const int blk = gb - base, sq = blk >> 2, br = (blk >> 1) & 1, bc = blk & 1;
+    const int a = tl.a, c = sq ? tl.c2 : tl.c1;
+    const int bi0 = a * kM + 64 * br, bj0 = c * kM + 64 * bc;
+    if (bi0 >= d || bj0 >= d || (c == a && br > bc)) continue;   // block-uniform
+    const float* src = part + (size_t)tl.first * kM * kN + (size_t)(64 * br + r) * kN + 128 * sq + 64 * bc + c4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < tl.ns; p0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int pp = 0; pp < 8; ++pp)
+        v[pp] = (p0 + pp < tl.ns) ? __ldcs(reinterpret_cast<const float4*>(src + (size_t)(p0 + pp) * kM * kN))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int pp = 0; pp < 8; ++pp)
+        if (p0 + pp < tl.ns) {
+          acc.x += v[pp].x; acc.y += v[pp].y; acc.z += v[pp].z; acc.w += v[pp].w;
+        }
+    }
+    S[r * kSLd + c4] = acc.x;
+    S[r * kSLd + c4 + 1] = acc.y;
+    S[r * kSLd + c4 + 2] = acc.z;
+    S[r * kSLd + c4 + 3] = acc.w;
+    __syncthreads();
+    if (c >= a) flush_block(smem_u32(S), kSLd, 1, bi0, bj0, H, d, t, kReduceThreads, set != 0);
+    else flush_block(smem_u32(S), 1, kSLd, bj0, bi0, H, d, t, kReduceThreads, set != 0);
     __syncthreads();
   }
 }
@@ -438,9 +562,84 @@ EncodeTiledFn encode_fn() {
 struct Plan {
   int tiles, nsplit;
   long long per;
+  PairWorks pw;     // pw.ncta > 0: square tiles (then tiles/nsplit/per are unused)
+  PairTiles pt;
+  int pair_blocks;  // 64 x 64 blocks of the squares, for the reduction
 };
 
+// Square tiles for widths of at most K(K+1)/2 <= kMaxPairCtas squares (see
+// PairWork): returns false otherwise.
+bool plan_pairs(int d, long long n, Plan& p) {
+  const int K = (d + kM - 1) / kM;
+  const int squares = K * (K + 1) / 2;
+  if (squares > kMaxPairCtas) return false;
+  // each row block's squares: list[a][0..cnt[a]), column blocks
+  static_assert(kMaxPairCtas < 256, "block numbers are bytes");
+  constexpr int kMaxK = 17;                        // K(K+1)/2 <= 148
+  unsigned char list[kMaxK][kMaxK + 1];
+  int cnt[kMaxK];
+  for (int a = 0; a < K; ++a) {
+    cnt[a] = (K & 1) ? (K + 1) / 2 : (a < K / 2 ? K / 2 + 1 : K / 2);
+    for (int o = 0; o < cnt[a]; ++o) list[a][o] = (unsigned char)((a + o) % K);
+  }
+  int odd = -1;
+  for (int a = 0; a < K; ++a) {
+    if (!(cnt[a] & 1)) continue;
+    if (odd < 0) {
+      odd = a;
+      continue;
+    }
+    // rows odd and a share the square {odd, a}: move it to the other one
+    const int b = odd;
+    odd = -1;
+    int from = -1, at = -1;
+    for (int o = 0; o < cnt[b] && from < 0; ++o)
+      if (list[b][o] == a && a != b) from = b, at = o;
+    for (int o = 0; o < cnt[a] && from < 0; ++o)
+      if (list[a][o] == b) from = a, at = o;
+    const int to = from == a ? b : a;
+    list[to][cnt[to]++] = (unsigned char)(from == a ? a : b);
+    for (int o = at; o + 1 < cnt[from]; ++o) list[from][o] = list[from][o + 1];
+    --cnt[from];
+  }
+  int ntiles = 0;
+  for (int a = 0; a < K; ++a) ntiles += (cnt[a] + 1) / 2;
+  const int s = std::max(1, kMaxPairCtas / ntiles);   // splits per tile
+  long long per = ((n + s - 1) / s + kBK - 1) / kBK * kBK;
+  per = std::max<long long>(per, 4 * kBK);             // >= 4 stages per split
+  const int ns = (int)((n + per - 1) / per);
+  p.pw.ncta = 0;
+  p.pt.ntiles = 0;
+  p.pair_blocks = 0;
+  for (int a = 0; a < K; ++a) {
+    for (int o = 0; o < cnt[a]; o += 2) {
+      PairTile tl;
+      tl.a = (unsigned char)a;
+      tl.c1 = list[a][o];
+      tl.nsq = (unsigned char)(o + 1 < cnt[a] ? 2 : 1);
+      tl.c2 = tl.nsq == 2 ? list[a][o + 1] : tl.c1;
+      tl.first = (short)p.pw.ncta;
+      tl.ns = (short)ns;
+      for (int sp = 0; sp < ns; ++sp) {
+        PairWork& w = p.pw.w[p.pw.ncta++];
+        w.a = tl.a;
+        w.c1 = tl.c1;
+        w.c2 = tl.c2;
+        w.nsq = tl.nsq;
+        w.t0 = (int)(sp * per);
+        w.t1 = (int)std::min<long long>(n, (sp + 1) * per);
+      }
+      p.pt.t[p.pt.ntiles++] = tl;
+      p.pair_blocks += 4 * tl.nsq;
+    }
+  }
+  return true;
+}
+
 Plan plan(int d, long long n) {
+  Plan p{};
+  if (plan_pairs(d, n, p)) return p;
+  p.pw.ncta = 0;
   const int tm = (d + kM - 1) / kM, tn = (d + kN - 1) / kN;
   const int tiles = (int)band_start(tm, tn);
   // split tokens when the tiles alone cannot fill the GPU, keeping the grid
@@ -451,7 +650,15 @@ Plan plan(int d, long long n) {
   ns = std::max<long long>(1, std::min(ns, max_split));
   long long per = ((n + ns - 1) / ns + kBK - 1) / kBK * kBK;
   ns = (n + per - 1) / per;
-  return {tiles, (int)std::max<long long>(1, ns), per};
+  p.tiles = tiles;
+  p.nsplit = (int)std::max<long long>(1, ns);
+  p.per = per;
+  return p;
+}
+
+size_t part_floats(const Plan& p) {
+  if (p.pw.ncta > 0) return (size_t)p.pw.ncta * kM * kN;
+  return p.nsplit > 1 ? (size_t)p.tiles * p.nsplit * kM * kN : 0;
 }
 
 }  // namespace
@@ -459,18 +666,18 @@ Plan plan(int d, long long n) {
 size_t hessian_ws_bytes(int d, long long n) {
   const Plan p = plan(d, n);
   Carve c(nullptr);
-  if (p.nsplit > 1) c.take<float>((size_t)p.tiles * p.nsplit * kM * kN);
+  if (part_floats(p)) c.take<float>(part_floats(p));
   return c.off + 256;
 }
 
 cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, void* ws, int* info,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool set) {
   if (n <= 0) return cudaSuccess;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const Plan p = plan(d, n);
   Carve c(ws);
-  float* part = p.nsplit > 1 ? c.take<float>((size_t)p.tiles * p.nsplit * kM * kN) : nullptr;
+  float* part = part_floats(p) ? c.take<float>(part_floats(p)) : nullptr;
 
 
   CUtensorMap map;
@@ -487,11 +694,15 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
     cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     attr = true;
   }
-  hessian_tc_kernel<<<p.tiles * p.nsplit, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info);
+  const int grid = p.pw.ncta > 0 ? p.pw.ncta : p.tiles * p.nsplit;
+  hessian_tc_kernel<<<grid, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info, p.pw, set ? 1 : 0);
   count_launches(1);
-  if (p.nsplit > 1) {
+  if (p.pw.ncta > 0) {
+    hessian_pair_reduce_kernel<<<p.pair_blocks, kReduceThreads, 0, st>>>(part, H, d, p.pt, info, set ? 1 : 0);
+    count_launches(1);
+  } else if (p.nsplit > 1) {
     const int g = (int)std::min<long long>((long long)p.tiles * 8, 8 * kNumSMs);
-    hessian_reduce_kernel<<<g, kReduceThreads, 0, st>>>(part, H, d, p.tiles, p.nsplit, info);
+    hessian_reduce_kernel<<<g, kReduceThreads, 0, st>>>(part, H, d, p.tiles, p.nsplit, info, set ? 1 : 0);
     count_launches(1);
   }
   return cudaGetLastError();

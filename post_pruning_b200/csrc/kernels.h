@@ -34,6 +34,6 @@ cudaError_t launch_recon(const float* W0, const float* W, int rows, int d, long 
 // hessian_tc.cu
 size_t hessian_ws_bytes(int d, long long n);
 cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, void* ws, int* info,
-                              cudaStream_t st);
+                              cudaStream_t st, bool set);
 
 }  // namespace sgpt

@@ -30,7 +30,7 @@ PATTERN_NM = 1
 EXPORTS = (
     "sgpt_status_string", "sgpt_abi_version", "sgpt_kernel_launches", "sgpt_workspace_bytes",
     "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
-    "sgpt_hessian_accumulate", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
+    "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
     "sgpt_recon_error", "sgpt_prune_layer",
 )
 
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
         "sgpt_sync_status": (i32, [vp, vp]),
         "sgpt_hessian_zero": (i32, [vp, i32, vp]),
         "sgpt_hessian_accumulate": (i32, [vp, vp, i64, i32, vp, sz, vp, vp]),
+        "sgpt_hessian_compute": (i32, [vp, vp, i64, i32, vp, sz, vp, vp]),
         "sgpt_factor": (i32, [vp, i64, i32, ctypes.c_float, vp, vp, sz, vp, vp]),
         "sgpt_prune": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, sz, vp, vp]),
         "sgpt_prune_noalloc": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, vp]),
@@ -190,6 +191,18 @@ def hessian_accumulate(H: torch.Tensor, X: torch.Tensor, ws: torch.Tensor, dev_i
         raise ValueError("H must be [d, d] and X [n, d], both contiguous")
     _check(lib().sgpt_hessian_accumulate(_ptr(H), _ptr(X), X.shape[0], d, _ptr(ws), ws.numel(),
                                          _ptr(dev_info), _stream(stream)), "sgpt_hessian_accumulate")
+
+
+def hessian_compute(H: torch.Tensor, X: torch.Tensor, ws: torch.Tensor, dev_info: torch.Tensor, stream=None):
+    """H = X^T X (sgpt_hessian_compute): like hessian_zero + hessian_accumulate
+    without reading H."""
+    _dev(H, torch.float32, "H")
+    _dev(X, torch.bfloat16, "X")
+    d = H.shape[0]
+    if H.shape != (d, d) or not H.is_contiguous() or X.dim() != 2 or X.shape[1] != d or not X.is_contiguous():
+        raise ValueError("H must be [d, d] and X [n, d], both contiguous")
+    _check(lib().sgpt_hessian_compute(_ptr(H), _ptr(X), X.shape[0], d, _ptr(ws), ws.numel(),
+                                      _ptr(dev_info), _stream(stream)), "sgpt_hessian_compute")
 
 
 def factor(H: torch.Tensor, n_total: int, damp: float, U: torch.Tensor, ws: torch.Tensor,
@@ -346,7 +359,7 @@ class LayerBuffers:
 class LayerGraphs:
     """The four phases of one layer prune captured as CUDA graphs.
 
-    hessian (zero + accumulate), factor, prune (row loss cleared + sweep) and,
+    hessian (H = X^T X), factor, prune (row loss cleared + sweep) and,
     for 2:4, pack. Replaying them in order does exactly what
     LayerBuffers.run does, with the launch overhead of one graph per phase.
     Capture reads no data: buffers are bound by address, so W and X must
@@ -377,8 +390,7 @@ class LayerGraphs:
         b, p = self.bufs, self.params
         if name == "hessian":
             info_clear(b.info)
-            hessian_zero(b.H)
-            hessian_accumulate(b.H, self.X, b.ws, b.info)
+            hessian_compute(b.H, self.X, b.ws, b.info)
         elif name == "factor":
             factor(b.H, b.n_tok, p.damp, b.U, b.ws, b.info)
         elif name == "prune":

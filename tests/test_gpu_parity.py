@@ -67,12 +67,14 @@ def test_hessian_matches_oracle(spec):
     assert np.all(np.abs(H2.cpu().numpy() - ref) <= 1e-5 * absref + 1e-30)
 
 
-@pytest.mark.parametrize("d", [2592, 4192])
-def test_hessian_super_block_order(d):
-    """Widths whose tiles span several 2048-channel super-blocks, with ragged
-    last super-blocks: 2592 (131 tiles, token-split, so the reduction decodes
-    the same tile order) and 4192 (305 tiles, unsplit). Every element of H is
-    compared with the float64 sum."""
+@pytest.mark.parametrize("d", [1440, 2592, 4192])
+def test_hessian_tile_orders(d):
+    """Each tiling of the Hessian, every element of H against the float64
+    sum: 1440 (12 blocks with a 32-wide last one: 78 square tiles of up to
+    two 128 x 128 squares, some below the diagonal, one token split per
+    square); 2592 and 4192, whose band tiles span several 2048-channel
+    super-blocks with ragged last ones (131 tiles, token-split, so the
+    reduction decodes the same tile order; 305 tiles, unsplit)."""
     spec = LayerSpec("wide", d_in=d, d_out=16, n_tok=1000, seed=7)
     dev = torch.device("cuda")
     X = gen_activations(spec, device="cpu")
@@ -86,6 +88,11 @@ def test_hessian_super_block_order(d):
     Hg = H.cpu().numpy().astype(np.float64)
     assert np.array_equal(Hg, Hg.T)
     assert np.all(np.abs(Hg - ref) <= 1e-5 * absref + 1e-30)
+    # H = X^T X without reading H: the same bits over any old contents
+    H2 = torch.full_like(H, float("nan"))
+    pp.hessian_compute(H2, X.to(dev), pp.workspace(spec.d_out, d, spec.n_tok), info)
+    pp.raise_on_info(info)
+    assert torch.equal(H2, H)
 
 
 # ------------------------------------------------------------ factor
