@@ -585,10 +585,10 @@ namespace {
 // The factorisation's internal streams (per device): the critical chain
 // diag(k) -> chain step(k) -> diag(k-1) on `crit`; the panel product of
 // the rows above and the update of block column k-1 on `pan`; the rest of
-// each trailing update on `upd`; the V and U block rows, which nothing in
-// the chain waits for, on `rows`. They fork from and join back to the
-// caller's stream, so the whole factorisation is ordered on it (and
-// captures into one graph).
+// each trailing update on `upd`; the block rows of U and the sums T they
+// come from, which nothing in the chain waits for, on `rows`. They fork
+// from and join back to the caller's stream, so the whole factorisation is
+// ordered on it (and captures into one graph).
 struct FactorStreams {
   cudaStream_t crit = nullptr, pan = nullptr, upd = nullptr, rows = nullptr;
   cudaEvent_t fork = nullptr, diag_done = nullptr, chain_done = nullptr, panel_done = nullptr,

@@ -121,10 +121,11 @@ def test_factor_matches_oracle(spec):
     assert torch.equal(Hd, U)
 
 
-# 17 column blocks with a 32-wide last one: the block-column loop runs its
-# rank-128 updates, V and U block rows on internal streams and joins them
-# back to the caller's stream, so check it eager, on a side stream behind a
-# pending producer, and captured in a CUDA graph.
+# 17 column blocks with a 32-wide last one (paired updates from 16 block
+# columns on): the block-column loop runs its panels, rank-128 updates, sums
+# T and block rows of U on internal streams and joins them back to the
+# caller's stream, so check it eager, on a side stream behind a pending
+# producer, and captured in a CUDA graph.
 WIDE = LayerSpec("wide_2080", d_in=2080, d_out=64, n_tok=4096, sigma=1.5, seed=11)
 
 
