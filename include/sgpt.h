@@ -56,7 +56,7 @@ typedef enum sgpt_status {
   SGPT_ERR_NONFINITE = 3,   /* NaN/Inf met in H, U or W                    */
   SGPT_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up          */
   SGPT_ERR_CUDA = 5,        /* a CUDA runtime call failed                  */
-  SGPT_ERR_UNSUPPORTED = 6, /* valid request this build does not implement */
+  SGPT_ERR_UNSUPPORTED = 6, /* valid request this library version does not implement */
   SGPT_ERR_BAD_MASK = 7,    /* pack: a group does not keep exactly 2 of 4  */
   SGPT_ERR_WORKSPACE = 8    /* ws too small or misaligned                  */
 } sgpt_status;

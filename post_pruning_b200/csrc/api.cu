@@ -64,7 +64,7 @@ const char* sgpt_status_string(sgpt_status s) {
     case SGPT_ERR_NONFINITE: return "non-finite value";
     case SGPT_ERR_TIMEOUT: return "device-side wait timed out";
     case SGPT_ERR_CUDA: return "CUDA runtime error";
-    case SGPT_ERR_UNSUPPORTED: return "unsupported by this build";
+    case SGPT_ERR_UNSUPPORTED: return "not supported by this library version";
     case SGPT_ERR_BAD_MASK: return "mask breaks the 2:4 pattern";
     case SGPT_ERR_WORKSPACE: return "workspace too small or misaligned";
   }
