@@ -62,12 +62,18 @@ __global__ void __launch_bounds__(1024) damp_lambda_kernel(const float* __restri
 }
 
 // R[i][j] = scale * H[i][j] (+ lam on the diagonal), upper triangle only.
+// In the same pass: zero row i of U_zero (when given: the output, which
+// then holds the sums T from zero), and for rows above column block col0
+// (>= 0) write the hi/lo planes of R[i][col0..] that the first panel reads.
 __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict__ R, int d,
-                                  double scale, const double* __restrict__ lam, const int* info) {
+                                  double scale, const double* __restrict__ lam, const int* info,
+                                  float* __restrict__ U_zero, float* __restrict__ A_hi,
+                                  float* __restrict__ A_lo, int col0) {
   if (cta_info_set(info)) return;
   const int i = blockIdx.y;
   const double l = *lam;
   for (int j4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4; j4 < d; j4 += gridDim.x * blockDim.x * 4) {
+    if (U_zero) st4(U_zero + (long long)i * d + j4, make_float4(0.f, 0.f, 0.f, 0.f));
     if (j4 + 3 < i) continue;
     const float4 h = ld4(H + (long long)i * d + j4);
     float v[4] = {h.x, h.y, h.z, h.w};
@@ -78,6 +84,12 @@ __global__ void scale_damp_kernel(const float* __restrict__ H, float* __restrict
       v[t] = (float)x;
     }
     st4(R + (long long)i * d + j4, make_float4(v[0], v[1], v[2], v[3]));
+    if (col0 >= 0 && i < col0 && j4 >= col0) {
+      const float4 h = make_float4(tf32_hi(v[0]), tf32_hi(v[1]), tf32_hi(v[2]), tf32_hi(v[3]));
+      const long long off = (long long)i * kTile + (j4 - col0);
+      st4(A_hi + off, h);
+      st4(A_lo + off, make_float4(v[0] - h.x, v[1] - h.y, v[2] - h.z, v[3] - h.w));
+    }
   }
 }
 
@@ -831,16 +843,15 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
   cudaError_t e = factor_streams(&f);
   if (e != cudaSuccess) return e;
   const double scale = 2.0 / (double)n_total;
-  if (U != H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
   damp_lambda_kernel<<<1, 1024, 0, st>>>(H, d, scale, (double)damp, w.lam, info);
   count_launches(1);
-  scale_damp_kernel<<<dim3(cdiv(d, 4 * 128), d), 128, 0, st>>>(H, w.R, d, scale, w.lam, info);
-  count_launches(1);
-  if (U == H) cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st);
+  // scaled, damped H into R; U zeroed in the same pass unless it is H; the
   // planes of the last column block above its diagonal block
-  if (K > 1 && (e = tc::launch_split(w.R + (K - 1) * kTile, d, (K - 1) * kTile, d - (K - 1) * kTile, w.A_hi,
-                                     w.A_lo, kTile, info, st)) != cudaSuccess)
-    return e;
+  scale_damp_kernel<<<dim3(cdiv(d, 4 * 128), d), 128, 0, st>>>(H, w.R, d, scale, w.lam, info,
+                                                               U != H ? U : nullptr, w.A_hi, w.A_lo,
+                                                               K > 1 ? (K - 1) * kTile : -1);
+  count_launches(1);
+  if (U == H && (e = cudaMemsetAsync(U, 0, (size_t)d * d * sizeof(float), st)) != cudaSuccess) return e;
   if ((e = cudaEventRecord(f->fork, st)) != cudaSuccess) return e;
   for (cudaStream_t s : {f->crit, f->pan, f->upd, f->rows})
     if ((e = cudaStreamWaitEvent(s, f->fork, 0)) != cudaSuccess) return e;
