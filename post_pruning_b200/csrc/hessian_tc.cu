@@ -421,7 +421,6 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   if (failed && threadIdx.x == 0) set_info(info, SGPT_INFO_TIMEOUT);
   if (!skip && !failed && warp >= 2) {
     const int r = q * 32 + lane;              // tile row
-    const int i = i0 + r;
     if (paired || nsplit > 1) {
       float* dst = part + (size_t)blockIdx.x * kM * kN + (size_t)r * kN + h * 128;
 #pragma unroll
