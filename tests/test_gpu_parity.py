@@ -121,6 +121,26 @@ def test_factor_matches_oracle(spec):
     assert torch.equal(Hd, U)
 
 
+@pytest.mark.parametrize("d", [1920, 2048])
+def test_factor_pairing_boundary(d):
+    """15 block columns (the widest factorisation whose updates go step by
+    step) and 16 (the narrowest that pairs them), against the oracle."""
+    spec = LayerSpec(f"pair_{d}", d_in=d, d_out=64, n_tok=2 * d, sigma=1.5, seed=17)
+    X64 = bf16_bits_to_f64(gen_activations(spec)).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)
+    _, U_ref = _oracle_factor(Hs, spec.n_tok)
+    dev = torch.device("cuda")
+    Hd = torch.from_numpy(Hs).to(dev)
+    U = torch.empty_like(Hd)
+    info = pp.new_info()
+    pp.factor(Hd, spec.n_tok, 0.01, U, pp.workspace(spec.d_out, d), info)
+    pp.raise_on_info(info)
+    Ug = U.cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(Ug, -1) == 0) and np.all(np.diag(Ug) > 0)
+    rel_rows = np.linalg.norm(Ug - U_ref, axis=1) / np.linalg.norm(U_ref, axis=1)
+    assert rel_rows.max() < 1e-4, rel_rows.max()
+
+
 # 17 column blocks with a 32-wide last one (paired updates from 16 block
 # columns on): the block-column loop runs its panels, rank-128 updates, sums
 # T and block rows of U on internal streams and joins them back to the
