@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/sgpt.h"
 
 namespace sgpt {
@@ -75,6 +77,27 @@ __device__ __forceinline__ float tf32_hi(float x) {
 
 // Host-side count of kernel launches (diagnostics, sgpt_kernel_launches).
 void count_launches(unsigned long long n);
+
+// One-time setup per device (kernel attributes such as the dynamic
+// shared-memory limit belong to the current device's context): runs `f` the
+// first time it is called for the current device, under a lock, and again
+// later if it failed.
+struct PerDevice {
+  std::mutex mu;
+  bool done[64] = {};
+};
+template <class F>
+cudaError_t once_per_device(PerDevice& pd, F&& f) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return f();
+  std::lock_guard<std::mutex> lock(pd.mu);
+  if (pd.done[dev]) return cudaSuccess;
+  e = f();
+  if (e == cudaSuccess) pd.done[dev] = true;
+  return e;
+}
 
 // Host-side workspace carving: consecutive 256-byte aligned sub-buffers.
 struct Carve {

@@ -833,14 +833,17 @@ cudaError_t launch_factor(const float* H, long long n_total, int d, float damp, 
   const int K = cdiv(d, kTile);
   const FactorWs w = carve_factor(ws, d, nullptr);
   std::lock_guard<std::mutex> lock(g_streams_mu);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(diag_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDiagSmem);
-    cudaFuncSetAttribute(chain_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChainSmem);
-    attr_done = true;
-  }
+  static PerDevice attrs;
+  cudaError_t e = once_per_device(attrs, [] {
+    cudaError_t r = cudaFuncSetAttribute(diag_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kDiagSmem);
+    return r != cudaSuccess ? r
+                            : cudaFuncSetAttribute(chain_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)kChainSmem);
+  });
+  if (e != cudaSuccess) return e;
   FactorStreams* f = nullptr;
-  cudaError_t e = factor_streams(&f);
+  e = factor_streams(&f);
   if (e != cudaSuccess) return e;
   const double scale = 2.0 / (double)n_total;
   damp_lambda_kernel<<<1, 1024, 0, st>>>(H, d, scale, (double)damp, w.lam, info);

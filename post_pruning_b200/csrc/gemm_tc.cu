@@ -516,11 +516,11 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
         !make_map(&bl, B.lo, B.rows, B.cols, B.ld, kKC, kN, false))
       return cudaErrorInvalidValue;
   }
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    attr = true;
-  }
+  static PerDevice attrs;
+  cudaError_t ea = once_per_device(attrs, [] {
+    return cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+  });
+  if (ea != cudaSuccess) return ea;
   // persistent: one CTA per SM at most, fewer when the job leaves SMs to others
   const int ctas = std::min(grid, job.max_ctas > 0 ? std::min(job.max_ctas, kNumSMs) : kNumSMs);
   // C comes in by TMA when it is read (beta != 0); otherwise the map is unused

@@ -688,11 +688,11 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    attr = true;
-  }
+  static PerDevice attrs;
+  cudaError_t ea = once_per_device(attrs, [] {
+    return cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+  });
+  if (ea != cudaSuccess) return ea;
   const int grid = p.pw.ncta > 0 ? p.pw.ncta : p.tiles * p.nsplit;
   hessian_tc_kernel<<<grid, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info, p.pw, set ? 1 : 0);
   count_launches(1);

@@ -261,12 +261,15 @@ template <int MODE>
 static void launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
                          uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
                          const unsigned long long* thr, int* info, cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(sweep_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    cudaFuncSetAttribute(sweep_kernel<MODE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    attr_done = true;
-  }
+  static PerDevice attrs;
+  once_per_device(attrs, [] {
+    const cudaError_t r =
+        cudaFuncSetAttribute(sweep_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    return r != cudaSuccess
+               ? r
+               : cudaFuncSetAttribute(sweep_kernel<MODE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kSweepSmem);
+  });
   const int grid = cdiv(rows, kSweepWarps * rpw);
   if (rpw == 2)
     sweep_kernel<MODE, 2><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
@@ -442,21 +445,25 @@ constexpr int kSelMaxSmem = 160 * 1024;         // bytes of saliency bits a CTA 
 
 static cudaError_t launch_select(const float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
                                  SelState* sel, unsigned int k, int* info, cudaStream_t st) {
-  static int max_grid = 0;
-  cudaError_t e = cudaSuccess;
-  if (!max_grid) {
-    if ((e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxSmem)) !=
-        cudaSuccess)
-      return e;
-    int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kSelThreads, kSelMaxSmem)) !=
-        cudaSuccess)
-      return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    max_grid = std::max(1, std::min(per_sm, 1) * sms);   // one CTA per SM: fewer histogram merges
-  }
+  static PerDevice attrs;
+  static int max_grid_dev[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if ((e = once_per_device(attrs, [dev] {
+         cudaError_t r = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelMaxSmem);
+         if (r != cudaSuccess) return r;
+         int per_sm = 0, sms = 0;
+         if ((r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kSelThreads, kSelMaxSmem)) !=
+             cudaSuccess)
+           return r;
+         if ((r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return r;
+         max_grid_dev[dev] = std::max(1, std::min(per_sm, 1) * sms);   // one CTA per SM: fewer histogram merges
+         return cudaSuccess;
+       })) != cudaSuccess)
+    return e;
+  const int max_grid = max_grid_dev[dev];
   if ((e = cudaMemsetAsync(sel, 0, sizeof(SelState), st)) != cudaSuccess) return e;
   const long long total4 = (long long)rows * (bw / 4);
   const int grid = (int)std::max<long long>(1, std::min<long long>(cdivll(total4, kSelThreads), max_grid));
