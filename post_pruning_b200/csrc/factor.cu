@@ -15,11 +15,12 @@
 // plain FP32 on 136 CTAs, the one panel tile R_{k-1,k} and the update of
 // diagonal block k-1 that diag(k-1) waits for. Every other product (the
 // panel R_ik = A_ik U_kk^T of the rows above, the rank-128 updates of the
-// leading part, V_im = U_ii R_im and the triangular inverse) runs off the
-// chain on the tensor cores as an FP32-accurate three-product TF32 GEMM
-// (gemm_tc.cu). Operands move between those GEMMs as hi/lo planes written
-// by the producing epilogue, so no separate split pass runs except once for
-// the last column block.
+// leading part, the sums T_iq = sum_m R_im U_mq over whole rectangles and
+// the block rows U_kq = -U_kk T_kq of the inverse) runs off the chain on the
+// tensor cores as an FP32-accurate three-product TF32 GEMM (gemm_tc.cu).
+// Operands move between those GEMMs as hi/lo planes written by the producing
+// epilogue; the planes of the first column block come from the
+// scale-and-damp pass, so no separate split pass runs.
 #include <cuda_runtime.h>
 
 #include <algorithm>

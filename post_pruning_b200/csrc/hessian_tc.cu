@@ -1,16 +1,18 @@
-// H += X^T X on the 5th-generation tensor cores (SparseGPT review, section 七:
-// the Hessian proxy of a linear layer is the Gram matrix of its inputs).
+// H += X^T X, or H = X^T X, on the 5th-generation tensor cores (SparseGPT
+// review, section 七: the Hessian proxy of a linear layer is the Gram matrix
+// of its inputs).
 //
 // X is bf16 [n x d] row-major, so both GEMM operands of C = X^T X are the same
 // tensor read "MN-major": for C[i][j] = sum_t X[t][i] X[t][j], A(i, t) and
-// B(j, t) are contiguous along i and j. One CTA owns a 128 x 256 tile of H
-// whose rows i0.. and columns j0.. meet the upper triangle (H is symmetric:
-// only those tiles are computed, and every element i <= j is written to both
-// H[i][j] and H[j][i]). Tokens are split across CTAs when there are too few
-// tiles to fill the GPU; split partials are summed in split order
-// by a separate reduction kernel (deterministic). Tiles are numbered in
-// super-blocks of 2048 x 2048 channels so that the CTAs resident together
-// share most of the columns of X they stream (L2 reuse).
+// B(j, t) are contiguous along i and j. H is symmetric: only tiles on the
+// upper triangle are computed, and each element is written once, to H[i][j]
+// and its mirror H[j][i]. Wide layers use 128 x 256 band tiles whose rows
+// i0.. and columns j0.. meet the upper triangle, numbered in super-blocks of
+// 2048 x 2048 channels so that the CTAs resident together share most of the
+// columns of X they stream (L2 reuse); tokens are split across CTAs when
+// there are too few tiles to fill the GPU. Narrow layers use square tiles
+// (see PairWork), always token-split. Split partials are summed in split
+// order by a separate reduction kernel (deterministic).
 //
 // Per CTA: warp 0 lane 0 streams 64-token stages with TMA (128-byte swizzle,
 // one box = 64 tokens x 64 channels), warp 1 lane 0 issues
