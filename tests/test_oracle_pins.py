@@ -42,39 +42,50 @@ def _factor(X, damp_ratio=0.01):
 
 # ---------------------------------------------------------------- references
 
-def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None):
+def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None, blocksize=None):
     """Sequential OBS written as explicit least-squares re-fits.
 
     For each column q in order: decide the mask if the pattern decides here
-    (saliency w_c^2 / [(H_d[c:, c:])^-1]_00 on the current weights), set a
-    pruned weight to zero, then re-fit every column right of q to minimise
+    (N:M at the first column of each group of M, per row; unstructured at the
+    first column of each block of ``blocksize``, over every row of the block
+    at once: exactly floor(s * rows * width) pruned, smallest saliency first,
+    ties by row then column), with the saliency w_c^2 / [(H_d[c:, c:])^-1]_00
+    taken on the current (already re-fitted) weights; set a pruned weight to
+    zero, then re-fit every column right of q to minimise
     (w - w^) H_d (w - w^)^T with the columns <= q frozen. Uses general linear
-    solves only: no Cholesky, no U, no blocking.
+    solves only: no Cholesky, no U, no lazy batching.
     """
     kind, n_keep, m_grp, sparsity = ref.parse_pattern(pattern)
-    assert kind == "nm" or forced_mask is not None
+    assert kind == "nm" or forced_mask is not None or blocksize
     r, d = W.shape
     sal_den = np.array([np.linalg.inv(Hd[c:, c:])[0, 0] for c in range(d)])
-    out = np.array(W, dtype=np.float64)
+    w0 = np.array(W, dtype=np.float64)
+    cur = w0.copy()
     mask = np.ones((r, d), dtype=bool) if forced_mask is None else forced_mask.copy()
-    for row in range(r):
-        w0 = np.array(W[row], dtype=np.float64)
-        cur = w0.copy()
-        for q in range(d):
-            if forced_mask is None and q % m_grp == 0:
-                S = cur[q:q + m_grp] ** 2 / sal_den[q:q + m_grp]
+    for q in range(d):
+        if forced_mask is None and kind == "nm" and q % m_grp == 0:
+            for row in range(r):
+                S = cur[row, q:q + m_grp] ** 2 / sal_den[q:q + m_grp]
                 order = sorted(range(m_grp), key=lambda j: (-S[j], j))
                 mask[row, q:q + m_grp] = False
                 mask[row, [q + j for j in order[:n_keep]]] = True
+        if forced_mask is None and kind == "unstructured" and q % blocksize == 0:
+            width = min(blocksize, d - q)
+            k = int(math.floor(sparsity * r * width))
+            keys = sorted((cur[row, q + j] ** 2 / sal_den[q + j], row, j)
+                          for row in range(r) for j in range(width))
+            mask[:, q:q + width] = True
+            for _, row, j in keys[:k]:
+                mask[row, q + j] = False
+        for row in range(r):
             if not mask[row, q]:
-                cur[q] = 0.0
+                cur[row, q] = 0.0
                 if q + 1 < d:
-                    D_fixed = w0[:q + 1] - cur[:q + 1]
+                    D_fixed = w0[row, :q + 1] - cur[row, :q + 1]
                     rhs = Hd[q + 1:, :q + 1] @ D_fixed
                     D_free = -np.linalg.solve(Hd[q + 1:, q + 1:], rhs)
-                    cur[q + 1:] = w0[q + 1:] - D_free
-        out[row] = cur
-    return out, mask
+                    cur[row, q + 1:] = w0[row, q + 1:] - D_free
+    return cur, mask
 
 
 def lstsq_fixed(X, w, fixed_idx, fixed_val):
@@ -180,6 +191,23 @@ def test_sweep_equals_frozen_prefix_least_squares(rng, blocksize):
     out = oracle.sweep(W, U, "2:4", blocksize=blocksize, forced_mask=forced)
     ref_W, _ = frozen_prefix_sweep(W, Hd, "2:4", forced_mask=forced)
     assert np.allclose(out["W"], ref_W, atol=1e-11)
+
+
+@pytest.mark.parametrize("blocksize,sparsity", [(4, 0.5), (8, 0.7), (8, 0.5), (16, 0.8)])
+def test_unstructured_sweep_equals_frozen_prefix_least_squares(rng, blocksize, sparsity):
+    """Unstructured selection across blocks ([SGPT] 八 and 十一 step four):
+    every block after the first is scored on weights that earlier blocks
+    compensated, over all rows at once; non-diagonal H, 3 to 6 blocks."""
+    W, X = _layer(rng, r=6, d=24, n=70, scale_spread=1.5)
+    _, Hd, U = _factor(X)
+    pat = f"unstructured:{sparsity}"
+    out = oracle.sweep(W, U, pat, blocksize=blocksize)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, pat, blocksize=blocksize)
+    assert np.array_equal(out["mask"], ref_mask)
+    assert np.allclose(out["W"], ref_W, atol=1e-11)
+    for b0 in range(0, 24, blocksize):
+        width = min(blocksize, 24 - b0)
+        assert (~ref_mask[:, b0:b0 + width]).sum() == math.floor(sparsity * 6 * width)
 
 
 def test_diagonal_hessian_is_wanda_and_magnitude(rng):
@@ -313,34 +341,76 @@ def test_pack_roundtrip_and_bits(rng):
         oracle.pack24(out["W"], bad)
 
 
+def test_pack_and_mask_word_layout_beyond_the_first_word():
+    """Hand-derived words for groups 8..15 and columns 32..63 of two rows
+    (golden file, [2:4] section on the 2:4 mechanism): pins the word index
+    and the shift of both the metadata and the mask bits, in both
+    directions."""
+    g = _golden("pack24_layout_64.json")
+    d = g["d_in"]
+    rows = len(g["kept_pairs"])
+    W = np.array([[1000.0 * (r + 1) + c for c in range(d)] for r in range(rows)])
+    mask = np.zeros((rows, d), dtype=bool)
+    for r, pairs in enumerate(g["kept_pairs"]):
+        for grp, (a, b) in enumerate(pairs):
+            mask[r, 4 * grp + a] = mask[r, 4 * grp + b] = True
+    Wm = np.where(mask, W, 0.0)
+    meta_want = np.array([[int(h, 16) for h in row] for row in g["meta_words_hex"]], dtype=np.uint32)
+    mask_want = np.array([[int(h, 16) for h in row] for row in g["mask_words_hex"]], dtype=np.uint32)
+    values, meta = oracle.pack24(Wm, mask)
+    assert np.array_equal(meta, meta_want)
+    assert np.array_equal(values[:, 16:32], np.array(g["values_groups_8_to_15"], dtype=np.float64))
+    assert np.array_equal(oracle.mask_bits(mask), mask_want)
+    # and back: the golden words alone decode to the same matrices
+    assert np.array_equal(oracle.bits_to_mask(mask_want, d), mask)
+    assert np.array_equal(oracle.unpack24(values, meta_want, d), Wm)
+
+
 # ---------------------------------------------------------------- mutations
 
 _MUTATIONS = [
-    ("wrong sign of the compensation", "W1[:, q:] -= np.outer(e, U[c, c:i2])",
-     "W1[:, q:] += np.outer(e, U[c, c:i2])"),
-    ("dropped lazy trailing update", "W[:, i2:] -= E1 @ U[i1:i2, i2:]", "pass"),
-    ("transposed U in the trailing update", "W[:, i2:] -= E1 @ U[i1:i2, i2:]",
-     "W[:, i2:] -= E1 @ U.T[i1:i2, i2:]"),
-    ("error not divided by U_qq", "e = (w - p) / U[c, c]", "e = (w - p)"),
-    ("saliency on the starting weights", "S = (W1[:, q:q + m_grp] / diagU[c:c + m_grp]) ** 2",
-     "S = (W[:, c:c + m_grp] / diagU[c:c + m_grp]) ** 2"),
-    ("saliency without U", "S = (W1[:, q:q + m_grp] / diagU[c:c + m_grp]) ** 2",
-     "S = (W1[:, q:q + m_grp]) ** 2"),
-    ("off-by-one in the rank-1 update", "W1[:, q:] -= np.outer(e, U[c, c:i2])",
-     "W1[:, q + 1:] -= np.outer(e, U[c, c:i2 - 1])"),
+    # (name, [(old, new), ...], pattern, blocksize)
+    ("wrong sign of the compensation", [("W1[:, q:] -= np.outer(e, U[c, c:i2])",
+                                         "W1[:, q:] += np.outer(e, U[c, c:i2])")], "2:4", 8),
+    ("dropped lazy trailing update", [("W[:, i2:] -= E1 @ U[i1:i2, i2:]", "pass")], "2:4", 8),
+    ("transposed U in the trailing update", [("W[:, i2:] -= E1 @ U[i1:i2, i2:]",
+                                              "W[:, i2:] -= E1 @ U.T[i1:i2, i2:]")], "2:4", 8),
+    ("error not divided by U_qq", [("e = (w - p) / U[c, c]", "e = (w - p)")], "2:4", 8),
+    ("saliency on the starting weights",
+     [("S = (W1[:, q:q + m_grp] / diagU[c:c + m_grp]) ** 2",
+       "S = (W[:, c:c + m_grp] / diagU[c:c + m_grp]) ** 2")], "2:4", 8),
+    ("saliency without U", [("S = (W1[:, q:q + m_grp] / diagU[c:c + m_grp]) ** 2",
+                             "S = (W1[:, q:q + m_grp]) ** 2")], "2:4", 8),
+    ("off-by-one in the rank-1 update", [("W1[:, q:] -= np.outer(e, U[c, c:i2])",
+                                          "W1[:, q + 1:] -= np.outer(e, U[c, c:i2 - 1])")], "2:4", 8),
+    # the unstructured branch scored on the weights as they were before any
+    # earlier block compensated them
+    ("unstructured saliency on the starting weights",
+     [("W = np.array(W, dtype=np.float64, copy=True)",
+       "W_start = np.array(W, dtype=np.float64, copy=True); W = W_start.copy()"),
+      ("S = (W1 / diagU[i1:i2]) ** 2", "S = (W_start[:, i1:i2] / diagU[i1:i2]) ** 2")],
+     "unstructured:0.5", 4),
+    ("unstructured saliency without U", [("S = (W1 / diagU[i1:i2]) ** 2", "S = W1 ** 2")],
+     "unstructured:0.5", 4),
+    ("unstructured count rounded up",
+     [("k = int(math.floor(sparsity * r * width))", "k = int(math.ceil(sparsity * r * width))")],
+     "unstructured:0.53", 4),
 ]
 
 
-@pytest.mark.parametrize("name,old,new", _MUTATIONS, ids=[m[0] for m in _MUTATIONS])
-def test_pins_catch_planted_mistakes(rng, name, old, new):
+@pytest.mark.parametrize("name,edits,pattern,blocksize", _MUTATIONS, ids=[m[0] for m in _MUTATIONS])
+def test_pins_catch_planted_mistakes(name, edits, pattern, blocksize):
     src = inspect.getsource(ref.sweep)
-    assert old in src, name
+    for old, new in edits:
+        assert old in src, name
+        src = src.replace(old, new)
     ns = dict(vars(ref))
-    exec(src.replace(old, new), ns)
+    exec(src, ns)
     mutated = ns["sweep"]
-    W, X = _layer(rng, r=5, d=16, n=60, scale_spread=1.5)
+    # own seed: the verdict must not depend on which tests ran before
+    W, X = _layer(np.random.default_rng(2024), r=16, d=32, n=80, scale_spread=1.5)
     _, Hd, U = _factor(X)
-    got = mutated(W, U, "2:4", blocksize=8)
-    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, "2:4")
+    got = mutated(W, U, pattern, blocksize=blocksize)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, pattern, blocksize=blocksize)
     same = np.array_equal(got["mask"], ref_mask) and np.allclose(got["W"], ref_W, atol=1e-9)
     assert not same, f"pins did not catch: {name}"
