@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define SGPT_ABI_VERSION 1
+#define SGPT_ABI_VERSION 2
 
 typedef enum sgpt_status {
   SGPT_OK = 0,
@@ -87,6 +87,18 @@ int sgpt_abi_version(void);
 /* Diagnostics: number of kernels this library has enqueued since it was
  * loaded (all devices, all streams). Memsets and copies are not counted. */
 uint64_t sgpt_kernel_launches(void);
+
+/* Failure-path testing and diagnostics (no counterpart in the pages): the
+ * number of SM clock cycles a device-side wait on other threads or CTAs (a
+ * tensor-core pipeline barrier, the selection's grid barrier) polls before
+ * it gives up and records SGPT_INFO_TIMEOUT. cycles <= 0 restores the
+ * default, 4e9 (about 2 s at the boost clock). Process-wide; read when a
+ * kernel is enqueued (a captured graph keeps the value it was captured
+ * with). A CTA that gave up still waits for its own copies and tensor-core
+ * operations in flight under a fixed limit before it exits, so a tiny value
+ * makes kernels report TIMEOUT and return, never leaves work behind. Returns
+ * the previous value. */
+int64_t sgpt_set_wait_limit(int64_t cycles);
 
 /* Scratch bytes needed by any call below for these sizes (n_tok only matters
  * for the Hessian; pass 0 when H is given). */
@@ -180,8 +192,11 @@ sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint
 
 /* Layer reconstruction error (SparseGPT review, section 六, the objective):
  * num_den[0] = tr(dW H dW^T), num_den[1] = tr(W0 H W0^T), dW = W0 - W, in
- * fp64 on the device. H is the full symmetric matrix (undamped; any positive
- * scale). Both W0 and W use leading dimension ldw. */
+ * fp64 on the device (FP32 products, fp64 sums in a fixed order: the result
+ * is the same to the last bit on every call). H is the full symmetric
+ * matrix (undamped; any positive scale). Both W0 and W use leading
+ * dimension ldw. ws: at least sgpt_workspace_bytes(d_out, d_in, 0, p)
+ * bytes (SGPT_ERR_WORKSPACE otherwise). */
 sgpt_status sgpt_recon_error(const float* W0, const float* W, int d_out, int d_in, int ldw,
                              const float* H, double* num_den, void* ws, size_t ws_bytes,
                              void* stream);

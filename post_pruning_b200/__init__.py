@@ -27,6 +27,7 @@ from .sgpt import (  # noqa: F401
     prune_noalloc,
     raise_on_info,
     recon_error,
+    set_wait_limit,
     sync_status,
     workspace,
     workspace_bytes,

@@ -14,6 +14,8 @@
 namespace sgpt {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+static std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
+long long wait_limit_cycles() { return g_wait_cycles.load(std::memory_order_relaxed); }
 }  // namespace sgpt
 
 namespace {
@@ -75,10 +77,15 @@ int sgpt_abi_version(void) { return SGPT_ABI_VERSION; }
 
 uint64_t sgpt_kernel_launches(void) { return sgpt::g_launches.load(std::memory_order_relaxed); }
 
+int64_t sgpt_set_wait_limit(int64_t cycles) {
+  const long long v = cycles > 0 ? (long long)cycles : kDefaultWaitCycles;
+  return (int64_t)sgpt::g_wait_cycles.exchange(v, std::memory_order_relaxed);
+}
+
 size_t sgpt_workspace_bytes(int d_out, int d_in, int64_t n_tok, const sgpt_params* p) {
   (void)p;
   if (!valid_din(d_in) || !valid_dout(d_out) || n_tok < 0) return 0;
-  size_t need = std::max(factor_ws_bytes(d_in), prune_ws_bytes(d_out, d_in));
+  size_t need = std::max({factor_ws_bytes(d_in), prune_ws_bytes(d_out, d_in), recon_ws_bytes(d_out, d_in)});
   if (n_tok > 0) need = std::max(need, hessian_ws_bytes(d_in, n_tok));
   return need;
 }
@@ -181,27 +188,34 @@ sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint
 
 sgpt_status sgpt_recon_error(const float* W0, const float* W, int d_out, int d_in, int ldw, const float* H,
                              double* num_den, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (!W0 || !W || !H || !num_den) return SGPT_ERR_INVALID_ARG;
   if (!aligned16(W0) || !aligned16(W) || !aligned16(H) || (reinterpret_cast<uintptr_t>(num_den) & 7u))
     return SGPT_ERR_INVALID_ARG;
   if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
-  return from_cuda(launch_recon(W0, W, d_out, d_in, ldw, H, num_den, as_stream(stream)));
+  const sgpt_status s = check_ws(ws, ws_bytes, recon_ws_bytes(d_out, d_in));
+  if (s != SGPT_OK) return s;
+  return from_cuda(launch_recon(W0, W, d_out, d_in, ldw, H, num_den, ws, as_stream(stream)));
 }
 
 sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint16_t* X, int64_t n_tok,
                              float* H, float* U, const sgpt_params* p, uint32_t* mask_bits, float* values,
                              uint32_t* meta, float* row_loss, void* ws, size_t ws_bytes, int* dev_info,
                              void* stream) {
+  // every argument of every step is checked here, before the first launch,
+  // so a bad one never leaves H or U half overwritten
   if (!H || !U || H == U || n_tok <= 0 || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (!W || !mask_bits || !aligned16(W) || !aligned16(mask_bits) || !aligned16(H) || !aligned16(U))
+    return SGPT_ERR_INVALID_ARG;
+  if (X && (!aligned16(X) || n_tok > (int64_t)INT32_MAX)) return SGPT_ERR_INVALID_ARG;
+  if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
   sgpt_status s = check_params(p);
   if (s != SGPT_OK) return s;
-  if (!valid_din(d_in) || !valid_dout(d_out)) return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
   s = check_ws(ws, ws_bytes, sgpt_workspace_bytes(d_out, d_in, X ? n_tok : 0, p));
   if (s != SGPT_OK) return s;
   const bool pack = p->pattern == SGPT_PATTERN_NM && values && meta;
   if ((values || meta) && !pack) return SGPT_ERR_INVALID_ARG;
+  if (pack && (!aligned16(values) || !aligned16(meta))) return SGPT_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
   if ((s = sgpt_info_clear(dev_info, stream)) != SGPT_OK) return s;
   if (X && (s = sgpt_hessian_compute(H, X, n_tok, d_in, ws, ws_bytes, dev_info, stream)) != SGPT_OK) return s;

@@ -14,9 +14,20 @@ constexpr int kNumSMs = 148;          // B200
 constexpr int kTile = 128;            // square tile of H, R, U and the GEMMs
 constexpr int kMaxBlock = 128;        // widest OBS block held by the sweep
 
-// Bounded spin: a device-side wait gives up after this many polls and
-// records SGPT_INFO_TIMEOUT instead of hanging the GPU.
-constexpr long long kSpinLimit = 1ll << 26;
+// Bounded waits. A device-side wait on another role of the same kernel or on
+// other CTAs (an mbarrier phase, a grid barrier) gives up after the launch's
+// wait limit in SM clock cycles (a kernel argument, from wait_limit_cycles())
+// and records SGPT_INFO_TIMEOUT instead of hanging the GPU. A CTA that gave
+// up still waits for its own asynchronous work in flight (TMA copies,
+// tensor-core MMAs) before it frees TMEM and exits; those drains complete by
+// themselves and use the fixed kDrainCycles, never the settable limit.
+constexpr long long kDefaultWaitCycles = 4000000000ll;   // ~2 s at the boost clock
+constexpr long long kDrainCycles = 4000000000ll;
+// Below this limit an mbarrier wait polls without suspending the thread.
+constexpr long long kShortWaitCycles = 1000000ll;
+
+// The wait limit kernels are launched with now (sgpt_set_wait_limit).
+long long wait_limit_cycles();
 
 // First error wins; later kernels of the chain see it and return early.
 __device__ __forceinline__ void set_info(int* info, int code) {

@@ -47,7 +47,6 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;   // producer, MMA issuer, epilogu
 // bytes, 16-byte chunks XOR-swizzled by row % 8 (TMA's 128-byte swizzle).
 constexpr size_t kStagingBytes = (size_t)kM * kN * 4;
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + kStagingBytes + 1024 + 256;
-constexpr long long kWaitCycles = 4000000000ll;
 constexpr int kChunk = 128 / kKC;               // stages (128 of K) per TMEM accumulation
 constexpr int kTmemCols = 2 * kN;               // two accumulators: one fills while one drains
 
@@ -117,11 +116,31 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Non-suspending test of a barrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.b32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false if the barrier phase did not complete within `limit`
+// SM clock cycles. try_wait may suspend the thread for a hardware-defined
+// time, longer than a short limit, so short limits (failure-path tests)
+// poll with the non-suspending test instead.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit) {
+  if (limit < kShortWaitCycles) {
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity))
+      if (clock64() - t0 > limit) return false;
+    return true;
+  }
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   return true;
 }
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
@@ -193,13 +212,14 @@ __device__ __forceinline__ Item decode_item(const Job& job, int w) {
 __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
     const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
     const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo, const Job job,
-    const __grid_constant__ CUtensorMap c_map, const int b_mn, const int items, int* info) {
+    const __grid_constant__ CUtensorMap c_map, const int b_mn, const int items, int* info,
+    const long long wait_cycles) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* T = smem + kStages * kStageBytes;   // epilogue tile (C in, result out)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kStagingBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 6);
   __shared__ int failed;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (cta_info_set(info)) return;
@@ -208,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
   const uint32_t s0 = smem_u32(smem);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
   const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16, cfull = tfull0 + 32;
+  const uint32_t mdone = tfull0 + 40;         // every MMA this CTA issued has completed
   if (threadIdx.x == 0) {
     // descriptors into the TMA unit's cache before the first copy needs them
     const CUtensorMap* maps[5] = {&a_hi, &a_lo, &b_hi, &b_lo, &c_map};
@@ -223,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
       mbar_init(tempty0 + 8 * b, kEpiWarps);
     }
     mbar_init(cfull, 1);
+    mbar_init(mdone, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -244,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
         const int iters = (it.ke - it.kb + kKC - 1) / kKC;
         for (int i = 0; i < iters; ++i, ++g) {
           const int st = g % kStages;
-          if (g >= kStages && !mbar_wait(empty0 + 8 * st, ((g / kStages) & 1) ^ 1)) {
+          if (g >= kStages && !mbar_wait(empty0 + 8 * st, ((g / kStages) & 1) ^ 1, wait_cycles)) {
             failed = 1;
             break;
           }
@@ -268,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
       }
       // never leave with copies in flight: wait for every stage still armed
       for (int x = (g > kStages ? g - kStages : 0); x < g; ++x)
-        if (!mbar_wait(full0 + 8 * (x % kStages), (x / kStages) & 1)) failed = 1;
+        if (!mbar_wait(full0 + 8 * (x % kStages), (x / kStages) & 1, kDrainCycles)) failed = 1;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -279,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
         const int iters = (it.ke - it.kb + kKC - 1) / kKC;
         for (int c0 = 0; c0 < iters && !failed; c0 += kChunk, ++u) {
           const int b = u & 1;
-          if (u >= 2 && !mbar_wait(tempty0 + 8 * b, ((u >> 1) - 1) & 1)) {
+          if (u >= 2 && !mbar_wait(tempty0 + 8 * b, ((u >> 1) - 1) & 1, wait_cycles)) {
             failed = 1;
             break;
           }
@@ -288,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
           const int c1 = min(iters, c0 + kChunk);
           for (int i = c0; i < c1; ++i, ++g) {
             const int st = g % kStages;
-            if (!mbar_wait(full0 + 8 * st, (g / kStages) & 1)) {
+            if (!mbar_wait(full0 + 8 * st, (g / kStages) & 1, wait_cycles)) {
               failed = 1;
               break;
             }
@@ -315,6 +337,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
           mma_commit(tfull0 + 8 * b);
         }
       }
+      // never free TMEM under a running MMA (after a timeout the epilogue
+      // may not have waited for the last ones): wait for all of them
+      mma_commit(mdone);
+      if (!mbar_wait(mdone, 0, kDrainCycles)) failed = 1;
     }
   } else {
     // Epilogue warps: warp w reads TMEM lanes 32*(w%4).. (tile rows) and
@@ -351,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
       for (int e = 0; e < 64; ++e) acc[e] = 0.f;
       for (int c0 = 0; c0 < iters; c0 += kChunk, ++u) {
         const int b = u & 1;
-        if (!failed && !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1)) failed = 1;
+        if (!failed && !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1, wait_cycles)) failed = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (!failed) {
 #pragma unroll
@@ -366,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty0 + 8 * b);
       }
-      if (read_c && !failed && !mbar_wait(cfull, nitem & 1)) failed = 1;
+      if (read_c && !failed && !mbar_wait(cfull, nitem & 1, wait_cycles)) failed = 1;
       // this thread's 64 columns = 16 chunks of 16 bytes in groups 2h, 2h+1
 #pragma unroll
       for (int cj = 0; cj < 16; ++cj) {
@@ -410,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
       }
     }
     // never leave with a C copy in flight (after a timeout some were not waited for)
-    if (read_c && issuer && c_issued > 0) mbar_wait(cfull, (c_issued - 1) & 1);
+    if (read_c && issuer && c_issued > 0) mbar_wait(cfull, (c_issued - 1) & 1, kDrainCycles);
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -528,7 +554,8 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
   if (job.C && job.beta != 0.f &&
       !make_map_c(&cm, job.C, (long long)job.c_row0 + job.Mlim, (long long)job.c_col0 + job.Nlim, job.ldc))
     return cudaErrorInvalidValue;
-  gemm_tf32x3_kernel<<<ctas, kThreads, kSmem, st>>>(ah, al, bh, bl, job, cm, b_mn ? 1 : 0, grid, info);
+  gemm_tf32x3_kernel<<<ctas, kThreads, kSmem, st>>>(ah, al, bh, bl, job, cm, b_mn ? 1 : 0, grid, info,
+                                                    wait_limit_cycles());
   count_launches(1);
   return cudaGetLastError();
 }

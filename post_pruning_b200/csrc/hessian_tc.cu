@@ -47,7 +47,6 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;   // warp 0: TMA, warp 1: MMA
 constexpr int kChunkIters = 8;                // stages (512 tokens) per TMEM accumulation
 constexpr int kTmemCols = 2 * kN;             // two accumulators, double-buffered
 constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-constexpr long long kWaitCycles = 4000000000ll;   // ~2 s at the B200 boost clock
 
 // instruction descriptor: D fp32, A/B bf16, both MN-major, N=256, M=128
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
@@ -90,13 +89,31 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the barrier phase did not complete in time.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Non-suspending test of a barrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.b32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false if the barrier phase did not complete within `limit`
+// SM clock cycles. try_wait may suspend the thread for a hardware-defined
+// time, longer than a short limit, so short limits (failure-path tests)
+// poll with the non-suspending test instead.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit) {
+  if (limit < kShortWaitCycles) {
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity))
+      if (clock64() - t0 > limit) return false;
+    return true;
+  }
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
-  }
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > limit) return false;
   return true;
 }
 
@@ -270,12 +287,12 @@ __device__ void flush_block(uint32_t S, int rs, int cs, int i0, int j0, float* _
 __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int d, long long n,
     int nsplit, long long per, float* __restrict__ part, int* info, const __grid_constant__ PairWorks pw,
-    int set) {
+    int set, long long wait_cycles) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   __shared__ int failed;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   const uint32_t s0 = smem_u32(smem);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
   const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16;
+  const uint32_t mdone = tfull0 + 32;         // every MMA this CTA issued has completed
 
   if (threadIdx.x == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
@@ -319,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, kEpiWarps);
     }
+    mbar_init(mdone, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -346,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     for (int it = 0; it < iters; ++it) {
       const int s = it % kStages;
       const uint32_t par = ((it / kStages) & 1) ^ 1;
-      if (it >= kStages && !mbar_wait(empty0 + 8 * s, par)) {
+      if (it >= kStages && !mbar_wait(empty0 + 8 * s, par, wait_cycles)) {
         failed = 1;
         break;
       }
@@ -363,13 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     }
     // never leave with copies in flight: wait for every stage that was armed
     for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
-      if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1)) failed = 1;
+      if (!mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1, kDrainCycles)) failed = 1;
   } else if (!skip && warp == 1 && lane == 0) {
     // MMA issuer: chunk c accumulates kChunkIters stages into buffer c & 1
     const uint32_t idesc = nsq == 2 ? kIdesc : kIdesc128;
     for (int c = 0; c < nchunks && !failed; ++c) {
       const int b = c & 1;
-      if (c >= 2 && !mbar_wait(tempty0 + 8 * b, ((c >> 1) - 1) & 1)) {
+      if (c >= 2 && !mbar_wait(tempty0 + 8 * b, ((c >> 1) - 1) & 1, wait_cycles)) {
         failed = 1;
         break;
       }
@@ -378,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       const int it_end = min(iters, (c + 1) * kChunkIters);
       for (int it = c * kChunkIters; it < it_end; ++it) {
         const int s = it % kStages;
-        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1, wait_cycles)) {
           failed = 1;
           break;
         }
@@ -392,11 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
       }
       mma_commit(tfull0 + 8 * b);
     }
+    // never free TMEM under a running MMA (after a timeout the epilogue may
+    // not have waited for the last ones): wait for all of them
+    mma_commit(mdone);
+    if (!mbar_wait(mdone, 0, kDrainCycles)) failed = 1;
   } else if (!skip && warp >= 2) {
     // Drain every chunk into the running sums, then hand the buffer back.
     for (int c = 0; c < nchunks; ++c) {
       const int b = c & 1;
-      if (!mbar_wait(tfull0 + 8 * b, (c >> 1) & 1)) {
+      if (!mbar_wait(tfull0 + 8 * b, (c >> 1) & 1, wait_cycles)) {
         failed = 1;
         break;
       }
@@ -696,7 +719,8 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
   });
   if (ea != cudaSuccess) return ea;
   const int grid = p.pw.ncta > 0 ? p.pw.ncta : p.tiles * p.nsplit;
-  hessian_tc_kernel<<<grid, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info, p.pw, set ? 1 : 0);
+  hessian_tc_kernel<<<grid, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info, p.pw, set ? 1 : 0,
+                                                   wait_limit_cycles());
   count_launches(1);
   if (p.pw.ncta > 0) {
     hessian_pair_reduce_kernel<<<p.pair_blocks, kReduceThreads, 0, st>>>(part, H, d, p.pt, info, set ? 1 : 0);

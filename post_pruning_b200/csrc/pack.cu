@@ -61,16 +61,18 @@ cudaError_t launch_pack24(const float* W, long long ldw, int rows, int d, const 
 
 // ------------------------------------------------- reconstruction error
 
-// out += sum over the tile of (A H)[m][n] * A[m][n], A = W0 - W (diff) or W0.
+// partial[tile] = sum over the tile of (A H)[m][n] * A[m][n], A = W0 - W
+// (diff) or W0; one partial per CTA, summed in a fixed order afterwards, so
+// the result is deterministic to the last bit.
 template <class OA>
 __global__ void __launch_bounds__(kGemmThreads) quad_form_kernel(OA A, const float* __restrict__ H,
                                                                  int d, const float* __restrict__ P,
                                                                  const float* __restrict__ Q,
                                                                  long long ldw, int rows,
-                                                                 double* __restrict__ out) {
+                                                                 double* __restrict__ partial) {
   extern __shared__ float smem[];
   __shared__ double red[kGemmThreads / 32];
-  const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile;
+  const int m0 = blockIdx.x * kTile, n0 = blockIdx.y * kTile;   // row tiles on x: up to 2^17 of them
   A.i0 = m0;
   A.I = rows - m0;
   float acc[8][8];
@@ -102,20 +104,43 @@ __global__ void __launch_bounds__(kGemmThreads) quad_form_kernel(OA A, const flo
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int w = 0; w < kGemmThreads / 32; ++w) t += red[w];
-    atomicAdd(out, t);
+    partial[(long long)blockIdx.x * gridDim.y + blockIdx.y] = t;
   }
 }
 
+// out[q] = sum of partial[q * n .. q * n + n) for q = 0, 1 (one CTA per q):
+// each thread sums a fixed stride of the partials, then a fixed tree.
+constexpr int kSumThreads = 1024;
+__global__ void __launch_bounds__(kSumThreads) recon_sum_kernel(const double* __restrict__ partial,
+                                                                long long n, double* __restrict__ out) {
+  __shared__ double red[kSumThreads];
+  const double* p = partial + blockIdx.x * n;
+  double s = 0.0;
+  for (long long i = threadIdx.x; i < n; i += kSumThreads) s += p[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kSumThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[blockIdx.x] = red[0];
+}
+
+size_t recon_ws_bytes(int rows, int d) {
+  return 2 * (size_t)cdiv(d, kTile) * (size_t)cdiv(rows, kTile) * sizeof(double) + 256;
+}
+
 cudaError_t launch_recon(const float* W0, const float* W, int rows, int d, long long ldw,
-                         const float* H, double* num_den, cudaStream_t st) {
-  cudaMemsetAsync(num_den, 0, 2 * sizeof(double), st);
-  dim3 grid(cdiv(d, kTile), cdiv(rows, kTile));
+                         const float* H, double* num_den, void* ws, cudaStream_t st) {
+  dim3 grid(cdiv(rows, kTile), cdiv(d, kTile));
+  const long long tiles = (long long)grid.x * grid.y;
+  double* partial = static_cast<double*>(ws);
   const OpKContigDiff dA{W0, W, ldw, 0, rows, d};
-  quad_form_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(dA, H, d, W0, W, ldw, rows, num_den);
-  count_launches(1);
+  quad_form_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(dA, H, d, W0, W, ldw, rows, partial);
   const OpKContig A0{W0, ldw, 0, rows, d};
-  quad_form_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(A0, H, d, W0, nullptr, ldw, rows, num_den + 1);
-  count_launches(1);
+  quad_form_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(A0, H, d, W0, nullptr, ldw, rows, partial + tiles);
+  recon_sum_kernel<<<2, kSumThreads, 0, st>>>(partial, tiles, num_den);
+  count_launches(3);
   return cudaGetLastError();
 }
 

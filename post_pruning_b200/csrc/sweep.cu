@@ -258,11 +258,11 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 2 : 1; }
 
 template <int MODE>
-static void launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
-                         uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
-                         const unsigned long long* thr, int* info, cudaStream_t st) {
+static cudaError_t launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
+                                uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
+                                const unsigned long long* thr, int* info, cudaStream_t st) {
   static PerDevice attrs;
-  once_per_device(attrs, [] {
+  const cudaError_t ea = once_per_device(attrs, [] {
     const cudaError_t r =
         cudaFuncSetAttribute(sweep_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
     return r != cudaSuccess
@@ -270,6 +270,7 @@ static void launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int 
                : cudaFuncSetAttribute(sweep_kernel<MODE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kSweepSmem);
   });
+  if (ea != cudaSuccess) return ea;
   const int grid = cdiv(rows, kSweepWarps * rpw);
   if (rpw == 2)
     sweep_kernel<MODE, 2><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
@@ -278,6 +279,7 @@ static void launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int 
     sweep_kernel<MODE, 1><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
                                                                    Err_lo, thr, info);
   count_launches(1);
+  return cudaGetLastError();
 }
 
 // --------------------------------------------------------- trailing update
@@ -309,7 +311,6 @@ struct SelState {
 };
 
 constexpr int kSelThreads = 1024;
-constexpr long long kGridWaitCycles = 2000000000ll;
 
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
   unsigned int v;
@@ -318,16 +319,17 @@ __device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
 }
 
 // Barrier over the whole grid (the launch is cooperative, so every CTA is
-// resident). The wait is bounded: on timeout the CTA records
-// SGPT_INFO_TIMEOUT and the caller returns.
-__device__ bool grid_sync(unsigned int* ctr, unsigned int target, int* info, int* failed) {
+// resident). The wait is bounded by `limit` SM clock cycles: on timeout the
+// CTA records SGPT_INFO_TIMEOUT and the caller returns (a CTA still waiting
+// elsewhere gives up on its own limit; none waits on one that returned).
+__device__ bool grid_sync(unsigned int* ctr, unsigned int target, int* info, int* failed, long long limit) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     atomicAdd(ctr, 1u);
     const long long t0 = clock64();
     while (ld_acquire(ctr) < target) {
-      if (clock64() - t0 > kGridWaitCycles) {
+      if (clock64() - t0 > limit) {
         set_info(info, SGPT_INFO_TIMEOUT);
         *failed = 1;
         break;
@@ -353,7 +355,7 @@ __device__ bool grid_sync(unsigned int* ctr, unsigned int target, int* info, int
 // 4e + j. st must be zeroed before the launch; CTA 0 writes the threshold.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
-    const float* __restrict__ U, SelState* st, unsigned int k, int keep_bits, int* info) {
+    const float* __restrict__ U, SelState* st, unsigned int k, int keep_bits, int* info, long long wait_cycles) {
   if (cta_info_set(info)) return;
   extern __shared__ unsigned int skey[];        // this CTA's saliency bits, if keep_bits
   __shared__ unsigned int h[256];
@@ -412,7 +414,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     }
     __syncthreads();
     if (t < 256 && h[t]) atomicAdd(&st->hist[pass][t], h[t]);
-    if (!grid_sync(&st->arrive, (unsigned)(pass + 1) * gridDim.x, info, &s_failed)) return;
+    if (!grid_sync(&st->arrive, (unsigned)(pass + 1) * gridDim.x, info, &s_failed, wait_cycles)) return;
     // every CTA: inclusive scan of the 256 bins and the bin holding rank k
     const unsigned int cnt = (t < 256) ? __ldcg(&st->hist[pass][t]) : 0u;
     unsigned int inc = cnt;
@@ -480,7 +482,8 @@ static cudaError_t launch_select(const float* W, long long ldw, int rows, int d,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, select_kernel, W, ldw, rows, d, i1, bw, U, sel, k, keep_bits, info);
+  e = cudaLaunchKernelEx(&cfg, select_kernel, W, ldw, rows, d, i1, bw, U, sel, k, keep_bits, info,
+                         wait_limit_cycles());
   count_launches(1);
   return e;
 }
@@ -526,16 +529,19 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
     if (p.forced) {
-      launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info, st);
+      e = launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr,
+                                    info, st);
     } else if (p.pattern == SGPT_PATTERN_NM) {
-      launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr, info, st);
+      e = launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr,
+                                  info, st);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
-      launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr,
-                                   info, st);
+      e = launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo,
+                                       &w.sel->thr, info, st);
     }
+    if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {
       tc::Job job{};
@@ -611,15 +617,18 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
     if (p.forced) {
-      launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info, st);
+      e = launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info,
+                                    st);
     } else if (p.pattern == SGPT_PATTERN_NM) {
-      launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info, st);
+      e = launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info, st);
     } else {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
-      launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info, st);
+      e = launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr,
+                                       info, st);
     }
+    if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {
       dim3 grid(cdiv(d - i2, kTile), cdiv(rows, kTile));

@@ -28,7 +28,8 @@ PATTERN_UNSTRUCTURED = 0
 PATTERN_NM = 1
 
 EXPORTS = (
-    "sgpt_status_string", "sgpt_abi_version", "sgpt_kernel_launches", "sgpt_workspace_bytes",
+    "sgpt_status_string", "sgpt_abi_version", "sgpt_kernel_launches", "sgpt_set_wait_limit",
+    "sgpt_workspace_bytes",
     "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
     "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
     "sgpt_recon_error", "sgpt_prune_layer",
@@ -90,6 +91,7 @@ def lib() -> ctypes.CDLL:
         "sgpt_status_string": (ctypes.c_char_p, [i32]),
         "sgpt_abi_version": (i32, []),
         "sgpt_kernel_launches": (ctypes.c_uint64, []),
+        "sgpt_set_wait_limit": (i64, [i64]),
         "sgpt_workspace_bytes": (sz, [i32, i32, i64, pp]),
         "sgpt_info_clear": (i32, [vp, vp]),
         "sgpt_sync_status": (i32, [vp, vp]),
@@ -145,6 +147,12 @@ def _check(status: int, where: str):
 def kernel_launches() -> int:
     """Kernels libsgpt has enqueued since it was loaded."""
     return int(lib().sgpt_kernel_launches())
+
+
+def set_wait_limit(cycles: int) -> int:
+    """Cycles a device-side wait polls before it records TIMEOUT (<= 0: the
+    default). Returns the previous value. For testing failure paths."""
+    return int(lib().sgpt_set_wait_limit(int(cycles)))
 
 
 def workspace_bytes(d_out: int, d_in: int, n_tok: int = 0, params: Params | None = None) -> int:
@@ -270,8 +278,9 @@ def pack24(W: torch.Tensor, mask: torch.Tensor, values: torch.Tensor, meta: torc
 
 
 def recon_error(W0: torch.Tensor, W: torch.Tensor, H: torch.Tensor, num_den: torch.Tensor,
-                stream=None):
-    """num_den (float64 [2], device) = (tr(dW H dW^T), tr(W0 H W0^T))."""
+                ws: torch.Tensor | None = None, stream=None):
+    """num_den (float64 [2], device) = (tr(dW H dW^T), tr(W0 H W0^T)).
+    ws: a workspace for these sizes (one is allocated when None)."""
     _dev(W0, torch.float32, "W0")
     _dev(W, torch.float32, "W")
     _dev(H, torch.float32, "H")
@@ -280,7 +289,9 @@ def recon_error(W0: torch.Tensor, W: torch.Tensor, H: torch.Tensor, num_den: tor
     if _rowmajor(W0, "W0") != ldw or W0.shape != W.shape:
         raise ValueError("W0 and W must share shape and leading dimension")
     r, d = W.shape
-    _check(lib().sgpt_recon_error(_ptr(W0), _ptr(W), r, d, ldw, _ptr(H), _ptr(num_den), None, 0,
+    if ws is None:
+        ws = workspace(r, d, device=W.device)
+    _check(lib().sgpt_recon_error(_ptr(W0), _ptr(W), r, d, ldw, _ptr(H), _ptr(num_den), _ptr(ws), ws.numel(),
                                   _stream(stream)), "sgpt_recon_error")
 
 

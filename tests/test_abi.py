@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "sgpt.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|sgpt_status|int|size_t|uint64_t)\s+(sgpt_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|sgpt_status|int|int64_t|size_t|uint64_t)\s+(sgpt_\w+)\s*\(",
                                  src, flags=re.M)))
 
 
@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
     L = pp.lib()
     for name in _declared():
         assert hasattr(L, name), name
-    assert L.sgpt_abi_version() == 1
+    assert L.sgpt_abi_version() == 2
 
 
 def test_status_strings():
@@ -97,6 +97,24 @@ def test_other_entry_points_validate():
     assert L.sgpt_hessian_accumulate(FAKE, FAKE, 100, 96 + 8, FAKE, 1 << 30, FAKE, None) == 1
     assert L.sgpt_pack24(FAKE, 8, 64, 64, FAKE, FAKE, None, FAKE, None) == 1
     assert L.sgpt_recon_error(FAKE, FAKE, 8, 64, 60, FAKE, FAKE, None, 0, None) == 1
+    assert L.sgpt_recon_error(FAKE, FAKE, 8, 64, 64, FAKE, FAKE, None, 0, None) == 8     # workspace
+    # prune_layer checks W, the mask and ldw before anything is launched
+    p24 = S.Params("2:4").to_c()
+    assert L.sgpt_prune_layer(None, 8, 64, 64, None, 10, FAKE, FAKE + 4096, ctypes.byref(p24), FAKE, None,
+                              None, None, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_prune_layer(FAKE, 8, 64, 60, None, 10, FAKE, FAKE + 4096, ctypes.byref(p24), FAKE, None,
+                              None, None, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_prune_layer(FAKE, 8, 64, 64, None, 10, FAKE, FAKE + 4096, ctypes.byref(p24), MISALIGNED,
+                              None, None, None, FAKE, 1 << 30, FAKE, None) == 1
+
+
+def test_wait_limit_setting():
+    L = pp.lib()
+    default = 4000000000
+    assert pp.set_wait_limit(1000) == default
+    assert pp.set_wait_limit(0) == 1000
+    assert pp.set_wait_limit(-5) == default
+    assert L.sgpt_set_wait_limit(0) == default
     assert L.sgpt_info_clear(None, None) == 1
     assert L.sgpt_sync_status(None, None) == 1
     p = S.Params("2:4").to_c()

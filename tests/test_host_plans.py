@@ -28,6 +28,7 @@ HARNESS = r'''
 
 namespace sgpt {
 void count_launches(unsigned long long) {}   // the library's counter lives in api.cu
+long long wait_limit_cycles() { return kDefaultWaitCycles; }   // the setting lives in api.cu too
 }
 
 int main() {
