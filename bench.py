@@ -1,16 +1,21 @@
 #!/usr/bin/env python
 """SparseGPT per-layer prune time and weights/s on B200.
 
-One step prunes the OPT-125M-shaped layer (W 768 x 768 fp32, X 262,144 x 768
-bf16 = 128 sequences x 2,048 tokens) twice from its activations, once 2:4 and
-once unstructured at 50%: each run is a full layer prune through the C ABI
-(Hessian accumulation, damping and factorisation, blocked OBS sweep, and for
-2:4 the packing). Inputs are resident in HBM; W is restored and L2 is flushed
+Default workload: one Qwen3-32B-shaped decoder block, 131,072 calibration
+tokens, every linear layer pruned 2:4 from its activations. One step prunes
+all seven matrices (q 5120->8192, k/v 5120->1024, o 8192->5120, gate/up
+5120->25600, down 25600->5120; 487,587,840 weights): for each of the four
+distinct inputs the Hessian H = X^T X and the damped factorisation run once,
+then every matrix that reads that input is swept (blocked OBS, 2:4 masks on
+the compensated weights, lazy trailing updates) and packed (values + 2-bit
+metadata), all through the C ABI. Inputs are resident in HBM (11.5 GB of
+bf16 activations, far above the 126 MB L2); W is restored and L2 flushed
 between steps (untimed). Device time per step comes from CUDA events on the
 launching stream; with N GPUs every rank prunes its own replica and the
 slowest rank's time counts (weak scaling, no collectives on the data path).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--config qwen3_32b_block|opt125m_768|llama7b_down|llama7b_q|...]
 
 Prints one JSON line on rank 0.
 """
@@ -30,49 +35,75 @@ sys.path.insert(0, ROOT)
 
 METRIC = "SparseGPT per-layer prune time & weights/s on 1 B200; % of HBM/tensor roofline"
 UNIT = "weights/s"
-CONFIG = "opt125m_768"
+CONFIG = "qwen3_32b_block"
 WORKLOADS = {
     "layer256": "256x256 layer, 2048 tokens, 2:4",
+    "opt125m_768": ("OPT-125M-shaped linear layer: W 768x768 fp32 ~N(0,1/768); X 262144x768 bf16 "
+                    "(128 seqs x 2048 tokens, lognormal(sigma=1) channel scales, 1% outlier channels x20); "
+                    "two layer prunes per step from X: 2:4 and unstructured 50%; blocksize 128; damp 0.01"),
     "llama7b_down": ("Llama-7B MLP down-proj: W 4096x11008 fp32, X 131072x11008 bf16 (lognormal sigma=1.5, "
                      "0.5% outlier channels x50), 2:4"),
     "llama7b_q": ("Llama-7B q_proj: W 4096x4096 fp32, X 262144x4096 bf16, unstructured 50/70/80% "
                   "(three layer prunes per step)"),
     "profile_4096": "4096x4096 layer, 32768 tokens, 2:4 (profiler captures)",
-    "qwen3_32b_block": ("Qwen3-32B-shaped block: q 5120->8192, k/v 5120->1024, o 8192->5120, gate/up "
-                        "5120->25600, down 25600->5120, 131072 tokens, 2:4; H and U shared by q/k/v and by "
-                        "gate/up (4 Hessians, 7 sweeps per step)"),
+    "qwen3_32b_block": ("Qwen3-32B-shaped decoder block, 2:4 along d_in: q 5120->8192, k/v 5120->1024, "
+                        "o 8192->5120, gate/up 5120->25600, down 25600->5120 (487,587,840 weights); "
+                        "X 131072 tokens per distinct input, bf16, lognormal(sigma=1) channel scales with 1% "
+                        "outlier channels x20, independent draws for the attention, o, MLP and down inputs; "
+                        "W fp32 ~N(0,1/d_in); H and U computed once for q/k/v and once for gate/up "
+                        "(4 Hessians + 4 factorisations + 7 sweeps and 2:4 packs per step); blocksize 128; "
+                        "damp 0.01"),
 }
-WORKLOAD = ("OPT-125M-shaped linear layer: W 768x768 fp32 ~N(0,1/768); X 262144x768 bf16 "
-            "(128 seqs x 2048 tokens, lognormal(sigma=1) channel scales, 1% outlier channels x20); "
-            "two layer prunes per step from X: 2:4 and unstructured 50%; blocksize 128; damp 0.01")
-WORKLOADS[CONFIG] = WORKLOAD
+
+# Oracle sample (cpu_baseline and the reference arm): per distinct input the
+# first SAMPLE_TOKENS tokens of its leading SAMPLE_D channels; the Hessian of
+# that slice, its damped factorisation, and the sweep and pack of SAMPLE_ROWS
+# evenly spaced rows of each matrix over those channels. Each time is scaled
+# to the full workload: Hessian x (n / tokens) x (d / SAMPLE_D)^2, factor x
+# (d / SAMPLE_D)^3, sweep x (d_out / rows) x (d / SAMPLE_D). The sweep's
+# scaling is linear in d although its trailing product grows as d^2, so the
+# scaled oracle time is, if anything, too short for the wide layers.
+SAMPLE_TOKENS = 512
+SAMPLE_D = 3072
+SAMPLE_ROWS = 8
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--config", default=CONFIG, help="workload (default: the OPT-125M-shaped layer)")
+    ap.add_argument("--config", default=CONFIG, help="workload (default: the Qwen3-32B-shaped block)")
     return ap.parse_args()
 
 
-# DRAM bytes (read + write) of one hessian_tc_kernel launch, from the ncu
-# capture summarised in profiles/hessian_tc_kernel_opt125m_768.md; re-capture
-# when the kernel changes.
-HESSIAN_TRAFFIC = {"opt125m_768": 407.6e6}
+# DRAM bytes (read + write) per launch of a phase's kernels, from ncu
+# captures of the current kernels on these workloads (none yet: null).
+TRAFFIC = {}
 
 
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained") or p["bf16_tflops"], "measured"
     except (OSError, KeyError, ValueError):
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# TF32 tensor rate over bf16 (nominal dense figures 1.1 and 2.25 PFLOP/s).
+TF32_OVER_BF16 = 1.1 / 2.25
+
+
+def group_by_input(specs):
+    """{x_key: [specs reading that input]} in order of first appearance."""
+    by_x = {}
+    for sp in specs:
+        by_x.setdefault(sp.x_key, []).append(sp)
+    return by_x
 
 
 # ------------------------------------------------------------------ clocks
@@ -127,68 +158,108 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle
 
-def cpu_baseline(spec, X_cpu, W_cpu, budget_tokens=32768):
-    """The float64 oracle as it stands, on a bounded sample of the workload:
-    the Hessian over the first `budget_tokens` tokens (time scaled to the full
-    token count), damping, factorisation, sweep and packing in full, for
-    both runs. Returns (weights/s, seconds, cores, sample description)."""
-    import numpy as np
-
-    import oracle
-    from workloads import bf16_bits_to_f64
-
+def host_cores() -> int:
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # noqa: BLE001
-        cores = os.cpu_count()
-    n = spec.n_tok
-    t_sample = min(budget_tokens, n)
-    Xs = bf16_bits_to_f64(X_cpu[:t_sample]).numpy()
-    W0 = W_cpu.numpy().astype(np.float64)
+        return os.cpu_count() or 1
+
+
+def oracle_sample_inputs(specs):
+    """What the oracle sample reads, generated on the host: the first
+    SAMPLE_TOKENS tokens x SAMPLE_D channels of each distinct input and
+    SAMPLE_ROWS evenly spaced rows (first SAMPLE_D columns) of every weight
+    matrix, as float64."""
+    from workloads import bf16_bits_to_f64, gen_activations, gen_weights
+    xs, ws, rows = {}, {}, {}
+    for key, group in group_by_input(specs).items():
+        sp = group[0]
+        X = gen_activations(sp, device="cpu", count=min(SAMPLE_TOKENS, sp.n_tok))
+        xs[key] = bf16_bits_to_f64(X[:, :min(SAMPLE_D, sp.d_in)]).numpy()
+    for sp in specs:
+        step = max(1, sp.d_out // SAMPLE_ROWS)
+        r = list(range(0, sp.d_out, step))[:SAMPLE_ROWS]
+        rows[sp.name] = r
+        ws[sp.name] = gen_weights(sp, rows=r)[:, :min(SAMPLE_D, sp.d_in)].numpy().astype("float64")
+    return xs, ws, rows
+
+
+def oracle_sample_time(specs, xs, ws, rows) -> float:
+    """The float64 oracle, as it stands, on the bounded sample; returns the
+    time scaled to one whole step of the workload (seconds)."""
+    import oracle
     total = 0.0
-    for run in spec.runs:
+    for key, group in group_by_input(specs).items():
+        sp0 = group[0]
+        n, d = sp0.n_tok, sp0.d_in
+        X = xs[key]
+        ds = X.shape[1]
         t0 = time.perf_counter()
-        H = oracle.hessian(Xs)
-        t_h = (time.perf_counter() - t0) * (n / t_sample)
+        H = oracle.hessian(X)
+        total += (time.perf_counter() - t0) * (n / X.shape[0]) * (d / ds) ** 2
         t0 = time.perf_counter()
-        oracle.prune_layer(W0, H=H, pattern=run, blocksize=128, damp_ratio=0.01)
-        total += t_h + (time.perf_counter() - t0)
-    weights = spec.weights * len(spec.runs)
-    sample = (f"per run: Hessian over {t_sample} of {n} tokens, time scaled x{n / t_sample:g}; "
-              f"damping, factor, sweep and 2:4 pack in full; runs {list(spec.runs)}")
-    return weights / total, total, cores, sample
+        Hd, _ = oracle.damp(H, 0.01)
+        U = oracle.inverse_cholesky_upper(Hd)
+        total += (time.perf_counter() - t0) * (d / ds) ** 3
+        for sp in group:
+            for run in sp.runs:
+                t0 = time.perf_counter()
+                out = oracle.sweep(ws[sp.name], U, run, 128)
+                if run == "2:4":
+                    oracle.pack24(out["W"], out["mask"])
+                total += (time.perf_counter() - t0) * (sp.d_out / len(rows[sp.name])) * (d / ds)
+    return total
 
 
-def reference_arm(args, spec):
-    """--impl reference: the oracle timed as it stands on the host cores."""
-    import torch
+def oracle_sample_text(specs) -> str:
+    return (f"per distinct input, its first {SAMPLE_TOKENS} tokens x first min(d, {SAMPLE_D}) channels: "
+            f"Hessian (time x n_tok/{SAMPLE_TOKENS} x (d/{SAMPLE_D})^2), damping and factorisation "
+            f"(time x (d/{SAMPLE_D})^3), and per matrix and run the sweep (+ 2:4 pack) of {SAMPLE_ROWS} evenly "
+            f"spaced rows over those channels (time x d_out/{SAMPLE_ROWS} x d/{SAMPLE_D}, linear in d although "
+            f"the trailing product grows as d^2); numpy float64, {len(specs)} matrices")
 
-    from workloads import gen_activations, gen_weights
+
+def cpu_baseline(specs, repeats=2):
+    """The oracle timed on the host cores over the bounded sample."""
+    xs, ws, rows = oracle_sample_inputs(specs)
+    times = [oracle_sample_time(specs, xs, ws, rows) for _ in range(repeats)]
+    t = sum(times) / len(times)
+    weights = sum(sp.weights * len(sp.runs) for sp in specs)
+    return weights / t, t, host_cores(), oracle_sample_text(specs) + f"; mean of {repeats} evaluations"
+
+
+def reference_arm(args, specs, workload):
+    """--impl reference: the oracle, as it stands, on the host cores. Each
+    step times the bounded sample; ms_per_step is that measured time, value
+    the whole workload's weights over the time scaled to it."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    X = gen_activations(spec, device="cpu", count=32768)
-    W = gen_weights(spec)
-    times = []
-    cores = 1
-    sample = ""
+    xs, ws, rows = oracle_sample_inputs(specs)
+    scaled, wall = [], []
     for i in range(args.warmup + args.steps):
-        v, t, cores, sample = cpu_baseline(spec, X, W, budget_tokens=8192)
+        w0 = time.perf_counter()
+        t = oracle_sample_time(specs, xs, ws, rows)
         if i >= args.warmup:
-            times.append(t)
-    t = sum(times) / len(times)
-    value = spec.weights * len(spec.runs) / t
+            scaled.append(t)
+            wall.append(time.perf_counter() - w0)
+    t_full = sum(scaled) / len(scaled)
+    weights = sum(sp.weights * len(sp.runs) for sp in specs)
+    value = weights / t_full
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(wall) / len(wall) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "data": "synthetic", "config": {"workload": workload, "name": args.config},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                         "sample": oracle_sample_text(specs),
+                         "scaled_ms_per_step": t_full * 1e3,
+                         "note": "ms_per_step is the measured time of one step's sample; value divides the "
+                                 "whole workload's weights by the sample time scaled to it"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    del torch
     print(json.dumps(line), flush=True)
 
 
@@ -212,13 +283,78 @@ def aggregate(weights_per_rank_step: int, steps: int, world: int, t_slowest: flo
     return {"value": total / t_slowest, "ms_per_step": t_slowest * 1e3 / steps}
 
 
+# ------------------------------------------------------------------ rooflines
+
+def phase_rooflines(jobs, phase_ms, sustained: bool) -> dict:
+    """Achieved rate of each phase against its bound, from the algorithmic
+    work of the phase (per step) and its measured time (per step).
+
+    hessian  bf16 tensor: n*d*(d+1) flop per input (the upper triangle with
+             the diagonal; symmetric tiles are what the kernel issues).
+    factor   FP32-accurate products on tensor cores (three TF32 products per
+             fp32 product): 2/3*d^3 flop per input (reverse Cholesky d^3/3 +
+             triangular inverse d^3/3); peak = TF32 rate / 3.
+    prune    sweep + selection + lazy trailing update: the larger of the
+             sweep's 12*r*d HBM bytes (W in, W out, errors) and the trailing
+             update's r*(d^2 - d*B) flop at the FP32-accurate rate.
+    pack     HBM: 6.25 bytes per weight (W and mask in, values and metadata
+             out).
+    """
+    hbm, bf16_burst, bf16_sust, kind = peaks()
+    bf16 = bf16_sust if sustained else bf16_burst
+    which = "sustained" if sustained else "burst"
+    fp32acc = bf16 * TF32_OVER_BF16 / 3.0
+    B = 128
+    h_flops = sum(xs.n_tok * xs.d_in * (xs.d_in + 1) for xs, _, _ in jobs)
+    f_flops = sum(2.0 / 3.0 * xs.d_in ** 3 for xs, _, _ in jobs)
+    sweep_bytes = sum(12.0 * sp.d_out * sp.d_in for _, _, mats in jobs for sp, _ in mats)
+    trail_flops = sum(float(sp.d_out) * (sp.d_in ** 2 - sp.d_in * B) for _, _, mats in jobs for sp, _ in mats)
+    pack_bytes = sum(6.25 * sp.d_out * sp.d_in for _, _, mats in jobs for sp, p in mats if p.is_nm)
+    out = {}
+
+    def entry(name, bound, achieved, peak, unit, work, extra=None):
+        e = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+             "frac": achieved / peak if peak else None, "traffic": TRAFFIC.get(name),
+             "work_per_step": work}
+        e.update(extra or {})
+        out[name] = e
+
+    t = phase_ms.get("hessian", 0.0) * 1e-3
+    if t > 0:
+        entry("hessian", "tensor", h_flops / t / 1e12, bf16, "TFLOP/s",
+              f"{h_flops:.4g} flop (n*d*(d+1) per distinct input)",
+              {"kernel": "hessian_tc_kernel", "peak_kind": f"{kind} bf16 {which}"})
+    t = phase_ms.get("factor", 0.0) * 1e-3
+    if t > 0:
+        entry("factor", "tensor", f_flops / t / 1e12, fp32acc, "TFLOP/s",
+              f"{f_flops:.4g} flop (2/3*d^3 per distinct input)",
+              {"kernel": "gemm_tf32x3_kernel + diag_factor_kernel + chain_step_kernel",
+               "peak_kind": f"{kind} bf16 {which} x {TF32_OVER_BF16:.3f} (TF32) / 3 (products per fp32 product)"})
+    t = phase_ms.get("prune", 0.0) * 1e-3
+    if t > 0:
+        t_roof = max(sweep_bytes / (hbm * 1e9), trail_flops / (fp32acc * 1e12))
+        entry("prune", "hbm+tensor", t_roof / t, 1.0, "fraction of roofline time",
+              f"sweep {sweep_bytes:.4g} B; trailing {trail_flops:.4g} flop",
+              {"kernel": "sweep_kernel + gemm_tf32x3_kernel (+ select_kernel)",
+               "roofline_ms": t_roof * 1e3, "measured_ms": t * 1e3,
+               "sweep_hbm_gbs": sweep_bytes / t / 1e9, "trailing_tflops": trail_flops / t / 1e12,
+               "peak_kind": f"{kind} HBM {hbm} GB/s; FP32-accurate tensor {fp32acc:.4g} TFLOP/s"})
+    t = phase_ms.get("pack", 0.0) * 1e-3
+    if t > 0 and pack_bytes:
+        entry("pack", "hbm", pack_bytes / t / 1e9, hbm, "GB/s", f"{pack_bytes:.4g} B (6.25 per weight)",
+              {"kernel": "pack24_kernel", "peak_kind": f"{kind} HBM copy"})
+    return out
+
+
 # ------------------------------------------------------------------ native
 
 def main():
     args = parse()
     from workloads import CONFIGS
+    specs = CONFIGS[args.config]
+    workload = WORKLOADS.get(args.config, args.config)
     if args.impl == "reference":
-        reference_arm(args, CONFIGS[CONFIG][0])
+        reference_arm(args, specs, workload)
         return
 
     import torch
@@ -239,23 +375,19 @@ def main():
     stream = torch.cuda.current_stream()
     # A job is one activation input: its Hessian and factor are computed once,
     # then every weight matrix reading that input is swept (and 2:4 packed).
-    # The OPT-125M workload prunes its layer twice from X (one job per run);
-    # the Qwen3-32B block has four inputs shared by q/k/v, o, gate/up, down.
+    # A single-layer workload with several runs prunes its layer once per run
+    # from X (one job per run).
     jobs = []
-    specs = CONFIGS[args.config]
     if len(specs) == 1:
         sp = specs[0]
         X = gen_activations(sp, device=dev)
         for run in sp.runs:
             jobs.append((sp, X, [(sp, pp.Params(run))]))
     else:
-        by_x = {}
-        for sp in specs:
-            by_x.setdefault(sp.x_key, []).append(sp)
-        for key, group in by_x.items():
+        for key, group in group_by_input(specs).items():
             X = gen_activations(group[0], device=dev)
             jobs.append((group[0], X, [(sp, pp.Params(sp.runs[0])) for sp in group]))
-    layers = []      # (W0, W, LayerGraphs)
+    layers = []      # (W0, W, LayerGraphs, spec, params)
     job_graphs = []
     for xs, X, mats in jobs:
         first = None
@@ -270,39 +402,41 @@ def main():
             else:
                 b = pp.LayerBuffers.sharing(first, sp.d_out, dev)
                 g = pp.LayerGraphs(b, W, None, p, phases=("prune", "pack"))
-            layers.append((W0, W, g))
+            layers.append((W0, W, g, sp, p))
             gl.append(g)
         job_graphs.append(gl)
     weights_per_step = sum(sp.weights for _, _, mats in jobs for sp, _ in mats)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     PH = pp.LayerGraphs.PHASES
 
-    def one_step(ev=None):
-        # ev[j][phase] pairs of events around every graph of job j
-        for j, gl in enumerate(job_graphs):
-            for g in gl:
-                for name in g.phases:
-                    if ev is not None:
-                        ev[j][name][0].record(stream)
-                    g.graphs[name].replay()
-                    if ev is not None:
-                        ev[j][name][1].record(stream)
-
     def prep():
-        for W0, W, _ in layers:
+        for W0, W, _, _, _ in layers:
             W.copy_(W0)
         flush.zero_()
 
+    def step_replay(evs_step=None):
+        # evs_step[j][phase]: one event pair around all graphs of that phase of job j
+        for j, gl in enumerate(job_graphs):
+            for name in PH:
+                ran = False
+                for g in gl:
+                    if name in g.graphs:
+                        if evs_step is not None and not ran:
+                            evs_step[j][name][0].record(stream)
+                        ran = True
+                        g.graphs[name].replay()
+                if ran and evs_step is not None:
+                    evs_step[j][name][1].record(stream)
+
     for _ in range(args.warmup):
         prep()
-        one_step()
+        step_replay()
     torch.cuda.synchronize()
-    for _, _, g in layers:
+    for _, _, g, _, _ in layers:
         pp.raise_on_info(g.bufs.info, where="warm-up")
 
     def mk():
         return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    # one event pair per (job, phase); graphs of the same phase in a job share it
     evs = [[{name: mk() for name in PH} for _ in job_graphs] for _ in range(args.steps)]
     step_ev = [mk() for _ in range(args.steps)]
     clocks = ClockSampler(local)
@@ -313,136 +447,153 @@ def main():
     torch.cuda.synchronize()
     launches0 = pp.kernel_launches()
     wall0 = time.perf_counter()
-    phase = {name: 0.0 for name in PH}
     for s_ in range(args.steps):
         prep()
         step_ev[s_][0].record(stream)
-        for j, gl in enumerate(job_graphs):
-            for name in PH:
-                e0, e1 = evs[s_][j][name]
-                ran = False
-                for g in gl:
-                    if name in g.graphs:
-                        if not ran:
-                            e0.record(stream)
-                            ran = True
-                        g.graphs[name].replay()
-                if ran:
-                    e1.record(stream)
+        step_replay(evs[s_])
         step_ev[s_][1].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
-    launches = pp.kernel_launches() - launches0 + args.steps * sum(sum(g.kernels.values()) for _, _, g in layers)
+    launches = pp.kernel_launches() - launches0 + args.steps * sum(sum(g.kernels.values()) for _, _, g, _, _ in layers)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    for _, _, g in layers:
+    for _, _, g, _, _ in layers:
         pp.raise_on_info(g.bufs.info, where="timed steps")
 
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    phase = {name: 0.0 for name in PH}
+    per_job = [{name: 0.0 for name in PH} for _ in job_graphs]
     for s_ in range(args.steps):
         for j, gl in enumerate(job_graphs):
             for name in PH:
                 if any(name in g.graphs for g in gl):
                     e0, e1 = evs[s_][j][name]
-                    phase[name] += e0.elapsed_time(e1)
+                    ms = e0.elapsed_time(e1)
+                    phase[name] += ms
+                    per_job[j][name] += ms
     phase = {k: v / args.steps for k, v in phase.items()}
+    per_job = [{k: v / args.steps for k, v in pj.items() if v} for pj in per_job]
     t_rank = max_over_ranks(sum(step_ms) / 1e3, dist if world > 1 else None, dev)
     agg = aggregate(weights_per_step, args.steps, world, t_rank)
     value, ms_per_step = agg["value"], agg["ms_per_step"]
-    spec = jobs[0][0]
-    n_hess = len(jobs)
-    n, d = spec.n_tok, spec.d_in
 
-    # roofline of the dominant kernel: the tensor-core Hessian (one launch per job)
-    hbm, bf16_burst, bf16_sust, peak_kind = peaks()
-    hess_flops = sum(xs.n_tok * xs.d_in * (xs.d_in + 1) for xs, _, _ in jobs)
-    achieved = hess_flops / (phase["hessian"] * 1e-3) / 1e12
-    roofline = {"kernel": "hessian_tc_kernel", "bound": "tensor", "achieved": achieved,
-                "peak": bf16_burst, "unit": "TFLOP/s", "frac": achieved / bf16_burst,
-                "traffic": HESSIAN_TRAFFIC.get(args.config), "traffic_unit": "bytes per launch",
-                "peak_kind": f"{peak_kind} bf16 burst",
-                "work": f"n*d*(d+1) = {hess_flops / n_hess:.4g} flop per launch (upper triangle incl. "
-                        f"diagonal), {n_hess} launches per step"}
+    sustained = ms_per_step * args.steps > 2000.0     # seconds-long run: the power-capped peak applies
+    roof = phase_rooflines([(xs, X, mats) for xs, X, mats in jobs], phase, sustained)
+    dominant = max(roof, key=lambda k: phase.get(k, 0.0))
+    roofline = dict(roof[dominant])
+    roofline["phase"] = dominant
+    roofline["share_of_step"] = phase[dominant] / ms_per_step
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "input_dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOADS.get(args.config, args.config), "name": args.config,
+        "config": {"workload": workload, "name": args.config,
                    "weights_per_step": weights_per_step,
                    "launch": "each phase of each layer replayed as a captured CUDA graph",
                    "l2": "flushed between steps (256 MiB write, untimed); every X exceeds the 126 MB L2",
                    "parallelism": f"replicas x{world}"},
         "phases_ms_per_step": phase,
+        "phases_ms_per_input": [{"input": f"{xs.d_in}-wide ({', '.join(sp.name for sp, _ in mats)})", **pj}
+                                for (xs, _, mats), pj in zip(jobs, per_job)],
         "roofline": roofline,
+        "rooflines": roof,
         "gpu_launches": launches,
         "clocks": clk,
         "wall_s_timed": wall,
     }
 
-    # end to end through the public API with host buffers (rank-local), for
-    # workloads whose layers each read their own input
-    single = all(len(m) == 1 for _, _, m in jobs)
-    if not args.no_e2e and single:
-        hp = [(pp.HostPruner(sp.d_out, sp.d_in, xs.n_tok, dev), p, xs, sp) for xs, _, ((sp, p),) in jobs]
-        X_host = {id(X): X.cpu().pin_memory() for _, X, _ in jobs}
-        W_host = [layers[k][0].cpu().pin_memory() for k in range(len(layers))]
-        xs_of = [X for _, X, _ in jobs]
-
-        # Each distinct input is copied from the host once per step, into one
-        # of two device buffers on a copy stream, while the previous step's
-        # prunes run on the compute stream from the other buffer; the layers
-        # that read the same input prune from that copy.
-        keys = list({id(X): X for X in xs_of}.keys())
-        xbuf = {key: [torch.empty_like(X_host[key], device=dev) for _ in range(2)] for key in keys}
+    # end to end through the public API with host buffers (rank-local): every
+    # step copies each distinct X and every W from pinned host memory, prunes
+    # each input's first matrix with sgpt_prune_layer (Hessian, factor,
+    # sweep, pack) and the matrices sharing its H and U with sgpt_prune and
+    # sgpt_pack24, and copies every result back.
+    if not args.no_e2e:
         copy_s, comp_s = torch.cuda.Stream(), torch.cuda.Stream()
+        distinct = {}                 # jobs that read the same X share one copy of it
+        x_of_job = [distinct.setdefault(id(X), len(distinct)) for _, X, _ in jobs]
+        X_dev = {id(X): X for _, X, _ in jobs}
+        X_host = [X_dev[k].cpu().pin_memory() for k in distinct]
+        xbuf = [[torch.empty_like(Xh, device=dev) for _ in range(2)] for Xh in X_host]
         ready = [torch.cuda.Event() for _ in range(2)]
         free = [torch.cuda.Event() for _ in range(2)]
+        pin = dict(pin_memory=True)
+        host = []     # per layer: W in, then W, mask, values, meta out
+        for W0, W, g, sp, p in layers:
+            b = g.bufs
+            host.append({"W_in": W0.cpu().pin_memory(),
+                         "W_out": torch.empty(W.shape, dtype=W.dtype, **pin),
+                         "mask": torch.empty(b.mask.shape, dtype=b.mask.dtype, **pin),
+                         "values": torch.empty(b.values.shape, dtype=b.values.dtype, **pin) if p.is_nm else None,
+                         "meta": torch.empty(b.meta.shape, dtype=b.meta.dtype, **pin) if p.is_nm else None})
+        h2d = sum(Xh.numel() * Xh.element_size() for Xh in X_host) + sum(h["W_in"].numel() * 4 for h in host)
+        d2h = sum(sum(t.numel() * t.element_size() for k, t in h.items() if k != "W_in" and t is not None)
+                  for h in host)
         step_no = [0]
 
         def e2e_step():
-            b = step_no[0] & 1
+            bsel = step_no[0] & 1
             step_no[0] += 1
             with torch.cuda.stream(copy_s):
-                copy_s.wait_event(free[b])          # the step two back is done with this buffer
-                for key in keys:
-                    xbuf[key][b].copy_(X_host[key], non_blocking=True)
-                ready[b].record(copy_s)
+                copy_s.wait_event(free[bsel])       # the step two back is done with this buffer
+                for j, Xh in enumerate(X_host):
+                    xbuf[j][bsel].copy_(Xh, non_blocking=True)
+                ready[bsel].record(copy_s)
             with torch.cuda.stream(comp_s):
-                comp_s.wait_event(ready[b])
-                for k, (h, p, xs, sp) in enumerate(hp):
-                    h.enqueue(W_host[k], None, p, X_device=xbuf[id(xs_of[k])][b])
-                free[b].record(comp_s)
+                comp_s.wait_event(ready[bsel])
+                k = 0
+                for j, (xs, _, mats) in enumerate(jobs):
+                    for m_i, (sp, p) in enumerate(mats):
+                        W0, W, g, _, _ = layers[k]
+                        b, h = g.bufs, host[k]
+                        W.copy_(h["W_in"], non_blocking=True)
+                        pack = p.is_nm
+                        if m_i == 0:
+                            pp.prune_layer(W, b.H, b.U, p, b.mask, b.ws, b.info, X=xbuf[x_of_job[j]][bsel],
+                                           values=b.values if pack else None, meta=b.meta if pack else None,
+                                           row_loss=b.row_loss)
+                        else:
+                            pp.info_clear(b.info)
+                            b.row_loss.zero_()
+                            pp.prune(W, b.U, p, b.mask, b.ws, b.info, row_loss=b.row_loss)
+                            if pack:
+                                pp.pack24(W, b.mask, b.values, b.meta, b.info)
+                        h["W_out"].copy_(W, non_blocking=True)
+                        h["mask"].copy_(b.mask, non_blocking=True)
+                        if pack:
+                            h["values"].copy_(b.values, non_blocking=True)
+                            h["meta"].copy_(b.meta, non_blocking=True)
+                        k += 1
+                free[bsel].record(comp_s)
 
-        for _ in range(max(1, args.warmup // 2)):
+        for _ in range(max(2, args.warmup // 2)):
             e2e_step()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ks = max(1, args.steps // 2)
+        ks = max(2, args.steps // 2)
         e0.record(copy_s)
         comp_s.wait_event(e0)
         for _ in range(ks):
             e2e_step()
         e1.record(comp_s)
         torch.cuda.synchronize()
-        for h, _, _, _ in hp:
-            pp.raise_on_info(h.bufs.info, where="e2e")
+        for _, _, g, _, _ in layers:
+            pp.raise_on_info(g.bufs.info, where="e2e")
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
-        x_bytes = sum(X.numel() * X.element_size() for X in {id(X): X for X in xs_of}.values())
         line["e2e"] = {"value": weights_per_step * ks * world / t_e2e, "unit": UNIT,
-                       "h2d_bytes_per_step": x_bytes + sum(h.W.numel() * 4 for h, _, _, _ in hp),
-                       "d2h_bytes_per_step": sum(h.d2h_bytes(p) for h, p, _, _ in hp),
-                       "ms_per_step": t_e2e * 1e3 / ks,
-                       "note": ("every step copies each distinct X and every W from pinned host memory "
-                                "and each layer's results back; the next step's X copy overlaps this "
-                                "step's pruning (two device buffers)")}
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": t_e2e * 1e3 / ks, "steps": ks,
+                       "note": ("every step copies each distinct X and every W from pinned host memory and "
+                                "every pruned W, mask, 2:4 values and metadata back; the next step's X copies "
+                                "overlap this step's pruning (two device buffers per input)")}
+        del xbuf
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and len(specs) == 1:
-        v, t, cores, sample = cpu_baseline(spec, jobs[0][1][:32768].cpu(), layers[0][0].cpu())
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, t, cores, sample = cpu_baseline(specs)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": sample, "seconds": t}
+                                "sample": sample, "scaled_seconds_per_step": t}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
