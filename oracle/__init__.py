@@ -13,9 +13,11 @@ from .sparsegpt_ref import (  # noqa: F401
     inverse_cholesky_upper,
     mask_bits,
     pack24,
+    pack_nm,
     parse_pattern,
     prune_layer,
     recon_error,
     sweep,
     unpack24,
+    unpack_nm,
 )

@@ -22,6 +22,10 @@ Sources (web pages; cited by title and section):
   "2:4 结构化稀疏的核心机制与生产状态分类": keep 2 of every 4 consecutive
   weights and record the kept positions in 2-bit metadata; worked example
   [0.42, -0.18, 0.07, 0.31] -> [0.42, 0, 0, 0.31].
+* [FT] review of "Sparse Fine-tuning for Inference Acceleration of Large
+  Language Models" (tqpw.cn), section 八 8.4: the GPU formats 2:4, 16:32,
+  16:64 and 16:128 (keep N of every M consecutive weights), the kept
+  positions recorded alongside the values.
 
 Readings where the pages are silent (each is listed in the design notes):
 * scale 2/n on H with n the number of token rows (a scalar; results do not
@@ -41,7 +45,10 @@ Readings where the pages are silent (each is listed in the design notes):
   smallest saliencies first, ties broken by row, then column;
 * the packed 2:4 form keeps the two survivors of each group in index order and
   a 4-bit code a | b << 2 per group (a < b the kept positions), eight codes per
-  32-bit word, least significant first.
+  32-bit word, least significant first;
+* the packed N:M form generalises it: the N survivors of each group of M in
+  index order, and each survivor's in-group position in log2(M) bits, packed
+  along the row least significant bit first (2:4 gives the same words).
 """
 
 from __future__ import annotations
@@ -230,6 +237,60 @@ def unpack24(values, meta, d_in: int):
     return out
 
 
+def pack_nm(W_hat, mask, n_keep: int, m_grp: int):
+    """General N:M packing: values [d_out, d_in*N/M] and meta uint32 words.
+
+    Group g of a row (columns M*g .. M*g+M-1) must keep exactly N weights;
+    they are stored in column order as values N*g .. N*g+N-1 of the row. The
+    in-group position of kept value k of the row (k = N*g + j) takes
+    b = log2(M) bits at bit offset k*b of the row's metadata bit string,
+    which fills uint32 words least significant bit first (a position may
+    continue into the next word); a row has ceil(d_in*N/M*b / 32) words.
+    For 2:4 this is pack24's layout: a | b << 2 per group, eight groups a
+    word.
+    """
+    W_hat = np.asarray(W_hat)
+    mask = np.asarray(mask, dtype=bool)
+    r, d = W_hat.shape
+    b = int(m_grp).bit_length() - 1
+    if m_grp != 1 << b or d % m_grp or not 1 <= n_keep <= m_grp:
+        raise ValueError("M must be a power of two dividing d_in, 1 <= N <= M")
+    groups = d // m_grp
+    nvals = groups * n_keep
+    words = (nvals * b + 31) // 32
+    values = np.zeros((r, nvals), dtype=W_hat.dtype)
+    bitstr = np.zeros((r, words * 32), dtype=np.uint8)
+    for g in range(groups):
+        grp = mask[:, m_grp * g:m_grp * g + m_grp]
+        if not np.all(grp.sum(axis=1) == n_keep):
+            raise ValueError(f"group {g} does not keep exactly {n_keep} of {m_grp}")
+        idx = np.argsort(~grp, axis=1, kind="stable")[:, :n_keep]      # kept, ascending
+        for j in range(n_keep):
+            k = n_keep * g + j
+            values[:, k] = W_hat[np.arange(r), m_grp * g + idx[:, j]]
+            for bit in range(b):
+                bitstr[:, k * b + bit] = (idx[:, j] >> bit) & 1
+    weights = np.uint64(1) << np.arange(32, dtype=np.uint64)
+    meta = (bitstr.reshape(r, words, 32).astype(np.uint64) * weights).sum(axis=2)
+    return values, meta.astype(np.uint32)
+
+
+def unpack_nm(values, meta, d_in: int, n_keep: int, m_grp: int):
+    """Inverse of pack_nm: the dense [d_out, d_in] matrix with zeros."""
+    values = np.asarray(values)
+    meta = np.asarray(meta, dtype=np.uint64)
+    r = values.shape[0]
+    b = int(m_grp).bit_length() - 1
+    bits = ((meta[:, :, None] >> np.arange(32, dtype=np.uint64)) & np.uint64(1)).reshape(r, -1)
+    out = np.zeros((r, d_in), dtype=values.dtype)
+    for k in range(d_in // m_grp * n_keep):
+        pos = np.zeros(r, dtype=np.int64)
+        for bit in range(b):
+            pos |= bits[:, k * b + bit].astype(np.int64) << bit
+        out[np.arange(r), m_grp * (k // n_keep) + pos] = values[:, k]
+    return out
+
+
 def mask_bits(mask) -> np.ndarray:
     """Bool mask [d_out, d_in] -> uint32 words, bit c%32 of word c//32."""
     mask = np.asarray(mask, dtype=bool)
@@ -277,4 +338,6 @@ def prune_layer(W, X=None, H=None, pattern="2:4", blocksize: int = 128,
     kind, n_keep, m_grp, _ = parse_pattern(pattern)
     if kind == "nm" and (n_keep, m_grp) == (2, 4):
         out["values"], out["meta"] = pack24(out["W"], out["mask"])
+    elif kind == "nm":
+        out["values"], out["meta"] = pack_nm(out["W"], out["mask"], n_keep, m_grp)
     return out

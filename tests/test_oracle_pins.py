@@ -366,6 +366,55 @@ def test_pack_and_mask_word_layout_beyond_the_first_word():
     assert np.array_equal(oracle.unpack24(values, meta_want, d), Wm)
 
 
+def test_pack_nm_hand_derived_words():
+    """General N:M layout (golden file): 3-bit positions of a 4:8 row, and
+    5-bit positions of a 16:32 row that run across word boundaries."""
+    g = _golden("pack_nm_layout.json")
+    for case in g["cases"]:
+        n, m = (int(x) for x in case["pattern"].split(":"))
+        d = case["d_in"]
+        W = np.array([[100.0 + c for c in range(d)]])
+        mask = np.zeros((1, d), dtype=bool)
+        for grp, kept in enumerate(case["kept"]):
+            mask[0, [m * grp + j for j in kept]] = True
+        Wm = np.where(mask, W, 0.0)
+        values, meta = oracle.pack_nm(Wm, mask, n, m)
+        want = np.array([[int(h, 16) for h in case["meta_words_hex"]]], dtype=np.uint32)
+        assert np.array_equal(meta, want), case["pattern"]
+        assert np.array_equal(values[0], np.array(case["values"], dtype=np.float64))
+        assert np.array_equal(oracle.unpack_nm(values, want, d, n, m), Wm)
+
+
+def test_pack_nm_reduces_to_pack24_and_round_trips(rng):
+    W, X = _layer(rng, r=5, d=128, n=200)
+    out = oracle.prune_layer(W, X=X, pattern="2:4", blocksize=64)
+    v24, m24 = oracle.pack24(out["W"], out["mask"])
+    v, m = oracle.pack_nm(out["W"], out["mask"], 2, 4)
+    assert np.array_equal(v, v24) and np.array_equal(m, m24)
+    for pat in ["1:4", "3:4", "4:8", "16:32", "16:64", "16:128", "8:16"]:
+        n, mm = (int(x) for x in pat.split(":"))
+        o = oracle.prune_layer(W, X=X, pattern=pat, blocksize=128)
+        groups = o["mask"].reshape(5, -1, mm).sum(axis=2)
+        assert np.all(groups == n), pat
+        assert np.array_equal(oracle.unpack_nm(o["values"], o["meta"], 128, n, mm), o["W"]), pat
+        b = mm.bit_length() - 1
+        assert o["meta"].shape == (5, (128 // mm * n * b + 31) // 32)
+    with pytest.raises(ValueError):
+        oracle.pack_nm(out["W"], np.ones_like(out["mask"]), 4, 8)
+
+
+@pytest.mark.parametrize("pattern", ["1:4", "3:4", "4:8", "8:16"])
+def test_nm_sweep_equals_frozen_prefix_least_squares(rng, pattern):
+    """N of M on the compensated weights at each group start ([SGPT] 十四
+    14.4), against the general-solve reference, across several blocks."""
+    W, X = _layer(rng, r=5, d=32, n=80, scale_spread=1.5)
+    _, Hd, U = _factor(X)
+    out = oracle.sweep(W, U, pattern, blocksize=16)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, pattern)
+    assert np.array_equal(out["mask"], ref_mask)
+    assert np.allclose(out["W"], ref_W, atol=1e-11)
+
+
 # ---------------------------------------------------------------- mutations
 
 _MUTATIONS = [
