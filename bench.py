@@ -526,8 +526,8 @@ def main():
             host.append({"W_in": W0.cpu().pin_memory(),
                          "W_out": torch.empty(W.shape, dtype=W.dtype, **pin),
                          "mask": torch.empty(b.mask.shape, dtype=b.mask.dtype, **pin),
-                         "values": torch.empty(b.values.shape, dtype=b.values.dtype, **pin) if p.is_nm else None,
-                         "meta": torch.empty(b.meta.shape, dtype=b.meta.dtype, **pin) if p.is_nm else None})
+                         "values": torch.empty(b.values.shape, dtype=b.values.dtype, **pin) if b.packs(p) else None,
+                         "meta": torch.empty(b.meta.shape, dtype=b.meta.dtype, **pin) if b.packs(p) else None})
         h2d = sum(Xh.numel() * Xh.element_size() for Xh in X_host) + sum(h["W_in"].numel() * 4 for h in host)
         d2h = sum(sum(t.numel() * t.element_size() for k, t in h.items() if k != "W_in" and t is not None)
                   for h in host)
@@ -549,7 +549,7 @@ def main():
                         W0, W, g, _, _ = layers[k]
                         b, h = g.bufs, host[k]
                         W.copy_(h["W_in"], non_blocking=True)
-                        pack = p.is_nm
+                        pack = b.packs(p)
                         if m_i == 0:
                             pp.prune_layer(W, b.H, b.U, p, b.mask, b.ws, b.info, X=xbuf[x_of_job[j]][bsel],
                                            values=b.values if pack else None, meta=b.meta if pack else None,
@@ -559,7 +559,7 @@ def main():
                             b.row_loss.zero_()
                             pp.prune(W, b.U, p, b.mask, b.ws, b.info, row_loss=b.row_loss)
                             if pack:
-                                pp.pack24(W, b.mask, b.values, b.meta, b.info)
+                                pp.pack_nm(W, b.mask, *p.nm, b.values, b.meta, b.info)
                         h["W_out"].copy_(W, non_blocking=True)
                         h["mask"].copy_(b.mask, non_blocking=True)
                         if pack:

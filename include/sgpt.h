@@ -10,7 +10,9 @@
  *   - Hessian proxy H = X X^T: same page, section 七.
  *   - Optimal-Brain-Surgeon removal with compensation: section 八.
  *   - Layer-wise pipeline, columns processed block by block: section 十一.
- *   - N:M (2:4) semi-structured sparsity: section 十四 14.4.
+ *   - N:M (2:4) semi-structured sparsity: section 十四 14.4. The N:M GPU formats
+ *     2:4, 16:32, 16:64 and 16:128: "Sparse Fine-tuning for Inference
+ *     Acceleration of Large Language Models" review (tqpw.cn), section 八 8.4.
  *   - 2:4 storage, values plus 2-bit position metadata: "LLM 2:4 structured
  *     sparsity production guide" (oh-bug.com), section "2:4 结构化稀疏的核心机制
  *     与生产状态分类".
@@ -57,7 +59,7 @@ typedef enum sgpt_status {
   SGPT_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up          */
   SGPT_ERR_CUDA = 5,        /* a CUDA runtime call failed                  */
   SGPT_ERR_UNSUPPORTED = 6, /* valid request this library version does not implement */
-  SGPT_ERR_BAD_MASK = 7,    /* pack: a group does not keep exactly 2 of 4  */
+  SGPT_ERR_BAD_MASK = 7,    /* pack: a group does not keep exactly n of m  */
   SGPT_ERR_WORKSPACE = 8    /* ws too small or misaligned                  */
 } sgpt_status;
 
@@ -71,7 +73,9 @@ typedef enum sgpt_status {
 
 typedef struct sgpt_params {
   int pattern;    /* SGPT_PATTERN_UNSTRUCTURED or SGPT_PATTERN_NM            */
-  int n, m;       /* N:M - keep n of every m consecutive inputs (2 and 4)    */
+  int n, m;       /* N:M - keep n of every m consecutive inputs: m a power
+                     of two from 4 to 128, 1 <= n <= m, blocksize % m == 0 and
+                     d_in % m == 0 (SGPT_ERR_UNSUPPORTED for other m)        */
   float sparsity; /* unstructured - fraction pruned in each block, [0, 1)    */
   int blocksize;  /* columns per OBS block: 32, 64, 96 or 128                */
   float damp;     /* damping ratio (0.01 = 1% of the mean diagonal), >= 0    */
@@ -190,6 +194,27 @@ sgpt_status sgpt_prune_noalloc(float* W, int d_out, int d_in, int ldw, const flo
 sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint32_t* mask_bits,
                         float* values, uint32_t* meta, int* dev_info, void* stream);
 
+/* N:M packing (sparse fine-tuning review, section 八 8.4: keep N of every M
+ * weights and record the kept positions; the 2:4 guide's 2-bit positions
+ * generalised to log2(M) bits):
+ *   values [d_out x d_in*n/m] fp32: the n kept weights of each group of m,
+ *          in column order (value g*n + j of a row is the j-th kept weight
+ *          of group g);
+ *   meta   [d_out x sgpt_pack_nm_meta_words(d_in, n, m)] uint32: the
+ *          in-group position of value k of a row takes log2(m) bits at bit
+ *          offset k*log2(m) of the row's bit string, which fills the row's
+ *          words least significant bit first (a position may continue into
+ *          the next word). For 2:4 the words equal sgpt_pack24's.
+ * m a power of two from 4 to 128 (else SGPT_ERR_UNSUPPORTED), 1 <= n <= m,
+ * d_in % m == 0. A group whose mask does not keep exactly n sets
+ * *dev_info = BAD_MASK. */
+sgpt_status sgpt_pack_nm(const float* W, int d_out, int d_in, int ldw, const uint32_t* mask_bits, int n, int m,
+                         float* values, uint32_t* meta, int* dev_info, void* stream);
+
+/* Metadata words per row of sgpt_pack_nm: ceil(d_in/m * n * log2(m) / 32),
+ * or -1 for arguments sgpt_pack_nm rejects. */
+int sgpt_pack_nm_meta_words(int d_in, int n, int m);
+
 /* Layer reconstruction error (SparseGPT review, section 六, the objective):
  * num_den[0] = tr(dW H dW^T), num_den[1] = tr(W0 H W0^T), dW = W0 - W, in
  * fp64 on the device (FP32 products, fp64 sums in a fixed order: the result
@@ -203,8 +228,9 @@ sgpt_status sgpt_recon_error(const float* W0, const float* W, int d_out, int d_i
 
 /* One layer end to end: if X != NULL, H = X^T X over its n_tok rows, else H
  * must already hold that sum; then U = sgpt_factor(H), sgpt_prune, and for
- * 2:4 sgpt_pack24 (values/meta may be NULL to skip packing). U and H must
- * not alias. *dev_info is cleared first. */
+ * N:M sgpt_pack_nm (values/meta sized as sgpt_pack_nm states; NULL to skip
+ * packing). U and H must not alias. *dev_info is cleared first. Every
+ * argument is checked before the first launch. */
 sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint16_t* X,
                              int64_t n_tok, float* H, float* U, const sgpt_params* p,
                              uint32_t* mask_bits, float* values, uint32_t* meta,

@@ -22,6 +22,8 @@ from .sgpt import (  # noqa: F401
     lib,
     new_info,
     pack24,
+    pack_nm,
+    pack_nm_meta_words,
     prune,
     prune_layer,
     prune_noalloc,

@@ -32,6 +32,9 @@ bool valid_dout(int d_out) { return d_out >= 1 && d_out <= (1 << 24); }
 
 sgpt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SGPT_OK : SGPT_ERR_CUDA; }
 
+// Group sizes the N:M sweep and pack support: powers of two from 4 to 128.
+bool valid_m(int m) { return m >= 4 && m <= 128 && (m & (m - 1)) == 0; }
+
 sgpt_status check_params(const sgpt_params* p) {
   if (!p) return SGPT_ERR_INVALID_ARG;
   if (p->blocksize < 32 || p->blocksize > kMaxBlock || p->blocksize % 32) return SGPT_ERR_INVALID_ARG;
@@ -39,7 +42,8 @@ sgpt_status check_params(const sgpt_params* p) {
   if (p->forced != 0 && p->forced != 1) return SGPT_ERR_INVALID_ARG;
   if (p->pattern == SGPT_PATTERN_NM) {
     if (p->n <= 0 || p->m <= 0 || p->n > p->m) return SGPT_ERR_INVALID_ARG;
-    if (!(p->n == 2 && p->m == 4)) return SGPT_ERR_UNSUPPORTED;
+    if (!valid_m(p->m)) return SGPT_ERR_UNSUPPORTED;
+    if (p->blocksize % p->m) return SGPT_ERR_INVALID_ARG;
   } else if (p->pattern == SGPT_PATTERN_UNSTRUCTURED) {
     if (!(p->sparsity >= 0.f && p->sparsity < 1.f)) return SGPT_ERR_INVALID_ARG;
   } else {
@@ -158,6 +162,7 @@ sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U, c
   if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
   sgpt_status s = check_params(p);
   if (s != SGPT_OK) return s;
+  if (p->pattern == SGPT_PATTERN_NM && d_in % p->m) return SGPT_ERR_INVALID_ARG;
   s = check_ws(ws, ws_bytes, prune_ws_bytes(d_out, d_in));
   if (s != SGPT_OK) return s;
   return from_cuda(launch_prune(W, d_out, d_in, ldw, U, *p, mask_bits, row_loss, ws, dev_info,
@@ -173,6 +178,7 @@ sgpt_status sgpt_prune_noalloc(float* W, int d_out, int d_in, int ldw, const flo
   if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
   sgpt_status s = check_params(p);
   if (s != SGPT_OK) return s;
+  if (p->pattern == SGPT_PATTERN_NM && d_in % p->m) return SGPT_ERR_INVALID_ARG;
   return from_cuda(launch_prune_noalloc(W, d_out, d_in, ldw, U, *p, mask_bits, row_loss, dev_info,
                                         as_stream(stream)));
 }
@@ -184,6 +190,25 @@ sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint
     return SGPT_ERR_INVALID_ARG;
   if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
   return from_cuda(launch_pack24(W, ldw, d_out, d_in, mask_bits, values, meta, dev_info, as_stream(stream)));
+}
+
+int sgpt_pack_nm_meta_words(int d_in, int n, int m) {
+  if (!valid_din(d_in) || !valid_m(m) || n < 1 || n > m || d_in % m) return -1;
+  return packnm_meta_words(d_in, n, m);
+}
+
+sgpt_status sgpt_pack_nm(const float* W, int d_out, int d_in, int ldw, const uint32_t* mask_bits, int n, int m,
+                         float* values, uint32_t* meta, int* dev_info, void* stream) {
+  if (!W || !mask_bits || !values || !meta || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(mask_bits) || !aligned16(meta))
+    return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  if (n < 1 || n > m || m < 1) return SGPT_ERR_INVALID_ARG;
+  if (!valid_m(m)) return SGPT_ERR_UNSUPPORTED;
+  if (d_in % m) return SGPT_ERR_INVALID_ARG;
+  if (n == 2 && m == 4)      // the same words, by the 2:4 kernel
+    return from_cuda(launch_pack24(W, ldw, d_out, d_in, mask_bits, values, meta, dev_info, as_stream(stream)));
+  return from_cuda(launch_packnm(W, ldw, d_out, d_in, mask_bits, n, m, values, meta, dev_info, as_stream(stream)));
 }
 
 sgpt_status sgpt_recon_error(const float* W0, const float* W, int d_out, int d_in, int ldw, const float* H,
@@ -213,6 +238,7 @@ sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint1
   if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
   s = check_ws(ws, ws_bytes, sgpt_workspace_bytes(d_out, d_in, X ? n_tok : 0, p));
   if (s != SGPT_OK) return s;
+  if (p->pattern == SGPT_PATTERN_NM && d_in % p->m) return SGPT_ERR_INVALID_ARG;
   const bool pack = p->pattern == SGPT_PATTERN_NM && values && meta;
   if ((values || meta) && !pack) return SGPT_ERR_INVALID_ARG;
   if (pack && (!aligned16(values) || !aligned16(meta))) return SGPT_ERR_INVALID_ARG;
@@ -224,7 +250,7 @@ sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint1
     return SGPT_ERR_CUDA;
   if ((s = sgpt_prune(W, d_out, d_in, ldw, U, p, mask_bits, row_loss, ws, ws_bytes, dev_info, stream)) != SGPT_OK)
     return s;
-  if (pack) s = sgpt_pack24(W, d_out, d_in, ldw, mask_bits, values, meta, dev_info, stream);
+  if (pack) s = sgpt_pack_nm(W, d_out, d_in, ldw, mask_bits, p->n, p->m, values, meta, dev_info, stream);
   return s;
 }
 

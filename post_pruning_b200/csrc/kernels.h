@@ -28,6 +28,9 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
 // pack.cu
 cudaError_t launch_pack24(const float* W, long long ldw, int rows, int d, const uint32_t* mask,
                           float* values, uint32_t* meta, int* info, cudaStream_t st);
+int packnm_meta_words(int d, int n, int m);
+cudaError_t launch_packnm(const float* W, long long ldw, int rows, int d, const uint32_t* mask, int n, int m,
+                          float* values, uint32_t* meta, int* info, cudaStream_t st);
 size_t recon_ws_bytes(int rows, int d);
 cudaError_t launch_recon(const float* W0, const float* W, int rows, int d, long long ldw,
                          const float* H, double* num_den, void* ws, cudaStream_t st);

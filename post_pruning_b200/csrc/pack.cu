@@ -1,9 +1,11 @@
-// 2:4 packing and the layer reconstruction error.
+// 2:4 and N:M packing and the layer reconstruction error.
 //
 // Packing follows the 2:4 production guide (oh-bug.com, section on the 2:4
 // mechanism): of every four consecutive weights along the input dimension two
 // are kept, stored in column order, and their positions are recorded as
-// 2-bit indices.
+// 2-bit indices. The N:M formats of the sparse fine-tuning review
+// (tqpw.cn, section 八 8.4: 16:32, 16:64, 16:128) keep N of every M and
+// record each kept position in log2(M) bits the same way.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -55,6 +57,70 @@ cudaError_t launch_pack24(const float* W, long long ldw, int rows, int d, const 
                           float* values, uint32_t* meta, int* info, cudaStream_t st) {
   const long long n = (long long)rows * (d / 32);
   pack24_kernel<<<(unsigned)cdivll(n, 256), 256, 0, st>>>(W, ldw, rows, d, mask, values, meta, info);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// General N:M packing: one thread per (row, group of M). The group's mask
+// bits (M <= 32: part of one word; M = 64, 128: whole words) give the kept
+// positions in column order; kept value j of group g goes to value g*N + j
+// of the row and its position (log2(M) bits) to bit offset (g*N + j) *
+// log2(M) of the row's metadata bits, least significant first. Positions
+// that continue into the next word, and words shared between groups, are
+// merged with atomicOr into metadata the launcher zeroed (OR is order-free:
+// the result is deterministic).
+__global__ void __launch_bounds__(256) packnm_kernel(const float* __restrict__ W, long long ldw, int rows, int d,
+                                                     const uint32_t* __restrict__ mask, int n, int m, int lg,
+                                                     int meta_words, float* __restrict__ values,
+                                                     uint32_t* __restrict__ meta, int* info) {
+  if (info_set(info)) return;
+  const int groups = d / m;
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (long long)rows * groups) return;
+  const int row = (int)(t / groups), g = (int)(t - (long long)row * groups);
+  const uint32_t* mrow = mask + (long long)row * (d / 32);
+  const float* wrow = W + (long long)row * ldw + (long long)g * m;
+  float* vrow = values + (long long)row * (d / m) * n;
+  uint32_t* meta_row = meta + (long long)row * meta_words;
+  int cnt = 0;
+  for (int w0 = 0; w0 < m; w0 += 32) {
+    const int c = g * m + w0;                       // first column of this 32-bit slice
+    uint32_t bitsw = mrow[c >> 5] >> (c & 31);
+    if (m < 32) bitsw &= (1u << m) - 1u;
+    while (bitsw) {
+      const int pos = w0 + __ffs(bitsw) - 1;          // in-group position, ascending
+      bitsw &= bitsw - 1u;
+      if (cnt < n) {
+        const long long k = (long long)g * n + cnt;
+        vrow[k] = wrow[pos];
+        const long long off = k * lg;
+        const int word = (int)(off >> 5), sh = (int)(off & 31);
+        atomicOr(meta_row + word, (uint32_t)pos << sh);
+        if (sh + lg > 32) atomicOr(meta_row + word + 1, (uint32_t)pos >> (32 - sh));
+      }
+      ++cnt;
+    }
+  }
+  if (cnt != n) set_info(info, SGPT_INFO_BAD_MASK);
+}
+
+int packnm_meta_words(int d, int n, int m) {
+  int lg = 0;
+  while ((1 << lg) < m) ++lg;
+  const long long bits = (long long)(d / m) * n * lg;
+  return (int)((bits + 31) / 32);
+}
+
+cudaError_t launch_packnm(const float* W, long long ldw, int rows, int d, const uint32_t* mask, int n, int m,
+                          float* values, uint32_t* meta, int* info, cudaStream_t st) {
+  int lg = 0;
+  while ((1 << lg) < m) ++lg;
+  const int words = packnm_meta_words(d, n, m);
+  cudaError_t e = cudaMemsetAsync(meta, 0, (size_t)rows * words * sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  const long long threads = (long long)rows * (d / m);
+  packnm_kernel<<<(unsigned)cdivll(threads, 256), 256, 0, st>>>(W, ldw, rows, d, mask, n, m, lg, words, values,
+                                                                 meta, info);
   count_launches(1);
   return cudaGetLastError();
 }

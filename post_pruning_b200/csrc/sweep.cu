@@ -6,7 +6,7 @@
 //      row * bw + column), one cooperative launch of select_kernel with a
 //      grid barrier per 8-bit digit;
 //   2. sweep_kernel: one warp per row, one 4-column group per lane; the
-//      groups are processed in order: mask decision (2:4 at each group start
+//      groups are processed in order: mask decision (N:M at each group start
 //      on the compensated weights), e = (w_q - p_q) / U_qq (as a product with
 //      the reciprocal), rank-4 update of the rest of the block with the U
 //      rows held in shared memory;
@@ -31,7 +31,10 @@ constexpr int kSweepWarps = 8;             // warps per CTA
 constexpr int kSweepThreads = kSweepWarps * 32;
 constexpr size_t kSweepSmem = (size_t)kMaxBlock * kMaxBlock * sizeof(float);
 
-enum SweepMode { kModeNM24 = 0, kModeThreshold = 1, kModeForced = 2 };
+// kModeNM4: N of every 4 (2:4 on the hot path); kModeNMG: N of every M for
+// M = 8 .. 128; kModeThreshold: unstructured, prune keys below a threshold
+// found by select_kernel; kModeForced: the mask is an input.
+enum SweepMode { kModeNM4 = 0, kModeThreshold = 1, kModeForced = 2, kModeNMG = 3 };
 
 __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsigned idx) {
   return ((unsigned long long)__float_as_uint(saliency(w, inv_u)) << 32) | idx;
@@ -53,12 +56,21 @@ __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsi
 // the U values are loaded before the weights arrive. Two rows per warp halve
 // the owner work per row (for tall layers); one row per warp gives more
 // parallelism to short ones.
-template <int MODE, int ROWS>
+// N:M with M > 4 (kModeNMG): at the first column of each group of M the
+// lanes holding the group's columns rank them by saliency on the weights as
+// compensated so far (every later column has received the updates of every
+// earlier group by then): each member lane receives the group's M
+// saliencies by shuffle and counts, for each of its own columns, the group
+// columns that beat it (larger saliency, or equal and lower column); the N
+// best are kept. An M-group covers M/4 consecutive lanes of one column span,
+// or (M = 128 with two rows per warp) every lane of both spans. The group
+// steps then apply the decided bits like a forced mask.
+template <int MODE, int ROWS, int M>
 __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
     const float* __restrict__ U, uint32_t* __restrict__ mask, float* __restrict__ row_loss,
     float* __restrict__ Err, float* __restrict__ Err_lo, const unsigned long long* __restrict__ thr,
-    int* info) {
+    int nkeep, int* info) {
   constexpr int LPR = 32 / ROWS;                 // lanes per row
   constexpr int CPL = 4 * ROWS;                  // columns per lane
   if (cta_info_set(info)) return;
@@ -158,9 +170,56 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 #pragma unroll
       for (int t = 0; t < 4; ++t) wo[t] = __shfl_sync(0xffffffffu, w[4 * gi + t], owner);
       const float r[4] = {ri.x, ri.y, ri.z, ri.w};
+      if (MODE == kModeNMG && (q0 & (M - 1)) == 0) {
+        // decide the M-group that starts here
+        constexpr int NSPAN = (M > SPAN) ? ROWS : 1;        // column spans the group covers
+        constexpr int NL = (M > SPAN) ? LPR : M / 4;        // lanes it covers in each span
+        const int gl0 = (M > SPAN) ? 0 : (q0 - gi * SPAN) / 4;   // its first lane (row-relative)
+        const bool member = sl >= gl0 && sl < gl0 + NL;
+        float ms[4 * NSPAN];
+        int rk[4 * NSPAN];
+#pragma unroll
+        for (int vv = 0; vv < NSPAN; ++vv)
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int v = (gi + vv < ROWS) ? gi + vv : gi;
+            ms[4 * vv + t] = saliency(w[4 * v + t], Uinv[c0 + v * SPAN + t]);
+            rk[4 * vv + t] = 0;
+          }
+#pragma unroll 1
+        for (int k = 0; k < NL; ++k) {
+          const int src = base + gl0 + k;
+#pragma unroll
+          for (int vv = 0; vv < NSPAN; ++vv)
+#pragma unroll
+            for (int t2 = 0; t2 < 4; ++t2) {
+              const float so = __shfl_sync(0xffffffffu, ms[4 * vv + t2], src);
+              const int co = (gi + vv) * SPAN + 4 * (gl0 + k) + t2;
+#pragma unroll
+              for (int vm = 0; vm < NSPAN; ++vm)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  const int mc = (gi + vm) * SPAN + c0 + t;
+                  const float mv = ms[4 * vm + t];
+                  if (so > mv || (so == mv && co < mc)) ++rk[4 * vm + t];
+                }
+            }
+        }
+        if (mine && member) {
+#pragma unroll
+          for (int vm = 0; vm < NSPAN; ++vm)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const int j = 4 * (gi + vm) + t;
+              if (j < CPL) keep = (keep & ~(1u << j)) | ((rk[4 * vm + t] < nkeep ? 1u : 0u) << j);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) kb[j] = __ballot_sync(0xffffffffu, (keep >> j) & 1u);
+      }
       uint32_t km;
-      if (MODE == kModeNM24) {
-        // 2 of 4 on the compensated weights; ties keep the lower column.
+      if (MODE == kModeNM4) {
+        // N of 4 on the compensated weights; ties keep the lower column.
         float slv[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) slv[t] = saliency(wo[t], r[t]);
@@ -171,7 +230,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 #pragma unroll
           for (int o = 0; o < 4; ++o)
             if (o != t && (slv[o] > slv[t] || (slv[o] == slv[t] && o < t))) ++rank;
-          if (rank < 2) km |= 1u << t;
+          if (rank < nkeep) km |= 1u << t;
         }
       } else {
         km = 0;
@@ -257,29 +316,50 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 // per row), one for short ones (twice the warps in flight).
 static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 2 : 1; }
 
-template <int MODE>
-static cudaError_t launch_sweep(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
-                                uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
-                                const unsigned long long* thr, int* info, cudaStream_t st) {
+template <int MODE, int M>
+static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
+                                  uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
+                                  const unsigned long long* thr, int nkeep, int* info, cudaStream_t st) {
   static PerDevice attrs;
   const cudaError_t ea = once_per_device(attrs, [] {
     const cudaError_t r =
-        cudaFuncSetAttribute(sweep_kernel<MODE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+        cudaFuncSetAttribute(sweep_kernel<MODE, 1, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
     return r != cudaSuccess
                ? r
-               : cudaFuncSetAttribute(sweep_kernel<MODE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+               : cudaFuncSetAttribute(sweep_kernel<MODE, 2, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kSweepSmem);
   });
   if (ea != cudaSuccess) return ea;
   const int grid = cdiv(rows, kSweepWarps * rpw);
   if (rpw == 2)
-    sweep_kernel<MODE, 2><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
-                                                                   Err_lo, thr, info);
+    sweep_kernel<MODE, 2, M><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss,
+                                                                      Err, Err_lo, thr, nkeep, info);
   else
-    sweep_kernel<MODE, 1><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss, Err,
-                                                                   Err_lo, thr, info);
+    sweep_kernel<MODE, 1, M><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss,
+                                                                      Err, Err_lo, thr, nkeep, info);
   count_launches(1);
   return cudaGetLastError();
+}
+
+// The sweep of one block for a pattern: forced mask, unstructured threshold,
+// N of 4, or N of M = 8 .. 128.
+static cudaError_t launch_sweep(const sgpt_params& p, int rpw, float* W, long long ldw, int rows, int d, int i1,
+                                int bw, const float* U, uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
+                                const unsigned long long* thr, int* info, cudaStream_t st) {
+#define SGPT_SWEEP(MODE, M) \
+  launch_sweep_m<MODE, M>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, p.n, info, st)
+  if (p.forced) return SGPT_SWEEP(kModeForced, 4);
+  if (p.pattern != SGPT_PATTERN_NM) return SGPT_SWEEP(kModeThreshold, 4);
+  switch (p.m) {
+    case 4: return SGPT_SWEEP(kModeNM4, 4);
+    case 8: return SGPT_SWEEP(kModeNMG, 8);
+    case 16: return SGPT_SWEEP(kModeNMG, 16);
+    case 32: return SGPT_SWEEP(kModeNMG, 32);
+    case 64: return SGPT_SWEEP(kModeNMG, 64);
+    case 128: return SGPT_SWEEP(kModeNMG, 128);
+  }
+#undef SGPT_SWEEP
+  return cudaErrorInvalidValue;
 }
 
 // --------------------------------------------------------- trailing update
@@ -528,19 +608,12 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
   const int rpw = sweep_rows_per_warp(rows);
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
-    if (p.forced) {
-      e = launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr,
-                                    info, st);
-    } else if (p.pattern == SGPT_PATTERN_NM) {
-      e = launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, nullptr,
-                                  info, st);
-    } else {
+    if (!p.forced && p.pattern == SGPT_PATTERN_UNSTRUCTURED) {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
-      e = launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo,
-                                       &w.sel->thr, info, st);
     }
+    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, info, st);
     if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {
@@ -616,18 +689,12 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
   const int rpw = sweep_rows_per_warp(rows);
   for (int i1 = 0; i1 < d; i1 += B) {
     const int bw = min(B, d - i1);
-    if (p.forced) {
-      e = launch_sweep<kModeForced>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info,
-                                    st);
-    } else if (p.pattern == SGPT_PATTERN_NM) {
-      e = launch_sweep<kModeNM24>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, nullptr, info, st);
-    } else {
+    if (!p.forced && p.pattern == SGPT_PATTERN_UNSTRUCTURED) {
       const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
-      e = launch_sweep<kModeThreshold>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr,
-                                       info, st);
     }
+    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info, st);
     if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {

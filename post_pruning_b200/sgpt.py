@@ -32,7 +32,7 @@ EXPORTS = (
     "sgpt_workspace_bytes",
     "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
     "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
-    "sgpt_recon_error", "sgpt_prune_layer",
+    "sgpt_pack_nm", "sgpt_pack_nm_meta_words", "sgpt_recon_error", "sgpt_prune_layer",
 )
 
 
@@ -52,7 +52,7 @@ class _Params(ctypes.Structure):
 @dataclass(frozen=True)
 class Params:
     """Sparsity pattern and solver knobs (mirrors sgpt_params)."""
-    pattern: str = "2:4"        # "2:4" or "unstructured:<fraction>"
+    pattern: str = "2:4"        # "N:M" (e.g. "2:4", "16:64") or "unstructured:<fraction>"
     blocksize: int = 128
     damp: float = 0.01
     forced: bool = False
@@ -60,6 +60,12 @@ class Params:
     @property
     def is_nm(self) -> bool:
         return not self.pattern.startswith("unstructured")
+
+    @property
+    def nm(self) -> tuple[int, int]:
+        """(N, M) of an N:M pattern."""
+        n, m = (int(x) for x in self.pattern.split(":"))
+        return n, m
 
     @property
     def sparsity(self) -> float:
@@ -102,6 +108,8 @@ def lib() -> ctypes.CDLL:
         "sgpt_prune": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, sz, vp, vp]),
         "sgpt_prune_noalloc": (i32, [vp, i32, i32, i32, vp, pp, vp, vp, vp, vp]),
         "sgpt_pack24": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "sgpt_pack_nm": (i32, [vp, i32, i32, i32, vp, i32, i32, vp, vp, vp, vp]),
+        "sgpt_pack_nm_meta_words": (i32, [i32, i32, i32]),
         "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
                                    vp, sz, vp, vp]),
@@ -277,6 +285,31 @@ def pack24(W: torch.Tensor, mask: torch.Tensor, values: torch.Tensor, meta: torc
                              _stream(stream)), "sgpt_pack24")
 
 
+def pack_nm_meta_words(d_in: int, n: int, m: int) -> int:
+    """uint32 metadata words per row of an N:M pack (-1 if unsupported)."""
+    return int(lib().sgpt_pack_nm_meta_words(d_in, n, m))
+
+
+def pack_nm(W: torch.Tensor, mask: torch.Tensor, n: int, m: int, values: torch.Tensor, meta: torch.Tensor,
+            dev_info: torch.Tensor, stream=None):
+    """N:M packing (sgpt_pack_nm): values [d_out, d_in*n/m] fp32, meta
+    [d_out, pack_nm_meta_words(d_in, n, m)] int32."""
+    _dev(W, torch.float32, "W")
+    _dev(values, torch.float32, "values")
+    _dev(mask, torch.int32, "mask")
+    _dev(meta, torch.int32, "meta")
+    ldw = _rowmajor(W, "W")
+    r, d = W.shape
+    words = pack_nm_meta_words(d, n, m)
+    if words < 0:
+        raise ValueError(f"unsupported N:M {n}:{m} for d_in {d}")
+    if values.shape != (r, d * n // m) or meta.shape != (r, words) or not values.is_contiguous() \
+            or not meta.is_contiguous():
+        raise ValueError(f"values must be [d_out, {d * n // m}] and meta [d_out, {words}], contiguous")
+    _check(lib().sgpt_pack_nm(_ptr(W), r, d, ldw, _ptr(mask), n, m, _ptr(values), _ptr(meta), _ptr(dev_info),
+                              _stream(stream)), "sgpt_pack_nm")
+
+
 def recon_error(W0: torch.Tensor, W: torch.Tensor, H: torch.Tensor, num_den: torch.Tensor,
                 ws: torch.Tensor | None = None, stream=None):
     """num_den (float64 [2], device) = (tr(dW H dW^T), tr(W0 H W0^T)).
@@ -338,30 +371,42 @@ class LayerBuffers:
     info: torch.Tensor
 
     @classmethod
-    def sharing(cls, other: "LayerBuffers", d_out: int, device="cuda") -> "LayerBuffers":
+    def sharing(cls, other: "LayerBuffers", d_out: int, device="cuda", nm=(2, 4)) -> "LayerBuffers":
         """Buffers for another weight matrix that reads the same input: it
         shares H and U (factor once, sweep each matrix) and has its own
         outputs and workspace."""
-        mine = cls.allocate(d_out, other.d_in, 0, device, with_hu=False)
+        mine = cls.allocate(d_out, other.d_in, 0, device, with_hu=False, nm=nm)
         mine.H, mine.U, mine.n_tok = other.H, other.U, other.n_tok
         return mine
 
     @classmethod
-    def allocate(cls, d_out: int, d_in: int, n_tok: int, device="cuda", with_hu: bool = True) -> "LayerBuffers":
+    def allocate(cls, d_out: int, d_in: int, n_tok: int, device="cuda", with_hu: bool = True,
+                 nm=(2, 4)) -> "LayerBuffers":
+        """nm: the (N, M) the packed outputs are sized for."""
         f32 = dict(dtype=torch.float32, device=device)
         i32 = dict(dtype=torch.int32, device=device)
         hu = (d_in, d_in) if with_hu else (0, 0)
+        n, m = nm
+        words = max(pack_nm_meta_words(d_in, n, m), 0)
         return cls(d_out, d_in, n_tok,
                    H=torch.empty(hu, **f32), U=torch.empty(hu, **f32),
                    mask=torch.empty((d_out, d_in // 32), **i32),
-                   values=torch.empty((d_out, d_in // 2), **f32),
-                   meta=torch.empty((d_out, d_in // 32), **i32),
+                   values=torch.empty((d_out, d_in * n // m), **f32),
+                   meta=torch.empty((d_out, words), **i32),
                    row_loss=torch.empty(d_out, **f32),
                    ws=workspace(d_out, d_in, n_tok, device=device),
                    info=new_info(device))
 
+    def packs(self, params: Params) -> bool:
+        """Whether the packed outputs are sized for this pattern."""
+        if not params.is_nm:
+            return False
+        n, m = params.nm
+        return self.values.shape[1] == self.d_in * n // m and \
+            self.meta.shape[1] == pack_nm_meta_words(self.d_in, n, m)
+
     def run(self, W: torch.Tensor, X: torch.Tensor | None, params: Params, stream=None):
-        pack = params.is_nm
+        pack = self.packs(params)
         prune_layer(W, self.H, self.U, params, self.mask, self.ws, self.info, X=X,
                     n_tok=self.n_tok, values=self.values if pack else None,
                     meta=self.meta if pack else None, row_loss=self.row_loss, stream=stream)
@@ -383,7 +428,7 @@ class LayerGraphs:
     def __init__(self, bufs: LayerBuffers, W: torch.Tensor, X: torch.Tensor | None, params: Params,
                  phases=PHASES):
         self.bufs, self.W, self.X, self.params = bufs, W, X, params
-        self.phases = tuple(ph for ph in phases if not (ph == "pack" and not params.is_nm))
+        self.phases = tuple(ph for ph in phases if not (ph == "pack" and not bufs.packs(params)))
         # one eager pass first: per-process kernel attributes are set outside capture
         self._eager()
         torch.cuda.synchronize()
@@ -408,7 +453,7 @@ class LayerGraphs:
             b.row_loss.zero_()
             prune(self.W, b.U, p, b.mask, b.ws, b.info, row_loss=b.row_loss)
         elif name == "pack":
-            pack24(self.W, b.mask, b.values, b.meta, b.info)
+            pack_nm(self.W, b.mask, *p.nm, b.values, b.meta, b.info)
 
     def _eager(self):
         for name in self.phases:
@@ -425,26 +470,27 @@ class HostPruner:
     Owns the device buffers of one layer shape and pinned host outputs.
     run() copies W and X from (pinned) host memory to the device, prunes the
     layer from X with sgpt_prune_layer, copies the pruned weights, the mask
-    and (for 2:4) the packed values and metadata back to the host, and checks
-    the device status. All copies are enqueued on the current stream.
+    and (for the N:M pattern it was sized for, 2:4 by default) the packed
+    values and metadata back to the host, and checks the device status. All
+    copies are enqueued on the current stream.
     """
 
-    def __init__(self, d_out: int, d_in: int, n_tok: int, device="cuda"):
-        self.bufs = LayerBuffers.allocate(d_out, d_in, n_tok, device)
+    def __init__(self, d_out: int, d_in: int, n_tok: int, device="cuda", nm=(2, 4)):
+        self.bufs = LayerBuffers.allocate(d_out, d_in, n_tok, device, nm=nm)
         self.W = torch.empty((d_out, d_in), dtype=torch.float32, device=device)
         self.X = torch.empty((n_tok, d_in), dtype=torch.bfloat16, device=device)
         pin = dict(pin_memory=True)
         self.W_out = torch.empty((d_out, d_in), dtype=torch.float32, **pin)
         self.mask_out = torch.empty((d_out, d_in // 32), dtype=torch.int32, **pin)
-        self.values_out = torch.empty((d_out, d_in // 2), dtype=torch.float32, **pin)
-        self.meta_out = torch.empty((d_out, d_in // 32), dtype=torch.int32, **pin)
+        self.values_out = torch.empty(self.bufs.values.shape, dtype=torch.float32, **pin)
+        self.meta_out = torch.empty(self.bufs.meta.shape, dtype=torch.int32, **pin)
 
     def h2d_bytes(self) -> int:
         return self.W.numel() * 4 + self.X.numel() * 2
 
     def d2h_bytes(self, params: Params) -> int:
         b = self.W_out.numel() * 4 + self.mask_out.numel() * 4
-        if params.is_nm:
+        if self.bufs.packs(params):
             b += self.values_out.numel() * 4 + self.meta_out.numel() * 4
         return b
 
@@ -460,13 +506,13 @@ class HostPruner:
         self.bufs.run(self.W, self.X if X_device is None else X_device, params, stream=stream)
         self.W_out.copy_(self.W, non_blocking=True)
         self.mask_out.copy_(self.bufs.mask, non_blocking=True)
-        if params.is_nm:
+        if self.bufs.packs(params):
             self.values_out.copy_(self.bufs.values, non_blocking=True)
             self.meta_out.copy_(self.bufs.meta, non_blocking=True)
 
     def run(self, W_host: torch.Tensor, X_host: torch.Tensor, params: Params, stream=None):
         self.enqueue(W_host, X_host, params, stream)
         raise_on_info(self.bufs.info, stream, "HostPruner.run")
-        if params.is_nm:
+        if self.bufs.packs(params):
             return self.W_out, self.mask_out, self.values_out, self.meta_out
         return self.W_out, self.mask_out, None, None

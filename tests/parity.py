@@ -42,7 +42,7 @@ def gpu_prune_layer(W: torch.Tensor, X: torch.Tensor | None, p: pp.Params,
     dev = torch.device("cuda")
     r, d = W.shape
     n = X.shape[0] if X is not None else n_tok
-    bufs = pp.LayerBuffers.allocate(r, d, n, dev)
+    bufs = pp.LayerBuffers.allocate(r, d, n, dev, nm=p.nm if p.is_nm else (2, 4))
     Wd = W.to(dev).contiguous()
     Xd = X.to(dev).contiguous() if X is not None else None
     if H_sum is not None:
@@ -138,7 +138,7 @@ def compare(gpu: dict, W0: np.ndarray, H: np.ndarray, U: np.ndarray, p: pp.Param
     m = {}
     m["mask_agree_free"] = float(np.mean(gpu["mask"] == free["mask"]))
     if p.is_nm:
-        differ, gap = nm_decisions_disagree(gpu["mask"], forced["S_dec"])
+        differ, gap = nm_decisions_disagree(gpu["mask"], forced["S_dec"], *p.nm)
         m["decisions"] = differ.size
         m["decision_flips"] = int(differ.sum())
         m["flip_max_gap"] = float(gap[differ].max()) if differ.any() else 0.0
@@ -159,9 +159,10 @@ def compare(gpu: dict, W0: np.ndarray, H: np.ndarray, U: np.ndarray, p: pp.Param
     m["loss_rel"] = float(np.abs(gpu["row_loss"].sum() - forced["loss"].sum()) / max(forced["loss"].sum(), 1e-300))
     m["pruned_zero"] = bool(np.all(gpu["W"][~gpu["mask"]] == 0.0))
     if p.is_nm:
-        groups = gpu["mask"].reshape(gpu["mask"].shape[0], -1, 4).sum(axis=2)
-        m["exact_24"] = bool(np.all(groups == 2))
-        vals, meta = oracle.pack24(gpu["W"].astype(np.float64), gpu["mask"])
+        n_keep, m_grp = p.nm
+        groups = gpu["mask"].reshape(gpu["mask"].shape[0], -1, m_grp).sum(axis=2)
+        m["exact_nm"] = bool(np.all(groups == n_keep))
+        vals, meta = oracle.pack_nm(gpu["W"].astype(np.float64), gpu["mask"], n_keep, m_grp)
         m["pack_exact"] = bool(np.array_equal(vals.astype(np.float32), gpu["values"])
                                and np.array_equal(meta, gpu["meta"]))
     else:
@@ -177,7 +178,7 @@ def compare(gpu: dict, W0: np.ndarray, H: np.ndarray, U: np.ndarray, p: pp.Param
 def assert_parity(m: dict, p: pp.Params):
     assert m["pruned_zero"]
     if p.is_nm:
-        assert m["exact_24"]
+        assert m["exact_nm"]
         assert m["pack_exact"]
     else:
         assert m["exact_count"]

@@ -56,7 +56,7 @@ MISALIGNED = FAKE + 4
 
 @pytest.mark.parametrize("case", [
     "null_W", "bad_din", "bad_ldw", "bad_blocksize", "bad_sparsity", "nm_unsupported",
-    "misaligned", "bad_pattern", "negative_damp",
+    "misaligned", "bad_pattern", "negative_damp", "nm_blocksize", "nm_din", "nm_n_above_m",
 ])
 def test_prune_rejects_bad_arguments(case):
     L = pp.lib()
@@ -74,7 +74,14 @@ def test_prune_rejects_bad_arguments(case):
     elif case == "bad_sparsity":
         p = S.Params("unstructured:1.0").to_c()
     elif case == "nm_unsupported":
-        p = S.Params("4:8").to_c()
+        p = S.Params("3:6").to_c()              # M not a power of two
+    elif case == "nm_blocksize":
+        p = S.Params("16:128", blocksize=64).to_c()
+    elif case == "nm_din":
+        p = S.Params("16:128").to_c()
+        args["d"] = args["ldw"] = 320
+    elif case == "nm_n_above_m":
+        p = S.Params("8:4").to_c()
     elif case == "misaligned":
         args["mask"] = MISALIGNED
     elif case == "bad_pattern":
@@ -106,6 +113,20 @@ def test_other_entry_points_validate():
                               None, None, FAKE, 1 << 30, FAKE, None) == 1
     assert L.sgpt_prune_layer(FAKE, 8, 64, 64, None, 10, FAKE, FAKE + 4096, ctypes.byref(p24), MISALIGNED,
                               None, None, None, FAKE, 1 << 30, FAKE, None) == 1
+
+
+def test_pack_nm_sizes_and_validation():
+    L = pp.lib()
+    assert L.sgpt_pack_nm_meta_words(64, 2, 4) == 2          # = d_in / 32, as pack24
+    assert L.sgpt_pack_nm_meta_words(32, 16, 32) == 3        # 16 x 5 bits
+    assert L.sgpt_pack_nm_meta_words(256, 16, 128) == 7      # 2 x 16 x 7 bits
+    assert L.sgpt_pack_nm_meta_words(64, 4, 8) == 3          # 8 groups x 4 x 3 bits = 96
+    assert L.sgpt_pack_nm_meta_words(64, 3, 6) == -1
+    assert L.sgpt_pack_nm_meta_words(96, 16, 64) == -1       # d_in % m
+    assert L.sgpt_pack_nm(FAKE, 8, 64, 64, FAKE, 3, 6, FAKE, FAKE, FAKE, None) == 6
+    assert L.sgpt_pack_nm(FAKE, 8, 96, 96, FAKE, 16, 64, FAKE, FAKE, FAKE, None) == 1
+    assert L.sgpt_pack_nm(FAKE, 8, 64, 64, FAKE, 9, 8, FAKE, FAKE, FAKE, None) == 1
+    assert L.sgpt_pack_nm(FAKE, 8, 64, 64, FAKE, 4, 8, MISALIGNED, FAKE, FAKE, None) == 1
 
 
 def test_wait_limit_setting():

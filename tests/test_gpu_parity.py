@@ -208,6 +208,50 @@ def test_sweep_matches_oracle_given_H(spec, p):
     assert_parity(m, p)
 
 
+# General N:M (sparse fine-tuning review, section 八 8.4: 16:32, 16:64,
+# 16:128; SparseGPT review, section 十四 14.4: 2:4, 4:8), against the oracle
+# on the same H: masks, weights, losses and the packed values and metadata.
+NM_PATTERNS = ["1:4", "3:4", "4:8", "8:16", "16:32", "16:64", "16:128"]
+TALL_2K = LayerSpec("tall_2k", d_in=256, d_out=2304, n_tok=1024, sigma=1.5, seed=9)
+
+
+@pytest.mark.parametrize("pattern", NM_PATTERNS)
+@pytest.mark.parametrize("spec", SMALL + [TALL_2K], ids=lambda s: s.name)
+def test_nm_sweep_and_pack_match_oracle(spec, pattern):
+    """layer256 and ragged (one row per warp, ragged last block for M <= 64),
+    tall (128 columns, 1000 rows), tall_2k (2304 rows: two rows per warp,
+    where a 128-group spans both of a lane's column spans)."""
+    n, m = (int(x) for x in pattern.split(":"))
+    if spec.d_in % m:
+        pytest.skip(f"d_in {spec.d_in} is not a multiple of {m}")
+    W, X = _inputs(spec)
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)
+    H, U_ref = _oracle_factor(Hs, spec.n_tok)
+    p = pp.Params(pattern)
+    gpu = gpu_prune_layer(W, None, p, H_sum=torch.from_numpy(Hs), n_tok=spec.n_tok)
+    m_ = compare(gpu, W.numpy().astype(np.float64), H, U_ref, p)
+    assert_parity(m_, p)
+
+
+def test_nm_blocksize_independence_and_pack_errors():
+    """N:M results do not depend on the block size; a mask that breaks the
+    pattern is reported by the pack."""
+    spec = SMALL[0]
+    W, X = _inputs(spec)
+    a = gpu_prune_layer(W, X, pp.Params("16:64", blocksize=128))
+    b = gpu_prune_layer(W, X, pp.Params("16:64", blocksize=64))
+    assert np.mean(a["mask"] == b["mask"]) > 0.999
+    dev = torch.device("cuda")
+    Wd = torch.randn(8, 128, device=dev)
+    mask = torch.full((8, 4), -1, dtype=torch.int32, device=dev)        # keeps all of every group
+    vals = torch.empty(8, 128 * 4 // 8, device=dev)
+    meta = torch.empty(8, pp.pack_nm_meta_words(128, 4, 8), dtype=torch.int32, device=dev)
+    info = pp.new_info()
+    pp.pack_nm(Wd, mask, 4, 8, vals, meta, info)
+    assert pp.sync_status(info) == 7
+
+
 def test_forced_mask_reproduces_oracle():
     spec = SMALL[1]
     W, X = _inputs(spec)
