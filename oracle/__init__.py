@@ -16,6 +16,8 @@ from .sparsegpt_ref import (  # noqa: F401
     pack_nm,
     parse_pattern,
     prune_layer,
+    quant_grid,
+    quantize,
     recon_error,
     sweep,
     unpack24,

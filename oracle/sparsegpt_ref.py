@@ -48,7 +48,12 @@ Readings where the pages are silent (each is listed in the design notes):
   32-bit word, least significant first;
 * the packed N:M form generalises it: the N survivors of each group of M in
   index order, and each survivor's in-group position in log2(M) bits, packed
-  along the row least significant bit first (2:4 gives the same words).
+  along the row least significant bit first (2:4 gives the same words);
+* joint sparsification and quantization: one uniform asymmetric grid of
+  2**bits levels per output row over the dense row's range widened to 0
+  (fp32 scale and zero point); each kept weight becomes its grid value when
+  its column is reached and the difference is compensated like a pruning
+  error; the integer code is decided in fp32.
 """
 
 from __future__ import annotations
@@ -109,6 +114,38 @@ def inverse_cholesky_upper(Hd: np.ndarray) -> np.ndarray:
 # The blocked OBS sweep  ([SGPT] sections 八 and 十一)
 # --------------------------------------------------------------------------
 
+def quant_grid(W, bits: int):
+    """Per-row uniform asymmetric grid of 2**bits levels ([SGPT] sections 十五
+    and 十七: survivors quantized to low-bit values, GPTQ-style).
+
+    The range of each row of the dense input weights, widened to include 0
+    (so a pruned weight stays exactly 0 on the grid); a row of zeros takes
+    [-1, 1]. scale = (max - min) / (2**bits - 1) and zero = rint(-min /
+    scale), both in fp32, the arithmetic the grid is stored in. Returns
+    (scale, zero) as float32 arrays [d_out].
+    """
+    W32 = np.asarray(W, dtype=np.float32)
+    maxq = np.float32(2 ** bits - 1)
+    lo = np.minimum(W32.min(axis=1), np.float32(0))
+    hi = np.maximum(W32.max(axis=1), np.float32(0))
+    flat = lo == hi
+    lo = np.where(flat, np.float32(-1), lo)
+    hi = np.where(flat, np.float32(1), hi)
+    scale = ((hi - lo) / maxq).astype(np.float32)
+    zero = np.rint(-lo / scale).astype(np.float32)
+    return scale, zero
+
+
+def quantize(x, scale, zero, bits: int):
+    """The grid value nearest x: scale * (clip(rint(x / scale) + zero, 0,
+    2**bits - 1) - zero). The integer code is decided in fp32 (x rounded to
+    fp32, fp32 division, ties to even), the precision the grid is stored in;
+    the value is formed in float64."""
+    x32 = np.asarray(x, dtype=np.float32)
+    code = np.clip(np.rint(x32 / scale) + zero, np.float32(0), np.float32(2 ** bits - 1))
+    return np.asarray(scale, dtype=np.float64) * (code.astype(np.float64) - np.asarray(zero, dtype=np.float64))
+
+
 def parse_pattern(pattern):
     """'2:4' -> ('nm', 2, 4, None); 'unstructured:0.5' -> ('unstructured', .., 0.5)."""
     if isinstance(pattern, tuple):
@@ -119,8 +156,14 @@ def parse_pattern(pattern):
     return ("nm", int(n), int(m), None)
 
 
-def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None):
+def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=None, qgrid=None):
     """Prune W [d_out, d_in] column by column with OBS compensation.
+
+    With ``qbits`` the sweep also quantizes ([SGPT] sections 十五 and 十七,
+    pruning and GPTQ-style quantization in the same second-order pass): a
+    kept weight is replaced by its value on the row's grid (``qgrid``, or
+    quant_grid of the input W), and the difference is compensated in the
+    later columns exactly like a pruning error.
 
     Returns a dict with
       W      the pruned, compensated weights (float64)
@@ -144,6 +187,8 @@ def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None):
     Err = np.zeros((r, d))
     loss = np.zeros(r)
     rows = np.arange(r)
+    if qbits:
+        qscale, qzero = quant_grid(W, qbits) if qgrid is None else qgrid
 
     for i1 in range(0, d, blocksize):
         i2 = min(i1 + blocksize, d)
@@ -177,7 +222,8 @@ def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None):
                     np.put_along_axis(keep, order[:, :n_keep], True, axis=1)
                     mask[:, c:c + m_grp] = keep
             w = W1[:, q]
-            p = np.where(mask[:, c], w, 0.0)
+            kept = quantize(w, qscale, qzero, qbits) if qbits else w
+            p = np.where(mask[:, c], kept, 0.0)
             e = (w - p) / U[c, c]
             W1[:, q:] -= np.outer(e, U[c, c:i2])
             W1[:, q] = p
@@ -327,13 +373,14 @@ def recon_error(W0, W_hat, H):
 # --------------------------------------------------------------------------
 
 def prune_layer(W, X=None, H=None, pattern="2:4", blocksize: int = 128,
-                damp_ratio: float = 0.01, forced_mask=None):
-    """Hessian (from X, or H given), damping, factor, sweep, and 2:4 pack."""
+                damp_ratio: float = 0.01, forced_mask=None, qbits=None):
+    """Hessian (from X, or H given), damping, factor, sweep (optionally with
+    quantization of the survivors), and N:M pack."""
     if H is None:
         H = hessian(X)
     Hd, lam = damp(H, damp_ratio)
     U = inverse_cholesky_upper(Hd)
-    out = sweep(W, U, pattern, blocksize, forced_mask)
+    out = sweep(W, U, pattern, blocksize, forced_mask, qbits=qbits)
     out.update(H=H, Hd=Hd, lam=lam, U=U)
     kind, n_keep, m_grp, _ = parse_pattern(pattern)
     if kind == "nm" and (n_keep, m_grp) == (2, 4):

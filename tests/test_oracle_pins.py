@@ -42,7 +42,7 @@ def _factor(X, damp_ratio=0.01):
 
 # ---------------------------------------------------------------- references
 
-def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None, blocksize=None):
+def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None, blocksize=None, qbits=None):
     """Sequential OBS written as explicit least-squares re-fits.
 
     For each column q in order: decide the mask if the pattern decides here
@@ -53,7 +53,9 @@ def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None, blocksize=None):
     taken on the current (already re-fitted) weights; set a pruned weight to
     zero, then re-fit every column right of q to minimise
     (w - w^) H_d (w - w^)^T with the columns <= q frozen. Uses general linear
-    solves only: no Cholesky, no U, no lazy batching.
+    solves only: no Cholesky, no U, no lazy batching. With ``qbits`` a kept
+    weight is set to its grid value (the grid of the input rows) instead and
+    the later columns are re-fitted the same way.
     """
     kind, n_keep, m_grp, sparsity = ref.parse_pattern(pattern)
     assert kind == "nm" or forced_mask is not None or blocksize
@@ -61,6 +63,8 @@ def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None, blocksize=None):
     sal_den = np.array([np.linalg.inv(Hd[c:, c:])[0, 0] for c in range(d)])
     w0 = np.array(W, dtype=np.float64)
     cur = w0.copy()
+    if qbits:
+        qs, qz = oracle.quant_grid(W, qbits)
     mask = np.ones((r, d), dtype=bool) if forced_mask is None else forced_mask.copy()
     for q in range(d):
         if forced_mask is None and kind == "nm" and q % m_grp == 0:
@@ -78,8 +82,11 @@ def frozen_prefix_sweep(W, Hd, pattern="2:4", forced_mask=None, blocksize=None):
             for _, row, j in keys[:k]:
                 mask[row, q + j] = False
         for row in range(r):
-            if not mask[row, q]:
-                cur[row, q] = 0.0
+            if not mask[row, q] or qbits:
+                if mask[row, q]:
+                    cur[row, q] = oracle.quantize(cur[row, q], qs[row], qz[row], qbits)
+                else:
+                    cur[row, q] = 0.0
                 if q + 1 < d:
                     D_fixed = w0[row, :q + 1] - cur[row, :q + 1]
                     rhs = Hd[q + 1:, :q + 1] @ D_fixed
@@ -415,6 +422,55 @@ def test_nm_sweep_equals_frozen_prefix_least_squares(rng, pattern):
     assert np.allclose(out["W"], ref_W, atol=1e-11)
 
 
+def test_quant_grid_hand_examples():
+    g = _golden("quant_grid.json")
+    for case in g["cases"]:
+        bits = case["bits"]
+        scale, zero = oracle.quant_grid(np.array([case["row"]]), bits)
+        want_scale = (np.float32(case["scale_fraction"][0]) / np.float32(case["scale_fraction"][1])
+                      if "scale_fraction" in case else np.float32(case["scale"]))
+        assert scale[0] == np.float32(want_scale) and zero[0] == case["zero"]
+        q = oracle.quantize(np.array(case["x"]), scale[0], zero[0], bits)
+        if "q" in case:
+            assert np.array_equal(q, np.array(case["q"]))
+        else:
+            assert np.array_equal(q, np.float64(scale[0]) * np.array(case["q_codes"], dtype=np.float64))
+
+
+def test_quantized_sweep_diagonal_hessian_is_rounding(rng):
+    """Diagonal H: no compensation, so every survivor is exactly its grid
+    value and the mask is the one the unquantized sweep takes."""
+    r, d, n = 6, 32, 64
+    X = np.zeros((n, d))
+    X[np.arange(n), np.arange(n) % d] = rng.standard_normal(n) * 3
+    W = rng.standard_normal((r, d)).astype(np.float32).astype(np.float64)
+    for bits in (3, 4, 8):
+        a = oracle.prune_layer(W, X=X, pattern="2:4", damp_ratio=0.0, blocksize=16, qbits=bits)
+        b = oracle.prune_layer(W, X=X, pattern="2:4", damp_ratio=0.0, blocksize=16)
+        assert np.array_equal(a["mask"], b["mask"])
+        s_, z_ = oracle.quant_grid(W, bits)
+        want = np.where(a["mask"], oracle.quantize(W, s_[:, None], z_[:, None], bits), 0.0)
+        assert np.array_equal(a["W"], want)
+
+
+@pytest.mark.parametrize("pattern,bits", [("2:4", 4), ("4:8", 3), ("unstructured:0.5", 4), ("unstructured:0.0", 3)])
+def test_quantized_sweep_equals_frozen_prefix_least_squares(rng, pattern, bits):
+    """Joint pruning and quantization ([SGPT] 十五, 十七) against the
+    general-solve reference: every pruned or quantized weight is frozen and
+    the later columns re-fitted."""
+    W, X = _layer(rng, r=5, d=24, n=70, scale_spread=1.5)
+    _, Hd, U = _factor(X)
+    out = oracle.sweep(W, U, pattern, blocksize=8, qbits=bits)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, pattern, blocksize=8, qbits=bits)
+    assert np.array_equal(out["mask"], ref_mask)
+    assert np.allclose(out["W"], ref_W, atol=1e-11)
+    s_, z_ = oracle.quant_grid(W, bits)
+    on_grid = np.where(out["mask"], oracle.quantize(out["W"], s_[:, None], z_[:, None], bits), 0.0)
+    assert np.allclose(out["W"], on_grid, atol=1e-12)      # every survivor sits on its row's grid
+    dW = W - out["W"]
+    assert out["loss"].sum() == pytest.approx(np.trace(dW @ Hd @ dW.T), rel=1e-10)
+
+
 # ---------------------------------------------------------------- mutations
 
 _MUTATIONS = [
@@ -444,6 +500,13 @@ _MUTATIONS = [
     ("unstructured count rounded up",
      [("k = int(math.floor(sparsity * r * width))", "k = int(math.ceil(sparsity * r * width))")],
      "unstructured:0.53", 4),
+    # joint quantization: the grid error left uncompensated, and the grid
+    # value taken of the weight before this block's updates
+    ("quantization error not compensated",
+     [("e = (w - p) / U[c, c]", "e = (w - np.where(mask[:, c], w, 0.0)) / U[c, c]")], ("2:4", 4), 8),
+    ("quantized before the in-block updates",
+     [("kept = quantize(w, qscale, qzero, qbits) if qbits else w",
+       "kept = quantize(W[:, c], qscale, qzero, qbits) if qbits else w")], ("2:4", 4), 8),
 ]
 
 
@@ -459,7 +522,10 @@ def test_pins_catch_planted_mistakes(name, edits, pattern, blocksize):
     # own seed: the verdict must not depend on which tests ran before
     W, X = _layer(np.random.default_rng(2024), r=16, d=32, n=80, scale_spread=1.5)
     _, Hd, U = _factor(X)
-    got = mutated(W, U, pattern, blocksize=blocksize)
-    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, pattern, blocksize=blocksize)
+    qbits = None
+    if isinstance(pattern, tuple):          # (pattern, bits): the quantized sweep
+        pattern, qbits = pattern
+    got = mutated(W, U, pattern, blocksize=blocksize, qbits=qbits)
+    ref_W, ref_mask = frozen_prefix_sweep(W, Hd, pattern, blocksize=blocksize, qbits=qbits)
     same = np.array_equal(got["mask"], ref_mask) and np.allclose(got["W"], ref_W, atol=1e-9)
     assert not same, f"pins did not catch: {name}"
