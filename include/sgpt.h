@@ -80,6 +80,14 @@ typedef struct sgpt_params {
   int blocksize;  /* columns per OBS block: 32, 64, 96 or 128                */
   float damp;     /* damping ratio (0.01 = 1% of the mean diagonal), >= 0    */
   int forced;     /* 1: mask_bits is an INPUT and no selection is made       */
+  int qbits;      /* 0: prune only. 2..16: joint sparsification and
+                     quantization (SparseGPT review, sections 十五 and 十七):
+                     every kept weight is replaced by its value on its row's
+                     grid of 2^qbits levels as its column is reached, and the
+                     difference is compensated like a pruning error          */
+  const float* qgrid; /* qbits > 0: the grid [d_out x 2] fp32 (scale, zero
+                     point per row, device), e.g. from sgpt_quant_grid; NULL:
+                     sgpt_prune computes it from the dense input W           */
 } sgpt_params;
 
 /* Human-readable name of a status. Never NULL. */
@@ -178,11 +186,27 @@ sgpt_status sgpt_prune(float* W, int d_out, int d_in, int ldw, const float* U,
  *     before any stream capture on the device.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race and must be serialised by the
- *     caller. Nothing in the array needs clearing between calls. */
+ *     caller. Nothing in the array needs clearing between calls.
+ *   - With p->qbits > 0 the caller passes the grid in p->qgrid (the array
+ *     has no room for it): SGPT_ERR_UNSUPPORTED when it is NULL. */
 #define SGPT_NOALLOC_MAX_ROWS 8192
 sgpt_status sgpt_prune_noalloc(float* W, int d_out, int d_in, int ldw, const float* U,
                                const sgpt_params* p, uint32_t* mask_bits, float* row_loss,
                                int* dev_info, void* stream);
+
+/* The per-row quantization grid of the joint sparse + quantized sweep
+ * (SparseGPT review, sections 十五 and 十七; the grid itself is this
+ * library's reading: uniform and asymmetric, 2^qbits levels over the row's
+ * range widened to include 0, so a pruned weight stays exactly 0):
+ *   grid [d_out x 2] fp32: grid[2r] = scale = (hi - lo) / (2^qbits - 1),
+ *        grid[2r + 1] = zero = rint(-lo / scale), with lo = min(row, 0) and
+ *        hi = max(row, 0) of the dense row (a row of zeros: lo = -1, hi = 1),
+ *        all in fp32. A weight x maps to scale * (clip(rint(x / scale) +
+ *        zero, 0, 2^qbits - 1) - zero); the integer code of a kept weight of
+ *        the result is rint(W / scale) + zero exactly.
+ * qbits in 2..16. Call it on the dense W before sgpt_prune (or leave
+ * qgrid NULL and sgpt_prune computes the same grid). */
+sgpt_status sgpt_quant_grid(const float* W, int d_out, int d_in, int ldw, int qbits, float* grid, void* stream);
 
 /* 2:4 packing (2:4 production guide, section on the 2:4 mechanism):
  *   values [d_out x d_in/2] fp32: the two kept weights of each group of four,

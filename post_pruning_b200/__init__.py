@@ -27,6 +27,7 @@ from .sgpt import (  # noqa: F401
     prune,
     prune_layer,
     prune_noalloc,
+    quant_grid,
     raise_on_info,
     recon_error,
     set_wait_limit,

@@ -40,6 +40,8 @@ sgpt_status check_params(const sgpt_params* p) {
   if (p->blocksize < 32 || p->blocksize > kMaxBlock || p->blocksize % 32) return SGPT_ERR_INVALID_ARG;
   if (!(p->damp >= 0.f) || !std::isfinite(p->damp)) return SGPT_ERR_INVALID_ARG;
   if (p->forced != 0 && p->forced != 1) return SGPT_ERR_INVALID_ARG;
+  if (p->qbits != 0 && (p->qbits < 2 || p->qbits > 16)) return SGPT_ERR_INVALID_ARG;
+  if (p->qbits && p->qgrid && !aligned16(p->qgrid)) return SGPT_ERR_INVALID_ARG;
   if (p->pattern == SGPT_PATTERN_NM) {
     if (p->n <= 0 || p->m <= 0 || p->n > p->m) return SGPT_ERR_INVALID_ARG;
     if (!valid_m(p->m)) return SGPT_ERR_UNSUPPORTED;
@@ -178,6 +180,7 @@ sgpt_status sgpt_prune_noalloc(float* W, int d_out, int d_in, int ldw, const flo
   if (row_loss && !aligned16(row_loss)) return SGPT_ERR_INVALID_ARG;
   sgpt_status s = check_params(p);
   if (s != SGPT_OK) return s;
+  if (p->qbits && !p->qgrid) return SGPT_ERR_UNSUPPORTED;
   if (p->pattern == SGPT_PATTERN_NM && d_in % p->m) return SGPT_ERR_INVALID_ARG;
   return from_cuda(launch_prune_noalloc(W, d_out, d_in, ldw, U, *p, mask_bits, row_loss, dev_info,
                                         as_stream(stream)));
@@ -190,6 +193,13 @@ sgpt_status sgpt_pack24(const float* W, int d_out, int d_in, int ldw, const uint
     return SGPT_ERR_INVALID_ARG;
   if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
   return from_cuda(launch_pack24(W, ldw, d_out, d_in, mask_bits, values, meta, dev_info, as_stream(stream)));
+}
+
+sgpt_status sgpt_quant_grid(const float* W, int d_out, int d_in, int ldw, int qbits, float* grid, void* stream) {
+  if (!W || !grid || !aligned16(W) || !aligned16(grid)) return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || ldw < d_in || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  if (qbits < 2 || qbits > 16) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_quant_grid(W, ldw, d_out, d_in, qbits, grid, as_stream(stream)));
 }
 
 int sgpt_pack_nm_meta_words(int d_in, int n, int m) {

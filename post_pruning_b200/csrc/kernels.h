@@ -21,6 +21,8 @@ size_t prune_ws_bytes(int d_out, int d_in);
 cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* U,
                          const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
                          int* info, cudaStream_t st);
+cudaError_t launch_quant_grid(const float* W, long long ldw, int rows, int d, int bits, float* grid,
+                              cudaStream_t st);
 cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const float* U,
                                  const sgpt_params& p, uint32_t* mask, float* row_loss, int* info,
                                  cudaStream_t st);

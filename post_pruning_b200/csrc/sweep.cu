@@ -36,6 +36,13 @@ constexpr size_t kSweepSmem = (size_t)kMaxBlock * kMaxBlock * sizeof(float);
 // found by select_kernel; kModeForced: the mask is an input.
 enum SweepMode { kModeNM4 = 0, kModeThreshold = 1, kModeForced = 2, kModeNMG = 3 };
 
+// The value of x on a row's quantization grid: scale * (clip(rint(x / scale)
+// + zero, 0, maxq) - zero); the code is decided in fp32 with ties to even.
+__device__ __forceinline__ float quant_value(float x, float scale, float zero, float maxq) {
+  const float c = fminf(fmaxf(rintf(__fdiv_rn(x, scale)) + zero, 0.f), maxq);
+  return __fmul_rn(scale, c - zero);
+}
+
 __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsigned idx) {
   return ((unsigned long long)__float_as_uint(saliency(w, inv_u)) << 32) | idx;
 }
@@ -65,12 +72,17 @@ __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsi
 // best are kept. An M-group covers M/4 consecutive lanes of one column span,
 // or (M = 128 with two rows per warp) every lane of both spans. The group
 // steps then apply the decided bits like a forced mask.
-template <int MODE, int ROWS, int M>
+//
+// QUANT (joint sparsification and quantization, SparseGPT review sections
+// 十五 and 十七): a kept weight is replaced by its value on the row's grid
+// (qgrid[2 * row] = scale, qgrid[2 * row + 1] = zero point) when its column
+// is reached, and (w - value) / U_qq is compensated like a pruning error.
+template <int MODE, int ROWS, int M, bool QUANT>
 __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
     const float* __restrict__ U, uint32_t* __restrict__ mask, float* __restrict__ row_loss,
     float* __restrict__ Err, float* __restrict__ Err_lo, const unsigned long long* __restrict__ thr,
-    int nkeep, int* info) {
+    int nkeep, const float* __restrict__ qgrid, float qmaxq, int* info) {
   constexpr int LPR = 32 / ROWS;                 // lanes per row
   constexpr int CPL = 4 * ROWS;                  // columns per lane
   if (cta_info_set(info)) return;
@@ -140,6 +152,11 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
       const unsigned idx = (unsigned)row * (unsigned)bw + (unsigned)c;
       if (c < bw && sal_key(w[j], Uinv[c], idx) >= t) keep |= 1u << j;
     }
+  }
+  float qs = 1.f, qz = 0.f;
+  if (QUANT && mine) {
+    qs = qgrid[2 * (long long)row];
+    qz = qgrid[2 * (long long)row + 1];
   }
   float loss = 0.f;
   // keep bit j of every lane, for the threshold and forced modes
@@ -238,16 +255,38 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
         for (int t = 0; t < 4; ++t) km |= ((kb[4 * gi + t] >> owner) & 1u) << t;
       }
       float e[4];
-      e[0] = (km & 1u) ? 0.f : __fmul_rn(wo[0], r[0]);
-      wo[1] = fmaf(-e[0], g0.y, wo[1]);
-      wo[2] = fmaf(-e[0], g0.z, wo[2]);
-      wo[3] = fmaf(-e[0], g0.w, wo[3]);
-      e[1] = (km & 2u) ? 0.f : __fmul_rn(wo[1], r[1]);
-      wo[2] = fmaf(-e[1], g1.z, wo[2]);
-      wo[3] = fmaf(-e[1], g1.w, wo[3]);
-      e[2] = (km & 4u) ? 0.f : __fmul_rn(wo[2], r[2]);
-      wo[3] = fmaf(-e[2], g2.w, wo[3]);
-      e[3] = (km & 8u) ? 0.f : __fmul_rn(wo[3], r[3]);
+      if constexpr (QUANT) {
+        // a kept weight becomes its grid value; the difference is
+        // compensated like a pruning error
+        float pq[4];
+        pq[0] = (km & 1u) ? quant_value(wo[0], qs, qz, qmaxq) : 0.f;
+        e[0] = __fmul_rn(__fsub_rn(wo[0], pq[0]), r[0]);
+        wo[1] = fmaf(-e[0], g0.y, wo[1]);
+        wo[2] = fmaf(-e[0], g0.z, wo[2]);
+        wo[3] = fmaf(-e[0], g0.w, wo[3]);
+        pq[1] = (km & 2u) ? quant_value(wo[1], qs, qz, qmaxq) : 0.f;
+        e[1] = __fmul_rn(__fsub_rn(wo[1], pq[1]), r[1]);
+        wo[2] = fmaf(-e[1], g1.z, wo[2]);
+        wo[3] = fmaf(-e[1], g1.w, wo[3]);
+        pq[2] = (km & 4u) ? quant_value(wo[2], qs, qz, qmaxq) : 0.f;
+        e[2] = __fmul_rn(__fsub_rn(wo[2], pq[2]), r[2]);
+        wo[3] = fmaf(-e[2], g2.w, wo[3]);
+        pq[3] = (km & 8u) ? quant_value(wo[3], qs, qz, qmaxq) : 0.f;
+        e[3] = __fmul_rn(__fsub_rn(wo[3], pq[3]), r[3]);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) wo[t] = pq[t];
+      } else {
+        e[0] = (km & 1u) ? 0.f : __fmul_rn(wo[0], r[0]);
+        wo[1] = fmaf(-e[0], g0.y, wo[1]);
+        wo[2] = fmaf(-e[0], g0.z, wo[2]);
+        wo[3] = fmaf(-e[0], g0.w, wo[3]);
+        e[1] = (km & 2u) ? 0.f : __fmul_rn(wo[1], r[1]);
+        wo[2] = fmaf(-e[1], g1.z, wo[2]);
+        wo[3] = fmaf(-e[1], g1.w, wo[3]);
+        e[2] = (km & 4u) ? 0.f : __fmul_rn(wo[2], r[2]);
+        wo[3] = fmaf(-e[2], g2.w, wo[3]);
+        e[3] = (km & 8u) ? 0.f : __fmul_rn(wo[3], r[3]);
+      }
       if (sl == gp) {
         // the owner keeps its group's result
 #pragma unroll
@@ -316,38 +355,40 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 // per row), one for short ones (twice the warps in flight).
 static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 2 : 1; }
 
-template <int MODE, int M>
+template <int MODE, int M, bool QUANT>
 static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
                                   uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
-                                  const unsigned long long* thr, int nkeep, int* info, cudaStream_t st) {
+                                  const unsigned long long* thr, int nkeep, const float* qgrid, float qmaxq,
+                                  int* info, cudaStream_t st) {
   static PerDevice attrs;
   const cudaError_t ea = once_per_device(attrs, [] {
-    const cudaError_t r =
-        cudaFuncSetAttribute(sweep_kernel<MODE, 1, M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    return r != cudaSuccess
-               ? r
-               : cudaFuncSetAttribute(sweep_kernel<MODE, 2, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kSweepSmem);
+    const cudaError_t r = cudaFuncSetAttribute(sweep_kernel<MODE, 1, M, QUANT>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    return r != cudaSuccess ? r
+                            : cudaFuncSetAttribute(sweep_kernel<MODE, 2, M, QUANT>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
   });
   if (ea != cudaSuccess) return ea;
   const int grid = cdiv(rows, kSweepWarps * rpw);
   if (rpw == 2)
-    sweep_kernel<MODE, 2, M><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss,
-                                                                      Err, Err_lo, thr, nkeep, info);
+    sweep_kernel<MODE, 2, M, QUANT><<<grid, kSweepThreads, kSweepSmem, st>>>(
+        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, nkeep, qgrid, qmaxq, info);
   else
-    sweep_kernel<MODE, 1, M><<<grid, kSweepThreads, kSweepSmem, st>>>(W, ldw, rows, d, i1, bw, U, mask, row_loss,
-                                                                      Err, Err_lo, thr, nkeep, info);
+    sweep_kernel<MODE, 1, M, QUANT><<<grid, kSweepThreads, kSweepSmem, st>>>(
+        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, nkeep, qgrid, qmaxq, info);
   count_launches(1);
   return cudaGetLastError();
 }
 
-// The sweep of one block for a pattern: forced mask, unstructured threshold,
-// N of 4, or N of M = 8 .. 128.
-static cudaError_t launch_sweep(const sgpt_params& p, int rpw, float* W, long long ldw, int rows, int d, int i1,
-                                int bw, const float* U, uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
-                                const unsigned long long* thr, int* info, cudaStream_t st) {
-#define SGPT_SWEEP(MODE, M) \
-  launch_sweep_m<MODE, M>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, p.n, info, st)
+template <bool QUANT>
+static cudaError_t launch_sweep_q(const sgpt_params& p, int rpw, float* W, long long ldw, int rows, int d, int i1,
+                                  int bw, const float* U, uint32_t* mask, float* row_loss, float* Err,
+                                  float* Err_lo, const unsigned long long* thr, const float* qgrid, int* info,
+                                  cudaStream_t st) {
+  const float qmaxq = QUANT ? (float)((1 << p.qbits) - 1) : 0.f;
+#define SGPT_SWEEP(MODE, M)                                                                                  \
+  launch_sweep_m<MODE, M, QUANT>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, p.n, qgrid, \
+                                 qmaxq, info, st)
   if (p.forced) return SGPT_SWEEP(kModeForced, 4);
   if (p.pattern != SGPT_PATTERN_NM) return SGPT_SWEEP(kModeThreshold, 4);
   switch (p.m) {
@@ -360,6 +401,58 @@ static cudaError_t launch_sweep(const sgpt_params& p, int rpw, float* W, long lo
   }
 #undef SGPT_SWEEP
   return cudaErrorInvalidValue;
+}
+
+// The sweep of one block for a pattern: forced mask, unstructured threshold,
+// N of 4, or N of M = 8 .. 128; with or without quantization of the kept
+// weights (qgrid: the per-row grid, when p.qbits > 0).
+static cudaError_t launch_sweep(const sgpt_params& p, int rpw, float* W, long long ldw, int rows, int d, int i1,
+                                int bw, const float* U, uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
+                                const unsigned long long* thr, const float* qgrid, int* info, cudaStream_t st) {
+  if (p.qbits > 0)
+    return launch_sweep_q<true>(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, qgrid, info,
+                                st);
+  return launch_sweep_q<false>(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, nullptr, info,
+                               st);
+}
+
+// ------------------------------------------------------ quantization grid
+
+// One warp per row: the range of the dense row widened to include 0 (a row
+// of zeros takes [-1, 1]); scale = (hi - lo) / maxq and zero =
+// rint(-lo / scale), in fp32.
+__global__ void __launch_bounds__(256) quant_grid_kernel(const float* __restrict__ W, long long ldw, int rows, int d,
+                                                        float maxq, float* __restrict__ grid) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* w = W + (long long)row * ldw;
+  float lo = 0.f, hi = 0.f;
+  for (int c = 4 * lane; c < d; c += 128) {
+    const float4 x = ld4(w + c);
+    lo = fminf(lo, fminf(fminf(x.x, x.y), fminf(x.z, x.w)));
+    hi = fmaxf(hi, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    if (lo == hi) {
+      lo = -1.f;
+      hi = 1.f;
+    }
+    const float scale = __fdiv_rn(__fsub_rn(hi, lo), maxq);
+    grid[2 * (long long)row] = scale;
+    grid[2 * (long long)row + 1] = rintf(__fdiv_rn(-lo, scale));
+  }
+}
+
+cudaError_t launch_quant_grid(const float* W, long long ldw, int rows, int d, int bits, float* grid,
+                              cudaStream_t st) {
+  quant_grid_kernel<<<cdiv(rows, 8), 256, 0, st>>>(W, ldw, rows, d, (float)((1 << bits) - 1), grid);
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 // --------------------------------------------------------- trailing update
@@ -576,6 +669,7 @@ struct PruneWs {
   float* U_hi;     // hi/lo planes of U (d_in x d_in)
   float* U_lo;
   SelState* sel;
+  float* qgrid;    // per-row quantization grid (scale, zero), d_out x 2
 };
 
 static PruneWs carve_prune(void* ws, int d_out, int d_in, size_t* bytes) {
@@ -586,6 +680,7 @@ static PruneWs carve_prune(void* ws, int d_out, int d_in, size_t* bytes) {
   w.U_hi = c.take<float>((size_t)d_in * d_in);
   w.U_lo = c.take<float>((size_t)d_in * d_in);
   w.sel = c.take<SelState>(1);
+  w.qgrid = c.take<float>((size_t)d_out * 2);
   if (bytes) *bytes = c.off + 256;
   return w;
 }
@@ -602,6 +697,12 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
   const PruneWs w = carve_prune(ws, rows, d, nullptr);
   cudaError_t e = tc::launch_split(U, d, d, d, w.U_hi, w.U_lo, d, info, st);
   if (e != cudaSuccess) return e;
+  // the quantization grid of the dense rows, before any column is touched
+  const float* qgrid = p.qgrid;
+  if (p.qbits > 0 && !qgrid) {
+    if ((e = launch_quant_grid(W, ldw, rows, d, p.qbits, w.qgrid, st)) != cudaSuccess) return e;
+    qgrid = w.qgrid;
+  }
   const tc::Operand Ep{w.Err_hi, w.Err_lo, rows, kMaxBlock, kMaxBlock};
   const tc::Operand Up{w.U_hi, w.U_lo, d, d, d};
   const int B = p.blocksize;
@@ -613,7 +714,8 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
     }
-    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, info, st);
+    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, qgrid,
+                     info, st);
     if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {
@@ -694,7 +796,8 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
     }
-    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, info, st);
+    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, p.qgrid, info,
+                     st);
     if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {

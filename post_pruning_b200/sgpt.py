@@ -12,7 +12,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import torch
 
@@ -32,7 +32,7 @@ EXPORTS = (
     "sgpt_workspace_bytes",
     "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
     "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
-    "sgpt_pack_nm", "sgpt_pack_nm_meta_words", "sgpt_recon_error", "sgpt_prune_layer",
+    "sgpt_pack_nm", "sgpt_pack_nm_meta_words", "sgpt_quant_grid", "sgpt_recon_error", "sgpt_prune_layer",
 )
 
 
@@ -46,7 +46,8 @@ class SgptError(RuntimeError):
 class _Params(ctypes.Structure):
     _fields_ = [("pattern", ctypes.c_int), ("n", ctypes.c_int), ("m", ctypes.c_int),
                 ("sparsity", ctypes.c_float), ("blocksize", ctypes.c_int),
-                ("damp", ctypes.c_float), ("forced", ctypes.c_int)]
+                ("damp", ctypes.c_float), ("forced", ctypes.c_int),
+                ("qbits", ctypes.c_int), ("qgrid", ctypes.c_void_p)]
 
 
 @dataclass(frozen=True)
@@ -56,6 +57,8 @@ class Params:
     blocksize: int = 128
     damp: float = 0.01
     forced: bool = False
+    qbits: int = 0              # >0: quantize the kept weights to 2**qbits levels per row
+    qgrid: object = field(default=None, compare=False)   # [d_out, 2] fp32 CUDA tensor or None
 
     @property
     def is_nm(self) -> bool:
@@ -72,11 +75,16 @@ class Params:
         return 0.0 if self.is_nm else float(self.pattern.split(":")[1])
 
     def to_c(self) -> _Params:
+        grid = None
+        if self.qgrid is not None:
+            _dev(self.qgrid, torch.float32, "qgrid")
+            grid = self.qgrid.data_ptr()
         if self.is_nm:
             n, m = (int(x) for x in self.pattern.split(":"))
-            return _Params(PATTERN_NM, n, m, 0.0, self.blocksize, self.damp, int(self.forced))
+            return _Params(PATTERN_NM, n, m, 0.0, self.blocksize, self.damp, int(self.forced),
+                           int(self.qbits), grid)
         return _Params(PATTERN_UNSTRUCTURED, 0, 0, self.sparsity, self.blocksize, self.damp,
-                       int(self.forced))
+                       int(self.forced), int(self.qbits), grid)
 
 
 _lib = None
@@ -110,6 +118,7 @@ def lib() -> ctypes.CDLL:
         "sgpt_pack24": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp]),
         "sgpt_pack_nm": (i32, [vp, i32, i32, i32, vp, i32, i32, vp, vp, vp, vp]),
         "sgpt_pack_nm_meta_words": (i32, [i32, i32, i32]),
+        "sgpt_quant_grid": (i32, [vp, i32, i32, i32, i32, vp, vp]),
         "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
                                    vp, sz, vp, vp]),
@@ -283,6 +292,18 @@ def pack24(W: torch.Tensor, mask: torch.Tensor, values: torch.Tensor, meta: torc
         raise ValueError("values must be [d_out, d_in/2] and meta [d_out, d_in/32]")
     _check(lib().sgpt_pack24(_ptr(W), r, d, ldw, _ptr(mask), _ptr(values), _ptr(meta), _ptr(dev_info),
                              _stream(stream)), "sgpt_pack24")
+
+
+def quant_grid(W: torch.Tensor, qbits: int, grid: torch.Tensor, stream=None):
+    """Per-row quantization grid of the dense W (sgpt_quant_grid): grid
+    [d_out, 2] fp32 = (scale, zero point)."""
+    _dev(W, torch.float32, "W")
+    _dev(grid, torch.float32, "grid")
+    ldw = _rowmajor(W, "W")
+    r, d = W.shape
+    if grid.shape != (r, 2) or not grid.is_contiguous():
+        raise ValueError("grid must be contiguous [d_out, 2]")
+    _check(lib().sgpt_quant_grid(_ptr(W), r, d, ldw, qbits, _ptr(grid), _stream(stream)), "sgpt_quant_grid")
 
 
 def pack_nm_meta_words(d_in: int, n: int, m: int) -> int:

@@ -133,8 +133,9 @@ def compare(gpu: dict, W0: np.ndarray, H: np.ndarray, U: np.ndarray, p: pp.Param
         gpu = restrict(gpu, rows)
         W0 = W0[rows]
     pat = pattern_of(p)
-    free = oracle.sweep(W0, U, pat, p.blocksize)
-    forced = oracle.sweep(W0, U, pat, p.blocksize, forced_mask=gpu["mask"])
+    qb = p.qbits or None
+    free = oracle.sweep(W0, U, pat, p.blocksize, qbits=qb)
+    forced = oracle.sweep(W0, U, pat, p.blocksize, forced_mask=gpu["mask"], qbits=qb)
     m = {}
     m["mask_agree_free"] = float(np.mean(gpu["mask"] == free["mask"]))
     if p.is_nm:
@@ -150,6 +151,15 @@ def compare(gpu: dict, W0: np.ndarray, H: np.ndarray, U: np.ndarray, p: pp.Param
         m["flip_max_gap"] = float(dist[differ].max()) if differ.any() else 0.0
         m["decision_agree"] = 1.0 - differ.mean()
     ref = forced["W"]
+    if qb:
+        # integer codes of the kept weights on each row's grid, GPU against
+        # the oracle's run along the GPU's mask
+        scale, zero = oracle.quant_grid(W0, qb)
+        kept = gpu["mask"]
+        cg = np.rint(gpu["W"].astype(np.float64) / scale[:, None].astype(np.float64))
+        co = np.rint(ref / scale[:, None].astype(np.float64))
+        m["code_agree"] = float(np.mean(cg[kept] == co[kept])) if kept.any() else 1.0
+        m["on_grid"] = bool(np.all(np.abs(gpu["W"] / scale[:, None] - cg) < 1e-3))
     m["weight_rel_l2"] = float(np.linalg.norm(gpu["W"] - ref) / max(np.linalg.norm(ref), 1e-300))
     num_g, den = oracle.recon_error(W0, gpu["W"], H)
     num_o, _ = oracle.recon_error(W0, free["W"], H)
@@ -188,5 +198,8 @@ def assert_parity(m: dict, p: pp.Params):
     # GPU's mask trajectory, each differing one a near-tie
     assert m["decision_agree"] >= MASK_AGREEMENT, m
     assert m["flip_max_gap"] < NEAR_TIE, m
+    if "code_agree" in m:
+        assert m["on_grid"], m
+        assert m["code_agree"] >= MASK_AGREEMENT, m
     assert m["weight_rel_l2"] <= WEIGHT_REL_L2, m
     assert m["recon_rel_diff"] <= RECON_REL, m

@@ -252,6 +252,46 @@ def test_nm_blocksize_independence_and_pack_errors():
     assert pp.sync_status(info) == 7
 
 
+# Joint sparsification and quantization (SparseGPT review, sections 十五
+# and 十七): every kept weight on its row's grid, the grid error compensated.
+QUANT_CASES = [pp.Params("2:4", qbits=4), pp.Params("2:4", qbits=8), pp.Params("16:64", qbits=4),
+               pp.Params("unstructured:0.5", qbits=4), pp.Params("unstructured:0.0", qbits=3)]
+
+
+@pytest.mark.parametrize("p", QUANT_CASES, ids=lambda p: f"{p.pattern}-q{p.qbits}")
+@pytest.mark.parametrize("spec", SMALL[:2] + [TALL_2K], ids=lambda s: s.name)
+def test_quantized_sweep_matches_oracle(spec, p):
+    W, X = _inputs(spec)
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs = (X64.T @ X64).astype(np.float32)
+    H, U_ref = _oracle_factor(Hs, spec.n_tok)
+    gpu = gpu_prune_layer(W, None, p, H_sum=torch.from_numpy(Hs), n_tok=spec.n_tok)
+    m_ = compare(gpu, W.numpy().astype(np.float64), H, U_ref, p)
+    assert_parity(m_, p)
+
+
+def test_quant_grid_is_bit_exact_and_reusable():
+    """sgpt_quant_grid equals the oracle's fp32 grid bit for bit; passing it
+    to the sweep gives the same result as letting the sweep compute it."""
+    spec = SMALL[1]
+    W, X = _inputs(spec)
+    dev = torch.device("cuda")
+    Wd = W.to(dev)
+    for bits in (2, 4, 8, 16):
+        grid = torch.empty(spec.d_out, 2, device=dev)
+        pp.quant_grid(Wd, bits, grid)
+        s_, z_ = oracle.quant_grid(W.numpy(), bits)
+        g = grid.cpu().numpy()
+        assert np.array_equal(g[:, 0], s_) and np.array_equal(g[:, 1], z_), bits
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs = torch.from_numpy((X64.T @ X64).astype(np.float32))
+    a = gpu_prune_layer(W, None, pp.Params("2:4", qbits=4), H_sum=Hs, n_tok=spec.n_tok)
+    grid = torch.empty(spec.d_out, 2, device=dev)
+    pp.quant_grid(Wd, 4, grid)
+    b = gpu_prune_layer(W, None, pp.Params("2:4", qbits=4, qgrid=grid), H_sum=Hs, n_tok=spec.n_tok)
+    assert np.array_equal(a["W"], b["W"]) and np.array_equal(a["mask"], b["mask"])
+
+
 def test_forced_mask_reproduces_oracle():
     spec = SMALL[1]
     W, X = _inputs(spec)
