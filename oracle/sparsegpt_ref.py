@@ -156,7 +156,8 @@ def parse_pattern(pattern):
     return ("nm", int(n), int(m), None)
 
 
-def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=None, qgrid=None):
+def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=None, qgrid=None,
+          forced_values=None):
     """Prune W [d_out, d_in] column by column with OBS compensation.
 
     With ``qbits`` the sweep also quantizes ([SGPT] sections 十五 and 十七,
@@ -172,7 +173,10 @@ def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=Non
       S_dec  the saliency each weight had when its mask was decided
       Err    the per-column errors e (float64 [d_out, d_in])
     With ``forced_mask`` the mask is taken as given and no selection is made
-    (S_dec is still recorded at the moment the pattern would decide).
+    (S_dec is still recorded at the moment the pattern would decide). With
+    ``forced_values`` as well, a kept weight takes the given value instead of
+    its grid value (W_dec records the weight each column had just before it
+    was replaced), so the sweep follows another run's decisions exactly.
     """
     kind, n_keep, m_grp, sparsity = parse_pattern(pattern)
     W = np.array(W, dtype=np.float64, copy=True)
@@ -184,6 +188,7 @@ def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=Non
     if forced_mask is not None:
         mask[:] = np.asarray(forced_mask, dtype=bool)
     S_dec = np.zeros((r, d))
+    W_dec = np.zeros((r, d))
     Err = np.zeros((r, d))
     loss = np.zeros(r)
     rows = np.arange(r)
@@ -222,7 +227,11 @@ def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=Non
                     np.put_along_axis(keep, order[:, :n_keep], True, axis=1)
                     mask[:, c:c + m_grp] = keep
             w = W1[:, q]
-            kept = quantize(w, qscale, qzero, qbits) if qbits else w
+            W_dec[:, c] = w
+            if forced_values is not None:
+                kept = np.asarray(forced_values[:, c], dtype=np.float64)
+            else:
+                kept = quantize(w, qscale, qzero, qbits) if qbits else w
             p = np.where(mask[:, c], kept, 0.0)
             e = (w - p) / U[c, c]
             W1[:, q:] -= np.outer(e, U[c, c:i2])
@@ -235,7 +244,7 @@ def sweep(W, U, pattern="2:4", blocksize: int = 128, forced_mask=None, qbits=Non
         # Lazy update of every column to the right of the block.
         W[:, i2:] -= E1 @ U[i1:i2, i2:]
 
-    return {"W": W, "mask": mask, "loss": loss, "S_dec": S_dec, "Err": Err}
+    return {"W": W, "mask": mask, "loss": loss, "S_dec": S_dec, "W_dec": W_dec, "Err": Err}
 
 
 # --------------------------------------------------------------------------
