@@ -261,6 +261,61 @@ sgpt_status sgpt_prune_layer(float* W, int d_out, int d_in, int ldw, const uint1
                              float* row_loss, void* ws, size_t ws_bytes, int* dev_info,
                              void* stream);
 
+/* ------------------------------------------------------------------------
+ * Multi-layer driver. The layer-wise procedure of the SparseGPT review,
+ * section 九 (collect the current layer's inputs, form its Hessian, prune
+ * and compensate, pass the pruned output to the next layer; section 十一,
+ * steps three to six), on one synthetic MLP block of a decoder:
+ *   x -> x' = x + W_down (silu(W_gate x) * (W_up x)),
+ * x [n_tok x hidden] and z = silu(W_gate x) * (W_up x) [n_tok x inter] bf16,
+ * the three products on the tensor cores in bf16 (the weights rounded to
+ * bf16) with fp32 accumulation, every rounding to bf16 to nearest even.
+ *   SGPT_DRIVER_SEQUENTIAL: gate and up are pruned from x (one Hessian and
+ *     factor), z is formed with the PRUNED gate and up, down is pruned from
+ *     z, and x' is the pruned block's output.
+ *   SGPT_DRIVER_PARALLEL (V-SparseGPT press release, voc.com.cn: the inputs
+ *     of every layer of the original model are recorded first, so layers are
+ *     sparsified side by side): z and x' come from the DENSE block; gate and
+ *     up are pruned from x and down from the recorded z, the down input's
+ *     Hessian on a second stream beside gate and up.
+ * blk: the three weight matrices (fp32, row-major, in: dense, out: pruned;
+ *   W_gate, W_up [inter x hidden], W_down [hidden x inter]) and their masks
+ *   ([inter x hidden/32], [hidden x inter/32]).
+ * X_next [n_tok x hidden] bf16 out; Z [n_tok x inter] bf16 out (the down
+ *   projection's input), or NULL to keep it in ws.
+ * p: pattern, block size, damping and qbits as for sgpt_prune (one grid per
+ *   matrix from its dense weights); p->forced and p->qgrid must be 0/NULL.
+ * ws: sgpt_mlp_block_workspace_bytes(hidden, inter, n_tok) bytes.
+ * *dev_info is cleared first; numeric errors as elsewhere. Stacked blocks
+ * are pruned by calling this once per block with X = the previous X_next. */
+#define SGPT_DRIVER_SEQUENTIAL 0
+#define SGPT_DRIVER_PARALLEL 1
+
+typedef struct sgpt_mlp_block {
+  float* W_gate;
+  float* W_up;
+  float* W_down;
+  uint32_t* mask_gate;
+  uint32_t* mask_up;
+  uint32_t* mask_down;
+} sgpt_mlp_block;
+
+size_t sgpt_mlp_block_workspace_bytes(int hidden, int inter, int64_t n_tok);
+sgpt_status sgpt_prune_mlp_block(const sgpt_mlp_block* blk, int hidden, int inter, const uint16_t* X, int64_t n_tok,
+                                 int mode, const sgpt_params* p, uint16_t* X_next, uint16_t* Z, void* ws,
+                                 size_t ws_bytes, int* dev_info, void* stream);
+
+/* The forward product of the driver: Y [n x d_out] fp32 = X [n x d_in] bf16
+ * times Wb^T, Wb [d_out x d_in] bf16, on the tensor cores
+ * (tcgen05.mma.kind::f16, fp32 accumulation in sums of at most 128 of K).
+ * d_in and d_out multiples of 32; 1 <= n < 2^31. */
+sgpt_status sgpt_linear_bf16(const uint16_t* X, const uint16_t* Wb, int64_t n, int d_in, int d_out, float* Y,
+                             int* dev_info, void* stream);
+
+/* Wb = W rounded to bf16 (to nearest even), rows x cols, W leading
+ * dimension ldw; Wb dense [rows x cols]. */
+sgpt_status sgpt_to_bf16(const float* W, int rows, int cols, int ldw, uint16_t* Wb, int* dev_info, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -5,6 +5,7 @@ of the bench use it. See ``sparsegpt_ref`` for what it computes and which
 passages of the pages each step follows.
 """
 
+from . import mlp_block_ref  # noqa: F401
 from .sparsegpt_ref import (  # noqa: F401
     NotPositiveDefinite,
     bits_to_mask,

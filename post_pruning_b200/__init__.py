@@ -6,6 +6,8 @@ kernels inside ``libsgpt.so``; see ``include/sgpt.h`` for the contract.
 """
 
 from .sgpt import (  # noqa: F401
+    DRIVER_PARALLEL,
+    DRIVER_SEQUENTIAL,
     EXPORTS,
     HostPruner,
     LIB_PATH,
@@ -20,18 +22,22 @@ from .sgpt import (  # noqa: F401
     info_clear,
     kernel_launches,
     lib,
+    linear_bf16,
+    mlp_block_workspace,
     new_info,
     pack24,
     pack_nm,
     pack_nm_meta_words,
     prune,
     prune_layer,
+    prune_mlp_block,
     prune_noalloc,
     quant_grid,
     raise_on_info,
     recon_error,
     set_wait_limit,
     sync_status,
+    to_bf16,
     workspace,
     workspace_bytes,
 )

@@ -202,6 +202,47 @@ sgpt_status sgpt_quant_grid(const float* W, int d_out, int d_in, int ldw, int qb
   return from_cuda(launch_quant_grid(W, ldw, d_out, d_in, qbits, grid, as_stream(stream)));
 }
 
+sgpt_status sgpt_to_bf16(const float* W, int rows, int cols, int ldw, uint16_t* Wb, int* dev_info, void* stream) {
+  if (!W || !Wb || !aligned16(W) || (reinterpret_cast<uintptr_t>(Wb) & 7u)) return SGPT_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 4 || cols % 4 || ldw < cols || ldw % 4) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_to_bf16(W, ldw, rows, cols, Wb, dev_info, as_stream(stream)));
+}
+
+sgpt_status sgpt_linear_bf16(const uint16_t* X, const uint16_t* Wb, int64_t n, int d_in, int d_out, float* Y,
+                             int* dev_info, void* stream) {
+  if (!X || !Wb || !Y || !dev_info || !aligned16(X) || !aligned16(Wb) || !aligned16(Y)) return SGPT_ERR_INVALID_ARG;
+  if (n < 1 || n > (int64_t)INT32_MAX || !valid_din(d_in) || !valid_din(d_out)) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_linear_bf16(X, Wb, n, d_in, d_out, Y, dev_info, as_stream(stream)));
+}
+
+size_t sgpt_mlp_block_workspace_bytes(int hidden, int inter, int64_t n_tok) {
+  if (!valid_din(hidden) || !valid_din(inter) || n_tok < 1 || n_tok > (int64_t)INT32_MAX) return 0;
+  return mlp_block_ws_bytes(hidden, inter, n_tok);
+}
+
+sgpt_status sgpt_prune_mlp_block(const sgpt_mlp_block* blk, int hidden, int inter, const uint16_t* X, int64_t n_tok,
+                                 int mode, const sgpt_params* p, uint16_t* X_next, uint16_t* Z, void* ws,
+                                 size_t ws_bytes, int* dev_info, void* stream) {
+  if (!blk || !X || !X_next || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (!blk->W_gate || !blk->W_up || !blk->W_down || !blk->mask_gate || !blk->mask_up || !blk->mask_down)
+    return SGPT_ERR_INVALID_ARG;
+  const void* ptrs[] = {blk->W_gate, blk->W_up, blk->W_down, blk->mask_gate, blk->mask_up, blk->mask_down, X, X_next};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return SGPT_ERR_INVALID_ARG;
+  if (Z && !aligned16(Z)) return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(hidden) || !valid_din(inter) || n_tok < 1 || n_tok > (int64_t)INT32_MAX) return SGPT_ERR_INVALID_ARG;
+  if (mode != SGPT_DRIVER_SEQUENTIAL && mode != SGPT_DRIVER_PARALLEL) return SGPT_ERR_INVALID_ARG;
+  sgpt_status s = check_params(p);
+  if (s != SGPT_OK) return s;
+  if (p->forced || p->qgrid) return SGPT_ERR_INVALID_ARG;     // each layer decides its own mask and grid
+  if (p->pattern == SGPT_PATTERN_NM && (hidden % p->m || inter % p->m)) return SGPT_ERR_INVALID_ARG;
+  s = check_ws(ws, ws_bytes, mlp_block_ws_bytes(hidden, inter, n_tok));
+  if (s != SGPT_OK) return s;
+  if ((s = sgpt_info_clear(dev_info, stream)) != SGPT_OK) return s;
+  return from_cuda(launch_prune_mlp_block(*blk, hidden, inter, X, n_tok, mode, *p, X_next, Z, ws, dev_info,
+                                          as_stream(stream)));
+}
+
 int sgpt_pack_nm_meta_words(int d_in, int n, int m) {
   if (!valid_din(d_in) || !valid_m(m) || n < 1 || n > m || d_in % m) return -1;
   return packnm_meta_words(d_in, n, m);

@@ -10,7 +10,9 @@
 //
 // Used for the panel products, the rank-128 updates and the triangular
 // inverse of the factorisation and for the lazy trailing update of the OBS
-// sweep.
+// sweep. The same kernel also runs plain bf16 products (one
+// tcgen05.mma.kind::f16 per K step of 16, K-major operands, fp32
+// accumulation), the forward passes between the layers of a block.
 //
 // Output tiles of 128 x 128, K in stages of 32 (one 128-byte swizzle row of
 // fp32) through a two-stage TMA ring of 64 KB stages (no multicast). Persistent: one CTA per
@@ -37,22 +39,39 @@ namespace tc {
 
 namespace {
 
-constexpr int kM = 128, kN = 128, kKC = 32;   // K per stage: one 128-byte swizzle row of fp32
-constexpr int kStages = 2;
-constexpr int kPlane = kM * kKC * 4;            // 16 KB: one operand plane of one stage
-constexpr int kStageBytes = 4 * kPlane;         // A hi/lo, B hi/lo
+constexpr int kM = 128, kN = 128;
+// The two arithmetic kinds of the kernel. kKindTf32x3: fp32 operands as hi/lo
+// TF32 planes, three tcgen05.mma.kind::tf32 products per K step of 8. kKindBf16:
+// bf16 operands, one tcgen05.mma.kind::f16 product per K step of 16. A stage
+// holds one 128-byte swizzle row of K per operand row in either case (32
+// fp32 or 64 bf16), so a plane is 16 KB; the bf16 ring has four stages in the
+// shared memory the fp32 one fills with two.
+constexpr int kKindTf32x3 = 0, kKindBf16 = 1;
+template <int KIND>
+struct Cfg {
+  static constexpr int KC = KIND == kKindTf32x3 ? 32 : 64;     // K per stage
+  static constexpr int PLANES = KIND == kKindTf32x3 ? 2 : 1;   // planes per operand
+  static constexpr int STAGES = KIND == kKindTf32x3 ? 2 : 4;
+  static constexpr int KSTEP = KIND == kKindTf32x3 ? 8 : 16;   // K per MMA
+};
+constexpr int kPlane = kM * 128;                // 16 KB: one operand plane of one stage
+template <int KIND>
+constexpr int stage_bytes() { return 2 * Cfg<KIND>::PLANES * kPlane; }
+constexpr int kRingBytes = 2 * stage_bytes<kKindTf32x3>();   // 128 KB, both kinds
+static_assert(Cfg<kKindBf16>::STAGES * stage_bytes<kKindBf16>() == kRingBytes, "same ring for both kinds");
 constexpr int kEpiWarps = 8;                    // two per TMEM lane quadrant, 64 columns each
 constexpr int kThreads = 64 + 32 * kEpiWarps;   // producer, MMA issuer, epilogue
 // Epilogue tile: 128 x 128 fp32 as four 32-column groups of 128 rows x 128
 // bytes, 16-byte chunks XOR-swizzled by row % 8 (TMA's 128-byte swizzle).
 constexpr size_t kStagingBytes = (size_t)kM * kN * 4;
-constexpr size_t kSmem = (size_t)kStages * kStageBytes + kStagingBytes + 1024 + 256;
-constexpr int kChunk = 128 / kKC;               // stages (128 of K) per TMEM accumulation
+constexpr size_t kSmem = (size_t)kRingBytes + kStagingBytes + 1024 + 256;
 constexpr int kTmemCols = 2 * kN;               // two accumulators: one fills while one drains
 
+template <int KIND>
 __host__ __device__ constexpr uint32_t make_idesc(bool b_mn) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(kN >> 3) << 17) |
-         ((uint32_t)(kM >> 4) << 24);
+  // D fp32; A and B tf32 (2) or bf16 (1); B MN-major bit 16; N/8, M/16
+  return (1u << 4) | ((KIND == kKindTf32x3 ? 2u : 1u) << 7) | ((KIND == kKindTf32x3 ? 2u : 1u) << 10) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -79,7 +98,7 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3fff);
-  d |= (uint64_t)((kKC * 128) >> 4) << 16;
+  d |= (uint64_t)((Cfg<kKindTf32x3>::KC * 128) >> 4) << 16;
   d |= (uint64_t)(512 >> 4) << 32;
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)1 << 61;
@@ -155,6 +174,12 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem, uint64_t a, uint64_t b, 
       " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
+__device__ __forceinline__ void mma_bf16(uint32_t tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
@@ -209,11 +234,15 @@ __device__ __forceinline__ Item decode_item(const Job& job, int w) {
 // one TMEM accumulator per unit of at most kChunk K steps, alternating two,
 // while the epilogue warps drain the other, so one tile's epilogue overlaps
 // the next tile's main loop.
-__global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
+template <int KIND>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
     const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo, const Job job,
     const __grid_constant__ CUtensorMap c_map, const int b_mn, const int items, int* info,
     const long long wait_cycles) {
+  constexpr int kStages = Cfg<KIND>::STAGES, kKC = Cfg<KIND>::KC, kPl = Cfg<KIND>::PLANES;
+  constexpr int kStageBytes = stage_bytes<KIND>();
+  constexpr int kChunk = 128 / kKC;             // stages (128 of K) per TMEM accumulation
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -224,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (cta_info_set(info)) return;
 
-  const uint32_t idesc = make_idesc(b_mn != 0);
+  const uint32_t idesc = make_idesc<KIND>(b_mn != 0);
   const uint32_t s0 = smem_u32(smem);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
   const uint32_t tfull0 = smem_u32(bars + 2 * kStages), tempty0 = tfull0 + 16, cfull = tfull0 + 32;
@@ -275,8 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
           const uint32_t sa = s0 + st * kStageBytes;
           const int k = it.kb + i * kKC;
           tma_2d(sa, &a_hi, bar, job.a_x0 + k, job.a_y0 + it.m0);
-          tma_2d(sa + kPlane, &a_lo, bar, job.a_x0 + k, job.a_y0 + it.m0);
-          if (b_mn) {
+          if (kPl == 2) tma_2d(sa + kPlane, &a_lo, bar, job.a_x0 + k, job.a_y0 + it.m0);
+          if (KIND == kKindBf16) {
+            tma_2d(sa + kPlane, &b_hi, bar, job.b_x0 + k, job.b_y0 + it.n0);
+          } else if (b_mn) {
 #pragma unroll
             for (int c = 0; c < kN / 32; ++c) {
               tma_2d(sa + 2 * kPlane + c * kKC * 128, &b_hi, bar, job.b_x0 + it.n0 + 32 * c, job.b_y0 + k);
@@ -317,7 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tf32x3_kernel(
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t sa = s0 + st * kStageBytes;
 #pragma unroll
-            for (int ks = 0; ks < kKC / 8; ++ks) {
+            for (int ks = 0; ks < kKC / Cfg<KIND>::KSTEP; ++ks) {
+              if constexpr (KIND == kKindBf16) {
+                // one K step of 16 bf16 is 32 bytes of each operand row
+                mma_bf16(acc_t, kmajor_desc(sa + ks * 32), kmajor_desc(sa + kPlane + ks * 32), idesc,
+                         (i == c0 && ks == 0) ? 0u : 1u);
+                continue;
+              }
               const uint64_t ah = kmajor_desc(sa + ks * 32), al = kmajor_desc(sa + kPlane + ks * 32);
               uint64_t bh, bl;
               if (b_mn) {
@@ -499,6 +536,20 @@ bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, lo
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map over a row-major bf16 matrix [rows x cols] (ld in elements):
+// boxes of 64 elements (one 128-byte swizzle row) x 128 rows.
+bool make_map_bf16(CUtensorMap* m, const uint16_t* p, long long rows, long long cols, long long ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)Cfg<kKindBf16>::KC, (cuuint32_t)kM};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tensor map over C for the epilogue: boxes of 32 columns x 128 rows with the
 // 128-byte swizzle.
 bool make_map_c(CUtensorMap* m, const float* p, long long rows, long long cols, long long ld) {
@@ -526,9 +577,35 @@ cudaError_t launch_split(const float* src, long long ld, int rows, int cols, flo
   return cudaGetLastError();
 }
 
+namespace {
+// Kernel attributes, the persistent grid, C's map and the launch: shared by
+// both arithmetic kinds.
+template <int KIND>
+cudaError_t launch_kind(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh, const CUtensorMap& bl,
+                        bool b_mn, const Job& job, int grid, int* info, cudaStream_t st) {
+  static PerDevice attrs;
+  cudaError_t ea = once_per_device(attrs, [] {
+    return cudaFuncSetAttribute(gemm_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+  });
+  if (ea != cudaSuccess) return ea;
+  // persistent: one CTA per SM at most, fewer when the job leaves SMs to others
+  const int ctas = std::min(grid, job.max_ctas > 0 ? std::min(job.max_ctas, kNumSMs) : kNumSMs);
+  // C comes in by TMA when it is read (beta != 0); otherwise the map is unused
+  CUtensorMap cm = ah;
+  if (job.C && job.beta != 0.f &&
+      !make_map_c(&cm, job.C, (long long)job.c_row0 + job.Mlim, (long long)job.c_col0 + job.Nlim, job.ldc))
+    return cudaErrorInvalidValue;
+  gemm_tc_kernel<KIND><<<ctas, kThreads, kSmem, st>>>(ah, al, bh, bl, job, cm, b_mn ? 1 : 0, grid, info,
+                                                      wait_limit_cycles());
+  count_launches(1);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
                         cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
+  constexpr int kKC = Cfg<kKindTf32x3>::KC;
   CUtensorMap ah, al, bh, bl;
   if (!make_map(&ah, A.hi, A.rows, A.cols, A.ld, kKC, kM, false) ||
       !make_map(&al, A.lo, A.rows, A.cols, A.ld, kKC, kM, false))
@@ -542,22 +619,16 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
         !make_map(&bl, B.lo, B.rows, B.cols, B.ld, kKC, kN, false))
       return cudaErrorInvalidValue;
   }
-  static PerDevice attrs;
-  cudaError_t ea = once_per_device(attrs, [] {
-    return cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-  });
-  if (ea != cudaSuccess) return ea;
-  // persistent: one CTA per SM at most, fewer when the job leaves SMs to others
-  const int ctas = std::min(grid, job.max_ctas > 0 ? std::min(job.max_ctas, kNumSMs) : kNumSMs);
-  // C comes in by TMA when it is read (beta != 0); otherwise the map is unused
-  CUtensorMap cm = ah;
-  if (job.C && job.beta != 0.f &&
-      !make_map_c(&cm, job.C, (long long)job.c_row0 + job.Mlim, (long long)job.c_col0 + job.Nlim, job.ldc))
+  return launch_kind<kKindTf32x3>(ah, al, bh, bl, b_mn, job, grid, info, st);
+}
+
+cudaError_t launch_gemm_bf16(const OperandBf16& A, const OperandBf16& B, const Job& job, int grid, int* info,
+                             cudaStream_t st) {
+  if (grid <= 0) return cudaSuccess;
+  CUtensorMap ah, bh;
+  if (!make_map_bf16(&ah, A.p, A.rows, A.cols, A.ld) || !make_map_bf16(&bh, B.p, B.rows, B.cols, B.ld))
     return cudaErrorInvalidValue;
-  gemm_tf32x3_kernel<<<ctas, kThreads, kSmem, st>>>(ah, al, bh, bl, job, cm, b_mn ? 1 : 0, grid, info,
-                                                    wait_limit_cycles());
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_kind<kKindBf16>(ah, ah, bh, bh, false, job, grid, info, st);
 }
 
 }  // namespace tc

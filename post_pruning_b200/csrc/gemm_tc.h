@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 namespace sgpt {
 namespace tc {
@@ -45,10 +46,22 @@ struct Job {
   int max_ctas;      // persistent CTAs at most (0: one per SM)
 };
 
+// A bf16 operand: row-major rows x cols, leading dimension ld (ld % 8 == 0,
+// 16-byte aligned base); K-major, i.e. K is the column index.
+struct OperandBf16 {
+  const uint16_t* p;
+  long long rows, cols, ld;
+};
+
 constexpr int kTileTC = 128;
 
 cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
                         cudaStream_t st);
+// C = alpha * A B^T + beta * C with A [M x K] and B [N x K] bf16 (both
+// K-major), fp32 accumulation and C; Job fields as above (mode 0 only, no
+// planes needed).
+cudaError_t launch_gemm_bf16(const OperandBf16& A, const OperandBf16& B, const Job& job, int grid, int* info,
+                             cudaStream_t st);
 cudaError_t launch_split(const float* src, long long ld, int rows, int cols, float* hi, float* lo, long long ldo,
                          const int* info, cudaStream_t st);
 

@@ -37,6 +37,16 @@ size_t recon_ws_bytes(int rows, int d);
 cudaError_t launch_recon(const float* W0, const float* W, int rows, int d, long long ldw,
                          const float* H, double* num_den, void* ws, cudaStream_t st);
 
+// driver.cu
+cudaError_t launch_to_bf16(const float* W, long long ld, long long rows, int cols, uint16_t* Wb, const int* info,
+                           cudaStream_t st);
+cudaError_t launch_linear_bf16(const uint16_t* X, const uint16_t* Wb, long long n, int d_in, int d_out, float* Y,
+                               int* info, cudaStream_t st);
+size_t mlp_block_ws_bytes(int h, int f, long long n);
+cudaError_t launch_prune_mlp_block(const sgpt_mlp_block& blk, int h, int f, const uint16_t* X, long long n,
+                                   int mode, const sgpt_params& p, uint16_t* X_next, uint16_t* Z, void* ws,
+                                   int* info, cudaStream_t st);
+
 // hessian_tc.cu
 size_t hessian_ws_bytes(int d, long long n);
 cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, void* ws, int* info,

@@ -33,7 +33,10 @@ EXPORTS = (
     "sgpt_info_clear", "sgpt_sync_status", "sgpt_hessian_zero",
     "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
     "sgpt_pack_nm", "sgpt_pack_nm_meta_words", "sgpt_quant_grid", "sgpt_recon_error", "sgpt_prune_layer",
+    "sgpt_mlp_block_workspace_bytes", "sgpt_prune_mlp_block", "sgpt_linear_bf16", "sgpt_to_bf16",
 )
+DRIVER_SEQUENTIAL = 0
+DRIVER_PARALLEL = 1
 
 
 class SgptError(RuntimeError):
@@ -87,6 +90,11 @@ class Params:
                        int(self.forced), int(self.qbits), grid)
 
 
+class _MlpBlock(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("W_gate", "W_up", "W_down", "mask_gate", "mask_up", "mask_down")]
+
+
 _lib = None
 
 
@@ -119,6 +127,11 @@ def lib() -> ctypes.CDLL:
         "sgpt_pack_nm": (i32, [vp, i32, i32, i32, vp, i32, i32, vp, vp, vp, vp]),
         "sgpt_pack_nm_meta_words": (i32, [i32, i32, i32]),
         "sgpt_quant_grid": (i32, [vp, i32, i32, i32, i32, vp, vp]),
+        "sgpt_mlp_block_workspace_bytes": (sz, [i32, i32, i64]),
+        "sgpt_prune_mlp_block": (i32, [ctypes.POINTER(_MlpBlock), i32, i32, vp, i64, i32, pp, vp, vp, vp, sz,
+                                       vp, vp]),
+        "sgpt_linear_bf16": (i32, [vp, vp, i64, i32, i32, vp, vp, vp]),
+        "sgpt_to_bf16": (i32, [vp, i32, i32, i32, vp, vp, vp]),
         "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
                                    vp, sz, vp, vp]),
@@ -304,6 +317,72 @@ def quant_grid(W: torch.Tensor, qbits: int, grid: torch.Tensor, stream=None):
     if grid.shape != (r, 2) or not grid.is_contiguous():
         raise ValueError("grid must be contiguous [d_out, 2]")
     _check(lib().sgpt_quant_grid(_ptr(W), r, d, ldw, qbits, _ptr(grid), _stream(stream)), "sgpt_quant_grid")
+
+
+def to_bf16(W: torch.Tensor, Wb: torch.Tensor, dev_info: torch.Tensor, stream=None):
+    """Wb = W rounded to bf16 (sgpt_to_bf16)."""
+    _dev(W, torch.float32, "W")
+    _dev(Wb, torch.bfloat16, "Wb")
+    ldw = _rowmajor(W, "W")
+    if Wb.shape != W.shape or not Wb.is_contiguous():
+        raise ValueError("Wb must be contiguous with W's shape")
+    _check(lib().sgpt_to_bf16(_ptr(W), W.shape[0], W.shape[1], ldw, _ptr(Wb), _ptr(dev_info), _stream(stream)),
+           "sgpt_to_bf16")
+
+
+def linear_bf16(X: torch.Tensor, Wb: torch.Tensor, Y: torch.Tensor, dev_info: torch.Tensor, stream=None):
+    """Y = X Wb^T on the tensor cores (sgpt_linear_bf16): X [n, d_in] and Wb
+    [d_out, d_in] bf16, Y [n, d_out] fp32."""
+    _dev(X, torch.bfloat16, "X")
+    _dev(Wb, torch.bfloat16, "Wb")
+    _dev(Y, torch.float32, "Y")
+    n, d_in = X.shape
+    d_out = Wb.shape[0]
+    if Wb.shape[1] != d_in or Y.shape != (n, d_out) or not (X.is_contiguous() and Wb.is_contiguous()
+                                                             and Y.is_contiguous()):
+        raise ValueError("X [n, d_in], Wb [d_out, d_in], Y [n, d_out], all contiguous")
+    _check(lib().sgpt_linear_bf16(_ptr(X), _ptr(Wb), n, d_in, d_out, _ptr(Y), _ptr(dev_info), _stream(stream)),
+           "sgpt_linear_bf16")
+
+
+def mlp_block_workspace(hidden: int, inter: int, n_tok: int, device="cuda") -> torch.Tensor:
+    b = int(lib().sgpt_mlp_block_workspace_bytes(hidden, inter, n_tok))
+    if b == 0:
+        raise ValueError("unsupported block sizes")
+    return torch.empty(b, dtype=torch.uint8, device=device)
+
+
+def prune_mlp_block(W_gate: torch.Tensor, W_up: torch.Tensor, W_down: torch.Tensor, masks, X: torch.Tensor,
+                    params: Params, X_next: torch.Tensor, ws: torch.Tensor, dev_info: torch.Tensor,
+                    mode: int = DRIVER_SEQUENTIAL, Z: torch.Tensor | None = None, stream=None):
+    """One synthetic MLP block pruned layer by layer (sgpt_prune_mlp_block).
+    masks: (gate, up, down) int32 mask-bit tensors."""
+    for t, name in ((W_gate, "W_gate"), (W_up, "W_up"), (W_down, "W_down")):
+        _dev(t, torch.float32, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _dev(X, torch.bfloat16, "X")
+    _dev(X_next, torch.bfloat16, "X_next")
+    inter, hidden = W_gate.shape
+    if W_up.shape != (inter, hidden) or W_down.shape != (hidden, inter):
+        raise ValueError("W_gate, W_up [inter, hidden] and W_down [hidden, inter]")
+    n = X.shape[0]
+    if X.shape != (n, hidden) or X_next.shape != (n, hidden):
+        raise ValueError("X and X_next must be [n_tok, hidden]")
+    if Z is not None:
+        _dev(Z, torch.bfloat16, "Z")
+        if Z.shape != (n, inter) or not Z.is_contiguous():
+            raise ValueError("Z must be contiguous [n_tok, inter]")
+    mg, mu, md = masks
+    for m_, shape in ((mg, (inter, hidden // 32)), (mu, (inter, hidden // 32)), (md, (hidden, inter // 32))):
+        _dev(m_, torch.int32, "mask")
+        if m_.shape != shape or not m_.is_contiguous():
+            raise ValueError(f"mask must be contiguous {shape}")
+    blk = _MlpBlock(_ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(mg), _ptr(mu), _ptr(md))
+    p = params.to_c()
+    _check(lib().sgpt_prune_mlp_block(ctypes.byref(blk), hidden, inter, _ptr(X), n, mode, ctypes.byref(p),
+                                      _ptr(X_next), _ptr(Z), _ptr(ws), ws.numel(), _ptr(dev_info),
+                                      _stream(stream)), "sgpt_prune_mlp_block")
 
 
 def pack_nm_meta_words(d_in: int, n: int, m: int) -> int:
