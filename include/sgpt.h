@@ -312,6 +312,20 @@ sgpt_status sgpt_prune_mlp_block(const sgpt_mlp_block* blk, int hidden, int inte
 sgpt_status sgpt_linear_bf16(const uint16_t* X, const uint16_t* Wb, int64_t n, int d_in, int d_out, float* Y,
                              int* dev_info, void* stream);
 
+/* A consumer of the 2:4 output (2:4 production guide, section on the 2:4
+ * mechanism: two kept weights of every four along the reduction axis and
+ * their 2-bit positions): Y [n x d_out] fp32 = X W^T, where W [d_out x d_in]
+ * is given ONLY in packed form,
+ *   values [d_out x d_in/2] bf16 (e.g. sgpt_pack24's values through
+ *          sgpt_to_bf16),
+ *   meta   [d_out x d_in/32] uint32, sgpt_pack24's metadata words,
+ * and X [n x d_in] bf16. Runs on the sparse tensor cores
+ * (tcgen05.mma.sp.kind::f16, fp32 accumulation); the library re-arranges
+ * the metadata into the layout the instruction reads (the 4-bit group codes
+ * are the same). d_in % 32 == 0; 1 <= n < 2^31. */
+sgpt_status sgpt_sparse24_linear(const uint16_t* values, const uint32_t* meta, int d_out, int d_in,
+                                 const uint16_t* X, int64_t n, float* Y, int* dev_info, void* stream);
+
 /* Wb = W rounded to bf16 (to nearest even), rows x cols, W leading
  * dimension ldw; Wb dense [rows x cols]. */
 sgpt_status sgpt_to_bf16(const float* W, int rows, int cols, int ldw, uint16_t* Wb, int* dev_info, void* stream);

@@ -36,6 +36,7 @@ from .sgpt import (  # noqa: F401
     raise_on_info,
     recon_error,
     set_wait_limit,
+    sparse24_linear,
     sync_status,
     to_bf16,
     workspace,

@@ -215,6 +215,14 @@ sgpt_status sgpt_linear_bf16(const uint16_t* X, const uint16_t* Wb, int64_t n, i
   return from_cuda(launch_linear_bf16(X, Wb, n, d_in, d_out, Y, dev_info, as_stream(stream)));
 }
 
+sgpt_status sgpt_sparse24_linear(const uint16_t* values, const uint32_t* meta, int d_out, int d_in,
+                                 const uint16_t* X, int64_t n, float* Y, int* dev_info, void* stream) {
+  if (!values || !meta || !X || !Y || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (!aligned16(values) || !aligned16(meta) || !aligned16(X) || !aligned16(Y)) return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out) || n < 1 || n > (int64_t)INT32_MAX) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_sparse24_gemm(values, meta, d_out, d_in, X, n, Y, dev_info, as_stream(stream)));
+}
+
 size_t sgpt_mlp_block_workspace_bytes(int hidden, int inter, int64_t n_tok) {
   if (!valid_din(hidden) || !valid_din(inter) || n_tok < 1 || n_tok > (int64_t)INT32_MAX) return 0;
   return mlp_block_ws_bytes(hidden, inter, n_tok);

@@ -47,6 +47,10 @@ cudaError_t launch_prune_mlp_block(const sgpt_mlp_block& blk, int h, int f, cons
                                    int mode, const sgpt_params& p, uint16_t* X_next, uint16_t* Z, void* ws,
                                    int* info, cudaStream_t st);
 
+// consumer.cu
+cudaError_t launch_sparse24_gemm(const uint16_t* values_bf16, const uint32_t* meta, int rows, int d,
+                                 const uint16_t* X, long long n, float* Y, int* info, cudaStream_t st);
+
 // hessian_tc.cu
 size_t hessian_ws_bytes(int d, long long n);
 cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, void* ws, int* info,

@@ -34,6 +34,7 @@ EXPORTS = (
     "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
     "sgpt_pack_nm", "sgpt_pack_nm_meta_words", "sgpt_quant_grid", "sgpt_recon_error", "sgpt_prune_layer",
     "sgpt_mlp_block_workspace_bytes", "sgpt_prune_mlp_block", "sgpt_linear_bf16", "sgpt_to_bf16",
+    "sgpt_sparse24_linear",
 )
 DRIVER_SEQUENTIAL = 0
 DRIVER_PARALLEL = 1
@@ -132,6 +133,7 @@ def lib() -> ctypes.CDLL:
                                        vp, vp]),
         "sgpt_linear_bf16": (i32, [vp, vp, i64, i32, i32, vp, vp, vp]),
         "sgpt_to_bf16": (i32, [vp, i32, i32, i32, vp, vp, vp]),
+        "sgpt_sparse24_linear": (i32, [vp, vp, i32, i32, vp, i64, vp, vp, vp]),
         "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
                                    vp, sz, vp, vp]),
@@ -343,6 +345,26 @@ def linear_bf16(X: torch.Tensor, Wb: torch.Tensor, Y: torch.Tensor, dev_info: to
         raise ValueError("X [n, d_in], Wb [d_out, d_in], Y [n, d_out], all contiguous")
     _check(lib().sgpt_linear_bf16(_ptr(X), _ptr(Wb), n, d_in, d_out, _ptr(Y), _ptr(dev_info), _stream(stream)),
            "sgpt_linear_bf16")
+
+
+def sparse24_linear(values: torch.Tensor, meta: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
+                    dev_info: torch.Tensor, stream=None):
+    """Y = X W^T from W's packed 2:4 form on the sparse tensor cores
+    (sgpt_sparse24_linear): values [d_out, d_in/2] bf16, meta [d_out,
+    d_in/32] int32 (sgpt_pack24's words), X [n, d_in] bf16, Y [n, d_out]
+    fp32."""
+    _dev(values, torch.bfloat16, "values")
+    _dev(meta, torch.int32, "meta")
+    _dev(X, torch.bfloat16, "X")
+    _dev(Y, torch.float32, "Y")
+    d_out, half = values.shape
+    n, d_in = X.shape
+    if half * 2 != d_in or meta.shape != (d_out, d_in // 32) or Y.shape != (n, d_out):
+        raise ValueError("values [d_out, d_in/2], meta [d_out, d_in/32], X [n, d_in], Y [n, d_out]")
+    if not (values.is_contiguous() and meta.is_contiguous() and X.is_contiguous() and Y.is_contiguous()):
+        raise ValueError("all operands must be contiguous")
+    _check(lib().sgpt_sparse24_linear(_ptr(values), _ptr(meta), d_out, d_in, _ptr(X), n, _ptr(Y), _ptr(dev_info),
+                                      _stream(stream)), "sgpt_sparse24_linear")
 
 
 def mlp_block_workspace(hidden: int, inter: int, n_tok: int, device="cuda") -> torch.Tensor:
