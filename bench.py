@@ -77,6 +77,12 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--config", default=CONFIG, help="workload (default: the Qwen3-32B-shaped block)")
+    ap.add_argument("--pattern", default=None,
+                    help="prune every matrix with this pattern instead (e.g. 16:64, unstructured:0.5)")
+    ap.add_argument("--qbits", type=int, default=0,
+                    help="joint sparsification and quantization of the kept weights to this many bits")
+    ap.add_argument("--driver", choices=["sequential", "parallel"], default="sequential",
+                    help="mode of the multi-layer driver (config qwen3_32b_mlp_block)")
     return ap.parse_args()
 
 
@@ -309,7 +315,8 @@ def phase_rooflines(jobs, phase_ms, sustained: bool) -> dict:
     f_flops = sum(2.0 / 3.0 * xs.d_in ** 3 for xs, _, _ in jobs)
     sweep_bytes = sum(12.0 * sp.d_out * sp.d_in for _, _, mats in jobs for sp, _ in mats)
     trail_flops = sum(float(sp.d_out) * (sp.d_in ** 2 - sp.d_in * B) for _, _, mats in jobs for sp, _ in mats)
-    pack_bytes = sum(6.25 * sp.d_out * sp.d_in for _, _, mats in jobs for sp, p in mats if p.is_nm)
+    pack_bytes = sum(6.25 * sp.d_out * sp.d_in for _, _, mats in jobs for sp, p in mats
+                     if p.is_nm and p.nm == (2, 4))
     out = {}
 
     def entry(name, bound, achieved, peak, unit, work, extra=None):
@@ -351,8 +358,16 @@ def phase_rooflines(jobs, phase_ms, sustained: bool) -> dict:
 def main():
     args = parse()
     from workloads import CONFIGS
+    if args.config in EXTRA_BENCHES:
+        EXTRA_BENCHES[args.config](args)
+        return
     specs = CONFIGS[args.config]
+    if args.pattern:
+        specs = [sp.with_(runs=(args.pattern,)) for sp in specs]
     workload = WORKLOADS.get(args.config, args.config)
+    if args.pattern or args.qbits:
+        workload += f" [pattern {args.pattern or 'as listed'}, quantized to {args.qbits} bits]" if args.qbits else \
+            f" [pattern {args.pattern}]"
     if args.impl == "reference":
         reference_arm(args, specs, workload)
         return
@@ -382,11 +397,11 @@ def main():
         sp = specs[0]
         X = gen_activations(sp, device=dev)
         for run in sp.runs:
-            jobs.append((sp, X, [(sp, pp.Params(run))]))
+            jobs.append((sp, X, [(sp, pp.Params(run, qbits=args.qbits))]))
     else:
         for key, group in group_by_input(specs).items():
             X = gen_activations(group[0], device=dev)
-            jobs.append((group[0], X, [(sp, pp.Params(sp.runs[0])) for sp in group]))
+            jobs.append((group[0], X, [(sp, pp.Params(sp.runs[0], qbits=args.qbits)) for sp in group]))
     layers = []      # (W0, W, LayerGraphs, spec, params)
     job_graphs = []
     for xs, X, mats in jobs:
@@ -396,11 +411,11 @@ def main():
             W0 = gen_weights(sp, device=dev)
             W = W0.clone()
             if first is None:
-                b = pp.LayerBuffers.allocate(sp.d_out, sp.d_in, xs.n_tok, dev)
+                b = pp.LayerBuffers.allocate(sp.d_out, sp.d_in, xs.n_tok, dev, nm=p.nm if p.is_nm else (2, 4))
                 g = pp.LayerGraphs(b, W, X, p)
                 first = b
             else:
-                b = pp.LayerBuffers.sharing(first, sp.d_out, dev)
+                b = pp.LayerBuffers.sharing(first, sp.d_out, dev, nm=p.nm if p.is_nm else (2, 4))
                 g = pp.LayerGraphs(b, W, None, p, phases=("prune", "pack"))
             layers.append((W0, W, g, sp, p))
             gl.append(g)
@@ -599,6 +614,156 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ other rows
+
+def _events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def bench_mlp_block(args):
+    """The multi-layer driver on one Qwen3-32B-shaped MLP block (hidden 5120,
+    intermediate 25600, 131,072 tokens, 2:4 unless --pattern): gate and up
+    pruned from the block input, the down input formed with the pruned (or,
+    --driver parallel, dense) gate and up, down pruned from it, the block
+    output formed; every step restores the dense weights (untimed). Also
+    times the driver's forward product alone (sgpt_linear_bf16 of the same
+    shape as gate) for its roofline."""
+    import torch
+
+    import post_pruning_b200 as pp
+    from workloads import LayerSpec, gen_activations, gen_weights
+    dev = torch.device("cuda")
+    h, f, n = 5120, 25600, 131072
+    spec = LayerSpec("mlp_in", d_in=h, d_out=f, n_tok=n, sigma=1.0, p_out=0.01, f_out=20.0, x_key=2)
+    X = gen_activations(spec, device=dev)
+    W0 = [gen_weights(spec.with_(w_key=4), device=dev), gen_weights(spec.with_(w_key=5), device=dev),
+          gen_weights(LayerSpec("down", d_in=f, d_out=h, n_tok=n, w_key=6), device=dev)]
+    W = [w.clone() for w in W0]
+    masks = (torch.empty(f, h // 32, dtype=torch.int32, device=dev), torch.empty(f, h // 32, dtype=torch.int32,
+             device=dev), torch.empty(h, f // 32, dtype=torch.int32, device=dev))
+    X_next = torch.empty(n, h, dtype=torch.bfloat16, device=dev)
+    ws = pp.mlp_block_workspace(h, f, n)
+    info = pp.new_info()
+    p = pp.Params(args.pattern or "2:4", qbits=args.qbits)
+    mode = pp.DRIVER_PARALLEL if args.driver == "parallel" else pp.DRIVER_SEQUENTIAL
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def step():
+        pp.prune_mlp_block(*W, masks, X, p, X_next, ws, info, mode=mode)
+
+    def prep():
+        for w, w0 in zip(W, W0):
+            w.copy_(w0)
+        flush.zero_()
+    for _ in range(args.warmup):
+        prep()
+        step()
+    pp.raise_on_info(info)
+    evs = [_events(torch) for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    l0 = pp.kernel_launches()
+    for e0, e1 in evs:
+        prep()
+        e0.record(st)
+        step()
+        e1.record(st)
+    torch.cuda.synchronize()
+    launches = pp.kernel_launches() - l0
+    clk = clocks.stop()
+    pp.raise_on_info(info)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    weights = 3 * h * f
+    # the forward product alone: x Wg^T, n x h x f
+    Wb = torch.empty(f, h, dtype=torch.bfloat16, device=dev)
+    pp.to_bf16(W0[0], Wb, info)
+    Y = torch.empty(n, f, device=dev)
+    for _ in range(3):
+        pp.linear_bf16(X, Wb, Y, info)
+    e0, e1 = _events(torch)
+    e0.record(st)
+    for _ in range(10):
+        pp.linear_bf16(X, Wb, Y, info)
+    e1.record(st)
+    torch.cuda.synchronize()
+    g_ms = e0.elapsed_time(e1) / 10
+    g_flops = 2.0 * n * h * f
+    hbm, bf16_burst, bf16_sust, kind = peaks()
+    line = {"metric": "multi-layer driver: one MLP block pruned layer by layer, weights/s", "value": weights / ms * 1e3,
+            "unit": "weights/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "f32 (forward products bf16)", "data": "synthetic",
+            "config": {"workload": f"Qwen3-32B-shaped MLP block h={h} f={f}, {n} tokens, {p.pattern}, "
+                                   f"driver {args.driver}", "name": "qwen3_32b_mlp_block"},
+            "gpu_launches": launches,
+            "forward_gemm": {"kernel": "gemm_tc_kernel<bf16>", "shape": f"{n}x{h} * {h}x{f}", "ms": g_ms,
+                             "achieved": g_flops / g_ms / 1e9, "unit": "TFLOP/s", "peak": bf16_burst,
+                             "frac": g_flops / g_ms / 1e9 / bf16_burst, "peak_kind": f"{kind} bf16 burst"},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
+def bench_consumer(args):
+    """The 2:4 consumer: Y = X W^T from the packed 2:4 form of the Qwen3-32B
+    down-proj (5120 x 25600) on the sparse tensor cores, against the dense
+    tensor-core product of the same (unpacked, bf16) weights; 8192 tokens."""
+    import torch
+
+    import post_pruning_b200 as pp
+    dev = torch.device("cuda")
+    d_out, d_in, n = 5120, 25600, 8192
+    g = torch.Generator(device=dev).manual_seed(0)
+    W = torch.randn(d_out, d_in, device=dev, generator=g)
+    keep = torch.zeros(d_out, d_in // 4, 4, dtype=torch.bool, device=dev)
+    keep.scatter_(2, torch.rand(d_out, d_in // 4, 4, device=dev, generator=g).topk(2, dim=2).indices, True)
+    keep = keep.reshape(d_out, d_in)
+    W = torch.where(keep, W, torch.zeros_like(W))
+    bits = (keep.reshape(d_out, d_in // 32, 32).to(torch.int64) << torch.arange(32, device=dev)).sum(2)
+    mask = torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits).to(torch.int32)   # the same 32 bits as int32
+    info = pp.new_info()
+    vals = torch.empty(d_out, d_in // 2, device=dev)
+    meta = torch.empty(d_out, d_in // 32, dtype=torch.int32, device=dev)
+    pp.pack24(W, mask, vals, meta, info)
+    vb = torch.empty(d_out, d_in // 2, dtype=torch.bfloat16, device=dev)
+    pp.to_bf16(vals, vb, info)
+    Wb = torch.empty(d_out, d_in, dtype=torch.bfloat16, device=dev)
+    pp.to_bf16(W, Wb, info)
+    X = torch.randn(n, d_in, device=dev, generator=g).to(torch.bfloat16)
+    Y = torch.empty(n, d_out, device=dev)
+    pp.raise_on_info(info)
+    st = torch.cuda.current_stream()
+    out = {}
+    for name, fn in (("sparse24", lambda: pp.sparse24_linear(vb, meta, X, Y, info)),
+                     ("dense", lambda: pp.linear_bf16(X, Wb, Y, info))):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = _events(torch)
+        e0.record(st)
+        for _ in range(args.steps):
+            fn()
+        e1.record(st)
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / args.steps
+    pp.raise_on_info(info)
+    flops = 2.0 * n * d_in * d_out
+    hbm, bf16_burst, bf16_sust, kind = peaks()
+    line = {"metric": "2:4 consumer: Y = X W^T from the packed 2:4 form, dense-equivalent TFLOP/s",
+            "value": flops / out["sparse24"] / 1e9, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": out["sparse24"], "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"X {n}x{d_in} bf16, W {d_out}x{d_in} 2:4 (values bf16 + 2-bit metadata)",
+                       "name": "consumer_qwen_down"},
+            "dense_ms": out["dense"], "dense_tflops": flops / out["dense"] / 1e9,
+            "speedup_vs_dense": out["dense"] / out["sparse24"],
+            "peak": {"bf16_dense": bf16_burst, "sparse_2to4_nominal": 2 * bf16_burst, "kind": f"{kind} burst"}}
+    print(json.dumps(line), flush=True)
+
+
+EXTRA_BENCHES = {"qwen3_32b_mlp_block": bench_mlp_block, "consumer_qwen_down": bench_consumer}
 
 
 if __name__ == "__main__":
