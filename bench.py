@@ -83,6 +83,8 @@ def parse():
                     help="joint sparsification and quantization of the kept weights to this many bits")
     ap.add_argument("--driver", choices=["sequential", "parallel"], default="sequential",
                     help="mode of the multi-layer driver (config qwen3_32b_mlp_block)")
+    ap.add_argument("--width", type=int, default=25600, help="d_in of config hessian")
+    ap.add_argument("--tokens", type=int, default=131072, help="tokens of config hessian")
     return ap.parse_args()
 
 
@@ -763,7 +765,43 @@ def bench_consumer(args):
     print(json.dumps(line), flush=True)
 
 
-EXTRA_BENCHES = {"qwen3_32b_mlp_block": bench_mlp_block, "consumer_qwen_down": bench_consumer}
+def bench_hessian(args):
+    """The Hessian kernel alone: H = X^T X for X [tokens x width] bf16 with
+    the Qwen-block channel-scale distribution (sgpt_hessian_compute), for
+    per-kernel timing and profiler captures at a chosen size."""
+    import torch
+
+    import post_pruning_b200 as pp
+    from workloads import LayerSpec, gen_activations
+    dev = torch.device("cuda")
+    spec = LayerSpec("hessian", d_in=args.width, d_out=128, n_tok=args.tokens, sigma=1.0, p_out=0.01, f_out=20.0,
+                     x_key=3)
+    X = gen_activations(spec, device=dev)
+    H = torch.empty(args.width, args.width, device=dev)
+    ws = pp.workspace(128, args.width, args.tokens)
+    info = pp.new_info()
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        pp.hessian_compute(H, X, ws, info)
+    e0, e1 = _events(torch)
+    e0.record(st)
+    for _ in range(args.steps):
+        pp.hessian_compute(H, X, ws, info)
+    e1.record(st)
+    torch.cuda.synchronize()
+    pp.raise_on_info(info)
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = float(args.tokens) * args.width * (args.width + 1)
+    hbm, bf16_burst, bf16_sust, kind = peaks()
+    print(json.dumps({"metric": "Hessian H = X^T X alone, TFLOP/s (n*d*(d+1) flop)", "value": flops / ms / 1e9,
+                      "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+                      "config": {"workload": f"X {args.tokens} x {args.width} bf16", "name": "hessian"},
+                      "peak": bf16_burst, "frac": flops / ms / 1e9 / bf16_burst, "peak_kind": f"{kind} bf16 burst"}),
+          flush=True)
+
+
+EXTRA_BENCHES = {"qwen3_32b_mlp_block": bench_mlp_block, "consumer_qwen_down": bench_consumer,
+                 "hessian": bench_hessian}
 
 
 if __name__ == "__main__":

@@ -796,32 +796,52 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
     }
     if (k > 0) {
       // T_iq += R_ik U_kq for i < k, q >= k (rows [0, c0), columns [c0, d)),
-      // with the planes of T's block row k-1, which this term completes
+      // with the planes of T's block row k-1, which this term completes.
+      // Paired steps (k+1, k): the first adds its term to block row k only
+      // (which the next block row of U needs); the second adds both steps'
+      // terms to the rows above, K = 256 over the columns right of the pair
+      // and K = 128 over block column k (U_{k+1,k} = 0), so the rectangle is
+      // read and written once per two block columns.
       if ((e = cudaStreamWaitEvent(f.rows, f.chain_done, 0)) != cudaSuccess) return e;
       if (k >= 2 && (e = cudaStreamWaitEvent(f.rows, f.panel_done, 0)) != cudaSuccess) return e;
-      tc::Job job{};
-      job.mode = 0;
-      job.mt = k;
-      job.nt = K - k;
-      job.kdim = bk;
-      job.a_x0 = c0;
-      job.b_x0 = c0;
-      job.b_y0 = c0;
-      job.C = U;
-      job.ldc = d;
-      job.c_col0 = c0;
-      job.Mlim = c0;
-      job.Nlim = d - c0;
-      job.alpha = 1.f;
-      job.beta = 1.f;
-      job.C_hi = w.T_hi;
-      job.C_lo = w.T_lo;
-      job.ldp = d;
-      job.p_row0 = c0 - kTile;
-      job.planes_one_row = 1;
-      job.planes_m0 = c0 - kTile;
-      job.max_ctas = kOffChainCtas;
-      if ((e = tc::launch_gemm(Rp, Ud, true, job, k * (K - k), info, f.rows)) != cudaSuccess) return e;
+      const bool t_second = paired && ((K - 1 - k) & 1) != 0;
+      const bool t_first = paired && !t_second;
+      auto t_job = [&](int row0, int rows, int col0, int cols, int kdim) {
+        tc::Job job{};
+        job.mode = 0;
+        job.mt = rows / kTile;
+        job.nt = cdiv(cols, kTile);
+        job.kdim = kdim;
+        job.a_x0 = c0;
+        job.a_y0 = row0;
+        job.b_x0 = col0;
+        job.b_y0 = c0;
+        job.C = U;
+        job.ldc = d;
+        job.c_row0 = row0;
+        job.c_col0 = col0;
+        job.Mlim = rows;
+        job.Nlim = cols;
+        job.alpha = 1.f;
+        job.beta = 1.f;
+        job.C_hi = w.T_hi;
+        job.C_lo = w.T_lo;
+        job.ldp = d;
+        job.p_row0 = c0 - kTile;
+        job.planes_one_row = 1;
+        job.planes_m0 = c0 - kTile - row0;
+        job.max_ctas = kOffChainCtas;
+        return tc::launch_gemm(Rp, Ud, true, job, job.mt * job.nt, info, f.rows);
+      };
+      if (t_first) {
+        if ((e = t_job(c0 - kTile, kTile, c0, d - c0, bk)) != cudaSuccess) return e;
+      } else if (t_second) {
+        const int c1 = c0 + kTile;
+        if (c1 < d && (e = t_job(0, c0, c1, d - c1, std::min(2 * kTile, d - c0))) != cudaSuccess) return e;
+        if ((e = t_job(0, c0, c0, bk, bk)) != cudaSuccess) return e;
+      } else {
+        if ((e = t_job(0, c0, c0, d - c0, bk)) != cudaSuccess) return e;
+      }
     }
   }
   return cudaSuccess;
