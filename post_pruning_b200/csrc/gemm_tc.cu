@@ -213,11 +213,23 @@ struct Item {
   int m0, n0, kb, ke;
 };
 
+// Dense grids are walked in groups of kGroupRows tile rows, rows fastest
+// inside a group: the CTAs resident together share the A panels of the
+// group's rows and the B panels of a few tile columns, which stay in L2
+// while the CTAs stream K (a row-major order walks every column of B for
+// each few rows and reads B from DRAM again and again when it exceeds L2).
+constexpr int kGroupRows = 16;
+
 __device__ __forceinline__ Item decode_item(const Job& job, int w) {
   Item it{0, 0, 0, 0};
   if (job.mode == 0) {
-    it.m0 = (w / job.nt) * kM;
-    it.n0 = (w % job.nt) * kN;
+    const int per_group = kGroupRows * job.nt;
+    const int g = w / per_group;
+    const int first = g * kGroupRows;
+    const int rows = min(kGroupRows, job.mt - first);
+    const int r = w - g * per_group;
+    it.m0 = (first + r % rows) * kM;
+    it.n0 = (r / rows) * kN;
     it.ke = job.kdim;
   } else if (job.mode == 1) {
     int i, j;
