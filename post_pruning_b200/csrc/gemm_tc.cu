@@ -495,84 +495,49 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(
 
 // ------------------------------------------------------------- wide tiles
 //
-// 128 x 256 output tiles for dense grids (mode 0). Per K stage a CTA loads
-// 128 rows of A and 256 of B, so each byte of operands feeds twice the
-// products of a 128 x 128 tile: with 128 x 128 tiles the tensor pipe needs
-// more operand bytes per cycle per SM than L2 delivers. Four 48 KB stages
-// (3xTF32: 16 of K per stage, 64-byte swizzle, hi/lo planes of A and B;
-// bf16: 64 of K, 128-byte swizzle); two 256-column TMEM accumulators (all
-// 512 columns); warp 0 loads, warp 1 issues N = 256 MMAs, warps 2-9 drain
-// TMEM (lane quadrant w % 4, columns 128 (w - 2) / 4 ..) and write their rows
-// of C straight from registers (16-byte accesses, each thread its own row),
-// with the optional hi/lo planes. Every wait is bounded as in the kernel
-// above.
+// 128 x 256 output tiles for the bf16 products on dense grids (mode 0). Per
+// K stage a CTA loads 128 rows of A and 256 of B, so each byte of operands
+// feeds twice the products of a 128 x 128 tile: with 128 x 128 tiles the
+// tensor pipe needs more operand bytes per cycle per SM than L2 delivers
+// (the 8192 x 5120 x 25600 product: 0.41 -> 0.63 of the bf16 peak). Four
+// 48 KB stages of 64 of K (128-byte swizzle); two 256-column TMEM
+// accumulators (all 512 columns); warp 0 loads, warp 1 issues N = 256 MMAs,
+// warps 2-9 drain TMEM (lane quadrant w % 4, columns 128 (w - 2) / 4 ..) and
+// write their rows of C straight from registers (16-byte accesses, each
+// thread its own row). The bf16 products have long K and no C to read, so
+// the epilogue is a small part of a tile. Every wait is bounded as in the
+// kernel above.
 namespace {
-template <int KIND>
-struct WideCfg {
-  static constexpr int KC = KIND == kKindTf32x3 ? 16 : 64;     // K per stage (one swizzle row)
-  static constexpr int PLANES = KIND == kKindTf32x3 ? 2 : 1;
-  static constexpr int KSTEP = KIND == kKindTf32x3 ? 8 : 16;
-  static constexpr int ELEM = KIND == kKindTf32x3 ? 4 : 2;
-  static constexpr int A_PLANE = kM * KC * ELEM;                 // 8 KB / 16 KB
-  static constexpr int B_PLANE = 256 * KC * ELEM;                // 16 KB / 32 KB
-  static constexpr int STAGE = PLANES * (A_PLANE + B_PLANE);     // 48 KB both
-};
-constexpr int kWN = 256, kWStages = 4;
-constexpr size_t kWideSmem = (size_t)kWStages * 48 * 1024 + 1024 + 256;
+constexpr int kWN = 256, kWStages = 4, kWKC = 64;
+constexpr int kWAPlane = kM * kWKC * 2;          // 16 KB
+constexpr int kWBPlane = kWN * kWKC * 2;         // 32 KB
+constexpr int kWStage = kWAPlane + kWBPlane;     // 48 KB
+constexpr size_t kWideSmem = (size_t)kWStages * kWStage + 1024 + 256;
 constexpr int kWTmemCols = 2 * kWN;
-static_assert(WideCfg<kKindTf32x3>::STAGE == 48 * 1024 && WideCfg<kKindBf16>::STAGE == 48 * 1024, "stage size");
-
-// K-major operand with the 64-byte swizzle (a stage of 16 fp32 per row):
-// 8-row groups of 512 bytes.
-__device__ __forceinline__ uint64_t kmajor_desc_sw64(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3fff);
-  d |= (uint64_t)1 << 16;
-  d |= (uint64_t)(512 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)4 << 61;                         // SWIZZLE_64B
-  return d;
-}
-// MN-major 32-bit operand in 32-column atoms (see mnmajor_desc) with 16 K
-// rows per box: LBO = one box (16 x 128 bytes), SBO = 4 K rows.
-__device__ __forceinline__ uint64_t mnmajor_desc_k16(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3fff);
-  d |= (uint64_t)((16 * 128) >> 4) << 16;
-  d |= (uint64_t)(512 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)1 << 61;
-  return d;
-}
 }  // namespace
 
-template <int KIND>
-__global__ void __launch_bounds__(kThreads, 1) gemm_wide_kernel(
-    const __grid_constant__ CUtensorMap a_hi, const __grid_constant__ CUtensorMap a_lo,
-    const __grid_constant__ CUtensorMap b_hi, const __grid_constant__ CUtensorMap b_lo, const Job job,
-    const int b_mn, const int items, int* info, const long long wait_cycles) {
-  using C = WideCfg<KIND>;
-  constexpr int kKC = C::KC, kChunk = 128 / C::KC;
+__global__ void __launch_bounds__(kThreads, 1) gemm_wide_bf16_kernel(
+    const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap b_map, const Job job,
+    const int items, int* info, const long long wait_cycles) {
+  constexpr int kChunk = 128 / kWKC;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWStages * C::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWStages * kWStage);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kWStages + 6);
   __shared__ int failed;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (cta_info_set(info)) return;
 
-  // D fp32; A, B tf32 or bf16; B MN-major (bit 16); N = 256, M = 128
-  const uint32_t idesc = (1u << 4) | ((KIND == kKindTf32x3 ? 2u : 1u) << 7) |
-                         ((KIND == kKindTf32x3 ? 2u : 1u) << 10) | ((b_mn ? 1u : 0u) << 16) |
-                         ((uint32_t)(kWN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+  // D fp32, A and B bf16, both K-major, N = 256, M = 128
+  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kWN >> 3) << 17) |
+                             ((uint32_t)(kM >> 4) << 24);
   const uint32_t s0 = smem_u32(smem);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kWStages);
   const uint32_t tfull0 = smem_u32(bars + 2 * kWStages), tempty0 = tfull0 + 16, mdone = tfull0 + 32;
   if (threadIdx.x == 0) {
-    const CUtensorMap* maps[4] = {&a_hi, &a_lo, &b_hi, &b_lo};
-    for (int i = 0; i < 4; ++i)
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(maps[i])) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a_map)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&b_map)) : "memory");
     failed = 0;
     for (int st = 0; st < kWStages; ++st) {
       mbar_init(full0 + 8 * st, 1);
@@ -604,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_wide_kernel(
     m0 = (first + r % rows) * kM;
     n0 = (r / rows) * kWN;
   };
-  const int iters = (job.kdim + kKC - 1) / kKC;
+  const int iters = (job.kdim + kWKC - 1) / kWKC;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -619,21 +584,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_wide_kernel(
             break;
           }
           const uint32_t bar = full0 + 8 * st;
-          mbar_expect_tx(bar, C::STAGE);
-          const uint32_t sa = s0 + st * C::STAGE, sb = sa + C::PLANES * C::A_PLANE;
-          const int k = i * kKC;
-          tma_2d(sa, &a_hi, bar, job.a_x0 + k, job.a_y0 + m0);
-          if (C::PLANES == 2) tma_2d(sa + C::A_PLANE, &a_lo, bar, job.a_x0 + k, job.a_y0 + m0);
-          if (KIND == kKindTf32x3 && b_mn) {
-#pragma unroll
-            for (int c = 0; c < kWN / 32; ++c) {
-              tma_2d(sb + c * kKC * 128, &b_hi, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
-              tma_2d(sb + C::B_PLANE + c * kKC * 128, &b_lo, bar, job.b_x0 + n0 + 32 * c, job.b_y0 + k);
-            }
-          } else {
-            tma_2d(sb, &b_hi, bar, job.b_x0 + k, job.b_y0 + n0);
-            if (C::PLANES == 2) tma_2d(sb + C::B_PLANE, &b_lo, bar, job.b_x0 + k, job.b_y0 + n0);
-          }
+          mbar_expect_tx(bar, kWStage);
+          const uint32_t sa = s0 + st * kWStage;
+          const int k = i * kWKC;
+          tma_2d(sa, &a_map, bar, job.a_x0 + k, job.a_y0 + m0);
+          tma_2d(sa + kWAPlane, &b_map, bar, job.b_x0 + k, job.b_y0 + n0);
         }
       }
       for (int x = (g > kWStages ? g - kWStages : 0); x < g; ++x)
@@ -659,27 +614,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_wide_kernel(
               break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t sa = s0 + st * C::STAGE, sb = sa + C::PLANES * C::A_PLANE;
+            const uint32_t sa = s0 + st * kWStage;
 #pragma unroll
-            for (int ks = 0; ks < kKC / C::KSTEP; ++ks) {
-              const uint32_t first = (i == c0 && ks == 0) ? 0u : 1u;
-              if constexpr (KIND == kKindBf16) {
-                mma_bf16(acc_t, kmajor_desc(sa + ks * 32), kmajor_desc(sb + ks * 32), idesc, first);
-              } else {
-                const uint64_t ah = kmajor_desc_sw64(sa + ks * 32), al = kmajor_desc_sw64(sa + C::A_PLANE + ks * 32);
-                uint64_t bh, bl;
-                if (b_mn) {
-                  bh = mnmajor_desc_k16(sb + ks * 1024);
-                  bl = mnmajor_desc_k16(sb + C::B_PLANE + ks * 1024);
-                } else {
-                  bh = kmajor_desc_sw64(sb + ks * 32);
-                  bl = kmajor_desc_sw64(sb + C::B_PLANE + ks * 32);
-                }
-                mma_tf32(acc_t, al, bh, idesc, first);   // small terms first
-                mma_tf32(acc_t, ah, bl, idesc, 1u);
-                mma_tf32(acc_t, ah, bh, idesc, 1u);
-              }
-            }
+            for (int ks = 0; ks < kWKC / 16; ++ks)   // K steps of 16 bf16 = 32 bytes of each row
+              mma_bf16(acc_t, kmajor_desc(sa + ks * 32), kmajor_desc(sa + kWAPlane + ks * 32), idesc,
+                       (i == c0 && ks == 0) ? 0u : 1u);
             mma_commit(empty0 + 8 * st);
           }
           mma_commit(tfull0 + 8 * b);
@@ -693,7 +632,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_wide_kernel(
     const int q = warp & 3, h = (warp - 2) >> 2;
     const int m = q * 32 + lane;                    // tile row = TMEM lane
     const bool read_c = job.C != nullptr && job.beta != 0.f;
-    const long long ldp = job.ldp ? job.ldp : job.ldc;
     int u = 0;
     for (int w = blockIdx.x; w < items; w += gridDim.x) {
       int m0, n0;
@@ -719,28 +657,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_wide_kernel(
         if (lane == 0) mbar_arrive(tempty0 + 8 * b);
       }
       const int row = m0 + m;
-      if (!failed && row < job.Mlim) {
-        const bool planes = job.C_hi != nullptr && (!job.planes_one_row || m0 == job.planes_m0);
-        const long long crow = (long long)(job.c_row0 + row) * job.ldc + job.c_col0;
-        const long long prow = (long long)(job.c_row0 + row - job.p_row0) * ldp + job.c_col0 - job.p_col0;
+      if (!failed && row < job.Mlim && job.C) {
+        float* crow = job.C + (long long)(job.c_row0 + row) * job.ldc + job.c_col0;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int col = n0 + h * 128 + 4 * j;
           if (col >= job.Nlim) continue;
           float4 o = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
-          if (read_c) {
-            const float4 cv = ld4(job.C + crow + col);
-            o = make_float4(fmaf(job.alpha, o.x, job.beta * cv.x), fmaf(job.alpha, o.y, job.beta * cv.y),
-                            fmaf(job.alpha, o.z, job.beta * cv.z), fmaf(job.alpha, o.w, job.beta * cv.w));
-          } else {
-            o = make_float4(job.alpha * o.x, job.alpha * o.y, job.alpha * o.z, job.alpha * o.w);
-          }
-          if (job.C) st4(job.C + crow + col, o);
-          if (planes) {
-            const float4 hv = make_float4(tf32_hi(o.x), tf32_hi(o.y), tf32_hi(o.z), tf32_hi(o.w));
-            st4(job.C_hi + prow + col, hv);
-            st4(job.C_lo + prow + col, make_float4(o.x - hv.x, o.y - hv.y, o.z - hv.z, o.w - hv.w));
-          }
+          const float4 cv = read_c ? ld4(crow + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+          o = make_float4(fmaf(job.alpha, o.x, job.beta * cv.x), fmaf(job.alpha, o.y, job.beta * cv.y),
+                          fmaf(job.alpha, o.z, job.beta * cv.z), fmaf(job.alpha, o.w, job.beta * cv.w));
+          st4(crow + col, o);
         }
       }
     }
@@ -803,21 +730,6 @@ bool make_map(CUtensorMap* m, const float* p, long long rows, long long cols, lo
              CU_TENSOR_MAP_INTERLEAVE_NONE,
              mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The same over fp32 with a chosen swizzle (the wide tiles' 64-byte K-major
-// boxes of 16 fp32).
-bool make_map_sw(CUtensorMap* m, const float* p, long long rows, long long cols, long long ld, int box_x, int box_y,
-                 CUtensorMapSwizzle sw) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
-  const cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_y};
-  const cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -889,49 +801,33 @@ cudaError_t launch_kind(const CUtensorMap& ah, const CUtensorMap& al, const CUte
 }  // namespace
 
 namespace {
-template <int KIND>
-cudaError_t launch_wide(const CUtensorMap& ah, const CUtensorMap& al, const CUtensorMap& bh, const CUtensorMap& bl,
-                        bool b_mn, const Job& job, int items, int* info, cudaStream_t st) {
+cudaError_t launch_wide_bf16(const CUtensorMap& a_map, const CUtensorMap& b_map, const Job& job, int items, int* info,
+                             cudaStream_t st) {
   static PerDevice attrs;
   cudaError_t ea = once_per_device(attrs, [] {
-    return cudaFuncSetAttribute(gemm_wide_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideSmem);
+    return cudaFuncSetAttribute(gemm_wide_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kWideSmem);
   });
   if (ea != cudaSuccess) return ea;
   const int ctas = std::min(items, job.max_ctas > 0 ? std::min(job.max_ctas, kNumSMs) : kNumSMs);
-  gemm_wide_kernel<KIND><<<ctas, kThreads, kWideSmem, st>>>(ah, al, bh, bl, job, b_mn ? 1 : 0, items, info,
-                                                           wait_limit_cycles());
+  gemm_wide_bf16_kernel<<<ctas, kThreads, kWideSmem, st>>>(a_map, b_map, job, items, info, wait_limit_cycles());
   count_launches(1);
   return cudaGetLastError();
 }
 
-// Dense grids more than one tile column wide go to the 128 x 256 tiles
-// (their job.nt counted in 256-column tiles), except jobs whose planes
-// belong to one 128-column tile column.
-bool use_wide(const Job& job) { return job.mode == 0 && !job.planes_one_col && job.Nlim > kN; }
+// bf16 dense grids more than one tile column wide go to the 128 x 256 tiles
+// (their job.nt counted in 256-column tiles). The 3xTF32 jobs stay on the
+// 128 x 128 tiles: they are read-modify-write updates with short K (128 or
+// 256), whose time is in the epilogue's C traffic, and the same wide tiles
+// with a register-direct epilogue measured slower for them than the
+// TMA-fed, coalesced one (factor 125 -> 149 ms, sweep 64 -> 103 ms on the
+// default workload).
+bool use_wide_bf16(const Job& job) { return job.mode == 0 && job.Nlim > kN; }
 }  // namespace
 
 cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job& job, int grid, int* info,
                         cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
-  if (use_wide(job)) {
-    constexpr int KC = WideCfg<kKindTf32x3>::KC;
-    CUtensorMap ah, al, bh, bl;
-    if (!make_map_sw(&ah, A.hi, A.rows, A.cols, A.ld, KC, kM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_sw(&al, A.lo, A.rows, A.cols, A.ld, KC, kM, CU_TENSOR_MAP_SWIZZLE_64B))
-      return cudaErrorInvalidValue;
-    if (b_mn) {
-      if (!make_map_sw(&bh, B.hi, B.rows, B.cols, B.ld, 32, KC, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
-          !make_map_sw(&bl, B.lo, B.rows, B.cols, B.ld, 32, KC, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
-        return cudaErrorInvalidValue;
-    } else {
-      if (!make_map_sw(&bh, B.hi, B.rows, B.cols, B.ld, KC, kWN, CU_TENSOR_MAP_SWIZZLE_64B) ||
-          !make_map_sw(&bl, B.lo, B.rows, B.cols, B.ld, KC, kWN, CU_TENSOR_MAP_SWIZZLE_64B))
-        return cudaErrorInvalidValue;
-    }
-    Job w = job;
-    w.nt = cdiv(job.Nlim, kWN);
-    return launch_wide<kKindTf32x3>(ah, al, bh, bl, b_mn, w, w.mt * w.nt, info, st);
-  }
   constexpr int kKC = Cfg<kKindTf32x3>::KC;
   CUtensorMap ah, al, bh, bl;
   if (!make_map(&ah, A.hi, A.rows, A.cols, A.ld, kKC, kM, false) ||
@@ -952,13 +848,13 @@ cudaError_t launch_gemm(const Operand& A, const Operand& B, bool b_mn, const Job
 cudaError_t launch_gemm_bf16(const OperandBf16& A, const OperandBf16& B, const Job& job, int grid, int* info,
                              cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
-  if (use_wide(job)) {
+  if (use_wide_bf16(job)) {
     CUtensorMap ah, bh;
     if (!make_map_bf16(&ah, A.p, A.rows, A.cols, A.ld) || !make_map_bf16(&bh, B.p, B.rows, B.cols, B.ld, kWN))
       return cudaErrorInvalidValue;
     Job w = job;
     w.nt = cdiv(job.Nlim, kWN);
-    return launch_wide<kKindBf16>(ah, ah, bh, bh, false, w, w.mt * w.nt, info, st);
+    return launch_wide_bf16(ah, bh, w, w.mt * w.nt, info, st);
   }
   CUtensorMap ah, bh;
   if (!make_map_bf16(&ah, A.p, A.rows, A.cols, A.ld) || !make_map_bf16(&bh, B.p, B.rows, B.cols, B.ld))
