@@ -737,10 +737,12 @@ def bench_consumer(args):
     X = torch.randn(n, d_in, device=dev, generator=g).to(torch.bfloat16)
     Y = torch.empty(n, d_out, device=dev)
     pp.raise_on_info(info)
+    tiles = pp.sparse24_meta_tiles(meta, d_in)      # once per weight matrix, timed apart below
     st = torch.cuda.current_stream()
     out = {}
-    for name, fn in (("sparse24", lambda: pp.sparse24_linear(vb, meta, X, Y, info)),
-                     ("dense", lambda: pp.linear_bf16(X, Wb, Y, info))):
+    for name, fn in (("sparse24", lambda: pp.sparse24_linear(vb, tiles, X, Y, info)),
+                     ("dense", lambda: pp.linear_bf16(X, Wb, Y, info)),
+                     ("tile_meta", lambda: pp.sparse24_meta_tiles(meta, d_in, out=tiles))):
         for _ in range(args.warmup):
             fn()
         e0, e1 = _events(torch)
@@ -760,6 +762,7 @@ def bench_consumer(args):
             "config": {"workload": f"X {n}x{d_in} bf16, W {d_out}x{d_in} 2:4 (values bf16 + 2-bit metadata)",
                        "name": "consumer_qwen_down"},
             "dense_ms": out["dense"], "dense_tflops": flops / out["dense"] / 1e9,
+            "tile_meta_ms": out["tile_meta"],
             "speedup_vs_dense": out["dense"] / out["sparse24"],
             "peak": {"bf16_dense": bf16_burst, "sparse_2to4_nominal": 2 * bf16_burst, "kind": f"{kind} burst"}}
     print(json.dumps(line), flush=True)

@@ -316,14 +316,27 @@ sgpt_status sgpt_linear_bf16(const uint16_t* X, const uint16_t* Wb, int64_t n, i
  * mechanism: two kept weights of every four along the reduction axis and
  * their 2-bit positions): Y [n x d_out] fp32 = X W^T, where W [d_out x d_in]
  * is given ONLY in packed form,
- *   values [d_out x d_in/2] bf16 (e.g. sgpt_pack24's values through
- *          sgpt_to_bf16),
- *   meta   [d_out x d_in/32] uint32, sgpt_pack24's metadata words,
+ *   values     [d_out x d_in/2] bf16 (e.g. sgpt_pack24's values through
+ *              sgpt_to_bf16),
+ *   meta_tiles sgpt_pack24's metadata words re-arranged once per weight
+ *              matrix by sgpt_sparse24_tile_meta,
  * and X [n x d_in] bf16. Runs on the sparse tensor cores
- * (tcgen05.mma.sp.kind::f16, fp32 accumulation); the library re-arranges
- * the metadata into the layout the instruction reads (the 4-bit group codes
- * are the same). d_in % 32 == 0; 1 <= n < 2^31. */
-sgpt_status sgpt_sparse24_linear(const uint16_t* values, const uint32_t* meta, int d_out, int d_in,
+ * (tcgen05.mma.sp.kind::f16, fp32 accumulation in one sum over all of K).
+ * d_in % 32 == 0; 1 <= n < 2^31. All pointers device, 16-byte aligned; Y is
+ * written, nothing else. A bounded wait that runs out sets
+ * SGPT_INFO_TIMEOUT in *dev_info.
+ *
+ * meta_tiles: sgpt_sparse24_meta_tiles_bytes(d_out, d_in) bytes (0 = bad
+ * sizes), caller-owned. The layout is the order in which the sparse tensor
+ * cores read the metadata from tensor memory, in 4 KB pieces per 256 rows
+ * and 128 columns of K (each 4-bit group code unchanged; rows and columns
+ * past the matrix hold a valid padding code). sgpt_sparse24_tile_meta
+ * reads meta [d_out x d_in/32] uint32 (sgpt_pack24's words) and writes
+ * meta_tiles on `stream`; its result is opaque and reusable for every
+ * product with the same weights. */
+size_t sgpt_sparse24_meta_tiles_bytes(int d_out, int d_in);
+sgpt_status sgpt_sparse24_tile_meta(const uint32_t* meta, int d_out, int d_in, uint32_t* meta_tiles, void* stream);
+sgpt_status sgpt_sparse24_linear(const uint16_t* values, const uint32_t* meta_tiles, int d_out, int d_in,
                                  const uint16_t* X, int64_t n, float* Y, int* dev_info, void* stream);
 
 /* Wb = W rounded to bf16 (to nearest even), rows x cols, W leading

@@ -37,6 +37,7 @@ from .sgpt import (  # noqa: F401
     recon_error,
     set_wait_limit,
     sparse24_linear,
+    sparse24_meta_tiles,
     sync_status,
     to_bf16,
     workspace,

@@ -215,12 +215,23 @@ sgpt_status sgpt_linear_bf16(const uint16_t* X, const uint16_t* Wb, int64_t n, i
   return from_cuda(launch_linear_bf16(X, Wb, n, d_in, d_out, Y, dev_info, as_stream(stream)));
 }
 
-sgpt_status sgpt_sparse24_linear(const uint16_t* values, const uint32_t* meta, int d_out, int d_in,
+size_t sgpt_sparse24_meta_tiles_bytes(int d_out, int d_in) {
+  if (!valid_din(d_in) || !valid_dout(d_out)) return 0;
+  return sparse24_meta_tiles_bytes(d_out, d_in);
+}
+
+sgpt_status sgpt_sparse24_tile_meta(const uint32_t* meta, int d_out, int d_in, uint32_t* meta_tiles, void* stream) {
+  if (!meta || !meta_tiles || !aligned16(meta_tiles)) return SGPT_ERR_INVALID_ARG;
+  if (!valid_din(d_in) || !valid_dout(d_out)) return SGPT_ERR_INVALID_ARG;
+  return from_cuda(launch_tile_meta(meta, d_out, d_in, meta_tiles, as_stream(stream)));
+}
+
+sgpt_status sgpt_sparse24_linear(const uint16_t* values, const uint32_t* meta_tiles, int d_out, int d_in,
                                  const uint16_t* X, int64_t n, float* Y, int* dev_info, void* stream) {
-  if (!values || !meta || !X || !Y || !dev_info) return SGPT_ERR_INVALID_ARG;
-  if (!aligned16(values) || !aligned16(meta) || !aligned16(X) || !aligned16(Y)) return SGPT_ERR_INVALID_ARG;
+  if (!values || !meta_tiles || !X || !Y || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (!aligned16(values) || !aligned16(meta_tiles) || !aligned16(X) || !aligned16(Y)) return SGPT_ERR_INVALID_ARG;
   if (!valid_din(d_in) || !valid_dout(d_out) || n < 1 || n > (int64_t)INT32_MAX) return SGPT_ERR_INVALID_ARG;
-  return from_cuda(launch_sparse24_gemm(values, meta, d_out, d_in, X, n, Y, dev_info, as_stream(stream)));
+  return from_cuda(launch_sparse24_gemm(values, meta_tiles, d_out, d_in, X, n, Y, dev_info, as_stream(stream)));
 }
 
 size_t sgpt_mlp_block_workspace_bytes(int hidden, int inter, int64_t n_tok) {

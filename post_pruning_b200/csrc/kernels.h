@@ -48,7 +48,9 @@ cudaError_t launch_prune_mlp_block(const sgpt_mlp_block& blk, int h, int f, cons
                                    int* info, cudaStream_t st);
 
 // consumer.cu
-cudaError_t launch_sparse24_gemm(const uint16_t* values_bf16, const uint32_t* meta, int rows, int d,
+size_t sparse24_meta_tiles_bytes(int rows, int d);
+cudaError_t launch_tile_meta(const uint32_t* meta, int rows, int d, uint32_t* tiles, cudaStream_t st);
+cudaError_t launch_sparse24_gemm(const uint16_t* values_bf16, const uint32_t* tiles, int rows, int d,
                                  const uint16_t* X, long long n, float* Y, int* info, cudaStream_t st);
 
 // hessian_tc.cu

@@ -34,7 +34,7 @@ EXPORTS = (
     "sgpt_hessian_accumulate", "sgpt_hessian_compute", "sgpt_factor", "sgpt_prune", "sgpt_prune_noalloc", "sgpt_pack24",
     "sgpt_pack_nm", "sgpt_pack_nm_meta_words", "sgpt_quant_grid", "sgpt_recon_error", "sgpt_prune_layer",
     "sgpt_mlp_block_workspace_bytes", "sgpt_prune_mlp_block", "sgpt_linear_bf16", "sgpt_to_bf16",
-    "sgpt_sparse24_linear",
+    "sgpt_sparse24_linear", "sgpt_sparse24_meta_tiles_bytes", "sgpt_sparse24_tile_meta",
 )
 DRIVER_SEQUENTIAL = 0
 DRIVER_PARALLEL = 1
@@ -134,6 +134,8 @@ def lib() -> ctypes.CDLL:
         "sgpt_linear_bf16": (i32, [vp, vp, i64, i32, i32, vp, vp, vp]),
         "sgpt_to_bf16": (i32, [vp, i32, i32, i32, vp, vp, vp]),
         "sgpt_sparse24_linear": (i32, [vp, vp, i32, i32, vp, i64, vp, vp, vp]),
+        "sgpt_sparse24_meta_tiles_bytes": (sz, [i32, i32]),
+        "sgpt_sparse24_tile_meta": (i32, [vp, i32, i32, vp, vp]),
         "sgpt_recon_error": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         "sgpt_prune_layer": (i32, [vp, i32, i32, i32, vp, i64, vp, vp, pp, vp, vp, vp, vp,
                                    vp, sz, vp, vp]),
@@ -347,24 +349,48 @@ def linear_bf16(X: torch.Tensor, Wb: torch.Tensor, Y: torch.Tensor, dev_info: to
            "sgpt_linear_bf16")
 
 
-def sparse24_linear(values: torch.Tensor, meta: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
+def sparse24_meta_tiles(meta: torch.Tensor, d_in: int, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """sgpt_pack24's metadata words meta [d_out, d_in/32] int32 re-arranged
+    for sparse24_linear (sgpt_sparse24_tile_meta); done once per weight
+    matrix. Returns (or fills) an int32 buffer of
+    sgpt_sparse24_meta_tiles_bytes(d_out, d_in) bytes."""
+    _dev(meta, torch.int32, "meta")
+    d_out = meta.shape[0]
+    if meta.shape != (d_out, d_in // 32) or not meta.is_contiguous():
+        raise ValueError("meta [d_out, d_in/32], contiguous")
+    nbytes = lib().sgpt_sparse24_meta_tiles_bytes(d_out, d_in)
+    if nbytes == 0:
+        raise ValueError(f"unsupported sizes d_out={d_out} d_in={d_in}")
+    if out is None:
+        out = torch.empty(nbytes // 4, dtype=torch.int32, device=meta.device)
+    _dev(out, torch.int32, "out")
+    if out.numel() * 4 < nbytes or not out.is_contiguous():
+        raise ValueError(f"out needs {nbytes} contiguous bytes")
+    _check(lib().sgpt_sparse24_tile_meta(_ptr(meta), d_out, d_in, _ptr(out), _stream(stream)),
+           "sgpt_sparse24_tile_meta")
+    return out
+
+
+def sparse24_linear(values: torch.Tensor, meta_tiles: torch.Tensor, X: torch.Tensor, Y: torch.Tensor,
                     dev_info: torch.Tensor, stream=None):
     """Y = X W^T from W's packed 2:4 form on the sparse tensor cores
-    (sgpt_sparse24_linear): values [d_out, d_in/2] bf16, meta [d_out,
-    d_in/32] int32 (sgpt_pack24's words), X [n, d_in] bf16, Y [n, d_out]
-    fp32."""
+    (sgpt_sparse24_linear): values [d_out, d_in/2] bf16, meta_tiles from
+    sparse24_meta_tiles, X [n, d_in] bf16, Y [n, d_out] fp32."""
     _dev(values, torch.bfloat16, "values")
-    _dev(meta, torch.int32, "meta")
+    _dev(meta_tiles, torch.int32, "meta_tiles")
     _dev(X, torch.bfloat16, "X")
     _dev(Y, torch.float32, "Y")
     d_out, half = values.shape
     n, d_in = X.shape
-    if half * 2 != d_in or meta.shape != (d_out, d_in // 32) or Y.shape != (n, d_out):
-        raise ValueError("values [d_out, d_in/2], meta [d_out, d_in/32], X [n, d_in], Y [n, d_out]")
-    if not (values.is_contiguous() and meta.is_contiguous() and X.is_contiguous() and Y.is_contiguous()):
+    if half * 2 != d_in or Y.shape != (n, d_out):
+        raise ValueError("values [d_out, d_in/2], X [n, d_in], Y [n, d_out]")
+    if meta_tiles.numel() * 4 < lib().sgpt_sparse24_meta_tiles_bytes(d_out, d_in):
+        raise ValueError("meta_tiles too small for these sizes")
+    if not (values.is_contiguous() and meta_tiles.is_contiguous() and X.is_contiguous() and Y.is_contiguous()):
         raise ValueError("all operands must be contiguous")
-    _check(lib().sgpt_sparse24_linear(_ptr(values), _ptr(meta), d_out, d_in, _ptr(X), n, _ptr(Y), _ptr(dev_info),
-                                      _stream(stream)), "sgpt_sparse24_linear")
+    _check(lib().sgpt_sparse24_linear(_ptr(values), _ptr(meta_tiles), d_out, d_in, _ptr(X), n, _ptr(Y),
+                                      _ptr(dev_info), _stream(stream)), "sgpt_sparse24_linear")
 
 
 def mlp_block_workspace(hidden: int, inter: int, n_tok: int, device="cuda") -> torch.Tensor:

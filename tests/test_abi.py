@@ -115,6 +115,20 @@ def test_other_entry_points_validate():
                               None, None, None, FAKE, 1 << 30, FAKE, None) == 1
 
 
+def test_sparse24_meta_tiles_sizes_and_validation():
+    L = pp.lib()
+    # 4 KB per 256 rows and 128 columns of K, both rounded up
+    assert L.sgpt_sparse24_meta_tiles_bytes(256, 128) == 4096
+    assert L.sgpt_sparse24_meta_tiles_bytes(5120, 25600) == 20 * 200 * 4096
+    assert L.sgpt_sparse24_meta_tiles_bytes(257, 160) == 2 * 2 * 4096
+    assert L.sgpt_sparse24_meta_tiles_bytes(256, 100) == 0            # d_in % 32
+    assert L.sgpt_sparse24_meta_tiles_bytes(0, 128) == 0
+    assert L.sgpt_sparse24_tile_meta(FAKE, 256, 128, MISALIGNED, None) == 1
+    assert L.sgpt_sparse24_tile_meta(None, 256, 128, FAKE, None) == 1
+    assert L.sgpt_sparse24_linear(FAKE, MISALIGNED, 256, 128, FAKE, 10, FAKE, FAKE, None) == 1
+    assert L.sgpt_sparse24_linear(FAKE, FAKE, 256, 128, FAKE, 0, FAKE, FAKE, None) == 1
+
+
 def test_pack_nm_sizes_and_validation():
     L = pp.lib()
     assert L.sgpt_pack_nm_meta_words(64, 2, 4) == 2          # = d_in / 32, as pack24
