@@ -10,8 +10,10 @@
 //      on the compensated weights), e = (w_q - p_q) / U_qq (as a product with
 //      the reciprocal), rank-4 update of the rest of the block with the U
 //      rows held in shared memory;
-//   3. W[:, i2:] -= Err * U[i1:i2, i2:] as an FP32-accurate tensor-core GEMM
-//      (three TF32 products on hi/lo planes of Err and U, gemm_tc.cu).
+//   3. W[:, i2:] -= Err * U[i1:i2, i2:] as FP32-accurate tensor-core GEMMs
+//      (three TF32 products on hi/lo planes of Err and U, gemm_tc.cu): at
+//      once for the rest of the block's group of blocks, once per group for
+//      the columns right of it (launch_prune).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -81,7 +83,7 @@ template <int MODE, int ROWS, int M, bool QUANT>
 __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
     float* __restrict__ W, long long ldw, int rows, int d, int i1, int bw,
     const float* __restrict__ U, uint32_t* __restrict__ mask, float* __restrict__ row_loss,
-    float* __restrict__ Err, float* __restrict__ Err_lo, const unsigned long long* __restrict__ thr,
+    float* __restrict__ Err, float* __restrict__ Err_lo, int err_ld, const unsigned long long* __restrict__ thr,
     int nkeep, const float* __restrict__ qgrid, float qmaxq, int* info) {
   constexpr int LPR = 32 / ROWS;                 // lanes per row
   constexpr int CPL = 4 * ROWS;                  // columns per lane
@@ -105,7 +107,6 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
   const int sub = lane / LPR, sl = lane % LPR;   // row within the warp, lane within the row
   const int base = sub * LPR;                    // first lane of this row
   const int row = (blockIdx.x * kSweepWarps + (tid >> 5)) * ROWS + sub;
-  const int ngroups = bw >> 2;
   constexpr int SPAN = 4 * LPR;                  // columns between a lane's groups
   const bool live = row < rows;
   const bool mine = live;
@@ -341,9 +342,9 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
           lo[j] = ev[j] - h;
           ev[j] = h;
         }
-        st4(Err_lo + (long long)row * kMaxBlock + c, make_float4(lo[0], lo[1], lo[2], lo[3]));
+        st4(Err_lo + (long long)row * err_ld + c, make_float4(lo[0], lo[1], lo[2], lo[3]));
       }
-      st4(Err + (long long)row * kMaxBlock + c, make_float4(ev[0], ev[1], ev[2], ev[3]));
+      st4(Err + (long long)row * err_ld + c, make_float4(ev[0], ev[1], ev[2], ev[3]));
       if (MODE != kModeForced && (sl & 7) == 0) mask[(long long)row * (d / 32) + (i1 + c) / 32] = bits[v];
     }
     if (sl == 0 && row_loss) row_loss[row] += tot;
@@ -357,7 +358,7 @@ static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 2 : 1; }
 
 template <int MODE, int M, bool QUANT>
 static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
-                                  uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
+                                  uint32_t* mask, float* row_loss, float* Err, float* Err_lo, int err_ld,
                                   const unsigned long long* thr, int nkeep, const float* qgrid, float qmaxq,
                                   int* info, cudaStream_t st) {
   static PerDevice attrs;
@@ -372,10 +373,10 @@ static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, in
   const int grid = cdiv(rows, kSweepWarps * rpw);
   if (rpw == 2)
     sweep_kernel<MODE, 2, M, QUANT><<<grid, kSweepThreads, kSweepSmem, st>>>(
-        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, nkeep, qgrid, qmaxq, info);
+        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, nkeep, qgrid, qmaxq, info);
   else
     sweep_kernel<MODE, 1, M, QUANT><<<grid, kSweepThreads, kSweepSmem, st>>>(
-        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, nkeep, qgrid, qmaxq, info);
+        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, nkeep, qgrid, qmaxq, info);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -383,12 +384,12 @@ static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, in
 template <bool QUANT>
 static cudaError_t launch_sweep_q(const sgpt_params& p, int rpw, float* W, long long ldw, int rows, int d, int i1,
                                   int bw, const float* U, uint32_t* mask, float* row_loss, float* Err,
-                                  float* Err_lo, const unsigned long long* thr, const float* qgrid, int* info,
-                                  cudaStream_t st) {
+                                  float* Err_lo, int err_ld, const unsigned long long* thr, const float* qgrid,
+                                  int* info, cudaStream_t st) {
   const float qmaxq = QUANT ? (float)((1 << p.qbits) - 1) : 0.f;
 #define SGPT_SWEEP(MODE, M)                                                                                  \
-  launch_sweep_m<MODE, M, QUANT>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, p.n, qgrid, \
-                                 qmaxq, info, st)
+  launch_sweep_m<MODE, M, QUANT>(rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, p.n, \
+                                 qgrid, qmaxq, info, st)
   if (p.forced) return SGPT_SWEEP(kModeForced, 4);
   if (p.pattern != SGPT_PATTERN_NM) return SGPT_SWEEP(kModeThreshold, 4);
   switch (p.m) {
@@ -408,12 +409,13 @@ static cudaError_t launch_sweep_q(const sgpt_params& p, int rpw, float* W, long 
 // weights (qgrid: the per-row grid, when p.qbits > 0).
 static cudaError_t launch_sweep(const sgpt_params& p, int rpw, float* W, long long ldw, int rows, int d, int i1,
                                 int bw, const float* U, uint32_t* mask, float* row_loss, float* Err, float* Err_lo,
-                                const unsigned long long* thr, const float* qgrid, int* info, cudaStream_t st) {
+                                int err_ld, const unsigned long long* thr, const float* qgrid, int* info,
+                                cudaStream_t st) {
   if (p.qbits > 0)
-    return launch_sweep_q<true>(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, qgrid, info,
-                                st);
-  return launch_sweep_q<false>(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, thr, nullptr, info,
-                               st);
+    return launch_sweep_q<true>(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, qgrid,
+                                info, st);
+  return launch_sweep_q<false>(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, nullptr,
+                               info, st);
 }
 
 // ------------------------------------------------------ quantization grid
@@ -663,20 +665,32 @@ static cudaError_t launch_select(const float* W, long long ldw, int rows, int d,
 
 // ----------------------------------------------------------------- driver
 
+// The trailing update is applied in two parts. The columns of the blocks
+// still to come in the current group (as many whole blocks as fit in
+// kGroupCols columns) get each block's error right after its sweep (K = one
+// block), since the next sweep reads them; every column right of the group
+// gets the errors of the whole group at once when the group ends (K = the
+// group's width). Each column receives the same sum of error-times-U terms
+// as with one update per block (the lazy batch update of the pages, batched
+// over more blocks), in another order; the trailing matrix is read and
+// written once per group instead of once per block.
+constexpr int kGroupCols = 4 * kMaxBlock;
+
 struct PruneWs {
-  float* Err_hi;   // error block of the current OBS block, hi/lo planes (d_out x 128)
+  float* Err_hi;   // error blocks of the current group, hi/lo planes (d_out x kGroupCols)
   float* Err_lo;
   float* U_hi;     // hi/lo planes of U (d_in x d_in)
   float* U_lo;
   SelState* sel;
   float* qgrid;    // per-row quantization grid (scale, zero), d_out x 2
 };
+constexpr int kErrLd = kGroupCols;
 
 static PruneWs carve_prune(void* ws, int d_out, int d_in, size_t* bytes) {
   Carve c(ws);
   PruneWs w;
-  w.Err_hi = c.take<float>((size_t)d_out * kMaxBlock);
-  w.Err_lo = c.take<float>((size_t)d_out * kMaxBlock);
+  w.Err_hi = c.take<float>((size_t)d_out * kErrLd);
+  w.Err_lo = c.take<float>((size_t)d_out * kErrLd);
   w.U_hi = c.take<float>((size_t)d_in * d_in);
   w.U_lo = c.take<float>((size_t)d_in * d_in);
   w.sel = c.take<SelState>(1);
@@ -691,6 +705,28 @@ size_t prune_ws_bytes(int d_out, int d_in) {
   return b;
 }
 
+// W[:, c0:c1] -= Err[:, e0:e0+k] U[u0:u0+k, c0:c1] (FP32-accurate GEMM).
+static cudaError_t trailing_update(const tc::Operand& Ep, const tc::Operand& Up, float* W, long long ldw, int rows,
+                                   int e0, int u0, int k, int c0, int c1, int* info, cudaStream_t st) {
+  if (c1 <= c0 || k <= 0) return cudaSuccess;
+  tc::Job job{};
+  job.mode = 0;
+  job.mt = cdiv(rows, kTile);
+  job.nt = cdiv(c1 - c0, kTile);
+  job.kdim = k;
+  job.a_x0 = e0;
+  job.b_x0 = c0;
+  job.b_y0 = u0;
+  job.C = W;
+  job.ldc = ldw;
+  job.c_col0 = c0;
+  job.Mlim = rows;
+  job.Nlim = c1 - c0;
+  job.alpha = -1.f;
+  job.beta = 1.f;
+  return tc::launch_gemm(Ep, Up, true, job, job.mt * job.nt, info, st);
+}
+
 cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* U,
                          const sgpt_params& p, uint32_t* mask, float* row_loss, void* ws,
                          int* info, cudaStream_t st) {
@@ -703,38 +739,29 @@ cudaError_t launch_prune(float* W, int rows, int d, long long ldw, const float* 
     if ((e = launch_quant_grid(W, ldw, rows, d, p.qbits, w.qgrid, st)) != cudaSuccess) return e;
     qgrid = w.qgrid;
   }
-  const tc::Operand Ep{w.Err_hi, w.Err_lo, rows, kMaxBlock, kMaxBlock};
+  const tc::Operand Ep{w.Err_hi, w.Err_lo, rows, kErrLd, kErrLd};
   const tc::Operand Up{w.U_hi, w.U_lo, d, d, d};
   const int B = p.blocksize;
   const int rpw = sweep_rows_per_warp(rows);
-  for (int i1 = 0; i1 < d; i1 += B) {
-    const int bw = min(B, d - i1);
-    if (!p.forced && p.pattern == SGPT_PATTERN_UNSTRUCTURED) {
-      const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
-      if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
-        return e;
+  const int gw = kGroupCols / B * B;                      // columns per group: whole blocks
+  for (int g1 = 0; g1 < d; g1 += gw) {
+    const int g2 = std::min(d, g1 + gw);                  // the group's columns [g1, g2)
+    for (int i1 = g1; i1 < g2; i1 += B) {
+      const int bw = min(B, d - i1), i2 = i1 + bw;
+      const int slot = i1 - g1;                           // this block's columns of the error buffer
+      if (!p.forced && p.pattern == SGPT_PATTERN_UNSTRUCTURED) {
+        const double kk = std::floor((double)p.sparsity * (double)rows * (double)bw);
+        if ((e = launch_select(W, ldw, rows, d, i1, bw, U, w.sel, (unsigned int)kk, info, st)) != cudaSuccess)
+          return e;
+      }
+      e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi + slot, w.Err_lo + slot,
+                       kErrLd, &w.sel->thr, qgrid, info, st);
+      if (e != cudaSuccess) return e;
+      // the group's later blocks need this block's error before their sweeps
+      if ((e = trailing_update(Ep, Up, W, ldw, rows, slot, i1, bw, i2, g2, info, st)) != cudaSuccess) return e;
     }
-    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, w.Err_hi, w.Err_lo, &w.sel->thr, qgrid,
-                     info, st);
-    if (e != cudaSuccess) return e;
-    const int i2 = i1 + bw;
-    if (i2 < d) {
-      tc::Job job{};
-      job.mode = 0;
-      job.mt = cdiv(rows, kTile);
-      job.nt = cdiv(d - i2, kTile);
-      job.kdim = bw;
-      job.b_x0 = i2;
-      job.b_y0 = i1;
-      job.C = W;
-      job.ldc = ldw;
-      job.c_col0 = i2;
-      job.Mlim = rows;
-      job.Nlim = d - i2;
-      job.alpha = -1.f;
-      job.beta = 1.f;
-      if ((e = tc::launch_gemm(Ep, Up, true, job, job.mt * job.nt, info, st)) != cudaSuccess) return e;
-    }
+    // the columns right of the group: all of the group's errors at once
+    if ((e = trailing_update(Ep, Up, W, ldw, rows, 0, g1, g2 - g1, g2, d, info, st)) != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -796,8 +823,8 @@ cudaError_t launch_prune_noalloc(float* W, int rows, int d, long long ldw, const
       if ((e = launch_select(W, ldw, rows, d, i1, bw, U, sel, (unsigned int)kk, info, st)) != cudaSuccess)
         return e;
     }
-    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, &sel->thr, p.qgrid, info,
-                     st);
+    e = launch_sweep(p, rpw, W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, nullptr, kMaxBlock, &sel->thr, p.qgrid,
+                     info, st);
     if (e != cudaSuccess) return e;
     const int i2 = i1 + bw;
     if (i2 < d) {
