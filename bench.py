@@ -526,25 +526,35 @@ def main():
     # step copies each distinct X and every W from pinned host memory, prunes
     # each input's first matrix with sgpt_prune_layer (Hessian, factor,
     # sweep, pack) and the matrices sharing its H and U with sgpt_prune and
-    # sgpt_pack24, and copies every result back.
+    # sgpt_pack_nm, and copies every pruned W, mask, value and metadata array
+    # back into pinned host memory. Three streams: uploads (h2d), pruning
+    # (comp) and downloads (d2h); step s+1's uploads and step s's downloads
+    # overlap step s's pruning. Each W, mask and packed output has two device
+    # buffers (steps alternate), so an upload never overwrites what a
+    # download of the step before still reads.
     if not args.no_e2e:
-        copy_s, comp_s = torch.cuda.Stream(), torch.cuda.Stream()
+        h2d_s, comp_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
         distinct = {}                 # jobs that read the same X share one copy of it
         x_of_job = [distinct.setdefault(id(X), len(distinct)) for _, X, _ in jobs]
         X_dev = {id(X): X for _, X, _ in jobs}
         X_host = [X_dev[k].cpu().pin_memory() for k in distinct]
         xbuf = [[torch.empty_like(Xh, device=dev) for _ in range(2)] for Xh in X_host]
-        ready = [torch.cuda.Event() for _ in range(2)]
-        free = [torch.cuda.Event() for _ in range(2)]
+        ready = [torch.cuda.Event() for _ in range(2)]      # step's inputs are on the device
+        free = [torch.cuda.Event() for _ in range(2)]       # step's outputs are on the host
+        done = [torch.cuda.Event() for _ in layers]        # layer pruned (per step)
         pin = dict(pin_memory=True)
-        host = []     # per layer: W in, then W, mask, values, meta out
+        host, devb = [], []     # per layer: pinned host tensors; two sets of device buffers
         for W0, W, g, sp, p in layers:
             b = g.bufs
+            pk = b.packs(p)
             host.append({"W_in": W0.cpu().pin_memory(),
                          "W_out": torch.empty(W.shape, dtype=W.dtype, **pin),
                          "mask": torch.empty(b.mask.shape, dtype=b.mask.dtype, **pin),
-                         "values": torch.empty(b.values.shape, dtype=b.values.dtype, **pin) if b.packs(p) else None,
-                         "meta": torch.empty(b.meta.shape, dtype=b.meta.dtype, **pin) if b.packs(p) else None})
+                         "values": torch.empty(b.values.shape, dtype=b.values.dtype, **pin) if pk else None,
+                         "meta": torch.empty(b.meta.shape, dtype=b.meta.dtype, **pin) if pk else None})
+            devb.append([{"W": torch.empty_like(W), "mask": torch.empty_like(b.mask),
+                          "values": torch.empty_like(b.values) if pk else None,
+                          "meta": torch.empty_like(b.meta) if pk else None} for _ in range(2)])
         h2d = sum(Xh.numel() * Xh.element_size() for Xh in X_host) + sum(h["W_in"].numel() * 4 for h in host)
         d2h = sum(sum(t.numel() * t.element_size() for k, t in h.items() if k != "W_in" and t is not None)
                   for h in host)
@@ -553,48 +563,51 @@ def main():
         def e2e_step():
             bsel = step_no[0] & 1
             step_no[0] += 1
-            with torch.cuda.stream(copy_s):
-                copy_s.wait_event(free[bsel])       # the step two back is done with this buffer
+            with torch.cuda.stream(h2d_s):
+                h2d_s.wait_event(free[bsel])        # step s-2's outputs in these buffers are on the host
                 for j, Xh in enumerate(X_host):
                     xbuf[j][bsel].copy_(Xh, non_blocking=True)
-                ready[bsel].record(copy_s)
+                for k, h in enumerate(host):
+                    devb[k][bsel]["W"].copy_(h["W_in"], non_blocking=True)
+                ready[bsel].record(h2d_s)
             with torch.cuda.stream(comp_s):
                 comp_s.wait_event(ready[bsel])
                 k = 0
                 for j, (xs, _, mats) in enumerate(jobs):
                     for m_i, (sp, p) in enumerate(mats):
-                        W0, W, g, _, _ = layers[k]
-                        b, h = g.bufs, host[k]
-                        W.copy_(h["W_in"], non_blocking=True)
+                        g, bd = layers[k][2], devb[k][bsel]
+                        b = g.bufs
                         pack = b.packs(p)
                         if m_i == 0:
-                            pp.prune_layer(W, b.H, b.U, p, b.mask, b.ws, b.info, X=xbuf[x_of_job[j]][bsel],
-                                           values=b.values if pack else None, meta=b.meta if pack else None,
+                            pp.prune_layer(bd["W"], b.H, b.U, p, bd["mask"], b.ws, b.info,
+                                           X=xbuf[x_of_job[j]][bsel], values=bd["values"], meta=bd["meta"],
                                            row_loss=b.row_loss)
                         else:
                             pp.info_clear(b.info)
                             b.row_loss.zero_()
-                            pp.prune(W, b.U, p, b.mask, b.ws, b.info, row_loss=b.row_loss)
+                            pp.prune(bd["W"], b.U, p, bd["mask"], b.ws, b.info, row_loss=b.row_loss)
                             if pack:
-                                pp.pack_nm(W, b.mask, *p.nm, b.values, b.meta, b.info)
-                        h["W_out"].copy_(W, non_blocking=True)
-                        h["mask"].copy_(b.mask, non_blocking=True)
-                        if pack:
-                            h["values"].copy_(b.values, non_blocking=True)
-                            h["meta"].copy_(b.meta, non_blocking=True)
+                                pp.pack_nm(bd["W"], bd["mask"], *p.nm, bd["values"], bd["meta"], b.info)
+                        done[k].record(comp_s)
                         k += 1
-                free[bsel].record(comp_s)
+            with torch.cuda.stream(d2h_s):
+                for k, h in enumerate(host):
+                    d2h_s.wait_event(done[k])
+                    bd = devb[k][bsel]
+                    for key in ("W", "mask", "values", "meta"):
+                        if bd[key] is not None:
+                            h["W_out" if key == "W" else key].copy_(bd[key], non_blocking=True)
+                free[bsel].record(d2h_s)
 
         for _ in range(max(2, args.warmup // 2)):
             e2e_step()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ks = max(2, args.steps // 2)
-        e0.record(copy_s)
-        comp_s.wait_event(e0)
+        e0.record(h2d_s)
         for _ in range(ks):
             e2e_step()
-        e1.record(comp_s)
+        e1.record(d2h_s)
         torch.cuda.synchronize()
         for _, _, g, _, _ in layers:
             pp.raise_on_info(g.bufs.info, where="e2e")
@@ -603,9 +616,11 @@ def main():
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": t_e2e * 1e3 / ks, "steps": ks,
                        "note": ("every step copies each distinct X and every W from pinned host memory and "
-                                "every pruned W, mask, 2:4 values and metadata back; the next step's X copies "
-                                "overlap this step's pruning (two device buffers per input)")}
-        del xbuf
+                                "every pruned W, mask, N:M values and metadata back into pinned host memory; "
+                                "uploads, pruning and downloads run on three streams, so step s+1's uploads "
+                                "and step s's downloads overlap step s's pruning (two device buffers per "
+                                "input and output)")}
+        del xbuf, devb
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, t, cores, sample = cpu_baseline(specs)
