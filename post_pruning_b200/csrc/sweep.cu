@@ -352,26 +352,38 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
   }
 }
 
-// Rows per warp for a layer: two for tall layers (halves the instructions
-// per row), one for short ones (twice the warps in flight).
-static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 2 : 1; }
+// Rows per warp for a layer: four for tall layers (every lane of a row
+// repeats the owner group's decision and in-group steps, so fewer lanes per
+// row means fewer instructions per row), one for short ones (more warps in
+// flight). N:M with M > 4 takes at most two (its groups span lanes).
+static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 4 : 1; }
 
 template <int MODE, int M, bool QUANT>
 static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, int d, int i1, int bw, const float* U,
                                   uint32_t* mask, float* row_loss, float* Err, float* Err_lo, int err_ld,
                                   const unsigned long long* thr, int nkeep, const float* qgrid, float qmaxq,
                                   int* info, cudaStream_t st) {
+  // four rows per warp only where an N:M group stays inside one lane (M = 4)
+  constexpr bool kFour = MODE != kModeNMG;
   static PerDevice attrs;
   const cudaError_t ea = once_per_device(attrs, [] {
-    const cudaError_t r = cudaFuncSetAttribute(sweep_kernel<MODE, 1, M, QUANT>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
-    return r != cudaSuccess ? r
-                            : cudaFuncSetAttribute(sweep_kernel<MODE, 2, M, QUANT>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    cudaError_t r = cudaFuncSetAttribute(sweep_kernel<MODE, 1, M, QUANT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    if (r == cudaSuccess)
+      r = cudaFuncSetAttribute(sweep_kernel<MODE, 2, M, QUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSweepSmem);
+    if (r == cudaSuccess && kFour)
+      r = cudaFuncSetAttribute(sweep_kernel<MODE, kFour ? 4 : 2, M, QUANT>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSweepSmem);
+    return r;
   });
   if (ea != cudaSuccess) return ea;
+  if (!kFour && rpw > 2) rpw = 2;
   const int grid = cdiv(rows, kSweepWarps * rpw);
-  if (rpw == 2)
+  if (rpw == 4)
+    sweep_kernel<MODE, kFour ? 4 : 2, M, QUANT><<<grid, kSweepThreads, kSweepSmem, st>>>(
+        W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, nkeep, qgrid, qmaxq, info);
+  else if (rpw == 2)
     sweep_kernel<MODE, 2, M, QUANT><<<grid, kSweepThreads, kSweepSmem, st>>>(
         W, ldw, rows, d, i1, bw, U, mask, row_loss, Err, Err_lo, err_ld, thr, nkeep, qgrid, qmaxq, info);
   else

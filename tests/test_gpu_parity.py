@@ -196,9 +196,14 @@ PATTERNS = [pp.Params("2:4"), pp.Params("2:4", blocksize=32), pp.Params("unstruc
             pp.Params("unstructured:0.7", blocksize=64)]
 
 
+TALL_2K = LayerSpec("tall_2k", d_in=256, d_out=2304, n_tok=1024, sigma=1.5, seed=9)
+
+
 @pytest.mark.parametrize("p", PATTERNS, ids=lambda p: f"{p.pattern}-b{p.blocksize}")
-@pytest.mark.parametrize("spec", SMALL[:2], ids=lambda s: s.name)
+@pytest.mark.parametrize("spec", SMALL[:2] + [TALL_2K], ids=lambda s: s.name)
 def test_sweep_matches_oracle_given_H(spec, p):
+    """tall_2k: 2304 rows, four rows per warp (2:4 and unstructured), block
+    sizes 32, 64 and 128."""
     W, X = _inputs(spec)
     X64 = bf16_bits_to_f64(X).numpy()
     Hs = (X64.T @ X64).astype(np.float32)
@@ -212,15 +217,15 @@ def test_sweep_matches_oracle_given_H(spec, p):
 # 16:128; SparseGPT review, section 十四 14.4: 2:4, 4:8), against the oracle
 # on the same H: masks, weights, losses and the packed values and metadata.
 NM_PATTERNS = ["1:4", "3:4", "4:8", "8:16", "16:32", "16:64", "16:128"]
-TALL_2K = LayerSpec("tall_2k", d_in=256, d_out=2304, n_tok=1024, sigma=1.5, seed=9)
 
 
 @pytest.mark.parametrize("pattern", NM_PATTERNS)
 @pytest.mark.parametrize("spec", SMALL + [TALL_2K], ids=lambda s: s.name)
 def test_nm_sweep_and_pack_match_oracle(spec, pattern):
     """layer256 and ragged (one row per warp, ragged last block for M <= 64),
-    tall (128 columns, 1000 rows), tall_2k (2304 rows: two rows per warp,
-    where a 128-group spans both of a lane's column spans)."""
+    tall (128 columns, 1000 rows), tall_2k (2304 rows: four rows per warp for
+    n:4, two for M > 4, where a 128-group spans both of a lane's column
+    spans)."""
     n, m = (int(x) for x in pattern.split(":"))
     if spec.d_in % m:
         pytest.skip(f"d_in {spec.d_in} is not a multiple of {m}")
