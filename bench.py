@@ -83,8 +83,8 @@ def parse():
                     help="joint sparsification and quantization of the kept weights to this many bits")
     ap.add_argument("--driver", choices=["sequential", "parallel"], default="sequential",
                     help="mode of the multi-layer driver (config qwen3_32b_mlp_block)")
-    ap.add_argument("--width", type=int, default=25600, help="d_in of config hessian")
-    ap.add_argument("--tokens", type=int, default=131072, help="tokens of config hessian")
+    ap.add_argument("--width", type=int, default=25600, help="d_in of configs hessian and factor")
+    ap.add_argument("--tokens", type=int, default=131072, help="tokens of configs hessian and factor")
     return ap.parse_args()
 
 
@@ -818,8 +818,49 @@ def bench_hessian(args):
           flush=True)
 
 
+def bench_factor(args):
+    """The factorisation alone: U = chol(H_d^-1) of the Hessian of X [tokens
+    x width] (sgpt_factor, damping included), for per-phase timing and
+    profiler captures at a chosen size."""
+    import torch
+
+    import post_pruning_b200 as pp
+    from workloads import LayerSpec, gen_activations
+    dev = torch.device("cuda")
+    spec = LayerSpec("factor", d_in=args.width, d_out=128, n_tok=args.tokens, sigma=1.0, p_out=0.01, f_out=20.0,
+                     x_key=3)
+    X = gen_activations(spec, device=dev)
+    H = torch.empty(args.width, args.width, device=dev)
+    U = torch.empty_like(H)
+    ws = pp.workspace(128, args.width, args.tokens)
+    info = pp.new_info()
+    pp.hessian_compute(H, X, ws, info)
+    del X
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        pp.factor(H, args.tokens, 0.01, U, ws, info)
+    e0, e1 = _events(torch)
+    e0.record(st)
+    for _ in range(args.steps):
+        pp.factor(H, args.tokens, 0.01, U, ws, info)
+    e1.record(st)
+    torch.cuda.synchronize()
+    pp.raise_on_info(info)
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.0 / 3.0 * float(args.width) ** 3
+    hbm, bf16_burst, bf16_sust, kind = peaks()
+    rate = bf16_burst * TF32_OVER_BF16 / 3.0
+    print(json.dumps({"metric": "factorisation U = chol(H_d^-1) alone, FP32-accurate TFLOP/s (2/3 d^3 flop)",
+                      "value": flops / ms / 1e9, "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps,
+                      "warmup": args.warmup,
+                      "config": {"workload": f"H of X {args.tokens} x {args.width} bf16", "name": "factor"},
+                      "peak": rate, "frac": flops / ms / 1e9 / rate,
+                      "peak_kind": f"{kind} bf16 burst x {TF32_OVER_BF16:.3f} (TF32) / 3 (products per fp32 product)"}),
+          flush=True)
+
+
 EXTRA_BENCHES = {"qwen3_32b_mlp_block": bench_mlp_block, "consumer_qwen_down": bench_consumer,
-                 "hessian": bench_hessian}
+                 "hessian": bench_hessian, "factor": bench_factor}
 
 
 if __name__ == "__main__":

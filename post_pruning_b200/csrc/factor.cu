@@ -645,8 +645,10 @@ cudaError_t after(cudaStream_t s2, cudaStream_t s1, cudaEvent_t ev) {
 // Off-chain GEMMs are persistent kernels that would otherwise hold every SM
 // for their whole duration; they leave some to the chain's launches.
 constexpr int kOffChainCtas = kNumSMs - 16;
-// Block columns from which the trailing updates go by pairs.
-constexpr int kPairFrom = 16;
+// Steps per group of the trailing updates and the sums T, and the number of
+// block columns from which they go by groups.
+constexpr int kGroup = 4;
+constexpr int kGroupFrom = 16;
 
 // Upper tiles of the leading part are numbered column by column: tile
 // (i, j), i <= j, is number j (j + 1) / 2 + i.
@@ -667,18 +669,30 @@ inline int tri_start(int j) { return j * (j + 1) / 2; }
 //         still-unused upper part of U (zero at the start); the product that
 //         completes block row k-1 of T also writes its hi/lo planes, which
 //         the next block row of U reads.
-// From kPairFrom block columns on, the updates go by pairs of steps
-// (k+1, k): the first one updates block column k-1 and the diagonal tile of
-// column k-2 with panel k+1 alone (both are needed before the next two chain
-// steps); the second one updates everything left of block column k with
-// both panels (K = 256), so that the bulk of the trailing matrix is read and
-// written once per two block columns.
+// From kGroupFrom block columns on, the steps go by groups of kGroup, k0
+// down to L (the groups counted from the last block column; the final group
+// ends at step 2 for the trailing updates and at step 1 for the sums T).
+// Trailing updates: a step k > L applies its own panel (K = 128) to the
+// group's block columns left of it, L .. k-1 (all but diagonal tile
+// (k-1, k-1), which the chain step updates), and to the diagonal tile
+// (L-1, L-1) that the chain step of L reads, writing the planes of block
+// column k-1 for the next panel; step L applies all of the group's panels
+// (K = up to 512) to block column L-1 above its diagonal tile and, off the
+// chain, to every tile left of it. The tiles of the first launch are
+// contiguous in the column-by-column numbering: (L-1, L-1) is the one just
+// before column L. Sums T: a step k > L adds its term to the group's block
+// rows below it (L .. k-1), which the group's next block rows of U need;
+// step L adds all of the group's terms to the rows above the group, column
+// block q of the group with the terms m <= q (U is upper triangular; its
+// planes are not written below the diagonal) and the columns right of the
+// group with all of them. So the bulk of the trailing matrix and of the
+// sums is read and written once per kGroup block columns.
 cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const FactorStreams& f) {
   const int K = cdiv(d, kTile);
   const tc::Operand Ud{w.U_hi, w.U_lo, d, d, d};
   const tc::Operand Rp{w.R, w.V_lo, d, d, d};
   const tc::Operand Tp{w.T_hi, w.T_lo, kTile, d, d};
-  const bool paired = K >= kPairFrom;
+  const int G = K >= kGroupFrom ? kGroup : 1;
   cudaError_t e = cudaSuccess;
   bool pan_pending = false, upd_pending = false;
   for (int k = K - 1; k >= 0; --k) {
@@ -699,11 +713,12 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
       if ((e = cudaEventRecord(f.chain_done, f.crit)) != cudaSuccess) return e;
     }
     if (k >= 2) {   // block 0 is all the chain step of k = 1 touches
-      const bool second = paired && ((K - 1 - k) & 1) != 0;   // k is the second step of its pair
-      const bool first = paired && !second;
-      // K of this step's updates: panel k, or panels k and k+1 (the last
-      // block may be narrower than 128)
-      const int kp = second ? std::min(2 * kTile, d - c0) : bk;
+      const int k0 = k + (K - 1 - k) % G;              // the group's first step
+      const int L = std::max(k0 - G + 1, 2);           // its last step with trailing updates
+      const bool last = k == L;
+      // K of this step's updates: panel k, or at the group's last step all
+      // of the group's panels (the last block may be narrower than 128)
+      const int kp = last ? std::min((k0 + 1) * kTile, d) - c0 : bk;
       const tc::Operand P{w.R + c0, w.V_lo + c0, c0, kp, d};
       {
         // panel R_ik = A_ik U_kk^T for i < k-1, as hi/lo planes (hi over R,
@@ -728,15 +743,16 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
         if ((e = cudaEventRecord(f.panel_done, f.pan)) != cudaSuccess) return e;
       }
       {
-        // block column k-1 above its diagonal block (and, for the first
-        // step of a pair, the diagonal tile of block column k-2, which comes
-        // just before it in the numbering); the planes of block column k-1
-        // for the next panel
+        // a step before the group's last: the group's block columns left of
+        // it and diagonal tile (L-1, L-1), with the planes of block column
+        // k-1 for the next panel; the last step: block column k-1 above its
+        // diagonal tile, with its planes
         if ((e = cudaStreamWaitEvent(f.pan, f.chain_done, 0)) != cudaSuccess) return e;
         tc::Job job{};
         job.mode = 1;
         job.kdim = kp;
-        job.t0 = tri_start(k - 1) - (first ? 1 : 0);
+        job.t0 = last ? tri_start(k - 1) : tri_start(L) - 1;
+        const int n_tiles = last ? k - 1 : tri_start(k) - tri_start(L);
         job.C = w.R;
         job.ldc = d;
         job.Mlim = job.Nlim = c0;
@@ -746,15 +762,14 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
         job.C_lo = w.A_lo;
         job.ldp = kTile;
         job.p_col0 = c0 - kTile;
-        job.planes_one_col = first ? 1 : 0;
+        job.planes_one_col = last ? 0 : 1;
         job.planes_n0 = c0 - kTile;
         job.max_ctas = kOffChainCtas;
-        if ((e = tc::launch_gemm(P, P, false, job, (k - 1) + (first ? 1 : 0), info, f.pan)) != cudaSuccess)
-          return e;
+        if ((e = tc::launch_gemm(P, P, false, job, n_tiles, info, f.pan)) != cudaSuccess) return e;
         if ((e = cudaEventRecord(f.pan_done, f.pan)) != cudaSuccess) return e;
         pan_pending = true;
       }
-      if (!first) {
+      if (last) {
         // the block columns left of k-1
         if ((e = cudaStreamWaitEvent(f.upd, f.panel_done, 0)) != cudaSuccess) return e;
         tc::Job job{};
@@ -797,15 +812,13 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
     if (k > 0) {
       // T_iq += R_ik U_kq for i < k, q >= k (rows [0, c0), columns [c0, d)),
       // with the planes of T's block row k-1, which this term completes.
-      // Paired steps (k+1, k): the first adds its term to block row k only
-      // (which the next block row of U needs); the second adds both steps'
-      // terms to the rows above, K = 256 over the columns right of the pair
-      // and K = 128 over block column k (U_{k+1,k} = 0), so the rectangle is
-      // read and written once per two block columns.
+      // Grouped steps (see above): a step before the group's last adds its
+      // term to the group's rows below it; the last adds all of the group's
+      // terms to the rows above the group.
       if ((e = cudaStreamWaitEvent(f.rows, f.chain_done, 0)) != cudaSuccess) return e;
       if (k >= 2 && (e = cudaStreamWaitEvent(f.rows, f.panel_done, 0)) != cudaSuccess) return e;
-      const bool t_second = paired && ((K - 1 - k) & 1) != 0;
-      const bool t_first = paired && !t_second;
+      const int k0 = k + (K - 1 - k) % G;
+      const int LT = std::max(k0 - G + 1, 1);
       auto t_job = [&](int row0, int rows, int col0, int cols, int kdim) {
         tc::Job job{};
         job.mode = 0;
@@ -833,14 +846,16 @@ cudaError_t factor_blocks(const FactorWs& w, int d, float* U, int* info, const F
         job.max_ctas = kOffChainCtas;
         return tc::launch_gemm(Rp, Ud, true, job, job.mt * job.nt, info, f.rows);
       };
-      if (t_first) {
-        if ((e = t_job(c0 - kTile, kTile, c0, d - c0, bk)) != cudaSuccess) return e;
-      } else if (t_second) {
-        const int c1 = c0 + kTile;
-        if (c1 < d && (e = t_job(0, c0, c1, d - c1, std::min(2 * kTile, d - c0))) != cudaSuccess) return e;
-        if ((e = t_job(0, c0, c0, bk, bk)) != cudaSuccess) return e;
+      if (k > LT) {
+        const int r0 = LT * kTile;
+        if ((e = t_job(r0, c0 - r0, c0, d - c0, bk)) != cudaSuccess) return e;
       } else {
-        if ((e = t_job(0, c0, c0, d - c0, bk)) != cudaSuccess) return e;
+        // column block q of the group takes the terms m = k .. q; the columns
+        // from block k0 on take all of them
+        for (int q = k; q < k0; ++q)
+          if ((e = t_job(0, c0, q * kTile, kTile, (q + 1) * kTile - c0)) != cudaSuccess) return e;
+        const int ck0 = k0 * kTile;
+        if ((e = t_job(0, c0, ck0, d - ck0, std::min((k0 + 1) * kTile, d) - c0)) != cudaSuccess) return e;
       }
     }
   }

@@ -121,11 +121,13 @@ def test_factor_matches_oracle(spec):
     assert torch.equal(Hd, U)
 
 
-@pytest.mark.parametrize("d", [1920, 2048])
-def test_factor_pairing_boundary(d):
+@pytest.mark.parametrize("d", [1920, 2048, 2304, 2432, 2560])
+def test_factor_grouping_boundary(d):
     """15 block columns (the widest factorisation whose updates go step by
-    step) and 16 (the narrowest that pairs them), against the oracle."""
-    spec = LayerSpec(f"pair_{d}", d_in=d, d_out=64, n_tok=2 * d, sigma=1.5, seed=17)
+    step), 16 (the narrowest that groups them by four) and 18-20 (every
+    length of the final group, which ends at step 2 for the trailing
+    updates and at step 1 for the sums T), against the oracle."""
+    spec = LayerSpec(f"group_{d}", d_in=d, d_out=64, n_tok=2 * d, sigma=1.5, seed=17)
     X64 = bf16_bits_to_f64(gen_activations(spec)).numpy()
     Hs = (X64.T @ X64).astype(np.float32)
     _, U_ref = _oracle_factor(Hs, spec.n_tok)
@@ -141,7 +143,7 @@ def test_factor_pairing_boundary(d):
     assert rel_rows.max() < 1e-4, rel_rows.max()
 
 
-# 17 column blocks with a 32-wide last one (paired updates from 16 block
+# 17 column blocks with a 32-wide last one (grouped updates from 16 block
 # columns on): the block-column loop runs its panels, rank-128 updates, sums
 # T and block rows of U on internal streams and joins them back to the
 # caller's stream, so check it eager, on a side stream behind a pending
