@@ -88,9 +88,11 @@ def parse():
     return ap.parse_args()
 
 
-# DRAM bytes (read + write) per launch of a phase's kernels, from ncu
-# captures of the current kernels on these workloads (none yet: null).
-TRAFFIC = {}
+# DRAM bytes (read + write) per step of each phase's kernels: the
+# dram__bytes_read.sum + dram__bytes_write.sum of every launch of one step of
+# the workload in one ncu capture, summed per phase; null for workloads and
+# overrides without a capture.
+TRAFFIC = {"qwen3_32b_block": {"hessian": 217.46e9, "factor": 160.14e9, "prune": 66.30e9, "pack": 2.87e9}}
 
 
 def peaks():
@@ -293,7 +295,7 @@ def aggregate(weights_per_rank_step: int, steps: int, world: int, t_slowest: flo
 
 # ------------------------------------------------------------------ rooflines
 
-def phase_rooflines(jobs, phase_ms, sustained: bool) -> dict:
+def phase_rooflines(jobs, phase_ms, sustained: bool, traffic=None) -> dict:
     """Achieved rate of each phase against its bound, from the algorithmic
     work of the phase (per step) and its measured time (per step).
 
@@ -323,7 +325,7 @@ def phase_rooflines(jobs, phase_ms, sustained: bool) -> dict:
 
     def entry(name, bound, achieved, peak, unit, work, extra=None):
         e = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-             "frac": achieved / peak if peak else None, "traffic": TRAFFIC.get(name),
+             "frac": achieved / peak if peak else None, "traffic": (traffic or {}).get(name),
              "work_per_step": work}
         e.update(extra or {})
         out[name] = e
@@ -496,7 +498,8 @@ def main():
     value, ms_per_step = agg["value"], agg["ms_per_step"]
 
     sustained = ms_per_step * args.steps > 2000.0     # seconds-long run: the power-capped peak applies
-    roof = phase_rooflines([(xs, X, mats) for xs, X, mats in jobs], phase, sustained)
+    roof = phase_rooflines([(xs, X, mats) for xs, X, mats in jobs], phase, sustained,
+                           None if (args.pattern or args.qbits) else TRAFFIC.get(args.config))
     dominant = max(roof, key=lambda k: phase.get(k, 0.0))
     roofline = dict(roof[dominant])
     roofline["phase"] = dominant
