@@ -433,17 +433,22 @@ def main():
             W.copy_(W0)
         flush.zero_()
 
-    def step_replay(evs_step=None):
-        # evs_step[j][phase]: one event pair around all graphs of that phase of job j
+    def step_replay(evs_step=None, evs_mat=None):
+        # evs_step[j][phase]: one event pair around all graphs of that phase of
+        # job j; evs_mat[(j, m)][phase]: one pair around matrix m's graph
         for j, gl in enumerate(job_graphs):
             for name in PH:
                 ran = False
-                for g in gl:
+                for m, g in enumerate(gl):
                     if name in g.graphs:
                         if evs_step is not None and not ran:
                             evs_step[j][name][0].record(stream)
                         ran = True
+                        if evs_mat is not None:
+                            evs_mat[(j, m)][name][0].record(stream)
                         g.graphs[name].replay()
+                        if evs_mat is not None:
+                            evs_mat[(j, m)][name][1].record(stream)
                 if ran and evs_step is not None:
                     evs_step[j][name][1].record(stream)
 
@@ -457,6 +462,8 @@ def main():
     def mk():
         return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     evs = [[{name: mk() for name in PH} for _ in job_graphs] for _ in range(args.steps)]
+    evs_mat = [{(j, m): {name: mk() for name in ("prune", "pack")} for j, gl in enumerate(job_graphs)
+                for m in range(len(gl))} for _ in range(args.steps)]
     step_ev = [mk() for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
@@ -469,7 +476,7 @@ def main():
     for s_ in range(args.steps):
         prep()
         step_ev[s_][0].record(stream)
-        step_replay(evs[s_])
+        step_replay(evs[s_], evs_mat[s_])
         step_ev[s_][1].record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
@@ -493,6 +500,16 @@ def main():
                     per_job[j][name] += ms
     phase = {k: v / args.steps for k, v in phase.items()}
     per_job = [{k: v / args.steps for k, v in pj.items() if v} for pj in per_job]
+    per_matrix = []
+    for j, (xs, _, mats) in enumerate(jobs):
+        for m, (sp, _) in enumerate(mats):
+            g = job_graphs[j][m]
+            row = {"matrix": sp.name, "d_out": sp.d_out, "d_in": sp.d_in}
+            for name in ("prune", "pack"):
+                if name in g.graphs:
+                    row[f"{name}_ms"] = sum(evs_mat[s_][(j, m)][name][0].elapsed_time(evs_mat[s_][(j, m)][name][1])
+                                            for s_ in range(args.steps)) / args.steps
+            per_matrix.append(row)
     t_rank = max_over_ranks(sum(step_ms) / 1e3, dist if world > 1 else None, dev)
     agg = aggregate(weights_per_step, args.steps, world, t_rank)
     value, ms_per_step = agg["value"], agg["ms_per_step"]
@@ -518,6 +535,11 @@ def main():
         "phases_ms_per_step": phase,
         "phases_ms_per_input": [{"input": f"{xs.d_in}-wide ({', '.join(sp.name for sp, _ in mats)})", **pj}
                                 for (xs, _, mats), pj in zip(jobs, per_job)],
+        "phases_ms_per_matrix": per_matrix,
+        "ms_per_step_median": statistics.median(step_ms),
+        # the same step from H (the Hessian phase left out): factor, sweep, pack
+        "from_H": {"value": weights_per_step * world / ((ms_per_step - phase["hessian"]) * 1e-3),
+                   "unit": UNIT, "ms_per_step": ms_per_step - phase["hessian"]},
         "roofline": roofline,
         "rooflines": roof,
         "gpu_launches": launches,

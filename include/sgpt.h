@@ -77,7 +77,10 @@ typedef struct sgpt_params {
                      of two from 4 to 128, 1 <= n <= m, blocksize % m == 0 and
                      d_in % m == 0 (SGPT_ERR_UNSUPPORTED for other m)        */
   float sparsity; /* unstructured - fraction pruned in each block, [0, 1)    */
-  int blocksize;  /* columns per OBS block: 32, 64, 96 or 128                */
+  int blocksize;  /* columns per OBS block: 32, 64, 96 or 128; the interval
+                     at which an unstructured mask is chosen on the weights
+                     compensated so far (the lazy batch of the trailing
+                     update is internal and changes only rounding order)    */
   float damp;     /* damping ratio (0.01 = 1% of the mean diagonal), >= 0    */
   int forced;     /* 1: mask_bits is an INPUT and no selection is made       */
   int qbits;      /* 0: prune only. 2..16: joint sparsification and
