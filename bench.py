@@ -444,11 +444,12 @@ def main():
                         if evs_step is not None and not ran:
                             evs_step[j][name][0].record(stream)
                         ran = True
-                        if evs_mat is not None:
-                            evs_mat[(j, m)][name][0].record(stream)
+                        mev = evs_mat[(j, m)].get(name) if evs_mat is not None else None
+                        if mev is not None:
+                            mev[0].record(stream)
                         g.graphs[name].replay()
-                        if evs_mat is not None:
-                            evs_mat[(j, m)][name][1].record(stream)
+                        if mev is not None:
+                            mev[1].record(stream)
                 if ran and evs_step is not None:
                     evs_step[j][name][1].record(stream)
 
