@@ -162,10 +162,13 @@ __host__ __device__ inline long long band_start(int ti, int tn) {
 // column tiles (G*256 channels each way), super-block rows in order and, in
 // each, the diagonal super-block first; tiles row by row inside a
 // super-block. CTAs that run together then read a few thousand channels of X
-// rather than all of them.
+// rather than all of them. G = 8 (2048 channels). At d = 25,600 and 131,072
+// tokens, launched alone, G = 2..6 measured 92-97 ms per launch against 100
+// for G = 8 or 12 and 106-107 for 16 or 24, but G = 4 read twice the DRAM
+// bytes (402 against 193 GB) and inside a whole power-capped step it was no
+// faster; narrower layers do not depend on it.
 constexpr int kGroup = 8;
-__host__ __device__ inline void grouped_tile(long long t, int tm, int tn, int& ti, int& tj) {
-  const int G = kGroup;
+__host__ __device__ inline void grouped_tile(long long t, int tm, int tn, int G, int& ti, int& tj) {
   for (int I = 0;; ++I) {
     const int r0 = 2 * G * I, nr = (r0 + 2 * G < tm ? r0 + 2 * G : tm) - r0;
     const int c_hi = G * (I + 1) < tn ? G * (I + 1) : tn;
@@ -287,7 +290,7 @@ __device__ void flush_block(uint32_t S, int rs, int cs, int i0, int j0, float* _
 __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     const __grid_constant__ CUtensorMap xmap, float* __restrict__ H, int d, long long n,
     int nsplit, long long per, float* __restrict__ part, int* info, const __grid_constant__ PairWorks pw,
-    int set, long long wait_cycles) {
+    int set, int group, long long wait_cycles) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -310,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
   } else {
     const int tile = blockIdx.x / nsplit, split = blockIdx.x - (blockIdx.x / nsplit) * nsplit;
     int ti, tj;
-    grouped_tile(tile, (d + kM - 1) / kM, (d + kN - 1) / kN, ti, tj);
+    grouped_tile(tile, (d + kM - 1) / kM, (d + kN - 1) / kN, group, ti, tj);
     i0 = ti * kM;
     j1 = tj * kN;
     j2 = j1 + 128;
@@ -482,7 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
 constexpr int kReduceThreads = 1024;
 __global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const float* __restrict__ part,
                                                                         float* __restrict__ H, int d, int tiles,
-                                                                        int nsplit, const int* info, int set) {
+                                                                        int nsplit, const int* info, int set,
+                                                                        int group) {
   if (cta_info_set(info)) return;
   __shared__ float S[64 * kSLd];
   const int tn = (d + kN - 1) / kN;
@@ -490,7 +494,7 @@ __global__ void __launch_bounds__(kReduceThreads) hessian_reduce_kernel(const fl
   for (int blk = blockIdx.x; blk < tiles * 8; blk += gridDim.x) {
     const int tile = blk >> 3, br = (blk & 7) >> 2, bc = blk & 3;
     int ti, tj;
-    grouped_tile(tile, (d + kM - 1) / kM, tn, ti, tj);
+    grouped_tile(tile, (d + kM - 1) / kM, tn, group, ti, tj);
     const int bi0 = ti * kM + 64 * br, bj0 = tj * kN + 64 * bc;
     if (!(bi0 < d && bj0 < d && bj0 + 63 >= bi0)) continue;   // block-uniform
     const float* src = part + (size_t)tile * nsplit * kM * kN + (size_t)(64 * br + r) * kN + 64 * bc + c4;
@@ -584,7 +588,7 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Plan {
-  int tiles, nsplit;
+  int tiles, nsplit, group;
   long long per;
   PairWorks pw;     // pw.ncta > 0: square tiles (then tiles/nsplit/per are unused)
   PairTiles pt;
@@ -675,6 +679,7 @@ Plan plan(int d, long long n) {
   long long per = ((n + ns - 1) / ns + kBK - 1) / kBK * kBK;
   ns = (n + per - 1) / per;
   p.tiles = tiles;
+  p.group = kGroup;
   p.nsplit = (int)std::max<long long>(1, ns);
   p.per = per;
   return p;
@@ -720,14 +725,15 @@ cudaError_t launch_hessian_tc(float* H, const uint16_t* X, long long n, int d, v
   if (ea != cudaSuccess) return ea;
   const int grid = p.pw.ncta > 0 ? p.pw.ncta : p.tiles * p.nsplit;
   hessian_tc_kernel<<<grid, kThreads, kSmem, st>>>(map, H, d, n, p.nsplit, p.per, part, info, p.pw, set ? 1 : 0,
-                                                   wait_limit_cycles());
+                                                   p.group, wait_limit_cycles());
   count_launches(1);
   if (p.pw.ncta > 0) {
     hessian_pair_reduce_kernel<<<p.pair_blocks, kReduceThreads, 0, st>>>(part, H, d, p.pt, info, set ? 1 : 0);
     count_launches(1);
   } else if (p.nsplit > 1) {
     const int g = (int)std::min<long long>((long long)p.tiles * 8, 8 * kNumSMs);
-    hessian_reduce_kernel<<<g, kReduceThreads, 0, st>>>(part, H, d, p.tiles, p.nsplit, info, set ? 1 : 0);
+    hessian_reduce_kernel<<<g, kReduceThreads, 0, st>>>(part, H, d, p.tiles, p.nsplit, info, set ? 1 : 0,
+                                                        p.group);
     count_launches(1);
   }
   return cudaGetLastError();

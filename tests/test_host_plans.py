@@ -37,13 +37,15 @@ int main() {
   for (int d = 32; d <= 32768; d += (d < 4096 ? 32 : 544)) {
     const int tm = (d + 127) / 128, tn = (d + 255) / 256;
     const long long T = band_start(tm, tn);
-    std::vector<char> seen((size_t)tm * tn, 0);
-    for (long long t = 0; t < T; ++t) {
-      int ti = -1, tj = -1;
-      grouped_tile(t, tm, tn, ti, tj);
-      if (ti < 0 || ti >= tm || tj < 0 || tj >= tn || tj < ti / 2 || seen[(size_t)ti * tn + tj]++) {
-        if (bad++ < 5) printf("band d=%d t=%lld -> (%d, %d)\n", d, t, ti, tj);
-        break;
+    for (int G : {4, 8, 12, 16, 24}) {
+      std::vector<char> seen((size_t)tm * tn, 0);
+      for (long long t = 0; t < T; ++t) {
+        int ti = -1, tj = -1;
+        grouped_tile(t, tm, tn, G, ti, tj);
+        if (ti < 0 || ti >= tm || tj < 0 || tj >= tn || tj < ti / 2 || seen[(size_t)ti * tn + tj]++) {
+          if (bad++ < 5) printf("band d=%d G=%d t=%lld -> (%d, %d)\n", d, G, t, ti, tj);
+          break;
+        }
       }
     }
   }
