@@ -72,8 +72,8 @@ __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsi
 // saliencies by shuffle and counts, for each of its own columns, the group
 // columns that beat it (larger saliency, or equal and lower column); the N
 // best are kept. An M-group covers M/4 consecutive lanes of one column span,
-// or (M = 128 with two rows per warp) every lane of both spans. The group
-// steps then apply the decided bits like a forced mask.
+// or, when M is wider than a span, every lane of M/span consecutive spans.
+// The group steps then apply the decided bits like a forced mask.
 //
 // QUANT (joint sparsification and quantization, SparseGPT review sections
 // 十五 and 十七): a kept weight is replaced by its value on the row's grid
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
       const float r[4] = {ri.x, ri.y, ri.z, ri.w};
       if (MODE == kModeNMG && (q0 & (M - 1)) == 0) {
         // decide the M-group that starts here
-        constexpr int NSPAN = (M > SPAN) ? ROWS : 1;        // column spans the group covers
+        constexpr int NSPAN = (M > SPAN) ? M / SPAN : 1;    // column spans the group covers
         constexpr int NL = (M > SPAN) ? LPR : M / 4;        // lanes it covers in each span
         const int gl0 = (M > SPAN) ? 0 : (q0 - gi * SPAN) / 4;   // its first lane (row-relative)
         const bool member = sl >= gl0 && sl < gl0 + NL;
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kSweepThreads) sweep_kernel(
 // Rows per warp for a layer: four for tall layers (every lane of a row
 // repeats the owner group's decision and in-group steps, so fewer lanes per
 // row means fewer instructions per row), one for short ones (more warps in
-// flight). N:M with M > 4 takes at most two (its groups span lanes).
+// flight). N:M with M > 4 takes at most two (see launch_sweep_m).
 static int sweep_rows_per_warp(int rows) { return rows >= 2048 ? 4 : 1; }
 
 template <int MODE, int M, bool QUANT>
@@ -363,7 +363,8 @@ static cudaError_t launch_sweep_m(int rpw, float* W, long long ldw, int rows, in
                                   uint32_t* mask, float* row_loss, float* Err, float* Err_lo, int err_ld,
                                   const unsigned long long* thr, int nkeep, const float* qgrid, float qmaxq,
                                   int* info, cudaStream_t st) {
-  // four rows per warp only where an N:M group stays inside one lane (M = 4)
+  // N:M with M > 4 stays at two rows per warp: at four its decision
+  // registers leave one CTA per SM and the sweep measured slower (16:64)
   constexpr bool kFour = MODE != kModeNMG;
   static PerDevice attrs;
   const cudaError_t ea = once_per_device(attrs, [] {
