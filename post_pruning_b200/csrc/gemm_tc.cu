@@ -426,9 +426,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(
       for (int e = 0; e < 64; ++e) acc[e] = 0.f;
       for (int c0 = 0; c0 < iters; c0 += kChunk, ++u) {
         const int b = u & 1;
-        if (!failed && !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1, wait_cycles)) failed = 1;
+        // one decision per warp: the TMEM loads below are warp-collective
+        int bad = failed;
+        if (!bad) bad = !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1, wait_cycles);
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad) failed = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (!failed) {
+        if (!bad) {
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             uint32_t v[32];
@@ -641,9 +645,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_wide_bf16_kernel(
       for (int e = 0; e < 128; ++e) acc[e] = 0.f;
       for (int c0 = 0; c0 < iters; c0 += kChunk, ++u) {
         const int b = u & 1;
-        if (!failed && !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1, wait_cycles)) failed = 1;
+        // one decision per warp: the TMEM loads below are warp-collective
+        int bad = failed;
+        if (!bad) bad = !mbar_wait(tfull0 + 8 * b, (u >> 1) & 1, wait_cycles);
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad) failed = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (!failed) {
+        if (!bad) {
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t v[32];

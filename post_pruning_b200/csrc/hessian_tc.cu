@@ -422,7 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(
     // Drain every chunk into the running sums, then hand the buffer back.
     for (int c = 0; c < nchunks; ++c) {
       const int b = c & 1;
-      if (!mbar_wait(tfull0 + 8 * b, (c >> 1) & 1, wait_cycles)) {
+      // one decision per warp: the TMEM loads and the __syncwarp below are
+      // warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * b, (c >> 1) & 1, wait_cycles) ? 1 : 0)) {
         failed = 1;
         break;
       }
