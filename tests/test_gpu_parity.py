@@ -230,7 +230,19 @@ def test_nm_sweep_and_pack_match_oracle(spec, pattern):
     spans)."""
     n, m = (int(x) for x in pattern.split(":"))
     if spec.d_in % m:
-        pytest.skip(f"d_in {spec.d_in} is not a multiple of {m}")
+        # a width that is not a whole number of groups: refused before any
+        # launch, W and the mask untouched
+        dev = torch.device("cuda")
+        W = torch.ones(spec.d_out, spec.d_in, device=dev)
+        U = torch.eye(spec.d_in, device=dev)
+        mask = torch.full((spec.d_out, spec.d_in // 32), 7, dtype=torch.int32, device=dev)
+        info = pp.new_info()
+        with pytest.raises(pp.SgptError) as err:
+            pp.prune(W, U, pp.Params(pattern), mask, pp.workspace(spec.d_out, spec.d_in), info)
+        assert err.value.name == "INVALID_ARG"
+        torch.cuda.synchronize()
+        assert bool((W == 1).all()) and bool((mask == 7).all())
+        return
     W, X = _inputs(spec)
     X64 = bf16_bits_to_f64(X).numpy()
     Hs = (X64.T @ X64).astype(np.float32)
