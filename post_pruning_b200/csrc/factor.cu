@@ -14,9 +14,9 @@
 // next is diag(k) -> chain step(k) -> diag(k-1): the chain step forms, in
 // plain FP32 on 136 CTAs, the one panel tile R_{k-1,k} and the update of
 // diagonal block k-1 that diag(k-1) waits for. Every other product (the
-// panel R_ik = A_ik U_kk^T of the rows above, the rank-128 updates of the
-// leading part, the sums T_iq = sum_m R_im U_mq over whole rectangles and
-// the block rows U_kq = -U_kk T_kq of the inverse) runs off the chain on the
+// panel R_ik = A_ik U_kk^T of the rows above, the rank-128 to rank-512
+// updates of the leading part, the sums T_iq = sum_m R_im U_mq over whole
+// rectangles and the block rows U_kq = -U_kk T_kq of the inverse) runs off the chain on the
 // tensor cores as an FP32-accurate three-product TF32 GEMM (gemm_tc.cu).
 // Operands move between those GEMMs as hi/lo planes written by the producing
 // epilogue; the planes of the first column block come from the
@@ -666,8 +666,8 @@ inline int tri_start(int j) { return j * (j + 1) / 2; }
 //   upd:  the update of the block columns left of k-1;
 //   rows: block row k of U, U_kq = -U_kk T_kq (q > k), then the step's
 //         terms R_ik U_kq (i < k, q >= k) of the sums
-//         T_iq = sum_{m=i+1..q} R_im U_mq: one rank-128 product over the
-//         whole rectangle above and right of block k. T lives in the
+//         T_iq = sum_{m=i+1..q} R_im U_mq: products over whole
+//         rectangles above and right of block k (grouped, below). T lives in the
 //         still-unused upper part of U (zero at the start); the product that
 //         completes block row k-1 of T also writes its hi/lo planes, which
 //         the next block row of U reads.

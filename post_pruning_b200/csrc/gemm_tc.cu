@@ -8,9 +8,9 @@
 // product is about 2^-21 relative, against 2^-24 for a plain fp32 FMA and
 // 2^-11 for a single TF32 product.
 //
-// Used for the panel products, the rank-128 updates and the triangular
-// inverse of the factorisation and for the lazy trailing update of the OBS
-// sweep. The same kernel also runs plain bf16 products (one
+// Used for the panel products, the rank-128 to rank-512 updates and the
+// triangular inverse of the factorisation and for the lazy trailing update of
+// the OBS sweep. The same kernel also runs plain bf16 products (one
 // tcgen05.mma.kind::f16 per K step of 16, K-major operands, fp32
 // accumulation), the forward passes between the layers of a block.
 //

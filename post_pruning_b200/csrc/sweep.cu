@@ -62,9 +62,9 @@ __device__ __forceinline__ unsigned long long sal_key(float w, float inv_u, unsi
 // Arithmetically this is the column-by-column sweep with the updates of the
 // four columns to the columns right of the group summed together. The chain
 // per group is one shuffle, the four in-group steps and one rank-4 update;
-// the U values are loaded before the weights arrive. Two rows per warp halve
-// the owner work per row (for tall layers); one row per warp gives more
-// parallelism to short ones.
+// the U values are loaded before the weights arrive. Several rows per warp
+// (four for tall layers, two for N:M with M > 4) cut the repeated owner work
+// per row; one row per warp gives more parallelism to short layers.
 // N:M with M > 4 (kModeNMG): at the first column of each group of M the
 // lanes holding the group's columns rank them by saliency on the weights as
 // compensated so far (every later column has received the updates of every
