@@ -131,7 +131,9 @@ sgpt_status sgpt_sync_status(const int* dev_info, void* stream);
  *   H   [d_in x d_in] fp32, full symmetric matrix, updated in place; both
  *       triangles are written. Zero it first (sgpt_hessian_zero) to start a
  *       new accumulation; call repeatedly to stream token chunks.
- *   X   [n_tok x d_in] bf16 bit patterns, row-major, 16-byte aligned rows.
+ *   X   [n_tok x d_in] bf16 bit patterns, row-major, 16-byte aligned rows;
+ *       may be NULL when n_tok == 0 (then nothing is launched and H is left
+ *       as it is).
  * Products are exact in fp32; sums are fp32 (tensor cores, fixed order). */
 sgpt_status sgpt_hessian_zero(float* H, int d_in, void* stream);
 sgpt_status sgpt_hessian_accumulate(float* H, const uint16_t* X, int64_t n_tok, int d_in,

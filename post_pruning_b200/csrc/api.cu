@@ -123,8 +123,9 @@ sgpt_status sgpt_hessian_zero(float* H, int d_in, void* stream) {
 namespace {
 sgpt_status hessian(float* H, const uint16_t* X, int64_t n_tok, int d_in, void* ws, size_t ws_bytes, int* dev_info,
                     void* stream, bool set) {
-  if (!H || !X || !aligned16(H) || !aligned16(X) || !valid_din(d_in) || n_tok < 0 || !dev_info)
-    return SGPT_ERR_INVALID_ARG;
+  // X may be NULL when there are no tokens
+  if (!H || !aligned16(H) || !valid_din(d_in) || n_tok < 0 || !dev_info) return SGPT_ERR_INVALID_ARG;
+  if (n_tok > 0 && (!X || !aligned16(X))) return SGPT_ERR_INVALID_ARG;
   if (n_tok > (int64_t)INT32_MAX) return SGPT_ERR_INVALID_ARG;   // TMA coordinates are 32-bit
   if (n_tok == 0) return set ? sgpt_hessian_zero(H, d_in, stream) : SGPT_OK;
   sgpt_status s = check_ws(ws, ws_bytes, hessian_ws_bytes(d_in, n_tok));

@@ -115,6 +115,16 @@ def test_other_entry_points_validate():
                               None, None, None, FAKE, 1 << 30, FAKE, None) == 1
 
 
+def test_hessian_without_tokens():
+    """n_tok == 0: X may be NULL and the accumulation is a no-op (nothing is
+    launched, so this runs without a GPU); a negative count or a NULL X with
+    tokens is refused."""
+    L = pp.lib()
+    assert L.sgpt_hessian_accumulate(FAKE, None, 0, 256, None, 0, FAKE, None) == 0
+    assert L.sgpt_hessian_accumulate(FAKE, None, 5, 256, FAKE, 1 << 30, FAKE, None) == 1
+    assert L.sgpt_hessian_accumulate(FAKE, FAKE, -1, 256, FAKE, 1 << 30, FAKE, None) == 1
+
+
 def test_sparse24_meta_tiles_sizes_and_validation():
     L = pp.lib()
     # 4 KB per 256 rows and 128 columns of K, both rounded up

@@ -482,3 +482,29 @@ def test_hessian_long_accumulation():
         absref = float(np.dot(np.abs(Xh[:, a]), np.abs(Xh[:, b])))
         assert abs(Hh[a, b] - ref) <= 2e-6 * absref
         assert Hh[a, b] == Hh[b, a]
+
+
+def test_edge_cases_no_tokens_and_smallest_layer():
+    """No tokens: sgpt_hessian_compute gives H = 0 and sgpt_hessian_accumulate
+    leaves H as it was. The smallest layer the library takes (one output row,
+    32 inputs) against the oracle, 2:4 and unstructured."""
+    dev = torch.device("cuda")
+    info = pp.new_info()
+    d = 256
+    X0 = torch.empty(0, d, dtype=torch.bfloat16, device=dev)
+    ws = pp.workspace(64, d)
+    H = torch.full((d, d), 3.0, device=dev)
+    pp.hessian_accumulate(H, X0, ws, info)
+    torch.cuda.synchronize()
+    assert bool((H == 3.0).all())
+    pp.hessian_compute(H, X0, ws, info)
+    torch.cuda.synchronize()
+    assert bool((H == 0).all())
+    assert pp.sync_status(info) == 0
+    spec = LayerSpec("min", d_in=32, d_out=1, n_tok=64, seed=23)
+    W, X = _inputs(spec)
+    X64 = bf16_bits_to_f64(X).numpy()
+    Hs, U_ref = _oracle_factor((X64.T @ X64).astype(np.float32), spec.n_tok)
+    for p in (pp.Params("2:4"), pp.Params("unstructured:0.5")):
+        gpu = gpu_prune_layer(W, X, p)
+        assert_parity(compare(gpu, W.numpy().astype(np.float64), Hs, U_ref, p), p)
